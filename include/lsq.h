@@ -1,0 +1,268 @@
+/*
+ * lsq.h - C ABI of the streamed NF4-LoRA training path on one B200 (sm_100a).
+ *
+ * The method: the frozen base of a Llama/Qwen decoder stack is quantised once,
+ * offline, to blockwise NF4 and kept in page-locked host RAM; during training
+ * each decoder layer's quantised bytes are copied into a small pool of HBM
+ * slots on a copy stream while the previous layer computes, forward
+ * 0 -> L-1 and, under gradient checkpointing, backward L-1 -> 0; only the LoRA
+ * adapters train.  Sources: "Soup" README snapshot (headline + "Citing Soup");
+ * soup-cli 0.72.0 -> 0.72.2 diff, CHANGELOG [0.72.2] and
+ * docs/performance-and-quantization.md "Layer Streaming" / "NF4 streaming";
+ * themenonlab blog "The trick: layer streaming"; aiany.app listing "How It
+ * Works".  The pages fix no kernel; formats that they leave open are stated
+ * below as readings.
+ *
+ * Conventions for every call:
+ *  - The caller owns every buffer.  Device pointers are CUDA device memory of
+ *    the current device; "host pinned" means page-locked host memory
+ *    (cudaHostAlloc / cudaHostRegister).  The library allocates no device
+ *    memory on any call below; scratch is passed in as `workspace`.
+ *  - bf16 means IEEE bfloat16 (2 bytes); all matrices are row-major, dense,
+ *    with the stated leading dimension equal to the row length.
+ *  - Calls are asynchronous: they validate, enqueue on the given stream and
+ *    return.  A NULL stream means the legacy default stream.
+ *  - Errors are returned, never thrown, and nothing is enqueued when a call
+ *    returns non-OK.  lsq_last_error() gives a message for the calling thread.
+ *    Kernels never trap: a bounded device-side wait that expires records
+ *    LSQ_ETIMEOUT in a device status word read by lsq_device_status().
+ */
+#ifndef LSQ_H_
+#define LSQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lsq_cuda_stream; /* a cudaStream_t */
+
+typedef enum lsq_status {
+  LSQ_OK = 0,
+  LSQ_EINVAL = 1,       /* bad argument: size, alignment, NULL pointer */
+  LSQ_ENOTPINNED = 2,   /* a host source is not page-locked */
+  LSQ_ECUDA = 3,        /* a CUDA runtime call failed (message in lsq_last_error) */
+  LSQ_ETIMEOUT = 4,     /* a bounded device wait expired */
+  LSQ_ESTATE = 5,       /* call out of order (stream scheduler) */
+  LSQ_EUNSUPPORTED = 6  /* device is not sm_100 or a limit of this build */
+} lsq_status;
+
+/* Static message for a status code. */
+const char* lsq_status_str(lsq_status s);
+/* Message of the last non-OK status returned on this host thread ("" if none). */
+const char* lsq_last_error(void);
+/* ABI version: 100 * major + minor. */
+int lsq_version(void);
+/* Reads and clears the device status word of the current device (a
+ * synchronous cudaMemcpy): *status = LSQ_OK or the first device-side error
+ * since the last read, *where = the site code of that error. */
+lsq_status lsq_device_status(int32_t* status, int32_t* where);
+
+/* ------------------------------------------------------------------------
+ * NF4 blockwise format.
+ *
+ * Pages: the streamed base is "quantised once, offline, one tensor at a
+ * time" to NF4 (soup-cli diff, docs "NF4 streaming (quantization: 4bit)";
+ * CHANGELOG [0.72.2]).  Readings (the pages give no format): the 16-level
+ * NormalFloat codebook of QLoRA (8 positive and 7 negative normal quantiles,
+ * an exact 0, scaled to [-1, 1]); block = 64 consecutive elements of a
+ * row-major [n_out, k_in] weight (k_in % 64 == 0); one fp32 absmax per block,
+ * stored row-major [n_out][k_in/64]; code = nearest level to w/absmax (fp32
+ * division, ties to the lower level, all-zero block -> absmax 0, codes 7);
+ * two codes per byte, first element in the high nibble; dequantised value
+ * bf16_rn(fp32(level) * absmax).
+ * ---------------------------------------------------------------------- */
+typedef struct lsq_nf4_weight {
+  const uint8_t* codes; /* device, n_out*k_in/2 bytes, 16-byte aligned */
+  const float* absmax;  /* device, n_out*(k_in/64) fp32, 4-byte aligned */
+  int64_t n_out;        /* rows (output features), >= 1, multiple of 8 */
+  int64_t k_in;         /* columns (input features), multiple of 64 */
+} lsq_nf4_weight;
+
+/* Copies the library's 16 NF4 levels (ascending fp32) into host array out. */
+lsq_status lsq_nf4_codebook(float out[16]);
+
+/* Quantise a bf16 weight (device, [n_out, k_in] row-major) into codes
+ * (device, n_out*k_in/2 bytes) and absmax (device, n_out*k_in/64 fp32).
+ * Definition: "NF4 blockwise format" above.  Bit-exact with a CPU
+ * implementation of that definition.  EINVAL on k_in % 64 or NULLs. */
+lsq_status lsq_nf4_quantize(const void* w_bf16, int64_t n_out, int64_t k_in, uint8_t* codes, float* absmax,
+                            lsq_cuda_stream stream);
+
+/* Dequantise into a bf16 [n_out, k_in] device buffer (the exact values the
+ * fused kernels feed to the tensor cores); for tests and diagnostics. */
+lsq_status lsq_nf4_dequantize(const lsq_nf4_weight* w, void* w_bf16, lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Fused NF4-dequant GEMM with LoRA, forward.
+ *
+ * Y = residual + X deq(W)^T + s (X A^T) B^T,   U = X A^T
+ * The frozen-base linear with a LoRA adapter that layer streaming trains
+ * (themenonlab blog, "only the small LoRA adapter is actually resident and
+ * trainable"; soup-cli diff docs "Layer Streaming", lora.r / lora.alpha).
+ * s = alpha / r.  The dequantised tile never reaches HBM: the kernel decodes
+ * NF4 into shared memory and multiplies on the tensor cores (tcgen05, fp32
+ * accumulation in TMEM); the rank-r path runs as two small MMAs, one in the
+ * main loop (U) and one before the epilogue (s U B^T); Y is rounded to bf16
+ * once.
+ *  x        device bf16 [M, k_in], 16-byte aligned
+ *  A        device bf16 [r, k_in]   (LoRA down), NULL with r = 0 disables LoRA
+ *  B        device bf16 [n_out, r]  (LoRA up)
+ *  residual device bf16 [M, n_out] or NULL; may alias y
+ *  y        device bf16 [M, n_out]
+ *  u_out    device fp32 [M, r] or NULL (kept for the backward)
+ * Limits: 1 <= M, 0 <= r <= 64.  Deterministic (no atomics, fixed order). */
+lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A, const void* B,
+                            int32_t r, float s, const void* residual, void* y, float* u_out,
+                            lsq_cuda_stream stream);
+
+/* Up to three linears that read the same x in one launch (q/k/v, gate/up);
+ * segment i uses W[i], A[i], B[i], residual[i], y[i], u_out[i] exactly as
+ * lsq_nf4_lora_fwd.  All W[i].k_in equal; r and s shared. */
+lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                  const void* const* A, const void* const* B, int32_t r, float s,
+                                  const void* const* residual, void* const* y, float* const* u_out,
+                                  lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Backward of the fused linear (frozen W: no weight gradient).
+ *
+ * G = dY B;  dX = dY deq(W) + s G A;  dB (+)= s dY^T U;  dA (+)= s G^T X.
+ * The gradients that make "non-zero gradients at layer 0" hold (soup-cli
+ * diff, CHANGELOG [0.72.2], "Correctness").  dX runs on the tensor cores
+ * against the dequantised tile in MN-major layout; dA and dB are
+ * deterministic two-stage reductions over M (no atomics).
+ *  x    device bf16 [M, k_in]   forward input
+ *  dy   device bf16 [M, n_out]  upstream gradient
+ *  u    device fp32 [M, r]      U from the forward
+ *  dx   device bf16 [M, k_in] or NULL
+ *  dA   device fp32 [r, k_in];  dB device fp32 [n_out, r]
+ *  accumulate  0: overwrite dA/dB, 1: add into them
+ *  workspace   device scratch of lsq_nf4_lora_bwd_workspace_size() bytes,
+ *              256-byte aligned; contents undefined after the call. */
+size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r);
+lsq_status lsq_nf4_lora_bwd(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M, const void* A,
+                            const void* B, int32_t r, float s, const float* u, void* dx, float* dA, float* dB,
+                            int32_t accumulate, void* workspace, size_t workspace_bytes,
+                            lsq_cuda_stream stream);
+
+/* Up to three linears that read the same x: dx = sum_i (dy[i] W[i] + s G[i] A[i]),
+ * per-segment dA[i], dB[i].  dx may be NULL (gradients of the adapters only). */
+lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, const void* const* dy,
+                                  int64_t M, const void* const* A, const void* const* B, int32_t r, float s,
+                                  const float* const* u, void* dx, float* const* dA, float* const* dB,
+                                  int32_t accumulate, void* workspace, size_t workspace_bytes,
+                                  lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Dense bf16 GEMM for the resident, unquantised lm_head ("Untied
+ * embed_tokens + lm_head stay resident and unquantised", soup-cli diff, docs
+ * "NF4 streaming").  tcgen05, fp32 accumulation.
+ *  trans_b = 0:  out[M,N] = a[M,K] b[N,K]^T   (logits = h E^T)
+ *  trans_b = 1:  out[M,N] = a[M,K] b[K,N]     (dh = dlogits E)
+ *  out_f32 = 1: fp32 output, else bf16.  K % 64 == 0, N % 8 == 0. */
+lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, int64_t M, int64_t N, int64_t K,
+                          int32_t trans_b, int32_t out_f32, lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Decoder-layer kernels around the linears (Llama / Qwen, "Llama / Qwen
+ * only", soup-cli diff docs "Layer Streaming", "Honest scope").  Activations
+ * bf16, reductions fp32.  Row-major [rows, d] unless stated.
+ * ---------------------------------------------------------------------- */
+/* y = x / sqrt(mean(x^2) + eps) * g;  rstd[row] = 1/sqrt(mean(x^2)+eps) (fp32, may be NULL). */
+lsq_status lsq_rmsnorm_fwd(const void* x, const void* g, void* y, float* rstd, int64_t rows, int64_t d, float eps,
+                           lsq_cuda_stream stream);
+/* dres_out = dres_in + d/dx of the norm given dy (g frozen); dres_in may be
+ * NULL (treated as 0) or alias dres_out. */
+lsq_status lsq_rmsnorm_bwd(const void* dy, const void* x, const void* g, const float* rstd, const void* dres_in,
+                           void* dres_out, int64_t rows, int64_t d, lsq_cuda_stream stream);
+/* In-place rotate-half RoPE on x viewed as [batch, seq, heads, hd] at
+ * positions 0..seq-1; inverse = 1 applies the transpose (backward). */
+lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t heads, int64_t hd, float theta, int32_t inverse,
+                    lsq_cuda_stream stream);
+/* Causal GQA attention: q [B,S,Hq,hd], k,v [B,S,Hkv,hd] -> o [B,S,Hq,hd],
+ * lse [B,Hq,S] fp32 (log-sum-exp of the scaled scores).  Scale 1/sqrt(hd). */
+lsq_status lsq_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t batch,
+                             int64_t seq, int64_t hq, int64_t hkv, int64_t hd, lsq_cuda_stream stream);
+/* Gradients dq, dk, dv (bf16, same layouts) from do; deterministic.
+ * workspace: lsq_attention_bwd_workspace_size() bytes (row dot products). */
+size_t lsq_attention_bwd_workspace_size(int64_t batch, int64_t seq, int64_t hq);
+lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,
+                             int64_t hkv, int64_t hd, void* workspace, size_t workspace_bytes,
+                             lsq_cuda_stream stream);
+/* m = silu(g) * u over n elements. */
+lsq_status lsq_swiglu_fwd(const void* g, const void* u, void* m, int64_t n, lsq_cuda_stream stream);
+/* dg, du from dm (dg/du may alias g/u: in-place). */
+lsq_status lsq_swiglu_bwd(const void* dm, const void* g, const void* u, void* dg, void* du, int64_t n,
+                          lsq_cuda_stream stream);
+/* h[i, :] = table[ids[i], :], ids int32 device [rows]; table bf16 [vocab, d]. */
+lsq_status lsq_embed_gather(const int32_t* ids, const void* table, void* h, int64_t rows, int64_t d,
+                            int64_t vocab, lsq_cuda_stream stream);
+/* Causal-LM cross entropy over logits fp32 [batch*seq, V]: target of row
+ * (b, t) is ids[b, t+1] for t < seq-1; the last row of each sequence is
+ * ignored.  loss (device fp32 scalar) = mean NLL over batch*(seq-1) rows;
+ * dlogits bf16 [batch*seq, V] = (softmax - onehot) / (batch*(seq-1)), zero
+ * on ignored rows.  workspace: lsq_xent_workspace_size() bytes. */
+size_t lsq_xent_workspace_size(int64_t rows);
+lsq_status lsq_xent_fwd_bwd(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
+                            float* loss, void* dlogits, void* workspace, size_t workspace_bytes,
+                            lsq_cuda_stream stream);
+/* AdamW on n fp32 masters p with grads g and moments m, v (all device fp32);
+ * writes the bf16 operand copies p_bf16 (device, may be NULL).  step >= 1. */
+lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int32_t step,
+                          float lr, float beta1, float beta2, float eps, float weight_decay,
+                          lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Layer streaming scheduler.
+ *
+ * "The frozen base lives in CPU RAM and is streamed into two pre-allocated
+ * VRAM buffers one decoder layer at a time" (soup-cli diff, CHANGELOG
+ * [0.72.0]); `stream_buffers` 2..8, default 2 (docs "Layer Streaming");
+ * page-locked RAM is what lets the copy overlap compute (docs "NF4
+ * streaming", point 2); backward under gradient checkpointing re-streams the
+ * layers in reverse.  The scheduler owns only CUDA events and bookkeeping;
+ * the caller owns the slots (device), the records (host pinned) and both
+ * streams.  Every layer record has the same size.
+ * ---------------------------------------------------------------------- */
+typedef struct lsq_stream lsq_stream;
+
+typedef struct lsq_stream_cfg {
+  int32_t n_layers;                  /* >= 1 */
+  int32_t n_slots;                   /* 2..8 (or n_layers for a resident run) */
+  size_t record_bytes;               /* bytes per layer record, > 0 */
+  void* const* slots;                /* n_slots device pointers, 256-byte aligned, >= record_bytes each */
+  const void* const* host_records;   /* n_layers host pointers, page-locked */
+} lsq_stream_cfg;
+
+/* Creates the scheduler; ENOTPINNED if any record is not page-locked (the
+ * pages fall back to pageable memory silently; here it is an error). */
+lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stream compute, lsq_cuda_stream copy,
+                             lsq_stream** out);
+/* Enqueue on the copy stream: wait until the compute stream is done with the
+ * slot's previous occupant, copy layer's record into the slot, record the
+ * layer's upload event.  ESTATE if the slot holds the layer in current use. */
+lsq_status lsq_layer_upload_async(lsq_stream* st, int32_t layer, int32_t slot);
+/* Begin compute on `layer`, walking in `direction` (+1 forward, -1
+ * backward): release the previously stepped layer's slot after the compute
+ * work enqueued so far; upload `layer` if no slot holds it; make the compute
+ * stream wait for its upload; prefetch layer + direction into the least
+ * recently used other slot.  *slot_ptr = device address of the record. */
+lsq_status lsq_stream_step(lsq_stream* st, int32_t layer, int32_t direction, void** slot_ptr);
+/* Counters since create: uploads issued, bytes copied, uploads skipped
+ * because the layer was still resident. */
+lsq_status lsq_stream_stats(const lsq_stream* st, int64_t* uploads, int64_t* bytes, int64_t* reused);
+/* Device time (ms) of the last completed upload of `layer` (event pair on the
+ * copy stream); synchronises on that upload. */
+lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float* ms);
+/* Forget all residency (next step re-uploads); waits for pending copies. */
+lsq_status lsq_stream_reset(lsq_stream* st);
+lsq_status lsq_stream_destroy(lsq_stream* st);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSQ_H_ */

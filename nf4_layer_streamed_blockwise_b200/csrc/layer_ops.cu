@@ -1,0 +1,394 @@
+// Decoder-layer kernels around the NF4-LoRA linears (Llama / Qwen): RMSNorm,
+// RoPE, SwiGLU, embedding gather, causal-LM cross entropy, AdamW.  All are
+// HBM-bound streaming kernels: 16-byte vector accesses, one CTA per row for
+// the row reductions, fixed reduction trees (deterministic).
+#include "common.cuh"
+#include "host_common.h"
+
+namespace lsq {
+namespace ops {
+
+__device__ __forceinline__ void unpack8(uint4 v, float* f) {
+  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+// block-wide sum with a fixed tree; every thread gets the result
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) t += red[i];
+  return t;
+}
+
+constexpr int RN_T = 256;
+
+// ---------------------------------------------------------------- RMSNorm
+__global__ void __launch_bounds__(RN_T) rmsnorm_fwd_kernel(const uint4* __restrict__ x, const uint4* __restrict__ g,
+                                                           uint4* __restrict__ y, float* __restrict__ rstd, int d8,
+                                                           float inv_d, float eps) {
+  __shared__ float red[RN_T / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * d8;
+  float ss = 0.0f;
+  for (int c = threadIdx.x; c < d8; c += RN_T) {
+    float f[8];
+    unpack8(xr[c], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+  }
+  const float tot = block_sum<RN_T>(ss, red);
+  const float rs = 1.0f / sqrtf(tot * inv_d + eps);
+  if (threadIdx.x == 0 && rstd) rstd[row] = rs;
+  for (int c = threadIdx.x; c < d8; c += RN_T) {
+    float f[8], gv[8];
+    unpack8(xr[c], f);
+    unpack8(g[c], gv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = f[i] * rs * gv[i];
+    y[row * d8 + c] = pack8(f);
+  }
+}
+
+// dx = rs*(dy*g) - x * rs^3 * mean(dy*g*x);  out = dres_in + dx
+__global__ void __launch_bounds__(RN_T) rmsnorm_bwd_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ x,
+                                                           const uint4* __restrict__ g, const float* __restrict__ rstd,
+                                                           const uint4* dres_in, uint4* dres_out, int d8, float inv_d) {
+  __shared__ float red[RN_T / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * d8;
+  const uint4* dr = dy + row * d8;
+  float dot = 0.0f;
+  for (int c = threadIdx.x; c < d8; c += RN_T) {
+    float f[8], dv[8], gv[8];
+    unpack8(xr[c], f);
+    unpack8(dr[c], dv);
+    unpack8(g[c], gv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dot = fmaf(dv[i] * gv[i], f[i], dot);
+  }
+  const float tot = block_sum<RN_T>(dot, red);
+  const float rs = rstd[row];
+  const float k = rs * rs * rs * tot * inv_d;
+  for (int c = threadIdx.x; c < d8; c += RN_T) {
+    float f[8], dv[8], gv[8], o[8];
+    unpack8(xr[c], f);
+    unpack8(dr[c], dv);
+    unpack8(g[c], gv);
+    if (dres_in) unpack8(dres_in[row * d8 + c], o);
+    else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] += rs * dv[i] * gv[i] - f[i] * k;
+    dres_out[row * d8 + c] = pack8(o);
+  }
+}
+
+// ---------------------------------------------------------------- RoPE
+// one CTA per (batch, position): the hd/2 angles pos * theta^(-2i/hd) are
+// computed once in double, then every head at that position is rotated.
+__global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int seq, int heads, int hd,
+                                                   double log_theta, int inverse) {
+  extern __shared__ float cs[];  // [hd/2] cos, [hd/2] sin
+  const int half = hd / 2;
+  const int64_t bs = blockIdx.x;
+  const int pos = (int)(bs % seq);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double inv = exp(-2.0 * i / hd * log_theta);
+    double s, c;
+    sincos((double)pos * inv, &s, &c);
+    cs[i] = (float)c;
+    cs[half + i] = inverse ? -(float)s : (float)s;
+  }
+  __syncthreads();
+  __nv_bfloat16* base = x + bs * (int64_t)heads * hd;
+  for (int idx = threadIdx.x; idx < heads * half; idx += blockDim.x) {
+    const int h = idx / half, i = idx % half;
+    __nv_bfloat16* p = base + (int64_t)h * hd + i;
+    const float x1 = __bfloat162float(p[0]), x2 = __bfloat162float(p[half]);
+    const float c = cs[i], s = cs[half + i];
+    p[0] = __float2bfloat16_rn(x1 * c - x2 * s);
+    p[half] = __float2bfloat16_rn(x2 * c + x1 * s);
+  }
+}
+
+// ---------------------------------------------------------------- SwiGLU
+__device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf(-g)); }
+
+__global__ void __launch_bounds__(256) swiglu_fwd_kernel(const uint4* __restrict__ g, const uint4* __restrict__ u,
+                                                         uint4* __restrict__ m, int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    float gv[8], uv[8], o[8];
+    unpack8(g[i], gv);
+    unpack8(u[i], uv);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = gv[k] * sigmoidf_(gv[k]) * uv[k];
+    m[i] = pack8(o);
+  }
+}
+
+__global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint4* __restrict__ dm, const uint4* g, const uint4* u,
+                                                         uint4* dg, uint4* du, int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    float dv[8], gv[8], uv[8], og[8], ou[8];
+    unpack8(dm[i], dv);
+    unpack8(g[i], gv);
+    unpack8(u[i], uv);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float sg = sigmoidf_(gv[k]);
+      const float silu = gv[k] * sg;
+      ou[k] = dv[k] * silu;
+      og[k] = dv[k] * uv[k] * sg * (1.0f + gv[k] * (1.0f - sg));
+    }
+    dg[i] = pack8(og);
+    du[i] = pack8(ou);
+  }
+}
+
+// ---------------------------------------------------------------- embedding
+__global__ void __launch_bounds__(128) embed_kernel(const int32_t* __restrict__ ids, const uint4* __restrict__ table,
+                                                    uint4* __restrict__ h, int d8, int64_t vocab) {
+  const int64_t row = blockIdx.x;
+  const int32_t id = ids[row];
+  const bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) report(LSQ_EINVAL, 801);
+  for (int c = threadIdx.x; c < d8; c += blockDim.x)
+    h[row * d8 + c] = ok ? table[(int64_t)id * d8 + c] : make_uint4(0, 0, 0, 0);
+}
+
+// ---------------------------------------------------------------- cross entropy
+constexpr int XE_T = 512;
+
+// per row: lse, row loss, dlogits = (softmax - onehot) * inv_count
+__global__ void __launch_bounds__(XE_T) xent_row_kernel(const float* __restrict__ logits, const int32_t* __restrict__ ids,
+                                                        int seq, int64_t V, float inv_count,
+                                                        __nv_bfloat16* __restrict__ dlogits,
+                                                        float* __restrict__ row_loss) {
+  __shared__ float rm[XE_T / 32], rsum[XE_T / 32];
+  const int64_t row = blockIdx.x;
+  const int t = (int)(row % seq);
+  const float* lr = logits + row * V;
+  __nv_bfloat16* dr = dlogits + row * V;
+  if (t == seq - 1) {  // no next token: ignored row
+    for (int64_t c = threadIdx.x; c < V; c += XE_T) dr[c] = __float2bfloat16_rn(0.0f);
+    if (threadIdx.x == 0) row_loss[row] = 0.0f;
+    return;
+  }
+  const int32_t tgt = ids[row + 1];
+  float m = -INFINITY, s = 0.0f;
+  for (int64_t c = threadIdx.x; c < V; c += XE_T) {
+    const float v = lr[c];
+    if (v > m) {
+      s = s * expf(m - v) + 1.0f;
+      m = v;
+    } else {
+      s += expf(v - m);
+    }
+  }
+  // combine (m, s) pairs: warp tree, then a fixed pass over the warps
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float mm = fmaxf(m, m2);
+    s = (m == -INFINITY ? 0.0f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.0f : s2 * expf(m2 - mm));
+    m = mm;
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    rm[w] = m;
+    rsum[w] = s;
+  }
+  __syncthreads();
+  float M = -INFINITY, SS = 0.0f;
+  for (int i = 0; i < XE_T / 32; ++i) {
+    const float mm = fmaxf(M, rm[i]);
+    SS = (M == -INFINITY ? 0.0f : SS * expf(M - mm)) + (rm[i] == -INFINITY ? 0.0f : rsum[i] * expf(rm[i] - mm));
+    M = mm;
+  }
+  const float lse = M + logf(SS);
+  const bool tgt_ok = tgt >= 0 && tgt < V;
+  if (threadIdx.x == 0) {
+    if (!tgt_ok) report(LSQ_EINVAL, 802);
+    row_loss[row] = tgt_ok ? lse - lr[tgt] : 0.0f;
+  }
+  for (int64_t c = threadIdx.x; c < V; c += XE_T) {
+    float p = expf(lr[c] - lse);
+    if (c == tgt) p -= 1.0f;
+    dr[c] = __float2bfloat16_rn(p * inv_count);
+  }
+}
+
+__global__ void __launch_bounds__(1024) xent_mean_kernel(const float* __restrict__ row_loss, int64_t rows, float inv_count,
+                                                         float* __restrict__ loss) {
+  __shared__ float red[32];
+  float s = 0.0f;
+  for (int64_t i = threadIdx.x; i < rows; i += 1024) s += row_loss[i];
+  const float tot = block_sum<1024>(s, red);
+  if (threadIdx.x == 0) *loss = tot * inv_count;
+}
+
+// ---------------------------------------------------------------- AdamW
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                                    float* __restrict__ m, float* __restrict__ v,
+                                                    __nv_bfloat16* __restrict__ pb, int64_t n, float lr, float b1,
+                                                    float b2, float eps, float wd, float bc1, float bc2) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float gi = g[i];
+    const float mi = b1 * m[i] + (1.0f - b1) * gi;
+    const float vi = b2 * v[i] + (1.0f - b2) * gi * gi;
+    m[i] = mi;
+    v[i] = vi;
+    const float mh = mi / bc1, vh = vi / bc2;
+    const float pi = p[i] - lr * (mh / (sqrtf(vh) + eps) + wd * p[i]);
+    p[i] = pi;
+    if (pb) pb[i] = __float2bfloat16_rn(pi);
+  }
+}
+
+static unsigned grid_for(int64_t n, int threads) {
+  int64_t g = (n + threads - 1) / threads;
+  const int64_t cap = (int64_t)num_sms() * 32;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (unsigned)g;
+}
+
+}  // namespace ops
+}  // namespace lsq
+
+using namespace lsq;
+using namespace lsq::ops;
+
+extern "C" lsq_status lsq_rmsnorm_fwd(const void* x, const void* g, void* y, float* rstd, int64_t rows, int64_t d,
+                                      float eps, lsq_cuda_stream stream) {
+  if (!x || !g || !y) return fail(LSQ_EINVAL, "lsq_rmsnorm_fwd: NULL argument");
+  if (rows < 1 || d < 8 || d % 8 != 0) return fail(LSQ_EINVAL, "lsq_rmsnorm_fwd: need rows >= 1, d % 8 == 0");
+  if (!aligned(x, 16) || !aligned(g, 16) || !aligned(y, 16)) return fail(LSQ_EINVAL, "lsq_rmsnorm_fwd: alignment");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  rmsnorm_fwd_kernel<<<(unsigned)rows, RN_T, 0, (cudaStream_t)stream>>>(
+      (const uint4*)x, (const uint4*)g, (uint4*)y, rstd, (int)(d / 8), 1.0f / (float)d, eps);
+  LSQ_LAUNCH_CHECK("rmsnorm_fwd_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_rmsnorm_bwd(const void* dy, const void* x, const void* g, const float* rstd,
+                                      const void* dres_in, void* dres_out, int64_t rows, int64_t d,
+                                      lsq_cuda_stream stream) {
+  if (!dy || !x || !g || !rstd || !dres_out) return fail(LSQ_EINVAL, "lsq_rmsnorm_bwd: NULL argument");
+  if (rows < 1 || d < 8 || d % 8 != 0) return fail(LSQ_EINVAL, "lsq_rmsnorm_bwd: need rows >= 1, d % 8 == 0");
+  if (!aligned(dy, 16) || !aligned(x, 16) || !aligned(g, 16) || !aligned(dres_out, 16) ||
+      (dres_in && !aligned(dres_in, 16)))
+    return fail(LSQ_EINVAL, "lsq_rmsnorm_bwd: alignment");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  rmsnorm_bwd_kernel<<<(unsigned)rows, RN_T, 0, (cudaStream_t)stream>>>(
+      (const uint4*)dy, (const uint4*)x, (const uint4*)g, rstd, (const uint4*)dres_in, (uint4*)dres_out, (int)(d / 8),
+      1.0f / (float)d);
+  LSQ_LAUNCH_CHECK("rmsnorm_bwd_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t heads, int64_t hd, float theta,
+                               int32_t inverse, lsq_cuda_stream stream) {
+  if (!x) return fail(LSQ_EINVAL, "lsq_rope: NULL argument");
+  if (batch < 1 || seq < 1 || heads < 1 || hd < 2 || hd % 2 != 0 || hd > 1024 || !(theta > 1.0f))
+    return fail(LSQ_EINVAL, "lsq_rope: bad shape or theta");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  rope_kernel<<<(unsigned)(batch * seq), 128, (size_t)hd * sizeof(float), (cudaStream_t)stream>>>(
+      static_cast<__nv_bfloat16*>(x), (int)seq, (int)heads, (int)hd, log((double)theta), inverse ? 1 : 0);
+  LSQ_LAUNCH_CHECK("rope_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_swiglu_fwd(const void* g, const void* u, void* m, int64_t n, lsq_cuda_stream stream) {
+  if (!g || !u || !m) return fail(LSQ_EINVAL, "lsq_swiglu_fwd: NULL argument");
+  if (n < 8 || n % 8 != 0) return fail(LSQ_EINVAL, "lsq_swiglu_fwd: n must be a multiple of 8");
+  if (!aligned(g, 16) || !aligned(u, 16) || !aligned(m, 16)) return fail(LSQ_EINVAL, "lsq_swiglu_fwd: alignment");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  swiglu_fwd_kernel<<<grid_for(n / 8, 256), 256, 0, (cudaStream_t)stream>>>((const uint4*)g, (const uint4*)u,
+                                                                            (uint4*)m, n / 8);
+  LSQ_LAUNCH_CHECK("swiglu_fwd_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_swiglu_bwd(const void* dm, const void* g, const void* u, void* dg, void* du, int64_t n,
+                                     lsq_cuda_stream stream) {
+  if (!dm || !g || !u || !dg || !du) return fail(LSQ_EINVAL, "lsq_swiglu_bwd: NULL argument");
+  if (n < 8 || n % 8 != 0) return fail(LSQ_EINVAL, "lsq_swiglu_bwd: n must be a multiple of 8");
+  if (!aligned(dm, 16) || !aligned(g, 16) || !aligned(u, 16) || !aligned(dg, 16) || !aligned(du, 16))
+    return fail(LSQ_EINVAL, "lsq_swiglu_bwd: alignment");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  swiglu_bwd_kernel<<<grid_for(n / 8, 256), 256, 0, (cudaStream_t)stream>>>(
+      (const uint4*)dm, (const uint4*)g, (const uint4*)u, (uint4*)dg, (uint4*)du, n / 8);
+  LSQ_LAUNCH_CHECK("swiglu_bwd_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_embed_gather(const int32_t* ids, const void* table, void* h, int64_t rows, int64_t d,
+                                       int64_t vocab, lsq_cuda_stream stream) {
+  if (!ids || !table || !h) return fail(LSQ_EINVAL, "lsq_embed_gather: NULL argument");
+  if (rows < 1 || d < 8 || d % 8 != 0 || vocab < 1) return fail(LSQ_EINVAL, "lsq_embed_gather: bad shape");
+  if (!aligned(table, 16) || !aligned(h, 16)) return fail(LSQ_EINVAL, "lsq_embed_gather: alignment");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  embed_kernel<<<(unsigned)rows, 128, 0, (cudaStream_t)stream>>>(ids, (const uint4*)table, (uint4*)h, (int)(d / 8),
+                                                                 vocab);
+  LSQ_LAUNCH_CHECK("embed_kernel");
+  return LSQ_OK;
+}
+
+extern "C" size_t lsq_xent_workspace_size(int64_t rows) {
+  return (size_t)((rows > 0 ? rows : 1) * sizeof(float) + 255) / 256 * 256;
+}
+
+extern "C" lsq_status lsq_xent_fwd_bwd(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
+                                       float* loss, void* dlogits, void* workspace, size_t workspace_bytes,
+                                       lsq_cuda_stream stream) {
+  if (!logits || !ids || !loss || !dlogits || !workspace) return fail(LSQ_EINVAL, "lsq_xent_fwd_bwd: NULL argument");
+  if (batch < 1 || seq < 2 || V < 2) return fail(LSQ_EINVAL, "lsq_xent_fwd_bwd: need batch >= 1, seq >= 2, V >= 2");
+  const int64_t rows = batch * seq;
+  if (workspace_bytes < lsq_xent_workspace_size(rows)) return fail(LSQ_EINVAL, "lsq_xent_fwd_bwd: workspace too small");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  const float inv = 1.0f / (float)(batch * (seq - 1));
+  float* rl = static_cast<float*>(workspace);
+  xent_row_kernel<<<(unsigned)rows, XE_T, 0, (cudaStream_t)stream>>>(logits, ids, (int)seq, V, inv,
+                                                                     static_cast<__nv_bfloat16*>(dlogits), rl);
+  LSQ_LAUNCH_CHECK("xent_row_kernel");
+  xent_mean_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(rl, rows, inv, loss);
+  LSQ_LAUNCH_CHECK("xent_mean_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n,
+                                     int32_t step, float lr, float beta1, float beta2, float eps, float weight_decay,
+                                     lsq_cuda_stream stream) {
+  if (!p || !g || !m || !v) return fail(LSQ_EINVAL, "lsq_adamw_step: NULL argument");
+  if (n < 1 || step < 1) return fail(LSQ_EINVAL, "lsq_adamw_step: need n >= 1 and step >= 1");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  const float bc1 = (float)(1.0 - pow((double)beta1, (double)step));
+  const float bc2 = (float)(1.0 - pow((double)beta2, (double)step));
+  adamw_kernel<<<grid_for(n, 256), 256, 0, (cudaStream_t)stream>>>(p, g, m, v, static_cast<__nv_bfloat16*>(p_bf16), n,
+                                                                   lr, beta1, beta2, eps, weight_decay, bc1, bc2);
+  LSQ_LAUNCH_CHECK("adamw_kernel");
+  return LSQ_OK;
+}

@@ -1,0 +1,6 @@
+// Single translation unit of the lsq library (one device module, so every
+// kernel sees the same device status word without relocatable device code).
+#include "abi.cu"
+#include "nf4_quant.cu"
+#include "gemm_tc.cu"
+#include "lora_grad.cu"

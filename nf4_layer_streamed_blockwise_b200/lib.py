@@ -1,0 +1,343 @@
+"""ctypes binding of the lsq C ABI (include/lsq.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors (or raw ints for pointers) and passes their device addresses, sizes
+and the stream handle through.  No computation happens on this side.  The
+shared library is loaded from this package directory; if it is missing the
+import fails loudly (there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsq.so")
+
+c_void_p = ctypes.c_void_p
+c_int32 = ctypes.c_int32
+c_int64 = ctypes.c_int64
+c_float = ctypes.c_float
+c_size_t = ctypes.c_size_t
+
+STATUS = {0: "LSQ_OK", 1: "LSQ_EINVAL", 2: "LSQ_ENOTPINNED", 3: "LSQ_ECUDA", 4: "LSQ_ETIMEOUT",
+          5: "LSQ_ESTATE", 6: "LSQ_EUNSUPPORTED"}
+
+
+class LsqError(RuntimeError):
+    def __init__(self, status: int, fn: str, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class lsq_nf4_weight(ctypes.Structure):
+    _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
+
+
+class lsq_stream_cfg(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("n_slots", c_int32), ("record_bytes", c_size_t),
+                ("slots", ctypes.POINTER(c_void_p)), ("host_records", ctypes.POINTER(c_void_p))]
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m nf4_layer_streamed_blockwise_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_SIGS = {
+    "lsq_status_str": (ctypes.c_char_p, [c_int32]),
+    "lsq_last_error": (ctypes.c_char_p, []),
+    "lsq_version": (c_int32, []),
+    "lsq_device_status": (c_int32, [ctypes.POINTER(c_int32), ctypes.POINTER(c_int32)]),
+    "lsq_nf4_codebook": (c_int32, [ctypes.POINTER(c_float)]),
+    "lsq_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "lsq_nf4_dequantize": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p]),
+    "lsq_nf4_lora_fwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64, c_void_p, c_void_p, c_int32,
+                                   c_float, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "lsq_nf4_lora_fwd_multi": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
+                                         ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int32, c_float,
+                                         ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
+                                         ctypes.POINTER(c_void_p), c_void_p]),
+    "lsq_nf4_lora_bwd_workspace_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
+    "lsq_nf4_lora_bwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
+                                   c_int32, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
+                                   c_size_t, c_void_p]),
+    "lsq_nf4_lora_bwd_multi": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p,
+                                         ctypes.POINTER(c_void_p), c_int64, ctypes.POINTER(c_void_p),
+                                         ctypes.POINTER(c_void_p), c_int32, c_float, ctypes.POINTER(c_void_p),
+                                         c_void_p, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int32,
+                                         c_void_p, c_size_t, c_void_p]),
+    "lsq_dense_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32,
+                                 c_void_p]),
+    "lsq_rmsnorm_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_float, c_void_p]),
+    "lsq_rmsnorm_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                                  c_void_p]),
+    "lsq_rope": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int64, c_float, c_int32, c_void_p]),
+    "lsq_attention_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
+                                    c_int64, c_int64, c_void_p]),
+    "lsq_attention_bwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
+    "lsq_attention_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_int64, c_int64, c_int64, c_int64, c_int64, c_void_p, c_size_t,
+                                    c_void_p]),
+    "lsq_swiglu_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+    "lsq_swiglu_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+    "lsq_embed_gather": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p]),
+    "lsq_xent_workspace_size": (c_size_t, [c_int64]),
+    "lsq_xent_fwd_bwd": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                   c_size_t, c_void_p]),
+    "lsq_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_float,
+                                 c_float, c_float, c_float, c_float, c_void_p]),
+    "lsq_stream_create": (c_int32, [ctypes.POINTER(lsq_stream_cfg), c_void_p, c_void_p, ctypes.POINTER(c_void_p)]),
+    "lsq_layer_upload_async": (c_int32, [c_void_p, c_int32, c_int32]),
+    "lsq_stream_step": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_void_p)]),
+    "lsq_stream_stats": (c_int32, [c_void_p, ctypes.POINTER(c_int64), ctypes.POINTER(c_int64),
+                                   ctypes.POINTER(c_int64)]),
+    "lsq_stream_upload_ms": (c_int32, [c_void_p, c_int32, ctypes.POINTER(c_float)]),
+    "lsq_stream_reset": (c_int32, [c_void_p]),
+    "lsq_stream_destroy": (c_int32, [c_void_p]),
+}
+
+
+def _fn(name):
+    f = getattr(_lib, name)
+    res, args = _SIGS[name]
+    f.restype, f.argtypes = res, args
+    return f
+
+
+def exported_symbols() -> list:
+    """Names of the declared entry points that the loaded library exports."""
+    out = []
+    for name in _SIGS:
+        try:
+            getattr(_lib, name)
+            out.append(name)
+        except AttributeError:
+            pass
+    return out
+
+
+def _check(name: str, status: int):
+    if status != 0:
+        msg = _fn("lsq_last_error")().decode(errors="replace")
+        raise LsqError(status, name, msg)
+
+
+def _call(name, *args):
+    _check(name, _fn(name)(*args))
+
+
+def _p(t) -> Optional[int]:
+    """device / host address of a tensor (None for None; ints pass through)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptrs(seq) -> ctypes.Array:
+    arr = (c_void_p * len(seq))()
+    for i, t in enumerate(seq):
+        arr[i] = _p(t)
+    return arr
+
+
+class NF4Weight:
+    """Device views of one NF4 weight: codes uint8 [n_out*k_in/2], absmax fp32 [n_out*k_in/64]."""
+
+    def __init__(self, codes: torch.Tensor, absmax: torch.Tensor, n_out: int, k_in: int):
+        self.codes, self.absmax, self.n_out, self.k_in = codes, absmax, int(n_out), int(k_in)
+
+    def c(self) -> lsq_nf4_weight:
+        return lsq_nf4_weight(_p(self.codes), _p(self.absmax), self.n_out, self.k_in)
+
+    @staticmethod
+    def empty(n_out: int, k_in: int, device="cuda") -> "NF4Weight":
+        return NF4Weight(torch.empty(n_out * k_in // 2, dtype=torch.uint8, device=device),
+                         torch.empty(n_out * (k_in // 64), dtype=torch.float32, device=device), n_out, k_in)
+
+
+# ---------------------------------------------------------------------------- misc
+def lsq_status_str(s: int) -> str:
+    return _fn("lsq_status_str")(s).decode()
+
+
+def lsq_last_error() -> str:
+    return _fn("lsq_last_error")().decode(errors="replace")
+
+
+def lsq_version() -> int:
+    return _fn("lsq_version")()
+
+
+def lsq_device_status():
+    s, w = c_int32(0), c_int32(0)
+    _call("lsq_device_status", ctypes.byref(s), ctypes.byref(w))
+    return s.value, w.value
+
+
+def lsq_nf4_codebook():
+    out = (c_float * 16)()
+    _call("lsq_nf4_codebook", out)
+    return list(out)
+
+
+# ---------------------------------------------------------------------------- NF4
+def lsq_nf4_quantize(w_bf16: torch.Tensor, codes: torch.Tensor, absmax: torch.Tensor, stream=None):
+    n, k = w_bf16.shape
+    _call("lsq_nf4_quantize", _p(w_bf16), n, k, _p(codes), _p(absmax), _stream(stream))
+
+
+def lsq_nf4_dequantize(w: NF4Weight, out_bf16: torch.Tensor, stream=None):
+    cw = w.c()
+    _call("lsq_nf4_dequantize", ctypes.byref(cw), _p(out_bf16), _stream(stream))
+
+
+def lsq_nf4_lora_fwd(W: NF4Weight, x, M: int, A, B, r: int, s: float, residual, y, u_out, stream=None):
+    cw = W.c()
+    _call("lsq_nf4_lora_fwd", ctypes.byref(cw), _p(x), M, _p(A), _p(B), r, s, _p(residual), _p(y), _p(u_out),
+          _stream(stream))
+
+
+def lsq_nf4_lora_fwd_multi(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: float, residual, y, u_out,
+                           stream=None):
+    n = len(Ws)
+    cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
+    res = residual if residual is not None else [None] * n
+    uo = u_out if u_out is not None else [None] * n
+    _call("lsq_nf4_lora_fwd_multi", n, cws, _p(x), M, _ptrs(A), _ptrs(B), r, s, _ptrs(res), _ptrs(y), _ptrs(uo),
+          _stream(stream))
+
+
+def lsq_nf4_lora_bwd_workspace_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
+    arr = (c_int64 * len(n_outs))(*n_outs)
+    return int(_fn("lsq_nf4_lora_bwd_workspace_size")(len(n_outs), M, k_in, arr, r))
+
+
+def lsq_nf4_lora_bwd(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB, accumulate: int,
+                     workspace, stream=None):
+    cw = W.c()
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _call("lsq_nf4_lora_bwd", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
+          _p(dB), accumulate, _p(workspace), wsb, _stream(stream))
+
+
+def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB,
+                           accumulate: int, workspace, stream=None):
+    n = len(Ws)
+    cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _call("lsq_nf4_lora_bwd_multi", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(dx),
+          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream))
+
+
+def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int, stream=None):
+    _call("lsq_dense_gemm", _p(a), _p(b), _p(out), M, N, K, trans_b, out_f32, _stream(stream))
+
+
+# ---------------------------------------------------------------------------- layer ops
+def lsq_rmsnorm_fwd(x, g, y, rstd, rows: int, d: int, eps: float, stream=None):
+    _call("lsq_rmsnorm_fwd", _p(x), _p(g), _p(y), _p(rstd), rows, d, eps, _stream(stream))
+
+
+def lsq_rmsnorm_bwd(dy, x, g, rstd, dres_in, dres_out, rows: int, d: int, stream=None):
+    _call("lsq_rmsnorm_bwd", _p(dy), _p(x), _p(g), _p(rstd), _p(dres_in), _p(dres_out), rows, d, _stream(stream))
+
+
+def lsq_rope(x, batch: int, seq: int, heads: int, hd: int, theta: float, inverse: int, stream=None):
+    _call("lsq_rope", _p(x), batch, seq, heads, hd, theta, inverse, _stream(stream))
+
+
+def lsq_attention_fwd(q, k, v, o, lse, batch: int, seq: int, hq: int, hkv: int, hd: int, stream=None):
+    _call("lsq_attention_fwd", _p(q), _p(k), _p(v), _p(o), _p(lse), batch, seq, hq, hkv, hd, _stream(stream))
+
+
+def lsq_attention_bwd_workspace_size(batch: int, seq: int, hq: int) -> int:
+    return int(_fn("lsq_attention_bwd_workspace_size")(batch, seq, hq))
+
+
+def lsq_attention_bwd(q, k, v, o, lse, d_o, dq, dk, dv, batch: int, seq: int, hq: int, hkv: int, hd: int,
+                      workspace, stream=None):
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _call("lsq_attention_bwd", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(d_o), _p(dq), _p(dk), _p(dv), batch, seq,
+          hq, hkv, hd, _p(workspace), wsb, _stream(stream))
+
+
+def lsq_swiglu_fwd(g, u, m, n: int, stream=None):
+    _call("lsq_swiglu_fwd", _p(g), _p(u), _p(m), n, _stream(stream))
+
+
+def lsq_swiglu_bwd(dm, g, u, dg, du, n: int, stream=None):
+    _call("lsq_swiglu_bwd", _p(dm), _p(g), _p(u), _p(dg), _p(du), n, _stream(stream))
+
+
+def lsq_embed_gather(ids, table, h, rows: int, d: int, vocab: int, stream=None):
+    _call("lsq_embed_gather", _p(ids), _p(table), _p(h), rows, d, vocab, _stream(stream))
+
+
+def lsq_xent_workspace_size(rows: int) -> int:
+    return int(_fn("lsq_xent_workspace_size")(rows))
+
+
+def lsq_xent_fwd_bwd(logits, ids, batch: int, seq: int, V: int, loss, dlogits, workspace, stream=None):
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _call("lsq_xent_fwd_bwd", _p(logits), _p(ids), batch, seq, V, _p(loss), _p(dlogits), _p(workspace), wsb,
+          _stream(stream))
+
+
+def lsq_adamw_step(p, g, m, v, p_bf16, n: int, step: int, lr: float, beta1: float, beta2: float, eps: float,
+                   weight_decay: float, stream=None):
+    _call("lsq_adamw_step", _p(p), _p(g), _p(m), _p(v), _p(p_bf16), n, step, lr, beta1, beta2, eps, weight_decay,
+          _stream(stream))
+
+
+# ---------------------------------------------------------------------------- streaming
+def lsq_stream_create(n_layers: int, n_slots: int, record_bytes: int, slots: Sequence[int],
+                      host_records: Sequence[int], compute_stream, copy_stream) -> int:
+    sl = (c_void_p * len(slots))(*[_p(s) for s in slots])
+    hr = (c_void_p * len(host_records))(*[_p(h) for h in host_records])
+    cfg = lsq_stream_cfg(n_layers, n_slots, record_bytes, sl, hr)
+    out = c_void_p()
+    _call("lsq_stream_create", ctypes.byref(cfg), _stream(compute_stream), _stream(copy_stream), ctypes.byref(out))
+    return out.value
+
+
+def lsq_layer_upload_async(st: int, layer: int, slot: int):
+    _call("lsq_layer_upload_async", st, layer, slot)
+
+
+def lsq_stream_step(st: int, layer: int, direction: int) -> int:
+    out = c_void_p()
+    _call("lsq_stream_step", st, layer, direction, ctypes.byref(out))
+    return out.value
+
+
+def lsq_stream_stats(st: int):
+    a, b, c = c_int64(0), c_int64(0), c_int64(0)
+    _call("lsq_stream_stats", st, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    return a.value, b.value, c.value
+
+
+def lsq_stream_upload_ms(st: int, layer: int) -> float:
+    ms = c_float(0)
+    _call("lsq_stream_upload_ms", st, layer, ctypes.byref(ms))
+    return ms.value
+
+
+def lsq_stream_reset(st: int):
+    _call("lsq_stream_reset", st)
+
+
+def lsq_stream_destroy(st: int):
+    _call("lsq_stream_destroy", st)

@@ -1,0 +1,240 @@
+"""GPU parity of the NF4 quantiser and the fused NF4-LoRA linear against the oracle.
+
+Bit-exact: packed codes, absmax and dequantised bf16.  Tolerance (see
+tolerances.py): forward Y, U; backward dX, dA, dB; dense GEMMs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import lora_linear as OL
+from oracle import nf4 as ON
+from tolerances import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_quant(W_bf16: torch.Tensor):
+    return ON.quantize(W_bf16.float().numpy())
+
+
+def _gpu_quant(lsq, W_bf16: torch.Tensor):
+    n, k = W_bf16.shape
+    w = lsq.NF4Weight.empty(n, k)
+    lsq.lsq_nf4_quantize(W_bf16.cuda(), w.codes, w.absmax)
+    torch.cuda.synchronize()
+    return w
+
+
+def _f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("shape", [(512, 512), (8, 64), (24, 576), (1000, 128)])
+def test_quantize_bitexact(lsq, shape):
+    W = S.bf16_weight(*shape, stream=31 + shape[0])
+    w = _gpu_quant(lsq, W)
+    packed, am = _oracle_quant(W)
+    assert np.array_equal(w.codes.cpu().numpy(), packed)
+    assert np.array_equal(w.absmax.cpu().numpy().view(np.uint32), am.reshape(-1).view(np.uint32))
+
+
+def test_quantize_edge_cases_bitexact(lsq):
+    # every bf16 value in [-1, 1] against absmax 1 (a block holding +1 or -1),
+    # all-zero blocks, signed zeros and random absmax scales
+    vals = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = ON.bf16_bits_to_f32(vals)
+    f = f[np.isfinite(f) & (np.abs(f) <= 1.0)]
+    n_blocks = (f.size + 62) // 63
+    buf = np.zeros(n_blocks * 64, dtype=np.float32)
+    for b in range(n_blocks):
+        chunk = f[b * 63:(b + 1) * 63]
+        buf[b * 64] = 1.0 if b % 2 == 0 else -1.0
+        buf[b * 64 + 1:b * 64 + 1 + chunk.size] = chunk
+    rng = np.random.default_rng(0)
+    scaled = (buf.reshape(-1, 64) * ON.bf16_round(rng.uniform(1e-4, 30, size=(n_blocks, 1)).astype(np.float32)))
+    extra = np.zeros((4, 64), np.float32)
+    extra[1, 5] = -0.0
+    extra[2, :] = -0.0
+    extra[3, 7] = 3e-39                 # a subnormal
+    blocks = np.concatenate([buf.reshape(-1, 64), ON.bf16_round(scaled.astype(np.float32)), extra])
+    pad = (-blocks.shape[0]) % 8
+    blocks = np.concatenate([blocks, np.zeros((pad, 64), np.float32)]).reshape(-1, 64 * 8)
+    W = torch.from_numpy(np.ascontiguousarray(blocks)).to(torch.bfloat16)
+    w = _gpu_quant(lsq, W)
+    packed, am = _oracle_quant(W)
+    assert np.array_equal(w.codes.cpu().numpy(), packed)
+    assert np.array_equal(w.absmax.cpu().numpy().view(np.uint32), am.reshape(-1).view(np.uint32))
+
+
+def test_dequantize_bitexact(lsq):
+    W = S.bf16_weight(256, 512, stream=5)
+    w = _gpu_quant(lsq, W)
+    out = torch.empty(256, 512, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_nf4_dequantize(w, out)
+    packed, am = _oracle_quant(W)
+    ref = ON.dequantize(packed, am, 256, 512)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+
+
+def _lora_bf16(case):
+    return case["A"].to(torch.bfloat16), case["B"].to(torch.bfloat16)
+
+
+def _oracle_fwd(case, packed, am, residual=None):
+    N, K = case["W"].shape
+    Wd = ON.dequantize_f64(packed, am, N, K)
+    A, B = _lora_bf16(case)
+    Y, U = OL.lora_forward(_f64(case["X"]), Wd, _f64(A), _f64(B), case["s"])
+    if residual is not None:
+        Y = Y + _f64(residual)
+    return Y, U, Wd
+
+
+@pytest.mark.parametrize("M,N,K,r", [(64, 512, 512, 8), (200, 328, 192, 16), (1, 64, 64, 3), (300, 256, 1024, 64),
+                                     (130, 1536, 576, 8)])
+def test_fwd_matches_oracle(lsq, M, N, K, r):
+    case = S.linear_case(M, N, K, r, s=16.0 / r, seed=M + N)
+    w = _gpu_quant(lsq, case["W"])
+    A, B = _lora_bf16(case)
+    x = case["X"].cuda()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    u = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    lsq.lsq_nf4_lora_fwd(w, x, M, A.cuda(), B.cuda(), r, case["s"], None, y, u)
+    torch.cuda.synchronize()
+    Y, U, _ = _oracle_fwd(case, *_oracle_quant(case["W"]))
+    assert_close(y.float().cpu().numpy(), Y, what="Y")
+    assert_close(u.cpu().numpy(), U, rel=1e-5, max_rms=1e-4, what="U")
+
+
+def test_fwd_with_residual_and_no_lora(lsq):
+    M, N, K = 96, 264, 256
+    case = S.linear_case(M, N, K, 8)
+    w = _gpu_quant(lsq, case["W"])
+    res = S.bf16(S.normal_f32(9, 9, (M, N)))
+    y = res.clone().cuda()                      # residual aliases y
+    lsq.lsq_nf4_lora_fwd(w, case["X"].cuda(), M, None, None, 0, 0.0, y, y, None)
+    torch.cuda.synchronize()
+    packed, am = _oracle_quant(case["W"])
+    ref = _f64(case["X"]) @ ON.dequantize_f64(packed, am, N, K).T + _f64(res)
+    assert_close(y.float().cpu().numpy(), ref, what="Y+res")
+
+
+def test_b_zero_equals_base_bitwise(lsq):
+    M, N, K, r = 128, 512, 512, 8
+    case = S.linear_case(M, N, K, r)
+    w = _gpu_quant(lsq, case["W"])
+    x = case["X"].cuda()
+    A = case["A"].to(torch.bfloat16).cuda()
+    Bz = torch.zeros(N, r, dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty_like(y1)
+    lsq.lsq_nf4_lora_fwd(w, x, M, A, Bz, r, 2.0, None, y1, None)
+    lsq.lsq_nf4_lora_fwd(w, x, M, None, None, 0, 0.0, None, y2, None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_fwd_multi_segments(lsq):
+    M, K, r = 257, 320, 16
+    shapes = [(384, K), (128, K), (200, K)]
+    cases = [S.linear_case(M, n, K, r, s=1.0, seed=i) for i, (n, _) in enumerate(shapes)]
+    x = cases[0]["X"]
+    ws = [_gpu_quant(lsq, c["W"]) for c in cases]
+    As = [c["A"].to(torch.bfloat16).cuda() for c in cases]
+    Bs = [c["B"].to(torch.bfloat16).cuda() for c in cases]
+    ys = [torch.empty(M, n, dtype=torch.bfloat16, device="cuda") for n, _ in shapes]
+    us = [torch.empty(M, r, dtype=torch.float32, device="cuda") for _ in shapes]
+    lsq.lsq_nf4_lora_fwd_multi(ws, x.cuda(), M, As, Bs, r, 1.0, None, ys, us)
+    torch.cuda.synchronize()
+    for i, c in enumerate(cases):
+        c = dict(c, X=x)
+        Y, U, _ = _oracle_fwd(c, *_oracle_quant(c["W"]))
+        assert_close(ys[i].float().cpu().numpy(), Y, what=f"Y{i}")
+        assert_close(us[i].cpu().numpy(), U, rel=1e-5, max_rms=1e-4, what=f"U{i}")
+
+
+@pytest.mark.parametrize("M,N,K,r", [(64, 512, 512, 8), (200, 328, 192, 16), (77, 192, 576, 8), (260, 512, 1024, 64)])
+def test_bwd_matches_oracle(lsq, M, N, K, r):
+    case = S.linear_case(M, N, K, r, s=16.0 / r, seed=3 * M + N)
+    w = _gpu_quant(lsq, case["W"])
+    A, B = _lora_bf16(case)
+    x, dy = case["X"].cuda(), case["dY"].cuda()
+    u = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_nf4_lora_fwd(w, x, M, A.cuda(), B.cuda(), r, case["s"], None, y, u)
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lsq.lsq_nf4_lora_bwd_workspace_size([N], M, K, r), dtype=torch.uint8, device="cuda")
+    lsq.lsq_nf4_lora_bwd(w, x, dy, M, A.cuda(), B.cuda(), r, case["s"], u, dx, dA, dB, 0, ws)
+    torch.cuda.synchronize()
+    packed, am = _oracle_quant(case["W"])
+    Wd = ON.dequantize_f64(packed, am, N, K)
+    rdX, rdA, rdB, _ = OL.lora_backward(_f64(case["X"]), Wd, _f64(A), _f64(B), case["s"], _f64(case["dY"]))
+    assert_close(dx.float().cpu().numpy(), rdX, what="dX")
+    assert_close(dA.cpu().numpy(), rdA, what="dA")
+    assert_close(dB.cpu().numpy(), rdB, what="dB")
+    # accumulate = 1 adds into the existing gradients
+    lsq.lsq_nf4_lora_bwd(w, x, dy, M, A.cuda(), B.cuda(), r, case["s"], u, None, dA, dB, 1, ws)
+    torch.cuda.synchronize()
+    assert_close(dA.cpu().numpy(), 2 * rdA, what="2dA")
+    assert_close(dB.cpu().numpy(), 2 * rdB, what="2dB")
+
+
+def test_bwd_multi_segments_sum(lsq):
+    M, K, r = 200, 256, 16
+    ns = [256, 64, 192]
+    cases = [S.linear_case(M, n, K, r, s=1.0, seed=10 + i) for i, n in enumerate(ns)]
+    x = cases[0]["X"]
+    ws_ = [_gpu_quant(lsq, c["W"]) for c in cases]
+    As = [c["A"].to(torch.bfloat16) for c in cases]
+    Bs = [c["B"].to(torch.bfloat16) for c in cases]
+    us, dys = [], []
+    for i, c in enumerate(cases):
+        u = torch.from_numpy((_f64(x) @ _f64(As[i]).T).astype(np.float32)).cuda()
+        us.append(u)
+        dys.append(c["dY"].cuda())
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dA = [torch.empty(r, K, dtype=torch.float32, device="cuda") for _ in ns]
+    dB = [torch.empty(n, r, dtype=torch.float32, device="cuda") for n in ns]
+    wsb = torch.empty(lsq.lsq_nf4_lora_bwd_workspace_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
+    lsq.lsq_nf4_lora_bwd_multi(ws_, x.cuda(), dys, M, [a.cuda() for a in As], [b.cuda() for b in Bs], r, 1.0, us, dx,
+                               dA, dB, 0, wsb)
+    torch.cuda.synchronize()
+    rdx = 0
+    for i, c in enumerate(cases):
+        packed, am = _oracle_quant(c["W"])
+        Wd = ON.dequantize_f64(packed, am, ns[i], K)
+        d_x, d_a, d_b, _ = OL.lora_backward(_f64(x), Wd, _f64(As[i]), _f64(Bs[i]), 1.0, _f64(c["dY"]))
+        rdx = rdx + d_x
+        assert_close(dA[i].cpu().numpy(), d_a, what=f"dA{i}")
+        assert_close(dB[i].cpu().numpy(), d_b, what=f"dB{i}")
+    assert_close(dx.float().cpu().numpy(), rdx, what="dX sum")
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 1000, 576), (64, 4096, 128)])
+@pytest.mark.parametrize("trans_b", [0, 1])
+def test_dense_gemm(lsq, M, N, K, trans_b):
+    a = S.bf16(S.normal_f32(7, 1, (M, K)))
+    b = S.bf16(S.normal_f32(7, 2, (K, N) if trans_b else (N, K), 0.05))
+    ref = _f64(a) @ (_f64(b) if trans_b else _f64(b).T)
+    for out_f32 in (1, 0):
+        out = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+        lsq.lsq_dense_gemm(a.cuda(), b.cuda(), out, M, N, K, trans_b, out_f32)
+        torch.cuda.synchronize()
+        tol = 5e-5 if out_f32 else 5e-3
+        assert_close(out.float().cpu().numpy(), ref, rel=tol, max_rms=2e-2, what=f"dense f32={out_f32}")
+
+
+def test_bad_arguments_rejected_before_launch(lsq):
+    w = lsq.NF4Weight.empty(64, 64)
+    x = torch.empty(4, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(4, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lsq.LsqError) as e:
+        lsq.lsq_nf4_lora_fwd(lsq.NF4Weight(w.codes, w.absmax, 64, 96), x, 4, None, None, 0, 0.0, None, y, None)
+    assert e.value.status == 1
+    with pytest.raises(lsq.LsqError):
+        lsq.lsq_nf4_lora_fwd(w, x, 4, None, None, 65, 1.0, None, y, None)
+    assert lsq.lsq_device_status() == (0, 0)

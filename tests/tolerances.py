@@ -1,0 +1,30 @@
+"""Acceptance tolerances for floating-point parity against the fp64 oracle.
+
+GEMM / LoRA outputs and gradients: relative Frobenius error <= 5e-3 and max
+elementwise error <= 2e-2 x RMS(reference).  The CUDA path multiplies bf16
+operands exactly and accumulates in fp32, then rounds the output to bf16
+once: the bf16 rounding alone is a relative error of at most 2^-9 ~ 2e-3 per
+element, which is what the 5e-3 Frobenius bound leaves room for.
+"""
+import numpy as np
+
+REL_FRO = 5e-3
+MAX_ABS_RMS = 2e-2
+
+
+def rel_fro(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def assert_close(got, ref, rel=REL_FRO, max_rms=MAX_ABS_RMS, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    rf = rel_fro(got, ref)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    mx = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    assert rf <= rel, f"{what}: relative Frobenius error {rf:.3e} > {rel:.1e}"
+    assert mx <= max_rms * rms + 1e-30, f"{what}: max error {mx:.3e} > {max_rms:.0e} x RMS {rms:.3e}"
