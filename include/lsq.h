@@ -162,7 +162,7 @@ lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
  * "NF4 streaming").  tcgen05, fp32 accumulation.
  *  trans_b = 0:  out[M,N] = a[M,K] b[N,K]^T   (logits = h E^T)
  *  trans_b = 1:  out[M,N] = a[M,K] b[K,N]     (dh = dlogits E)
- *  out_f32 = 1: fp32 output, else bf16.  K % 64 == 0, N % 8 == 0. */
+ *  out_f32 = 1: fp32 output, else bf16.  K % 8 == 0, N % 8 == 0. */
 lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, int64_t M, int64_t N, int64_t K,
                           int32_t trans_b, int32_t out_f32, lsq_cuda_stream stream);
 

@@ -622,8 +622,11 @@ extern "C" lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, in
                                      int32_t trans_b, int32_t out_f32, lsq_cuda_stream stream) {
   const char* who = "lsq_dense_gemm";
   if (!a || !b || !out) return fail(LSQ_EINVAL, "%s: NULL argument", who);
-  lsq_status st = common_checks(M, K, 0, who);
+  lsq_status st = check_device();
   if (st != LSQ_OK) return st;
+  if (M < 1 || M > (1 << 30)) return fail(LSQ_EINVAL, "%s: M out of range (%lld)", who, (long long)M);
+  if (K < 8 || K % 8 != 0 || K > (1 << 30))
+    return fail(LSQ_EINVAL, "%s: K must be a positive multiple of 8 (got %lld)", who, (long long)K);
   if (N < 8 || N % 8 != 0 || N > (1 << 30)) return fail(LSQ_EINVAL, "%s: N must be a positive multiple of 8", who);
   if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16))
     return fail(LSQ_EINVAL, "%s: operands must be 16-byte aligned", who);
@@ -635,7 +638,7 @@ extern "C" lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, in
   p.N = (int)N;
   p.out = out;
   p.out_f32 = out_f32 ? 1 : 0;
-  p.nkb = (int)(K / BK);
+  p.nkb = (int)((K + BK - 1) / BK);  // the K tail reads as zeros (TMA out-of-bounds fill)
   Maps maps;
   memset(&maps, 0, sizeof(maps));
   if ((st = encode_tmap_2d(&maps.a[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, K, M, K * 2, BK, BM,

@@ -4,3 +4,6 @@
 #include "nf4_quant.cu"
 #include "gemm_tc.cu"
 #include "lora_grad.cu"
+#include "layer_ops.cu"
+#include "attention.cu"
+#include "stream.cu"

@@ -125,8 +125,18 @@ def _check(name: str, status: int):
         raise LsqError(status, name, msg)
 
 
-def _call(name, *args):
+# kernel launches issued by the library, counted per call on this side
+# (lsq_nf4_lora_bwd: the dX GEMM plus two reduction kernels for each of dA, dB)
+LAUNCHES = [0]
+_KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_nf4_lora_fwd": 1, "lsq_nf4_lora_fwd_multi": 1,
+            "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
+            "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
+            "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1}
+
+
+def _call(name, *args, launches=None):
     _check(name, _fn(name)(*args))
+    LAUNCHES[0] += _KERNELS.get(name, 0) if launches is None else launches
 
 
 def _p(t) -> Optional[int]:
@@ -230,7 +240,7 @@ def lsq_nf4_lora_bwd(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx,
     cw = W.c()
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
-          _p(dB), accumulate, _p(workspace), wsb, _stream(stream))
+          _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (4 if r > 0 else 0))
 
 
 def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB,
@@ -239,7 +249,7 @@ def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int,
     cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd_multi", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(dx),
-          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream))
+          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (4 * n if r > 0 else 0))
 
 
 def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int, stream=None):

@@ -1,0 +1,375 @@
+"""Streamed NF4-LoRA training step on one GPU, sequenced over the lsq C ABI.
+
+The method (soup-cli 0.72.0 -> 0.72.2 diff, CHANGELOG [0.72.2] and docs
+"Layer Streaming" / "NF4 streaming"; "Soup" README headline): the frozen base
+is quantised once, offline, to NF4 and kept in page-locked host RAM as one
+record per decoder layer; each training step streams the records through a
+small ring of HBM slots, forward 0 -> L-1, and under gradient checkpointing
+re-streams them L-1 -> 0 for the backward, recomputing each layer from its
+saved input; embed_tokens and lm_head stay resident and unquantised; only the
+LoRA adapters train (optimizer step at the end).
+
+This module only allocates memory (torch), builds the host store and calls
+the library in order.  Every arithmetic step runs in the library's kernels.
+
+Layer record layout (bytes, each piece 256-byte aligned): NF4 codes of
+q, k, v, o, gate, up, down; then their fp32 absmax arrays in the same order;
+then the two RMSNorm gains (bf16 [d] each).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import torch
+
+import synthetic as S
+from . import lib as L
+
+ALIGN = 256
+
+
+def _al(n: int, a: int = ALIGN) -> int:
+    return (n + a - 1) // a * a
+
+
+@dataclasses.dataclass
+class RecordLayout:
+    """Byte offsets of one layer record."""
+    codes: Dict[str, int]
+    absmax: Dict[str, int]
+    ln1: int
+    ln2: int
+    nbytes: int
+
+    @staticmethod
+    def of(shape: S.ModelShape) -> "RecordLayout":
+        off = 0
+        codes, absmax = {}, {}
+        for name, (n, k) in shape.linear_shapes().items():
+            codes[name] = off
+            off = _al(off + n * k // 2)
+        for name, (n, k) in shape.linear_shapes().items():
+            absmax[name] = off
+            off = _al(off + n * (k // 64) * 4)
+        ln1 = off
+        off = _al(off + shape.d * 2)
+        ln2 = off
+        off = _al(off + shape.d * 2)
+        return RecordLayout(codes, absmax, ln1, ln2, _al(off, 4096))
+
+
+class LayerView:
+    """Typed device views into one layer record that sits in an HBM slot."""
+
+    def __init__(self, shape: S.ModelShape, lay: RecordLayout, base: int):
+        self.W = {}
+        for name, (n, k) in shape.linear_shapes().items():
+            self.W[name] = L.NF4Weight(base + lay.codes[name], base + lay.absmax[name], n, k)
+        self.ln1 = base + lay.ln1
+        self.ln2 = base + lay.ln2
+
+
+class LoraParams:
+    """All LoRA tensors of the stack in flat buffers: fp32 masters, grads, AdamW
+    moments, and the bf16 operand copies the kernels read."""
+
+    def __init__(self, shape: S.ModelShape, device="cuda"):
+        self.shape = shape
+        self.offsets = []  # per layer: {name: {"A": (off, (r, K)), "B": (off, (N, r))}}
+        off = 0
+        for _ in range(shape.n_layers):
+            per = {}
+            for name, (n, k) in shape.linear_shapes().items():
+                per[name] = {"A": (off, (shape.r, k))}
+                off = _al(off + shape.r * k, 64)
+                per[name]["B"] = (off, (n, shape.r))
+                off = _al(off + n * shape.r, 64)
+            self.offsets.append(per)
+        self.numel = off
+        self.master = torch.zeros(off, dtype=torch.float32, device=device)
+        self.grad = torch.zeros(off, dtype=torch.float32, device=device)
+        self.m = torch.zeros(off, dtype=torch.float32, device=device)
+        self.v = torch.zeros(off, dtype=torch.float32, device=device)
+        self.op = torch.zeros(off, dtype=torch.bfloat16, device=device)
+        self.step = 0
+
+    def view(self, buf: torch.Tensor, l: int, name: str, ab: str) -> torch.Tensor:
+        o, shp = self.offsets[l][name][ab]
+        return buf[o:o + shp[0] * shp[1]].view(*shp)
+
+    def init_host(self):
+        """Masters from the seeded numpy streams (reproducible by the oracle)."""
+        for l, per in enumerate(S.lora_init(self.shape)):
+            for name, t in per.items():
+                for ab in ("A", "B"):
+                    self.view(self.master, l, name, ab).copy_(t[ab])
+        self.op.copy_(self.master)
+
+    def init_device(self, seed: int = S.LORA_SEED):
+        for l in range(self.shape.n_layers):
+            for i, (name, (n, k)) in enumerate(self.shape.linear_shapes().items()):
+                st = 1000 + 16 * l + i
+                self.view(self.master, l, name, "A").copy_(
+                    S.device_normal_f32((self.shape.r, k), 1.0 / math.sqrt(k), seed, st))
+                self.view(self.master, l, name, "B").copy_(
+                    S.device_normal_f32((n, self.shape.r), S.LORA_B_STD, seed, st + 8))
+        self.op.copy_(self.master)
+
+
+class StreamedLoraTrainer:
+    """One GPU, one batch of [batch, seq] token ids per step.
+
+    n_slots: HBM slots for streamed layer records (2..8), or None for a
+    resident run (one slot per layer, every layer uploaded once).
+    init: "host" draws every weight from the seeded numpy streams that the
+    oracle also reads; "device" draws them with the CUDA RNG (full-size runs).
+    """
+
+    def __init__(self, shape: S.ModelShape, batch: int, seq: int, n_slots: Optional[int] = 2,
+                 init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None):
+        self.shape, self.B, self.S = shape, batch, seq
+        self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
+        self.M = batch * seq
+        self.lr = lr
+        self.dev = device
+        self.resident = n_slots is None
+        self.n_slots = shape.n_layers if self.resident else int(n_slots)
+        self.layout = RecordLayout.of(shape)
+        self.compute = torch.cuda.current_stream()
+        self.copy = torch.cuda.Stream()
+        if share is not None:       # reuse another trainer's host store and resident tensors
+            self.host_records = share.host_records
+            self.embed, self.lm_head, self.final_norm = share.embed, share.lm_head, share.final_norm
+        else:
+            self._build_store(init)
+            self._build_resident(init)
+        self.lora = LoraParams(shape, device)
+        if init == "host":
+            self.lora.init_host()
+        else:
+            self.lora.init_device()
+        self._alloc_activations()
+        self.slots = [torch.empty(self.layout.nbytes, dtype=torch.uint8, device=device) for _ in range(self.n_slots)]
+        self.sched = L.lsq_stream_create(shape.n_layers, self.n_slots, self.layout.nbytes,
+                                         [s.data_ptr() for s in self.slots],
+                                         [h.data_ptr() for h in self.host_records], self.compute, self.copy)
+        if self.resident:
+            for l in range(shape.n_layers):
+                L.lsq_layer_upload_async(self.sched, l, l)
+            torch.cuda.synchronize()
+        self.loss_dev = torch.zeros(1, dtype=torch.float32, device=device)
+
+    # ------------------------------------------------------------------ setup
+    def _build_store(self, init: str):
+        """Quantise every layer once on the GPU and keep the records pinned on the host."""
+        sh, lay = self.shape, self.layout
+        stage = torch.zeros(lay.nbytes, dtype=torch.uint8, device=self.dev)
+        base = stage.data_ptr()
+        self.host_records: List[torch.Tensor] = []
+        for l in range(sh.n_layers):
+            if init == "host":
+                Wl = S.layer_weights(sh, l)
+            for i, (name, (n, k)) in enumerate(sh.linear_shapes().items()):
+                if init == "host":
+                    w = Wl[name].to(self.dev)
+                else:
+                    w = S.device_normal_bf16((n, k), S.BASE_STD, S.WEIGHT_SEED, 1000 + 16 * l + i)
+                L.lsq_nf4_quantize(w, base + lay.codes[name], base + lay.absmax[name])
+                del w
+            ones = torch.ones(sh.d, dtype=torch.bfloat16, device=self.dev)
+            stage[lay.ln1:lay.ln1 + 2 * sh.d].copy_(ones.view(torch.uint8))
+            stage[lay.ln2:lay.ln2 + 2 * sh.d].copy_(ones.view(torch.uint8))
+            rec = torch.empty(lay.nbytes, dtype=torch.uint8, pin_memory=True)
+            rec.copy_(stage)
+            self.host_records.append(rec)
+        del stage
+        torch.cuda.synchronize()
+
+    def _build_resident(self, init: str):
+        sh = self.shape
+        if init == "host":
+            e = S.embeddings(sh)
+            self.embed = e["embed"].to(self.dev)
+            self.lm_head = self.embed if sh.tied else e["lm_head"].to(self.dev)
+        else:
+            self.embed = S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD, S.WEIGHT_SEED, 11)
+            self.lm_head = self.embed if sh.tied else S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD,
+                                                                            S.WEIGHT_SEED, 12)
+        self.final_norm = torch.ones(sh.d, dtype=torch.bfloat16, device=self.dev)
+
+    def _alloc_activations(self):
+        sh, M, dev = self.shape, self.M, self.dev
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        d, f, kv, r = sh.d, sh.f, sh.kv, sh.r
+        self.ids = torch.zeros(M, dtype=torch.int32, device=dev)
+        self.h = torch.empty(sh.n_layers + 1, M, d, **bf)        # checkpointed layer inputs
+        self.x1, self.q, self.a, self.hmid, self.x2 = (torch.empty(M, d, **bf) for _ in range(5))
+        self.k, self.v = torch.empty(M, kv, **bf), torch.empty(M, kv, **bf)
+        self.g, self.u, self.mm = (torch.empty(M, f, **bf) for _ in range(3))
+        self.rstd1, self.rstd2, self.rstdf = (torch.empty(M, **f32) for _ in range(3))
+        self.lse = torch.empty(self.B * sh.n_q * self.S, **f32)
+        self.U = {n: torch.empty(M, r, **f32) for n in S.LINEARS}
+        self.dh, self.dhmid, self.dx, self.dq, self.da = (torch.empty(M, d, **bf) for _ in range(5))
+        self.dk, self.dv = torch.empty(M, kv, **bf), torch.empty(M, kv, **bf)
+        self.dmm = torch.empty(M, f, **bf)
+        self.hn = torch.empty(M, d, **bf)
+        self.logits = torch.empty(M, sh.vocab, **f32)
+        self.dlogits = torch.empty(M, sh.vocab, **bf)
+        ws = max(L.lsq_nf4_lora_bwd_workspace_size([d, kv, kv], M, d, r),
+                 L.lsq_nf4_lora_bwd_workspace_size([d], M, d, r),
+                 L.lsq_nf4_lora_bwd_workspace_size([f, f], M, d, r),
+                 L.lsq_nf4_lora_bwd_workspace_size([d], M, f, r))
+        self.ws_lora = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.ws_attn = torch.empty(L.lsq_attention_bwd_workspace_size(self.B, self.S, sh.n_q), dtype=torch.uint8,
+                                   device=dev)
+        self.ws_xent = torch.empty(L.lsq_xent_workspace_size(M), dtype=torch.uint8, device=dev)
+
+    # ------------------------------------------------------------------ timing
+    def _t0(self):
+        if self.timeline is None:
+            return None
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.compute)
+        return e
+
+    def _t1(self, start, kind: str, flops: float):
+        if start is None:
+            return
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.compute)
+        self.timeline.append((kind, flops, start, e))
+
+    def _fwd_flops(self, ns, K):
+        M, r = self.M, self.shape.r
+        return sum(2.0 * M * n * K + 2.0 * M * r * K + 2.0 * M * n * r for n in ns)
+
+    def _bwd_flops(self, ns, K):
+        M, r = self.M, self.shape.r
+        return sum(2.0 * M * n * K + 2.0 * M * n * r + 2.0 * M * r * K for n in ns)
+
+    # ------------------------------------------------------------------ layer
+    def _ops(self, l: int):
+        lp = self.lora
+        A = {n: lp.view(lp.op, l, n, "A") for n in S.LINEARS}
+        B = {n: lp.view(lp.op, l, n, "B") for n in S.LINEARS}
+        return A, B
+
+    def _layer_fwd(self, l: int, W: LayerView, save: bool):
+        sh, M, r, s = self.shape, self.M, self.shape.r, self.shape.s
+        A, B = self._ops(l)
+        hin, hout = self.h[l], self.h[l + 1]
+        U = self.U if save else {n: None for n in S.LINEARS}
+        L.lsq_rmsnorm_fwd(hin, W.ln1, self.x1, self.rstd1, M, sh.d, sh.eps)
+        t = self._t0()
+        L.lsq_nf4_lora_fwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, M, [A["q"], A["k"], A["v"]],
+                                 [B["q"], B["k"], B["v"]], r, s, None, [self.q, self.k, self.v],
+                                 [U["q"], U["k"], U["v"]])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d))
+        L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
+        L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
+        L.lsq_attention_fwd(self.q, self.k, self.v, self.a, self.lse, self.B, self.S, sh.n_q, sh.n_kv, sh.hd)
+        t = self._t0()
+        L.lsq_nf4_lora_fwd(W.W["o"], self.a, M, A["o"], B["o"], r, s, hin, self.hmid, U["o"])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d))
+        L.lsq_rmsnorm_fwd(self.hmid, W.ln2, self.x2, self.rstd2, M, sh.d, sh.eps)
+        t = self._t0()
+        L.lsq_nf4_lora_fwd_multi([W.W["gate"], W.W["up"]], self.x2, M, [A["gate"], A["up"]], [B["gate"], B["up"]],
+                                 r, s, None, [self.g, self.u], [U["gate"], U["up"]])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d))
+        L.lsq_swiglu_fwd(self.g, self.u, self.mm, M * sh.f)
+        t = self._t0()
+        L.lsq_nf4_lora_fwd(W.W["down"], self.mm, M, A["down"], B["down"], r, s, self.hmid, hout, U["down"])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f))
+
+    def _layer_bwd(self, l: int, W: LayerView):
+        """self.dh holds dLoss/dh[l+1] on entry and dLoss/dh[l] on exit."""
+        sh, M, r, s = self.shape, self.M, self.shape.r, self.shape.s
+        A, B = self._ops(l)
+        lp = self.lora
+        gA = {n: lp.view(lp.grad, l, n, "A") for n in S.LINEARS}
+        gB = {n: lp.view(lp.grad, l, n, "B") for n in S.LINEARS}
+        U = self.U
+        # down:  h_out = h_mid + down(m)
+        t = self._t0()
+        L.lsq_nf4_lora_bwd(W.W["down"], self.mm, self.dh, M, A["down"], B["down"], r, s, U["down"], self.dmm,
+                           gA["down"], gB["down"], 0, self.ws_lora)
+        self._t1(t, "nf4_bwd", self._bwd_flops([sh.d], sh.f))
+        L.lsq_swiglu_bwd(self.dmm, self.g, self.u, self.g, self.u, M * sh.f)   # g, u <- dg, du
+        t = self._t0()
+        L.lsq_nf4_lora_bwd_multi([W.W["gate"], W.W["up"]], self.x2, [self.g, self.u], M, [A["gate"], A["up"]],
+                                 [B["gate"], B["up"]], r, s, [U["gate"], U["up"]], self.dx,
+                                 [gA["gate"], gA["up"]], [gB["gate"], gB["up"]], 0, self.ws_lora)
+        self._t1(t, "nf4_bwd", self._bwd_flops([sh.f, sh.f], sh.d))
+        L.lsq_rmsnorm_bwd(self.dx, self.hmid, W.ln2, self.rstd2, self.dh, self.dhmid, M, sh.d)
+        # o:  h_mid = h_in + o(a)
+        t = self._t0()
+        L.lsq_nf4_lora_bwd(W.W["o"], self.a, self.dhmid, M, A["o"], B["o"], r, s, U["o"], self.da, gA["o"],
+                           gB["o"], 0, self.ws_lora)
+        self._t1(t, "nf4_bwd", self._bwd_flops([sh.d], sh.d))
+        L.lsq_attention_bwd(self.q, self.k, self.v, self.a, self.lse, self.da, self.dq, self.dk, self.dv, self.B,
+                            self.S, sh.n_q, sh.n_kv, sh.hd, self.ws_attn)
+        L.lsq_rope(self.dq, self.B, self.S, sh.n_q, sh.hd, sh.theta, 1)
+        L.lsq_rope(self.dk, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 1)
+        t = self._t0()
+        L.lsq_nf4_lora_bwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, [self.dq, self.dk, self.dv], M,
+                                 [A["q"], A["k"], A["v"]], [B["q"], B["k"], B["v"]], r, s,
+                                 [U["q"], U["k"], U["v"]], self.dx, [gA["q"], gA["k"], gA["v"]],
+                                 [gB["q"], gB["k"], gB["v"]], 0, self.ws_lora)
+        self._t1(t, "nf4_bwd", self._bwd_flops([sh.d, sh.kv, sh.kv], sh.d))
+        L.lsq_rmsnorm_bwd(self.dx, self.h[l], W.ln1, self.rstd1, self.dhmid, self.dh, M, sh.d)
+
+    def _view(self, l: int, direction: int) -> LayerView:
+        return LayerView(self.shape, self.layout, L.lsq_stream_step(self.sched, l, direction))
+
+    # ------------------------------------------------------------------ step
+    def set_ids(self, ids: torch.Tensor):
+        self.ids.copy_(ids.reshape(-1).to(torch.int32), non_blocking=True)
+
+    def forward_backward(self):
+        """Loss into self.loss_dev and LoRA gradients into self.lora.grad."""
+        sh, M = self.shape, self.M
+        L.lsq_embed_gather(self.ids, self.embed, self.h[0], M, sh.d, sh.vocab)
+        for l in range(sh.n_layers):
+            self._layer_fwd(l, self._view(l, +1), save=False)
+        L.lsq_rmsnorm_fwd(self.h[sh.n_layers], self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
+        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        L.lsq_xent_fwd_bwd(self.logits, self.ids, self.B, self.S, sh.vocab, self.loss_dev, self.dlogits,
+                           self.ws_xent)
+        L.lsq_dense_gemm(self.dlogits, self.lm_head, self.hn, M, sh.d, sh.vocab, 1, 0)   # hn <- d hn
+        L.lsq_rmsnorm_bwd(self.hn, self.h[sh.n_layers], self.final_norm, self.rstdf, None, self.dh, M, sh.d)
+        for l in reversed(range(sh.n_layers)):
+            W = self._view(l, -1)
+            self._layer_fwd(l, W, save=True)
+            self._layer_bwd(l, W)
+
+    def optimizer_step(self):
+        lp = self.lora
+        lp.step += 1
+        L.lsq_adamw_step(lp.master, lp.grad, lp.m, lp.v, lp.op, lp.numel, lp.step, self.lr, 0.9, 0.999, 1e-8, 0.0)
+
+    def train_step(self, ids: Optional[torch.Tensor] = None):
+        if ids is not None:
+            self.set_ids(ids)
+        self.forward_backward()
+        self.optimizer_step()
+
+    def logits_of_last_forward(self) -> torch.Tensor:
+        return self.logits
+
+    def stats(self):
+        return L.lsq_stream_stats(self.sched)
+
+    def close(self):
+        if getattr(self, "sched", None):
+            torch.cuda.synchronize()
+            L.lsq_stream_destroy(self.sched)
+            self.sched = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -85,7 +85,7 @@ QWEN3B = ModelShape("qwen2.5-3b", 36, 2048, 11008, 16, 2, 151936, 1e6, 1e-6, Tru
 LLAMA8B = ModelShape("llama-3.1-8b", 32, 4096, 14336, 32, 8, 128256, 5e5, 1e-5, False, 16)
 DENSE32B = ModelShape("dense-32b", 64, 5120, 27648, 40, 8, 152064, 1e6, 1e-5, False, 16)
 # Small stacks for tests that the fp64 oracle finishes in seconds.
-TINY = ModelShape("tiny", 2, 128, 320, 4, 2, 512, 1e4, 1e-5, True, 8)
+TINY = ModelShape("tiny", 2, 256, 704, 4, 2, 512, 1e4, 1e-5, True, 8)
 TINY_UNTIED = ModelShape("tiny-untied", 3, 256, 704, 4, 1, 1000, 5e5, 1e-5, False, 16)
 
 SHAPES = {s.name: s for s in (SMOL, QWEN3B, LLAMA8B, DENSE32B, TINY, TINY_UNTIED)}
@@ -178,3 +178,21 @@ def lora_init(shape: ModelShape) -> List[Dict[str, Dict[str, torch.Tensor]]]:
 def tokens(shape: ModelShape, batch: int, seq: int, step: int = 0) -> torch.Tensor:
     """int32 token ids [batch, seq]; targets are the ids shifted by one."""
     return uniform_ids(DATA_SEED, 500 + step, (batch, seq), shape.vocab)
+
+
+# ----------------------------------------------------------------------------
+# device-side draws (fast path for full-size workloads; not reproducible by
+# the oracle, which uses the numpy streams above)
+# ----------------------------------------------------------------------------
+
+def device_normal_bf16(shape, std: float, seed: int, stream: int, device="cuda") -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) << 32) | int(stream))
+    t = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    return (t * std).to(torch.bfloat16)
+
+
+def device_normal_f32(shape, std: float, seed: int, stream: int, device="cuda") -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) << 32) | int(stream))
+    return torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * std

@@ -1,0 +1,177 @@
+"""GPU parity of the decoder-layer kernels against the fp64 oracle (forward
+values, and backward values against torch.autograd through the oracle's
+forward in float64)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import decoder as D
+from tolerances import assert_close, assert_close_ew
+
+pytestmark = pytest.mark.gpu
+F64 = torch.float64
+
+
+def _rand(shape, std=1.0, stream=0):
+    return S.bf16(S.normal_f32(S.DATA_SEED, 9000 + stream, shape, std))
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _grad(fn, inputs, dy):
+    xs = [x.detach().to(F64).requires_grad_(True) for x in inputs]
+    out = fn(*xs)
+    gr = torch.autograd.grad(out, xs, grad_outputs=dy.to(F64))
+    return out.detach(), gr
+
+
+@pytest.mark.parametrize("M,d", [(130, 576), (64, 4096), (1, 256)])
+def test_rmsnorm_fwd_bwd(lsq, M, d):
+    x = _rand((M, d), 2.0, 1)
+    g = _rand((d,), 0.3, 2) + 1
+    g = g.to(torch.bfloat16)
+    dy = _rand((M, d), 1.0, 3)
+    res = _rand((M, d), 1.0, 4)
+    eps = 1e-5
+    y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    rstd = torch.empty(M, dtype=torch.float32, device="cuda")
+    lsq.lsq_rmsnorm_fwd(x.cuda(), g.cuda(), y, rstd, M, d, eps)
+    out = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_rmsnorm_bwd(dy.cuda(), x.cuda(), g.cuda(), rstd, res.cuda(), out, M, d)
+    torch.cuda.synchronize()
+    ref, (dx, _) = _grad(lambda a, b: D.rmsnorm(a, b, eps), [x, g], dy)
+    assert_close_ew(_np(y), ref.numpy(), what="rmsnorm y")
+    rr = 1.0 / np.sqrt((_np(x) ** 2).mean(-1) + eps)
+    assert_close(rstd.cpu().numpy(), rr, rel=1e-6, max_rms=1e-5, what="rstd")
+    assert_close_ew(_np(out), dx.numpy() + _np(res), what="rmsnorm dx + res")
+
+
+@pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5)])
+def test_rope_fwd_and_transpose(lsq, B, Sq, H, hd, theta):
+    x = _rand((B, Sq, H, hd), 1.0, 5)
+    dy = _rand((B, Sq, H, hd), 1.0, 6)
+    xg = x.cuda().contiguous()
+    lsq.lsq_rope(xg, B, Sq, H, hd, theta, 0)
+    dg = dy.cuda().contiguous()
+    lsq.lsq_rope(dg, B, Sq, H, hd, theta, 1)
+    torch.cuda.synchronize()
+    ref, (dx,) = _grad(lambda a: D.rope(a, theta), [x], dy)
+    assert_close_ew(_np(xg), ref.numpy(), what="rope")
+    assert_close_ew(_np(dg), dx.numpy(), what="rope transpose")
+
+
+def test_swiglu_fwd_bwd(lsq):
+    n = 4096 * 3
+    g, u, dm = _rand((n,), 2.0, 7), _rand((n,), 1.0, 8), _rand((n,), 1.0, 9)
+    m = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_swiglu_fwd(g.cuda(), u.cuda(), m, n)
+    gg, uu = g.cuda().clone(), u.cuda().clone()
+    lsq.lsq_swiglu_bwd(dm.cuda(), gg, uu, gg, uu, n)   # in place
+    torch.cuda.synchronize()
+    ref, (dg, du) = _grad(lambda a, b: D.silu(a) * b, [g, u], dm)
+    assert_close_ew(_np(m), ref.numpy(), what="swiglu")
+    assert_close_ew(_np(gg), dg.numpy(), what="dg")
+    assert_close_ew(_np(uu), du.numpy(), what="du")
+
+
+def _attn_case(B, Sq, Hq, Hkv, hd, seed):
+    q = _rand((B, Sq, Hq, hd), 1.0, 20 + seed)
+    k = _rand((B, Sq, Hkv, hd), 1.0, 21 + seed)
+    v = _rand((B, Sq, Hkv, hd), 1.0, 22 + seed)
+    do = _rand((B, Sq, Hq, hd), 1.0, 23 + seed)
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("B,Sq,Hq,Hkv,hd", [(1, 512, 9, 3, 64), (2, 200, 4, 1, 128), (1, 64, 2, 2, 64),
+                                            (1, 1, 4, 2, 128), (2, 130, 8, 2, 128)])
+def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
+    q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, Sq)
+    o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device="cuda")
+    lsq.lsq_attention_fwd(q.cuda(), k.cuda(), v.cuda(), o, lse, B, Sq, Hq, Hkv, hd)
+    dq = torch.empty_like(o)
+    dk = torch.empty(B, Sq, Hkv, hd, dtype=torch.bfloat16, device="cuda")
+    dv = torch.empty_like(dk)
+    ws = torch.empty(lsq.lsq_attention_bwd_workspace_size(B, Sq, Hq), dtype=torch.uint8, device="cuda")
+    lsq.lsq_attention_bwd(q.cuda(), k.cuda(), v.cuda(), o, lse, do.cuda(), dq, dk, dv, B, Sq, Hq, Hkv, hd, ws)
+    torch.cuda.synchronize()
+    ref, (rq, rk, rv) = _grad(D.causal_gqa_attention, [q, k, v], do)
+    assert_close_ew(_np(o), ref.numpy(), what="attn out")
+    # lse of the scaled scores
+    kk = k.to(F64).repeat_interleave(Hq // Hkv, dim=2)
+    sc = torch.einsum("bihd,bjhd->bhij", q.to(F64), kk) / math.sqrt(hd)
+    sc = sc.masked_fill(torch.triu(torch.ones(Sq, Sq, dtype=torch.bool), 1), float("-inf"))
+    assert_close(lse.cpu().numpy(), torch.logsumexp(sc, -1).numpy(), rel=1e-5, max_rms=1e-4, what="lse")
+    # P and dS enter the tensor cores as bf16: relative error up to ~2^-8 per
+    # term.  With a single key the softmax gradient is exactly zero; the kernel
+    # leaves a residue of dP - D (two fp32 sums of the same products in
+    # different orders), about 1e-6 here.
+    kw = dict(rel=1e-2, ew_rel=2e-2, ew_abs_rms=5e-2, zero_atol=1e-4)
+    assert_close_ew(_np(dq), rq.numpy(), what="dq", **kw)
+    assert_close_ew(_np(dk), rk.numpy(), what="dk", **kw)
+    assert_close_ew(_np(dv), rv.numpy(), what="dv", **kw)
+
+
+def test_attention_deterministic(lsq):
+    B, Sq, Hq, Hkv, hd = 2, 256, 8, 2, 128
+    q, k, v, do = (t.cuda() for t in _attn_case(B, Sq, Hq, Hkv, hd, 7))
+    outs = []
+    for _ in range(2):
+        o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device="cuda")
+        lsq.lsq_attention_fwd(q, k, v, o, lse, B, Sq, Hq, Hkv, hd)
+        dq, dk, dv = torch.empty_like(o), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(lsq.lsq_attention_bwd_workspace_size(B, Sq, Hq), dtype=torch.uint8, device="cuda")
+        lsq.lsq_attention_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Sq, Hq, Hkv, hd, ws)
+        outs.append((o, lse, dq, dk, dv))
+    torch.cuda.synchronize()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B,Sq,V", [(2, 64, 1000), (1, 512, 49152)])
+def test_cross_entropy(lsq, B, Sq, V):
+    logits = torch.from_numpy(S.normal_f32(S.DATA_SEED, 77, (B * Sq, V), 2.0))
+    ids = S.uniform_ids(S.DATA_SEED, 78, (B, Sq), V)
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    dl = torch.empty(B * Sq, V, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(lsq.lsq_xent_workspace_size(B * Sq), dtype=torch.uint8, device="cuda")
+    lsq.lsq_xent_fwd_bwd(logits.cuda(), ids.cuda(), B, Sq, V, loss, dl, ws)
+    torch.cuda.synchronize()
+    lg = logits.to(F64).reshape(B, Sq, V).requires_grad_(True)
+    ref = D.cross_entropy_next_token(lg, ids)
+    (g,) = torch.autograd.grad(ref, [lg])
+    assert abs(loss.item() - ref.item()) <= 1e-5 * abs(ref.item())
+    assert_close_ew(_np(dl), g.reshape(B * Sq, V).numpy(), what="dlogits")
+
+
+def test_embed_gather_exact(lsq):
+    V, d, M = 1000, 256, 300
+    table = _rand((V, d), 1.0, 40)
+    ids = S.uniform_ids(S.DATA_SEED, 41, (M,), V)
+    h = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_embed_gather(ids.cuda(), table.cuda(), h, M, d, V)
+    torch.cuda.synchronize()
+    assert torch.equal(h.cpu(), table[ids.long()])
+
+
+def test_adamw_matches_oracle(lsq):
+    n = 10000
+    p = torch.from_numpy(S.normal_f32(1, 50, (n,)))
+    m = torch.zeros(n)
+    v = torch.zeros(n)
+    pg, mg, vg = p.cuda(), m.cuda(), v.cuda()
+    pb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    ref = (p.to(F64), m.to(F64), v.to(F64))
+    for t in range(1, 4):
+        g = torch.from_numpy(S.normal_f32(1, 50 + t, (n,), 1e-2))
+        lsq.lsq_adamw_step(pg, g.cuda(), mg, vg, pb, n, t, 1e-3, 0.9, 0.999, 1e-8, 0.01)
+        ref = D.adamw(ref[0], g, ref[1], ref[2], t, lr=1e-3, wd=0.01)
+    torch.cuda.synchronize()
+    assert_close(pg.cpu().numpy(), ref[0].numpy(), rel=1e-6, max_rms=1e-6, what="adamw p")
+    assert torch.equal(pb.cpu(), pg.cpu().to(torch.bfloat16))

@@ -214,7 +214,7 @@ def test_bwd_multi_segments_sum(lsq):
     assert_close(dx.float().cpu().numpy(), rdx, what="dX sum")
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 1000, 576), (64, 4096, 128)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 1000, 576), (64, 4096, 128), (96, 512, 1000)])
 @pytest.mark.parametrize("trans_b", [0, 1])
 def test_dense_gemm(lsq, M, N, K, trans_b):
     a = S.bf16(S.normal_f32(7, 1, (M, K)))

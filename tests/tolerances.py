@@ -28,3 +28,31 @@ def assert_close(got, ref, rel=REL_FRO, max_rms=MAX_ABS_RMS, what=""):
     mx = float(np.max(np.abs(got - ref))) if got.size else 0.0
     assert rf <= rel, f"{what}: relative Frobenius error {rf:.3e} > {rel:.1e}"
     assert mx <= max_rms * rms + 1e-30, f"{what}: max error {mx:.3e} > {max_rms:.0e} x RMS {rms:.3e}"
+
+
+# Elementwise ops and attention (outputs rounded to bf16 once, inputs bf16):
+# error per element <= EW_REL |ref| (a bf16 ulp is 2^-8 relative, rounding
+# half of it, plus fp32 arithmetic) + EW_ABS_RMS x RMS(ref), with the same
+# Frobenius bound as the GEMMs.
+EW_REL = 8e-3
+EW_ABS_RMS = 2e-2
+
+
+def assert_close_ew(got, ref, rel=REL_FRO, ew_rel=EW_REL, ew_abs_rms=EW_ABS_RMS, what="", zero_atol=1e-6):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    nref = float(np.linalg.norm(ref))
+    if nref == 0.0:
+        mx = float(np.max(np.abs(got))) if got.size else 0.0
+        assert mx <= zero_atol, f"{what}: reference is exactly zero, got max |x| = {mx:.3e}"
+        return
+    rf = rel_fro(got, ref)
+    assert rf <= rel, f"{what}: relative Frobenius error {rf:.3e} > {rel:.1e}"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    err = np.abs(got - ref)
+    bound = ew_rel * np.abs(ref) + ew_abs_rms * rms
+    worst = int(np.argmax(err - bound))
+    assert np.all(err <= bound), (f"{what}: element {worst} error {err.flat[worst]:.3e} > "
+                                  f"{ew_rel:.0e} x |{ref.flat[worst]:.3e}| + {ew_abs_rms:.0e} x RMS {rms:.3e}")
