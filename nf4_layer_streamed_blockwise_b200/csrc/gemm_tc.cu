@@ -34,22 +34,27 @@ constexpr int TMA_WARP = 4, MMA_WARP = 5, DQ_WARP0 = 6;
 constexpr int KE_MAX = 64;  // columns of the rank-r products held in TMEM
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
-constexpr int L_BYTES = KE_MAX * BK * 2;
+constexpr int L_BYTES = KE_MAX * BK * 2;   // LoRA operand of the main loop (rp rows x 64)
+constexpr int C_BYTES = BN * BK / 2;       // packed NF4 codes of one stage (8 KB)
 constexpr int UE_BYTES = BM * KE_MAX * 2;
 constexpr int BE_BYTES = BN * KE_MAX * 2;
 constexpr uint32_t TMEM_COLS = 512;
 
+// Shared memory.  The epilogue's LoRA operands (UE, BE) alias the activation
+// stages: they are written only after every main-loop MMA has retired.
 template <int MODE>
 struct Layout {
   static constexpr bool NF4 = (MODE == NF4_FWD || MODE == NF4_DX);
   static constexpr int NST = NF4 ? 3 : 4;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + NST * A_BYTES;
-  static constexpr int OFF_L = OFF_B + NST * B_BYTES;
-  static constexpr int OFF_UE = OFF_L + (NF4 ? NST * L_BYTES : 0);
-  static constexpr int OFF_BE = OFF_UE + (NF4 ? UE_BYTES : 0);
-  static constexpr int OFF_BAR = OFF_BE + (NF4 ? BE_BYTES : 0);
-  static constexpr int NBAR = 2 * NST + 4;
+  static constexpr int OFF_C = OFF_B + NST * B_BYTES;
+  static constexpr int OFF_L = OFF_C + (NF4 ? NST * C_BYTES : 0);
+  static constexpr int OFF_BAR = OFF_L + (NF4 ? NST * L_BYTES : 0);
+  static constexpr int OFF_UE = OFF_A;
+  static constexpr int OFF_BE = OFF_A + UE_BYTES;
+  static_assert(!NF4 || UE_BYTES + BE_BYTES <= NST * (A_BYTES + B_BYTES), "epilogue operands must fit the stages");
+  static constexpr int NBAR = 3 * NST + 4;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int BYTES = OFF_MISC + 128 + 1024;  // + alignment slack
 };
@@ -79,8 +84,10 @@ struct Params {
 };
 
 struct Maps {
-  CUtensorMap a[3];
-  CUtensorMap b;
+  CUtensorMap a[3];  // activation (forward: x; dX: dy of each segment)
+  CUtensorMap b;     // dense: bf16 weight
+  CUtensorMap c[3];  // NF4: packed codes of each segment (uint8 [n, K/2])
+  CUtensorMap l[3];  // forward: LoRA A of each segment (bf16 [r, K], box rp rows)
 };
 
 __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
@@ -131,7 +138,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* empty = full + NST;
-  uint64_t* ufull = empty + NST;
+  uint64_t* cfull = empty + NST;  // packed codes of stage s landed (NF4)
+  uint64_t* ufull = cfull + NST;
   uint64_t* lready = ufull + 1;
   uint64_t* afull = ufull + 2;
   uint64_t* drain = ufull + 3;
@@ -154,6 +162,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1 + (NF4 ? 8 : 0));
       mbar_init(&empty[s], 1);
+      mbar_init(&cfull[s], 1);
     }
     mbar_init(ufull, 1);
     mbar_init(lready, 1);
@@ -173,6 +182,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
 
   if (warp == TMA_WARP) {
     // ------------------------------------------------------------ TMA producer
+    // per stage: the activation tile, the bf16 weight tile (dense) or the
+    // packed NF4 codes (into their own buffer, signalled on cfull[s]) and, in
+    // the forward, the LoRA-down tile A[0:rp, k-block] (rows >= r read as 0).
     if (lane == 0) {
       tma_prefetch_desc(&maps.a[0]);
       for (int i = 0; i < p.nkb; ++i) {
@@ -181,12 +193,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
         if (!mbar_wait(&empty[s], ph ^ 1u, 401)) break;
         uint8_t* a_dst = smem + L::OFF_A + s * A_BYTES;
         uint8_t* b_dst = smem + L::OFF_B + s * B_BYTES;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + (NF4 ? 0 : B_BYTES)));
+        uint32_t bytes = A_BYTES;
+        if (!NF4) bytes += B_BYTES;
+        if (MODE == NF4_FWD && lora) bytes += p.rp * 128;
+        mbar_arrive_expect_tx(&full[s], bytes);
         if (MODE == NF4_DX) {
           const int sg = seg_of_block(p, i);
-          tma_load_2d(a_dst, &maps.a[sg], &full[s], (i - p.seg[sg].first) * BK, m0);
+          const int nb = i - p.seg[sg].first;
+          tma_load_2d(a_dst, &maps.a[sg], &full[s], nb * BK, m0);
+          mbar_arrive_expect_tx(&cfull[s], C_BYTES);
+          tma_load_2d(smem + L::OFF_C + s * C_BYTES, &maps.c[sg], &cfull[s], n0 / 2, nb * BK);
         } else {
           tma_load_2d(a_dst, &maps.a[0], &full[s], i * BK, m0);
+        }
+        if (MODE == NF4_FWD) {
+          mbar_arrive_expect_tx(&cfull[s], C_BYTES);
+          tma_load_2d(smem + L::OFF_C + s * C_BYTES, &maps.c[seg], &cfull[s], i * (BK / 2), n0);
+          if (lora) tma_load_2d(smem + L::OFF_L + s * L_BYTES, &maps.l[seg], &full[s], i * BK, 0);
         }
         if (MODE == DENSE_NT) tma_load_2d(b_dst, &maps.b, &full[s], i * BK, n0);
         if (MODE == DENSE_NN) {
@@ -254,6 +277,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
     }
   } else if (warp >= DQ_WARP0) {
     // ------------------------------------------------------------ NF4 dequantisers
+    // Each thread turns one 64-element NF4 block per stage (32 code bytes from
+    // the TMA-filled codes tile, one absmax from registers, fetched ahead) into
+    // one 128-byte row of the swizzled bf16 operand tile.
     if (NF4) {
       const int t = threadIdx.x - DQ_WARP0 * 32;  // 0..255
       const int KB = p.K / 64;
@@ -261,65 +287,68 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
         const Seg& sg = p.seg[seg];
         const int n = n0 + t;
         const bool valid = n < sg.n;
-        const uint8_t* crow = sg.codes + (int64_t)(valid ? n : 0) * (p.K / 2);
         const float* arow = sg.absmax + (int64_t)(valid ? n : 0) * KB;
+        // absmax: four blocks per 16-byte load when rows are 16-byte aligned,
+        // one group fetched ahead; else a 2-deep scalar prefetch
+        const bool vec = (KB % 4) == 0;
+        float4 acur = make_float4(0.f, 0.f, 0.f, 0.f), anext = acur;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+        if (valid) {
+          if (vec) {
+            acur = __ldg(reinterpret_cast<const float4*>(arow));
+            if (KB > 4) anext = __ldg(reinterpret_cast<const float4*>(arow + 4));
+          } else {
+            s0 = __ldg(arow);
+            if (KB > 1) s1 = __ldg(arow + 1);
+            if (KB > 2) s2 = __ldg(arow + 2);
+          }
+        }
         for (int i = 0; i < p.nkb; ++i) {
           const int s = i % NST;
           const uint32_t ph = (uint32_t)(i / NST) & 1u;
-          uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-          float a = 0.0f;
-          if (valid) {
-            c0 = __ldg(reinterpret_cast<const uint4*>(crow + i * 32));
-            c1 = __ldg(reinterpret_cast<const uint4*>(crow + i * 32 + 16));
-            a = __ldg(arow + i);
+          float a;
+          if (vec) {
+            const int q = i & 3;
+            a = q == 0 ? acur.x : q == 1 ? acur.y : q == 2 ? acur.z : acur.w;
+          } else {
+            a = s0;
           }
-          uint4 lv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-          if (lora) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int idx = t + q * 256, j = idx >> 3, ch = idx & 7;
-              if (j < p.r) lv[q] = __ldg(reinterpret_cast<const uint4*>(sg.la + (int64_t)j * p.K + i * 64 + ch * 8));
-            }
-          }
-          if (!mbar_wait(&empty[s], ph ^ 1u, 601)) break;
-          store_block_row(smem_u32(smem + L::OFF_B + s * B_BYTES) + t * 128, t, c0, c1, a, s_cb);
-          if (lora) {
-            const uint32_t lb = smem_u32(smem + L::OFF_L + s * L_BYTES);
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int idx = t + q * 256, j = idx >> 3, ch = idx & 7;
-              if (j < p.rp) st_shared_v4(lb + j * 128 + ((uint32_t)(ch ^ (j & 7)) << 4), lv[q]);
-            }
-          }
+          if (!mbar_wait(&cfull[s], ph, 601)) break;
+          const uint8_t* crow = smem + L::OFF_C + s * C_BYTES + t * 32;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
+          store_block_row(smem_u32(smem + L::OFF_B + s * B_BYTES) + t * 128, t, c0, c1, valid ? a : 0.0f, s_cb);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&full[s]);
+          if (valid) {
+            if (vec) {
+              if ((i & 3) == 3) {
+                acur = anext;
+                if (i + 5 < KB) anext = __ldg(reinterpret_cast<const float4*>(arow + i + 5));
+              }
+            } else {
+              s0 = s1;
+              s1 = s2;
+              if (i + 3 < KB) s2 = __ldg(arow + i + 3);
+            }
+          }
         }
       } else {  // NF4_DX: tile = 64 contraction rows (n) x 256 output columns (k)
         const int nl = t >> 2, kc = t & 3;
         const int kcol = n0 + kc * 64;
         const int jq = p.rp / 4;  // LoRA B^T values per thread (rp <= 64 -> <= 16)
-        for (int i = 0; i < p.nkb; ++i) {
-          const int s = i % NST;
-          const uint32_t ph = (uint32_t)(i / NST) & 1u;
+        const int bn = t & 63, bj0 = (t >> 6) * jq;
+        float a_nx = 0.f;
+        uint16_t bl_nx[16];
+        // fetch absmax and the LoRA operand of contraction block i
+        auto fetch = [&](int i, float& a, uint16_t* bl) {
           const int sgi = seg_of_block(p, i);
           const Seg& sg = p.seg[sgi];
           const int nrow = (i - sg.first) * BK + nl;
-          const bool valid = nrow < sg.n && kcol < p.K;
-          uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-          float a = 0.0f;
-          if (valid) {
-            const uint8_t* cp = sg.codes + (int64_t)nrow * (p.K / 2) + kcol / 2;
-            c0 = __ldg(reinterpret_cast<const uint4*>(cp));
-            c1 = __ldg(reinterpret_cast<const uint4*>(cp + 16));
-            a = __ldg(sg.absmax + (int64_t)nrow * KB + kcol / 64);
-          }
-          // LoRA operand of the main loop: B^T tile [rp rows (j) x 64 (n)],
-          // thread handles n = (t & 63), j in [(t >> 6) * jq, +jq)
-          uint16_t bl[16];
-          const int bn = t & 63, bj0 = (t >> 6) * jq;
-          const int brow = (i - sg.first) * BK + bn;
+          a = (nrow < sg.n && kcol < p.K) ? __ldg(sg.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
           if (lora) {
+            const int brow = (i - sg.first) * BK + bn;
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
               const int j = bj0 + q;
@@ -328,7 +357,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
                 bl[q] = __ldg(reinterpret_cast<const unsigned short*>(sg.lb) + (int64_t)brow * p.r + j);
             }
           }
-          if (!mbar_wait(&empty[s], ph ^ 1u, 602)) break;
+        };
+        if (p.nkb > 0) fetch(0, a_nx, bl_nx);
+        for (int i = 0; i < p.nkb; ++i) {
+          const int s = i % NST;
+          const uint32_t ph = (uint32_t)(i / NST) & 1u;
+          const float a = a_nx;
+          uint16_t bl[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) bl[q] = bl_nx[q];
+          if (i + 1 < p.nkb) fetch(i + 1, a_nx, bl_nx);
+          if (!mbar_wait(&cfull[s], ph, 602)) break;
+          const uint8_t* crow = smem + L::OFF_C + s * C_BYTES + nl * 128 + kc * 32;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
           store_block_row(smem_u32(smem + L::OFF_B + s * B_BYTES) + kc * 8192 + nl * 128, nl, c0, c1, a, s_cb);
           if (lora) {
             const uint32_t lbase = smem_u32(smem + L::OFF_L + s * L_BYTES);
@@ -350,9 +392,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
     const int e = threadIdx.x;  // accumulator row / TMEM lane
     const int m = m0 + e;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    if (lora) {
-      // LoRA operand of the epilogue MMA, no-swizzle K-major [BN rows x KE]:
-      // forward: B[n0 + row, j]; dX: A_seg[j, n0 + row] at column seg*rp + j
+    bool ok = mbar_wait(ufull, 0, 701);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) tc_fence_after();
+    if (ok && lora) {
+      // Every main-loop MMA has retired: the stage buffers are free and hold
+      // the epilogue's LoRA operands now (no-swizzle K-major):
+      //   sBe [BN rows x KE]: forward B[n0 + row, j]; dX A_seg[j, n0 + row] at column seg*rp + j
+      //   sUe [128 rows x KE]: s*U (forward) or s*G (dX) as bf16
       const uint32_t be = smem_u32(smem + L::OFF_BE);
       for (int row = e; row < BN; row += 128) {
         for (int jc = 0; jc < KE / 8; ++jc) {
@@ -378,11 +425,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
           st_shared_v4(be + (row >> 3) * (KE * 16) + jc * 128 + (row & 7) * 16, make_uint4(w[0], w[1], w[2], w[3]));
         }
       }
-    }
-    bool ok = mbar_wait(ufull, 0, 701);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) tc_fence_after();
-    if (ok && lora) {
       const uint32_t ue = smem_u32(smem + L::OFF_UE);
       for (int c = 0; c < KE / 16; ++c) {
         float v[16];
@@ -561,6 +603,16 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
   if ((st = encode_tmap_2d(&maps.a[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, BK, BM,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
     return st;
+  for (int i = 0; i < nseg; ++i) {
+    // packed codes: rows of K/2 bytes, one stage = 256 rows x 32 bytes
+    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
+                             BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
+      return st;
+    // LoRA A [r, K]: one stage = rp rows x 64 columns; rows r..rp-1 read as zero
+    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A[i], K, r, K * 2, BK, p.rp,
+                                      CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+      return st;
+  }
   dim3 grid(tiles, (unsigned)((M + BM - 1) / BM));
   return launch<NF4_FWD>(maps, p, grid, (cudaStream_t)stream);
 }
@@ -609,6 +661,10 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
     blocks += (int)((W[i].n_out + BK - 1) / BK);
     if ((st = encode_tmap_2d(&maps.a[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy[i], W[i].n_out, M, W[i].n_out * 2, BK,
                              BM, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+      return st;
+    // packed codes: one stage = 64 rows (contraction) x 128 bytes (256 output columns)
+    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
+                             BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
   }
   p.nkb = blocks;

@@ -2,10 +2,12 @@
 //   dX = sum_seg dY_seg deq(W_seg) + s G_seg A_seg     (tensor cores, gemm_tc.cu)
 //   dB_seg = s dY_seg^T U_seg,  dA_seg = s G_seg^T X    (here)
 // dA and dB are skinny products (r <= 64 columns) reduced over the M token
-// rows.  They are HBM-bound reads of dY and X, done as a deterministic
-// two-stage reduction: stage 1 gives each CTA a 64-column panel and a chunk of
-// rows and writes fp32 partial sums; stage 2 adds the partials in a fixed
-// order.  No atomics, so the result is bit-identical run to run.
+// rows, i.e. HBM-bound reads of dY and X.  Deterministic two-stage reduction:
+// stage 1 gives each CTA a 128-column panel and a chunk of rows (row tiles of
+// P and Q double-buffered through shared memory with cp.async) and writes fp32
+// partial sums; stage 2 adds the partials of each output in a fixed order.
+// No atomics, so results are bit-identical run to run.  Every reduction of one
+// backward call (dA and dB of up to three linears) shares one launch per stage.
 #include "common.cuh"
 #include "host_common.h"
 
@@ -17,105 +19,164 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
 
 namespace lg {
 
-constexpr int PANEL = 64;
-constexpr int ROWS = 32;        // rows of Q staged per step
+constexpr int PANEL = 128;      // columns per CTA (2 per thread)
+constexpr int TR = 32;          // rows per shared-memory tile
+constexpr int THREADS = 256;
 constexpr int TARGET_CTAS = 296;
+constexpr int MAXRED = 6;
 
-// part[chunk][c][j] = sum_{m in chunk} P[m, c] * Q[m, j]
-__global__ void __launch_bounds__(256) skinny_partial(const __nv_bfloat16* __restrict__ P, int64_t M, int64_t C,
-                                                      const float* __restrict__ Q, int r, int64_t mchunk,
-                                                      float* __restrict__ part) {
-  __shared__ float sQ[ROWS * 64];
-  const int64_t c = (int64_t)blockIdx.x * PANEL + (threadIdx.x & 63);
-  const int jg = threadIdx.x >> 6;  // j = jg + 4 q
-  const int64_t mb0 = (int64_t)blockIdx.y * mchunk;
-  const int64_t mb1 = mb0 + mchunk < M ? mb0 + mchunk : M;
-  float acc[16];
+struct Red {
+  const __nv_bfloat16* P;  // [M, C]
+  const float* Q;          // [M, r]
+  float* out;              // [C, r] or, transposed, [r, C]
+  float* part;             // [chunks, C, r]
+  int64_t C;
+  int64_t mchunk;          // rows per chunk (multiple of TR)
+  int chunks, panels, transpose;
+};
+
+struct RedSet {
+  Red red[MAXRED];
+  int n;
+  int64_t M;
+  int r, accumulate;
+  float s;
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = smem_u32(dst);
+  const int sz = valid ? 16 : 0;  // 0: fill with zeros
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// stage 1: blockIdx.x = panel (+ offsets of earlier reductions), blockIdx.y = row chunk
+__global__ void __launch_bounds__(THREADS) skinny_partial(const __grid_constant__ RedSet rs) {
+  __shared__ __align__(16) __nv_bfloat16 sP[2][TR][PANEL];
+  __shared__ __align__(16) float sQ[2][TR][64];
+  int rid = 0, px = blockIdx.x;
+  while (rid + 1 < rs.n && px >= rs.red[rid].panels) {
+    px -= rs.red[rid].panels;
+    ++rid;
+  }
+  const Red& R = rs.red[rid];
+  if ((int)blockIdx.y >= R.chunks) return;
+  const int r = rs.r;
+  const int64_t M = rs.M, C = R.C;
+  const int64_t c0 = (int64_t)px * PANEL;
+  const int64_t mb0 = (int64_t)blockIdx.y * R.mchunk;
+  const int64_t mb1 = mb0 + R.mchunk < M ? mb0 + R.mchunk : M;
+  const int tid = threadIdx.x;
+  const int cp = tid & 63, jg = tid >> 6;  // columns c0 + 2cp, +1; j in [jg*jq, jg*jq + jq)
+  const int jq = (r + 3) / 4;
+  float acc[2][16];
 #pragma unroll
-  for (int q = 0; q < 16; ++q) acc[q] = 0.0f;
-  for (int64_t mb = mb0; mb < mb1; mb += ROWS) {
-    const int rows = (int)((mb1 - mb) < ROWS ? (mb1 - mb) : ROWS);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < rows * r; idx += 256) sQ[idx] = Q[mb * r + idx];
-    __syncthreads();
-    if (c < C) {
-      const __nv_bfloat16* pp = P + mb * C + c;
-      int mm = 0;
-      for (; mm + 4 <= rows; mm += 4) {
-        float pv[4];
+  for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) pv[u] = __bfloat162float(pp[(int64_t)(mm + u) * C]);
+    for (int q = 0; q < 16; ++q) acc[a][q] = 0.0f;
+
+  auto load = [&](int buf, int64_t mb) {
+    // P: TR rows x 128 columns = 512 chunks of 16 bytes (2 per thread)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int j = jg + 4 * q;
-            if (j < r) acc[q] = fmaf(pv[u], sQ[(mm + u) * r + j], acc[q]);
-          }
-        }
+    for (int u = 0; u < 2; ++u) {
+      const int idx = tid + u * THREADS;
+      const int row = idx >> 4, ch = idx & 15;
+      const int64_t m = mb + row, c = c0 + ch * 8;
+      const bool v = m < mb1 && c < C;
+      cp_async16(&sP[buf][row][ch * 8], v ? (const void*)(R.P + m * C + c) : (const void*)R.P, v);
+    }
+    // Q: TR rows x r floats, as 16-byte chunks of whole rows (r % 4 == 0) or scalars
+    if ((r & 3) == 0) {
+      const int per = r / 4;
+      for (int idx = tid; idx < TR * per; idx += THREADS) {
+        const int row = idx / per, ch = idx % per;
+        const int64_t m = mb + row;
+        const bool v = m < mb1;
+        cp_async16(&sQ[buf][row][ch * 4], v ? (const void*)(R.Q + m * r + ch * 4) : (const void*)R.Q, v);
       }
-      for (; mm < rows; ++mm) {
-        const float pv = __bfloat162float(pp[(int64_t)mm * C]);
+    } else {
+      for (int idx = tid; idx < TR * r; idx += THREADS) {
+        const int row = idx / r, j = idx % r;
+        const int64_t m = mb + row;
+        sQ[buf][row][j] = m < mb1 ? R.Q[m * r + j] : 0.0f;
+      }
+    }
+    cp_async_commit();
+  };
+
+  int buf = 0;
+  if (mb0 < mb1) load(0, mb0);
+  for (int64_t mb = mb0; mb < mb1; mb += TR) {
+    const bool more = mb + TR < mb1;
+    if (more) load(buf ^ 1, mb + TR);
+    if (more) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 4
+    for (int row = 0; row < TR; ++row) {
+      const uint32_t pp = *reinterpret_cast<const uint32_t*>(&sP[buf][row][cp * 2]);
+      const float p0 = bf16lo(pp), p1 = bf16hi(pp);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int j = jg + 4 * q;
-          if (j < r) acc[q] = fmaf(pv, sQ[mm * r + j], acc[q]);
+      for (int q = 0; q < 16; ++q) {
+        if (q < jq) {
+          const float qv = sQ[buf][row][jg * jq + q];
+          acc[0][q] = fmaf(p0, qv, acc[0][q]);
+          acc[1][q] = fmaf(p1, qv, acc[1][q]);
         }
       }
     }
+    __syncthreads();
+    buf ^= 1;
   }
-  if (c < C) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int64_t c = c0 + cp * 2 + a;
+    if (c >= C) continue;
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
-      const int j = jg + 4 * q;
-      if (j < r) part[((int64_t)blockIdx.y * C + c) * r + j] = acc[q];
+      const int j = jg * jq + q;
+      if (q < jq && j < r) R.part[((int64_t)blockIdx.y * C + c) * r + j] = acc[a][q];
     }
   }
 }
 
-// out[c, j] (transpose: out[j, c]) (+)= s * sum_k part[k][c][j], k ascending
-__global__ void __launch_bounds__(256) skinny_reduce(const float* __restrict__ part, int nchunks, int64_t C, int r,
-                                                     float s, float* __restrict__ out, int transpose, int accumulate) {
-  const int64_t n = C * r;
+// stage 2: out (+)= s * sum over chunks (ascending) of the partials
+__global__ void __launch_bounds__(256) skinny_reduce(const __grid_constant__ RedSet rs) {
+  const int rid = blockIdx.y;
+  const Red& R = rs.red[rid];
+  const int r = rs.r;
+  const int64_t n = R.C * r;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
     float sum = 0.0f;
-    for (int k = 0; k < nchunks; ++k) sum += part[(int64_t)k * n + idx];
+    for (int k = 0; k < R.chunks; ++k) sum += R.part[(int64_t)k * n + idx];
     const int64_t c = idx / r, j = idx % r;
-    float* dst = transpose ? out + j * C + c : out + idx;
-    const float v = s * sum;
-    *dst = accumulate ? *dst + v : v;
+    float* dst = R.transpose ? R.out + j * R.C + c : R.out + idx;
+    const float v = rs.s * sum;
+    *dst = rs.accumulate ? *dst + v : v;
   }
 }
 
-static int64_t nchunks_for(int64_t M, int64_t C) {
-  const int64_t panels = (C + PANEL - 1) / PANEL;
-  int64_t k = (TARGET_CTAS + panels - 1) / panels;
-  const int64_t maxk = (M + ROWS - 1) / ROWS;
+static int64_t panels_for(int64_t C) { return (C + PANEL - 1) / PANEL; }
+
+static int64_t chunks_for(int64_t M, int64_t C) {
+  int64_t k = (TARGET_CTAS + panels_for(C) - 1) / panels_for(C);
+  const int64_t maxk = (M + TR - 1) / TR;
   if (k > maxk) k = maxk;
   if (k < 1) k = 1;
   return k;
 }
 
+static int64_t mchunk_for(int64_t M, int64_t k) { return ((M + k - 1) / k + TR - 1) / TR * TR; }
+
 static size_t partial_bytes(int64_t M, int64_t C, int r) {
-  return (size_t)nchunks_for(M, C) * (size_t)C * (size_t)r * sizeof(float);
+  const int64_t k = chunks_for(M, C);
+  const int64_t kk = (M + mchunk_for(M, k) - 1) / mchunk_for(M, k);
+  return ((size_t)kk * (size_t)C * (size_t)r * sizeof(float) + 255) / 256 * 256;
 }
 
 static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
-
-static lsq_status skinny(const void* P, int64_t M, int64_t C, const float* Q, int r, float s, float* out,
-                         int transpose, int accumulate, float* part, cudaStream_t stream) {
-  const int64_t k = nchunks_for(M, C);
-  const int64_t mchunk = ((M + k - 1) / k + ROWS - 1) / ROWS * ROWS;
-  const int64_t kk = (M + mchunk - 1) / mchunk;
-  dim3 g1((unsigned)((C + PANEL - 1) / PANEL), (unsigned)kk);
-  skinny_partial<<<g1, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(P), M, C, Q, r, mchunk, part);
-  LSQ_LAUNCH_CHECK("skinny_partial");
-  int64_t g2 = (C * r + 255) / 256;
-  if (g2 > 4096) g2 = 4096;
-  skinny_reduce<<<(unsigned)g2, 256, 0, stream>>>(part, (int)kk, C, r, s, out, transpose, accumulate);
-  LSQ_LAUNCH_CHECK("skinny_reduce");
-  return LSQ_OK;
-}
 
 }  // namespace lg
 }  // namespace lsq
@@ -125,13 +186,9 @@ using namespace lsq;
 extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
   if (nseg < 1 || nseg > 3 || r <= 0 || M < 1 || !n_out) return 256;
-  size_t g = lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
-  size_t part = lg::partial_bytes(M, k_in, r);
-  for (int i = 0; i < nseg; ++i) {
-    const size_t b = lg::partial_bytes(M, n_out[i], r);
-    if (b > part) part = b;
-  }
-  return g + lg::round256(part);
+  size_t b = lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
+  for (int i = 0; i < nseg; ++i) b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
+  return b;
 }
 
 extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x,
@@ -151,6 +208,7 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   const int rp = r > 0 ? (r + 15) / 16 * 16 : 0;
   if (nseg * rp > 64) return fail(LSQ_EUNSUPPORTED, "%s: nseg * round16(r) must be <= 64", who);
   if (dx && !aligned(dx, 16)) return fail(LSQ_EINVAL, "%s: dx must be 16-byte aligned", who);
+  if (r > 0 && (!x || !aligned(x, 16))) return fail(LSQ_EINVAL, "%s: x NULL or not 16-byte aligned", who);
   int64_t n_out[3];
   for (int i = 0; i < nseg; ++i) {
     const lsq_nf4_weight& w = W[i];
@@ -160,14 +218,15 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     if (!dy[i] || !aligned(dy[i], 16)) return fail(LSQ_EINVAL, "%s: dy[%d] NULL or not 16-byte aligned", who, i);
     n_out[i] = w.n_out;
     if (r > 0) {
-      if (!x || !A || !B || !u || !dA || !dB || !A[i] || !B[i] || !u[i] || !dA[i] || !dB[i])
+      if (!A || !B || !u || !dA || !dB || !A[i] || !B[i] || !u[i] || !dA[i] || !dB[i])
         return fail(LSQ_EINVAL, "%s: LoRA operands/gradients NULL with r > 0", who);
-      if (!aligned(A[i], 16)) return fail(LSQ_EINVAL, "%s: LoRA A must be 16-byte aligned", who);
+      if (!aligned(A[i], 16) || !aligned(u[i], 16))
+        return fail(LSQ_EINVAL, "%s: LoRA A and U must be 16-byte aligned", who);
     }
   }
   if (r == 0 && !dx) return LSQ_OK;
   float* g[3] = {nullptr, nullptr, nullptr};
-  float* part = nullptr;
+  char* part = nullptr;
   if (r > 0) {
     const size_t need = lsq_nf4_lora_bwd_workspace_size(nseg, M, K, n_out, r);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
@@ -175,16 +234,44 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
                   workspace_bytes);
     float* ws = static_cast<float*>(workspace);
     for (int i = 0; i < nseg; ++i) g[i] = ws + (size_t)i * M * r;
-    part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                    lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float)));
+    part = static_cast<char*>(workspace) + lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
   }
   cudaStream_t cs = (cudaStream_t)stream;
   if ((st = tc::launch_dx(nseg, W, dy, M, A, B, r, s, dx, g, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
+  lg::RedSet rs;
+  memset(&rs, 0, sizeof(rs));
+  rs.M = M;
+  rs.r = r;
+  rs.s = s;
+  rs.accumulate = accumulate ? 1 : 0;
+  int panels = 0, maxchunks = 1;
+  int64_t maxn = 0;
   for (int i = 0; i < nseg; ++i) {
-    if ((st = lg::skinny(dy[i], M, n_out[i], u[i], r, s, dB[i], 0, accumulate, part, cs)) != LSQ_OK) return st;
-    if ((st = lg::skinny(x, M, K, g[i], r, s, dA[i], 1, accumulate, part, cs)) != LSQ_OK) return st;
+    for (int which = 0; which < 2; ++which) {  // dB_i = s dy_i^T U_i ; dA_i = s G_i^T x
+      lg::Red& R = rs.red[rs.n++];
+      R.P = static_cast<const __nv_bfloat16*>(which == 0 ? dy[i] : x);
+      R.Q = which == 0 ? u[i] : g[i];
+      R.out = which == 0 ? dB[i] : dA[i];
+      R.C = which == 0 ? n_out[i] : K;
+      R.transpose = which;
+      const int64_t k = lg::chunks_for(M, R.C);
+      R.mchunk = lg::mchunk_for(M, k);
+      R.chunks = (int)((M + R.mchunk - 1) / R.mchunk);
+      R.panels = (int)lg::panels_for(R.C);
+      R.part = reinterpret_cast<float*>(part);
+      part += lg::partial_bytes(M, R.C, r);
+      panels += R.panels;
+      if (R.chunks > maxchunks) maxchunks = R.chunks;
+      if (R.C * r > maxn) maxn = R.C * r;
+    }
   }
+  lg::skinny_partial<<<dim3(panels, maxchunks), lg::THREADS, 0, cs>>>(rs);
+  LSQ_LAUNCH_CHECK("skinny_partial");
+  int64_t g2 = (maxn + 255) / 256;
+  if (g2 > 1024) g2 = 1024;
+  lg::skinny_reduce<<<dim3((unsigned)g2, rs.n), 256, 0, cs>>>(rs);
+  LSQ_LAUNCH_CHECK("skinny_reduce");
   return LSQ_OK;
 }
 
