@@ -156,6 +156,29 @@ lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
                                   int32_t accumulate, void* workspace, size_t workspace_bytes,
                                   lsq_cuda_stream stream);
 
+/* Backward of one fused linear for callers that cannot allocate device
+ * memory.  The paper has no counterpart (its trainer allocates through
+ * PyTorch); this entry point exists for code that runs where a cudaMalloc is
+ * unavailable or unsafe: inside a host framework that owns the whole device
+ * pool and exposes no allocator, in a process held to a hard memory cap where
+ * an extra allocation mid-step could fail, or while a stream is being
+ * captured.
+ * Same arguments and results as lsq_nf4_lora_bwd without the workspace: the
+ * scratch (G and the dA/dB partial sums) is one fixed array of
+ * lsq_nf4_lora_bwd_noalloc_max_scratch() bytes (8 MiB) in the device memory of
+ * every GPU that loads the library, held until the process exits.  A size
+ * whose scratch exceeds it is rejected with LSQ_EINVAL before anything is
+ * enqueued.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current: make that first call
+ * before any stream capture.  Every call shares the array and leaves its last
+ * contents there; nothing in it needs to start at zero (each call writes all
+ * the scratch it reads).  Calls that overlap on the GPU (other streams or
+ * host threads) race on the array: the caller must serialise them. */
+size_t lsq_nf4_lora_bwd_noalloc_max_scratch(void);
+lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M,
+                                    const void* A, const void* B, int32_t r, float s, const float* u, void* dx,
+                                    float* dA, float* dB, int32_t accumulate, lsq_cuda_stream stream);
+
 /* ------------------------------------------------------------------------
  * Dense bf16 GEMM for the resident, unquantised lm_head ("Untied
  * embed_tokens + lm_head stay resident and unquantised", soup-cli diff, docs

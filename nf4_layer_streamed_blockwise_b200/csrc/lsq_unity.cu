@@ -7,3 +7,4 @@
 #include "layer_ops.cu"
 #include "attention.cu"
 #include "stream.cu"
+#include "noalloc.cu"

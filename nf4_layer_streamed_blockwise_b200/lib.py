@@ -69,6 +69,10 @@ _SIGS = {
                                          ctypes.POINTER(c_void_p), c_int32, c_float, ctypes.POINTER(c_void_p),
                                          c_void_p, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int32,
                                          c_void_p, c_size_t, c_void_p]),
+    "lsq_nf4_lora_bwd_noalloc_max_scratch": (c_size_t, []),
+    "lsq_nf4_lora_bwd_noalloc": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p, c_int64, c_void_p,
+                                           c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_int32, c_void_p]),
     "lsq_dense_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32,
                                  c_void_p]),
     "lsq_rmsnorm_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_float, c_void_p]),
@@ -250,6 +254,19 @@ def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int,
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd_multi", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(dx),
           _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (4 * n if r > 0 else 0))
+
+
+def lsq_nf4_lora_bwd_noalloc_max_scratch() -> int:
+    return int(_fn("lsq_nf4_lora_bwd_noalloc_max_scratch")())
+
+
+def lsq_nf4_lora_bwd_noalloc(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB, accumulate: int,
+                             stream=None):
+    """lsq_nf4_lora_bwd without a workspace argument: the library's own fixed
+    scratch array is used, for callers that cannot allocate device memory."""
+    cw = W.c()
+    _call("lsq_nf4_lora_bwd_noalloc", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
+          _p(dB), accumulate, _stream(stream), launches=1 + (4 if r > 0 else 0))
 
 
 def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int, stream=None):
