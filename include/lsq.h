@@ -100,8 +100,8 @@ lsq_status lsq_nf4_dequantize(const lsq_nf4_weight* w, void* w_bf16, lsq_cuda_st
  *
  * Y = residual + X deq(W)^T + s (X A^T) B^T,   U = X A^T
  * The frozen-base linear with a LoRA adapter that layer streaming trains
- * (themenonlab blog, "only the small LoRA adapter is actually resident and
- * trainable"; soup-cli diff docs "Layer Streaming", lora.r / lora.alpha).
+ * (themenonlab blog, "The trick: layer streaming": the adapter is the only
+ * trained part; soup-cli diff docs "Layer Streaming", lora.r / lora.alpha).
  * s = alpha / r.  The dequantised tile never reaches HBM: the kernel decodes
  * NF4 into shared memory and multiplies on the tensor cores (tcgen05, fp32
  * accumulation in TMEM); the rank-r path runs as two small MMAs, one in the
@@ -130,7 +130,7 @@ lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
  * Backward of the fused linear (frozen W: no weight gradient).
  *
  * G = dY B;  dX = dY deq(W) + s G A;  dB (+)= s dY^T U;  dA (+)= s G^T X.
- * The gradients that make "non-zero gradients at layer 0" hold (soup-cli
+ * The gradients whose presence at the first layer the pages test (soup-cli
  * diff, CHANGELOG [0.72.2], "Correctness").  dX runs on the tensor cores
  * against the dequantised tile in MN-major layout; dA and dB are
  * deterministic two-stage reductions over M (no atomics).
@@ -180,9 +180,8 @@ lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const void* x, cons
                                     float* dA, float* dB, int32_t accumulate, lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
- * Dense bf16 GEMM for the resident, unquantised lm_head ("Untied
- * embed_tokens + lm_head stay resident and unquantised", soup-cli diff, docs
- * "NF4 streaming").  tcgen05, fp32 accumulation.
+ * Dense bf16 GEMM for the lm_head, which the pages keep on the GPU and
+ * unquantised (soup-cli diff, docs "NF4 streaming").  tcgen05, fp32 accumulation.
  *  trans_b = 0:  out[M,N] = a[M,K] b[N,K]^T   (logits = h E^T)
  *  trans_b = 1:  out[M,N] = a[M,K] b[K,N]     (dh = dlogits E)
  *  out_f32 = 1: fp32 output, else bf16.  K % 8 == 0, N % 8 == 0. */
@@ -242,8 +241,8 @@ lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_
 /* ------------------------------------------------------------------------
  * Layer streaming scheduler.
  *
- * "The frozen base lives in CPU RAM and is streamed into two pre-allocated
- * VRAM buffers one decoder layer at a time" (soup-cli diff, CHANGELOG
+ * The frozen base sits in host RAM and reaches the GPU one decoder layer at a
+ * time through a pair of buffers allocated up front (soup-cli diff, CHANGELOG
  * [0.72.0]); `stream_buffers` 2..8, default 2 (docs "Layer Streaming");
  * page-locked RAM is what lets the copy overlap compute (docs "NF4
  * streaming", point 2); backward under gradient checkpointing re-streams the

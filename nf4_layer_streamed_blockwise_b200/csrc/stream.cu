@@ -8,9 +8,9 @@
 //  * compute on a layer starts only after that layer's upload completed
 //    (up_done event);
 //  * the layer currently being computed is never evicted.
-// The pages' design ("two pre-allocated VRAM buffers", stream_buffers 2..8,
-// a pinned store so the copy overlaps compute) is kept; the silent fallback to
-// pageable memory becomes LSQ_ENOTPINNED.
+// The pages' design (a pair of GPU buffers allocated up front, stream_buffers
+// 2..8, a page-locked store so that the copy overlaps compute) is kept; their
+// silent fallback to pageable memory becomes LSQ_ENOTPINNED.
 #include <vector>
 
 #include "host_common.h"

@@ -6,8 +6,8 @@ is quantised once, offline, to NF4 and kept in page-locked host RAM as one
 record per decoder layer; each training step streams the records through a
 small ring of HBM slots, forward 0 -> L-1, and under gradient checkpointing
 re-streams them L-1 -> 0 for the backward, recomputing each layer from its
-saved input; embed_tokens and lm_head stay resident and unquantised; only the
-LoRA adapters train (optimizer step at the end).
+saved input; the embedding and lm_head remain on the GPU unquantised; the
+LoRA adapters are the only trained parameters (optimizer step at the end).
 
 This module only allocates memory (torch), builds the host store and calls
 the library in order.  Every arithmetic step runs in the library's kernels.

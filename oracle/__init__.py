@@ -12,8 +12,9 @@ beyond what the definitions state.
 
 Sources.  The pages ("Soup" README snapshot; soup-cli 0.72.0 -> 0.72.2 diff,
 CHANGELOG [0.72.2] and docs/performance-and-quantization.md "Layer Streaming")
-say only that the frozen base is quantised once, offline, to NF4 and streamed
-as "the same quantised bytes through the same kernels", and that the trainer is
+say only that the frozen base is quantised to NF4 once, ahead of training, and
+that a streamed run feeds identical quantised bytes to identical kernels as a
+resident run, and that the trainer is
 a LoRA SFT trainer with gradient checkpointing.  They fix neither the codebook,
 the block size, the absmax type, the nibble order nor the LoRA maths; where
 they are silent the reading taken is stated in the function that takes it.

@@ -2,11 +2,11 @@
 
 TEST INFRASTRUCTURE ONLY: see ``oracle/__init__.py``.
 
-The pages name the architectures ("Llama / Qwen only", soup-cli 0.72.0 ->
-0.72.2 diff, docs "Layer Streaming", "Honest scope"), the task (causal-LM SFT,
-``task: sft``), gradient checkpointing "handled per-layer by the streamer"
-(same section, example config) and that embed_tokens and lm_head stay
-resident and unquantised (same section, "NF4 streaming").  They give no
+The pages restrict streaming to Llama and Qwen models (soup-cli 0.72.0 ->
+0.72.2 diff, docs "Layer Streaming", "Honest scope"), name the task (causal-LM
+SFT, ``task: sft``), say the streamer applies gradient checkpointing layer by
+layer (same section, example config) and keep the embedding and lm_head on the
+GPU in full precision (same section, "NF4 streaming").  They give no
 formula.  The forward here is the plain definition of a pre-norm Llama/Qwen
 decoder layer, written in PyTorch CPU ops in float64:
 

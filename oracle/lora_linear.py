@@ -2,11 +2,11 @@
 
 TEST INFRASTRUCTURE ONLY: see ``oracle/__init__.py``.
 
-The pages describe the trainer as LoRA on a frozen NF4 base where "only the
-small LoRA adapter is actually resident and trainable" (themenonlab blog, "The
-trick: layer streaming"; soup-cli 0.72.0 -> 0.72.2 diff, docs "Layer
-Streaming", config keys lora.r / lora.alpha) and require non-zero gradients at
-layer 0 (CHANGELOG [0.72.2], "Correctness").  The maths is the plain LoRA
+The pages describe the trainer as LoRA on a frozen NF4 base in which the
+adapter is the only trained and permanently resident part (themenonlab blog,
+"The trick: layer streaming"; soup-cli 0.72.0 -> 0.72.2 diff, docs "Layer
+Streaming", config keys lora.r / lora.alpha), and they test that the first
+layer still receives gradients (CHANGELOG [0.72.2], "Correctness").  The maths is the plain LoRA
 definition (Hu et al. 2021): with W' = deq(W) [N, K], A [r, K], B [N, r] and
 s = alpha / r,
 

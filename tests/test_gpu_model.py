@@ -3,9 +3,10 @@
 * per-step loss against the fp64 oracle within 1e-3 relative (whole-model
   configurations), LoRA gradients within the derived tolerance below;
 * streamed == resident bit for bit: logits, every LoRA gradient and a 5-step
-  loss curve, for several slot counts (the pages' regression test: "the same
-  quantised bytes through the same kernels");
-* non-zero gradients at layer 0 (the pages' other streaming regression test).
+  loss curve, for several slot counts (the pages' regression test: a
+  streamed run feeds identical quantised bytes to identical kernels);
+* the first layer's LoRA gradients are not zero (the pages' other streaming
+  regression check).
 
 Gradient tolerance: the GPU keeps activations in bf16 between kernels (as the
 pages' bf16 trainer does) while the oracle is fp64 end to end; each bf16
