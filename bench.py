@@ -213,6 +213,7 @@ def h2d_bandwidth(torch, nbytes=128 << 20, reps=10):
 
 def timed_steps(torch, dist, tr, steps, ids_list, world, instrument=False, e2e=False, host_ids=None,
                 loss_host=None):
+    from nf4_layer_streamed_blockwise_b200 import dist as DP
     if instrument:
         tr.timeline = []
     if dist is not None:
@@ -226,19 +227,14 @@ def timed_steps(torch, dist, tr, steps, ids_list, world, instrument=False, e2e=F
         else:
             tr.set_ids(ids_list[i % len(ids_list)])
         tr.forward_backward()
-        if world > 1:
-            dist.all_reduce(tr.lora.grad)
-            tr.lora.grad.div_(world)
+        DP.average_gradients(tr.lora.grad, world)
         tr.optimizer_step()
         if e2e:
             loss_host[i].copy_(tr.loss_dev, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = DP.max_over_ranks(e0.elapsed_time(e1), world, device="cuda")
     if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     if instrument:
         tl, tr.timeline = tr.timeline, None
@@ -252,15 +248,14 @@ def our_arm(a):
     from nf4_layer_streamed_blockwise_b200 import lib as L
     from nf4_layer_streamed_blockwise_b200.trainer import StreamedLoraTrainer
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from nf4_layer_streamed_blockwise_b200 import dist as DP
+    rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
+    rank, world, local = DP.init_from_env("nccl")
     dist = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     shape = S.SHAPES[a.shape]
     peaks, peaks_src = load_peaks()
 
@@ -270,9 +265,7 @@ def our_arm(a):
     for i in range(a.warmup):
         tr.set_ids(ids_list[i % 4])
         tr.forward_backward()
-        if world > 1:
-            dist.all_reduce(tr.lora.grad)
-            tr.lora.grad.div_(world)
+        DP.average_gradients(tr.lora.grad, world)
         tr.optimizer_step()
     torch.cuda.synchronize()
     torch.cuda.reset_peak_memory_stats()

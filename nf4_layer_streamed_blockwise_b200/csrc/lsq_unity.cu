@@ -3,6 +3,7 @@
 #include "abi.cu"
 #include "nf4_quant.cu"
 #include "gemm_tc.cu"
+#include "gemm_nf4.cu"
 #include "lora_grad.cu"
 #include "layer_ops.cu"
 #include "attention.cu"
