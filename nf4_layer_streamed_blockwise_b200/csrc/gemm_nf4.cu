@@ -61,6 +61,7 @@ struct Seg {
   const float* absmax;
   const __nv_bfloat16* la;   // LoRA A [r, K_in]
   const __nv_bfloat16* lb;   // LoRA B [n, r]
+  const __nv_bfloat16* lat;  // DX: A^T [K_in, rp], columns >= r zero
   __nv_bfloat16* y;          // FWD output [M, n]
   const __nv_bfloat16* res;  // FWD residual [M, n] or null
   float* uo;                 // U (FWD) or G (DX) [M, r] or null
@@ -82,7 +83,7 @@ struct Params {
 struct Maps {
   CUtensorMap a[3];  // FWD: x; DX: dy of each segment (box 64 x 256 rows, 128B swizzle)
   CUtensorMap c[3];  // packed codes of each segment
-  CUtensorMap l[3];  // FWD: LoRA A of each segment (box 64 x rp)
+  CUtensorMap l[3];  // LoRA operand of the main loop, box 64 x rp rows: FWD A [r, K]; DX B^T [rp, n]
 };
 
 __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
@@ -175,13 +176,14 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         if (!mbar_wait(&empty[s], ph ^ 1u, 411)) break;
         uint8_t* a_dst = smem + C::OFF_A + s * A_BYTES;
         uint8_t* c_dst = smem + C::OFF_C + s * C::C_BYTES;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + ((MODE == FWD && lora) ? p.rp * 128 : 0)));
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + (lora ? p.rp * 128 : 0)));
         mbar_arrive_expect_tx(&cfull[s], (uint32_t)C::C_BYTES);
         if (MODE == DX) {
           const int sg = seg_of_block(p, i);
           const int nb = i - p.seg[sg].first;
           tma_load_2d(a_dst, &maps.a[sg], &full[s], nb * BK, m0);
           tma_load_2d(c_dst, &maps.c[sg], &cfull[s], n0 / 2, nb * BK);
+          if (lora) tma_load_2d(smem + C::OFF_L + s * C::L_BYTES, &maps.l[sg], &full[s], nb * BK, 0);
         } else {
           tma_load_2d(a_dst, &maps.a[0], &full[s], i * BK, m0);
           tma_load_2d(c_dst, &maps.c[seg], &cfull[s], i * (BK / 2), n0);
@@ -306,50 +308,23 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
       constexpr int KC = BN / 64;
       const int nl = t / KC, kc = t % KC;
       const int kcol = n0 + kc * 64;
-      // LoRA B^T tile [rp rows (j) x 64 (n)]: thread takes n = t & 63, j in [g*jq, g*jq + jq)
-      const int bn = t & 63, g = t >> 6;
-      const int jq = (p.rp + KC - 1) / KC;  // <= 32
-      float a_nx = 0.f;
-      uint16_t bl_nx[32];
-      auto fetch = [&](int i, float& a, uint16_t* bl) {
+      auto absmax_of = [&](int i) {
         const int sgi = seg_of_block(p, i);
         const Seg& sg = p.seg[sgi];
         const int nrow = (i - sg.first) * BK + nl;
-        a = (nrow < sg.n && kcol < p.K) ? __ldg(sg.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
-        if (lora) {
-          const int brow = (i - sg.first) * BK + bn;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = g * jq + q;
-            bl[q] = 0;
-            if (q < jq && j < p.r && brow < sg.n)
-              bl[q] = __ldg(reinterpret_cast<const unsigned short*>(sg.lb) + (int64_t)brow * p.r + j);
-          }
-        }
+        return (nrow < sg.n && kcol < p.K) ? __ldg(sg.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
       };
-      if (p.nkb > 0) fetch(0, a_nx, bl_nx);
+      float a_nx = p.nkb > 0 ? absmax_of(0) : 0.0f;
       for (int i = 0; i < p.nkb; ++i) {
         const int s = i % NST;
         const uint32_t ph = (uint32_t)(i / NST) & 1u;
         const float a = a_nx;
-        uint16_t bl[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) bl[q] = bl_nx[q];
-        if (i + 1 < p.nkb) fetch(i + 1, a_nx, bl_nx);
+        if (i + 1 < p.nkb) a_nx = absmax_of(i + 1);
         if (!mbar_wait(&cfull[s], ph, 612)) break;
         const uint8_t* crow = smem + C::OFF_C + s * C::C_BYTES + nl * (BN / 2) + kc * 32;
         const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
         const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
         store_block_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + kc * 8192 + nl * 128, nl, c0, c1, a, s_cb);
-        if (lora) {
-          const uint32_t lbase = smem_u32(smem + C::OFF_L + s * C::L_BYTES);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = g * jq + q;
-            if (q < jq && j < p.rp)
-              st_shared_u16(lbase + j * 128 + ((uint32_t)((bn >> 3) ^ (j & 7)) << 4) + (bn & 7) * 2, bl[q]);
-          }
-        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
@@ -368,26 +343,26 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
       const uint32_t be = smem_u32(smem + C::OFF_BE);
       for (int row = e; row < BN; row += 128) {
         for (int jc = 0; jc < KE / 8; ++jc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float v2[2];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int j = jc * 8 + q * 2 + hh;
-              float v = 0.0f;
-              if (MODE == FWD) {
-                const int n = n0 + row;
-                if (j < p.r && n < p.seg[seg].n) v = __bfloat162float(p.seg[seg].lb[(int64_t)n * p.r + j]);
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (MODE == FWD) {
+            const int n = n0 + row, j0 = jc * 8;
+            if (n < p.seg[seg].n && j0 < p.r) {
+              const __nv_bfloat16* src = p.seg[seg].lb + (int64_t)n * p.r + j0;
+              if ((p.r & 7) == 0) {
+                w = __ldg(reinterpret_cast<const uint4*>(src));
               } else {
-                const int sg = j / p.rp, jj = j % p.rp, k = n0 + row;
-                if (jj < p.r && k < p.K) v = __bfloat162float(p.seg[sg].la[(int64_t)jj * p.K + k]);
+                float v[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = (j0 + q < p.r) ? __bfloat162float(src[q]) : 0.0f;
+                w = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                               pack_bf16x2(v[6], v[7]));
               }
-              v2[hh] = v;
             }
-            w[q] = pack_bf16x2(v2[0], v2[1]);
+          } else {
+            const int sg = (jc * 8) / p.rp, jj = (jc * 8) % p.rp, k = n0 + row;
+            if (k < p.K) w = __ldg(reinterpret_cast<const uint4*>(p.seg[sg].lat + (int64_t)k * p.rp + jj));
           }
-          st_shared_v4(be + (row >> 3) * (KE * 16) + jc * 128 + (row & 7) * 16, make_uint4(w[0], w[1], w[2], w[3]));
+          st_shared_v4(be + (row >> 3) * (KE * 16) + jc * 128 + (row & 7) * 16, w);
         }
       }
       // s * U (or s * G) as bf16, one operand per half
@@ -543,8 +518,9 @@ static lsq_status check_weight(const lsq_nf4_weight& w, int64_t K, const char* w
   return LSQ_OK;
 }
 
-lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const void* const* A,
-                     const void* const* B, int r, float s, void* dx, float* const* g_out, cudaStream_t stream) {
+lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
+                     const __nv_bfloat16* const* Bt, const __nv_bfloat16* const* At, int r, float s, void* dx,
+                     float* const* g_out, cudaStream_t stream) {
   const int64_t K = W[0].k_in;
   Params p;
   memset(&p, 0, sizeof(p));
@@ -566,8 +542,7 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
   for (int i = 0; i < nseg; ++i) {
     Seg& g = p.seg[i];
     g.absmax = W[i].absmax;
-    g.la = r > 0 ? static_cast<const __nv_bfloat16*>(A[i]) : nullptr;
-    g.lb = r > 0 ? static_cast<const __nv_bfloat16*>(B[i]) : nullptr;
+    g.lat = r > 0 ? At[i] : nullptr;
     g.uo = r > 0 ? g_out[i] : nullptr;
     g.n = (int)W[i].n_out;
     g.first = blocks;
@@ -577,6 +552,9 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
       return st;
     if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2, BN / 2,
                              BK, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
+      return st;
+    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bt[i], W[i].n_out, p.rp,
+                                      W[i].n_out * 2, BK, p.rp, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
       return st;
   }
   p.nkb = blocks;

@@ -3,24 +3,27 @@
 //   dB_seg = s dY_seg^T U_seg,  dA_seg = s G_seg^T X    (here)
 // dA and dB are skinny products (r <= 64 columns) reduced over the M token
 // rows, i.e. HBM-bound reads of dY and X.  Deterministic two-stage reduction:
-// stage 1 gives each CTA a 128-column panel and a chunk of rows (row tiles of
+// stage 1 gives each CTA a 256-column panel and a chunk of rows (row tiles of
 // P and Q double-buffered through shared memory with cp.async) and writes fp32
 // partial sums; stage 2 adds the partials of each output in a fixed order.
 // No atomics, so results are bit-identical run to run.  Every reduction of one
 // backward call (dA and dB of up to three linears) shares one launch per stage.
+#include <algorithm>
+
 #include "common.cuh"
 #include "host_common.h"
 
 namespace lsq {
 namespace tc {
-lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const void* const* A,
-                     const void* const* B, int r, float s, void* dx, float* const* g_out, cudaStream_t stream);
+lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
+                     const __nv_bfloat16* const* Bt, const __nv_bfloat16* const* At, int r, float s, void* dx,
+                     float* const* g_out, cudaStream_t stream);
 }
 
 namespace lg {
 
-constexpr int PANEL = 128;      // columns per CTA (2 per thread)
-constexpr int TR = 32;          // rows per shared-memory tile
+constexpr int PANEL = 256;      // columns per CTA (4 per thread)
+constexpr int TR = 16;          // rows per shared-memory tile
 constexpr int THREADS = 256;
 constexpr int TARGET_CTAS = 296;
 constexpr int MAXRED = 6;
@@ -52,42 +55,35 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// stage 1: blockIdx.x = panel (+ offsets of earlier reductions), blockIdx.y = row chunk
-__global__ void __launch_bounds__(THREADS) skinny_partial(const __grid_constant__ RedSet rs) {
-  __shared__ __align__(16) __nv_bfloat16 sP[2][TR][PANEL];
-  __shared__ __align__(16) float sQ[2][TR][64];
-  int rid = 0, px = blockIdx.x;
-  while (rid + 1 < rs.n && px >= rs.red[rid].panels) {
-    px -= rs.red[rid].panels;
-    ++rid;
-  }
-  const Red& R = rs.red[rid];
-  if ((int)blockIdx.y >= R.chunks) return;
-  const int r = rs.r;
-  const int64_t M = rs.M, C = R.C;
+// stage 1: blockIdx.x = panel (+ offsets of earlier reductions), blockIdx.y = row chunk.
+// Thread (cg, jg): columns c0 + 4 cg .. + 3, ranks j in [jg*jq, jg*jq + jq), jq = ceil(r/4);
+// per row it reads 4 bf16 of P (one 8-byte load) and its jq values of Q
+// (16-byte loads, the same address for the whole warp) for 4*jq FMAs.
+template <int JQ>
+__device__ __forceinline__ void skinny_body(const Red& R, int64_t M, int r, int blocky, int px,
+                                            __nv_bfloat16 (*sP)[TR][PANEL], float (*sQ)[TR][64]) {
+  const int64_t C = R.C;
   const int64_t c0 = (int64_t)px * PANEL;
-  const int64_t mb0 = (int64_t)blockIdx.y * R.mchunk;
+  const int64_t mb0 = (int64_t)blocky * R.mchunk;
   const int64_t mb1 = mb0 + R.mchunk < M ? mb0 + R.mchunk : M;
   const int tid = threadIdx.x;
-  const int cp = tid & 63, jg = tid >> 6;  // columns c0 + 2cp, +1; j in [jg*jq, jg*jq + jq)
-  const int jq = (r + 3) / 4;
-  float acc[2][16];
+  const int cg = tid & 63, jg = tid >> 6;
+  float acc[4][JQ];
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int q = 0; q < 16; ++q) acc[a][q] = 0.0f;
+    for (int q = 0; q < JQ; ++q) acc[a][q] = 0.0f;
 
   auto load = [&](int buf, int64_t mb) {
-    // P: TR rows x 128 columns = 512 chunks of 16 bytes (2 per thread)
+    // P: TR rows x 256 columns = 512 chunks of 16 bytes (2 per thread)
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = tid + u * THREADS;
-      const int row = idx >> 4, ch = idx & 15;
+      const int row = idx >> 5, ch = idx & 31;
       const int64_t m = mb + row, c = c0 + ch * 8;
       const bool v = m < mb1 && c < C;
       cp_async16(&sP[buf][row][ch * 8], v ? (const void*)(R.P + m * C + c) : (const void*)R.P, v);
     }
-    // Q: TR rows x r floats, as 16-byte chunks of whole rows (r % 4 == 0) or scalars
     if ((r & 3) == 0) {
       const int per = r / 4;
       for (int idx = tid; idx < TR * per; idx += THREADS) {
@@ -116,30 +112,59 @@ __global__ void __launch_bounds__(THREADS) skinny_partial(const __grid_constant_
     __syncthreads();
 #pragma unroll 4
     for (int row = 0; row < TR; ++row) {
-      const uint32_t pp = *reinterpret_cast<const uint32_t*>(&sP[buf][row][cp * 2]);
-      const float p0 = bf16lo(pp), p1 = bf16hi(pp);
+      const uint2 pp = *reinterpret_cast<const uint2*>(&sP[buf][row][cg * 4]);
+      const float p[4] = {bf16lo(pp.x), bf16hi(pp.x), bf16lo(pp.y), bf16hi(pp.y)};
+      float qv[JQ];
+      const float* qr = &sQ[buf][row][jg * JQ];
+      if (JQ % 4 == 0) {
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        if (q < jq) {
-          const float qv = sQ[buf][row][jg * jq + q];
-          acc[0][q] = fmaf(p0, qv, acc[0][q]);
-          acc[1][q] = fmaf(p1, qv, acc[1][q]);
+        for (int q = 0; q < JQ; q += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(qr + q);
+          qv[q] = f.x;
+          qv[q + 1] = f.y;
+          qv[q + 2] = f.z;
+          qv[q + 3] = f.w;
         }
+      } else {
+#pragma unroll
+        for (int q = 0; q < JQ; ++q) qv[q] = qr[q];
       }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int q = 0; q < JQ; ++q) acc[a][q] = fmaf(p[a], qv[q], acc[a][q]);
     }
     __syncthreads();
     buf ^= 1;
   }
 #pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    const int64_t c = c0 + cp * 2 + a;
+  for (int a = 0; a < 4; ++a) {
+    const int64_t c = c0 + cg * 4 + a;
     if (c >= C) continue;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const int j = jg * jq + q;
-      if (q < jq && j < r) R.part[((int64_t)blockIdx.y * C + c) * r + j] = acc[a][q];
+    for (int q = 0; q < JQ; ++q) {
+      const int j = jg * JQ + q;
+      if (j < r) R.part[((int64_t)blocky * C + c) * r + j] = acc[a][q];
     }
   }
+}
+
+__global__ void __launch_bounds__(THREADS) skinny_partial(const __grid_constant__ RedSet rs) {
+  __shared__ __align__(16) __nv_bfloat16 sP[2][TR][PANEL];
+  __shared__ __align__(16) float sQ[2][TR][64];
+  int rid = 0, px = blockIdx.x;
+  while (rid + 1 < rs.n && px >= rs.red[rid].panels) {
+    px -= rs.red[rid].panels;
+    ++rid;
+  }
+  const Red& R = rs.red[rid];
+  if ((int)blockIdx.y >= R.chunks) return;
+  const int jq = (rs.r + 3) / 4;
+  if (jq <= 1) skinny_body<1>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
+  else if (jq <= 2) skinny_body<2>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
+  else if (jq <= 4) skinny_body<4>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
+  else if (jq <= 8) skinny_body<8>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
+  else skinny_body<16>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
 }
 
 // stage 2: out (+)= s * sum over chunks (ascending) of the partials
@@ -155,6 +180,33 @@ __global__ void __launch_bounds__(256) skinny_reduce(const __grid_constant__ Red
     float* dst = R.transpose ? R.out + j * R.C + c : R.out + idx;
     const float v = rs.s * sum;
     *dst = rs.accumulate ? *dst + v : v;
+  }
+}
+
+// Rank-padded transposed copies of the LoRA operands for the dX kernel:
+// Bt [rp, n] (its main-loop operand, fetched by TMA) and At [K, rp] (its
+// epilogue operand, fetched as 16-byte rows); rows / columns >= r are zero.
+struct Prep {
+  const __nv_bfloat16* A[3];
+  const __nv_bfloat16* B[3];
+  __nv_bfloat16* At[3];
+  __nv_bfloat16* Bt[3];
+  int64_t n[3];
+  int64_t K;
+  int r, rp;
+};
+
+__global__ void __launch_bounds__(256) lora_prep(const __grid_constant__ Prep P) {
+  const int seg = blockIdx.y >> 1, which = blockIdx.y & 1;
+  const int64_t total = which == 0 ? (int64_t)P.rp * P.n[seg] : P.K * P.rp;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
+    if (which == 0) {  // Bt[j][n] = B[n][j]
+      const int64_t j = idx / P.n[seg], n = idx % P.n[seg];
+      P.Bt[seg][idx] = j < P.r ? P.B[seg][n * P.r + j] : __float2bfloat16_rn(0.0f);
+    } else {           // At[k][j] = A[j][k]
+      const int64_t j = idx / P.K, k = idx % P.K;
+      P.At[seg][k * P.rp + j] = j < P.r ? P.A[seg][j * P.K + k] : __float2bfloat16_rn(0.0f);
+    }
   }
 }
 
@@ -186,8 +238,12 @@ using namespace lsq;
 extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
   if (nseg < 1 || nseg > 3 || r <= 0 || M < 1 || !n_out) return 256;
+  const size_t rp = (size_t)(r + 15) / 16 * 16;
   size_t b = lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
-  for (int i = 0; i < nseg; ++i) b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
+  for (int i = 0; i < nseg; ++i) {
+    b += lg::round256(rp * (size_t)n_out[i] * 2) + lg::round256((size_t)k_in * rp * 2);
+    b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
+  }
   return b;
 }
 
@@ -226,6 +282,8 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   }
   if (r == 0 && !dx) return LSQ_OK;
   float* g[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* bt[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* at[3] = {nullptr, nullptr, nullptr};
   char* part = nullptr;
   if (r > 0) {
     const size_t need = lsq_nf4_lora_bwd_workspace_size(nseg, M, K, n_out, r);
@@ -235,9 +293,35 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     float* ws = static_cast<float*>(workspace);
     for (int i = 0; i < nseg; ++i) g[i] = ws + (size_t)i * M * r;
     part = static_cast<char*>(workspace) + lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
+    for (int i = 0; i < nseg; ++i) {
+      bt[i] = reinterpret_cast<__nv_bfloat16*>(part);
+      part += lg::round256((size_t)rp * (size_t)n_out[i] * 2);
+      at[i] = reinterpret_cast<__nv_bfloat16*>(part);
+      part += lg::round256((size_t)K * (size_t)rp * 2);
+    }
   }
   cudaStream_t cs = (cudaStream_t)stream;
-  if ((st = tc::launch_dx(nseg, W, dy, M, A, B, r, s, dx, g, cs)) != LSQ_OK) return st;
+  if (r > 0) {
+    lg::Prep P;
+    memset(&P, 0, sizeof(P));
+    int64_t most = 0;
+    for (int i = 0; i < nseg; ++i) {
+      P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
+      P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+      P.At[i] = at[i];
+      P.Bt[i] = bt[i];
+      P.n[i] = n_out[i];
+      most = std::max<int64_t>(most, std::max<int64_t>((int64_t)rp * n_out[i], K * rp));
+    }
+    P.K = K;
+    P.r = r;
+    P.rp = rp;
+    int64_t gx = (most + 255) / 256;
+    if (gx > 512) gx = 512;
+    lg::lora_prep<<<dim3((unsigned)gx, 2 * nseg), 256, 0, cs>>>(P);
+    LSQ_LAUNCH_CHECK("lora_prep");
+  }
+  if ((st = tc::launch_dx(nseg, W, dy, M, bt, at, r, s, dx, g, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
   lg::RedSet rs;
   memset(&rs, 0, sizeof(rs));

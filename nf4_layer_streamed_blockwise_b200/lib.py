@@ -130,7 +130,7 @@ def _check(name: str, status: int):
 
 
 # kernel launches issued by the library, counted per call on this side
-# (lsq_nf4_lora_bwd: the dX GEMM plus two reduction kernels for each of dA, dB)
+# (lsq_nf4_lora_bwd: a LoRA-operand transpose, the dX GEMM and two reduction kernels)
 LAUNCHES = [0]
 _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_nf4_lora_fwd": 1, "lsq_nf4_lora_fwd_multi": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
@@ -160,7 +160,9 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def _ptrs(seq) -> ctypes.Array:
+def _ptrs(seq) -> Optional[ctypes.Array]:
+    if seq is None:
+        return None
     arr = (c_void_p * len(seq))()
     for i, t in enumerate(seq):
         arr[i] = _p(t)
@@ -244,7 +246,7 @@ def lsq_nf4_lora_bwd(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx,
     cw = W.c()
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
-          _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (4 if r > 0 else 0))
+          _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (3 if r > 0 else 0))
 
 
 def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB,
@@ -253,7 +255,7 @@ def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int,
     cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd_multi", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(dx),
-          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (4 * n if r > 0 else 0))
+          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (3 if r > 0 else 0))
 
 
 def lsq_nf4_lora_bwd_noalloc_max_scratch() -> int:
@@ -266,7 +268,7 @@ def lsq_nf4_lora_bwd_noalloc(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float
     scratch array is used, for callers that cannot allocate device memory."""
     cw = W.c()
     _call("lsq_nf4_lora_bwd_noalloc", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
-          _p(dB), accumulate, _stream(stream), launches=1 + (4 if r > 0 else 0))
+          _p(dB), accumulate, _stream(stream), launches=1 + (3 if r > 0 else 0))
 
 
 def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int, stream=None):

@@ -93,6 +93,9 @@ def main():
         dB = [torch.empty(n, r, dtype=torch.float32, device="cuda") for n in ns]
         ws = torch.empty(L.lsq_nf4_lora_bwd_workspace_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
         run(f"bwd_{g}", fl, lambda: L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, A, B, r, s, us, dx, dA, dB, 0, ws))
+        fl0 = sum(2.0 * M * n * K for n in ns)
+        run(f"dx_{g}", fl0, lambda: L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, None, None, 0, 0.0, None, dx, None, None,
+                                                                0, None))
         del Ws, x, A, B, ys, us, dys, dx, dA, dB, ws
     hn = torch.randn(M, sh.d, **bf)
     E = torch.randn(sh.vocab, sh.d, **bf) * 0.02
