@@ -4,7 +4,7 @@
 Workload: Llama-3.1-8B-shaped stack (32 layers, hidden 4096, SwiGLU 14336,
 32 q / 8 kv heads, vocab 128256, RoPE theta 5e5), random-init bf16 weights
 quantised to NF4 (blocksize 64, fp32 absmax) and kept in page-locked host
-RAM, streamed per decoder layer through 2 HBM slots, forward 0 -> 31 and
+RAM, streamed per decoder layer through 8 HBM slots (the top of the 2..8 range), forward 0 -> 31 and
 re-streamed 31 -> 0 under gradient checkpointing; LoRA r=16 (alpha 16) on all
 seven linears; AdamW on the adapters; seeded uniform token ids, seq 512.
 
@@ -55,7 +55,7 @@ def args_():
     p.add_argument("--shape", default="llama-3.1-8b")
     p.add_argument("--batch", type=int, default=4)
     p.add_argument("--seq", type=int, default=512)
-    p.add_argument("--slots", type=int, default=2)
+    p.add_argument("--slots", type=int, default=8)
     p.add_argument("--no-resident", action="store_true")
     p.add_argument("--no-batch1", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")

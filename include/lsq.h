@@ -272,8 +272,20 @@ lsq_status lsq_layer_upload_async(lsq_stream* st, int32_t layer, int32_t slot);
  * backward): release the previously stepped layer's slot after the compute
  * work enqueued so far; upload `layer` if no slot holds it; make the compute
  * stream wait for its upload; prefetch layer + direction into the least
- * recently used other slot.  *slot_ptr = device address of the record. */
+ * recently used other slots (up to n_slots - 1 layers ahead, never evicting
+ * the layer in use or one already inside that window).  *slot_ptr = device
+ * address of the record. */
 lsq_status lsq_stream_step(lsq_stream* st, int32_t layer, int32_t direction, void** slot_ptr);
+/* The scheduler's slot policy without CUDA (for tests and planning): runs the
+ * same decisions lsq_stream_step makes for the n_steps (layers[i],
+ * directions[i]) calls and writes each action as three int32 (kind, layer,
+ * slot) into `actions` (host, 3 * max_actions ints): kind 1 = release the
+ * slot once the compute enqueued so far is done, 2 = upload the layer into
+ * the slot (after that release), 3 = compute waits for the layer's upload.
+ * *n_actions = the number written; EINVAL if more than max_actions. */
+lsq_status lsq_stream_simulate(int32_t n_layers, int32_t n_slots, int32_t n_steps, const int32_t* layers,
+                               const int32_t* directions, int32_t* actions, int32_t max_actions,
+                               int32_t* n_actions);
 /* Counters since create: uploads issued, bytes copied, uploads skipped
  * because the layer was still resident. */
 lsq_status lsq_stream_stats(const lsq_stream* st, int64_t* uploads, int64_t* bytes, int64_t* reused);

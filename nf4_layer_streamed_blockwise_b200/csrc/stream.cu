@@ -11,53 +11,133 @@
 // The pages' design (a pair of GPU buffers allocated up front, stream_buffers
 // 2..8, a page-locked store so that the copy overlaps compute) is kept; their
 // silent fallback to pageable memory becomes LSQ_ENOTPINNED.
+//
+// The slot policy (which slot to fill, how far to prefetch) is a CUDA-free
+// core that emits actions; the scheduler executes them with CUDA calls and
+// lsq_stream_simulate returns them, so the policy is testable without a GPU.
 #include <vector>
 
 #include "host_common.h"
 
-struct lsq_stream {
+namespace lsq {
+namespace sched {
+
+enum ActKind { RELEASE = 1, UPLOAD = 2, WAIT = 3 };
+struct Act {
+  int kind, layer, slot;
+};
+
+struct Policy {
   int n_layers = 0, n_slots = 0;
-  size_t record_bytes = 0;
-  std::vector<void*> slots;
-  std::vector<const void*> host;
-  cudaStream_t compute = nullptr, copy = nullptr;
   std::vector<int> slot_layer;         // layer held by a slot, -1 if none
   std::vector<int64_t> slot_tick;      // last step() use, for LRU
   std::vector<int> layer_slot;         // slot holding a layer, -1 if none
   std::vector<char> used_since_upload; // stepped since its last upload
-  std::vector<char> free_recorded;     // slot_free[slot] has been recorded
+  int cur = -1;                        // layer of the last step()
+  int64_t tick = 0, uploads = 0, reused = 0;
+
+  void init(int L, int S) {
+    n_layers = L;
+    n_slots = S;
+    slot_layer.assign(S, -1);
+    slot_tick.assign(S, 0);
+    layer_slot.assign(L, -1);
+    used_since_upload.assign(L, 0);
+    cur = -1;
+    tick = uploads = reused = 0;
+  }
+
+  // An empty slot if any, else the least recently used one, skipping slots
+  // whose layer is in `keep` (the layer in use and those prefetched ahead).
+  int victim(const int* keep, int nkeep) const {
+    int best = -1;
+    for (int s = 0; s < n_slots; ++s) {
+      bool kept = false;
+      for (int i = 0; i < nkeep; ++i) kept |= (keep[i] >= 0 && slot_layer[s] == keep[i]);
+      if (kept) continue;
+      if (slot_layer[s] < 0) return s;
+      if (best < 0 || slot_tick[s] < slot_tick[best]) best = s;
+    }
+    return best;
+  }
+
+  void place(int layer, int slot, std::vector<Act>& out) {
+    const int old = slot_layer[slot];
+    if (old >= 0) layer_slot[old] = -1;
+    if (layer_slot[layer] >= 0) slot_layer[layer_slot[layer]] = -1;
+    slot_layer[slot] = layer;
+    layer_slot[layer] = slot;
+    used_since_upload[layer] = 0;
+    uploads += 1;
+    out.push_back({UPLOAD, layer, slot});
+  }
+
+  // Begin compute on `layer` walking in `direction`; appends the actions.
+  void step(int layer, int direction, std::vector<Act>& out) {
+    if (cur >= 0 && cur != layer && layer_slot[cur] >= 0) out.push_back({RELEASE, cur, layer_slot[cur]});
+    if (layer_slot[layer] < 0) {
+      place(layer, victim(nullptr, 0), out);
+    } else if (used_since_upload[layer]) {
+      reused += 1;
+    }
+    const int slot = layer_slot[layer];
+    out.push_back({WAIT, layer, slot});
+    slot_tick[slot] = ++tick;
+    used_since_upload[layer] = 1;
+    cur = layer;
+    // prefetch up to n_slots - 1 layers ahead in the walking direction
+    int keep[8] = {layer, -1, -1, -1, -1, -1, -1, -1};
+    int nkeep = 1;
+    const int ahead = n_slots - 1 < 7 ? n_slots - 1 : 7;
+    for (int k = 1; k <= ahead; ++k) {
+      const int nxt = layer + k * direction;
+      if (nxt < 0 || nxt >= n_layers) break;
+      if (layer_slot[nxt] < 0) {
+        const int v = victim(keep, nkeep);
+        if (v < 0) break;
+        place(nxt, v, out);
+      }
+      keep[nkeep++] = nxt;
+    }
+  }
+};
+
+}  // namespace sched
+}  // namespace lsq
+
+struct lsq_stream {
+  lsq::sched::Policy pol;
+  size_t record_bytes = 0;
+  std::vector<void*> slots;
+  std::vector<const void*> host;
+  cudaStream_t compute = nullptr, copy = nullptr;
+  std::vector<char> free_recorded;  // slot_free[slot] has been recorded
   std::vector<cudaEvent_t> up_start, up_done, slot_free;
-  int cur = -1;  // layer of the last step()
-  int64_t tick = 0, uploads = 0, bytes = 0, reused = 0;
+  int64_t bytes = 0;
+  std::vector<lsq::sched::Act> acts;
 };
 
 namespace lsq {
 namespace sched {
 
-static lsq_status upload(lsq_stream* st, int layer, int slot) {
-  const int old = st->slot_layer[slot];
-  if (old >= 0) st->layer_slot[old] = -1;
-  if (st->free_recorded[slot]) LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[slot], 0));
-  LSQ_CUDA_TRY(cudaEventRecord(st->up_start[layer], st->copy));
-  LSQ_CUDA_TRY(cudaMemcpyAsync(st->slots[slot], st->host[layer], st->record_bytes, cudaMemcpyHostToDevice, st->copy));
-  LSQ_CUDA_TRY(cudaEventRecord(st->up_done[layer], st->copy));
-  st->slot_layer[slot] = layer;
-  st->layer_slot[layer] = slot;
-  st->used_since_upload[layer] = 0;
-  st->uploads += 1;
-  st->bytes += (int64_t)st->record_bytes;
-  return LSQ_OK;
-}
-
-// an empty slot if any, else the least recently used one; `keep` is excluded
-static int victim(const lsq_stream* st, int keep) {
-  int best = -1;
-  for (int s = 0; s < st->n_slots; ++s) {
-    if (s == keep) continue;
-    if (st->slot_layer[s] < 0) return s;
-    if (best < 0 || st->slot_tick[s] < st->slot_tick[best]) best = s;
+static lsq_status execute(lsq_stream* st) {
+  for (const Act& a : st->acts) {
+    if (a.kind == RELEASE) {
+      LSQ_CUDA_TRY(cudaEventRecord(st->slot_free[a.slot], st->compute));
+      st->free_recorded[a.slot] = 1;
+    } else if (a.kind == UPLOAD) {
+      if (st->free_recorded[a.slot]) LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[a.slot], 0));
+      LSQ_CUDA_TRY(cudaEventRecord(st->up_start[a.layer], st->copy));
+      LSQ_CUDA_TRY(cudaMemcpyAsync(st->slots[a.slot], st->host[a.layer], st->record_bytes, cudaMemcpyHostToDevice,
+                                   st->copy));
+      LSQ_CUDA_TRY(cudaEventRecord(st->up_done[a.layer], st->copy));
+      st->bytes += (int64_t)st->record_bytes;
+    } else if (a.kind == WAIT) {
+      LSQ_CUDA_TRY(cudaStreamWaitEvent(st->compute, st->up_done[a.layer], 0));
+    }
   }
-  return best;
+  st->acts.clear();
+  return LSQ_OK;
 }
 
 static bool is_pinned_host(const void* p) {
@@ -75,6 +155,10 @@ static void destroy_events(lsq_stream* st) {
       if (e) cudaEventDestroy(e);
 }
 
+static bool valid_slots(int n_layers, int n_slots) {
+  return n_slots >= 2 && (n_slots <= 8 || n_slots == n_layers);
+}
+
 }  // namespace sched
 }  // namespace lsq
 
@@ -86,7 +170,7 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   if (!cfg || !out || !cfg->slots || !cfg->host_records) return fail(LSQ_EINVAL, "lsq_stream_create: NULL argument");
   *out = nullptr;
   if (cfg->n_layers < 1 || cfg->record_bytes == 0) return fail(LSQ_EINVAL, "lsq_stream_create: empty model");
-  if (cfg->n_slots < 2 || (cfg->n_slots > 8 && cfg->n_slots != cfg->n_layers))
+  if (!valid_slots(cfg->n_layers, cfg->n_slots))
     return fail(LSQ_EINVAL, "lsq_stream_create: n_slots must be 2..8 or n_layers (resident), got %d", cfg->n_slots);
   if ((cudaStream_t)compute == (cudaStream_t)copy)
     return fail(LSQ_EINVAL, "lsq_stream_create: the copy stream must differ from the compute stream");
@@ -107,27 +191,22 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
       return fail(LSQ_ENOTPINNED, "lsq_stream_create: record %d is not page-locked host memory", l);
   }
   lsq_stream* st = new lsq_stream();
-  st->n_layers = cfg->n_layers;
-  st->n_slots = cfg->n_slots;
+  st->pol.init(cfg->n_layers, cfg->n_slots);
   st->record_bytes = cfg->record_bytes;
   st->slots.assign(cfg->slots, cfg->slots + cfg->n_slots);
   st->host.assign(cfg->host_records, cfg->host_records + cfg->n_layers);
   st->compute = (cudaStream_t)compute;
   st->copy = (cudaStream_t)copy;
-  st->slot_layer.assign(st->n_slots, -1);
-  st->slot_tick.assign(st->n_slots, 0);
-  st->free_recorded.assign(st->n_slots, 0);
-  st->layer_slot.assign(st->n_layers, -1);
-  st->used_since_upload.assign(st->n_layers, 0);
-  st->up_start.assign(st->n_layers, nullptr);
-  st->up_done.assign(st->n_layers, nullptr);
-  st->slot_free.assign(st->n_slots, nullptr);
+  st->free_recorded.assign(cfg->n_slots, 0);
+  st->up_start.assign(cfg->n_layers, nullptr);
+  st->up_done.assign(cfg->n_layers, nullptr);
+  st->slot_free.assign(cfg->n_slots, nullptr);
   cudaError_t e = cudaSuccess;
-  for (int l = 0; l < st->n_layers && e == cudaSuccess; ++l) {
+  for (int l = 0; l < cfg->n_layers && e == cudaSuccess; ++l) {
     e = cudaEventCreate(&st->up_start[l]);
     if (e == cudaSuccess) e = cudaEventCreate(&st->up_done[l]);
   }
-  for (int i = 0; i < st->n_slots && e == cudaSuccess; ++i)
+  for (int i = 0; i < cfg->n_slots && e == cudaSuccess; ++i)
     e = cudaEventCreateWithFlags(&st->slot_free[i], cudaEventDisableTiming);
   if (e != cudaSuccess) {
     destroy_events(st);
@@ -140,60 +219,63 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
 
 extern "C" lsq_status lsq_layer_upload_async(lsq_stream* st, int32_t layer, int32_t slot) {
   if (!st) return fail(LSQ_EINVAL, "lsq_layer_upload_async: NULL scheduler");
-  if (layer < 0 || layer >= st->n_layers || slot < 0 || slot >= st->n_slots)
+  Policy& p = st->pol;
+  if (layer < 0 || layer >= p.n_layers || slot < 0 || slot >= p.n_slots)
     return fail(LSQ_EINVAL, "lsq_layer_upload_async: layer %d / slot %d out of range", layer, slot);
-  if (st->cur >= 0 && st->layer_slot[st->cur] == slot && st->cur != layer)
-    return fail(LSQ_ESTATE, "lsq_layer_upload_async: slot %d holds layer %d, which is in use", slot, st->cur);
-  if (st->layer_slot[layer] == slot) return LSQ_OK;  // already there
-  if (st->layer_slot[layer] >= 0) {                 // move: forget the old copy
-    st->slot_layer[st->layer_slot[layer]] = -1;
-    st->layer_slot[layer] = -1;
-  }
-  return upload(st, layer, slot);
+  if (p.cur >= 0 && p.layer_slot[p.cur] == slot && p.cur != layer)
+    return fail(LSQ_ESTATE, "lsq_layer_upload_async: slot %d holds layer %d, which is in use", slot, p.cur);
+  if (p.layer_slot[layer] == slot) return LSQ_OK;  // already there
+  p.place(layer, slot, st->acts);
+  return execute(st);
 }
 
 extern "C" lsq_status lsq_stream_step(lsq_stream* st, int32_t layer, int32_t direction, void** slot_ptr) {
   if (!st || !slot_ptr) return fail(LSQ_EINVAL, "lsq_stream_step: NULL argument");
-  if (layer < 0 || layer >= st->n_layers) return fail(LSQ_EINVAL, "lsq_stream_step: layer %d out of range", layer);
+  if (layer < 0 || layer >= st->pol.n_layers) return fail(LSQ_EINVAL, "lsq_stream_step: layer %d out of range", layer);
   if (direction != 1 && direction != -1) return fail(LSQ_EINVAL, "lsq_stream_step: direction must be +1 or -1");
-  lsq_status s;
-  // release the previous layer once the compute work enqueued so far is done
-  if (st->cur >= 0 && st->cur != layer && st->layer_slot[st->cur] >= 0) {
-    const int ps = st->layer_slot[st->cur];
-    LSQ_CUDA_TRY(cudaEventRecord(st->slot_free[ps], st->compute));
-    st->free_recorded[ps] = 1;
+  st->pol.step(layer, direction, st->acts);
+  lsq_status s = execute(st);
+  if (s != LSQ_OK) return s;
+  *slot_ptr = st->slots[st->pol.layer_slot[layer]];
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_simulate(int32_t n_layers, int32_t n_slots, int32_t n_steps, const int32_t* layers,
+                                          const int32_t* directions, int32_t* actions, int32_t max_actions,
+                                          int32_t* n_actions) {
+  if (!layers || !directions || !actions || !n_actions) return fail(LSQ_EINVAL, "lsq_stream_simulate: NULL argument");
+  if (n_layers < 1 || !valid_slots(n_layers, n_slots) || n_steps < 0 || max_actions < 0)
+    return fail(LSQ_EINVAL, "lsq_stream_simulate: bad sizes");
+  Policy p;
+  p.init(n_layers, n_slots);
+  std::vector<Act> acts;
+  for (int i = 0; i < n_steps; ++i) {
+    if (layers[i] < 0 || layers[i] >= n_layers || (directions[i] != 1 && directions[i] != -1))
+      return fail(LSQ_EINVAL, "lsq_stream_simulate: step %d out of range", i);
+    p.step(layers[i], directions[i], acts);
   }
-  if (st->layer_slot[layer] < 0) {
-    const int v = victim(st, -1);
-    if ((s = upload(st, layer, v)) != LSQ_OK) return s;
-  } else if (st->used_since_upload[layer]) {
-    st->reused += 1;
+  if ((int64_t)acts.size() > max_actions)
+    return fail(LSQ_EINVAL, "lsq_stream_simulate: %zu actions exceed max_actions", acts.size());
+  for (size_t i = 0; i < acts.size(); ++i) {
+    actions[3 * i] = acts[i].kind;
+    actions[3 * i + 1] = acts[i].layer;
+    actions[3 * i + 2] = acts[i].slot;
   }
-  const int slot = st->layer_slot[layer];
-  LSQ_CUDA_TRY(cudaStreamWaitEvent(st->compute, st->up_done[layer], 0));
-  st->slot_tick[slot] = ++st->tick;
-  st->used_since_upload[layer] = 1;
-  st->cur = layer;
-  const int nxt = layer + direction;
-  if (nxt >= 0 && nxt < st->n_layers && st->layer_slot[nxt] < 0) {
-    const int v = victim(st, slot);
-    if (v >= 0 && (s = upload(st, nxt, v)) != LSQ_OK) return s;
-  }
-  *slot_ptr = st->slots[slot];
+  *n_actions = (int32_t)acts.size();
   return LSQ_OK;
 }
 
 extern "C" lsq_status lsq_stream_stats(const lsq_stream* st, int64_t* uploads, int64_t* bytes, int64_t* reused) {
   if (!st || !uploads || !bytes || !reused) return fail(LSQ_EINVAL, "lsq_stream_stats: NULL argument");
-  *uploads = st->uploads;
+  *uploads = st->pol.uploads;
   *bytes = st->bytes;
-  *reused = st->reused;
+  *reused = st->pol.reused;
   return LSQ_OK;
 }
 
 extern "C" lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float* ms) {
   if (!st || !ms) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: NULL argument");
-  if (layer < 0 || layer >= st->n_layers) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: layer out of range");
+  if (layer < 0 || layer >= st->pol.n_layers) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: layer out of range");
   LSQ_CUDA_TRY(cudaEventSynchronize(st->up_done[layer]));
   LSQ_CUDA_TRY(cudaEventElapsedTime(ms, st->up_start[layer], st->up_done[layer]));
   return LSQ_OK;
@@ -203,12 +285,11 @@ extern "C" lsq_status lsq_stream_reset(lsq_stream* st) {
   if (!st) return fail(LSQ_EINVAL, "lsq_stream_reset: NULL scheduler");
   LSQ_CUDA_TRY(cudaStreamSynchronize(st->copy));
   LSQ_CUDA_TRY(cudaStreamSynchronize(st->compute));
-  std::fill(st->slot_layer.begin(), st->slot_layer.end(), -1);
-  std::fill(st->layer_slot.begin(), st->layer_slot.end(), -1);
-  std::fill(st->slot_tick.begin(), st->slot_tick.end(), 0);
+  const int64_t up = st->pol.uploads, re = st->pol.reused;
+  st->pol.init(st->pol.n_layers, st->pol.n_slots);
+  st->pol.uploads = up;
+  st->pol.reused = re;
   std::fill(st->free_recorded.begin(), st->free_recorded.end(), 0);
-  std::fill(st->used_since_upload.begin(), st->used_since_upload.end(), 0);
-  st->cur = -1;
   return LSQ_OK;
 }
 

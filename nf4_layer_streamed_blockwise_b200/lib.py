@@ -96,6 +96,8 @@ _SIGS = {
     "lsq_stream_create": (c_int32, [ctypes.POINTER(lsq_stream_cfg), c_void_p, c_void_p, ctypes.POINTER(c_void_p)]),
     "lsq_layer_upload_async": (c_int32, [c_void_p, c_int32, c_int32]),
     "lsq_stream_step": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_void_p)]),
+    "lsq_stream_simulate": (c_int32, [c_int32, c_int32, c_int32, ctypes.POINTER(c_int32), ctypes.POINTER(c_int32),
+                                      ctypes.POINTER(c_int32), c_int32, ctypes.POINTER(c_int32)]),
     "lsq_stream_stats": (c_int32, [c_void_p, ctypes.POINTER(c_int64), ctypes.POINTER(c_int64),
                                    ctypes.POINTER(c_int64)]),
     "lsq_stream_upload_ms": (c_int32, [c_void_p, c_int32, ctypes.POINTER(c_float)]),
@@ -350,6 +352,18 @@ def lsq_stream_step(st: int, layer: int, direction: int) -> int:
     out = c_void_p()
     _call("lsq_stream_step", st, layer, direction, ctypes.byref(out))
     return out.value
+
+
+def lsq_stream_simulate(n_layers: int, n_slots: int, steps):
+    """steps: [(layer, direction), ...] -> [(kind, layer, slot), ...] (1 release, 2 upload, 3 wait)."""
+    n = len(steps)
+    layers = (c_int32 * max(n, 1))(*[l for l, _ in steps])
+    dirs = (c_int32 * max(n, 1))(*[d for _, d in steps])
+    cap = 4 * n * (n_slots + 2) + 16
+    acts = (c_int32 * (3 * cap))()
+    cnt = c_int32(0)
+    _call("lsq_stream_simulate", n_layers, n_slots, n, layers, dirs, acts, cap, ctypes.byref(cnt))
+    return [(acts[3 * i], acts[3 * i + 1], acts[3 * i + 2]) for i in range(cnt.value)]
 
 
 def lsq_stream_stats(st: int):
