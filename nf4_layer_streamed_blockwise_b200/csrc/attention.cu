@@ -56,6 +56,25 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* s, const __nv_bfloat16*
   }
 }
 
+// the same copy with cp.async (16-byte chunks, rows past S zero-filled); the
+// caller commits the group
+template <int D>
+__device__ __forceinline__ void load_tile_async(__nv_bfloat16* s, const __nv_bfloat16* g, int b, int p0, int rows,
+                                                int S, int H, int h, int nthreads) {
+  constexpr int C = D / 8;
+  for (int idx = threadIdx.x; idx < rows * C; idx += nthreads) {
+    const int r = idx / C, c = idx % C;
+    const int p = p0 + r;
+    const bool v = p < S;
+    const __nv_bfloat16* src = v ? g + (((int64_t)b * S + p) * H + h) * D + c * 8 : g;
+    const uint32_t dst = smem_u32(s + r * Tile<D>::LD + c * 8);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(v ? 16 : 0) : "memory");
+  }
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // A fragment (16 x 16, rows r0.., cols c0..) of a row-major smem tile
 template <int D>
 __device__ __forceinline__ void frag_a(const __nv_bfloat16* s, int r0, int c0, uint32_t* a) {
@@ -96,17 +115,18 @@ __global__ void __launch_bounds__(128) fwd_kernel(const __nv_bfloat16* __restric
                                                   float* __restrict__ lse, int S, int Hq, int Hkv, float scale_log2) {
   extern __shared__ __align__(16) uint8_t smem[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sK = sQ + BQ * Tile<D>::LD;
-  __nv_bfloat16* sV = sK + BKV * Tile<D>::LD;
+  __nv_bfloat16* sKb = sQ + BQ * Tile<D>::LD;        // 2 buffers of K
+  __nv_bfloat16* sVb = sKb + 2 * BKV * Tile<D>::LD;  // 2 buffers of V
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (Hq / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = qb * BQ;
-  load_tile<D>(sQ, q, b, q0, BQ, S, Hq, h, 128);
-  __syncthreads();
+  const int nkb = (min(q0 + BQ, S) + BKV - 1) / BKV;
+  load_tile_async<D>(sQ, q, b, q0, BQ, S, Hq, h, 128);
+  load_tile_async<D>(sKb, k, b, 0, BKV, S, Hkv, hk, 128);
+  load_tile_async<D>(sVb, v, b, 0, BKV, S, Hkv, hk, 128);
+  cp_commit();
   uint32_t qf[D / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks) frag_a<D>(sQ, warp * 16, ks * 16, qf[ks]);
 
   float oacc[D / 8][4];
 #pragma unroll
@@ -114,12 +134,24 @@ __global__ void __launch_bounds__(128) fwd_kernel(const __nv_bfloat16* __restric
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.0f, 0.0f};
   const int qi0 = q0 + warp * 16 + (lane >> 2);  // rows qi0 and qi0 + 8
 
-  const int nkb = (min(q0 + BQ, S) + BKV - 1) / BKV;
   for (int kb = 0; kb < nkb; ++kb) {
+    // prefetch the next key/value tile into the other buffer
+    if (kb + 1 < nkb) {
+      const int nb = (kb + 1) & 1;
+      load_tile_async<D>(sKb + nb * BKV * Tile<D>::LD, k, b, (kb + 1) * BKV, BKV, S, Hkv, hk, 128);
+      load_tile_async<D>(sVb + nb * BKV * Tile<D>::LD, v, b, (kb + 1) * BKV, BKV, S, Hkv, hk, 128);
+      cp_commit();
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
     __syncthreads();
-    load_tile<D>(sK, k, b, kb * BKV, BKV, S, Hkv, hk, 128);
-    load_tile<D>(sV, v, b, kb * BKV, BKV, S, Hkv, hk, 128);
-    __syncthreads();
+    if (kb == 0) {
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) frag_a<D>(sQ, warp * 16, ks * 16, qf[ks]);
+    }
+    const __nv_bfloat16* sK = sKb + (kb & 1) * BKV * Tile<D>::LD;
+    const __nv_bfloat16* sV = sVb + (kb & 1) * BKV * Tile<D>::LD;
     float sacc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.0f;
@@ -186,6 +218,7 @@ __global__ void __launch_bounds__(128) fwd_kernel(const __nv_bfloat16* __restric
         mma16816(oacc[2 * dp + 1], a, bb[2], bb[3]);
       }
     }
+    __syncthreads();  // this buffer is refilled by the prefetch two iterations on
   }
   // normalise and store
 #pragma unroll
@@ -242,14 +275,18 @@ __global__ void __launch_bounds__(128) dq_kernel(const __nv_bfloat16* __restrict
   extern __shared__ __align__(16) uint8_t smem[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
   __nv_bfloat16* sdO = sQ + BQ * Tile<D>::LD;
-  __nv_bfloat16* sK = sdO + BQ * Tile<D>::LD;
-  __nv_bfloat16* sV = sK + BKV * Tile<D>::LD;
+  __nv_bfloat16* sKb = sdO + BQ * Tile<D>::LD;       // 2 buffers of K
+  __nv_bfloat16* sVb = sKb + 2 * BKV * Tile<D>::LD;  // 2 buffers of V
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (Hq / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = qb * BQ;
-  load_tile<D>(sQ, q, b, q0, BQ, S, Hq, h, 128);
-  load_tile<D>(sdO, d_o, b, q0, BQ, S, Hq, h, 128);
+  const int nkb = (min(q0 + BQ, S) + BKV - 1) / BKV;
+  load_tile_async<D>(sQ, q, b, q0, BQ, S, Hq, h, 128);
+  load_tile_async<D>(sdO, d_o, b, q0, BQ, S, Hq, h, 128);
+  load_tile_async<D>(sKb, k, b, 0, BKV, S, Hkv, hk, 128);
+  load_tile_async<D>(sVb, v, b, 0, BKV, S, Hkv, hk, 128);
+  cp_commit();
   const int qi0 = q0 + warp * 16 + (lane >> 2);
   float lse2[2], dv[2];
 #pragma unroll
@@ -262,12 +299,19 @@ __global__ void __launch_bounds__(128) dq_kernel(const __nv_bfloat16* __restrict
   float dqacc[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) dqacc[i][0] = dqacc[i][1] = dqacc[i][2] = dqacc[i][3] = 0.0f;
-  const int nkb = (min(q0 + BQ, S) + BKV - 1) / BKV;
   for (int kb = 0; kb < nkb; ++kb) {
+    if (kb + 1 < nkb) {
+      const int nb = (kb + 1) & 1;
+      load_tile_async<D>(sKb + nb * BKV * Tile<D>::LD, k, b, (kb + 1) * BKV, BKV, S, Hkv, hk, 128);
+      load_tile_async<D>(sVb + nb * BKV * Tile<D>::LD, v, b, (kb + 1) * BKV, BKV, S, Hkv, hk, 128);
+      cp_commit();
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
     __syncthreads();
-    load_tile<D>(sK, k, b, kb * BKV, BKV, S, Hkv, hk, 128);
-    load_tile<D>(sV, v, b, kb * BKV, BKV, S, Hkv, hk, 128);
-    __syncthreads();
+    const __nv_bfloat16* sK = sKb + (kb & 1) * BKV * Tile<D>::LD;
+    const __nv_bfloat16* sV = sVb + (kb & 1) * BKV * Tile<D>::LD;
     float sacc[8][4], pacc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -313,6 +357,7 @@ __global__ void __launch_bounds__(128) dq_kernel(const __nv_bfloat16* __restrict
         mma16816(dqacc[2 * dp + 1], a, bb[2], bb[3]);
       }
     }
+    __syncthreads();
   }
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -340,35 +385,53 @@ __global__ void __launch_bounds__(128) dkv_kernel(const __nv_bfloat16* __restric
   extern __shared__ __align__(16) uint8_t smem[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);
   __nv_bfloat16* sV = sK + BKV * Tile<D>::LD;
-  __nv_bfloat16* sQ = sV + BKV * Tile<D>::LD;
-  __nv_bfloat16* sdO = sQ + BQ2 * Tile<D>::LD;
-  float* sL = reinterpret_cast<float*>(sdO + BQ2 * Tile<D>::LD);
-  float* sD = sL + BQ2;
+  __nv_bfloat16* sQb = sV + BKV * Tile<D>::LD;        // 2 buffers of Q
+  __nv_bfloat16* sdOb = sQb + 2 * BQ2 * Tile<D>::LD;  // 2 buffers of dO
+  float* sLb = reinterpret_cast<float*>(sdOb + 2 * BQ2 * Tile<D>::LD);
+  float* sDb = sLb + 2 * BQ2;
   const int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int group = Hq / Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = kb * BKV;
-  load_tile<D>(sK, k, b, k0, BKV, S, Hkv, hk, 128);
-  load_tile<D>(sV, v, b, k0, BKV, S, Hkv, hk, 128);
+  const int nq = (S - k0 + BQ2 - 1) / BQ2;  // query blocks at or after the key block, per head
+  const int total = group * nq;
+  auto issue = [&](int it, int buf) {
+    const int h = hk * group + it / nq, qs = k0 + (it % nq) * BQ2;
+    load_tile_async<D>(sQb + buf * BQ2 * Tile<D>::LD, q, b, qs, BQ2, S, Hq, h, 128);
+    load_tile_async<D>(sdOb + buf * BQ2 * Tile<D>::LD, d_o, b, qs, BQ2, S, Hq, h, 128);
+    cp_commit();
+    if (threadIdx.x < BQ2) {
+      const int qi = qs + threadIdx.x;
+      const int64_t idx = ((int64_t)b * Hq + h) * S + (qi < S ? qi : 0);
+      sLb[buf * BQ2 + threadIdx.x] = lse[idx] * LOG2E;
+      sDb[buf * BQ2 + threadIdx.x] = dvec[idx];
+    }
+  };
+  load_tile_async<D>(sK, k, b, k0, BKV, S, Hkv, hk, 128);
+  load_tile_async<D>(sV, v, b, k0, BKV, S, Hkv, hk, 128);
+  cp_commit();
+  if (total > 0) issue(0, 0);
   float dkacc[D / 8][4], dvacc[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dkacc[i][e] = dvacc[i][e] = 0.0f;
   const int kj0 = k0 + warp * 16 + (lane >> 2);  // this thread's key rows kj0, kj0 + 8
-  for (int hh = 0; hh < group; ++hh) {
-    const int h = hk * group + hh;
-    for (int qs = k0; qs < S; qs += BQ2) {
-      __syncthreads();
-      load_tile<D>(sQ, q, b, qs, BQ2, S, Hq, h, 128);
-      load_tile<D>(sdO, d_o, b, qs, BQ2, S, Hq, h, 128);
-      if (threadIdx.x < BQ2) {
-        const int qi = qs + threadIdx.x;
-        const int64_t idx = ((int64_t)b * Hq + h) * S + (qi < S ? qi : 0);
-        sL[threadIdx.x] = lse[idx] * LOG2E;
-        sD[threadIdx.x] = dvec[idx];
-      }
-      __syncthreads();
+  for (int it = 0; it < total; ++it) {
+    const int buf = it & 1;
+    const int qs = k0 + (it % nq) * BQ2;
+    if (it + 1 < total) {
+      issue(it + 1, buf ^ 1);
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
+    __syncthreads();
+    const __nv_bfloat16* sQ = sQb + buf * BQ2 * Tile<D>::LD;
+    const __nv_bfloat16* sdO = sdOb + buf * BQ2 * Tile<D>::LD;
+    const float* sL = sLb + buf * BQ2;
+    const float* sD = sDb + buf * BQ2;
+    {
       // S^T (16 keys x 32 queries) and dP^T = V dO^T
       float st[4][4], dpt[4][4];
 #pragma unroll
@@ -421,6 +484,7 @@ __global__ void __launch_bounds__(128) dkv_kernel(const __nv_bfloat16* __restric
         }
       }
     }
+    __syncthreads();
   }
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -439,7 +503,7 @@ __global__ void __launch_bounds__(128) dkv_kernel(const __nv_bfloat16* __restric
 template <int D>
 static lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int Hq,
                           int Hkv, cudaStream_t st) {
-  const size_t smem = (size_t)(BQ + 2 * BKV) * Tile<D>::LD * 2;
+  const size_t smem = (size_t)(BQ + 4 * BKV) * Tile<D>::LD * 2;
   static int cfg[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -459,8 +523,8 @@ template <int D>
 static lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o, const float* lse,
                           const float* dvec, void* dq, void* dk, void* dv, int B, int S, int Hq, int Hkv,
                           cudaStream_t st) {
-  const size_t smem_q = (size_t)(2 * BQ + 2 * BKV) * Tile<D>::LD * 2;
-  const size_t smem_kv = (size_t)(2 * BKV + 2 * BQ2) * Tile<D>::LD * 2 + 2 * BQ2 * sizeof(float);
+  const size_t smem_q = (size_t)(2 * BQ + 4 * BKV) * Tile<D>::LD * 2;
+  const size_t smem_kv = (size_t)(2 * BKV + 4 * BQ2) * Tile<D>::LD * 2 + 4 * BQ2 * sizeof(float);
   static int cfg[64];
   int dev = 0;
   cudaGetDevice(&dev);

@@ -13,10 +13,16 @@
 //   4          TMA producer: activation tile (256 rows, 128-byte swizzle),
 //              packed NF4 codes, and (FWD) the LoRA-down tile
 //   5          MMA issuer + TMEM owner
-//   6 ..       BN/32 dequantiser warps: one thread per 64-element NF4 block per
-//              stage -> one 128-byte row of the swizzled bf16 operand
-// TMEM columns: acc half h at [h*BN, h*BN + BN); rank-r product of half h at
-// [2*BN + h*KE, 2*BN + h*KE + KE), KE = (DX: nseg) * rp.  2*BN + 2*KE <= 512.
+//   6 ..       BN/16 dequantiser warps: two threads per 64-element NF4 block per
+//              stage, each writing half of one 128-byte row of the swizzled
+//              bf16 operand
+// The rank-r down product rides in the same MMA as the base GEMM: the LoRA
+// operand tile sits right after the weight tile in shared memory, so one MMA
+// per half (N = BN + LW) reads the activation slice once and writes
+// [acc | U] (FWD, LW = rp: A's rows appended to W's) or [dX | G] (DX, LW = 64:
+// each segment's B in its own rank-padded column range, so the segments' G
+// stay apart).  TMEM columns of half h: [h*NW, h*NW + BN) accumulator,
+// [h*NW + BN, h*NW + NW) the rank-r product; NW = BN + LW, 2*NW <= 512.
 //
 // The LoRA-up product runs on the tensor cores: after the main loop the
 // epilogue writes s*U (or s*G) as bf16 into shared memory and the MMA warp adds
@@ -37,16 +43,15 @@ constexpr int A_BYTES = BM * BK * 2;  // 32 KB
 
 template <int BN>
 struct Cfg {
-  static constexpr int DQ_WARPS = BN / 32;
+  static constexpr int DQ_WARPS = BN / 16;  // two threads per 64-element NF4 block
   static constexpr int NTHREADS = (6 + DQ_WARPS) * 32;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int W_BYTES = BN * BK * 2;             // dequantised weight tile
+  static constexpr int B_BYTES = W_BYTES + KE_MAX * BK * 2;  // + LoRA operand tile (<= 64 x 64)
   static constexpr int C_BYTES = BN * BK / 2;
-  static constexpr int L_BYTES = KE_MAX * BK * 2;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + NST * A_BYTES;
   static constexpr int OFF_C = OFF_B + NST * B_BYTES;
-  static constexpr int OFF_L = OFF_C + NST * C_BYTES;
-  static constexpr int OFF_BAR = OFF_L + NST * L_BYTES;
+  static constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
   // epilogue LoRA operands, aliased onto the stages (used after the main loop)
   static constexpr int OFF_UE = 0;                          // 2 x [128 x KE] bf16
   static constexpr int OFF_BE = 2 * HM * KE_MAX * 2;        // [BN x KE] bf16
@@ -83,7 +88,8 @@ struct Params {
 struct Maps {
   CUtensorMap a[3];  // FWD: x; DX: dy of each segment (box 64 x 256 rows, 128B swizzle)
   CUtensorMap c[3];  // packed codes of each segment
-  CUtensorMap l[3];  // LoRA operand of the main loop, box 64 x rp rows: FWD A [r, K]; DX B^T [rp, n]
+  CUtensorMap l[3];  // LoRA operand of the main loop: FWD A [r, K] (box 64 x rp rows);
+                     // DX rank-padded B [n, 64] (box 64 x 64 rows)
 };
 
 __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
@@ -110,12 +116,14 @@ __device__ __forceinline__ uint4 dq8(uint32_t w, float a, const float* cb) {
   return o;
 }
 
-// one NF4 block (64 values) -> one 128-byte row of a 128B-swizzled tile
-__device__ __forceinline__ void store_block_row(uint32_t row_addr, int row, uint4 c0, uint4 c1, float a,
-                                                const float* cb) {
-  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+// half of an NF4 block (32 values, 16 code bytes) -> 16-byte chunks
+// half*4 .. half*4+3 of one 128-byte row of a 128B-swizzled tile
+__device__ __forceinline__ void store_half_row(uint32_t row_addr, int row, int half, uint4 c, float a,
+                                               const float* cb) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) st_shared_v4(row_addr + ((uint32_t)(j ^ (row & 7)) << 4), dq8(w[j], a, cb));
+  for (int q = 0; q < 4; ++q)
+    st_shared_v4(row_addr + ((uint32_t)((half * 4 + q) ^ (row & 7)) << 4), dq8(w[q], a, cb));
 }
 
 template <int MODE, int BN>
@@ -176,26 +184,29 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         if (!mbar_wait(&empty[s], ph ^ 1u, 411)) break;
         uint8_t* a_dst = smem + C::OFF_A + s * A_BYTES;
         uint8_t* c_dst = smem + C::OFF_C + s * C::C_BYTES;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + (lora ? p.rp * 128 : 0)));
+        const uint32_t lbytes = lora ? (MODE == DX ? 64u * 128u : (uint32_t)p.rp * 128u) : 0u;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)A_BYTES + lbytes);
+        uint8_t* l_dst = smem + C::OFF_B + s * C::B_BYTES + C::W_BYTES;
         mbar_arrive_expect_tx(&cfull[s], (uint32_t)C::C_BYTES);
         if (MODE == DX) {
           const int sg = seg_of_block(p, i);
           const int nb = i - p.seg[sg].first;
           tma_load_2d(a_dst, &maps.a[sg], &full[s], nb * BK, m0);
           tma_load_2d(c_dst, &maps.c[sg], &cfull[s], n0 / 2, nb * BK);
-          if (lora) tma_load_2d(smem + C::OFF_L + s * C::L_BYTES, &maps.l[sg], &full[s], nb * BK, 0);
+          if (lora) tma_load_2d(l_dst, &maps.l[sg], &full[s], 0, nb * BK);
         } else {
           tma_load_2d(a_dst, &maps.a[0], &full[s], i * BK, m0);
           tma_load_2d(c_dst, &maps.c[seg], &cfull[s], i * (BK / 2), n0);
-          if (lora) tma_load_2d(smem + C::OFF_L + s * C::L_BYTES, &maps.l[seg], &full[s], i * BK, 0);
+          if (lora) tma_load_2d(l_dst, &maps.l[seg], &full[s], i * BK, 0);
         }
       }
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t id_main = idesc_bf16(HM, BN, 0, MODE == DX ? 1 : 0);
-      const uint32_t id_lora = idesc_bf16(HM, p.rp > 0 ? p.rp : 16, 0, 0);
+      const int LW = lora ? (MODE == DX ? 64 : p.rp) : 0;  // LoRA columns appended to the weight tile
+      const int NW = BN + LW;
+      const uint32_t id_main = idesc_bf16(HM, NW, 0, MODE == DX ? 1 : 0);
       const uint32_t id_ep = idesc_bf16(HM, BN, 0, 0);
       bool ok = true;
       for (int i = 0; i < p.nkb; ++i) {
@@ -208,14 +219,6 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         tc_fence_after();
         const uint32_t a_base = smem_u32(smem + C::OFF_A + s * A_BYTES);
         const uint32_t b_base = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
-        const uint32_t l_base = smem_u32(smem + C::OFF_L + s * C::L_BYTES);
-        uint32_t ucol = 2 * BN;
-        bool first = (i == 0);
-        if (MODE == DX) {
-          const int sg = seg_of_block(p, i);
-          ucol = 2 * BN + sg * p.rp;
-          first = (i == p.seg[sg].first);
-        }
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bd = (MODE == DX) ? smem_desc(b_base + kk * 2048, 8192, 1024, 2)
@@ -223,10 +226,7 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint64_t ad = smem_desc(a_base + h * (HM * 128) + kk * 32, 16, 1024, 2);
-            tc_mma(tmem + h * BN, ad, bd, id_main, (i | kk) != 0);
-            if (lora)
-              tc_mma(tmem + ucol + h * KE, ad, smem_desc(l_base + kk * 32, 16, 1024, 2), id_lora,
-                     !(first && kk == 0));
+            tc_mma(tmem + h * NW, ad, bd, id_main, (i | kk) != 0);
           }
         }
         tc_commit(&empty[s]);
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
             for (int h = 0; h < 2; ++h) {
               const uint32_t ue = smem_u32(smem + C::OFF_UE + h * HM * KE_MAX * 2);
               for (int kk = 0; kk < KE / 16; ++kk)
-                tc_mma(tmem + h * BN, smem_desc(ue + kk * 256, 128, KE * 16, 0),
+                tc_mma(tmem + h * NW, smem_desc(ue + kk * 256, 128, KE * 16, 0),
                        smem_desc(be + kk * 256, 128, KE * 16, 0), id_ep, 1);
             }
             tc_commit(afull);
@@ -257,11 +257,14 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
     }
   } else if (warp >= 6) {
     // ---------------------------------------------------------------- NF4 dequantisers
-    const int t = threadIdx.x - 6 * 32;  // 0 .. BN-1
+    const int t = threadIdx.x - 6 * 32;  // 0 .. 2*BN-1
     const int KB = p.K / 64;
     if (MODE == FWD) {
+      // thread -> (row, half): consecutive lanes read consecutive 16-byte code
+      // chunks and write conflict-free swizzled chunks
+      const int row = t >> 1, half = t & 1;
       const Seg& sg = p.seg[seg];
-      const int n = n0 + t;
+      const int n = n0 + row;
       const bool valid = n < sg.n;
       const float* arow = sg.absmax + (int64_t)(valid ? n : 0) * KB;
       const bool vec = (KB % 4) == 0;
@@ -283,10 +286,8 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         const int q = i & 3;
         const float a = vec ? (q == 0 ? acur.x : q == 1 ? acur.y : q == 2 ? acur.z : acur.w) : s0;
         if (!mbar_wait(&cfull[s], ph, 611)) break;
-        const uint8_t* crow = smem + C::OFF_C + s * C::C_BYTES + t * 32;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
-        store_block_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + t * 128, t, c0, c1, valid ? a : 0.0f, s_cb);
+        const uint4 c = *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C::C_BYTES + t * 16);
+        store_half_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + row * 128, row, half, c, valid ? a : 0.0f, s_cb);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
@@ -304,9 +305,10 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         }
       }
     } else {
-      // DX stage tile: 64 contraction rows (n) x BN output columns (k) = 64 x BN/64 blocks
-      constexpr int KC = BN / 64;
-      const int nl = t / KC, kc = t % KC;
+      // DX stage tile: 64 contraction rows (n) x BN output columns (k) = 64 x BN/64
+      // blocks; thread -> (k chunk, row, half) so that the 8 lanes of each
+      // store phase write 8 different swizzled chunks of 4 rows of one chunk
+      const int kc = t >> 7, nl = (t & 127) >> 1, half = t & 1;
       const int kcol = n0 + kc * 64;
       auto absmax_of = [&](int i) {
         const int sgi = seg_of_block(p, i);
@@ -321,10 +323,9 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         const float a = a_nx;
         if (i + 1 < p.nkb) a_nx = absmax_of(i + 1);
         if (!mbar_wait(&cfull[s], ph, 612)) break;
-        const uint8_t* crow = smem + C::OFF_C + s * C::C_BYTES + nl * (BN / 2) + kc * 32;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
-        store_block_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + kc * 8192 + nl * 128, nl, c0, c1, a, s_cb);
+        const uint4 c =
+            *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C::C_BYTES + nl * (BN / 2) + kc * 32 + half * 16);
+        store_half_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + kc * 8192 + nl * 128, nl, half, c, a, s_cb);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
@@ -334,6 +335,7 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
     // ---------------------------------------------------------------- epilogue (warps 0-3)
     const int e = threadIdx.x;  // TMEM lane = row of each half
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int NW = BN + (lora ? (MODE == DX ? 64 : p.rp) : 0);
     bool ok = mbar_wait(ufull, 0, 711);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) tc_fence_after();
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         const uint32_t ue = smem_u32(smem + C::OFF_UE + h * HM * KE_MAX * 2);
         for (int c = 0; c < KE / 16; ++c) {
           float v[16];
-          tmem_ld16(tmem + lane_base + 2 * BN + h * KE + c * 16, v);
+          tmem_ld16(tmem + lane_base + h * NW + BN + c * 16, v);
           tc_wait_ld();
           if (m < p.M) {
 #pragma unroll
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
         const int m = m0 + h * HM + e;
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_base + h * BN + c * 32, v);
+          tmem_ld32(tmem + lane_base + h * NW + c * 32, v);
           tc_wait_ld();
           if (m >= p.M) continue;
 #pragma unroll
@@ -519,7 +521,7 @@ static lsq_status check_weight(const lsq_nf4_weight& w, int64_t K, const char* w
 }
 
 lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
-                     const __nv_bfloat16* const* Bt, const __nv_bfloat16* const* At, int r, float s, void* dx,
+                     const __nv_bfloat16* const* Bp, const __nv_bfloat16* const* At, int r, float s, void* dx,
                      float* const* g_out, cudaStream_t stream) {
   const int64_t K = W[0].k_in;
   Params p;
@@ -553,8 +555,8 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
     if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2, BN / 2,
                              BK, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
-    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bt[i], W[i].n_out, p.rp,
-                                      W[i].n_out * 2, BK, p.rp, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp[i], 64, W[i].n_out, 64 * 2,
+                                      64, BK, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
       return st;
   }
   p.nkb = blocks;

@@ -16,7 +16,7 @@
 namespace lsq {
 namespace tc {
 lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
-                     const __nv_bfloat16* const* Bt, const __nv_bfloat16* const* At, int r, float s, void* dx,
+                     const __nv_bfloat16* const* Bp, const __nv_bfloat16* const* At, int r, float s, void* dx,
                      float* const* g_out, cudaStream_t stream);
 }
 
@@ -183,14 +183,16 @@ __global__ void __launch_bounds__(256) skinny_reduce(const __grid_constant__ Red
   }
 }
 
-// Rank-padded transposed copies of the LoRA operands for the dX kernel:
-// Bt [rp, n] (its main-loop operand, fetched by TMA) and At [K, rp] (its
-// epilogue operand, fetched as 16-byte rows); rows / columns >= r are zero.
+// Rank-padded copies of the LoRA operands for the dX kernel: Bp [n, 64] holds
+// segment seg's B in columns seg*rp .. seg*rp + r - 1 and zeros elsewhere (its
+// main-loop operand, appended to the weight tile, so each segment's G = dY B
+// lands in its own accumulator columns); At [K, rp] = A^T with zero columns
+// >= r (its epilogue operand, fetched as 16-byte rows).
 struct Prep {
   const __nv_bfloat16* A[3];
   const __nv_bfloat16* B[3];
   __nv_bfloat16* At[3];
-  __nv_bfloat16* Bt[3];
+  __nv_bfloat16* Bp[3];
   int64_t n[3];
   int64_t K;
   int r, rp;
@@ -198,11 +200,11 @@ struct Prep {
 
 __global__ void __launch_bounds__(256) lora_prep(const __grid_constant__ Prep P) {
   const int seg = blockIdx.y >> 1, which = blockIdx.y & 1;
-  const int64_t total = which == 0 ? (int64_t)P.rp * P.n[seg] : P.K * P.rp;
+  const int64_t total = which == 0 ? 64 * P.n[seg] : P.K * P.rp;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
-    if (which == 0) {  // Bt[j][n] = B[n][j]
-      const int64_t j = idx / P.n[seg], n = idx % P.n[seg];
-      P.Bt[seg][idx] = j < P.r ? P.B[seg][n * P.r + j] : __float2bfloat16_rn(0.0f);
+    if (which == 0) {  // Bp[n][c] = B[n][c - seg*rp] inside the segment's range, else 0
+      const int64_t n = idx / 64, c = idx % 64, j = c - (int64_t)seg * P.rp;
+      P.Bp[seg][idx] = (j >= 0 && j < P.r) ? P.B[seg][n * P.r + j] : __float2bfloat16_rn(0.0f);
     } else {           // At[k][j] = A[j][k]
       const int64_t j = idx / P.K, k = idx % P.K;
       P.At[seg][k * P.rp + j] = j < P.r ? P.A[seg][j * P.K + k] : __float2bfloat16_rn(0.0f);
@@ -241,7 +243,7 @@ extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64
   const size_t rp = (size_t)(r + 15) / 16 * 16;
   size_t b = lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
   for (int i = 0; i < nseg; ++i) {
-    b += lg::round256(rp * (size_t)n_out[i] * 2) + lg::round256((size_t)k_in * rp * 2);
+    b += lg::round256((size_t)64 * (size_t)n_out[i] * 2) + lg::round256((size_t)k_in * rp * 2);
     b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
   }
   return b;
@@ -282,7 +284,7 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   }
   if (r == 0 && !dx) return LSQ_OK;
   float* g[3] = {nullptr, nullptr, nullptr};
-  __nv_bfloat16* bt[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* bp[3] = {nullptr, nullptr, nullptr};
   __nv_bfloat16* at[3] = {nullptr, nullptr, nullptr};
   char* part = nullptr;
   if (r > 0) {
@@ -294,8 +296,8 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     for (int i = 0; i < nseg; ++i) g[i] = ws + (size_t)i * M * r;
     part = static_cast<char*>(workspace) + lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
     for (int i = 0; i < nseg; ++i) {
-      bt[i] = reinterpret_cast<__nv_bfloat16*>(part);
-      part += lg::round256((size_t)rp * (size_t)n_out[i] * 2);
+      bp[i] = reinterpret_cast<__nv_bfloat16*>(part);
+      part += lg::round256((size_t)64 * (size_t)n_out[i] * 2);
       at[i] = reinterpret_cast<__nv_bfloat16*>(part);
       part += lg::round256((size_t)K * (size_t)rp * 2);
     }
@@ -309,9 +311,9 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
       P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
       P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
       P.At[i] = at[i];
-      P.Bt[i] = bt[i];
+      P.Bp[i] = bp[i];
       P.n[i] = n_out[i];
-      most = std::max<int64_t>(most, std::max<int64_t>((int64_t)rp * n_out[i], K * rp));
+      most = std::max<int64_t>(most, std::max<int64_t>((int64_t)64 * n_out[i], K * rp));
     }
     P.K = K;
     P.r = r;
@@ -321,7 +323,7 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     lg::lora_prep<<<dim3((unsigned)gx, 2 * nseg), 256, 0, cs>>>(P);
     LSQ_LAUNCH_CHECK("lora_prep");
   }
-  if ((st = tc::launch_dx(nseg, W, dy, M, bt, at, r, s, dx, g, cs)) != LSQ_OK) return st;
+  if ((st = tc::launch_dx(nseg, W, dy, M, bp, at, r, s, dx, g, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
   lg::RedSet rs;
   memset(&rs, 0, sizeof(rs));
