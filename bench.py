@@ -362,7 +362,9 @@ def our_arm(a):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded uniform token ids, random-init weights)",
                 "config": workload_config(a, shape),
-                "roofline": {"bound": "tensor", "kernel": f"gemm_kernel ({dom})", "achieved": ach, "peak": peak,
+                "roofline": {"bound": "tensor",
+                             "kernel": f"fused NF4-LoRA linear, {dom} (nf4_pair_kernel + lora_down_kernel)",
+                             "achieved": ach, "peak": peak,
                              "unit": "TFLOP/s", "frac": ach / peak, "traffic": NCU_TRAFFIC,
                              "peak_source": f"{peaks_src} bf16_tflops_sustained"},
                 "fused_gemm": {"frac_of_sustained_peak": (all_flops / (all_ms * 1e-3) / 1e12) / peak,

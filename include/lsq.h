@@ -102,37 +102,44 @@ lsq_status lsq_nf4_dequantize(const lsq_nf4_weight* w, void* w_bf16, lsq_cuda_st
  * The frozen-base linear with a LoRA adapter that layer streaming trains
  * (themenonlab blog, "The trick: layer streaming": the adapter is the only
  * trained part; soup-cli diff docs "Layer Streaming", lora.r / lora.alpha).
- * s = alpha / r.  The dequantised tile never reaches HBM: the kernel decodes
- * NF4 into shared memory and multiplies on the tensor cores (tcgen05, fp32
- * accumulation in TMEM); the rank-r path runs as two small MMAs, one in the
- * main loop (U) and one before the epilogue (s U B^T); Y is rounded to bf16
- * once.
+ * s = alpha / r.  The dequantised tile never reaches HBM: pairs of SMs decode
+ * NF4 into shared memory and multiply on the tensor cores (tcgen05 with
+ * cta_group::2, fp32 accumulation in TMEM).  U is computed first by a split-K
+ * tensor-core kernel (kept in fp32 in u_out, and as s*U in bf16 in the
+ * workspace); (s U) B^T then runs as one more contraction block of the main
+ * GEMM, so Y is rounded to bf16 once.
  *  x        device bf16 [M, k_in], 16-byte aligned
  *  A        device bf16 [r, k_in]   (LoRA down), NULL with r = 0 disables LoRA
  *  B        device bf16 [n_out, r]  (LoRA up)
  *  residual device bf16 [M, n_out] or NULL; may alias y
  *  y        device bf16 [M, n_out]
  *  u_out    device fp32 [M, r] or NULL (kept for the backward)
+ *  workspace  device scratch of lsq_nf4_lora_fwd_workspace_size() bytes,
+ *             256-byte aligned (may be NULL when r = 0); contents undefined
+ *             after the call.  LSQ_EINVAL if missing or too small.
  * Limits: 1 <= M, 0 <= r <= 64.  Deterministic (no atomics, fixed order). */
+size_t lsq_nf4_lora_fwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r);
 lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A, const void* B,
-                            int32_t r, float s, const void* residual, void* y, float* u_out,
-                            lsq_cuda_stream stream);
+                            int32_t r, float s, const void* residual, void* y, float* u_out, void* workspace,
+                            size_t workspace_bytes, lsq_cuda_stream stream);
 
 /* Up to three linears that read the same x in one launch (q/k/v, gate/up);
  * segment i uses W[i], A[i], B[i], residual[i], y[i], u_out[i] exactly as
- * lsq_nf4_lora_fwd.  All W[i].k_in equal; r and s shared. */
+ * lsq_nf4_lora_fwd.  All W[i].k_in equal; r and s shared; the workspace size
+ * is lsq_nf4_lora_fwd_workspace_size(nseg, ...) over the n_out of every segment. */
 lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
                                   const void* const* A, const void* const* B, int32_t r, float s,
                                   const void* const* residual, void* const* y, float* const* u_out,
-                                  lsq_cuda_stream stream);
+                                  void* workspace, size_t workspace_bytes, lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
  * Backward of the fused linear (frozen W: no weight gradient).
  *
  * G = dY B;  dX = dY deq(W) + s G A;  dB (+)= s dY^T U;  dA (+)= s G^T X.
  * The gradients whose presence at the first layer the pages test (soup-cli
- * diff, CHANGELOG [0.72.2], "Correctness").  dX runs on the tensor cores
- * against the dequantised tile in MN-major layout; dA and dB are
+ * diff, CHANGELOG [0.72.2], "Correctness").  G comes from a split-K
+ * tensor-core kernel; dX runs on SM pairs against the dequantised tile in
+ * MN-major layout with (s G) A as one extra contraction block; dA and dB are
  * deterministic two-stage reductions over M (no atomics).
  *  x    device bf16 [M, k_in]   forward input
  *  dy   device bf16 [M, n_out]  upstream gradient
@@ -164,8 +171,8 @@ lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
  * an extra allocation mid-step could fail, or while a stream is being
  * captured.
  * Same arguments and results as lsq_nf4_lora_bwd without the workspace: the
- * scratch (G and the dA/dB partial sums) is one fixed array of
- * lsq_nf4_lora_bwd_noalloc_max_scratch() bytes (8 MiB) in the device memory of
+ * scratch (G, the padded LoRA operands and the partial sums) is one fixed array
+ * of lsq_nf4_lora_bwd_noalloc_max_scratch() bytes (32 MiB) in the device memory of
  * every GPU that loads the library, held until the process exits.  A size
  * whose scratch exceeds it is rejected with LSQ_EINVAL before anything is
  * enqueued.  The first call on a device looks up the array's device address

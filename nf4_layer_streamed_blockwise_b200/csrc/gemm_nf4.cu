@@ -1,34 +1,40 @@
-// Fused NF4-dequant GEMMs with the LoRA path, sm_100a (tcgen05 + TMEM + TMA).
+// Fused NF4-dequant GEMMs with the LoRA path, sm_100a: tcgen05 on SM pairs.
 //
-//   FWD: Y = residual + X deq(W)^T + s (X A^T) B^T,  U = X A^T
-//   DX : dX = sum_seg dY_seg deq(W_seg) + s sum_seg G_seg A_seg,  G_seg = dY_seg B_seg
+//   FWD: Y = residual + X deq(W)^T + s U B^T,          U = X A^T
+//   DX : dX = sum_seg dY_seg deq(W_seg) + s G A,       G = [G_seg] = [dY_seg B_seg]
 //
-// One CTA computes a 256 x BN output tile (BN = 128 or 192) as two 128-row
-// halves that share one dequantised weight tile per stage: the NF4 decode work
-// per tensor-core FLOP is half that of a 128-row tile.  Contraction blocks of
-// 64; NST shared-memory stages.
+// Main kernel (nf4_pair_kernel).  A cluster of two CTAs on two SMs computes a
+// 256 x 256 output tile with tcgen05.mma.cta_group::2 (M = 256, N = 256): each
+// CTA stages its own 128 activation rows and decodes its own 128 columns of
+// the weight tile into shared memory, and the pair's tensor cores read both
+// halves.  Per SM that is half the weight-operand reads and half the decode
+// work per FLOP of a one-SM 128 x 256 tile, and half the activation reads of
+// a 256 x 128 one.  The kernel is persistent: cluster c takes tiles c, c + C,
+// c + 2C, ... (C clusters, m index fastest so that the clusters in flight
+// share weight columns in L2); the two TMEM accumulators (2 x 256 fp32
+// columns) alternate, so the epilogue of one tile overlaps the main loop of
+// the next.  Six shared-memory stages of 64 contraction steps.
 //
-// Warp roles:
-//   0-3        epilogue warpgroup (TMEM lanes 0-127; both halves)
-//   4          TMA producer: activation tile (256 rows, 128-byte swizzle),
-//              packed NF4 codes, and (FWD) the LoRA-down tile
-//   5          MMA issuer + TMEM owner
-//   6 ..       BN/16 dequantiser warps: two threads per 64-element NF4 block per
-//              stage, each writing half of one 128-byte row of the swizzled
-//              bf16 operand
-// The rank-r down product rides in the same MMA as the base GEMM: the LoRA
-// operand tile sits right after the weight tile in shared memory, so one MMA
-// per half (N = BN + LW) reads the activation slice once and writes
-// [acc | U] (FWD, LW = rp: A's rows appended to W's) or [dX | G] (DX, LW = 64:
-// each segment's B in its own rank-padded column range, so the segments' G
-// stay apart).  TMEM columns of half h: [h*NW, h*NW + BN) accumulator,
-// [h*NW + BN, h*NW + NW) the rank-r product; NW = BN + LW, 2*NW <= 512.
+// The rank-r products stay off the main loop: a split-K tcgen05 kernel
+// (lora_down_kernel) computes U = X A^T (or G = dY B) and a reduction writes it
+// in fp32 (kept for the backward) and as s*U (s*G) in bf16, zero-padded to 64
+// columns.  The main loop then runs (s U) B^T (or (s G) A) as one extra
+// contraction block of width 64 whose two operands are TMA-loaded like the
+// activation tile, so the output is still rounded to bf16 once.
 //
-// The LoRA-up product runs on the tensor cores: after the main loop the
-// epilogue writes s*U (or s*G) as bf16 into shared memory and the MMA warp adds
-// (sU) B^T (or (sG) A) into the same accumulators (K = KE), so the output is
-// rounded to bf16 once.  Every wait is bounded (common.cuh); there are no
-// atomics, so results do not depend on timing or buffer addresses.
+// Warp roles in each CTA of the pair:
+//   0-3   epilogue: TMEM lanes 0-127 -> the CTA's 128 output rows
+//   4     TMA producer: activation tile, packed codes, the LoRA block's tiles
+//   5     TMEM owner; in the leader CTA (rank 0) also the MMA issuer
+//   6-13  NF4 decoders: two threads per 64-value block of the stage, each
+//         writing half of one 128-byte row of the swizzled bf16 operand
+// The leader's "full" barrier of a stage completes when both CTAs' TMA bytes
+// have landed and all 16 decoder warps of the pair have arrived; the MMA
+// commit releases the stage in both CTAs at once (commit multicast).  Every
+// wait is bounded (common.cuh); there are no atomics, so results do not
+// depend on timing or on which SM ran which tile.
+#include <algorithm>
+
 #include "common.cuh"
 #include "host_common.h"
 
@@ -37,73 +43,76 @@ namespace nf4g {
 
 enum Mode { FWD = 0, DX = 1 };
 
-constexpr int BM = 256, HM = 128, BK = 64, NST = 3;
-constexpr int KE_MAX = 64;
-constexpr int A_BYTES = BM * BK * 2;  // 32 KB
-
-template <int BN>
-struct Cfg {
-  static constexpr int DQ_WARPS = BN / 16;  // two threads per 64-element NF4 block
-  static constexpr int NTHREADS = (6 + DQ_WARPS) * 32;
-  static constexpr int W_BYTES = BN * BK * 2;             // dequantised weight tile
-  static constexpr int B_BYTES = W_BYTES + KE_MAX * BK * 2;  // + LoRA operand tile (<= 64 x 64)
-  static constexpr int C_BYTES = BN * BK / 2;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + NST * A_BYTES;
-  static constexpr int OFF_C = OFF_B + NST * B_BYTES;
-  static constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
-  // epilogue LoRA operands, aliased onto the stages (used after the main loop)
-  static constexpr int OFF_UE = 0;                          // 2 x [128 x KE] bf16
-  static constexpr int OFF_BE = 2 * HM * KE_MAX * 2;        // [BN x KE] bf16
-  static_assert(OFF_BE + BN * KE_MAX * 2 <= OFF_C, "epilogue operands must fit the stage buffers");
-  static constexpr int NBAR = 3 * NST + 4;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-  static constexpr int BYTES = OFF_MISC + 128 + 1024;
-  static_assert(BYTES <= 232448, "shared memory");
-};
-
-struct Seg {
-  const float* absmax;
-  const __nv_bfloat16* la;   // LoRA A [r, K_in]
-  const __nv_bfloat16* lb;   // LoRA B [n, r]
-  const __nv_bfloat16* lat;  // DX: A^T [K_in, rp], columns >= r zero
-  __nv_bfloat16* y;          // FWD output [M, n]
-  const __nv_bfloat16* res;  // FWD residual [M, n] or null
-  float* uo;                 // U (FWD) or G (DX) [M, r] or null
-  int n;                     // rows of W
-  int first;                 // FWD: first n-tile of the segment; DX: first contraction block
-};
-
-struct Params {
-  Seg seg[3];
-  int nseg;
-  int M, K;     // K = k_in
-  int r, rp;
-  float s;
-  float cb[16];
-  __nv_bfloat16* dx;  // DX output [M, K] or null
-  int nkb;
-};
-
-struct Maps {
-  CUtensorMap a[3];  // FWD: x; DX: dy of each segment (box 64 x 256 rows, 128B swizzle)
-  CUtensorMap c[3];  // packed codes of each segment
-  CUtensorMap l[3];  // LoRA operand of the main loop: FWD A [r, K] (box 64 x rp rows);
-                     // DX rank-padded B [n, 64] (box 64 x 64 rows)
-};
-
-__device__ __forceinline__ int seg_of_block(const Params& p, int i) {
-  int sg = 0;
-  while (sg + 1 < p.nseg && i >= p.seg[sg + 1].first) ++sg;
-  return sg;
+// ---------------------------------------------------------------- cluster / CTA-pair PTX
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of this CTA's variable p as seen in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier of either CTA of the pair (default .release.cta
+// semantics).  The writes this arrival publishes are shared-memory tiles that
+// the tensor cores read through the async proxy: the writer's
+// fence.proxy.async orders them, so a cluster-scope release, which costs a
+// full memory fence on every arrival, buys nothing here.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// all threads of both CTAs
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 2-D tile load into this CTA's shared memory that completes on an mbarrier of
+// either CTA of the pair (here always the leader's)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_caddr, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(m), "r"(bar_caddr), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A B^T over the pair: A rows 0-127 from the leader's shared memory,
+// 128-255 from the peer's; B rows (output columns) split the same way.
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in every CTA of `mask` once all MMAs issued so far complete
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                   "r"(smem_u32(bar)),
+               "h"(mask)
+               : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
-}
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
 // eight codes (one 32-bit word; first element = high nibble of byte 0) -> eight bf16
@@ -126,48 +135,441 @@ __device__ __forceinline__ void store_half_row(uint32_t row_addr, int row, int h
     st_shared_v4(row_addr + ((uint32_t)((half * 4 + q) ^ (row & 7)) << 4), dq8(w[q], a, cb));
 }
 
-template <int MODE, int BN>
-__global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __grid_constant__ Maps maps,
-                                                                         const __grid_constant__ Params p) {
-  using C = Cfg<BN>;
+// ================================================================ main kernel
+constexpr int BMC = 128;  // activation rows per CTA (256 per pair)
+constexpr int BNC = 128;  // weight columns decoded per CTA
+constexpr int BT = 256;   // tile edge of the pair: 256 rows x 256 output columns
+constexpr int BK = 64;
+constexpr int NST = 6;
+constexpr int A_BYTES = BMC * BK * 2;  // 16 KB
+constexpr int W_BYTES = BNC * BK * 2;  // 16 KB
+constexpr int C_BYTES = BNC * BK / 2;  // 4 KB
+constexpr int DQ_WARPS = 8;
+constexpr int NTHREADS = (6 + DQ_WARPS) * 32;
+constexpr int OFF_A = 0;
+constexpr int OFF_W = OFF_A + NST * A_BYTES;
+constexpr int OFF_C = OFF_W + NST * W_BYTES;
+constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
+constexpr int NBAR = 3 * NST + 5;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+constexpr int SMEM_BYTES = OFF_MISC + 128 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+struct Seg {
+  const float* absmax;
+  __nv_bfloat16* y;          // FWD output [M, n]
+  const __nv_bfloat16* res;  // FWD residual [M, n] or null (may alias y)
+  int n;                     // rows of W
+  int first;                 // FWD: first n-tile of the segment; DX: first contraction block
+};
+
+struct Params {
+  Seg seg[3];
+  int nseg, M, K;
+  int lora;          // 1: one LoRA contraction block follows the weight blocks
+  int nkb;           // weight contraction blocks per tile
+  int mtiles, tiles;
+  __nv_bfloat16* dx;  // DX output [M, K]
+  float cb[16];
+};
+
+struct Maps {
+  CUtensorMap a[3];   // FWD: x [M, K]; DX: dy of each segment [M, n]  (box 64 x 128 rows, 128B swizzle)
+  CUtensorMap c[3];   // packed codes of each segment: FWD box 32 B x 128 rows; DX box 64 B x 64 rows
+  CUtensorMap la[3];  // LoRA block, activation side: FWD s*U of each segment [M, 64]; DX s*G [M, 64]
+  CUtensorMap lb[3];  // LoRA block, weight side: FWD B of each segment, padded [n, 64]; DX A^T of all
+                      // segments side by side [K, 64]
+};
+
+__device__ __forceinline__ int seg_of_block(const Params& p, int i) {
+  int sg = 0;
+  while (sg + 1 < p.nseg && i >= p.seg[sg + 1].first) ++sg;
+  return sg;
+}
+
+template <int MODE>
+__device__ __forceinline__ void tile_at(const Params& p, int t, int& m0, int& sg, int& n0) {
+  const int mt = t % p.mtiles, nt = t / p.mtiles;
+  m0 = mt * BT;
+  sg = 0;
+  if (MODE == FWD) {
+    while (sg + 1 < p.nseg && nt >= p.seg[sg + 1].first) ++sg;
+    n0 = (nt - p.seg[sg].first) * BT;
+  } else {
+    n0 = nt * BT;
+  }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    nf4_pair_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* empty = full + NST;
   uint64_t* cfull = empty + NST;
-  uint64_t* ufull = cfull + NST;
-  uint64_t* lready = ufull + 1;
-  uint64_t* afull = ufull + 2;
-  uint64_t* drain = ufull + 3;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  float* s_cb = reinterpret_cast<float*>(smem + C::OFF_MISC + 16);
+  uint64_t* tfull = cfull + NST;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  float* s_cb = reinterpret_cast<float*>(smem + OFF_MISC + 16);
 
+  const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  int seg = 0, tile = blockIdx.x;
-  if (MODE == FWD) {
-    while (seg + 1 < p.nseg && (int)blockIdx.x >= p.seg[seg + 1].first) ++seg;
-    tile = blockIdx.x - p.seg[seg].first;
-  }
-  const int n0 = tile * BN;  // FWD: output column in the segment; DX: k_in column
-  const bool lora = p.rp > 0;
-  const int KE = (MODE == DX) ? p.nseg * p.rp : p.rp;
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+  const int nkb_all = p.nkb + p.lora;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1 + C::DQ_WARPS);
+      mbar_init(&full[s], 1 + 2 * DQ_WARPS);  // leader's producer + every decoder warp of the pair
       mbar_init(&empty[s], 1);
       mbar_init(&cfull[s], 1);
     }
-    mbar_init(ufull, 1);
-    mbar_init(lready, 1);
-    mbar_init(afull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2);  // one epilogue arrival per CTA
+    }
     mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (threadIdx.x < 16) s_cb[threadIdx.x] = p.cb[threadIdx.x];
   if (warp == 5) {
-    tmem_alloc(s_tmem, 512);
+    tmem_alloc_pair(s_tmem, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int t = cid; t < p.tiles && ok; t += ncl) {
+        int m0, sg, n0;
+        tile_at<MODE>(p, t, m0, sg, n0);
+        const int mrow = m0 + (int)rank * BMC, wcol = n0 + (int)rank * BNC;
+        for (int i = 0; i < nkb_all; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, 421)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fl = cluster_addr(&full[s], 0);
+          uint8_t* a_dst = smem + OFF_A + s * A_BYTES;
+          if (i < p.nkb) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * A_BYTES);
+            mbar_arrive_expect_tx(&cfull[s], (uint32_t)C_BYTES);
+            uint8_t* c_dst = smem + OFF_C + s * C_BYTES;
+            if (MODE == DX) {
+              const int bs = seg_of_block(p, i);
+              const int nb = i - p.seg[bs].first;
+              tma_load_2d_pair(a_dst, &maps.a[bs], fl, nb * BK, mrow);
+              tma_load_2d(c_dst, &maps.c[bs], &cfull[s], wcol / 2, nb * BK);
+            } else {
+              tma_load_2d_pair(a_dst, &maps.a[0], fl, i * BK, mrow);
+              tma_load_2d(c_dst, &maps.c[sg], &cfull[s], i * (BK / 2), wcol);
+            }
+          } else {
+            // no codes for the LoRA block, but cfull[s] still completes one phase per
+            // block, so that every barrier's parity follows the block counter
+            mbar_arrive(&cfull[s]);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (A_BYTES + W_BYTES));
+            tma_load_2d_pair(a_dst, &maps.la[sg], fl, 0, mrow);
+            tma_load_2d_pair(smem + OFF_W + s * W_BYTES, &maps.lb[sg], fl, 0, wcol);
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer (leader CTA)
+    if (rank == 0 && lane == 0) {
+      const uint32_t id_k = idesc_bf16(2 * BMC, BT, 0, 0);   // both operands K-major
+      const uint32_t id_mn = idesc_bf16(2 * BMC, BT, 0, 1);  // DX weight tile: MN-major
+      uint32_t g = 0;
+      int j = 0;
+      bool ok = true;
+      for (int t = cid; t < p.tiles && ok; t += ncl, ++j) {
+        const int buf = j & 1;
+        const uint32_t tph = (uint32_t)(j >> 1) & 1u;
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, 521)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BT);
+        for (int i = 0; i < nkb_all; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          if (!mbar_wait(&full[s], ph, 522)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + OFF_A + s * A_BYTES);
+          const uint32_t w_base = smem_u32(smem + OFF_W + s * W_BYTES);
+          const bool mn = (MODE == DX) && i < p.nkb;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, 2);
+            const uint64_t bd =
+                mn ? smem_desc(w_base + kk * 2048, 8192, 1024, 2) : smem_desc(w_base + kk * 32, 16, 1024, 2);
+            tc_mma_pair(d, ad, bd, mn ? id_mn : id_k, (i | kk) != 0);
+          }
+          tc_commit_pair_mc(&empty[s], 0x3);
+        }
+        if (ok) tc_commit_pair_mc(&tfull[buf], 0x3);
+      }
+      if (!ok) {
+        tc_commit_pair(drain);
+        mbar_wait(drain, 0, 523);
+      }
+    }
+  } else if (warp >= 6) {
+    // ---------------------------------------------------------------- NF4 decoders
+    const int t = threadIdx.x - 6 * 32;  // 0 .. 255
+    const int KB = p.K / 64;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int tt = cid; tt < p.tiles && ok; tt += ncl) {
+      int m0, sg, n0;
+      tile_at<MODE>(p, tt, m0, sg, n0);
+      const int wcol = n0 + (int)rank * BNC;
+      if (MODE == FWD) {
+        // thread -> (row, half): consecutive lanes read consecutive 16-byte code
+        // chunks and write conflict-free swizzled chunks
+        const int row = t >> 1, half = t & 1;
+        const Seg& S = p.seg[sg];
+        const int n = wcol + row;
+        const bool valid = n < S.n;
+        const float* arow = S.absmax + (int64_t)(valid ? n : 0) * KB;
+        // 16-byte absmax loads need every row start 16-byte aligned (the ABI promises 4)
+        const bool vec = (KB % 4) == 0 && (reinterpret_cast<uintptr_t>(S.absmax) & 15) == 0;
+        float4 acur = make_float4(0.f, 0.f, 0.f, 0.f), anext = acur;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+        if (valid) {
+          if (vec) {
+            acur = __ldg(reinterpret_cast<const float4*>(arow));
+            if (KB > 4) anext = __ldg(reinterpret_cast<const float4*>(arow + 4));
+          } else {
+            s0 = __ldg(arow);
+            if (KB > 1) s1 = __ldg(arow + 1);
+            if (KB > 2) s2 = __ldg(arow + 2);
+          }
+        }
+        for (int i = 0; i < nkb_all; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          const uint32_t fl = cluster_addr(&full[s], 0);
+          if (i < p.nkb) {
+            const int q = i & 3;
+            const float a = vec ? (q == 0 ? acur.x : q == 1 ? acur.y : q == 2 ? acur.z : acur.w) : s0;
+            if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], ph, 631))) {
+              ok = false;
+              break;
+            }
+            const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + t * 16);
+            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + row * 128, row, half, c, valid ? a : 0.0f, s_cb);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(fl);
+            if (valid) {
+              if (vec) {
+                if (q == 3) {
+                  acur = anext;
+                  if (i + 5 < KB) anext = __ldg(reinterpret_cast<const float4*>(arow + i + 5));
+                }
+              } else {
+                s0 = s1;
+                s1 = s2;
+                if (i + 3 < KB) s2 = __ldg(arow + i + 3);
+              }
+            }
+          } else {
+            // LoRA block: its weight-side tile comes by TMA; arrive once the producer
+            // has claimed the stage (cfull[s] completes without bytes for this block)
+            if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], ph, 632))) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) mbar_arrive_cluster(fl);
+          }
+        }
+      } else {
+        // DX stage tile: 64 contraction rows (n) x 128 output columns (k) = 64 x 2
+        // blocks; thread -> (k chunk, row, half) so that the 8 lanes of each
+        // store phase write 8 different swizzled chunks of 4 rows of one chunk
+        const int kc = t >> 7, nl = (t & 127) >> 1, half = t & 1;
+        const int kcol = wcol + kc * 64;
+        auto absmax_of = [&](int i) {
+          const int bs = seg_of_block(p, i);
+          const Seg& S = p.seg[bs];
+          const int nrow = (i - S.first) * BK + nl;
+          return (nrow < S.n && kcol < p.K) ? __ldg(S.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
+        };
+        // absmax of the next four blocks in flight (global-load latency > one block)
+        float a0 = absmax_of(0);
+        float a1 = p.nkb > 1 ? absmax_of(1) : 0.0f;
+        float a2 = p.nkb > 2 ? absmax_of(2) : 0.0f;
+        float a3 = p.nkb > 3 ? absmax_of(3) : 0.0f;
+        for (int i = 0; i < nkb_all; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          const uint32_t fl = cluster_addr(&full[s], 0);
+          if (i < p.nkb) {
+            const float a = a0;
+            a0 = a1;
+            a1 = a2;
+            a2 = a3;
+            a3 = i + 4 < p.nkb ? absmax_of(i + 4) : 0.0f;
+            if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], ph, 633))) {
+              ok = false;
+              break;
+            }
+            const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + nl * (BNC / 2) + kc * 32 +
+                                                            half * 16);
+            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + kc * 8192 + nl * 128, nl, half, c, a, s_cb);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(fl);
+          } else {
+            if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], ph, 634))) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) mbar_arrive_cluster(fl);
+          }
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 0-3)
+    const int e = threadIdx.x;  // TMEM lane = row within the CTA's 128
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int j = 0;
+    for (int t = cid; t < p.tiles; t += ncl, ++j) {
+      int m0, sg, n0;
+      tile_at<MODE>(p, t, m0, sg, n0);
+      const int buf = j & 1;
+      const uint32_t tph = (uint32_t)(j >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
+      tc_fence_after();
+      const int m = m0 + (int)rank * BMC + e;
+      const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
+      for (int c = 0; c < BT / 32; ++c) {
+        if (n0 + c * 32 >= ncols) break;
+        float v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(buf * BT + c * 32), v);
+        tc_wait_ld();
+        if (m >= p.M) continue;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+          const int col = n0 + c * 32 + gq * 8;
+          if (col >= ncols) continue;
+          float* x = v + gq * 8;
+          if (MODE == FWD) {
+            const Seg& S = p.seg[sg];
+            const int64_t off = (int64_t)m * S.n + col;
+            if (S.res) {
+              const uint4 rv = *reinterpret_cast<const uint4*>(S.res + off);
+              x[0] += bf16lo(rv.x);
+              x[1] += bf16hi(rv.x);
+              x[2] += bf16lo(rv.y);
+              x[3] += bf16hi(rv.y);
+              x[4] += bf16lo(rv.z);
+              x[5] += bf16hi(rv.z);
+              x[6] += bf16lo(rv.w);
+              x[7] += bf16hi(rv.w);
+            }
+            *reinterpret_cast<uint4*>(S.y + off) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                                              pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+          } else {
+            *reinterpret_cast<uint4*>(p.dx + (int64_t)m * p.K + col) =
+                make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                           pack_bf16x2(x[6], x[7]));
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(1, 128);
+      if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ================================================================ rank-r products: U = X A^T, G = dY B
+// Split-K tcgen05 GEMM with a narrow N: CTA (m tile, split, problem) multiplies
+// 128 activation rows by the problem's np = nsub * rp weight-side rows over
+// its share of the contraction, and writes fp32 partial sums; a second kernel
+// adds the splits in a fixed order.
+namespace ldn {
+constexpr int BM = 128, BK = 64, NST = 4, NMAX = 192;
+constexpr int A_BYTES = BM * BK * 2;    // 16 KB
+constexpr int B_BYTES = NMAX * BK * 2;  // 24 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + NST * A_BYTES;
+constexpr int OFF_BAR = OFF_B + NST * B_BYTES;
+constexpr int NBAR = 2 * NST + 1;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int NTHREADS = 192;
+constexpr int TARGET_CTAS = 296;
+
+struct Prob {
+  float* part;    // [splits][M][np]
+  int nkb;        // contraction blocks of 64 (the last may be partial: zero-filled)
+  int splits;     // split k covers blocks [k*kbps, min(nkb, (k+1)*kbps))
+  int nsub;       // weight-side maps wl[first .. first + nsub), rp rows each
+  int first;
+};
+struct Params {
+  Prob pr[3];
+  int nprob, M, rp, kbps;
+};
+struct Maps {
+  CUtensorMap in[3];  // activation side of each problem [M, Kr] (box 64 x 128 rows, 128B swizzle)
+  CUtensorMap wl[3];  // weight side [rows, Kr] (box 64 x rp rows; rows past the tensor read as zero)
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_constant__ Maps maps,
+                                                                const __grid_constant__ Params p) {
+  const Prob& P = p.pr[blockIdx.z];
+  const int split = blockIdx.y;
+  if (split >= P.splits) return;
+  const int kb0 = split * p.kbps;
+  const int nk = min(P.nkb, kb0 + p.kbps) - kb0;
+  const int np = P.nsub * p.rp;
+  const int m0 = blockIdx.x * BM;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + NST;
+  uint64_t* done = empty + NST;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = np <= 32 ? 32u : np <= 64 ? 64u : np <= 128 ? 128u : 256u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -175,317 +577,229 @@ __global__ void __launch_bounds__(Cfg<BN>::NTHREADS, 1) nf4_gemm_kernel(const __
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- TMA producer
+  if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < p.nkb; ++i) {
+      for (int i = 0; i < nk; ++i) {
         const int s = i % NST;
         const uint32_t ph = (uint32_t)(i / NST) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, 411)) break;
-        uint8_t* a_dst = smem + C::OFF_A + s * A_BYTES;
-        uint8_t* c_dst = smem + C::OFF_C + s * C::C_BYTES;
-        const uint32_t lbytes = lora ? (MODE == DX ? 64u * 128u : (uint32_t)p.rp * 128u) : 0u;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)A_BYTES + lbytes);
-        uint8_t* l_dst = smem + C::OFF_B + s * C::B_BYTES + C::W_BYTES;
-        mbar_arrive_expect_tx(&cfull[s], (uint32_t)C::C_BYTES);
-        if (MODE == DX) {
-          const int sg = seg_of_block(p, i);
-          const int nb = i - p.seg[sg].first;
-          tma_load_2d(a_dst, &maps.a[sg], &full[s], nb * BK, m0);
-          tma_load_2d(c_dst, &maps.c[sg], &cfull[s], n0 / 2, nb * BK);
-          if (lora) tma_load_2d(l_dst, &maps.l[sg], &full[s], 0, nb * BK);
-        } else {
-          tma_load_2d(a_dst, &maps.a[0], &full[s], i * BK, m0);
-          tma_load_2d(c_dst, &maps.c[seg], &cfull[s], i * (BK / 2), n0);
-          if (lora) tma_load_2d(l_dst, &maps.l[seg], &full[s], i * BK, 0);
-        }
+        if (!mbar_wait(&empty[s], ph ^ 1u, 441)) break;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + np * 128));
+        const int x = (kb0 + i) * BK;
+        tma_load_2d(smem + OFF_A + s * A_BYTES, &maps.in[blockIdx.z], &full[s], x, m0);
+        for (int q = 0; q < P.nsub; ++q)
+          tma_load_2d(smem + OFF_B + s * B_BYTES + q * p.rp * 128, &maps.wl[P.first + q], &full[s], x, 0);
       }
     }
-  } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1) {
     if (lane == 0) {
-      const int LW = lora ? (MODE == DX ? 64 : p.rp) : 0;  // LoRA columns appended to the weight tile
-      const int NW = BN + LW;
-      const uint32_t id_main = idesc_bf16(HM, NW, 0, MODE == DX ? 1 : 0);
-      const uint32_t id_ep = idesc_bf16(HM, BN, 0, 0);
+      const uint32_t id = idesc_bf16(BM, np, 0, 0);
       bool ok = true;
-      for (int i = 0; i < p.nkb; ++i) {
+      for (int i = 0; i < nk; ++i) {
         const int s = i % NST;
         const uint32_t ph = (uint32_t)(i / NST) & 1u;
-        if (!mbar_wait(&full[s], ph, 511)) {
+        if (!mbar_wait(&full[s], ph, 541)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + C::OFF_A + s * A_BYTES);
-        const uint32_t b_base = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
+        const uint32_t a_base = smem_u32(smem + OFF_A + s * A_BYTES);
+        const uint32_t b_base = smem_u32(smem + OFF_B + s * B_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bd = (MODE == DX) ? smem_desc(b_base + kk * 2048, 8192, 1024, 2)
-                                           : smem_desc(b_base + kk * 32, 16, 1024, 2);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint64_t ad = smem_desc(a_base + h * (HM * 128) + kk * 32, 16, 1024, 2);
-            tc_mma(tmem + h * NW, ad, bd, id_main, (i | kk) != 0);
-          }
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma(tmem, smem_desc(a_base + kk * 32, 16, 1024, 2), smem_desc(b_base + kk * 32, 16, 1024, 2), id,
+                 (i | kk) != 0);
         tc_commit(&empty[s]);
       }
-      if (ok) {
-        tc_commit(ufull);
-        if (lora) {
-          if (mbar_wait(lready, 0, 512)) {
-            tc_fence_after();
-            const uint32_t be = smem_u32(smem + C::OFF_BE);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t ue = smem_u32(smem + C::OFF_UE + h * HM * KE_MAX * 2);
-              for (int kk = 0; kk < KE / 16; ++kk)
-                tc_mma(tmem + h * NW, smem_desc(ue + kk * 256, 128, KE * 16, 0),
-                       smem_desc(be + kk * 256, 128, KE * 16, 0), id_ep, 1);
-            }
-            tc_commit(afull);
-          } else {
-            ok = false;
-          }
-        }
-      }
-      if (!ok) {
-        tc_commit(drain);
-        mbar_wait(drain, 0, 513);
-      }
-    }
-  } else if (warp >= 6) {
-    // ---------------------------------------------------------------- NF4 dequantisers
-    const int t = threadIdx.x - 6 * 32;  // 0 .. 2*BN-1
-    const int KB = p.K / 64;
-    if (MODE == FWD) {
-      // thread -> (row, half): consecutive lanes read consecutive 16-byte code
-      // chunks and write conflict-free swizzled chunks
-      const int row = t >> 1, half = t & 1;
-      const Seg& sg = p.seg[seg];
-      const int n = n0 + row;
-      const bool valid = n < sg.n;
-      const float* arow = sg.absmax + (int64_t)(valid ? n : 0) * KB;
-      const bool vec = (KB % 4) == 0;
-      float4 acur = make_float4(0.f, 0.f, 0.f, 0.f), anext = acur;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f;
-      if (valid) {
-        if (vec) {
-          acur = __ldg(reinterpret_cast<const float4*>(arow));
-          if (KB > 4) anext = __ldg(reinterpret_cast<const float4*>(arow + 4));
-        } else {
-          s0 = __ldg(arow);
-          if (KB > 1) s1 = __ldg(arow + 1);
-          if (KB > 2) s2 = __ldg(arow + 2);
-        }
-      }
-      for (int i = 0; i < p.nkb; ++i) {
-        const int s = i % NST;
-        const uint32_t ph = (uint32_t)(i / NST) & 1u;
-        const int q = i & 3;
-        const float a = vec ? (q == 0 ? acur.x : q == 1 ? acur.y : q == 2 ? acur.z : acur.w) : s0;
-        if (!mbar_wait(&cfull[s], ph, 611)) break;
-        const uint4 c = *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C::C_BYTES + t * 16);
-        store_half_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + row * 128, row, half, c, valid ? a : 0.0f, s_cb);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-        if (valid) {
-          if (vec) {
-            if (q == 3) {
-              acur = anext;
-              if (i + 5 < KB) anext = __ldg(reinterpret_cast<const float4*>(arow + i + 5));
-            }
-          } else {
-            s0 = s1;
-            s1 = s2;
-            if (i + 3 < KB) s2 = __ldg(arow + i + 3);
-          }
-        }
-      }
-    } else {
-      // DX stage tile: 64 contraction rows (n) x BN output columns (k) = 64 x BN/64
-      // blocks; thread -> (k chunk, row, half) so that the 8 lanes of each
-      // store phase write 8 different swizzled chunks of 4 rows of one chunk
-      const int kc = t >> 7, nl = (t & 127) >> 1, half = t & 1;
-      const int kcol = n0 + kc * 64;
-      auto absmax_of = [&](int i) {
-        const int sgi = seg_of_block(p, i);
-        const Seg& sg = p.seg[sgi];
-        const int nrow = (i - sg.first) * BK + nl;
-        return (nrow < sg.n && kcol < p.K) ? __ldg(sg.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
-      };
-      float a_nx = p.nkb > 0 ? absmax_of(0) : 0.0f;
-      for (int i = 0; i < p.nkb; ++i) {
-        const int s = i % NST;
-        const uint32_t ph = (uint32_t)(i / NST) & 1u;
-        const float a = a_nx;
-        if (i + 1 < p.nkb) a_nx = absmax_of(i + 1);
-        if (!mbar_wait(&cfull[s], ph, 612)) break;
-        const uint4 c =
-            *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C::C_BYTES + nl * (BN / 2) + kc * 32 + half * 16);
-        store_half_row(smem_u32(smem + C::OFF_B + s * C::B_BYTES) + kc * 8192 + nl * 128, nl, half, c, a, s_cb);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-      }
+      tc_commit(done);  // also the drain when the loop stopped early
+      if (!ok) mbar_wait(done, 0, 542);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 0-3)
-    const int e = threadIdx.x;  // TMEM lane = row of each half
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int NW = BN + (lora ? (MODE == DX ? 64 : p.rp) : 0);
-    bool ok = mbar_wait(ufull, 0, 711);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) tc_fence_after();
-    if (ok && lora) {
-      // LoRA-up operand sBe [BN rows x KE], no-swizzle K-major:
-      //   FWD: B[n0 + row, j];  DX: A_seg[j, n0 + row] at column seg*rp + j
-      const uint32_t be = smem_u32(smem + C::OFF_BE);
-      for (int row = e; row < BN; row += 128) {
-        for (int jc = 0; jc < KE / 8; ++jc) {
-          uint4 w = make_uint4(0, 0, 0, 0);
-          if (MODE == FWD) {
-            const int n = n0 + row, j0 = jc * 8;
-            if (n < p.seg[seg].n && j0 < p.r) {
-              const __nv_bfloat16* src = p.seg[seg].lb + (int64_t)n * p.r + j0;
-              if ((p.r & 7) == 0) {
-                w = __ldg(reinterpret_cast<const uint4*>(src));
-              } else {
-                float v[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = (j0 + q < p.r) ? __bfloat162float(src[q]) : 0.0f;
-                w = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                               pack_bf16x2(v[6], v[7]));
-              }
-            }
-          } else {
-            const int sg = (jc * 8) / p.rp, jj = (jc * 8) % p.rp, k = n0 + row;
-            if (k < p.K) w = __ldg(reinterpret_cast<const uint4*>(p.seg[sg].lat + (int64_t)k * p.rp + jj));
-          }
-          st_shared_v4(be + (row >> 3) * (KE * 16) + jc * 128 + (row & 7) * 16, w);
-        }
-      }
-      // s * U (or s * G) as bf16, one operand per half
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int m = m0 + h * HM + e;
-        const uint32_t ue = smem_u32(smem + C::OFF_UE + h * HM * KE_MAX * 2);
-        for (int c = 0; c < KE / 16; ++c) {
-          float v[16];
-          tmem_ld16(tmem + lane_base + h * NW + BN + c * 16, v);
-          tc_wait_ld();
-          if (m < p.M) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const int j = c * 16 + q;
-              if (MODE == FWD) {
-                if (tile == 0 && p.seg[seg].uo && j < p.r) p.seg[seg].uo[(int64_t)m * p.r + j] = v[q];
-              } else {
-                const int sg = j / p.rp, jj = j % p.rp;
-                if (blockIdx.x == 0 && p.seg[sg].uo && jj < p.r) p.seg[sg].uo[(int64_t)m * p.r + jj] = v[q];
-              }
-            }
-          }
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint4 o;
-            o.x = pack_bf16x2(v[hh * 8 + 0] * p.s, v[hh * 8 + 1] * p.s);
-            o.y = pack_bf16x2(v[hh * 8 + 2] * p.s, v[hh * 8 + 3] * p.s);
-            o.z = pack_bf16x2(v[hh * 8 + 4] * p.s, v[hh * 8 + 5] * p.s);
-            o.w = pack_bf16x2(v[hh * 8 + 6] * p.s, v[hh * 8 + 7] * p.s);
-            st_shared_v4(ue + (e >> 3) * (KE * 16) + (c * 2 + hh) * 128 + (e & 7) * 16, o);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (e == 0) mbar_arrive(lready);
-      ok = mbar_wait(afull, 0, 712);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) tc_fence_after();
-    }
-    if (ok) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int m = m0 + h * HM + e;
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + h * NW + c * 32, v);
-          tc_wait_ld();
-          if (m >= p.M) continue;
-#pragma unroll
-          for (int gq = 0; gq < 4; ++gq) {
-            const int col = n0 + c * 32 + gq * 8;
-            float* x = v + gq * 8;
-            if (MODE == FWD) {
-              const Seg& sg = p.seg[seg];
-              if (col >= sg.n) continue;
-              const int64_t off = (int64_t)m * sg.n + col;
-              if (sg.res) {
-                const uint4 rv = *reinterpret_cast<const uint4*>(sg.res + off);
-                x[0] += bf16lo(rv.x); x[1] += bf16hi(rv.x);
-                x[2] += bf16lo(rv.y); x[3] += bf16hi(rv.y);
-                x[4] += bf16lo(rv.z); x[5] += bf16hi(rv.z);
-                x[6] += bf16lo(rv.w); x[7] += bf16hi(rv.w);
-              }
-              *reinterpret_cast<uint4*>(sg.y + off) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                                                 pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-            } else {
-              if (col >= p.K || p.dx == nullptr) continue;
-              *reinterpret_cast<uint4*>(p.dx + (int64_t)m * p.K + col) =
-                  make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                             pack_bf16x2(x[6], x[7]));
-            }
-          }
+    // epilogue warps 2-5: TMEM lane quarter = warp % 4
+    const int qd = warp & 3;
+    const int m = m0 + qd * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    if (__all_sync(0xffffffffu, mbar_wait(done, 0, 741))) {
+      tc_fence_after();
+      for (int c = 0; c < np / 16; ++c) {
+        float v[16];
+        tmem_ld16(tmem + lane_base + (uint32_t)(c * 16), v);
+        tc_wait_ld();
+        if (m < p.M) {
+          float4* dst = reinterpret_cast<float4*>(P.part + ((int64_t)split * p.M + m) * np + c * 16);
+          dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+          dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+          dst[2] = make_float4(v[8], v[9], v[10], v[11]);
+          dst[3] = make_float4(v[12], v[13], v[14], v[15]);
         }
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
-template <int MODE, int BN>
-static lsq_status launch(const Maps& maps, const Params& p, dim3 grid, cudaStream_t stream) {
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    LSQ_CUDA_TRY(cudaFuncSetAttribute(nf4_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      Cfg<BN>::BYTES));
-    configured[dev] = 1;
+// Sum the splits (ascending) and write the outputs.
+//   FWD (one problem, segment q in columns q*rp ..): u_out[q] [M, r] fp32 (if
+//        given) and s*U of segment q as bf16 [M, 64], zero in columns >= r.
+//   DX  (problem q = segment q): G_q [M, r] fp32 and s*G as bf16 [M, 64] with
+//        segment q in columns q*rp .. q*rp + r - 1, zero elsewhere.
+struct Red {
+  const float* part[3];
+  int splits[3];
+  int np[3];
+  float* out32[3];
+  __nv_bfloat16* out16[3];
+  int dx, nseg, M, r, rp;
+  float s;
+};
+
+__global__ void __launch_bounds__(256) lora_down_reduce(const __grid_constant__ Red R) {
+  const int64_t per = (int64_t)R.M * 64;
+  const int64_t total = R.dx ? per : per * R.nseg;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int q0 = (int)(idx / per);
+    const int64_t rem = idx % per;
+    const int64_t m = rem / 64;
+    const int c = (int)(rem % 64);
+    int pb, col, seg, j;
+    bool live;
+    if (R.dx) {
+      seg = c / R.rp;
+      j = c % R.rp;
+      live = seg < R.nseg && j < R.r;
+      pb = seg;
+      col = j;
+    } else {
+      seg = q0;
+      j = c;
+      live = j < R.r;
+      pb = 0;
+      col = seg * R.rp + j;
+    }
+    float sum = 0.0f;
+    if (live) {
+      const float* part = R.part[pb];
+      const int np = R.np[pb];
+      for (int k = 0; k < R.splits[pb]; ++k) sum += part[((int64_t)k * R.M + m) * np + col];
+      if (R.out32[seg]) R.out32[seg][m * R.r + j] = sum;
+    }
+    __nv_bfloat16* o = R.out16[R.dx ? 0 : seg];
+    o[m * 64 + c] = __float2bfloat16_rn(live ? R.s * sum : 0.0f);
   }
-  nf4_gemm_kernel<MODE, BN><<<grid, Cfg<BN>::NTHREADS, Cfg<BN>::BYTES, stream>>>(maps, p);
-  LSQ_LAUNCH_CHECK("nf4_gemm_kernel");
+}
+
+// Padded copies of the LoRA operands.
+//   FWD job q: Bpad_q [n_q, 64] = B_q in columns < r, zero elsewhere
+//   DX  job q < nseg: Bt_q [rp, n_q] = B_q^T, zero rows >= r
+//   DX  job nseg: At [K, 64] = A_q^T of every segment q in columns q*rp .., zero elsewhere
+struct Pad {
+  const __nv_bfloat16* A[3];
+  const __nv_bfloat16* B[3];
+  __nv_bfloat16* Bpad[3];
+  __nv_bfloat16* Bt[3];
+  __nv_bfloat16* At;
+  int64_t n[3];
+  int64_t K;
+  int nseg, r, rp, dx;
+};
+
+__global__ void __launch_bounds__(256) lora_pad(const __grid_constant__ Pad P) {
+  const int job = blockIdx.y;
+  const bool at = P.dx && job == P.nseg;
+  const int64_t total = at ? P.K * 64 : P.dx ? (int64_t)P.rp * P.n[job] : P.n[job] * 64;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    if (at) {
+      const int64_t k = idx / 64;
+      const int c = (int)(idx % 64), q = c / P.rp, j = c % P.rp;
+      P.At[idx] = (q < P.nseg && j < P.r) ? P.A[q][(int64_t)j * P.K + k] : zero;
+    } else if (P.dx) {
+      const int64_t j = idx / P.n[job], n = idx % P.n[job];
+      P.Bt[job][idx] = j < P.r ? P.B[job][n * P.r + j] : zero;
+    } else {
+      const int64_t n = idx / 64;
+      const int c = (int)(idx % 64);
+      P.Bpad[job][idx] = c < P.r ? P.B[job][n * P.r + c] : zero;
+    }
+  }
+}
+
+// contraction blocks per split for problems of nkb[i] blocks over mtiles row tiles
+static int plan_kbps(const int* nkb, int nprob, int mtiles) {
+  int64_t tot = 0;
+  for (int i = 0; i < nprob; ++i) tot += nkb[i];
+  int64_t k = (tot * mtiles + TARGET_CTAS - 1) / TARGET_CTAS;
+  return (int)std::max<int64_t>(1, k);
+}
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace ldn
+
+// ---------------------------------------------------------------- launch helpers
+template <int MODE>
+static lsq_status launch_pair(const Maps& maps, const Params& p, cudaStream_t stream) {
+  static int max_clusters[64] = {0};
+  int dev = 0;
+  LSQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(LSQ_EUNSUPPORTED, "nf4 GEMM: device %d out of range", dev);
+  if (!max_clusters[dev]) {
+    LSQ_CUDA_TRY(
+        cudaFuncSetAttribute(nf4_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * num_sms());
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, nf4_pair_kernel<MODE>, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_clusters[dev] = n;
+  }
+  const int ncl = std::min(p.tiles, max_clusters[dev]);
+  nf4_pair_kernel<MODE><<<2 * ncl, NTHREADS, SMEM_BYTES, stream>>>(maps, p);
+  LSQ_LAUNCH_CHECK("nf4_pair_kernel");
   return LSQ_OK;
 }
 
-// N-tile width: the one whose wave count on the SMs times tile width is smaller
-// (ties to the wider tile, which re-reads the activation tile less often).
-static int pick_bn(const int64_t* ns, int nseg, int64_t M, bool lora_ok192) {
-  const int64_t mt = (M + BM - 1) / BM;
-  const int sms = num_sms();
-  int64_t best = -1;
-  int bn_best = 192;
-  for (int bn : {192, 128}) {
-    if (bn == 192 && !lora_ok192) continue;
-    int64_t tiles = 0;
-    for (int i = 0; i < nseg; ++i) tiles += (ns[i] + bn - 1) / bn;
-    const int64_t waves = (tiles * mt + sms - 1) / sms;
-    const int64_t cost = waves * bn;
-    if (best < 0 || cost < best) {
-      best = cost;
-      bn_best = bn;
-    }
+static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int maxsplits, cudaStream_t stream) {
+  static int configured[64] = {0};
+  int dev = 0;
+  LSQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(ldn::lora_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      ldn::SMEM_BYTES));
+    configured[dev] = 1;
   }
-  return bn_best;
+  const int mtiles = (p.M + ldn::BM - 1) / ldn::BM;
+  ldn::lora_down_kernel<<<dim3(mtiles, maxsplits, p.nprob), ldn::NTHREADS, ldn::SMEM_BYTES, stream>>>(maps, p);
+  LSQ_LAUNCH_CHECK("lora_down_kernel");
+  return LSQ_OK;
+}
+
+static lsq_status launch_reduce(const ldn::Red& R, cudaStream_t stream) {
+  const int64_t total = (int64_t)R.M * 64 * (R.dx ? 1 : R.nseg);
+  int64_t g = (total + 255) / 256;
+  if (g > 1184) g = 1184;
+  ldn::lora_down_reduce<<<(unsigned)g, 256, 0, stream>>>(R);
+  LSQ_LAUNCH_CHECK("lora_down_reduce");
+  return LSQ_OK;
+}
+
+static lsq_status launch_pad(const ldn::Pad& P, int64_t most, cudaStream_t stream) {
+  int64_t g = (most + 255) / 256;
+  if (g > 512) g = 512;
+  if (g < 1) g = 1;
+  ldn::lora_pad<<<dim3((unsigned)g, P.dx ? P.nseg + 1 : P.nseg), 256, 0, stream>>>(P);
+  LSQ_LAUNCH_CHECK("lora_pad");
+  return LSQ_OK;
 }
 
 static void fill_cb(Params& p) {
@@ -493,12 +807,18 @@ static void fill_cb(Params& p) {
   for (int i = 0; i < 16; ++i) p.cb[i] = cb[i];
 }
 
-}  // namespace nf4g
-}  // namespace lsq
+static lsq_status tmap_act(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, uint32_t box_outer) {
+  return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)inner, (uint64_t)outer,
+                        (uint64_t)inner * 2, 64, box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
-namespace lsq {
+}  // namespace nf4g
+
+// ================================================================ host paths
 namespace tc {
 using namespace lsq::nf4g;
+
+static int rpad(int r) { return r > 0 ? (r + 15) / 16 * 16 : 0; }
 
 static lsq_status nf4_checks(int64_t M, int64_t K, int32_t r, const char* who) {
   lsq_status st = check_device();
@@ -520,23 +840,159 @@ static lsq_status check_weight(const lsq_nf4_weight& w, int64_t K, const char* w
   return LSQ_OK;
 }
 
-lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
-                     const __nv_bfloat16* const* Bp, const __nv_bfloat16* const* At, int r, float s, void* dx,
-                     float* const* g_out, cudaStream_t stream) {
+// ---- forward: workspace = s*U per segment [M, 64] bf16 | padded B per segment [n, 64] bf16 | U partials
+struct FwdPlan {
+  int kbps, splits, np;
+  size_t su, bpad[3], part, total;
+};
+static FwdPlan fwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
+  FwdPlan f;
+  memset(&f, 0, sizeof(f));
+  const int nkb = (int)(K / 64);
+  const int mtiles = (int)((M + ldn::BM - 1) / ldn::BM);
+  f.kbps = ldn::plan_kbps(&nkb, 1, mtiles);
+  f.splits = (nkb + f.kbps - 1) / f.kbps;
+  f.np = nseg * rpad(r);
+  f.su = ldn::round256((size_t)M * 64 * 2);
+  f.total = (size_t)nseg * f.su;
+  for (int i = 0; i < nseg; ++i) {
+    f.bpad[i] = ldn::round256((size_t)n_out[i] * 64 * 2);
+    f.total += f.bpad[i];
+  }
+  f.part = ldn::round256((size_t)f.splits * (size_t)M * (size_t)f.np * sizeof(float));
+  f.total += f.part;
+  return f;
+}
+
+// ---- backward rank-r part: G fp32 | s*G bf16 [M, 64] | A^T side by side [K, 64] | B_q^T [rp, n_q] | G partials
+struct BwdPlan {
+  int kbps, splits[3];
+  size_t g32, sg, at, bt[3], part[3], total;
+};
+static BwdPlan bwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
+  BwdPlan b;
+  memset(&b, 0, sizeof(b));
+  const int rp = rpad(r);
+  int nkb[3];
+  for (int i = 0; i < nseg; ++i) nkb[i] = (int)((n_out[i] + 63) / 64);
+  const int mtiles = (int)((M + ldn::BM - 1) / ldn::BM);
+  b.kbps = ldn::plan_kbps(nkb, nseg, mtiles);
+  b.g32 = ldn::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
+  b.sg = ldn::round256((size_t)M * 64 * 2);
+  b.at = ldn::round256((size_t)K * 64 * 2);
+  b.total = b.g32 + b.sg + b.at;
+  for (int i = 0; i < nseg; ++i) {
+    b.splits[i] = (nkb[i] + b.kbps - 1) / b.kbps;
+    b.bt[i] = ldn::round256((size_t)rp * (size_t)n_out[i] * 2);
+    b.part[i] = ldn::round256((size_t)b.splits[i] * (size_t)M * (size_t)rp * sizeof(float));
+    b.total += b.bt[i] + b.part[i];
+  }
+  return b;
+}
+
+size_t bwd_rank_bytes(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
+  return bwd_plan(nseg, M, K, n_out, r).total;
+}
+
+// G = dY B per segment (fp32 into g_out[q], s*G bf16 into the workspace) and
+// the dX GEMM's LoRA-block operands; ws starts with the layout of bwd_plan.
+// Returns the bf16 s*G and A^T pointers through sg / at.
+lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const void* const* A,
+                         const void* const* B, int r, float s, char* ws, float** g_out, __nv_bfloat16** sg,
+                         __nv_bfloat16** at, cudaStream_t stream) {
+  const int64_t K = W[0].k_in;
+  const int rp = rpad(r);
+  int64_t n_out[3];
+  for (int i = 0; i < nseg; ++i) n_out[i] = W[i].n_out;
+  const BwdPlan b = bwd_plan(nseg, M, K, n_out, r);
+  char* cur = ws;
+  for (int i = 0; i < nseg; ++i) g_out[i] = reinterpret_cast<float*>(cur) + (size_t)i * M * r;
+  cur += b.g32;
+  *sg = reinterpret_cast<__nv_bfloat16*>(cur);
+  cur += b.sg;
+  *at = reinterpret_cast<__nv_bfloat16*>(cur);
+  cur += b.at;
+  __nv_bfloat16* bt[3];
+  float* part[3];
+  for (int i = 0; i < nseg; ++i) {
+    bt[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+    cur += b.bt[i];
+  }
+  for (int i = 0; i < nseg; ++i) {
+    part[i] = reinterpret_cast<float*>(cur);
+    cur += b.part[i];
+  }
+  lsq_status st;
+  ldn::Pad P;
+  memset(&P, 0, sizeof(P));
+  int64_t most = K * 64;
+  for (int i = 0; i < nseg; ++i) {
+    P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
+    P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+    P.Bt[i] = bt[i];
+    P.n[i] = n_out[i];
+    most = std::max<int64_t>(most, (int64_t)rp * n_out[i]);
+  }
+  P.At = *at;
+  P.K = K;
+  P.nseg = nseg;
+  P.r = r;
+  P.rp = rp;
+  P.dx = 1;
+  if ((st = launch_pad(P, most, stream)) != LSQ_OK) return st;
+
+  ldn::Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  ldn::Params p;
+  memset(&p, 0, sizeof(p));
+  p.nprob = nseg;
+  p.M = (int)M;
+  p.rp = rp;
+  p.kbps = b.kbps;
+  int maxsplits = 1;
+  for (int i = 0; i < nseg; ++i) {
+    if ((st = tmap_act(&maps.in[i], dy[i], n_out[i], M, ldn::BM)) != LSQ_OK) return st;
+    if ((st = tmap_act(&maps.wl[i], bt[i], n_out[i], rp, (uint32_t)rp)) != LSQ_OK) return st;
+    ldn::Prob& pr = p.pr[i];
+    pr.part = part[i];
+    pr.nkb = (int)((n_out[i] + 63) / 64);
+    pr.splits = b.splits[i];
+    pr.nsub = 1;
+    pr.first = i;
+    maxsplits = std::max(maxsplits, pr.splits);
+  }
+  if ((st = launch_down(maps, p, maxsplits, stream)) != LSQ_OK) return st;
+
+  ldn::Red R;
+  memset(&R, 0, sizeof(R));
+  for (int i = 0; i < nseg; ++i) {
+    R.part[i] = part[i];
+    R.splits[i] = b.splits[i];
+    R.np[i] = rp;
+    R.out32[i] = g_out[i];
+  }
+  R.out16[0] = *sg;
+  R.dx = 1;
+  R.nseg = nseg;
+  R.M = (int)M;
+  R.r = r;
+  R.rp = rp;
+  R.s = s;
+  return launch_reduce(R, stream);
+}
+
+// dX = sum_q dY_q deq(W_q) (+ (s G) A when sg != null)
+lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const __nv_bfloat16* sg,
+                     const __nv_bfloat16* at, void* dx, cudaStream_t stream) {
   const int64_t K = W[0].k_in;
   Params p;
   memset(&p, 0, sizeof(p));
   p.nseg = nseg;
   p.M = (int)M;
   p.K = (int)K;
-  p.r = r;
-  p.rp = r > 0 ? (r + 15) / 16 * 16 : 0;
-  p.s = s;
+  p.lora = sg ? 1 : 0;
   p.dx = static_cast<__nv_bfloat16*>(dx);
   fill_cb(p);
-  if (nseg * p.rp > KE_MAX) return fail(LSQ_EUNSUPPORTED, "lsq_nf4_lora_bwd: nseg * round16(r) must be <= 64");
-  const int64_t kk[1] = {K};
-  const int BN = pick_bn(kk, 1, M, true);
   Maps maps;
   memset(&maps, 0, sizeof(maps));
   int blocks = 0;
@@ -544,34 +1000,37 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
   for (int i = 0; i < nseg; ++i) {
     Seg& g = p.seg[i];
     g.absmax = W[i].absmax;
-    g.lat = r > 0 ? At[i] : nullptr;
-    g.uo = r > 0 ? g_out[i] : nullptr;
     g.n = (int)W[i].n_out;
     g.first = blocks;
     blocks += (int)((W[i].n_out + BK - 1) / BK);
-    if ((st = encode_tmap_2d(&maps.a[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy[i], W[i].n_out, M, W[i].n_out * 2, BK,
-                             BM, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
-      return st;
-    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2, BN / 2,
-                             BK, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
-      return st;
-    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp[i], 64, W[i].n_out, 64 * 2,
-                                      64, BK, CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+    if ((st = tmap_act(&maps.a[i], dy[i], W[i].n_out, M, BMC)) != LSQ_OK) return st;
+    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
+                             BNC / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
   }
+  if (sg) {
+    if ((st = tmap_act(&maps.la[0], sg, 64, M, BMC)) != LSQ_OK) return st;
+    if ((st = tmap_act(&maps.lb[0], at, 64, K, BNC)) != LSQ_OK) return st;
+  }
   p.nkb = blocks;
-  dim3 grid((unsigned)((K + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-  if (BN == 192) return launch<DX, 192>(maps, p, grid, stream);
-  return launch<DX, 128>(maps, p, grid, stream);
+  p.mtiles = (int)((M + BT - 1) / BT);
+  p.tiles = p.mtiles * (int)((K + BT - 1) / BT);
+  return launch_pair<DX>(maps, p, stream);
 }
 
 }  // namespace tc
 }  // namespace lsq
 
+extern "C" size_t lsq_nf4_lora_fwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
+                                                  int32_t r) {
+  if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
+  return lsq::tc::fwd_plan(nseg, M, k_in, n_out, r).total;
+}
+
 extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
                                              const void* const* A, const void* const* B, int32_t r, float s,
                                              const void* const* residual, void* const* y, float* const* u_out,
-                                             lsq_cuda_stream stream) {
+                                             void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
   using namespace lsq;
   using namespace lsq::nf4g;
   const char* who = "lsq_nf4_lora_fwd";
@@ -581,29 +1040,10 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
   lsq_status st = tc::nf4_checks(M, K, r, who);
   if (st != LSQ_OK) return st;
   if (!aligned(x, 16)) return fail(LSQ_EINVAL, "%s: x must be 16-byte aligned", who);
-  Params p;
-  memset(&p, 0, sizeof(p));
-  p.nseg = nseg;
-  p.M = (int)M;
-  p.K = (int)K;
-  p.r = r;
-  p.rp = r > 0 ? (r + 15) / 16 * 16 : 0;
-  p.s = s;
-  p.nkb = (int)(K / BK);
-  fill_cb(p);
   int64_t ns[3];
   for (int i = 0; i < nseg; ++i) {
     if ((st = tc::check_weight(W[i], K, who)) != LSQ_OK) return st;
     ns[i] = W[i].n_out;
-  }
-  const int BN = pick_bn(ns, nseg, M, true);
-  Maps maps;
-  memset(&maps, 0, sizeof(maps));
-  if ((st = encode_tmap_2d(&maps.a[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, BK, BM,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
-    return st;
-  int tiles = 0;
-  for (int i = 0; i < nseg; ++i) {
     if (!y[i] || !aligned(y[i], 16)) return fail(LSQ_EINVAL, "%s: y[%d] NULL or not 16-byte aligned", who, i);
     const void* res = residual ? residual[i] : nullptr;
     if (res && !aligned(res, 16)) return fail(LSQ_EINVAL, "%s: residual must be 16-byte aligned", who);
@@ -611,35 +1051,123 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
       if (!A || !B || !A[i] || !B[i]) return fail(LSQ_EINVAL, "%s: LoRA A/B NULL with r > 0", who);
       if (!aligned(A[i], 16) || !aligned(B[i], 2)) return fail(LSQ_EINVAL, "%s: LoRA A must be 16-byte aligned", who);
     }
+  }
+  const int rp = tc::rpad(r);
+  const tc::FwdPlan f = tc::fwd_plan(nseg, M, K, ns, r);
+  if (r > 0 && (!workspace || workspace_bytes < f.total || !aligned(workspace, 256)))
+    return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, f.total,
+                workspace_bytes);
+  cudaStream_t cs = (cudaStream_t)stream;
+
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.nseg = nseg;
+  p.M = (int)M;
+  p.K = (int)K;
+  p.lora = r > 0 ? 1 : 0;
+  p.nkb = (int)(K / BK);
+  fill_cb(p);
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if ((st = tmap_act(&maps.a[0], x, K, M, BMC)) != LSQ_OK) return st;
+  int tiles_n = 0;
+  for (int i = 0; i < nseg; ++i) {
     Seg& g = p.seg[i];
     g.absmax = W[i].absmax;
-    g.la = r > 0 ? static_cast<const __nv_bfloat16*>(A[i]) : nullptr;
-    g.lb = r > 0 ? static_cast<const __nv_bfloat16*>(B[i]) : nullptr;
     g.y = static_cast<__nv_bfloat16*>(y[i]);
-    g.res = static_cast<const __nv_bfloat16*>(res);
-    g.uo = (u_out && r > 0) ? u_out[i] : nullptr;
+    g.res = static_cast<const __nv_bfloat16*>(residual ? residual[i] : nullptr);
     g.n = (int)W[i].n_out;
-    g.first = tiles;
-    tiles += (int)((W[i].n_out + BN - 1) / BN);
-    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2, BK / 2,
-                             BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
-      return st;
-    if (r > 0 && (st = encode_tmap_2d(&maps.l[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A[i], K, r, K * 2, BK, p.rp,
-                                      CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+    g.first = tiles_n;
+    tiles_n += (int)((W[i].n_out + BT - 1) / BT);
+    if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
+                             BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
   }
-  dim3 grid(tiles, (unsigned)((M + BM - 1) / BM));
-  if (BN == 192) return launch<FWD, 192>(maps, p, grid, (cudaStream_t)stream);
-  return launch<FWD, 128>(maps, p, grid, (cudaStream_t)stream);
+  p.mtiles = (int)((M + BT - 1) / BT);
+  p.tiles = p.mtiles * tiles_n;
+
+  if (r > 0) {
+    // workspace: s*U per segment | padded B per segment | U partials
+    char* cur = static_cast<char*>(workspace);
+    __nv_bfloat16* su[3];
+    __nv_bfloat16* bpad[3];
+    for (int i = 0; i < nseg; ++i) {
+      su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+      cur += f.su;
+    }
+    for (int i = 0; i < nseg; ++i) {
+      bpad[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+      cur += f.bpad[i];
+    }
+    float* part = reinterpret_cast<float*>(cur);
+
+    ldn::Pad P;
+    memset(&P, 0, sizeof(P));
+    int64_t most = 0;
+    for (int i = 0; i < nseg; ++i) {
+      P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+      P.Bpad[i] = bpad[i];
+      P.n[i] = ns[i];
+      most = std::max<int64_t>(most, ns[i] * 64);
+    }
+    P.K = K;
+    P.nseg = nseg;
+    P.r = r;
+    P.rp = rp;
+    P.dx = 0;
+    if ((st = launch_pad(P, most, cs)) != LSQ_OK) return st;
+
+    ldn::Maps dm;
+    memset(&dm, 0, sizeof(dm));
+    ldn::Params dp;
+    memset(&dp, 0, sizeof(dp));
+    if ((st = tmap_act(&dm.in[0], x, K, M, ldn::BM)) != LSQ_OK) return st;
+    for (int i = 0; i < nseg; ++i)
+      if ((st = tmap_act(&dm.wl[i], A[i], K, r, (uint32_t)rp)) != LSQ_OK) return st;
+    dp.nprob = 1;
+    dp.M = (int)M;
+    dp.rp = rp;
+    dp.kbps = f.kbps;
+    dp.pr[0].part = part;
+    dp.pr[0].nkb = (int)(K / 64);
+    dp.pr[0].splits = f.splits;
+    dp.pr[0].nsub = nseg;
+    dp.pr[0].first = 0;
+    if ((st = launch_down(dm, dp, f.splits, cs)) != LSQ_OK) return st;
+
+    ldn::Red R;
+    memset(&R, 0, sizeof(R));
+    R.part[0] = part;
+    R.splits[0] = f.splits;
+    R.np[0] = f.np;
+    for (int i = 0; i < nseg; ++i) {
+      R.out32[i] = u_out ? u_out[i] : nullptr;
+      R.out16[i] = su[i];
+    }
+    R.dx = 0;
+    R.nseg = nseg;
+    R.M = (int)M;
+    R.r = r;
+    R.rp = rp;
+    R.s = s;
+    if ((st = launch_reduce(R, cs)) != LSQ_OK) return st;
+
+    for (int i = 0; i < nseg; ++i) {
+      if ((st = tmap_act(&maps.la[i], su[i], 64, M, BMC)) != LSQ_OK) return st;
+      if ((st = tmap_act(&maps.lb[i], bpad[i], 64, ns[i], BNC)) != LSQ_OK) return st;
+    }
+  }
+  return launch_pair<FWD>(maps, p, cs);
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A,
                                        const void* B, int32_t r, float s, const void* residual, void* y,
-                                       float* u_out, lsq_cuda_stream stream) {
+                                       float* u_out, void* workspace, size_t workspace_bytes,
+                                       lsq_cuda_stream stream) {
   const void* a[1] = {A};
   const void* b[1] = {B};
   const void* res[1] = {residual};
   void* yy[1] = {y};
   float* uu[1] = {u_out};
-  return lsq_nf4_lora_fwd_multi(1, W, x, M, a, b, r, s, res, yy, uu, stream);
+  return lsq_nf4_lora_fwd_multi(1, W, x, M, a, b, r, s, res, yy, uu, workspace, workspace_bytes, stream);
 }

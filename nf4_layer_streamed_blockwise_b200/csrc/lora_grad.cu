@@ -1,6 +1,7 @@
 // Backward of the fused NF4-LoRA linear:
-//   dX = sum_seg dY_seg deq(W_seg) + s G_seg A_seg     (tensor cores, gemm_tc.cu)
-//   dB_seg = s dY_seg^T U_seg,  dA_seg = s G_seg^T X    (here)
+//   G_seg = dY_seg B_seg                                 (split-K tensor-core kernel, gemm_nf4.cu)
+//   dX = sum_seg dY_seg deq(W_seg) + s G_seg A_seg       (CTA-pair tensor-core kernel, gemm_nf4.cu)
+//   dB_seg = s dY_seg^T U_seg,  dA_seg = s G_seg^T X      (here)
 // dA and dB are skinny products (r <= 64 columns) reduced over the M token
 // rows, i.e. HBM-bound reads of dY and X.  Deterministic two-stage reduction:
 // stage 1 gives each CTA a 256-column panel and a chunk of rows (row tiles of
@@ -14,12 +15,6 @@
 #include "host_common.h"
 
 namespace lsq {
-namespace tc {
-lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M,
-                     const __nv_bfloat16* const* Bp, const __nv_bfloat16* const* At, int r, float s, void* dx,
-                     float* const* g_out, cudaStream_t stream);
-}
-
 namespace lg {
 
 constexpr int PANEL = 256;      // columns per CTA (4 per thread)
@@ -183,35 +178,6 @@ __global__ void __launch_bounds__(256) skinny_reduce(const __grid_constant__ Red
   }
 }
 
-// Rank-padded copies of the LoRA operands for the dX kernel: Bp [n, 64] holds
-// segment seg's B in columns seg*rp .. seg*rp + r - 1 and zeros elsewhere (its
-// main-loop operand, appended to the weight tile, so each segment's G = dY B
-// lands in its own accumulator columns); At [K, rp] = A^T with zero columns
-// >= r (its epilogue operand, fetched as 16-byte rows).
-struct Prep {
-  const __nv_bfloat16* A[3];
-  const __nv_bfloat16* B[3];
-  __nv_bfloat16* At[3];
-  __nv_bfloat16* Bp[3];
-  int64_t n[3];
-  int64_t K;
-  int r, rp;
-};
-
-__global__ void __launch_bounds__(256) lora_prep(const __grid_constant__ Prep P) {
-  const int seg = blockIdx.y >> 1, which = blockIdx.y & 1;
-  const int64_t total = which == 0 ? 64 * P.n[seg] : P.K * P.rp;
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
-    if (which == 0) {  // Bp[n][c] = B[n][c - seg*rp] inside the segment's range, else 0
-      const int64_t n = idx / 64, c = idx % 64, j = c - (int64_t)seg * P.rp;
-      P.Bp[seg][idx] = (j >= 0 && j < P.r) ? P.B[seg][n * P.r + j] : __float2bfloat16_rn(0.0f);
-    } else {           // At[k][j] = A[j][k]
-      const int64_t j = idx / P.K, k = idx % P.K;
-      P.At[seg][k * P.rp + j] = j < P.r ? P.A[seg][j * P.K + k] : __float2bfloat16_rn(0.0f);
-    }
-  }
-}
-
 static int64_t panels_for(int64_t C) { return (C + PANEL - 1) / PANEL; }
 
 static int64_t chunks_for(int64_t M, int64_t C) {
@@ -239,13 +205,9 @@ using namespace lsq;
 
 extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || M < 1 || !n_out) return 256;
-  const size_t rp = (size_t)(r + 15) / 16 * 16;
-  size_t b = lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
-  for (int i = 0; i < nseg; ++i) {
-    b += lg::round256((size_t)64 * (size_t)n_out[i] * 2) + lg::round256((size_t)k_in * rp * 2);
-    b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
-  }
+  if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
+  size_t b = tc::bwd_rank_bytes(nseg, M, k_in, n_out, r);
+  for (int i = 0; i < nseg; ++i) b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
   return b;
 }
 
@@ -284,46 +246,21 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   }
   if (r == 0 && !dx) return LSQ_OK;
   float* g[3] = {nullptr, nullptr, nullptr};
-  __nv_bfloat16* bp[3] = {nullptr, nullptr, nullptr};
-  __nv_bfloat16* at[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* sg = nullptr;
+  __nv_bfloat16* at = nullptr;
   char* part = nullptr;
+  cudaStream_t cs = (cudaStream_t)stream;
   if (r > 0) {
     const size_t need = lsq_nf4_lora_bwd_workspace_size(nseg, M, K, n_out, r);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
       return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, need,
                   workspace_bytes);
-    float* ws = static_cast<float*>(workspace);
-    for (int i = 0; i < nseg; ++i) g[i] = ws + (size_t)i * M * r;
-    part = static_cast<char*>(workspace) + lg::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
-    for (int i = 0; i < nseg; ++i) {
-      bp[i] = reinterpret_cast<__nv_bfloat16*>(part);
-      part += lg::round256((size_t)64 * (size_t)n_out[i] * 2);
-      at[i] = reinterpret_cast<__nv_bfloat16*>(part);
-      part += lg::round256((size_t)K * (size_t)rp * 2);
-    }
+    char* ws = static_cast<char*>(workspace);
+    // G = dY B (fp32 for dA, s*G in bf16 for the dX kernel) and the padded operands
+    if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, r, s, ws, g, &sg, &at, cs)) != LSQ_OK) return st;
+    part = ws + tc::bwd_rank_bytes(nseg, M, K, n_out, r);
   }
-  cudaStream_t cs = (cudaStream_t)stream;
-  if (r > 0) {
-    lg::Prep P;
-    memset(&P, 0, sizeof(P));
-    int64_t most = 0;
-    for (int i = 0; i < nseg; ++i) {
-      P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
-      P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
-      P.At[i] = at[i];
-      P.Bp[i] = bp[i];
-      P.n[i] = n_out[i];
-      most = std::max<int64_t>(most, std::max<int64_t>((int64_t)64 * n_out[i], K * rp));
-    }
-    P.K = K;
-    P.r = r;
-    P.rp = rp;
-    int64_t gx = (most + 255) / 256;
-    if (gx > 512) gx = 512;
-    lg::lora_prep<<<dim3((unsigned)gx, 2 * nseg), 256, 0, cs>>>(P);
-    LSQ_LAUNCH_CHECK("lora_prep");
-  }
-  if ((st = tc::launch_dx(nseg, W, dy, M, bp, at, r, s, dx, g, cs)) != LSQ_OK) return st;
+  if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
   lg::RedSet rs;
   memset(&rs, 0, sizeof(rs));

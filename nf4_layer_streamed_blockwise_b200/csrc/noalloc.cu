@@ -1,7 +1,8 @@
 // Backward of the fused NF4-LoRA linear for callers that cannot allocate
 // device memory.  Same computation and kernels as lsq_nf4_lora_bwd; the
-// scratch (G = dY B and the dA/dB partial sums) lives in a fixed array that
-// the library itself holds in device memory.
+// scratch (G = dY B, its partial sums, the padded LoRA operands and the dA/dB
+// partial sums) lives in a fixed array that the library itself holds in
+// device memory.
 //
 // Who needs it: code that runs where a cudaMalloc is not allowed or not
 // possible - a host framework that owns the whole device memory pool and hands
@@ -16,10 +17,11 @@
 namespace lsq {
 namespace noalloc {
 
-// Largest scratch the entry point serves: 8 MiB, which covers one linear of
-// the 8B shape at 2048 tokens and r = 16 with room to spare.  Every GPU that
+// Largest scratch the entry point serves: 32 MiB, which covers any one linear
+// of the 8B shape at 2048 tokens and r = 16 (12.5 MiB for a 4096 x 4096
+// projection, 14.3 MiB for the 14336-wide down projection).  Every GPU that
 // loads the library keeps this array for as long as the process lives.
-constexpr size_t SCRATCH_BYTES = size_t(8) << 20;
+constexpr size_t SCRATCH_BYTES = size_t(32) << 20;
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[SCRATCH_BYTES];
 

@@ -54,12 +54,13 @@ _SIGS = {
     "lsq_nf4_codebook": (c_int32, [ctypes.POINTER(c_float)]),
     "lsq_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "lsq_nf4_dequantize": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p]),
+    "lsq_nf4_lora_fwd_workspace_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
     "lsq_nf4_lora_fwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64, c_void_p, c_void_p, c_int32,
-                                   c_float, c_void_p, c_void_p, c_void_p, c_void_p]),
+                                   c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsq_nf4_lora_fwd_multi": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
                                          ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int32, c_float,
                                          ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
-                                         ctypes.POINTER(c_void_p), c_void_p]),
+                                         ctypes.POINTER(c_void_p), c_void_p, c_size_t, c_void_p]),
     "lsq_nf4_lora_bwd_workspace_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
     "lsq_nf4_lora_bwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                    c_int32, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
@@ -132,9 +133,11 @@ def _check(name: str, status: int):
 
 
 # kernel launches issued by the library, counted per call on this side
-# (lsq_nf4_lora_bwd: a LoRA-operand transpose, the dX GEMM and two reduction kernels)
+# (with a LoRA adapter the fused linear's forward is 4 kernels: operand padding,
+# the split-K rank-r product, its reduction and the main GEMM; the backward is
+# those three, the dX GEMM when dx is wanted, and the two dA/dB reduction kernels)
 LAUNCHES = [0]
-_KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_nf4_lora_fwd": 1, "lsq_nf4_lora_fwd_multi": 1,
+_KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
             "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
             "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1}
@@ -222,20 +225,39 @@ def lsq_nf4_dequantize(w: NF4Weight, out_bf16: torch.Tensor, stream=None):
     _call("lsq_nf4_dequantize", ctypes.byref(cw), _p(out_bf16), _stream(stream))
 
 
-def lsq_nf4_lora_fwd(W: NF4Weight, x, M: int, A, B, r: int, s: float, residual, y, u_out, stream=None):
+def lsq_nf4_lora_fwd_workspace_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
+    arr = (c_int64 * len(n_outs))(*n_outs)
+    return int(_fn("lsq_nf4_lora_fwd_workspace_size")(len(n_outs), M, k_in, arr, r))
+
+
+def _fwd_workspace(workspace, n_outs, M, k_in, r, device):
+    """The caller's workspace, or (when None and r > 0) a fresh one of the size the library asks for."""
+    if workspace is not None or r == 0:
+        return workspace
+    return torch.empty(lsq_nf4_lora_fwd_workspace_size(n_outs, M, k_in, r), dtype=torch.uint8, device=device)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def lsq_nf4_lora_fwd(W: NF4Weight, x, M: int, A, B, r: int, s: float, residual, y, u_out, stream=None,
+                     workspace=None):
     cw = W.c()
+    ws = _fwd_workspace(workspace, [W.n_out], M, W.k_in, r, y.device)
     _call("lsq_nf4_lora_fwd", ctypes.byref(cw), _p(x), M, _p(A), _p(B), r, s, _p(residual), _p(y), _p(u_out),
-          _stream(stream))
+          _p(ws), _nbytes(ws), _stream(stream), launches=4 if r > 0 else 1)
 
 
 def lsq_nf4_lora_fwd_multi(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: float, residual, y, u_out,
-                           stream=None):
+                           stream=None, workspace=None):
     n = len(Ws)
     cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
     res = residual if residual is not None else [None] * n
     uo = u_out if u_out is not None else [None] * n
+    ws = _fwd_workspace(workspace, [w.n_out for w in Ws], M, Ws[0].k_in, r, y[0].device)
     _call("lsq_nf4_lora_fwd_multi", n, cws, _p(x), M, _ptrs(A), _ptrs(B), r, s, _ptrs(res), _ptrs(y), _ptrs(uo),
-          _stream(stream))
+          _p(ws), _nbytes(ws), _stream(stream), launches=4 if r > 0 else 1)
 
 
 def lsq_nf4_lora_bwd_workspace_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
@@ -248,7 +270,11 @@ def lsq_nf4_lora_bwd(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx,
     cw = W.c()
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
-          _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (3 if r > 0 else 0))
+          _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=_bwd_launches(r, dx))
+
+
+def _bwd_launches(r: int, dx) -> int:
+    return (1 if dx is not None else 0) + (5 if r > 0 else 0)
 
 
 def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB,
@@ -257,7 +283,7 @@ def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int,
     cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_nf4_lora_bwd_multi", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(dx),
-          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=1 + (3 if r > 0 else 0))
+          _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=_bwd_launches(r, dx))
 
 
 def lsq_nf4_lora_bwd_noalloc_max_scratch() -> int:
@@ -270,7 +296,7 @@ def lsq_nf4_lora_bwd_noalloc(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float
     scratch array is used, for callers that cannot allocate device memory."""
     cw = W.c()
     _call("lsq_nf4_lora_bwd_noalloc", ctypes.byref(cw), _p(x), _p(dy), M, _p(A), _p(B), r, s, _p(u), _p(dx), _p(dA),
-          _p(dB), accumulate, _stream(stream), launches=1 + (3 if r > 0 else 0))
+          _p(dB), accumulate, _stream(stream), launches=_bwd_launches(r, dx))
 
 
 def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int, stream=None):

@@ -4,7 +4,8 @@
         [--iters 20] [--only fwd_qkv,...]
 
 For every linear group of a decoder layer (q/k/v fused, o, gate/up fused,
-down) it times the forward kernel and the dX kernel, and the lm_head GEMMs,
+down) it times the forward call (all its kernels), the backward call, the dX
+GEMM alone (no adapter), and the lm_head GEMMs,
 with CUDA events around each launch and a 256 MB L2 flush between launches;
 prints one JSON line per kernel (median ms, TFLOP/s, fraction of the
 measured bf16 peak).  Inputs are random; only timing is reported.
@@ -86,7 +87,8 @@ def main():
         ys = [torch.empty(M, n, **bf) for n in ns]
         us = [torch.empty(M, r, dtype=torch.float32, device="cuda") for _ in ns]
         fl = sum(2.0 * M * n * K + 2.0 * M * r * K + 2.0 * M * n * r for n in ns)
-        run(f"fwd_{g}", fl, lambda: L.lsq_nf4_lora_fwd_multi(Ws, x, M, A, B, r, s, None, ys, us))
+        wsf = torch.empty(L.lsq_nf4_lora_fwd_workspace_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
+        run(f"fwd_{g}", fl, lambda: L.lsq_nf4_lora_fwd_multi(Ws, x, M, A, B, r, s, None, ys, us, workspace=wsf))
         dys = [torch.randn(M, n, **bf) for n in ns]
         dx = torch.empty(M, K, **bf)
         dA = [torch.empty(r, K, dtype=torch.float32, device="cuda") for _ in ns]
@@ -96,7 +98,7 @@ def main():
         fl0 = sum(2.0 * M * n * K for n in ns)
         run(f"dx_{g}", fl0, lambda: L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, None, None, 0, 0.0, None, dx, None, None,
                                                                 0, None))
-        del Ws, x, A, B, ys, us, dys, dx, dA, dB, ws
+        del Ws, x, A, B, ys, us, dys, dx, dA, dB, ws, wsf
     hn = torch.randn(M, sh.d, **bf)
     E = torch.randn(sh.vocab, sh.d, **bf) * 0.02
     logits = torch.empty(M, sh.vocab, dtype=torch.float32, device="cuda")

@@ -218,10 +218,10 @@ class StreamedLoraTrainer:
         self.hn = torch.empty(M, d, **bf)
         self.logits = torch.empty(M, sh.vocab, **f32)
         self.dlogits = torch.empty(M, sh.vocab, **bf)
-        ws = max(L.lsq_nf4_lora_bwd_workspace_size([d, kv, kv], M, d, r),
-                 L.lsq_nf4_lora_bwd_workspace_size([d], M, d, r),
-                 L.lsq_nf4_lora_bwd_workspace_size([f, f], M, d, r),
-                 L.lsq_nf4_lora_bwd_workspace_size([d], M, f, r))
+        # one scratch buffer serves every fused linear, forward and backward (they run in order on one stream)
+        groups = [([d, kv, kv], d), ([d], d), ([f, f], d), ([d], f)]
+        ws = max(max(L.lsq_nf4_lora_bwd_workspace_size(ns, M, k, r), L.lsq_nf4_lora_fwd_workspace_size(ns, M, k, r))
+                 for ns, k in groups)
         self.ws_lora = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(L.lsq_attention_bwd_workspace_size(self.B, self.S, sh.n_q), dtype=torch.uint8,
                                    device=dev)
@@ -266,22 +266,23 @@ class StreamedLoraTrainer:
         t = self._t0()
         L.lsq_nf4_lora_fwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, M, [A["q"], A["k"], A["v"]],
                                  [B["q"], B["k"], B["v"]], r, s, None, [self.q, self.k, self.v],
-                                 [U["q"], U["k"], U["v"]])
+                                 [U["q"], U["k"], U["v"]], workspace=self.ws_lora)
         self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d))
         L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
         L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
         L.lsq_attention_fwd(self.q, self.k, self.v, self.a, self.lse, self.B, self.S, sh.n_q, sh.n_kv, sh.hd)
         t = self._t0()
-        L.lsq_nf4_lora_fwd(W.W["o"], self.a, M, A["o"], B["o"], r, s, hin, self.hmid, U["o"])
+        L.lsq_nf4_lora_fwd(W.W["o"], self.a, M, A["o"], B["o"], r, s, hin, self.hmid, U["o"], workspace=self.ws_lora)
         self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d))
         L.lsq_rmsnorm_fwd(self.hmid, W.ln2, self.x2, self.rstd2, M, sh.d, sh.eps)
         t = self._t0()
         L.lsq_nf4_lora_fwd_multi([W.W["gate"], W.W["up"]], self.x2, M, [A["gate"], A["up"]], [B["gate"], B["up"]],
-                                 r, s, None, [self.g, self.u], [U["gate"], U["up"]])
+                                 r, s, None, [self.g, self.u], [U["gate"], U["up"]], workspace=self.ws_lora)
         self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d))
         L.lsq_swiglu_fwd(self.g, self.u, self.mm, M * sh.f)
         t = self._t0()
-        L.lsq_nf4_lora_fwd(W.W["down"], self.mm, M, A["down"], B["down"], r, s, self.hmid, hout, U["down"])
+        L.lsq_nf4_lora_fwd(W.W["down"], self.mm, M, A["down"], B["down"], r, s, self.hmid, hout, U["down"],
+                           workspace=self.ws_lora)
         self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f))
 
     def _layer_bwd(self, l: int, W: LayerView):

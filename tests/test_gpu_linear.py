@@ -108,6 +108,23 @@ def test_fwd_matches_oracle(lsq, M, N, K, r):
     assert_close(u.cpu().numpy(), U, rel=1e-5, max_rms=1e-4, what="U")
 
 
+def test_fwd_many_tiles_per_cluster(lsq):
+    """256 output tiles of 256 x 256 (8 x 32): every SM pair of the persistent
+    kernel takes several, so both TMEM accumulators are reused and their
+    barriers change phase more than once; M and N also leave ragged edges."""
+    M, N, K, r = 1960, 8184, 128, 16
+    case = S.linear_case(M, N, K, r, s=16.0 / r, seed=77)
+    w = _gpu_quant(lsq, case["W"])
+    A, B = _lora_bf16(case)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    u = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    lsq.lsq_nf4_lora_fwd(w, case["X"].cuda(), M, A.cuda(), B.cuda(), r, case["s"], None, y, u)
+    torch.cuda.synchronize()
+    Y, U, _ = _oracle_fwd(case, *_oracle_quant(case["W"]))
+    assert_close(y.float().cpu().numpy(), Y, what="Y")
+    assert_close(u.cpu().numpy(), U, rel=1e-5, max_rms=1e-4, what="U")
+
+
 def test_fwd_with_residual_and_no_lora(lsq):
     M, N, K = 96, 264, 256
     case = S.linear_case(M, N, K, 8)
@@ -181,6 +198,29 @@ def test_bwd_matches_oracle(lsq, M, N, K, r):
     torch.cuda.synchronize()
     assert_close(dA.cpu().numpy(), 2 * rdA, what="2dA")
     assert_close(dB.cpu().numpy(), 2 * rdB, what="2dB")
+
+
+def test_bwd_many_tiles_per_cluster(lsq):
+    """dX over 256 tiles (8 x 32 of 256 x 256): several per SM pair; n_out = 136
+    leaves a partial contraction block, M = 2000 a partial row tile."""
+    M, N, K, r = 2000, 136, 8192, 16
+    case = S.linear_case(M, N, K, r, s=16.0 / r, seed=78)
+    w = _gpu_quant(lsq, case["W"])
+    A, B = _lora_bf16(case)
+    x, dy = case["X"].cuda(), case["dY"].cuda()
+    u = torch.from_numpy((_f64(case["X"]) @ _f64(A).T).astype(np.float32)).cuda()
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lsq.lsq_nf4_lora_bwd_workspace_size([N], M, K, r), dtype=torch.uint8, device="cuda")
+    lsq.lsq_nf4_lora_bwd(w, x, dy, M, A.cuda(), B.cuda(), r, case["s"], u, dx, dA, dB, 0, ws)
+    torch.cuda.synchronize()
+    packed, am = _oracle_quant(case["W"])
+    Wd = ON.dequantize_f64(packed, am, N, K)
+    rdX, rdA, rdB, _ = OL.lora_backward(_f64(case["X"]), Wd, _f64(A), _f64(B), case["s"], _f64(case["dY"]))
+    assert_close(dx.float().cpu().numpy(), rdX, what="dX")
+    assert_close(dA.cpu().numpy(), rdA, what="dA")
+    assert_close(dB.cpu().numpy(), rdB, what="dB")
 
 
 def test_bwd_multi_segments_sum(lsq):
