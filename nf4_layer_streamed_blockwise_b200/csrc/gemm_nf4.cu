@@ -27,7 +27,8 @@
 //   4     TMA producer: activation tile, packed codes, the LoRA block's tiles
 //   5     TMEM owner; in the leader CTA (rank 0) also the MMA issuer
 //   6-13  NF4 decoders: two threads per 64-value block of the stage, each
-//         writing half of one 128-byte row of the swizzled bf16 operand
+//         writing half of one 128-byte row of the swizzled bf16 operand; the
+//         block's 16 possible values live in registers (byte-permute decode)
 // The leader's "full" barrier of a stage completes when both CTAs' TMA bytes
 // have landed and all 16 decoder warps of the pair have arrived; the MMA
 // commit releases the stage in both CTAs at once (commit multicast).  Every
@@ -115,24 +116,56 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-// eight codes (one 32-bit word; first element = high nibble of byte 0) -> eight bf16
-__device__ __forceinline__ uint4 dq8(uint32_t w, float a, const float* cb) {
-  uint4 o;
-  o.x = pack_bf16x2(__fmul_rn(cb[(w >> 4) & 15], a), __fmul_rn(cb[w & 15], a));
-  o.y = pack_bf16x2(__fmul_rn(cb[(w >> 12) & 15], a), __fmul_rn(cb[(w >> 8) & 15], a));
-  o.z = pack_bf16x2(__fmul_rn(cb[(w >> 20) & 15], a), __fmul_rn(cb[(w >> 16) & 15], a));
-  o.w = pack_bf16x2(__fmul_rn(cb[(w >> 28) & 15], a), __fmul_rn(cb[(w >> 24) & 15], a));
-  return o;
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// The 16 dequantised values bf16(code_value[c] * absmax) of one NF4 block, held
+// in registers as byte planes: lo[j] / hi[j] are the low / high bytes of
+// entries 4j .. 4j+3.  Decoding then selects bytes with prmt instead of
+// looking the codebook up in shared memory per value: the same fp32 product
+// and round-to-nearest-even as lsq_nf4_dequantize, computed once per code
+// value and block, and no shared-memory traffic per value.
+struct DqTab {
+  uint32_t lo[4], hi[4];
+};
+__device__ __forceinline__ DqTab dq_table(float a, const float (&cb)[16]) {
+  DqTab t;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t t0 = pack_bf16x2(__fmul_rn(cb[4 * j], a), __fmul_rn(cb[4 * j + 1], a));
+    const uint32_t t1 = pack_bf16x2(__fmul_rn(cb[4 * j + 2], a), __fmul_rn(cb[4 * j + 3], a));
+    t.lo[j] = prmt(t0, t1, 0x6420u);
+    t.hi[j] = prmt(t0, t1, 0x7531u);
+  }
+  return t;
+}
+// Four codes in the low 16 bits of ch (byte 0 = codes 0 | 1, high nibble
+// first) -> four bf16 as two words.  prmt selects one of 8 bytes by the low 3
+// bits of a selector nibble, so each plane is read as two 8-entry halves and
+// the half is chosen per byte by bit 3 of the code (mask m: 0xFF where set).
+__device__ __forceinline__ uint2 dq4(uint32_t ch, const DqTab& t) {
+  const uint32_t s7 = ch & 0x7777u, c8 = ch & 0x8888u;
+  const uint32_t m = prmt(0u, 0x80u, c8 | (c8 >> 1));  // nibble 0xC: sign of byte 4 (0x80) -> 0xFF; 0 -> 0x00
+  const uint32_t lo = (prmt(t.lo[0], t.lo[1], s7) & ~m) | (prmt(t.lo[2], t.lo[3], s7) & m);
+  const uint32_t hi = (prmt(t.hi[0], t.hi[1], s7) & ~m) | (prmt(t.hi[2], t.hi[3], s7) & m);
+  // lo / hi bytes are ordered (code 1, code 0, code 3, code 2): interleave to bf16 words
+  return make_uint2(prmt(lo, hi, 0x4051u), prmt(lo, hi, 0x6273u));
+}
+// eight codes (one 32-bit word) -> eight bf16
+__device__ __forceinline__ uint4 dq8(uint32_t w, const DqTab& t) {
+  const uint2 a = dq4(w, t), b = dq4(w >> 16, t);
+  return make_uint4(a.x, a.y, b.x, b.y);
 }
 
 // half of an NF4 block (32 values, 16 code bytes) -> 16-byte chunks
 // half*4 .. half*4+3 of one 128-byte row of a 128B-swizzled tile
-__device__ __forceinline__ void store_half_row(uint32_t row_addr, int row, int half, uint4 c, float a,
-                                               const float* cb) {
+__device__ __forceinline__ void store_half_row(uint32_t row_addr, int row, int half, uint4 c, const DqTab& t) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    st_shared_v4(row_addr + ((uint32_t)((half * 4 + q) ^ (row & 7)) << 4), dq8(w[q], a, cb));
+  for (int q = 0; q < 4; ++q) st_shared_v4(row_addr + ((uint32_t)((half * 4 + q) ^ (row & 7)) << 4), dq8(w[q], t));
 }
 
 // ================================================================ main kernel
@@ -212,7 +245,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  float* s_cb = reinterpret_cast<float*>(smem + OFF_MISC + 16);
 
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,7 +264,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  if (threadIdx.x < 16) s_cb[threadIdx.x] = p.cb[threadIdx.x];
   if (warp == 5) {
     tmem_alloc_pair(s_tmem, 512);
     tmem_relinquish_pair();
@@ -372,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               break;
             }
             const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + t * 16);
-            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + row * 128, row, half, c, valid ? a : 0.0f, s_cb);
+            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + row * 128, row, half, c, dq_table(valid ? a : 0.0f, p.cb));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(fl);
@@ -431,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + nl * (BNC / 2) + kc * 32 +
                                                             half * 16);
-            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + kc * 8192 + nl * 128, nl, half, c, a, s_cb);
+            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + kc * 8192 + nl * 128, nl, half, c, dq_table(a, p.cb));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(fl);
