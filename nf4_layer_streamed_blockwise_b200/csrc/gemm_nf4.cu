@@ -35,6 +35,7 @@
 // wait is bounded (common.cuh); there are no atomics, so results do not
 // depend on timing or on which SM ran which tile.
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "host_common.h"
@@ -169,24 +170,35 @@ __device__ __forceinline__ void store_half_row(uint32_t row_addr, int row, int h
 }
 
 // ================================================================ main kernel
-constexpr int BMC = 128;  // activation rows per CTA (256 per pair)
+constexpr int BMC = 128;  // activation rows per CTA and half (256 per pair)
 constexpr int BNC = 128;  // weight columns decoded per CTA
-constexpr int BT = 256;   // tile edge of the pair: 256 rows x 256 output columns
+constexpr int BT = 256;   // output columns of a pair tile (its rows: 256 * H)
 constexpr int BK = 64;
-constexpr int NST = 6;
-constexpr int A_BYTES = BMC * BK * 2;  // 16 KB
+constexpr int A_BYTES = BMC * BK * 2;  // 16 KB per 128-row activation tile
 constexpr int W_BYTES = BNC * BK * 2;  // 16 KB
 constexpr int C_BYTES = BNC * BK / 2;  // 4 KB
 constexpr int DQ_WARPS = 8;
 constexpr int NTHREADS = (6 + DQ_WARPS) * 32;
-constexpr int OFF_A = 0;
-constexpr int OFF_W = OFF_A + NST * A_BYTES;
-constexpr int OFF_C = OFF_W + NST * W_BYTES;
-constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
-constexpr int NBAR = 3 * NST + 5;
-constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-constexpr int SMEM_BYTES = OFF_MISC + 128 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+// H = 256-row halves per pair tile.  H = 1: six stages and two accumulator
+// buffers, so the epilogue of one tile overlaps the main loop of the next.
+// H = 2: a 512 x 256 tile whose two halves share every decoded weight tile
+// (half the decode work per FLOP); both accumulators fill TMEM, four stages.
+template <int H>
+struct PCfg {
+  static constexpr int NST = H == 1 ? 6 : 4;
+  static constexpr int NBUF = H == 1 ? 2 : 1;
+  static constexpr int A_STAGE = H * A_BYTES;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_W = OFF_A + NST * A_STAGE;
+  static constexpr int OFF_C = OFF_W + NST * W_BYTES;
+  static constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
+  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+  static constexpr int SMEM_BYTES = OFF_MISC + 128 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(NBUF * H * BT <= 512, "TMEM columns");
+};
 
 struct Seg {
   const float* absmax;
@@ -220,10 +232,10 @@ __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
   return sg;
 }
 
-template <int MODE>
+template <int MODE, int H>
 __device__ __forceinline__ void tile_at(const Params& p, int t, int& m0, int& sg, int& n0) {
   const int mt = t % p.mtiles, nt = t / p.mtiles;
-  m0 = mt * BT;
+  m0 = mt * BT * H;
   sg = 0;
   if (MODE == FWD) {
     while (sg + 1 < p.nseg && nt >= p.seg[sg + 1].first) ++sg;
@@ -233,18 +245,20 @@ __device__ __forceinline__ void tile_at(const Params& p, int t, int& m0, int& sg
   }
 }
 
-template <int MODE>
+template <int MODE, int H>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     nf4_pair_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
+  using C = PCfg<H>;
+  constexpr int NST = C::NST, NBUF = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + NST;
   uint64_t* cfull = empty + NST;
   uint64_t* tfull = cfull + NST;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  uint64_t* tempty = tfull + NBUF;
+  uint64_t* drain = tempty + NBUF;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
 
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&empty[s], 1);
       mbar_init(&cfull[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 2);  // one epilogue arrival per CTA
     }
@@ -280,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       for (int t = cid; t < p.tiles && ok; t += ncl) {
         int m0, sg, n0;
-        tile_at<MODE>(p, t, m0, sg, n0);
+        tile_at<MODE, H>(p, t, m0, sg, n0);
         const int mrow = m0 + (int)rank * BMC, wcol = n0 + (int)rank * BNC;
         for (int i = 0; i < nkb_all; ++i, ++g) {
           const int s = (int)(g % NST);
@@ -290,27 +304,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             break;
           }
           const uint32_t fl = cluster_addr(&full[s], 0);
-          uint8_t* a_dst = smem + OFF_A + s * A_BYTES;
+          uint8_t* a_dst = smem + C::OFF_A + s * C::A_STAGE;
           if (i < p.nkb) {
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * A_BYTES);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * H * A_BYTES);
             mbar_arrive_expect_tx(&cfull[s], (uint32_t)C_BYTES);
-            uint8_t* c_dst = smem + OFF_C + s * C_BYTES;
-            if (MODE == DX) {
-              const int bs = seg_of_block(p, i);
-              const int nb = i - p.seg[bs].first;
-              tma_load_2d_pair(a_dst, &maps.a[bs], fl, nb * BK, mrow);
-              tma_load_2d(c_dst, &maps.c[bs], &cfull[s], wcol / 2, nb * BK);
-            } else {
-              tma_load_2d_pair(a_dst, &maps.a[0], fl, i * BK, mrow);
-              tma_load_2d(c_dst, &maps.c[sg], &cfull[s], i * (BK / 2), wcol);
-            }
+            uint8_t* c_dst = smem + C::OFF_C + s * C_BYTES;
+            const int bs = (MODE == DX) ? seg_of_block(p, i) : 0;
+            const int x = (MODE == DX) ? (i - p.seg[bs].first) * BK : i * BK;
+#pragma unroll
+            for (int h = 0; h < H; ++h) tma_load_2d_pair(a_dst + h * A_BYTES, &maps.a[bs], fl, x, mrow + h * BT);
+            if (MODE == DX) tma_load_2d(c_dst, &maps.c[bs], &cfull[s], wcol / 2, x);
+            else tma_load_2d(c_dst, &maps.c[sg], &cfull[s], i * (BK / 2), wcol);
           } else {
             // no codes for the LoRA block, but cfull[s] still completes one phase per
             // block, so that every barrier's parity follows the block counter
             mbar_arrive(&cfull[s]);
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (A_BYTES + W_BYTES));
-            tma_load_2d_pair(a_dst, &maps.la[sg], fl, 0, mrow);
-            tma_load_2d_pair(smem + OFF_W + s * W_BYTES, &maps.lb[sg], fl, 0, wcol);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (H * A_BYTES + W_BYTES));
+#pragma unroll
+            for (int h = 0; h < H; ++h) tma_load_2d_pair(a_dst + h * A_BYTES, &maps.la[sg], fl, 0, mrow + h * BT);
+            tma_load_2d_pair(smem + C::OFF_W + s * W_BYTES, &maps.lb[sg], fl, 0, wcol);
           }
         }
       }
@@ -324,14 +336,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       int j = 0;
       bool ok = true;
       for (int t = cid; t < p.tiles && ok; t += ncl, ++j) {
-        const int buf = j & 1;
-        const uint32_t tph = (uint32_t)(j >> 1) & 1u;
+        const int buf = j % NBUF;
+        const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
         if (!mbar_wait(&tempty[buf], tph ^ 1u, 521)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(buf * BT);
+        const uint32_t d = tmem + (uint32_t)(buf * H * BT);
         for (int i = 0; i < nkb_all; ++i, ++g) {
           const int s = (int)(g % NST);
           const uint32_t ph = (g / NST) & 1u;
@@ -340,15 +352,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + OFF_A + s * A_BYTES);
-          const uint32_t w_base = smem_u32(smem + OFF_W + s * W_BYTES);
+          const uint32_t a_base = smem_u32(smem + C::OFF_A + s * C::A_STAGE);
+          const uint32_t w_base = smem_u32(smem + C::OFF_W + s * W_BYTES);
           const bool mn = (MODE == DX) && i < p.nkb;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, 2);
             const uint64_t bd =
                 mn ? smem_desc(w_base + kk * 2048, 8192, 1024, 2) : smem_desc(w_base + kk * 32, 16, 1024, 2);
-            tc_mma_pair(d, ad, bd, mn ? id_mn : id_k, (i | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+              tc_mma_pair(d + (uint32_t)(h * BT), smem_desc(a_base + h * A_BYTES + kk * 32, 16, 1024, 2), bd,
+                          mn ? id_mn : id_k, (i | kk) != 0);
           }
           tc_commit_pair_mc(&empty[s], 0x3);
         }
@@ -367,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int tt = cid; tt < p.tiles && ok; tt += ncl) {
       int m0, sg, n0;
-      tile_at<MODE>(p, tt, m0, sg, n0);
+      tile_at<MODE, H>(p, tt, m0, sg, n0);
       const int wcol = n0 + (int)rank * BNC;
       if (MODE == FWD) {
         // thread -> (row, half): consecutive lanes read consecutive 16-byte code
@@ -402,8 +416,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               ok = false;
               break;
             }
-            const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + t * 16);
-            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + row * 128, row, half, c, dq_table(valid ? a : 0.0f, p.cb));
+            const uint4 c = *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C_BYTES + t * 16);
+            store_half_row(smem_u32(smem + C::OFF_W + s * W_BYTES) + row * 128, row, half, c, dq_table(valid ? a : 0.0f, p.cb));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(fl);
@@ -460,9 +474,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               ok = false;
               break;
             }
-            const uint4 c = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + nl * (BNC / 2) + kc * 32 +
+            const uint4 c = *reinterpret_cast<const uint4*>(smem + C::OFF_C + s * C_BYTES + nl * (BNC / 2) + kc * 32 +
                                                             half * 16);
-            store_half_row(smem_u32(smem + OFF_W + s * W_BYTES) + kc * 8192 + nl * 128, nl, half, c, dq_table(a, p.cb));
+            store_half_row(smem_u32(smem + C::OFF_W + s * W_BYTES) + kc * 8192 + nl * 128, nl, half, c, dq_table(a, p.cb));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(fl);
@@ -483,17 +497,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     int j = 0;
     for (int t = cid; t < p.tiles; t += ncl, ++j) {
       int m0, sg, n0;
-      tile_at<MODE>(p, t, m0, sg, n0);
-      const int buf = j & 1;
-      const uint32_t tph = (uint32_t)(j >> 1) & 1u;
+      tile_at<MODE, H>(p, t, m0, sg, n0);
+      const int buf = j % NBUF;
+      const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
       tc_fence_after();
-      const int m = m0 + (int)rank * BMC + e;
       const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
-      for (int c = 0; c < BT / 32; ++c) {
-        if (n0 + c * 32 >= ncols) break;
+      for (int hc = 0; hc < H * (BT / 32); ++hc) {
+        const int h = hc / (BT / 32), c = hc % (BT / 32);
+        if (n0 + c * 32 >= ncols) continue;
+        const int m = m0 + h * BT + (int)rank * BMC + e;
         float v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(buf * BT + c * 32), v);
+        tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
         tc_wait_ld();
         if (m >= p.M) continue;
 #pragma unroll
@@ -728,25 +743,35 @@ __global__ void __launch_bounds__(256) lora_down_reduce(const __grid_constant__ 
 //   FWD job q: Bpad_q [n_q, 64] = B_q in columns < r, zero elsewhere
 //   DX  job q < nseg: Bt_q [rp, n_q] = B_q^T, zero rows >= r
 //   DX  job nseg: At [K, 64] = A_q^T of every segment q in columns q*rp .., zero elsewhere
+//   DX  job nseg + 1 + q: SU_q [M, 64] = bf16(s * U_q) in columns < r, zero elsewhere
 struct Pad {
   const __nv_bfloat16* A[3];
   const __nv_bfloat16* B[3];
+  const float* U[3];
   __nv_bfloat16* Bpad[3];
   __nv_bfloat16* Bt[3];
+  __nv_bfloat16* SU[3];
   __nv_bfloat16* At;
   int64_t n[3];
-  int64_t K;
+  int64_t K, M;
   int nseg, r, rp, dx;
+  float s;
 };
 
 __global__ void __launch_bounds__(256) lora_pad(const __grid_constant__ Pad P) {
   const int job = blockIdx.y;
   const bool at = P.dx && job == P.nseg;
-  const int64_t total = at ? P.K * 64 : P.dx ? (int64_t)P.rp * P.n[job] : P.n[job] * 64;
+  const bool su = P.dx && job > P.nseg;
+  const int64_t total = su ? P.M * 64 : at ? P.K * 64 : P.dx ? (int64_t)P.rp * P.n[job] : P.n[job] * 64;
   const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
-    if (at) {
+    if (su) {
+      const int q = job - P.nseg - 1;
+      const int64_t m = idx / 64;
+      const int c = (int)(idx % 64);
+      P.SU[q][idx] = c < P.r ? __float2bfloat16_rn(P.s * P.U[q][m * P.r + c]) : zero;
+    } else if (at) {
       const int64_t k = idx / 64;
       const int c = (int)(idx % 64), q = c / P.rp, j = c % P.rp;
       P.At[idx] = (q < P.nseg && j < P.r) ? P.A[q][(int64_t)j * P.K + k] : zero;
@@ -773,31 +798,75 @@ static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 }  // namespace ldn
 
 // ---------------------------------------------------------------- launch helpers
-template <int MODE>
-static lsq_status launch_pair(const Maps& maps, const Params& p, cudaStream_t stream) {
+template <int MODE, int H>
+static lsq_status launch_pair_h(const Maps& maps, const Params& p, int ncl, cudaStream_t stream) {
+  nf4_pair_kernel<MODE, H><<<2 * ncl, NTHREADS, PCfg<H>::SMEM_BYTES, stream>>>(maps, p);
+  LSQ_LAUNCH_CHECK("nf4_pair_kernel");
+  return LSQ_OK;
+}
+
+// Pair clusters that fit on the GPU at once (74 on 148 SMs), queried once per device.
+static lsq_status max_pair_clusters(int* out) {
   static int max_clusters[64] = {0};
   int dev = 0;
   LSQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(LSQ_EUNSUPPORTED, "nf4 GEMM: device %d out of range", dev);
   if (!max_clusters[dev]) {
-    LSQ_CUDA_TRY(
-        cudaFuncSetAttribute(nf4_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(nf4_pair_kernel<FWD, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PCfg<1>::SMEM_BYTES));
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(nf4_pair_kernel<DX, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PCfg<1>::SMEM_BYTES));
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(nf4_pair_kernel<FWD, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PCfg<2>::SMEM_BYTES));
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(nf4_pair_kernel<DX, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PCfg<2>::SMEM_BYTES));
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(2 * num_sms());
     cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = PCfg<1>::SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, nf4_pair_kernel<MODE>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, nf4_pair_kernel<FWD, 1>, &cfg) != cudaSuccess || n < 1) {
       (void)cudaGetLastError();
       n = num_sms() / 2;
     }
     max_clusters[dev] = n;
   }
-  const int ncl = std::min(p.tiles, max_clusters[dev]);
-  nf4_pair_kernel<MODE><<<2 * ncl, NTHREADS, SMEM_BYTES, stream>>>(maps, p);
-  LSQ_LAUNCH_CHECK("nf4_pair_kernel");
+  *out = max_clusters[dev];
   return LSQ_OK;
+}
+
+// Rows per pair tile: 512 (H = 2) halves the NF4 decode work per FLOP but
+// leaves no second accumulator for the epilogue to overlap; 256 (H = 1) keeps
+// the overlap.  Pick the one with fewer rounds of work per cluster, an H = 2
+// tile costing 1.25 times an H = 1 tile (measured on B200 at the 8B shapes:
+// 1.4-1.7x the TFLOP/s of H = 1 at 2048 rows); LSQ_NF4_TILE_ROWS=256|512
+// overrides.
+template <int MODE>
+static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, cudaStream_t stream) {
+  int ncl_max = 0;
+  lsq_status st = max_pair_clusters(&ncl_max);
+  if (st != LSQ_OK) return st;
+  int64_t best = -1;
+  int hbest = 1;
+  for (int h = 1; h <= 2; ++h) {
+    const int64_t tiles = (int64_t)((p.M + BT * h - 1) / (BT * h)) * ntiles_n;
+    const int64_t rounds = (tiles + ncl_max - 1) / ncl_max;
+    const int64_t cost = rounds * (h == 1 ? 4 : 5);
+    if (best < 0 || cost < best) {
+      best = cost;
+      hbest = h;
+    }
+  }
+  if (const char* e = getenv("LSQ_NF4_TILE_ROWS")) {
+    const int rows = atoi(e);
+    if (rows == 256) hbest = 1;
+    if (rows == 512) hbest = 2;
+  }
+  p.mtiles = (p.M + BT * hbest - 1) / (BT * hbest);
+  p.tiles = p.mtiles * ntiles_n;
+  const int ncl = std::min(p.tiles, ncl_max);
+  return hbest == 2 ? launch_pair_h<MODE, 2>(maps, p, ncl, stream) : launch_pair_h<MODE, 1>(maps, p, ncl, stream);
 }
 
 static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int maxsplits, cudaStream_t stream) {
@@ -828,7 +897,7 @@ static lsq_status launch_pad(const ldn::Pad& P, int64_t most, cudaStream_t strea
   int64_t g = (most + 255) / 256;
   if (g > 512) g = 512;
   if (g < 1) g = 1;
-  ldn::lora_pad<<<dim3((unsigned)g, P.dx ? P.nseg + 1 : P.nseg), 256, 0, stream>>>(P);
+  ldn::lora_pad<<<dim3((unsigned)g, P.dx ? 2 * P.nseg + 1 : P.nseg), 256, 0, stream>>>(P);
   LSQ_LAUNCH_CHECK("lora_pad");
   return LSQ_OK;
 }
@@ -898,7 +967,7 @@ static FwdPlan fwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, in
 // ---- backward rank-r part: G fp32 | s*G bf16 [M, 64] | A^T side by side [K, 64] | B_q^T [rp, n_q] | G partials
 struct BwdPlan {
   int kbps, splits[3];
-  size_t g32, sg, at, bt[3], part[3], total;
+  size_t sg, at, bt[3], su, part[3], total;
 };
 static BwdPlan bwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
   BwdPlan b;
@@ -908,10 +977,10 @@ static BwdPlan bwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, in
   for (int i = 0; i < nseg; ++i) nkb[i] = (int)((n_out[i] + 63) / 64);
   const int mtiles = (int)((M + ldn::BM - 1) / ldn::BM);
   b.kbps = ldn::plan_kbps(nkb, nseg, mtiles);
-  b.g32 = ldn::round256((size_t)nseg * (size_t)M * (size_t)r * sizeof(float));
   b.sg = ldn::round256((size_t)M * 64 * 2);
   b.at = ldn::round256((size_t)K * 64 * 2);
-  b.total = b.g32 + b.sg + b.at;
+  b.su = b.sg;
+  b.total = b.sg + b.at + (size_t)nseg * b.su;
   for (int i = 0; i < nseg; ++i) {
     b.splits[i] = (nkb[i] + b.kbps - 1) / b.kbps;
     b.bt[i] = ldn::round256((size_t)rp * (size_t)n_out[i] * 2);
@@ -925,20 +994,19 @@ size_t bwd_rank_bytes(int nseg, int64_t M, int64_t K, const int64_t* n_out, int 
   return bwd_plan(nseg, M, K, n_out, r).total;
 }
 
-// G = dY B per segment (fp32 into g_out[q], s*G bf16 into the workspace) and
-// the dX GEMM's LoRA-block operands; ws starts with the layout of bwd_plan.
-// Returns the bf16 s*G and A^T pointers through sg / at.
+// s*G = s dY B of every segment side by side in bf16 [M, 64] (the dX GEMM's
+// LoRA block and dA's operand), s*U of each segment in bf16 [M, 64] (dB's
+// operand), and A^T of every segment side by side [K, 64]; ws starts with the
+// layout of bwd_plan.  The bf16 pointers come back through sg / su / at.
 lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const void* const* A,
-                         const void* const* B, int r, float s, char* ws, float** g_out, __nv_bfloat16** sg,
-                         __nv_bfloat16** at, cudaStream_t stream) {
+                         const void* const* B, const float* const* U, int r, float s, char* ws, __nv_bfloat16** sg,
+                         __nv_bfloat16** su, __nv_bfloat16** at, cudaStream_t stream) {
   const int64_t K = W[0].k_in;
   const int rp = rpad(r);
   int64_t n_out[3];
   for (int i = 0; i < nseg; ++i) n_out[i] = W[i].n_out;
   const BwdPlan b = bwd_plan(nseg, M, K, n_out, r);
   char* cur = ws;
-  for (int i = 0; i < nseg; ++i) g_out[i] = reinterpret_cast<float*>(cur) + (size_t)i * M * r;
-  cur += b.g32;
   *sg = reinterpret_cast<__nv_bfloat16*>(cur);
   cur += b.sg;
   *at = reinterpret_cast<__nv_bfloat16*>(cur);
@@ -948,6 +1016,10 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   for (int i = 0; i < nseg; ++i) {
     bt[i] = reinterpret_cast<__nv_bfloat16*>(cur);
     cur += b.bt[i];
+  }
+  for (int i = 0; i < nseg; ++i) {
+    su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+    cur += b.su;
   }
   for (int i = 0; i < nseg; ++i) {
     part[i] = reinterpret_cast<float*>(cur);
@@ -960,12 +1032,17 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   for (int i = 0; i < nseg; ++i) {
     P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
     P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+    P.U[i] = U[i];
     P.Bt[i] = bt[i];
+    P.SU[i] = su[i];
     P.n[i] = n_out[i];
     most = std::max<int64_t>(most, (int64_t)rp * n_out[i]);
   }
+  most = std::max<int64_t>(most, M * 64);
   P.At = *at;
   P.K = K;
+  P.M = M;
+  P.s = s;
   P.nseg = nseg;
   P.r = r;
   P.rp = rp;
@@ -1000,7 +1077,6 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
     R.part[i] = part[i];
     R.splits[i] = b.splits[i];
     R.np[i] = rp;
-    R.out32[i] = g_out[i];
   }
   R.out16[0] = *sg;
   R.dx = 1;
@@ -1044,9 +1120,7 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
     if ((st = tmap_act(&maps.lb[0], at, 64, K, BNC)) != LSQ_OK) return st;
   }
   p.nkb = blocks;
-  p.mtiles = (int)((M + BT - 1) / BT);
-  p.tiles = p.mtiles * (int)((K + BT - 1) / BT);
-  return launch_pair<DX>(maps, p, stream);
+  return launch_pair<DX>(maps, p, (int)((K + BT - 1) / BT), stream);
 }
 
 }  // namespace tc
@@ -1114,8 +1188,6 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
                              BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
   }
-  p.mtiles = (int)((M + BT - 1) / BT);
-  p.tiles = p.mtiles * tiles_n;
 
   if (r > 0) {
     // workspace: s*U per segment | padded B per segment | U partials
@@ -1188,7 +1260,7 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
       if ((st = tmap_act(&maps.lb[i], bpad[i], 64, ns[i], BNC)) != LSQ_OK) return st;
     }
   }
-  return launch_pair<FWD>(maps, p, cs);
+  return launch_pair<FWD>(maps, p, tiles_n, cs);
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A,

@@ -1,14 +1,15 @@
 // Backward of the fused NF4-LoRA linear:
-//   G_seg = dY_seg B_seg                                 (split-K tensor-core kernel, gemm_nf4.cu)
-//   dX = sum_seg dY_seg deq(W_seg) + s G_seg A_seg       (CTA-pair tensor-core kernel, gemm_nf4.cu)
-//   dB_seg = s dY_seg^T U_seg,  dA_seg = s G_seg^T X      (here)
-// dA and dB are skinny products (r <= 64 columns) reduced over the M token
-// rows, i.e. HBM-bound reads of dY and X.  Deterministic two-stage reduction:
-// stage 1 gives each CTA a 256-column panel and a chunk of rows (row tiles of
-// P and Q double-buffered through shared memory with cp.async) and writes fp32
-// partial sums; stage 2 adds the partials of each output in a fixed order.
-// No atomics, so results are bit-identical run to run.  Every reduction of one
-// backward call (dA and dB of up to three linears) shares one launch per stage.
+//   s*G = s [dY_seg B_seg]                      (split-K tensor-core kernel, gemm_nf4.cu)
+//   dX = sum_seg dY_seg deq(W_seg) + (s G) A    (SM-pair tensor-core kernel, gemm_nf4.cu)
+//   dA_seg = (s G_seg)^T X,  dB_seg = dY_seg^T (s U_seg)      (here)
+// dA of every segment is one product X^T [s G_1 | s G_2 | ...] with N = 64
+// columns (the segments' ranks side by side, zero-padded), dB of segment q is
+// dY_q^T (s U_q) with N = 64: tensor-core GEMMs over the M token rows, both
+// operands read "MN-major" straight from their row-major tensors by TMA.  The
+// token range is split across CTAs; a second kernel adds the fp32 partials in
+// a fixed order (no atomics, results bit-identical run to run) and writes the
+// gradients in their own layouts (dA [r, k_in], dB [n_out, r]), overwriting or
+// adding.  s*G and s*U are bf16, the tensor cores' input type.
 #include <algorithm>
 
 #include "common.cuh"
@@ -17,186 +18,273 @@
 namespace lsq {
 namespace lg {
 
-constexpr int PANEL = 256;      // columns per CTA (4 per thread)
-constexpr int TR = 16;          // rows per shared-memory tile
-constexpr int THREADS = 256;
+constexpr int BM = 128;    // output rows per CTA (k for dA, n for dB)
+constexpr int BN = 64;     // output columns (ranks, zero-padded)
+constexpr int BKT = 64;    // token rows per stage
+constexpr int NST = 4;
+constexpr int A_BYTES = BM * BKT * 2;  // two 64-row MN chunks, 16 KB
+constexpr int B_BYTES = BN * BKT * 2;  // 8 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + NST * A_BYTES;
+constexpr int OFF_BAR = OFF_B + NST * B_BYTES;
+constexpr int NBAR = 2 * NST + 1;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int NTHREADS = 192;
 constexpr int TARGET_CTAS = 296;
-constexpr int MAXRED = 6;
+constexpr int MAXP = 4;  // dA + up to three dB
 
-struct Red {
-  const __nv_bfloat16* P;  // [M, C]
-  const float* Q;          // [M, r]
-  float* out;              // [C, r] or, transposed, [r, C]
-  float* part;             // [chunks, C, r]
-  int64_t C;
-  int64_t mchunk;          // rows per chunk (multiple of TR)
-  int chunks, panels, transpose;
+struct Prob {
+  float* part;  // [splits][rows][64]
+  int rows;     // k_in (dA) or n_out of the segment (dB)
+  int first;    // first 128-row tile of this problem in the grid
+};
+struct Params {
+  Prob pr[MAXP];
+  int nprob, M, kbps, splits;
+};
+struct Maps {
+  CUtensorMap a[MAXP];  // token-major activation side: x [M, k_in] or dy_q [M, n_q] (box 64 x 64 rows)
+  CUtensorMap b[MAXP];  // token-major rank side: s*G or s*U_q [M, 64] (box 64 x 64 rows)
 };
 
-struct RedSet {
-  Red red[MAXRED];
-  int n;
-  int64_t M;
-  int r, accumulate;
-  float s;
-};
+__global__ void __launch_bounds__(NTHREADS, 1) lora_grad_kernel(const __grid_constant__ Maps maps,
+                                                                const __grid_constant__ Params p) {
+  int pi = 0;
+  while (pi + 1 < p.nprob && (int)blockIdx.x >= p.pr[pi + 1].first) ++pi;
+  const Prob& P = p.pr[pi];
+  const int r0 = ((int)blockIdx.x - P.first) * BM;
+  const int split = blockIdx.y;
+  const int nblk = (p.M + BKT - 1) / BKT;
+  const int kb0 = split * p.kbps;
+  const int nk = min(nblk, kb0 + p.kbps) - kb0;  // >= 1: splits = ceil(nblk / kbps)
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const uint32_t d = smem_u32(dst);
-  const int sz = valid ? 16 : 0;  // 0: fill with zeros
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(sz) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + NST;
+  uint64_t* done = empty + NST;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-// stage 1: blockIdx.x = panel (+ offsets of earlier reductions), blockIdx.y = row chunk.
-// Thread (cg, jg): columns c0 + 4 cg .. + 3, ranks j in [jg*jq, jg*jq + jq), jq = ceil(r/4);
-// per row it reads 4 bf16 of P (one 8-byte load) and its jq values of Q
-// (16-byte loads, the same address for the whole warp) for 4*jq FMAs.
-template <int JQ>
-__device__ __forceinline__ void skinny_body(const Red& R, int64_t M, int r, int blocky, int px,
-                                            __nv_bfloat16 (*sP)[TR][PANEL], float (*sQ)[TR][64]) {
-  const int64_t C = R.C;
-  const int64_t c0 = (int64_t)px * PANEL;
-  const int64_t mb0 = (int64_t)blocky * R.mchunk;
-  const int64_t mb1 = mb0 + R.mchunk < M ? mb0 + R.mchunk : M;
-  const int tid = threadIdx.x;
-  const int cg = tid & 63, jg = tid >> 6;
-  float acc[4][JQ];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int q = 0; q < JQ; ++q) acc[a][q] = 0.0f;
-
-  auto load = [&](int buf, int64_t mb) {
-    // P: TR rows x 256 columns = 512 chunks of 16 bytes (2 per thread)
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int idx = tid + u * THREADS;
-      const int row = idx >> 5, ch = idx & 31;
-      const int64_t m = mb + row, c = c0 + ch * 8;
-      const bool v = m < mb1 && c < C;
-      cp_async16(&sP[buf][row][ch * 8], v ? (const void*)(R.P + m * C + c) : (const void*)R.P, v);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    if ((r & 3) == 0) {
-      const int per = r / 4;
-      for (int idx = tid; idx < TR * per; idx += THREADS) {
-        const int row = idx / per, ch = idx % per;
-        const int64_t m = mb + row;
-        const bool v = m < mb1;
-        cp_async16(&sQ[buf][row][ch * 4], v ? (const void*)(R.Q + m * r + ch * 4) : (const void*)R.Q, v);
-      }
-    } else {
-      for (int idx = tid; idx < TR * r; idx += THREADS) {
-        const int row = idx / r, j = idx % r;
-        const int64_t m = mb + row;
-        sQ[buf][row][j] = m < mb1 ? R.Q[m * r + j] : 0.0f;
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % NST;
+        const uint32_t ph = (uint32_t)(i / NST) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, 451)) break;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES));
+        const int y = (kb0 + i) * BKT;
+        uint8_t* a = smem + OFF_A + s * A_BYTES;
+        tma_load_2d(a, &maps.a[pi], &full[s], r0, y);
+        tma_load_2d(a + A_BYTES / 2, &maps.a[pi], &full[s], r0 + 64, y);
+        tma_load_2d(smem + OFF_B + s * B_BYTES, &maps.b[pi], &full[s], 0, y);
       }
     }
-    cp_async_commit();
-  };
-
-  int buf = 0;
-  if (mb0 < mb1) load(0, mb0);
-  for (int64_t mb = mb0; mb < mb1; mb += TR) {
-    const bool more = mb + TR < mb1;
-    if (more) load(buf ^ 1, mb + TR);
-    if (more) cp_async_wait<1>();
-    else cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll 4
-    for (int row = 0; row < TR; ++row) {
-      const uint2 pp = *reinterpret_cast<const uint2*>(&sP[buf][row][cg * 4]);
-      const float p[4] = {bf16lo(pp.x), bf16hi(pp.x), bf16lo(pp.y), bf16hi(pp.y)};
-      float qv[JQ];
-      const float* qr = &sQ[buf][row][jg * JQ];
-      if (JQ % 4 == 0) {
-#pragma unroll
-        for (int q = 0; q < JQ; q += 4) {
-          const float4 f = *reinterpret_cast<const float4*>(qr + q);
-          qv[q] = f.x;
-          qv[q + 1] = f.y;
-          qv[q + 2] = f.z;
-          qv[q + 3] = f.w;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(BM, BN, 1, 1);  // both operands MN-major (contiguous along rows / ranks)
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % NST;
+        const uint32_t ph = (uint32_t)(i / NST) & 1u;
+        if (!mbar_wait(&full[s], ph, 551)) {
+          ok = false;
+          break;
         }
-      } else {
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + OFF_A + s * A_BYTES);
+        const uint32_t b = smem_u32(smem + OFF_B + s * B_BYTES);
 #pragma unroll
-        for (int q = 0; q < JQ; ++q) qv[q] = qr[q];
+        for (int kk = 0; kk < BKT / 16; ++kk)  // 16 tokens = 16 rows of 128 bytes
+          tc_mma(tmem, smem_desc(a + kk * 2048, A_BYTES / 2, 1024, 2), smem_desc(b + kk * 2048, B_BYTES, 1024, 2),
+                 id, (i | kk) != 0);
+        tc_commit(&empty[s]);
       }
+      tc_commit(done);
+      if (!ok) mbar_wait(done, 0, 552);
+    }
+  } else {
+    const int qd = warp & 3;
+    const int row = r0 + qd * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    if (__all_sync(0xffffffffu, mbar_wait(done, 0, 751))) {
+      tc_fence_after();
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), v);
+        tc_wait_ld();
+        if (row < P.rows) {
+          float4* dst = reinterpret_cast<float4*>(P.part + ((int64_t)split * P.rows + row) * BN + c * 32);
 #pragma unroll
-        for (int q = 0; q < JQ; ++q) acc[a][q] = fmaf(p[a], qv[q], acc[a][q]);
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// Adds the splits (ascending) and writes the gradients.
+//   dA (problem 0): blocks of 32 k-rows; dA_q[j][k] = sum part[k][q*rp + j],
+//                   transposed through shared memory so both sides coalesce
+//   dB_q (problem q + 1): dB_q[n][j] = sum part[n][j]
+struct Red {
+  const float* part[MAXP];
+  int rows[MAXP];
+  int blocks[MAXP];  // reduce blocks of each problem
+  float* dA[3];
+  float* dB[3];
+  int nseg, r, rp, splits, accumulate;
+};
+
+__global__ void __launch_bounds__(256) lora_grad_reduce(const __grid_constant__ Red R) {
+  __shared__ float tile[32][65];
+  int pi = 0, b = blockIdx.x;
+  while (b >= R.blocks[pi]) {
+    b -= R.blocks[pi];
+    ++pi;
+  }
+  const int rows = R.rows[pi];
+  const float* part = R.part[pi];
+  if (pi == 0) {
+    const int k0 = b * 32;
+    for (int e = threadIdx.x; e < 32 * BN; e += 256) {
+      const int rl = e / BN, c = e % BN, k = k0 + rl;
+      float sum = 0.0f;
+      if (k < rows)
+        for (int sp = 0; sp < R.splits; ++sp) sum += part[((int64_t)sp * rows + k) * BN + c];
+      tile[rl][c] = sum;
     }
     __syncthreads();
-    buf ^= 1;
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int64_t c = c0 + cg * 4 + a;
-    if (c >= C) continue;
-#pragma unroll
-    for (int q = 0; q < JQ; ++q) {
-      const int j = jg * JQ + q;
-      if (j < r) R.part[((int64_t)blocky * C + c) * r + j] = acc[a][q];
+    const int live = R.nseg * R.r;
+    for (int e = threadIdx.x; e < 32 * live; e += 256) {
+      const int kl = e % 32, qj = e / 32, q = qj / R.r, j = qj % R.r, k = k0 + kl;
+      if (k >= rows) continue;
+      float* dst = R.dA[q] + (int64_t)j * rows + k;
+      const float v = tile[kl][q * R.rp + j];
+      *dst = R.accumulate ? *dst + v : v;
+    }
+  } else {
+    const int q = pi - 1;
+    const int64_t n_el = (int64_t)rows * R.r;
+    for (int64_t e = (int64_t)b * 256 + threadIdx.x; e < n_el && e < ((int64_t)b + 1) * 256; e += 256) {
+      const int64_t n = e / R.r;
+      const int j = (int)(e % R.r);
+      float sum = 0.0f;
+      for (int sp = 0; sp < R.splits; ++sp) sum += part[((int64_t)sp * rows + n) * BN + j];
+      float* dst = R.dB[q] + e;
+      *dst = R.accumulate ? *dst + sum : sum;
     }
   }
 }
 
-__global__ void __launch_bounds__(THREADS) skinny_partial(const __grid_constant__ RedSet rs) {
-  __shared__ __align__(16) __nv_bfloat16 sP[2][TR][PANEL];
-  __shared__ __align__(16) float sQ[2][TR][64];
-  int rid = 0, px = blockIdx.x;
-  while (rid + 1 < rs.n && px >= rs.red[rid].panels) {
-    px -= rs.red[rid].panels;
-    ++rid;
+struct Plan {
+  int kbps, splits, tiles;
+  size_t part[MAXP], total;
+};
+static Plan plan(int nseg, int64_t M, int64_t K, const int64_t* n_out) {
+  Plan pl;
+  memset(&pl, 0, sizeof(pl));
+  const int64_t rows[MAXP] = {K, nseg > 0 ? n_out[0] : 0, nseg > 1 ? n_out[1] : 0, nseg > 2 ? n_out[2] : 0};
+  for (int i = 0; i <= nseg; ++i) pl.tiles += (int)((rows[i] + BM - 1) / BM);
+  const int nblk = (int)((M + BKT - 1) / BKT);
+  int want = (TARGET_CTAS + pl.tiles - 1) / pl.tiles;
+  want = std::max(1, std::min(want, std::min(4, nblk)));
+  pl.kbps = (nblk + want - 1) / want;
+  pl.splits = (nblk + pl.kbps - 1) / pl.kbps;
+  for (int i = 0; i <= nseg; ++i) {
+    pl.part[i] = ((size_t)pl.splits * (size_t)rows[i] * BN * sizeof(float) + 255) / 256 * 256;
+    pl.total += pl.part[i];
   }
-  const Red& R = rs.red[rid];
-  if ((int)blockIdx.y >= R.chunks) return;
-  const int jq = (rs.r + 3) / 4;
-  if (jq <= 1) skinny_body<1>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
-  else if (jq <= 2) skinny_body<2>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
-  else if (jq <= 4) skinny_body<4>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
-  else if (jq <= 8) skinny_body<8>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
-  else skinny_body<16>(R, rs.M, rs.r, blockIdx.y, px, sP, sQ);
+  return pl;
 }
 
-// stage 2: out (+)= s * sum over chunks (ascending) of the partials
-__global__ void __launch_bounds__(256) skinny_reduce(const __grid_constant__ RedSet rs) {
-  const int rid = blockIdx.y;
-  const Red& R = rs.red[rid];
-  const int r = rs.r;
-  const int64_t n = R.C * r;
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
-    float sum = 0.0f;
-    for (int k = 0; k < R.chunks; ++k) sum += R.part[(int64_t)k * n + idx];
-    const int64_t c = idx / r, j = idx % r;
-    float* dst = R.transpose ? R.out + j * R.C + c : R.out + idx;
-    const float v = rs.s * sum;
-    *dst = rs.accumulate ? *dst + v : v;
+static lsq_status tmap_rows(CUtensorMap* m, const void* base, int64_t inner, int64_t M) {
+  return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)inner, (uint64_t)M,
+                        (uint64_t)inner * 2, 64, BKT, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// dA of every segment and dB of each: partial GEMMs, then the ordered reduction
+static lsq_status launch(int nseg, int64_t M, int64_t K, const int64_t* n_out, const void* x, const void* const* dy,
+                         const __nv_bfloat16* sg, __nv_bfloat16* const* su, float* const* dA, float* const* dB,
+                         int r, int rp, int accumulate, char* ws, cudaStream_t stream) {
+  const Plan pl = plan(nseg, M, K, n_out);
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  Params p;
+  memset(&p, 0, sizeof(p));
+  Red R;
+  memset(&R, 0, sizeof(R));
+  p.nprob = nseg + 1;
+  p.M = (int)M;
+  p.kbps = pl.kbps;
+  p.splits = pl.splits;
+  lsq_status st;
+  int first = 0;
+  char* cur = ws;
+  for (int i = 0; i <= nseg; ++i) {
+    const int64_t rows = i == 0 ? K : n_out[i - 1];
+    if ((st = tmap_rows(&maps.a[i], i == 0 ? x : dy[i - 1], rows, M)) != LSQ_OK) return st;
+    if ((st = tmap_rows(&maps.b[i], i == 0 ? (const void*)sg : (const void*)su[i - 1], 64, M)) != LSQ_OK)
+      return st;
+    Prob& pr = p.pr[i];
+    pr.part = reinterpret_cast<float*>(cur);
+    pr.rows = (int)rows;
+    pr.first = first;
+    first += (int)((rows + BM - 1) / BM);
+    cur += pl.part[i];
+    R.part[i] = pr.part;
+    R.rows[i] = (int)rows;
+    R.blocks[i] = i == 0 ? (int)((rows + 31) / 32) : (int)((rows * r + 255) / 256);
   }
+  static int configured[64] = {0};
+  int dev = 0;
+  LSQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(lora_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    configured[dev] = 1;
+  }
+  lora_grad_kernel<<<dim3(first, pl.splits), NTHREADS, SMEM_BYTES, stream>>>(maps, p);
+  LSQ_LAUNCH_CHECK("lora_grad_kernel");
+  for (int i = 0; i < nseg; ++i) {
+    R.dA[i] = dA[i];
+    R.dB[i] = dB[i];
+  }
+  R.nseg = nseg;
+  R.r = r;
+  R.rp = rp;
+  R.splits = pl.splits;
+  R.accumulate = accumulate ? 1 : 0;
+  int nb = 0;
+  for (int i = 0; i <= nseg; ++i) nb += R.blocks[i];
+  lora_grad_reduce<<<nb, 256, 0, stream>>>(R);
+  LSQ_LAUNCH_CHECK("lora_grad_reduce");
+  return LSQ_OK;
 }
-
-static int64_t panels_for(int64_t C) { return (C + PANEL - 1) / PANEL; }
-
-static int64_t chunks_for(int64_t M, int64_t C) {
-  int64_t k = (TARGET_CTAS + panels_for(C) - 1) / panels_for(C);
-  const int64_t maxk = (M + TR - 1) / TR;
-  if (k > maxk) k = maxk;
-  if (k < 1) k = 1;
-  return k;
-}
-
-static int64_t mchunk_for(int64_t M, int64_t k) { return ((M + k - 1) / k + TR - 1) / TR * TR; }
-
-static size_t partial_bytes(int64_t M, int64_t C, int r) {
-  const int64_t k = chunks_for(M, C);
-  const int64_t kk = (M + mchunk_for(M, k) - 1) / mchunk_for(M, k);
-  return ((size_t)kk * (size_t)C * (size_t)r * sizeof(float) + 255) / 256 * 256;
-}
-
-static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace lg
 }  // namespace lsq
@@ -206,9 +294,7 @@ using namespace lsq;
 extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
   if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
-  size_t b = tc::bwd_rank_bytes(nseg, M, k_in, n_out, r);
-  for (int i = 0; i < nseg; ++i) b += lg::partial_bytes(M, n_out[i], r) + lg::partial_bytes(M, k_in, r);
-  return b;
+  return tc::bwd_rank_bytes(nseg, M, k_in, n_out, r) + lg::plan(nseg, M, k_in, n_out).total;
 }
 
 extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x,
@@ -245,9 +331,9 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     }
   }
   if (r == 0 && !dx) return LSQ_OK;
-  float* g[3] = {nullptr, nullptr, nullptr};
   __nv_bfloat16* sg = nullptr;
   __nv_bfloat16* at = nullptr;
+  __nv_bfloat16* su[3] = {nullptr, nullptr, nullptr};
   char* part = nullptr;
   cudaStream_t cs = (cudaStream_t)stream;
   if (r > 0) {
@@ -256,46 +342,13 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
       return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, need,
                   workspace_bytes);
     char* ws = static_cast<char*>(workspace);
-    // G = dY B (fp32 for dA, s*G in bf16 for the dX kernel) and the padded operands
-    if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, r, s, ws, g, &sg, &at, cs)) != LSQ_OK) return st;
+    // s*G = s dY B (bf16, the dX kernel's LoRA block and dA's operand), s*U, A^T
+    if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, u, r, s, ws, &sg, su, &at, cs)) != LSQ_OK) return st;
     part = ws + tc::bwd_rank_bytes(nseg, M, K, n_out, r);
   }
   if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
-  lg::RedSet rs;
-  memset(&rs, 0, sizeof(rs));
-  rs.M = M;
-  rs.r = r;
-  rs.s = s;
-  rs.accumulate = accumulate ? 1 : 0;
-  int panels = 0, maxchunks = 1;
-  int64_t maxn = 0;
-  for (int i = 0; i < nseg; ++i) {
-    for (int which = 0; which < 2; ++which) {  // dB_i = s dy_i^T U_i ; dA_i = s G_i^T x
-      lg::Red& R = rs.red[rs.n++];
-      R.P = static_cast<const __nv_bfloat16*>(which == 0 ? dy[i] : x);
-      R.Q = which == 0 ? u[i] : g[i];
-      R.out = which == 0 ? dB[i] : dA[i];
-      R.C = which == 0 ? n_out[i] : K;
-      R.transpose = which;
-      const int64_t k = lg::chunks_for(M, R.C);
-      R.mchunk = lg::mchunk_for(M, k);
-      R.chunks = (int)((M + R.mchunk - 1) / R.mchunk);
-      R.panels = (int)lg::panels_for(R.C);
-      R.part = reinterpret_cast<float*>(part);
-      part += lg::partial_bytes(M, R.C, r);
-      panels += R.panels;
-      if (R.chunks > maxchunks) maxchunks = R.chunks;
-      if (R.C * r > maxn) maxn = R.C * r;
-    }
-  }
-  lg::skinny_partial<<<dim3(panels, maxchunks), lg::THREADS, 0, cs>>>(rs);
-  LSQ_LAUNCH_CHECK("skinny_partial");
-  int64_t g2 = (maxn + 255) / 256;
-  if (g2 > 1024) g2 = 1024;
-  lg::skinny_reduce<<<dim3((unsigned)g2, rs.n), 256, 0, cs>>>(rs);
-  LSQ_LAUNCH_CHECK("skinny_reduce");
-  return LSQ_OK;
+  return lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, cs);
 }
 
 extern "C" lsq_status lsq_nf4_lora_bwd(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M,

@@ -135,7 +135,7 @@ def _check(name: str, status: int):
 # kernel launches issued by the library, counted per call on this side
 # (with a LoRA adapter the fused linear's forward is 4 kernels: operand padding,
 # the split-K rank-r product, its reduction and the main GEMM; the backward is
-# those three, the dX GEMM when dx is wanted, and the two dA/dB reduction kernels)
+# those three, the dX GEMM when dx is wanted, and the dA/dB GEMM with its reduction)
 LAUNCHES = [0]
 _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
