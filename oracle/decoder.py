@@ -136,6 +136,65 @@ def model_loss_and_grads(ids, layers, emb, lora, shape):
     return float(loss.detach()), grads
 
 
+# ---------------------------------------------------------------- preference loss (DPO)
+# The pages name DPO among the preference losses that streaming serves and say
+# the reference model is the same streamed base with the adapters switched off
+# (aiany.app listing, "How It Works (concise)"; soup-cli docs "Layer
+# Streaming", preference losses v0.72.4).  They give no formula; the reading is
+# the DPO objective of Rafailov et al. (2023, eq. 7):
+#   z_i  = beta * ((pi(y_c) - ref(y_c)) - (pi(y_r) - ref(y_r)))
+#   loss = mean_i -log sigmoid(z_i)
+# over pairs i of sequences (chosen = row 2i, rejected = row 2i+1), where pi(y)
+# and ref(y) are the summed next-token log-probabilities of a whole sequence
+# (synthetic ids have no prompt/response split, so every position t < S-1
+# counts) under the adapted model and under the same base with the LoRA path
+# off (s = 0).  beta = 0.1 (reading).
+
+DPO_BETA = 0.1
+
+
+def sequence_logprob(logits: torch.Tensor, ids: torch.Tensor) -> torch.Tensor:
+    """Summed log p(ids[b, t+1] | logits[b, t]) over t < S-1, per sequence -> [B] (fp64)."""
+    lg = logits[:, :-1, :]
+    tgt = ids[:, 1:].long()
+    logp = lg - torch.logsumexp(lg, dim=-1, keepdim=True)
+    return torch.gather(logp, -1, tgt[..., None])[..., 0].sum(dim=1)
+
+
+def dpo_loss(pi_logp: torch.Tensor, ref_logp: torch.Tensor, beta: float = DPO_BETA) -> torch.Tensor:
+    """DPO loss over pairs (rows 2i, 2i+1) = (chosen, rejected) of [2P] sequence log-probs."""
+    pc, pr = pi_logp[0::2], pi_logp[1::2]
+    rc, rr = ref_logp[0::2], ref_logp[1::2]
+    z = beta * ((pc - rc) - (pr - rr))
+    return torch.nn.functional.softplus(-z).mean()  # -log sigmoid(z) = log(1 + exp(-z))
+
+
+def model_logits(ids, layers, emb, lora, shape, s: float) -> torch.Tensor:
+    """Logits [B, S, V] of the stack with LoRA scale s (s = 0: the base alone)."""
+    h = emb["embed"][ids.long()]
+    for l, W in enumerate(layers):
+        h = decoder_layer(h, W, lora[l], shape, s)
+    h = rmsnorm(h, emb["final_norm"], shape.eps)
+    return h @ emb["lm_head"].T
+
+
+def model_dpo_loss_and_grads(ids, layers, emb, lora, shape, beta: float = DPO_BETA):
+    """-> (loss, grads, policy_logp, ref_logp); grads[l][name]["A"|"B"] = d loss / d LoRA operand."""
+    leaves = [{n: {"A": t["A"].detach().clone().requires_grad_(True),
+                   "B": t["B"].detach().clone().requires_grad_(True)} for n, t in per.items()}
+              for per in lora]
+    with torch.no_grad():
+        ref = sequence_logprob(model_logits(ids, layers, emb, lora, shape, 0.0), ids)
+    pi = sequence_logprob(model_logits(ids, layers, emb, leaves, shape, shape.s), ids)
+    loss = dpo_loss(pi, ref, beta)
+    flat = [leaves[l][n][ab] for l in range(len(leaves)) for n in leaves[l] for ab in ("A", "B")]
+    gr = torch.autograd.grad(loss, flat)
+    grads, it = [], iter(gr)
+    for per in leaves:
+        grads.append({n: {"A": next(it), "B": next(it)} for n in per})
+    return float(loss.detach()), grads, pi.detach(), ref
+
+
 def adamw(master, grad, m, v, t: int, lr: float = 2e-5, b1: float = 0.9, b2: float = 0.999,
           eps: float = 1e-8, wd: float = 0.0):
     """One AdamW step in fp64 (Loshchilov & Hutter); returns (master, m, v).
