@@ -59,6 +59,9 @@ def args_():
     p.add_argument("--no-resident", action="store_true")
     p.add_argument("--no-batch1", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--dpo", action="store_true",
+                   help="DPO over pairs of sequences with the adapter-off reference on the same streamed base")
+    p.add_argument("--beta", type=float, default=0.1)
     return p.parse_args()
 
 
@@ -176,7 +179,7 @@ def reference_arm(a):
     value = tokens / sec
     sample = (f"one full-width {shape.name} decoder layer fwd+bwd (fp64 oracle) on batch 1 x {tokens} tokens, "
               f"plus lm_head+CE on 1/32 of the vocabulary; extrapolated x{shape.n_layers} layers, x32 vocab")
-    line = {"impl": "reference", "metric": "streamed NF4-LoRA train tok/s (8B shape, seq 512)", "value": value,
+    line = {"impl": "reference", "metric": metric_name(a, shape), "value": value,
             "unit": "tok/s", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": sec * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(a, shape),
@@ -186,11 +189,27 @@ def reference_arm(a):
 
 
 def workload_config(a, shape):
+    task = (f"DPO (beta {a.beta}, {a.batch // 2} chosen/rejected pairs, reference = the base with the adapters "
+            f"off, run on each layer while it is resident)") if a.dpo else "causal-LM SFT"
+    store_gb = shape.n_layers * record_bytes(shape) / 1e9
     return {"workload": f"{shape.name} shape, NF4 (bs64, fp32 absmax) base streamed from pinned host RAM through "
                         f"{a.slots} HBM slots, grad checkpointing with re-stream, LoRA r={shape.r} on all linears, "
-                        f"AdamW",
+                        f"{task}, AdamW",
             "batch": a.batch, "seq_len": a.seq, "n_slots": a.slots, "parallelism": f"dp{a.gpus}",
-            "l2": "inputs larger than L2 (3.93 GB of layer records streamed per pass)"}
+            "l2": f"inputs larger than L2 ({store_gb:.2f} GB of layer records streamed per pass)"}
+
+
+def record_bytes(shape):
+    """Bytes of one streamed layer record: NF4 codes + fp32 absmax of the 7 linears + 2 RMSNorm gains."""
+    w = sum(n * k for n, k in shape.linear_shapes().values())
+    return w // 2 + w // 64 * 4 + 2 * shape.d * 2
+
+
+def metric_name(a, shape):
+    task = "DPO train" if a.dpo else "train"
+    short = {"llama-3.1-8b": "8B", "dense-32b": "32B", "qwen2.5-3b": "3B", "smollm2-135m": "135M"}.get(shape.name,
+                                                                                                      shape.name)
+    return f"streamed NF4-LoRA {task} tok/s ({short} shape, seq {a.seq})"
 
 
 # ---------------------------------------------------------------------------- our arm
@@ -211,8 +230,16 @@ def h2d_bandwidth(torch, nbytes=128 << 20, reps=10):
     return best
 
 
+def step_fb(tr, a):
+    """The forward/backward of one training step of the benchmarked task."""
+    if getattr(a, "dpo", False):
+        tr.forward_backward_dpo(a.beta)
+    else:
+        tr.forward_backward()
+
+
 def timed_steps(torch, dist, tr, steps, ids_list, world, instrument=False, e2e=False, host_ids=None,
-                loss_host=None):
+                loss_host=None, a=None):
     from nf4_layer_streamed_blockwise_b200 import dist as DP
     if instrument:
         tr.timeline = []
@@ -226,7 +253,7 @@ def timed_steps(torch, dist, tr, steps, ids_list, world, instrument=False, e2e=F
             tr.ids.copy_(host_ids[i % len(host_ids)].view(-1), non_blocking=True)
         else:
             tr.set_ids(ids_list[i % len(ids_list)])
-        tr.forward_backward()
+        step_fb(tr, a)
         DP.average_gradients(tr.lora.grad, world)
         tr.optimizer_step()
         if e2e:
@@ -264,7 +291,7 @@ def our_arm(a):
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
         tr.set_ids(ids_list[i % 4])
-        tr.forward_backward()
+        step_fb(tr, a)
         DP.average_gradients(tr.lora.grad, world)
         tr.optimizer_step()
     torch.cuda.synchronize()
@@ -273,7 +300,7 @@ def our_arm(a):
     L.LAUNCHES[0] = 0
     clocks = ClockSampler(local)
     clocks.start()
-    ms, timeline = timed_steps(torch, dist, tr, a.steps, ids_list, world, instrument=True)
+    ms, timeline = timed_steps(torch, dist, tr, a.steps, ids_list, world, instrument=True, a=a)
     clk = clocks.stop()
     launches = L.LAUNCHES[0]
     up1, by1, re1 = tr.stats()
@@ -312,7 +339,7 @@ def our_arm(a):
     host_ids = [t.cpu().pin_memory() for t in ids_list]
     loss_host = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(a.steps)]
     ms_e2e, _ = timed_steps(torch, dist, tr, a.steps, ids_list, world, e2e=True, host_ids=host_ids,
-                            loss_host=loss_host)
+                            loss_host=loss_host, a=a)
     e2e = {"value": world * tokens * a.steps / (ms_e2e * 1e-3), "unit": "tok/s",
            "h2d_bytes_per_step": tokens * 4 + streaming["h2d_bytes_per_step"], "d2h_bytes_per_step": 4,
            "h2d_breakdown": {"token_ids": tokens * 4, "layer_records": streaming["h2d_bytes_per_step"]},
@@ -324,10 +351,12 @@ def our_arm(a):
     if not a.no_resident:
         trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store)
         for i in range(2):
-            trr.train_step(ids_list[i % 4])
+            trr.set_ids(ids_list[i % 4])
+            step_fb(trr, a)
+            trr.optimizer_step()
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats()
-        ms_r, _ = timed_steps(torch, dist, trr, a.steps, ids_list, world)
+        ms_r, _ = timed_steps(torch, dist, trr, a.steps, ids_list, world, a=a)
         streaming["ms_per_step_resident"] = ms_r / a.steps
         streaming["exposed_copy_ms_per_step"] = max(0.0, ms_step - ms_r / a.steps)
         streaming["exposed_copy_frac"] = streaming["exposed_copy_ms_per_step"] / ms_step
@@ -336,7 +365,7 @@ def our_arm(a):
         del trr
 
     batch1 = None
-    if not a.no_batch1 and a.batch != 1:
+    if not a.no_batch1 and a.batch != 1 and not a.dpo:
         tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store)
         ids1 = [t[:1] for t in ids_list]
         for i in range(2):
@@ -357,7 +386,7 @@ def our_arm(a):
                          f"({det['head_slice_s']} s) x 32"}
 
     if rank == 0:
-        line = {"metric": "streamed NF4-LoRA train tok/s (8B shape, seq 512)", "value": value, "unit": "tok/s",
+        line = {"metric": metric_name(a, shape), "value": value, "unit": "tok/s",
                 "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded uniform token ids, random-init weights)",

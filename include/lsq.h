@@ -239,6 +239,35 @@ size_t lsq_xent_workspace_size(int64_t rows);
 lsq_status lsq_xent_fwd_bwd(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
                             float* loss, void* dlogits, void* workspace, size_t workspace_bytes,
                             lsq_cuda_stream stream);
+/* ------------------------------------------------------------------------
+ * Preference loss (DPO) on the streamed base.  The pages serve preference
+ * losses from the same streamed base, taking the base with the adapters
+ * switched off as the reference model (aiany.app listing, "How It Works
+ * (concise)"; soup-cli docs "Layer Streaming", preference losses v0.72.4).
+ * They give no formula: the reading is DPO (Rafailov et al. 2023, eq. 7)
+ * over pairs of sequences, chosen = row 2i, rejected = row 2i+1 of the batch,
+ * with whole-sequence summed next-token log-probabilities.
+ *
+ * lsq_seq_logprob: seq_logp[b] = sum over t < seq-1 of log softmax(logits[b, t])[ids[b, t+1]];
+ *   logits fp32 [batch*seq, V], ids int32 [batch*seq] (device); row_lse fp32
+ *   [batch*seq] receives each row's log-sum-exp (for the backward); seq_logp
+ *   fp32 [batch]; workspace lsq_seq_logprob_workspace_size(batch*seq) bytes.
+ *   Fixed-order reductions (deterministic).
+ * lsq_dpo_loss: z_i = beta ((pi[2i] - ref[2i]) - (pi[2i+1] - ref[2i+1])),
+ *   loss (device fp32 scalar) = mean_i log(1 + exp(-z_i)); dseq fp32 [2 npairs]
+ *   = d loss / d pi.  All pointers device memory.
+ * lsq_seq_logprob_bwd: dlogits bf16 [batch*seq, V] = dseq[b] * (onehot(ids[b, t+1])
+ *   - softmax(logits[b, t])), zero on each sequence's last row (the gradient of
+ *   the loss through seq_logp). */
+size_t lsq_seq_logprob_workspace_size(int64_t rows);
+lsq_status lsq_seq_logprob(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
+                           float* row_lse, float* seq_logp, void* workspace, size_t workspace_bytes,
+                           lsq_cuda_stream stream);
+lsq_status lsq_dpo_loss(const float* policy_logp, const float* ref_logp, int32_t npairs, float beta, float* loss,
+                        float* dseq, lsq_cuda_stream stream);
+lsq_status lsq_seq_logprob_bwd(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
+                               const float* row_lse, const float* dseq, void* dlogits, lsq_cuda_stream stream);
+
 /* AdamW on n fp32 masters p with grads g and moments m, v (all device fp32);
  * writes the bf16 operand copies p_bf16 (device, may be NULL).  step >= 1. */
 lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int32_t step,

@@ -16,9 +16,9 @@
 // the next.  Six shared-memory stages of 64 contraction steps.
 //
 // The rank-r products stay off the main loop: a split-K tcgen05 kernel
-// (lora_down_kernel) computes U = X A^T (or G = dY B) and a reduction writes it
-// in fp32 (kept for the backward) and as s*U (s*G) in bf16, zero-padded to 64
-// columns.  The main loop then runs (s U) B^T (or (s G) A) as one extra
+// (lora_down_kernel) computes U = X A^T (or G = dY B), reduces its splits
+// inside a thread-block cluster and writes U in fp32 (kept for the backward)
+// and s*U (s*G) in bf16, zero-padded to 64 columns.  The main loop then runs (s U) B^T (or (s G) A) as one extra
 // contraction block of width 64 whose two operands are TMA-loaded like the
 // activation tile, so the output is still rounded to bf16 once.
 //
@@ -554,10 +554,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 // ================================================================ rank-r products: U = X A^T, G = dY B
-// Split-K tcgen05 GEMM with a narrow N: CTA (m tile, split, problem) multiplies
-// 128 activation rows by the problem's np = nsub * rp weight-side rows over
-// its share of the contraction, and writes fp32 partial sums; a second kernel
-// adds the splits in a fixed order.
+// Split-K tcgen05 GEMM with a narrow N, reduced inside a thread-block cluster:
+// the S CTAs of a cluster (S <= 8) take one 128-row tile of one problem and
+// split its contraction; each parks its fp32 partial [128 x np] in its own
+// shared memory, then rank k adds the S partials of rows [k*128/S, ...) in
+// rank order through distributed shared memory (a fixed order: results do not
+// depend on timing) and writes the outputs:
+//   FWD (one problem, segment q in columns q*rp ..): u_out[q] [M, r] fp32 (if
+//        given) and s*U of segment q as bf16 [M, 64], zero in columns >= r;
+//        meanwhile the epilogue warps of every CTA, idle until their MMAs
+//        finish, write the padded copies of B that the main GEMM reads.
+//   DX  (problem q = segment q): s*G as bf16 [M, 64] with segment q in columns
+//        q*rp .. q*rp + rp - 1 and zeros from nseg*rp on.
 namespace ldn {
 constexpr int BM = 128, BK = 64, NST = 4, NMAX = 192;
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB
@@ -570,31 +578,48 @@ constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr int NTHREADS = 192;
 constexpr int TARGET_CTAS = 296;
+constexpr int MAX_SPLITS = 8;  // portable cluster size
+static_assert(BM * (NMAX + 4) * 4 <= OFF_BAR, "partial tile must fit the stage buffers");
 
 struct Prob {
-  float* part;    // [splits][M][np]
-  int nkb;        // contraction blocks of 64 (the last may be partial: zero-filled)
-  int splits;     // split k covers blocks [k*kbps, min(nkb, (k+1)*kbps))
-  int nsub;       // weight-side maps wl[first .. first + nsub), rp rows each
+  int nkb;   // contraction blocks of 64 (the last may be partial: zero-filled)
+  int kbps;  // blocks per split: split k covers [k*kbps, min(nkb, (k+1)*kbps))
+  int nsub;  // weight-side maps wl[first .. first + nsub), rp rows each
   int first;
 };
 struct Params {
   Prob pr[3];
-  int nprob, M, rp, kbps;
+  int nprob, M, r, rp, dx, nseg;
+  float s;
+  float* out32[3];          // FWD: U of each segment (or null)
+  __nv_bfloat16* out16[3];  // FWD: s*U of each segment [M, 64]; DX: s*G [M, 64] in out16[0]
+  const __nv_bfloat16* B[3];  // FWD: LoRA B of each segment [n, r] ...
+  __nv_bfloat16* Bpad[3];     // ... and its padded copy [n, 64]
+  int64_t nB[3];
 };
 struct Maps {
   CUtensorMap in[3];  // activation side of each problem [M, Kr] (box 64 x 128 rows, 128B swizzle)
   CUtensorMap wl[3];  // weight side [rows, Kr] (box 64 x rp rows; rows past the tensor read as zero)
 };
 
+// plain load from a cluster peer's shared memory (after a cluster barrier: the
+// compiler may batch these, so a thread's loads from all peers overlap)
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t caddr) {
+  float4 v;
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(caddr));
+  return v;
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_constant__ Maps maps,
                                                                 const __grid_constant__ Params p) {
-  const Prob& P = p.pr[blockIdx.z];
-  const int split = blockIdx.y;
-  if (split >= P.splits) return;
-  const int kb0 = split * p.kbps;
-  const int nk = min(P.nkb, kb0 + p.kbps) - kb0;
+  const int pi = blockIdx.z;
+  const Prob& P = p.pr[pi];
+  const int split = blockIdx.y;  // rank in the cluster (the cluster spans y)
+  const int S = gridDim.y;
+  const int kb0 = split * P.kbps;
+  const int nk = max(0, min(P.nkb, kb0 + P.kbps) - kb0);
   const int np = P.nsub * p.rp;
+  const int ldp = np + 4;  // row stride of the parked partial (floats): 16-byte rows, no bank conflicts
   const int m0 = blockIdx.x * BM;
 
   extern __shared__ uint8_t smem_raw[];
@@ -603,6 +628,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
   uint64_t* empty = full + NST;
   uint64_t* done = empty + NST;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  float* park = reinterpret_cast<float*>(smem);  // [128][ldp], over the stage buffers once the MMAs are done
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = np <= 32 ? 32u : np <= 64 ? 64u : np <= 128 ? 128u : 256u;
 
@@ -631,7 +657,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
         if (!mbar_wait(&empty[s], ph ^ 1u, 441)) break;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + np * 128));
         const int x = (kb0 + i) * BK;
-        tma_load_2d(smem + OFF_A + s * A_BYTES, &maps.in[blockIdx.z], &full[s], x, m0);
+        tma_load_2d(smem + OFF_A + s * A_BYTES, &maps.in[pi], &full[s], x, m0);
         for (int q = 0; q < P.nsub; ++q)
           tma_load_2d(smem + OFF_B + s * B_BYTES + q * p.rp * 128, &maps.wl[P.first + q], &full[s], x, 0);
       }
@@ -656,113 +682,141 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
                  (i | kk) != 0);
         tc_commit(&empty[s]);
       }
-      tc_commit(done);  // also the drain when the loop stopped early
+      tc_commit(done);  // also the drain when the loop stopped early; completes at once if nk == 0
       if (!ok) mbar_wait(done, 0, 542);
     }
   } else {
     // epilogue warps 2-5: TMEM lane quarter = warp % 4
     const int qd = warp & 3;
-    const int m = m0 + qd * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-    if (__all_sync(0xffffffffu, mbar_wait(done, 0, 741))) {
-      tc_fence_after();
-      for (int c = 0; c < np / 16; ++c) {
-        float v[16];
-        tmem_ld16(tmem + lane_base + (uint32_t)(c * 16), v);
-        tc_wait_ld();
-        if (m < p.M) {
-          float4* dst = reinterpret_cast<float4*>(P.part + ((int64_t)split * p.M + m) * np + c * 16);
-          dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-          dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-          dst[2] = make_float4(v[8], v[9], v[10], v[11]);
-          dst[3] = make_float4(v[12], v[13], v[14], v[15]);
+    const int e = qd * 32 + lane;  // row of the tile
+    if (!p.dx) {
+      // padded copies of B, spread over every CTA of the grid while its MMAs run
+      const int64_t cta = ((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+      const int64_t stride = (int64_t)gridDim.x * gridDim.y * gridDim.z * 128;
+      for (int q = 0; q < p.nseg; ++q) {
+        const int64_t total = p.nB[q] * 8;  // 16-byte chunks of Bpad[q]
+        for (int64_t c = cta * 128 + (threadIdx.x - 64); c < total; c += stride) {
+          const int64_t n = c >> 3;
+          const int j0 = (int)(c & 7) * 8;
+          float v[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) v[t] = j0 + t < p.r ? __bfloat162float(p.B[q][n * p.r + j0 + t]) : 0.0f;
+          *reinterpret_cast<uint4*>(p.Bpad[q] + n * 64 + j0) =
+              make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                         pack_bf16x2(v[6], v[7]));
         }
       }
     }
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, 741));
+    if (ok && nk > 0) tc_fence_after();
+    for (int c = 0; c < np / 16; ++c) {
+      float v[16];
+      if (ok && nk > 0) {
+        tmem_ld16(tmem + lane_base + (uint32_t)(c * 16), v);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) v[t] = 0.0f;
+      }
+      float4* dst = reinterpret_cast<float4*>(park + e * ldp + c * 16);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) dst[t] = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // every CTA's partial is parked
+  if (warp >= 2) {
+    // rank k adds the cluster's partials for its own slice of rows, in rank order
+    const int per = (BM + S - 1) / S, r0 = split * per, r1 = min(BM, r0 + per);
+    const int nch = np / 8;  // 8-column chunks per row
+    const int t = threadIdx.x - 64;
+    for (int it = t; it < (r1 - r0) * nch; it += 128) {
+      const int e = r0 + it / nch, c = (it % nch) * 8;
+      const int64_t m = m0 + e;
+      if (m >= p.M) continue;
+      const uint32_t local = smem_u32(park + e * ldp + c);
+      float4 x0[MAX_SPLITS], x1[MAX_SPLITS];
+#pragma unroll
+      for (int k = 0; k < MAX_SPLITS; ++k) {
+        if (k < S) {
+          uint32_t a;
+          asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(k));
+          x0[k] = ld_dsmem_f4(a);
+          x1[k] = ld_dsmem_f4(a + 16);
+        }
+      }
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < MAX_SPLITS; ++k) {
+        if (k < S) {
+          v[0] += x0[k].x; v[1] += x0[k].y; v[2] += x0[k].z; v[3] += x0[k].w;
+          v[4] += x1[k].x; v[5] += x1[k].y; v[6] += x1[k].z; v[7] += x1[k].w;
+        }
+      }
+      const int q = c / p.rp, j0 = c % p.rp;  // segment and rank of the first column
+      const uint4 o = make_uint4(pack_bf16x2(p.s * v[0], p.s * v[1]), pack_bf16x2(p.s * v[2], p.s * v[3]),
+                                 pack_bf16x2(p.s * v[4], p.s * v[5]), pack_bf16x2(p.s * v[6], p.s * v[7]));
+      if (p.dx) {
+        *reinterpret_cast<uint4*>(p.out16[0] + m * 64 + pi * p.rp + j0) = o;
+      } else {
+        *reinterpret_cast<uint4*>(p.out16[q] + m * 64 + j0) = o;
+        if (p.out32[q])
+          for (int u = 0; u < 8; ++u)
+            if (j0 + u < p.r) p.out32[q][m * p.r + j0 + u] = v[u];
+      }
+    }
+    // zero padding of the bf16 operands for the same rows
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int e = r0 + t; e < r1; e += 128) {
+      const int64_t m = m0 + e;
+      if (m >= p.M) continue;
+      if (p.dx) {
+        if (pi == 0)
+          for (int c = p.nseg * p.rp; c < 64; c += 8) *reinterpret_cast<uint4*>(p.out16[0] + m * 64 + c) = z;
+      } else {
+        for (int q = 0; q < p.nseg; ++q)
+          for (int c = p.rp; c < 64; c += 8) *reinterpret_cast<uint4*>(p.out16[q] + m * 64 + c) = z;
+      }
+    }
+  }
+  cluster_sync_all();  // every CTA keeps its shared memory until the others have read it
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
   }
 }
 
-// Sum the splits (ascending) and write the outputs.
-//   FWD (one problem, segment q in columns q*rp ..): u_out[q] [M, r] fp32 (if
-//        given) and s*U of segment q as bf16 [M, 64], zero in columns >= r.
-//   DX  (problem q = segment q): G_q [M, r] fp32 and s*G as bf16 [M, 64] with
-//        segment q in columns q*rp .. q*rp + r - 1, zero elsewhere.
-struct Red {
-  const float* part[3];
-  int splits[3];
-  int np[3];
-  float* out32[3];
-  __nv_bfloat16* out16[3];
-  int dx, nseg, M, r, rp;
-  float s;
-};
-
-__global__ void __launch_bounds__(256) lora_down_reduce(const __grid_constant__ Red R) {
-  const int64_t per = (int64_t)R.M * 64;
-  const int64_t total = R.dx ? per : per * R.nseg;
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int q0 = (int)(idx / per);
-    const int64_t rem = idx % per;
-    const int64_t m = rem / 64;
-    const int c = (int)(rem % 64);
-    int pb, col, seg, j;
-    bool live;
-    if (R.dx) {
-      seg = c / R.rp;
-      j = c % R.rp;
-      live = seg < R.nseg && j < R.r;
-      pb = seg;
-      col = j;
-    } else {
-      seg = q0;
-      j = c;
-      live = j < R.r;
-      pb = 0;
-      col = seg * R.rp + j;
-    }
-    float sum = 0.0f;
-    if (live) {
-      const float* part = R.part[pb];
-      const int np = R.np[pb];
-      for (int k = 0; k < R.splits[pb]; ++k) sum += part[((int64_t)k * R.M + m) * np + col];
-      if (R.out32[seg]) R.out32[seg][m * R.r + j] = sum;
-    }
-    __nv_bfloat16* o = R.out16[R.dx ? 0 : seg];
-    o[m * 64 + c] = __float2bfloat16_rn(live ? R.s * sum : 0.0f);
-  }
+// splits (cluster size) so that about TARGET_CTAS CTAs run; at most 8 and at most the blocks
+static int plan_splits(int ctas_per_split, int nkb_max) {
+  int s = (TARGET_CTAS + ctas_per_split - 1) / ctas_per_split;
+  return std::max(1, std::min(s, std::min(MAX_SPLITS, nkb_max)));
 }
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
-// Padded copies of the LoRA operands.
-//   FWD job q: Bpad_q [n_q, 64] = B_q in columns < r, zero elsewhere
-//   DX  job q < nseg: Bt_q [rp, n_q] = B_q^T, zero rows >= r
-//   DX  job nseg: At [K, 64] = A_q^T of every segment q in columns q*rp .., zero elsewhere
-//   DX  job nseg + 1 + q: SU_q [M, 64] = bf16(s * U_q) in columns < r, zero elsewhere
+// Padded copies of the LoRA operands for the backward (the forward's padded B
+// is written inside lora_down_kernel):
+//   job q < nseg: Bt_q [rp, n_q] = B_q^T, zero rows >= r
+//   job nseg: At [K, 64] = A_q^T of every segment q in columns q*rp .., zero elsewhere
+//   job nseg + 1 + q: SU_q [M, 64] = bf16(s * U_q) in columns < r, zero elsewhere
 struct Pad {
   const __nv_bfloat16* A[3];
   const __nv_bfloat16* B[3];
   const float* U[3];
-  __nv_bfloat16* Bpad[3];
   __nv_bfloat16* Bt[3];
   __nv_bfloat16* SU[3];
   __nv_bfloat16* At;
   int64_t n[3];
   int64_t K, M;
-  int nseg, r, rp, dx;
+  int nseg, r, rp;
   float s;
 };
 
 __global__ void __launch_bounds__(256) lora_pad(const __grid_constant__ Pad P) {
   const int job = blockIdx.y;
-  const bool at = P.dx && job == P.nseg;
-  const bool su = P.dx && job > P.nseg;
-  const int64_t total = su ? P.M * 64 : at ? P.K * 64 : P.dx ? (int64_t)P.rp * P.n[job] : P.n[job] * 64;
+  const bool at = job == P.nseg;
+  const bool su = job > P.nseg;
+  const int64_t total = su ? P.M * 64 : at ? P.K * 64 : (int64_t)P.rp * P.n[job];
   const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -775,25 +829,12 @@ __global__ void __launch_bounds__(256) lora_pad(const __grid_constant__ Pad P) {
       const int64_t k = idx / 64;
       const int c = (int)(idx % 64), q = c / P.rp, j = c % P.rp;
       P.At[idx] = (q < P.nseg && j < P.r) ? P.A[q][(int64_t)j * P.K + k] : zero;
-    } else if (P.dx) {
+    } else {
       const int64_t j = idx / P.n[job], n = idx % P.n[job];
       P.Bt[job][idx] = j < P.r ? P.B[job][n * P.r + j] : zero;
-    } else {
-      const int64_t n = idx / 64;
-      const int c = (int)(idx % 64);
-      P.Bpad[job][idx] = c < P.r ? P.B[job][n * P.r + c] : zero;
     }
   }
 }
-
-// contraction blocks per split for problems of nkb[i] blocks over mtiles row tiles
-static int plan_kbps(const int* nkb, int nprob, int mtiles) {
-  int64_t tot = 0;
-  for (int i = 0; i < nprob; ++i) tot += nkb[i];
-  int64_t k = (tot * mtiles + TARGET_CTAS - 1) / TARGET_CTAS;
-  return (int)std::max<int64_t>(1, k);
-}
-static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace ldn
 
@@ -869,7 +910,8 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, cudaStre
   return hbest == 2 ? launch_pair_h<MODE, 2>(maps, p, ncl, stream) : launch_pair_h<MODE, 1>(maps, p, ncl, stream);
 }
 
-static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int maxsplits, cudaStream_t stream) {
+// one cluster of `splits` CTAs per (row tile, problem)
+static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int splits, cudaStream_t stream) {
   static int configured[64] = {0};
   int dev = 0;
   LSQ_CUDA_TRY(cudaGetDevice(&dev));
@@ -878,18 +920,20 @@ static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int m
                                       ldn::SMEM_BYTES));
     configured[dev] = 1;
   }
-  const int mtiles = (p.M + ldn::BM - 1) / ldn::BM;
-  ldn::lora_down_kernel<<<dim3(mtiles, maxsplits, p.nprob), ldn::NTHREADS, ldn::SMEM_BYTES, stream>>>(maps, p);
-  LSQ_LAUNCH_CHECK("lora_down_kernel");
-  return LSQ_OK;
-}
-
-static lsq_status launch_reduce(const ldn::Red& R, cudaStream_t stream) {
-  const int64_t total = (int64_t)R.M * 64 * (R.dx ? 1 : R.nseg);
-  int64_t g = (total + 255) / 256;
-  if (g > 1184) g = 1184;
-  ldn::lora_down_reduce<<<(unsigned)g, 256, 0, stream>>>(R);
-  LSQ_LAUNCH_CHECK("lora_down_reduce");
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((p.M + ldn::BM - 1) / ldn::BM), (unsigned)splits, (unsigned)p.nprob);
+  cfg.blockDim = dim3(ldn::NTHREADS);
+  cfg.dynamicSmemBytes = ldn::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)splits;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LSQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, ldn::lora_down_kernel, maps, p));
   return LSQ_OK;
 }
 
@@ -897,7 +941,7 @@ static lsq_status launch_pad(const ldn::Pad& P, int64_t most, cudaStream_t strea
   int64_t g = (most + 255) / 256;
   if (g > 512) g = 512;
   if (g < 1) g = 1;
-  ldn::lora_pad<<<dim3((unsigned)g, P.dx ? 2 * P.nseg + 1 : P.nseg), 256, 0, stream>>>(P);
+  ldn::lora_pad<<<dim3((unsigned)g, 2 * P.nseg + 1), 256, 0, stream>>>(P);
   LSQ_LAUNCH_CHECK("lora_pad");
   return LSQ_OK;
 }
@@ -940,52 +984,48 @@ static lsq_status check_weight(const lsq_nf4_weight& w, int64_t K, const char* w
   return LSQ_OK;
 }
 
-// ---- forward: workspace = s*U per segment [M, 64] bf16 | padded B per segment [n, 64] bf16 | U partials
+// ---- forward: workspace = s*U per segment [M, 64] bf16 | padded B per segment [n, 64] bf16
 struct FwdPlan {
-  int kbps, splits, np;
-  size_t su, bpad[3], part, total;
+  int splits, kbps;
+  size_t su, bpad[3], total;
 };
 static FwdPlan fwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
+  (void)r;
   FwdPlan f;
   memset(&f, 0, sizeof(f));
   const int nkb = (int)(K / 64);
   const int mtiles = (int)((M + ldn::BM - 1) / ldn::BM);
-  f.kbps = ldn::plan_kbps(&nkb, 1, mtiles);
-  f.splits = (nkb + f.kbps - 1) / f.kbps;
-  f.np = nseg * rpad(r);
+  f.splits = ldn::plan_splits(mtiles, nkb);
+  f.kbps = (nkb + f.splits - 1) / f.splits;
   f.su = ldn::round256((size_t)M * 64 * 2);
   f.total = (size_t)nseg * f.su;
   for (int i = 0; i < nseg; ++i) {
     f.bpad[i] = ldn::round256((size_t)n_out[i] * 64 * 2);
     f.total += f.bpad[i];
   }
-  f.part = ldn::round256((size_t)f.splits * (size_t)M * (size_t)f.np * sizeof(float));
-  f.total += f.part;
   return f;
 }
 
-// ---- backward rank-r part: G fp32 | s*G bf16 [M, 64] | A^T side by side [K, 64] | B_q^T [rp, n_q] | G partials
+// ---- backward rank-r part: s*G bf16 [M, 64] | A^T side by side [K, 64] | B_q^T [rp, n_q] | s*U_q [M, 64]
 struct BwdPlan {
-  int kbps, splits[3];
-  size_t sg, at, bt[3], su, part[3], total;
+  int splits;
+  size_t sg, at, bt[3], su, total;
 };
 static BwdPlan bwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
   BwdPlan b;
   memset(&b, 0, sizeof(b));
   const int rp = rpad(r);
-  int nkb[3];
-  for (int i = 0; i < nseg; ++i) nkb[i] = (int)((n_out[i] + 63) / 64);
+  int nkb_max = 1;
+  for (int i = 0; i < nseg; ++i) nkb_max = std::max(nkb_max, (int)((n_out[i] + 63) / 64));
   const int mtiles = (int)((M + ldn::BM - 1) / ldn::BM);
-  b.kbps = ldn::plan_kbps(nkb, nseg, mtiles);
+  b.splits = ldn::plan_splits(mtiles * nseg, nkb_max);
   b.sg = ldn::round256((size_t)M * 64 * 2);
   b.at = ldn::round256((size_t)K * 64 * 2);
   b.su = b.sg;
   b.total = b.sg + b.at + (size_t)nseg * b.su;
   for (int i = 0; i < nseg; ++i) {
-    b.splits[i] = (nkb[i] + b.kbps - 1) / b.kbps;
     b.bt[i] = ldn::round256((size_t)rp * (size_t)n_out[i] * 2);
-    b.part[i] = ldn::round256((size_t)b.splits[i] * (size_t)M * (size_t)rp * sizeof(float));
-    b.total += b.bt[i] + b.part[i];
+    b.total += b.bt[i];
   }
   return b;
 }
@@ -1012,7 +1052,6 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   *at = reinterpret_cast<__nv_bfloat16*>(cur);
   cur += b.at;
   __nv_bfloat16* bt[3];
-  float* part[3];
   for (int i = 0; i < nseg; ++i) {
     bt[i] = reinterpret_cast<__nv_bfloat16*>(cur);
     cur += b.bt[i];
@@ -1020,10 +1059,6 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   for (int i = 0; i < nseg; ++i) {
     su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
     cur += b.su;
-  }
-  for (int i = 0; i < nseg; ++i) {
-    part[i] = reinterpret_cast<float*>(cur);
-    cur += b.part[i];
   }
   lsq_status st;
   ldn::Pad P;
@@ -1046,7 +1081,6 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   P.nseg = nseg;
   P.r = r;
   P.rp = rp;
-  P.dx = 1;
   if ((st = launch_pad(P, most, stream)) != LSQ_OK) return st;
 
   ldn::Maps maps;
@@ -1055,37 +1089,22 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   memset(&p, 0, sizeof(p));
   p.nprob = nseg;
   p.M = (int)M;
+  p.r = r;
   p.rp = rp;
-  p.kbps = b.kbps;
-  int maxsplits = 1;
+  p.dx = 1;
+  p.nseg = nseg;
+  p.s = s;
+  p.out16[0] = *sg;
   for (int i = 0; i < nseg; ++i) {
     if ((st = tmap_act(&maps.in[i], dy[i], n_out[i], M, ldn::BM)) != LSQ_OK) return st;
     if ((st = tmap_act(&maps.wl[i], bt[i], n_out[i], rp, (uint32_t)rp)) != LSQ_OK) return st;
     ldn::Prob& pr = p.pr[i];
-    pr.part = part[i];
     pr.nkb = (int)((n_out[i] + 63) / 64);
-    pr.splits = b.splits[i];
+    pr.kbps = (pr.nkb + b.splits - 1) / b.splits;
     pr.nsub = 1;
     pr.first = i;
-    maxsplits = std::max(maxsplits, pr.splits);
   }
-  if ((st = launch_down(maps, p, maxsplits, stream)) != LSQ_OK) return st;
-
-  ldn::Red R;
-  memset(&R, 0, sizeof(R));
-  for (int i = 0; i < nseg; ++i) {
-    R.part[i] = part[i];
-    R.splits[i] = b.splits[i];
-    R.np[i] = rp;
-  }
-  R.out16[0] = *sg;
-  R.dx = 1;
-  R.nseg = nseg;
-  R.M = (int)M;
-  R.r = r;
-  R.rp = rp;
-  R.s = s;
-  return launch_reduce(R, stream);
+  return launch_down(maps, p, b.splits, stream);
 }
 
 // dX = sum_q dY_q deq(W_q) (+ (s G) A when sg != null)
@@ -1190,7 +1209,7 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
   }
 
   if (r > 0) {
-    // workspace: s*U per segment | padded B per segment | U partials
+    // workspace: s*U per segment | padded B per segment
     char* cur = static_cast<char*>(workspace);
     __nv_bfloat16* su[3];
     __nv_bfloat16* bpad[3];
@@ -1202,58 +1221,31 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
       bpad[i] = reinterpret_cast<__nv_bfloat16*>(cur);
       cur += f.bpad[i];
     }
-    float* part = reinterpret_cast<float*>(cur);
-
-    ldn::Pad P;
-    memset(&P, 0, sizeof(P));
-    int64_t most = 0;
-    for (int i = 0; i < nseg; ++i) {
-      P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
-      P.Bpad[i] = bpad[i];
-      P.n[i] = ns[i];
-      most = std::max<int64_t>(most, ns[i] * 64);
-    }
-    P.K = K;
-    P.nseg = nseg;
-    P.r = r;
-    P.rp = rp;
-    P.dx = 0;
-    if ((st = launch_pad(P, most, cs)) != LSQ_OK) return st;
-
     ldn::Maps dm;
     memset(&dm, 0, sizeof(dm));
     ldn::Params dp;
     memset(&dp, 0, sizeof(dp));
     if ((st = tmap_act(&dm.in[0], x, K, M, ldn::BM)) != LSQ_OK) return st;
-    for (int i = 0; i < nseg; ++i)
+    for (int i = 0; i < nseg; ++i) {
       if ((st = tmap_act(&dm.wl[i], A[i], K, r, (uint32_t)rp)) != LSQ_OK) return st;
+      dp.out32[i] = u_out ? u_out[i] : nullptr;
+      dp.out16[i] = su[i];
+      dp.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+      dp.Bpad[i] = bpad[i];
+      dp.nB[i] = ns[i];
+    }
     dp.nprob = 1;
     dp.M = (int)M;
+    dp.r = r;
     dp.rp = rp;
-    dp.kbps = f.kbps;
-    dp.pr[0].part = part;
+    dp.dx = 0;
+    dp.nseg = nseg;
+    dp.s = s;
     dp.pr[0].nkb = (int)(K / 64);
-    dp.pr[0].splits = f.splits;
+    dp.pr[0].kbps = f.kbps;
     dp.pr[0].nsub = nseg;
     dp.pr[0].first = 0;
     if ((st = launch_down(dm, dp, f.splits, cs)) != LSQ_OK) return st;
-
-    ldn::Red R;
-    memset(&R, 0, sizeof(R));
-    R.part[0] = part;
-    R.splits[0] = f.splits;
-    R.np[0] = f.np;
-    for (int i = 0; i < nseg; ++i) {
-      R.out32[i] = u_out ? u_out[i] : nullptr;
-      R.out16[i] = su[i];
-    }
-    R.dx = 0;
-    R.nseg = nseg;
-    R.M = (int)M;
-    R.r = r;
-    R.rp = rp;
-    R.s = s;
-    if ((st = launch_reduce(R, cs)) != LSQ_OK) return st;
 
     for (int i = 0; i < nseg; ++i) {
       if ((st = tmap_act(&maps.la[i], su[i], 64, M, BMC)) != LSQ_OK) return st;

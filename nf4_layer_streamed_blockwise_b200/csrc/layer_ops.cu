@@ -241,6 +241,112 @@ __global__ void __launch_bounds__(1024) xent_mean_kernel(const float* __restrict
   if (threadIdx.x == 0) *loss = tot * inv_count;
 }
 
+// ---------------------------------------------------------------- sequence log-probabilities and DPO
+// (preference losses on the same streamed base with the adapter off as the
+// reference: aiany.app listing, "How It Works (concise)"; the objective is
+// DPO, Rafailov et al. 2023, eq. 7)
+
+// per row: lse and log p(target) (0 on the last row of a sequence)
+__global__ void __launch_bounds__(XE_T) seqlp_row_kernel(const float* __restrict__ logits,
+                                                         const int32_t* __restrict__ ids, int seq, int64_t V,
+                                                         float* __restrict__ row_lse, float* __restrict__ row_lp) {
+  __shared__ float rm[XE_T / 32], rsum[XE_T / 32];
+  const int64_t row = blockIdx.x;
+  const int t = (int)(row % seq);
+  const float* lr = logits + row * V;
+  float m = -INFINITY, s = 0.0f;
+  for (int64_t c = threadIdx.x; c < V; c += XE_T) {
+    const float v = lr[c];
+    if (v > m) {
+      s = s * expf(m - v) + 1.0f;
+      m = v;
+    } else {
+      s += expf(v - m);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float mm = fmaxf(m, m2);
+    s = (m == -INFINITY ? 0.0f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.0f : s2 * expf(m2 - mm));
+    m = mm;
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    rm[w] = m;
+    rsum[w] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = -INFINITY, SS = 0.0f;
+    for (int i = 0; i < XE_T / 32; ++i) {
+      const float mm = fmaxf(M, rm[i]);
+      SS = (M == -INFINITY ? 0.0f : SS * expf(M - mm)) + (rm[i] == -INFINITY ? 0.0f : rsum[i] * expf(rm[i] - mm));
+      M = mm;
+    }
+    const float lse = M + logf(SS);
+    row_lse[row] = lse;
+    float lp = 0.0f;
+    if (t < seq - 1) {
+      const int32_t tgt = ids[row + 1];
+      if (tgt >= 0 && tgt < V) lp = lr[tgt] - lse;
+      else report(LSQ_EINVAL, 803);
+    }
+    row_lp[row] = lp;
+  }
+}
+
+// per sequence: sum of its rows' log p in a fixed order
+__global__ void __launch_bounds__(1024) seqlp_sum_kernel(const float* __restrict__ row_lp, int seq,
+                                                         float* __restrict__ seq_logp) {
+  __shared__ float red[32];
+  const int64_t b = blockIdx.x;
+  float s = 0.0f;
+  for (int t = threadIdx.x; t < seq; t += 1024) s += row_lp[b * seq + t];
+  const float tot = block_sum<1024>(s, red);
+  if (threadIdx.x == 0) seq_logp[b] = tot;
+}
+
+// loss = mean_i softplus(-z_i), z_i = beta ((pi_c - ref_c) - (pi_r - ref_r)); dseq = d loss / d pi
+__global__ void __launch_bounds__(32) dpo_loss_kernel(const float* __restrict__ pi, const float* __restrict__ ref,
+                                                      int npairs, float beta, float* __restrict__ loss,
+                                                      float* __restrict__ dseq) {
+  if (threadIdx.x != 0) return;
+  float tot = 0.0f;
+  for (int i = 0; i < npairs; ++i) {
+    const float z = beta * ((pi[2 * i] - ref[2 * i]) - (pi[2 * i + 1] - ref[2 * i + 1]));
+    tot += fmaxf(-z, 0.0f) + log1pf(expf(-fabsf(z)));           // softplus(-z), no overflow
+    const float sig_neg = z >= 0.0f ? expf(-z) / (1.0f + expf(-z)) : 1.0f / (1.0f + expf(z));  // sigmoid(-z)
+    const float g = beta * sig_neg / (float)npairs;
+    dseq[2 * i] = -g;
+    dseq[2 * i + 1] = g;
+  }
+  *loss = tot / (float)npairs;
+}
+
+// dlogits = dseq[b] * (onehot(target) - softmax), zero on the last row of a sequence
+__global__ void __launch_bounds__(XE_T) seqlp_bwd_kernel(const float* __restrict__ logits,
+                                                         const int32_t* __restrict__ ids, int seq, int64_t V,
+                                                         const float* __restrict__ row_lse,
+                                                         const float* __restrict__ dseq,
+                                                         __nv_bfloat16* __restrict__ dlogits) {
+  const int64_t row = blockIdx.x;
+  const int t = (int)(row % seq);
+  const float* lr = logits + row * V;
+  __nv_bfloat16* dr = dlogits + row * V;
+  if (t == seq - 1) {
+    for (int64_t c = threadIdx.x; c < V; c += XE_T) dr[c] = __float2bfloat16_rn(0.0f);
+    return;
+  }
+  const float g = dseq[row / seq], lse = row_lse[row];
+  const int32_t tgt = ids[row + 1];
+  for (int64_t c = threadIdx.x; c < V; c += XE_T) {
+    float p = -expf(lr[c] - lse);
+    if (c == tgt) p += 1.0f;
+    dr[c] = __float2bfloat16_rn(g * p);
+  }
+}
+
 // ---------------------------------------------------------------- AdamW
 __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
                                                     float* __restrict__ m, float* __restrict__ v,
@@ -375,6 +481,52 @@ extern "C" lsq_status lsq_xent_fwd_bwd(const float* logits, const int32_t* ids, 
   LSQ_LAUNCH_CHECK("xent_row_kernel");
   xent_mean_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(rl, rows, inv, loss);
   LSQ_LAUNCH_CHECK("xent_mean_kernel");
+  return LSQ_OK;
+}
+
+extern "C" size_t lsq_seq_logprob_workspace_size(int64_t rows) {
+  return (size_t)((rows > 0 ? rows : 1) * sizeof(float) + 255) / 256 * 256;
+}
+
+extern "C" lsq_status lsq_seq_logprob(const float* logits, const int32_t* ids, int64_t batch, int64_t seq, int64_t V,
+                                      float* row_lse, float* seq_logp, void* workspace, size_t workspace_bytes,
+                                      lsq_cuda_stream stream) {
+  if (!logits || !ids || !row_lse || !seq_logp || !workspace) return fail(LSQ_EINVAL, "lsq_seq_logprob: NULL argument");
+  if (batch < 1 || seq < 2 || V < 2) return fail(LSQ_EINVAL, "lsq_seq_logprob: need batch >= 1, seq >= 2, V >= 2");
+  const int64_t rows = batch * seq;
+  if (workspace_bytes < lsq_seq_logprob_workspace_size(rows))
+    return fail(LSQ_EINVAL, "lsq_seq_logprob: workspace too small");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  float* rl = static_cast<float*>(workspace);
+  seqlp_row_kernel<<<(unsigned)rows, XE_T, 0, (cudaStream_t)stream>>>(logits, ids, (int)seq, V, row_lse, rl);
+  LSQ_LAUNCH_CHECK("seqlp_row_kernel");
+  seqlp_sum_kernel<<<(unsigned)batch, 1024, 0, (cudaStream_t)stream>>>(rl, (int)seq, seq_logp);
+  LSQ_LAUNCH_CHECK("seqlp_sum_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_dpo_loss(const float* policy_logp, const float* ref_logp, int32_t npairs, float beta,
+                                   float* loss, float* dseq, lsq_cuda_stream stream) {
+  if (!policy_logp || !ref_logp || !loss || !dseq) return fail(LSQ_EINVAL, "lsq_dpo_loss: NULL argument");
+  if (npairs < 1) return fail(LSQ_EINVAL, "lsq_dpo_loss: npairs must be >= 1");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  dpo_loss_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(policy_logp, ref_logp, npairs, beta, loss, dseq);
+  LSQ_LAUNCH_CHECK("dpo_loss_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_seq_logprob_bwd(const float* logits, const int32_t* ids, int64_t batch, int64_t seq,
+                                          int64_t V, const float* row_lse, const float* dseq, void* dlogits,
+                                          lsq_cuda_stream stream) {
+  if (!logits || !ids || !row_lse || !dseq || !dlogits) return fail(LSQ_EINVAL, "lsq_seq_logprob_bwd: NULL argument");
+  if (batch < 1 || seq < 2 || V < 2) return fail(LSQ_EINVAL, "lsq_seq_logprob_bwd: need batch >= 1, seq >= 2, V >= 2");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  seqlp_bwd_kernel<<<(unsigned)(batch * seq), XE_T, 0, (cudaStream_t)stream>>>(
+      logits, ids, (int)seq, V, row_lse, dseq, static_cast<__nv_bfloat16*>(dlogits));
+  LSQ_LAUNCH_CHECK("seqlp_bwd_kernel");
   return LSQ_OK;
 }
 

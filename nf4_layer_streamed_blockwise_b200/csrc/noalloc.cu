@@ -18,9 +18,10 @@ namespace lsq {
 namespace noalloc {
 
 // Largest scratch the entry point serves: 32 MiB, which covers any one linear
-// of the 8B shape at 2048 tokens and r = 16 (12.5 MiB for a 4096 x 4096
-// projection, 14.3 MiB for the 14336-wide down projection).  Every GPU that
-// loads the library keeps this array for as long as the process lives.
+// of the 8B shape at 2048 tokens and r = 16 (9.1 MiB for a 4096 x 4096
+// projection, 14.9 MiB for gate or up, 15.9 MiB for the 14336-wide down
+// projection).  Every GPU that loads the library keeps this array for as
+// long as the process lives.
 constexpr size_t SCRATCH_BYTES = size_t(32) << 20;
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[SCRATCH_BYTES];

@@ -92,6 +92,12 @@ _SIGS = {
     "lsq_xent_workspace_size": (c_size_t, [c_int64]),
     "lsq_xent_fwd_bwd": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                    c_size_t, c_void_p]),
+    "lsq_seq_logprob_workspace_size": (c_size_t, [c_int64]),
+    "lsq_seq_logprob": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                  c_size_t, c_void_p]),
+    "lsq_dpo_loss": (c_int32, [c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p]),
+    "lsq_seq_logprob_bwd": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
     "lsq_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_float,
                                  c_float, c_float, c_float, c_float, c_void_p]),
     "lsq_stream_create": (c_int32, [ctypes.POINTER(lsq_stream_cfg), c_void_p, c_void_p, ctypes.POINTER(c_void_p)]),
@@ -140,7 +146,8 @@ LAUNCHES = [0]
 _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
             "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
-            "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1}
+            "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1, "lsq_seq_logprob": 2,
+            "lsq_dpo_loss": 1, "lsq_seq_logprob_bwd": 1}
 
 
 def _call(name, *args, launches=None):
@@ -350,6 +357,24 @@ def lsq_xent_workspace_size(rows: int) -> int:
 def lsq_xent_fwd_bwd(logits, ids, batch: int, seq: int, V: int, loss, dlogits, workspace, stream=None):
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_xent_fwd_bwd", _p(logits), _p(ids), batch, seq, V, _p(loss), _p(dlogits), _p(workspace), wsb,
+          _stream(stream))
+
+
+def lsq_seq_logprob_workspace_size(rows: int) -> int:
+    return int(_fn("lsq_seq_logprob_workspace_size")(rows))
+
+
+def lsq_seq_logprob(logits, ids, batch: int, seq: int, V: int, row_lse, seq_logp, workspace, stream=None):
+    _call("lsq_seq_logprob", _p(logits), _p(ids), batch, seq, V, _p(row_lse), _p(seq_logp), _p(workspace),
+          _nbytes(workspace), _stream(stream))
+
+
+def lsq_dpo_loss(policy_logp, ref_logp, npairs: int, beta: float, loss, dseq, stream=None):
+    _call("lsq_dpo_loss", _p(policy_logp), _p(ref_logp), npairs, beta, _p(loss), _p(dseq), _stream(stream))
+
+
+def lsq_seq_logprob_bwd(logits, ids, batch: int, seq: int, V: int, row_lse, dseq, dlogits, stream=None):
+    _call("lsq_seq_logprob_bwd", _p(logits), _p(ids), batch, seq, V, _p(row_lse), _p(dseq), _p(dlogits),
           _stream(stream))
 
 

@@ -5,7 +5,8 @@
 
 For every linear group of a decoder layer (q/k/v fused, o, gate/up fused,
 down) it times the forward call (all its kernels), the backward call, the dX
-GEMM alone (no adapter), and the lm_head GEMMs,
+GEMM alone (no adapter), the causal attention of one layer (forward; backward
+counted as 2.5x the forward FLOPs), and the lm_head GEMMs,
 with CUDA events around each launch and a 256 MB L2 flush between launches;
 prints one JSON line per kernel (median ms, TFLOP/s, fraction of the
 measured bf16 peak).  Inputs are random; only timing is reported.
@@ -99,6 +100,17 @@ def main():
         run(f"dx_{g}", fl0, lambda: L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, None, None, 0, 0.0, None, dx, None, None,
                                                                 0, None))
         del Ws, x, A, B, ys, us, dys, dx, dA, dB, ws, wsf
+    # causal GQA attention of one layer (the batch's sequences), forward and backward
+    Hq, Hkv, hd, Bt, Sq = sh.n_q, sh.n_kv, sh.hd, a.batch, a.seq
+    q, o, do = (torch.randn(Bt * Sq, Hq * hd, **bf) for _ in range(3))
+    k, v = (torch.randn(Bt * Sq, Hkv * hd, **bf) for _ in range(2))
+    lse = torch.empty(Bt * Hq * Sq, dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsa = torch.empty(L.lsq_attention_bwd_workspace_size(Bt, Sq, Hq), dtype=torch.uint8, device="cuda")
+    fa = 4.0 * Bt * Hq * Sq * Sq * hd / 2  # causal: half of the two S x S x hd products
+    run("attn_fwd", fa, lambda: L.lsq_attention_fwd(q, k, v, o, lse, Bt, Sq, Hq, Hkv, hd))
+    run("attn_bwd", 2.5 * fa, lambda: L.lsq_attention_bwd(q, k, v, o, lse, do, dq, dk, dv, Bt, Sq, Hq, Hkv, hd, wsa))
+    del q, o, do, k, v, lse, dq, dk, dv, wsa
     hn = torch.randn(M, sh.d, **bf)
     E = torch.randn(sh.vocab, sh.d, **bf) * 0.02
     logits = torch.empty(M, sh.vocab, dtype=torch.float32, device="cuda")

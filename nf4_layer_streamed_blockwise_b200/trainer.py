@@ -242,8 +242,8 @@ class StreamedLoraTrainer:
         e.record(self.compute)
         self.timeline.append((kind, flops, start, e))
 
-    def _fwd_flops(self, ns, K):
-        M, r = self.M, self.shape.r
+    def _fwd_flops(self, ns, K, r=None):
+        M, r = self.M, self.shape.r if r is None else r
         return sum(2.0 * M * n * K + 2.0 * M * r * K + 2.0 * M * n * r for n in ns)
 
     def _bwd_flops(self, ns, K):
@@ -257,33 +257,41 @@ class StreamedLoraTrainer:
         B = {n: lp.view(lp.op, l, n, "B") for n in S.LINEARS}
         return A, B
 
-    def _layer_fwd(self, l: int, W: LayerView, save: bool):
-        sh, M, r, s = self.shape, self.M, self.shape.r, self.shape.s
-        A, B = self._ops(l)
-        hin, hout = self.h[l], self.h[l + 1]
-        U = self.U if save else {n: None for n in S.LINEARS}
+    def _layer_fwd(self, l: int, W: LayerView, save: bool, hin=None, hout=None, adapter: bool = True):
+        """Layer l: hin (default h[l]) -> hout (default h[l+1], may alias hin).
+        adapter=False runs the frozen base alone (r = 0): the reference model
+        of the preference loss."""
+        sh, M = self.shape, self.M
+        r, s = (sh.r, sh.s) if adapter else (0, 0.0)
+        if adapter:
+            A, B = self._ops(l)
+        else:
+            A = B = {n: None for n in S.LINEARS}
+        hin = self.h[l] if hin is None else hin
+        hout = self.h[l + 1] if hout is None else hout
+        U = self.U if save and adapter else {n: None for n in S.LINEARS}
         L.lsq_rmsnorm_fwd(hin, W.ln1, self.x1, self.rstd1, M, sh.d, sh.eps)
         t = self._t0()
         L.lsq_nf4_lora_fwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, M, [A["q"], A["k"], A["v"]],
                                  [B["q"], B["k"], B["v"]], r, s, None, [self.q, self.k, self.v],
                                  [U["q"], U["k"], U["v"]], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d))
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d, r))
         L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
         L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
         L.lsq_attention_fwd(self.q, self.k, self.v, self.a, self.lse, self.B, self.S, sh.n_q, sh.n_kv, sh.hd)
         t = self._t0()
         L.lsq_nf4_lora_fwd(W.W["o"], self.a, M, A["o"], B["o"], r, s, hin, self.hmid, U["o"], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d))
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d, r))
         L.lsq_rmsnorm_fwd(self.hmid, W.ln2, self.x2, self.rstd2, M, sh.d, sh.eps)
         t = self._t0()
         L.lsq_nf4_lora_fwd_multi([W.W["gate"], W.W["up"]], self.x2, M, [A["gate"], A["up"]], [B["gate"], B["up"]],
                                  r, s, None, [self.g, self.u], [U["gate"], U["up"]], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d))
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d, r))
         L.lsq_swiglu_fwd(self.g, self.u, self.mm, M * sh.f)
         t = self._t0()
         L.lsq_nf4_lora_fwd(W.W["down"], self.mm, M, A["down"], B["down"], r, s, self.hmid, hout, U["down"],
                            workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f))
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f, r))
 
     def _layer_bwd(self, l: int, W: LayerView):
         """self.dh holds dLoss/dh[l+1] on entry and dLoss/dh[l] on exit."""
@@ -345,6 +353,57 @@ class StreamedLoraTrainer:
             W = self._view(l, -1)
             self._layer_fwd(l, W, save=True)
             self._layer_bwd(l, W)
+
+    def _dpo_buffers(self):
+        if getattr(self, "h_ref", None) is None:
+            dev, M = self.h.device, self.M
+            self.h_ref = torch.empty(M, self.shape.d, dtype=torch.bfloat16, device=dev)
+            self.row_lse = torch.empty(M, dtype=torch.float32, device=dev)
+            self.pi_logp, self.ref_logp, self.dseq = (torch.empty(self.B, dtype=torch.float32, device=dev)
+                                                      for _ in range(3))
+            self.ws_seqlp = torch.empty(L.lsq_seq_logprob_workspace_size(M), dtype=torch.uint8, device=dev)
+
+    def forward_backward_dpo(self, beta: float = 0.1):
+        """DPO over the batch as pairs (chosen = sequence 2i, rejected = 2i+1):
+        loss into self.loss_dev, LoRA gradients into self.lora.grad.
+
+        The reference model is the same streamed base with the adapters off:
+        while a layer's record is on the GPU for the policy forward, the
+        reference forward of that layer runs too (fused linears with r = 0), so
+        the reference costs compute but no extra layer uploads."""
+        sh, M = self.shape, self.M
+        if self.B % 2:
+            raise ValueError("DPO needs an even batch (pairs of chosen / rejected sequences)")
+        self._dpo_buffers()
+        L.lsq_embed_gather(self.ids, self.embed, self.h[0], M, sh.d, sh.vocab)
+        L.lsq_embed_gather(self.ids, self.embed, self.h_ref, M, sh.d, sh.vocab)
+        for l in range(sh.n_layers):
+            W = self._view(l, +1)
+            self._layer_fwd(l, W, save=False)
+            self._layer_fwd(l, W, save=False, hin=self.h_ref, hout=self.h_ref, adapter=False)
+        # reference sequence log-probabilities
+        L.lsq_rmsnorm_fwd(self.h_ref, self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
+        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        L.lsq_seq_logprob(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.ref_logp, self.ws_seqlp)
+        # policy sequence log-probabilities, loss, d loss / d logits
+        L.lsq_rmsnorm_fwd(self.h[sh.n_layers], self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
+        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        L.lsq_seq_logprob(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.pi_logp, self.ws_seqlp)
+        L.lsq_dpo_loss(self.pi_logp, self.ref_logp, self.B // 2, beta, self.loss_dev, self.dseq)
+        L.lsq_seq_logprob_bwd(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.dseq,
+                              self.dlogits)
+        L.lsq_dense_gemm(self.dlogits, self.lm_head, self.hn, M, sh.d, sh.vocab, 1, 0)   # hn <- d hn
+        L.lsq_rmsnorm_bwd(self.hn, self.h[sh.n_layers], self.final_norm, self.rstdf, None, self.dh, M, sh.d)
+        for l in reversed(range(sh.n_layers)):
+            W = self._view(l, -1)
+            self._layer_fwd(l, W, save=True)
+            self._layer_bwd(l, W)
+
+    def train_step_dpo(self, ids: Optional[torch.Tensor] = None, beta: float = 0.1):
+        if ids is not None:
+            self.set_ids(ids)
+        self.forward_backward_dpo(beta)
+        self.optimizer_step()
 
     def optimizer_step(self):
         lp = self.lora

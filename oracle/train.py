@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 from . import nf4
-from .decoder import F64, adamw, model_loss_and_grads
+from .decoder import DPO_BETA, F64, adamw, model_dpo_loss_and_grads, model_loss_and_grads
 
 
 def dequantized_layer(Wbf16: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
@@ -66,3 +66,12 @@ def train(shape, layers_bf16, emb_bf16, lora_masters, ids_per_step: List[torch.T
                     per[n][ab] = p.to(torch.float32).to(F64)
                     mom[l][n][ab], vel[l][n][ab] = m, v
     return losses, first_grads, masters
+
+
+def dpo_step(shape, layers_bf16, emb_bf16, lora_masters, ids: torch.Tensor, beta: float = DPO_BETA):
+    """One DPO forward/backward on the NF4 base (reference = the same base with
+    the adapters off): -> (loss, grads, policy sequence log-probs, reference ones)."""
+    layers = [dequantized_layer(W) for W in layers_bf16]
+    emb = {k: v.to(F64) for k, v in emb_bf16.items()}
+    ops = [{n: {ab: operand(t[ab]) for ab in ("A", "B")} for n, t in per.items()} for per in lora_masters]
+    return model_dpo_loss_and_grads(ids, layers, emb, ops, shape, beta)
