@@ -1,8 +1,9 @@
 // Causal GQA attention for the decoder layers (Llama / Qwen), forward and
 // backward, flash-style: scores stay in registers, softmax is online in fp32,
 // operands go through the tensor cores as bf16 (mma.sync m16n8k16, fp32
-// accumulate).  At seq 512 attention is ~1% of a layer's FLOPs, so these are
-// plain tiled kernels rather than tcgen05 pipelines.
+// accumulate).  These serve every shape; at head dim 128 and up to 512
+// positions the forward and backward run on the tcgen05 kernels of
+// attention_tc.cu instead.
 //
 // Layouts: q, o [B, S, Hq, D]; k, v [B, S, Hkv, D]; lse [B, Hq, S] (natural
 // log of the sum of exp of the scaled scores).  Query head h reads kv head
@@ -567,6 +568,9 @@ extern "C" lsq_status lsq_attention_fwd(const void* q, const void* k, const void
     return fail(LSQ_EINVAL, "lsq_attention_fwd: alignment");
   lsq_status st = check_args("lsq_attention_fwd", batch, seq, hq, hkv, hd);
   if (st != LSQ_OK) return st;
+  // head dim 128 at up to 512 positions: the tcgen05 kernel (attention_tc.cu)
+  if (atc::fwd_supported(seq, hd))
+    return atc::run_fwd(q, k, v, o, lse, (int)batch, (int)seq, (int)hq, (int)hkv, (cudaStream_t)stream);
   if (hd == 64) return run_fwd<64>(q, k, v, o, lse, (int)batch, (int)seq, (int)hq, (int)hkv, (cudaStream_t)stream);
   return run_fwd<128>(q, k, v, o, lse, (int)batch, (int)seq, (int)hq, (int)hkv, (cudaStream_t)stream);
 }
@@ -594,6 +598,8 @@ extern "C" lsq_status lsq_attention_bwd(const void* q, const void* k, const void
   dvec_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, cs>>>((const __nv_bfloat16*)o, (const __nv_bfloat16*)d_o,
                                                                   dvec, rows, (int)seq, (int)hq, (int)hd);
   LSQ_LAUNCH_CHECK("attention dvec_kernel");
+  if (atc::bwd_supported(seq, hd))
+    return atc::run_bwd(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
   if (hd == 64)
     return run_bwd<64>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
   return run_bwd<128>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);

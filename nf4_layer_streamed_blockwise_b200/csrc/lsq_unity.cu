@@ -6,6 +6,7 @@
 #include "gemm_nf4.cu"
 #include "lora_grad.cu"
 #include "layer_ops.cu"
+#include "attention_tc.cu"
 #include "attention.cu"
 #include "stream.cu"
 #include "noalloc.cu"

@@ -9,7 +9,7 @@ import torch
 
 import synthetic as S
 from oracle import decoder as D
-from tolerances import assert_close, assert_close_ew
+from tolerances import assert_close, assert_close_ew, assert_close_rows
 
 pytestmark = pytest.mark.gpu
 F64 = torch.float64
@@ -88,7 +88,8 @@ def _attn_case(B, Sq, Hq, Hkv, hd, seed):
 
 
 @pytest.mark.parametrize("B,Sq,Hq,Hkv,hd", [(1, 512, 9, 3, 64), (2, 200, 4, 1, 128), (1, 64, 2, 2, 64),
-                                            (1, 1, 4, 2, 128), (2, 130, 8, 2, 128)])
+                                            (1, 1, 4, 2, 128), (2, 130, 8, 2, 128), (2, 512, 32, 8, 128),
+                                            (1, 384, 4, 4, 128)])
 def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
     q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, Sq)
     o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
@@ -108,13 +109,13 @@ def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
     sc = sc.masked_fill(torch.triu(torch.ones(Sq, Sq, dtype=torch.bool), 1), float("-inf"))
     assert_close(lse.cpu().numpy(), torch.logsumexp(sc, -1).numpy(), rel=1e-5, max_rms=1e-4, what="lse")
     # P and dS enter the tensor cores as bf16: relative error up to ~2^-8 per
-    # term.  With a single key the softmax gradient is exactly zero; the kernel
-    # leaves a residue of dP - D (two fp32 sums of the same products in
-    # different orders), about 1e-6 here.
-    kw = dict(rel=1e-2, ew_rel=2e-2, ew_abs_rms=5e-2, zero_atol=1e-4)
-    assert_close_ew(_np(dq), rq.numpy(), what="dq", **kw)
-    assert_close_ew(_np(dk), rk.numpy(), what="dk", **kw)
-    assert_close_ew(_np(dv), rv.numpy(), what="dv", **kw)
+    # term, so each gradient row (one position, one head) is checked against
+    # its own norm (tolerances.assert_close_rows).  With a single key the
+    # softmax gradient is exactly zero; the kernel leaves a residue of dP - D
+    # (two fp32 sums of the same products in different orders), about 1e-6.
+    assert_close_rows(_np(dq), rq.numpy(), what="dq")
+    assert_close_rows(_np(dk), rk.numpy(), what="dk")
+    assert_close_rows(_np(dv), rv.numpy(), what="dv")
 
 
 def test_attention_deterministic(lsq):
