@@ -24,5 +24,8 @@ independent inverse-normal routine; brute-force argmin on every element;
 the round trip deq o quant o deq == deq; B = 0 reduces LoRA to the base linear;
 central finite differences for every analytic gradient; S = 1 attention equals
 the V projection; RoPE at position 0 is the identity; the SmolLM2-135M
-parameter count the pages print; the loss at init near ln(V).
+parameter count the pages print; the loss at init near ln(V); for the
+double-quantised absmax, the E4M3 table and rounding against torch's
+float8_e4m3fn, exact round trips on representable blocks and the half-ulp
+error bound.
 """

@@ -150,3 +150,108 @@ def dequantize(packed: np.ndarray, absmax: np.ndarray, N: int, K: int) -> np.nda
 
 def dequantize_f64(packed: np.ndarray, absmax: np.ndarray, N: int, K: int) -> np.ndarray:
     return bf16_bits_to_f32(dequantize(packed, absmax, N, K)).astype(np.float64)
+
+
+# ------------------------------------------------------------------------
+# Double quantisation of the absmax array (8-bit second level).
+#
+# The pages give only its footprint: the 8B base store at 3.60 GB and layer
+# buffers of 113 MB ("Soup" README, layer-streaming figure caption and the
+# 8B row of its benchmark table), which is what 4-bit codes plus roughly one
+# byte per 64-element block come to, not the 4 bytes of an fp32 absmax.  The
+# construction is the QLoRA paper's "double quantization" (Dettmers et al.
+# 2023, sec. 3): the first-level constants are themselves quantised to 8-bit
+# floats in blocks of 256, after centring.  Readings taken where that text
+# leaves the details open:
+# * 8-bit float = E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+#   bits, exponent field 0 subnormal, no infinities, S.1111.111 the only NaN;
+#   largest finite 448);
+# * block = 256 consecutive absmax values of one tensor (row-major [N, K/64]
+#   flattened; the last block of a tensor may be shorter);
+# * centring and scale per block: centre = fp32(fp32(hi + lo) * 0.5), half =
+#   fp32(fp32(hi - lo) * 0.5), scale = fp32(half / 448) (lo, hi: the block's
+#   smallest and largest absmax), so the block's extremes land on -448 and
+#   +448;
+# * code = the E4M3 value nearest to fp32(fp32(a - centre) / scale), ties to
+#   the even code, magnitudes beyond 448 saturating to 448, a zero result
+#   stored as +0 (code 0); a block with scale 0 stores every code 0;
+# * expansion: a' = fp32(fp32(e4m3(code) * scale) + centre), two roundings.
+# ------------------------------------------------------------------------
+DQ_BLOCK = 256
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 bit pattern, from the field definitions."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def e4m3_table() -> np.ndarray:
+    """float64 [256]: the value of every code (NaN at 0x7F and 0xFF)."""
+    return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest E4M3 code to each fp32 value (brute force over the 127
+    non-negative finite codes, distances exact in fp64); ties go to the even
+    code; magnitudes above 448 end on 448 (the nearest finite value); a result
+    of zero is +0."""
+    x = np.asarray(x, dtype=np.float32).reshape(-1)
+    mags = e4m3_table()[:0x7F]                      # codes 0..126, increasing
+    # saturate first: every magnitude at or above 448 takes the largest finite code
+    # (this also keeps the distances below exact in fp64)
+    a = np.minimum(np.abs(x.astype(np.float64)), E4M3_MAX)
+    dist = np.abs(a[:, None] - mags[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    tied = dist == best
+    # among the (at most two, adjacent) nearest codes prefer the even one
+    even = tied & ((np.arange(0x7F) % 2) == 0)[None, :]
+    code = np.where(even.any(axis=1), even.argmax(axis=1), tied.argmax(axis=1)).astype(np.uint8)
+    neg = (x < 0) & (code != 0)
+    code[neg] |= 0x80
+    return code
+
+
+def double_quantize_absmax(absmax: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 absmax (any shape, row-major) -> (codes uint8 [n], params fp32
+    [ceil(n / 256), 2] holding (centre, scale) per block of 256)."""
+    a = np.asarray(absmax, dtype=np.float32).reshape(-1)
+    n = a.size
+    nblk = (n + DQ_BLOCK - 1) // DQ_BLOCK
+    codes = np.zeros(n, dtype=np.uint8)
+    params = np.zeros((nblk, 2), dtype=np.float32)
+    half_f, max_f = np.float32(0.5), np.float32(E4M3_MAX)
+    for b in range(nblk):
+        blk = a[b * DQ_BLOCK:(b + 1) * DQ_BLOCK]
+        lo, hi = blk.min(), blk.max()
+        centre = np.float32(np.float32(hi + lo) * half_f)
+        half = np.float32(np.float32(hi - lo) * half_f)
+        scale = np.float32(half / max_f)
+        params[b] = (centre, scale)
+        if scale != 0:
+            x = ((blk - centre).astype(np.float32) / scale).astype(np.float32)
+            codes[b * DQ_BLOCK:b * DQ_BLOCK + blk.size] = e4m3_round(x)
+    return codes, params
+
+
+def expand_absmax(codes: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """(codes, (centre, scale) per 256) -> fp32 absmax [n]: fp32(fp32(e4m3 * scale) + centre)."""
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    p = np.asarray(params, dtype=np.float32).reshape(-1, 2)
+    blk = np.arange(c.size) // DQ_BLOCK
+    v = e4m3_table()[c].astype(np.float32)           # exact: every E4M3 value is an fp32
+    prod = (v * p[blk, 1]).astype(np.float32)
+    return (prod + p[blk, 0]).astype(np.float32)
+
+
+def double_quantized(absmax: np.ndarray) -> np.ndarray:
+    """The absmax a double-quantised store hands to the dequantiser: expand(quantise(absmax)), same shape."""
+    am = np.asarray(absmax, dtype=np.float32)
+    return expand_absmax(*double_quantize_absmax(am)).reshape(am.shape)

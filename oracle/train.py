@@ -24,7 +24,9 @@ from . import nf4
 from .decoder import DPO_BETA, F64, adamw, model_dpo_loss_and_grads, model_loss_and_grads
 
 
-def dequantized_layer(Wbf16: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
+def dequantized_layer(Wbf16: Dict[str, torch.Tensor], double_quant: bool = False) -> Dict[str, torch.Tensor]:
+    """fp64 weights the layer computes with: NF4 quantise, then dequantise; with
+    double_quant the absmax array goes through its 8-bit second level first."""
     out = {}
     for name, w in Wbf16.items():
         if name in ("ln1", "ln2"):
@@ -33,6 +35,8 @@ def dequantized_layer(Wbf16: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]
         a = w.float().numpy()
         N, K = a.shape
         packed, am = nf4.quantize(a)
+        if double_quant:
+            am = nf4.double_quantized(am)
         out[name] = torch.from_numpy(nf4.dequantize_f64(packed, am, N, K))
     return out
 
@@ -43,9 +47,9 @@ def operand(master: torch.Tensor) -> torch.Tensor:
 
 
 def train(shape, layers_bf16, emb_bf16, lora_masters, ids_per_step: List[torch.Tensor],
-          lr: float = 2e-5):
+          lr: float = 2e-5, double_quant: bool = False):
     """Run len(ids_per_step) steps; returns (losses, grads of the first step, final masters)."""
-    layers = [dequantized_layer(W) for W in layers_bf16]
+    layers = [dequantized_layer(W, double_quant) for W in layers_bf16]
     emb = {k: v.to(F64) for k, v in emb_bf16.items()}
     masters = [{n: {ab: t[ab].detach().to(F64).clone() for ab in ("A", "B")} for n, t in per.items()}
                for per in lora_masters]
