@@ -62,6 +62,9 @@ def args_():
     p.add_argument("--dpo", action="store_true",
                    help="DPO over pairs of sequences with the adapter-off reference on the same streamed base")
     p.add_argument("--beta", type=float, default=0.1)
+    p.add_argument("--absmax", default="fp32", choices=["fp32", "dq8"],
+                   help="absmax format of the streamed records: fp32, or double-quantised (8-bit E4M3 codes, "
+                        "blocks of 256, expanded to fp32 in HBM after each upload)")
     return p.parse_args()
 
 
@@ -191,25 +194,33 @@ def reference_arm(a):
 def workload_config(a, shape):
     task = (f"DPO (beta {a.beta}, {a.batch // 2} chosen/rejected pairs, reference = the base with the adapters "
             f"off, run on each layer while it is resident)") if a.dpo else "causal-LM SFT"
-    store_gb = shape.n_layers * record_bytes(shape) / 1e9
-    return {"workload": f"{shape.name} shape, NF4 (bs64, fp32 absmax) base streamed from pinned host RAM through "
+    store_gb = shape.n_layers * record_bytes(shape, a.absmax) / 1e9
+    am = "fp32 absmax" if a.absmax == "fp32" else "double-quantised absmax: E4M3 codes, blocks of 256"
+    return {"workload": f"{shape.name} shape, NF4 (bs64, {am}) base streamed from pinned host RAM through "
                         f"{a.slots} HBM slots, grad checkpointing with re-stream, LoRA r={shape.r} on all linears, "
                         f"{task}, AdamW",
             "batch": a.batch, "seq_len": a.seq, "n_slots": a.slots, "parallelism": f"dp{a.gpus}",
             "l2": f"inputs larger than L2 ({store_gb:.2f} GB of layer records streamed per pass)"}
 
 
-def record_bytes(shape):
-    """Bytes of one streamed layer record: NF4 codes + fp32 absmax of the 7 linears + 2 RMSNorm gains."""
-    w = sum(n * k for n, k in shape.linear_shapes().values())
-    return w // 2 + w // 64 * 4 + 2 * shape.d * 2
+def record_bytes(shape, absmax="fp32"):
+    """Bytes of one streamed layer record: NF4 codes + absmax of the 7 linears + 2 RMSNorm gains
+    (fp32 absmax: 4 bytes per 64-weight block; double-quantised: 1 byte per block + 8 per 256 blocks)."""
+    lin = shape.linear_shapes().values()
+    w = sum(n * k for n, k in lin)
+    if absmax == "fp32":
+        am = w // 64 * 4
+    else:
+        am = sum(n * k // 64 + 8 * ((n * k // 64 + 255) // 256) for n, k in lin)
+    return w // 2 + am + 2 * shape.d * 2
 
 
 def metric_name(a, shape):
     task = "DPO train" if a.dpo else "train"
     short = {"llama-3.1-8b": "8B", "dense-32b": "32B", "qwen2.5-3b": "3B", "smollm2-135m": "135M"}.get(shape.name,
                                                                                                       shape.name)
-    return f"streamed NF4-LoRA {task} tok/s ({short} shape, seq {a.seq})"
+    dq = ", double-quantised absmax" if a.absmax == "dq8" else ""
+    return f"streamed NF4-LoRA {task} tok/s ({short} shape, seq {a.seq}{dq})"
 
 
 # ---------------------------------------------------------------------------- our arm
@@ -287,7 +298,7 @@ def our_arm(a):
     peaks, peaks_src = load_peaks()
 
     h2d = h2d_bandwidth(torch)
-    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device")
+    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", absmax=a.absmax)
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
         tr.set_ids(ids_list[i % 4])
@@ -349,7 +360,8 @@ def our_arm(a):
 
     # resident run on the same store: exposed copy time and peak HBM
     if not a.no_resident:
-        trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store)
+        trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store,
+                                  absmax=a.absmax)
         for i in range(2):
             trr.set_ids(ids_list[i % 4])
             step_fb(trr, a)
@@ -366,7 +378,7 @@ def our_arm(a):
 
     batch1 = None
     if not a.no_batch1 and a.batch != 1 and not a.dpo:
-        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store)
+        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store, absmax=a.absmax)
         ids1 = [t[:1] for t in ids_list]
         for i in range(2):
             tr1.train_step(ids1[i % 4])

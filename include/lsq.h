@@ -96,6 +96,36 @@ lsq_status lsq_nf4_quantize(const void* w_bf16, int64_t n_out, int64_t k_in, uin
 lsq_status lsq_nf4_dequantize(const lsq_nf4_weight* w, void* w_bf16, lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Double-quantised absmax (8-bit second level).
+ *
+ * Pages: the 8B base store is 3.60 GB and each layer buffer 113 MB ("Soup"
+ * README, layer-streaming figure and its benchmark table) - the size of 4-bit
+ * codes plus about one byte, not four, per 64-weight block.  Construction:
+ * QLoRA's double quantization (Dettmers et al. 2023, sec. 3: the absmax
+ * constants quantised again to 8-bit floats in blocks of 256, after
+ * centring).  Readings: the 8-bit float is E4M3 (bias 7, 3 mantissa bits,
+ * largest finite 448); per block of 256 consecutive absmax values of one
+ * tensor (the last block may be shorter), lo / hi = its smallest / largest
+ * value, centre = fp32(fp32(hi + lo) * 0.5), half = fp32(fp32(hi - lo) * 0.5),
+ * scale = fp32(half / 448); code = E4M3 nearest to fp32(fp32(a - centre) /
+ * scale), ties to even, saturating at +-448, zero stored as +0; scale 0
+ * stores code 0.  Expansion: a' = fp32(fp32(e4m3(code) * scale) + centre).
+ *
+ * lsq_absmax_double_quantize: absmax fp32 [nb] -> codes u8 [nb] and params
+ *   fp32 [ceil(nb/256)][2] = (centre, scale).  Device pointers; absmax 4-byte,
+ *   params 8-byte aligned.  Bit-exact with a CPU implementation of the
+ *   definition.  EINVAL on NULLs, nb < 1 or alignment.
+ * lsq_absmax_expand: codes + params -> absmax fp32 [nb] (the values the fused
+ *   GEMMs then read).  Same pointer rules.
+ * The streaming scheduler runs the expansion itself after each upload when
+ * given the record's layout (lsq_stream_set_absmax_expand).
+ * ---------------------------------------------------------------------- */
+lsq_status lsq_absmax_double_quantize(const float* absmax, int64_t nb, uint8_t* codes, float* params,
+                                      lsq_cuda_stream stream);
+lsq_status lsq_absmax_expand(const uint8_t* codes, const float* params, int64_t nb, float* absmax,
+                             lsq_cuda_stream stream);
+
+/* ------------------------------------------------------------------------
  * Fused NF4-dequant GEMM with LoRA, forward.
  *
  * Y = residual + X deq(W)^T + s (X A^T) B^T,   U = X A^T
@@ -304,6 +334,25 @@ lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stream compute,
  * slot's previous occupant, copy layer's record into the slot, record the
  * layer's upload event.  ESTATE if the slot holds the layer in current use. */
 lsq_status lsq_layer_upload_async(lsq_stream* st, int32_t layer, int32_t slot);
+/* One double-quantised absmax array of a layer record: byte offsets from the
+ * slot's start of its codes (u8 [nb]) and params (fp32 pairs, 8-byte
+ * aligned), both inside the record, and of the fp32 [nb] output, which lies
+ * past the record's end and within the slot (4-byte aligned). */
+typedef struct lsq_absmax_dq_item {
+  uint64_t codes_off;
+  uint64_t params_off;
+  uint64_t out_off;
+  int64_t nb;
+} lsq_absmax_dq_item;
+/* Records carry double-quantised absmax: after every upload the scheduler
+ * expands the n_items (0..8; 0 switches it off) arrays into fp32 inside the
+ * slot, on the copy stream, before the upload's event - compute sees the
+ * layer only once its fp32 absmax is in place.  slot_bytes: the size of every
+ * slot (the caller's allocations; >= the largest out_off + 4 nb).  Call before
+ * the first upload (ESTATE otherwise); EINVAL on bounds, alignment or
+ * overlapping outputs. */
+lsq_status lsq_stream_set_absmax_expand(lsq_stream* st, const lsq_absmax_dq_item* items, int32_t n_items,
+                                        size_t slot_bytes);
 /* Begin compute on `layer`, walking in `direction` (+1 forward, -1
  * backward): release the previously stepped layer's slot after the compute
  * work enqueued so far; upload `layer` if no slot holds it; make the compute

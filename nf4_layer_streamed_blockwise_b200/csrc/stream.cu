@@ -115,6 +115,11 @@ struct lsq_stream {
   std::vector<cudaEvent_t> up_start, up_done, slot_free;
   int64_t bytes = 0;
   std::vector<lsq::sched::Act> acts;
+  // double-quantised absmax: expanded to fp32 inside the slot after each upload
+  int n_expand = 0;
+  uint64_t ex_codes[8], ex_params[8], ex_out[8];
+  int64_t ex_nb[8];
+  int64_t expands = 0;
 };
 
 namespace lsq {
@@ -130,6 +135,12 @@ static lsq_status execute(lsq_stream* st) {
       LSQ_CUDA_TRY(cudaEventRecord(st->up_start[a.layer], st->copy));
       LSQ_CUDA_TRY(cudaMemcpyAsync(st->slots[a.slot], st->host[a.layer], st->record_bytes, cudaMemcpyHostToDevice,
                                    st->copy));
+      if (st->n_expand > 0) {
+        lsq_status s = dq::launch_expand(static_cast<const char*>(st->slots[a.slot]), st->ex_codes, st->ex_params,
+                                         st->ex_out, st->ex_nb, st->n_expand, st->copy);
+        if (s != LSQ_OK) return s;
+        st->expands += 1;
+      }
       LSQ_CUDA_TRY(cudaEventRecord(st->up_done[a.layer], st->copy));
       st->bytes += (int64_t)st->record_bytes;
     } else if (a.kind == WAIT) {
@@ -214,6 +225,34 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
     return cuda_fail(e, "lsq_stream_create: cudaEventCreate");
   }
   *out = st;
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_set_absmax_expand(lsq_stream* st, const lsq_absmax_dq_item* items,
+                                                  int32_t n_items, size_t slot_bytes) {
+  if (!st || (n_items > 0 && !items)) return fail(LSQ_EINVAL, "lsq_stream_set_absmax_expand: NULL argument");
+  if (n_items < 0 || n_items > 8) return fail(LSQ_EINVAL, "lsq_stream_set_absmax_expand: 0..8 items, got %d", n_items);
+  if (st->pol.uploads > 0) return fail(LSQ_ESTATE, "lsq_stream_set_absmax_expand: call before the first upload");
+  const uint64_t rec = st->record_bytes;
+  for (int k = 0; k < n_items; ++k) {
+    const lsq_absmax_dq_item& it = items[k];
+    const uint64_t nb = (uint64_t)it.nb, nblk = (nb + 255) / 256;
+    if (it.nb < 1 || it.codes_off + nb > rec || it.params_off % 8 || it.params_off + 8 * nblk > rec ||
+        it.out_off % 4 || it.out_off < rec || it.out_off + 4 * nb > slot_bytes)
+      return fail(LSQ_EINVAL,
+                  "lsq_stream_set_absmax_expand: item %d out of bounds (codes and params inside the record, "
+                  "params 8-byte aligned, output 4-byte aligned between the record's end and slot_bytes)", k);
+    for (int j = 0; j < k; ++j)
+      if (it.out_off < items[j].out_off + 4 * (uint64_t)items[j].nb && items[j].out_off < it.out_off + 4 * nb)
+        return fail(LSQ_EINVAL, "lsq_stream_set_absmax_expand: outputs of items %d and %d overlap", j, k);
+  }
+  st->n_expand = n_items;
+  for (int k = 0; k < n_items; ++k) {
+    st->ex_codes[k] = items[k].codes_off;
+    st->ex_params[k] = items[k].params_off;
+    st->ex_out[k] = items[k].out_off;
+    st->ex_nb[k] = items[k].nb;
+  }
   return LSQ_OK;
 }
 

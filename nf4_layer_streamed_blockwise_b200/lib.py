@@ -37,6 +37,11 @@ class lsq_nf4_weight(ctypes.Structure):
     _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
 
 
+class lsq_absmax_dq_item(ctypes.Structure):
+    _fields_ = [("codes_off", ctypes.c_uint64), ("params_off", ctypes.c_uint64), ("out_off", ctypes.c_uint64),
+                ("nb", c_int64)]
+
+
 class lsq_stream_cfg(ctypes.Structure):
     _fields_ = [("n_layers", c_int32), ("n_slots", c_int32), ("record_bytes", c_size_t),
                 ("slots", ctypes.POINTER(c_void_p)), ("host_records", ctypes.POINTER(c_void_p))]
@@ -54,6 +59,8 @@ _SIGS = {
     "lsq_nf4_codebook": (c_int32, [ctypes.POINTER(c_float)]),
     "lsq_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "lsq_nf4_dequantize": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p]),
+    "lsq_absmax_double_quantize": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "lsq_absmax_expand": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
     "lsq_nf4_lora_fwd_workspace_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
     "lsq_nf4_lora_fwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64, c_void_p, c_void_p, c_int32,
                                    c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -101,6 +108,7 @@ _SIGS = {
     "lsq_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_float,
                                  c_float, c_float, c_float, c_float, c_void_p]),
     "lsq_stream_create": (c_int32, [ctypes.POINTER(lsq_stream_cfg), c_void_p, c_void_p, ctypes.POINTER(c_void_p)]),
+    "lsq_stream_set_absmax_expand": (c_int32, [c_void_p, ctypes.POINTER(lsq_absmax_dq_item), c_int32, c_size_t]),
     "lsq_layer_upload_async": (c_int32, [c_void_p, c_int32, c_int32]),
     "lsq_stream_step": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_void_p)]),
     "lsq_stream_simulate": (c_int32, [c_int32, c_int32, c_int32, ctypes.POINTER(c_int32), ctypes.POINTER(c_int32),
@@ -143,7 +151,7 @@ def _check(name: str, status: int):
 # the split-K rank-r product, its reduction and the main GEMM; the backward is
 # those three, the dX GEMM when dx is wanted, and the dA/dB GEMM with its reduction)
 LAUNCHES = [0]
-_KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1,
+_KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_absmax_double_quantize": 1, "lsq_absmax_expand": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
             "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
             "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1, "lsq_seq_logprob": 2,
@@ -230,6 +238,15 @@ def lsq_nf4_quantize(w_bf16: torch.Tensor, codes: torch.Tensor, absmax: torch.Te
 def lsq_nf4_dequantize(w: NF4Weight, out_bf16: torch.Tensor, stream=None):
     cw = w.c()
     _call("lsq_nf4_dequantize", ctypes.byref(cw), _p(out_bf16), _stream(stream))
+
+
+def lsq_absmax_double_quantize(absmax, nb: int, codes, params, stream=None):
+    """absmax fp32 [nb] -> codes u8 [nb], params fp32 [ceil(nb/256), 2] (centre, scale); device memory."""
+    _call("lsq_absmax_double_quantize", _p(absmax), nb, _p(codes), _p(params), _stream(stream))
+
+
+def lsq_absmax_expand(codes, params, nb: int, absmax, stream=None):
+    _call("lsq_absmax_expand", _p(codes), _p(params), nb, _p(absmax), _stream(stream))
 
 
 def lsq_nf4_lora_fwd_workspace_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
@@ -395,13 +412,36 @@ def lsq_stream_create(n_layers: int, n_slots: int, record_bytes: int, slots: Seq
     return out.value
 
 
+_EXPANDING = set()  # schedulers that launch an absmax expansion after every upload
+
+
+def lsq_stream_set_absmax_expand(st: int, items, slot_bytes: int):
+    """items: [(codes_off, params_off, out_off, nb), ...] (byte offsets from a slot's start)."""
+    arr = (lsq_absmax_dq_item * max(len(items), 1))(*[lsq_absmax_dq_item(*it) for it in items])
+    _call("lsq_stream_set_absmax_expand", st, arr, len(items), slot_bytes)
+    if items:
+        _EXPANDING.add(st)
+    else:
+        _EXPANDING.discard(st)
+
+
+def _with_uploads(st: int, fn):
+    """run fn(); count the expansion kernels of the uploads it issued"""
+    if st not in _EXPANDING:
+        return fn()
+    before = lsq_stream_stats(st)[0]
+    out = fn()
+    LAUNCHES[0] += lsq_stream_stats(st)[0] - before
+    return out
+
+
 def lsq_layer_upload_async(st: int, layer: int, slot: int):
-    _call("lsq_layer_upload_async", st, layer, slot)
+    _with_uploads(st, lambda: _call("lsq_layer_upload_async", st, layer, slot))
 
 
 def lsq_stream_step(st: int, layer: int, direction: int) -> int:
     out = c_void_p()
-    _call("lsq_stream_step", st, layer, direction, ctypes.byref(out))
+    _with_uploads(st, lambda: _call("lsq_stream_step", st, layer, direction, ctypes.byref(out)))
     return out.value
 
 
@@ -434,4 +474,5 @@ def lsq_stream_reset(st: int):
 
 
 def lsq_stream_destroy(st: int):
+    _EXPANDING.discard(st)
     _call("lsq_stream_destroy", st)

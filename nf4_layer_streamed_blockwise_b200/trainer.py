@@ -14,7 +14,12 @@ the library in order.  Every arithmetic step runs in the library's kernels.
 
 Layer record layout (bytes, each piece 256-byte aligned): NF4 codes of
 q, k, v, o, gate, up, down; then their fp32 absmax arrays in the same order;
-then the two RMSNorm gains (bf16 [d] each).
+then the two RMSNorm gains (bf16 [d] each).  With double-quantised absmax
+(absmax="dq8") the record carries, instead of the fp32 arrays, each weight's
+8-bit absmax codes and its (centre, scale) pairs per 256 blocks; the slot is
+longer than the record by the fp32 arrays, which the scheduler expands into
+after each upload (the host link carries 112.5 MB instead of 122.7 MB per 8B
+layer).
 """
 from __future__ import annotations
 
@@ -36,28 +41,53 @@ def _al(n: int, a: int = ALIGN) -> int:
 
 @dataclasses.dataclass
 class RecordLayout:
-    """Byte offsets of one layer record."""
+    """Byte offsets of one layer record (and of the fp32 absmax the kernels read,
+    which lie past the record when it carries double-quantised absmax)."""
     codes: Dict[str, int]
     absmax: Dict[str, int]
     ln1: int
     ln2: int
-    nbytes: int
+    nbytes: int                    # bytes per record: what each upload copies
+    slot_bytes: int                # bytes per HBM slot
+    dq: Optional[Dict[str, tuple]] = None   # name -> (codes8 offset, params offset, n blocks)
 
     @staticmethod
-    def of(shape: S.ModelShape) -> "RecordLayout":
+    def of(shape: S.ModelShape, absmax: str = "fp32") -> "RecordLayout":
+        if absmax not in ("fp32", "dq8"):
+            raise ValueError(f"absmax must be 'fp32' or 'dq8', got {absmax!r}")
         off = 0
-        codes, absmax = {}, {}
-        for name, (n, k) in shape.linear_shapes().items():
+        codes, am, dq = {}, {}, {}
+        lin = shape.linear_shapes()
+        for name, (n, k) in lin.items():
             codes[name] = off
             off = _al(off + n * k // 2)
-        for name, (n, k) in shape.linear_shapes().items():
-            absmax[name] = off
-            off = _al(off + n * (k // 64) * 4)
+        for name, (n, k) in lin.items():
+            nb = n * (k // 64)
+            if absmax == "fp32":
+                am[name] = off
+                off = _al(off + nb * 4)
+            else:
+                c8 = off
+                off = _al(off + nb)
+                dq[name] = (c8, off, nb)
+                off = _al(off + 8 * ((nb + 255) // 256))
         ln1 = off
         off = _al(off + shape.d * 2)
         ln2 = off
         off = _al(off + shape.d * 2)
-        return RecordLayout(codes, absmax, ln1, ln2, _al(off, 4096))
+        nbytes = _al(off, 4096)
+        slot = nbytes
+        if absmax == "dq8":
+            for name, (n, k) in lin.items():
+                am[name] = slot
+                slot = _al(slot + n * (k // 64) * 4)
+        return RecordLayout(codes, am, ln1, ln2, nbytes, _al(slot, 4096), dq or None)
+
+    def expand_items(self):
+        """(codes8, params, fp32 out, n blocks) per weight, for the scheduler."""
+        if not self.dq:
+            return []
+        return [(c8, pp, self.absmax[name], nb) for name, (c8, pp, nb) in self.dq.items()]
 
 
 class LayerView:
@@ -128,7 +158,8 @@ class StreamedLoraTrainer:
     """
 
     def __init__(self, shape: S.ModelShape, batch: int, seq: int, n_slots: Optional[int] = 2,
-                 init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None):
+                 init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None,
+                 absmax: str = "fp32"):
         self.shape, self.B, self.S = shape, batch, seq
         self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
         self.M = batch * seq
@@ -136,9 +167,12 @@ class StreamedLoraTrainer:
         self.dev = device
         self.resident = n_slots is None
         self.n_slots = shape.n_layers if self.resident else int(n_slots)
-        self.layout = RecordLayout.of(shape)
+        self.layout = RecordLayout.of(shape, absmax)
+        self.absmax_kind = absmax
         self.compute = torch.cuda.current_stream()
         self.copy = torch.cuda.Stream()
+        if share is not None and share.absmax_kind != absmax:
+            raise ValueError("a shared host store must have the same absmax format")
         if share is not None:       # reuse another trainer's host store and resident tensors
             self.host_records = share.host_records
             self.embed, self.lm_head, self.final_norm = share.embed, share.lm_head, share.final_norm
@@ -151,10 +185,13 @@ class StreamedLoraTrainer:
         else:
             self.lora.init_device()
         self._alloc_activations()
-        self.slots = [torch.empty(self.layout.nbytes, dtype=torch.uint8, device=device) for _ in range(self.n_slots)]
+        self.slots = [torch.empty(self.layout.slot_bytes, dtype=torch.uint8, device=device)
+                      for _ in range(self.n_slots)]
         self.sched = L.lsq_stream_create(shape.n_layers, self.n_slots, self.layout.nbytes,
                                          [s.data_ptr() for s in self.slots],
                                          [h.data_ptr() for h in self.host_records], self.compute, self.copy)
+        if self.layout.dq:
+            L.lsq_stream_set_absmax_expand(self.sched, self.layout.expand_items(), self.layout.slot_bytes)
         if self.resident:
             for l in range(shape.n_layers):
                 L.lsq_layer_upload_async(self.sched, l, l)
@@ -165,7 +202,7 @@ class StreamedLoraTrainer:
     def _build_store(self, init: str):
         """Quantise every layer once on the GPU and keep the records pinned on the host."""
         sh, lay = self.shape, self.layout
-        stage = torch.zeros(lay.nbytes, dtype=torch.uint8, device=self.dev)
+        stage = torch.zeros(lay.slot_bytes, dtype=torch.uint8, device=self.dev)
         base = stage.data_ptr()
         self.host_records: List[torch.Tensor] = []
         for l in range(sh.n_layers):
@@ -177,12 +214,15 @@ class StreamedLoraTrainer:
                 else:
                     w = S.device_normal_bf16((n, k), S.BASE_STD, S.WEIGHT_SEED, 1000 + 16 * l + i)
                 L.lsq_nf4_quantize(w, base + lay.codes[name], base + lay.absmax[name])
+                if lay.dq:   # second level: the record keeps the 8-bit codes and block params
+                    c8, pp, nb = lay.dq[name]
+                    L.lsq_absmax_double_quantize(base + lay.absmax[name], nb, base + c8, base + pp)
                 del w
             ones = torch.ones(sh.d, dtype=torch.bfloat16, device=self.dev)
             stage[lay.ln1:lay.ln1 + 2 * sh.d].copy_(ones.view(torch.uint8))
             stage[lay.ln2:lay.ln2 + 2 * sh.d].copy_(ones.view(torch.uint8))
             rec = torch.empty(lay.nbytes, dtype=torch.uint8, pin_memory=True)
-            rec.copy_(stage)
+            rec.copy_(stage[:lay.nbytes])
             self.host_records.append(rec)
         del stage
         torch.cuda.synchronize()

@@ -102,3 +102,32 @@ def test_bad_arguments():
         lib.lsq_stream_simulate(4, 2, [(4, 1)])
     with pytest.raises(lib.LsqError):
         lib.lsq_stream_simulate(4, 2, [(0, 0)])
+
+
+@pytest.mark.parametrize("name", ["tiny", "smollm2-135m", "llama-3.1-8b", "dense-32b"])
+def test_record_layout_double_quant(name):
+    """The double-quantised record: smaller than the fp32 one by 3 bytes per block
+    (less the params), every piece aligned and disjoint, the expanded fp32
+    arrays after the record inside the slot, and the byte count bench.py reports."""
+    import bench
+    import synthetic as S
+    from nf4_layer_streamed_blockwise_b200.trainer import RecordLayout
+    sh = S.SHAPES[name]
+    f, q = RecordLayout.of(sh, "fp32"), RecordLayout.of(sh, "dq8")
+    assert f.slot_bytes == f.nbytes and f.dq is None
+    assert q.nbytes < f.nbytes and q.slot_bytes > q.nbytes
+    assert abs(q.nbytes - bench.record_bytes(sh, "dq8")) < 64 * 256       # alignment padding only
+    spans = [(q.codes[n], q.codes[n] + a * b // 2) for n, (a, b) in sh.linear_shapes().items()]
+    spans += [(c8, c8 + nb) for c8, _, nb in q.dq.values()]
+    spans += [(pp, pp + 8 * ((nb + 255) // 256)) for _, pp, nb in q.dq.values()]
+    spans += [(q.ln1, q.ln1 + 2 * sh.d), (q.ln2, q.ln2 + 2 * sh.d)]
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])) and spans[-1][1] <= q.nbytes
+    assert all(s % 256 == 0 for s, _ in spans)
+    outs = sorted((o, o + 4 * nb) for _, _, o, nb in q.expand_items())
+    assert outs[0][0] >= q.nbytes and outs[-1][1] <= q.slot_bytes
+    assert all(a[1] <= b[0] for a, b in zip(outs, outs[1:]))
+    if name == "llama-3.1-8b":
+        assert abs(q.nbytes / 1e6 - 112.5) < 0.2 and abs(f.nbytes / 1e6 - 122.7) < 0.1
+    with pytest.raises(ValueError):
+        RecordLayout.of(sh, "int8")
