@@ -62,6 +62,10 @@ def args_():
     p.add_argument("--dpo", action="store_true",
                    help="DPO over pairs of sequences with the adapter-off reference on the same streamed base")
     p.add_argument("--beta", type=float, default=0.1)
+    p.add_argument("--upload", default="auto", choices=["auto", "replicated", "sharded"],
+                   help="with several GPUs: every rank streams whole records over its own host link "
+                        "(replicated), or each rank copies 1/N of every record and an NCCL all-gather over "
+                        "NVLink completes the slot (sharded; the default when N > 1)")
     p.add_argument("--absmax", default="fp32", choices=["fp32", "dq8"],
                    help="absmax format of the streamed records: fp32, or double-quantised (8-bit E4M3 codes, "
                         "blocks of 256, expanded to fp32 in HBM after each upload)")
@@ -200,6 +204,7 @@ def workload_config(a, shape):
                         f"{a.slots} HBM slots, grad checkpointing with re-stream, LoRA r={shape.r} on all linears, "
                         f"{task}, AdamW",
             "batch": a.batch, "seq_len": a.seq, "n_slots": a.slots, "parallelism": f"dp{a.gpus}",
+            "upload": a.upload if a.upload != "auto" else ("sharded" if a.gpus > 1 else "replicated"),
             "l2": f"inputs larger than L2 ({store_gb:.2f} GB of layer records streamed per pass)"}
 
 
@@ -298,7 +303,10 @@ def our_arm(a):
     peaks, peaks_src = load_peaks()
 
     h2d = h2d_bandwidth(torch)
-    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", absmax=a.absmax)
+    sharded = a.upload == "sharded" or (a.upload == "auto" and world > 1)
+    a.upload = "sharded" if sharded else "replicated"
+    shard = (rank, world) if sharded else None
+    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", absmax=a.absmax, shard=shard)
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
         tr.set_ids(ids_list[i % 4])
@@ -361,7 +369,7 @@ def our_arm(a):
     # resident run on the same store: exposed copy time and peak HBM
     if not a.no_resident:
         trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store,
-                                  absmax=a.absmax)
+                                  absmax=a.absmax, shard=shard)
         for i in range(2):
             trr.set_ids(ids_list[i % 4])
             step_fb(trr, a)
@@ -378,7 +386,8 @@ def our_arm(a):
 
     batch1 = None
     if not a.no_batch1 and a.batch != 1 and not a.dpo:
-        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store, absmax=a.absmax)
+        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store, absmax=a.absmax,
+                                  shard=shard)
         ids1 = [t[:1] for t in ids_list]
         for i in range(2):
             tr1.train_step(ids1[i % 4])

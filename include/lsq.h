@@ -46,7 +46,8 @@ typedef enum lsq_status {
   LSQ_ECUDA = 3,        /* a CUDA runtime call failed (message in lsq_last_error) */
   LSQ_ETIMEOUT = 4,     /* a bounded device wait expired */
   LSQ_ESTATE = 5,       /* call out of order (stream scheduler) */
-  LSQ_EUNSUPPORTED = 6  /* device is not sm_100 or a limit of this build */
+  LSQ_EUNSUPPORTED = 6, /* device is not sm_100 or a limit of this build */
+  LSQ_ECALLBACK = 7     /* a caller-supplied callback reported failure */
 } lsq_status;
 
 /* Static message for a status code. */
@@ -318,16 +319,36 @@ lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_
  * ---------------------------------------------------------------------- */
 typedef struct lsq_stream lsq_stream;
 
+/* Sharded upload (several GPUs, one process each, training data-parallel on
+ * the same frozen base): rank r of W holds only bytes [r S, (r + 1) S) of
+ * every record (S = record_bytes / W) in its page-locked store and copies
+ * only those into the slot, at the same offset; the gather callback then
+ * completes the slot from the other ranks (an all-gather over NVLink),
+ * enqueued on `copy` after this rank's copy and before the upload's event.
+ * Each GPU's host link carries 1/W of the bytes, and the node pins the store
+ * once instead of once per rank.  The callback must return 0 on success; the
+ * scheduler calls it for every upload, in the policy's order, which is the
+ * same on every rank given the same sequence of steps. */
+typedef int32_t (*lsq_gather_fn)(void* user, int32_t layer, int32_t slot, void* slot_ptr, size_t record_bytes,
+                                 lsq_cuda_stream copy);
+
 typedef struct lsq_stream_cfg {
   int32_t n_layers;                  /* >= 1 */
   int32_t n_slots;                   /* 2..8 (or n_layers for a resident run) */
-  size_t record_bytes;               /* bytes per layer record, > 0 */
+  size_t record_bytes;               /* bytes per layer record, > 0, a multiple of 256 x max(1, shard_world) */
   void* const* slots;                /* n_slots device pointers, 256-byte aligned, >= record_bytes each */
-  const void* const* host_records;   /* n_layers host pointers, page-locked */
+  const void* const* host_records;   /* n_layers host pointers, page-locked; with sharding each points
+                                        at this rank's record_bytes / shard_world bytes */
+  int32_t shard_rank;                /* sharded upload: this rank, 0 <= shard_rank < shard_world */
+  int32_t shard_world;               /* ranks sharing each record; record_bytes % (256 shard_world) == 0 */
+  lsq_gather_fn gather;              /* NULL: no sharding (shard_rank 0, shard_world 0 or 1) */
+  void* gather_user;                 /* passed to gather */
 } lsq_stream_cfg;
 
 /* Creates the scheduler; ENOTPINNED if any record is not page-locked (the
- * pages fall back to pageable memory silently; here it is an error). */
+ * pages fall back to pageable memory silently; here it is an error).  Upload
+ * calls that run the gather callback return ECALLBACK if it fails (the slot
+ * is then incomplete: destroy the scheduler). */
 lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stream compute, lsq_cuda_stream copy,
                              lsq_stream** out);
 /* Enqueue on the copy stream: wait until the compute stream is done with the

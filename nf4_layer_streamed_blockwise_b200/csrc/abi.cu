@@ -188,6 +188,7 @@ const char* lsq_status_str(lsq_status s) {
     case LSQ_ETIMEOUT: return "device wait timed out";
     case LSQ_ESTATE: return "call out of order";
     case LSQ_EUNSUPPORTED: return "unsupported device or size";
+    case LSQ_ECALLBACK: return "a caller-supplied callback failed";
   }
   return "unknown status";
 }

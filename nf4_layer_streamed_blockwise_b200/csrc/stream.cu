@@ -108,6 +108,11 @@ struct Policy {
 struct lsq_stream {
   lsq::sched::Policy pol;
   size_t record_bytes = 0;
+  // sharded upload: this rank copies shard_bytes at shard_rank * shard_bytes; gather completes the slot
+  size_t shard_bytes = 0;
+  int shard_rank = 0;
+  lsq_gather_fn gather = nullptr;
+  void* gather_user = nullptr;
   std::vector<void*> slots;
   std::vector<const void*> host;
   cudaStream_t compute = nullptr, copy = nullptr;
@@ -133,8 +138,13 @@ static lsq_status execute(lsq_stream* st) {
     } else if (a.kind == UPLOAD) {
       if (st->free_recorded[a.slot]) LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[a.slot], 0));
       LSQ_CUDA_TRY(cudaEventRecord(st->up_start[a.layer], st->copy));
-      LSQ_CUDA_TRY(cudaMemcpyAsync(st->slots[a.slot], st->host[a.layer], st->record_bytes, cudaMemcpyHostToDevice,
-                                   st->copy));
+      char* dst = static_cast<char*>(st->slots[a.slot]) + (size_t)st->shard_rank * st->shard_bytes;
+      LSQ_CUDA_TRY(cudaMemcpyAsync(dst, st->host[a.layer], st->shard_bytes, cudaMemcpyHostToDevice, st->copy));
+      if (st->gather) {
+        const int32_t rc = st->gather(st->gather_user, a.layer, a.slot, st->slots[a.slot], st->record_bytes,
+                                      (lsq_cuda_stream)st->copy);
+        if (rc != 0) return fail(LSQ_ECALLBACK, "gather callback returned %d for layer %d", rc, a.layer);
+      }
       if (st->n_expand > 0) {
         lsq_status s = dq::launch_expand(static_cast<const char*>(st->slots[a.slot]), st->ex_codes, st->ex_params,
                                          st->ex_out, st->ex_nb, st->n_expand, st->copy);
@@ -142,7 +152,7 @@ static lsq_status execute(lsq_stream* st) {
         st->expands += 1;
       }
       LSQ_CUDA_TRY(cudaEventRecord(st->up_done[a.layer], st->copy));
-      st->bytes += (int64_t)st->record_bytes;
+      st->bytes += (int64_t)st->shard_bytes;
     } else if (a.kind == WAIT) {
       LSQ_CUDA_TRY(cudaStreamWaitEvent(st->compute, st->up_done[a.layer], 0));
     }
@@ -195,15 +205,26 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
       return fail(LSQ_EINVAL, "lsq_stream_create: slot %d is not a 256-byte aligned device pointer", i);
     }
   }
+  const int world = cfg->shard_world > 1 ? cfg->shard_world : 1;
+  if (cfg->shard_world < 0 || cfg->shard_rank < 0 || cfg->shard_rank >= world)
+    return fail(LSQ_EINVAL, "lsq_stream_create: shard rank %d of %d", cfg->shard_rank, cfg->shard_world);
+  if (world > 1 && !cfg->gather) return fail(LSQ_EINVAL, "lsq_stream_create: sharded upload needs a gather callback");
+  if (cfg->record_bytes % (256 * (size_t)world) != 0)
+    return fail(LSQ_EINVAL, "lsq_stream_create: record_bytes must be a multiple of 256 x shard_world");
+  const size_t shard = cfg->record_bytes / world;
   for (int l = 0; l < cfg->n_layers; ++l) {
     const char* h = static_cast<const char*>(cfg->host_records[l]);
     if (!h) return fail(LSQ_EINVAL, "lsq_stream_create: record %d is NULL", l);
-    if (!is_pinned_host(h) || !is_pinned_host(h + cfg->record_bytes - 1))
+    if (!is_pinned_host(h) || !is_pinned_host(h + shard - 1))
       return fail(LSQ_ENOTPINNED, "lsq_stream_create: record %d is not page-locked host memory", l);
   }
   lsq_stream* st = new lsq_stream();
   st->pol.init(cfg->n_layers, cfg->n_slots);
   st->record_bytes = cfg->record_bytes;
+  st->shard_bytes = shard;
+  st->shard_rank = cfg->shard_rank;
+  st->gather = cfg->gather;
+  st->gather_user = cfg->gather_user;
   st->slots.assign(cfg->slots, cfg->slots + cfg->n_slots);
   st->host.assign(cfg->host_records, cfg->host_records + cfg->n_layers);
   st->compute = (cudaStream_t)compute;

@@ -24,7 +24,7 @@ c_float = ctypes.c_float
 c_size_t = ctypes.c_size_t
 
 STATUS = {0: "LSQ_OK", 1: "LSQ_EINVAL", 2: "LSQ_ENOTPINNED", 3: "LSQ_ECUDA", 4: "LSQ_ETIMEOUT",
-          5: "LSQ_ESTATE", 6: "LSQ_EUNSUPPORTED"}
+          5: "LSQ_ESTATE", 6: "LSQ_EUNSUPPORTED", 7: "LSQ_ECALLBACK"}
 
 
 class LsqError(RuntimeError):
@@ -42,9 +42,15 @@ class lsq_absmax_dq_item(ctypes.Structure):
                 ("nb", c_int64)]
 
 
+# int32 gather(void* user, int32 layer, int32 slot, void* slot_ptr, size_t record_bytes, cudaStream_t copy)
+lsq_gather_fn = ctypes.CFUNCTYPE(c_int32, c_void_p, c_int32, c_int32, c_void_p, c_size_t, c_void_p)
+
+
 class lsq_stream_cfg(ctypes.Structure):
     _fields_ = [("n_layers", c_int32), ("n_slots", c_int32), ("record_bytes", c_size_t),
-                ("slots", ctypes.POINTER(c_void_p)), ("host_records", ctypes.POINTER(c_void_p))]
+                ("slots", ctypes.POINTER(c_void_p)), ("host_records", ctypes.POINTER(c_void_p)),
+                ("shard_rank", c_int32), ("shard_world", c_int32), ("gather", lsq_gather_fn),
+                ("gather_user", c_void_p)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -402,13 +408,35 @@ def lsq_adamw_step(p, g, m, v, p_bf16, n: int, step: int, lr: float, beta1: floa
 
 
 # ---------------------------------------------------------------------------- streaming
+_GATHERS = {}  # scheduler handle -> its ctypes callback (kept alive while the scheduler lives)
+
+
 def lsq_stream_create(n_layers: int, n_slots: int, record_bytes: int, slots: Sequence[int],
-                      host_records: Sequence[int], compute_stream, copy_stream) -> int:
+                      host_records: Sequence[int], compute_stream, copy_stream, shard=None) -> int:
+    """shard: None, or (rank, world, gather) for the sharded upload, where
+    gather(layer, slot, slot_ptr, record_bytes, copy_stream_handle) enqueues the
+    completion of the slot on the copy stream (an all-gather) and raises on failure."""
     sl = (c_void_p * len(slots))(*[_p(s) for s in slots])
     hr = (c_void_p * len(host_records))(*[_p(h) for h in host_records])
-    cfg = lsq_stream_cfg(n_layers, n_slots, record_bytes, sl, hr)
+    cb = lsq_gather_fn()
+    rank = world = 0
+    if shard is not None:
+        rank, world, fn = shard
+
+        def _gather(user, layer, slot, slot_ptr, nbytes, stream):
+            try:
+                fn(int(layer), int(slot), int(slot_ptr or 0), int(nbytes), int(stream or 0))
+                return 0
+            except Exception as e:  # reported through the scheduler's status
+                import sys
+                print(f"lsq gather callback failed: {e!r}", file=sys.stderr)
+                return 1
+        cb = lsq_gather_fn(_gather)
+    cfg = lsq_stream_cfg(n_layers, n_slots, record_bytes, sl, hr, rank, world, cb, None)
     out = c_void_p()
     _call("lsq_stream_create", ctypes.byref(cfg), _stream(compute_stream), _stream(copy_stream), ctypes.byref(out))
+    if shard is not None:
+        _GATHERS[out.value] = cb
     return out.value
 
 
@@ -476,3 +504,4 @@ def lsq_stream_reset(st: int):
 def lsq_stream_destroy(st: int):
     _EXPANDING.discard(st)
     _call("lsq_stream_destroy", st)
+    _GATHERS.pop(st, None)

@@ -30,6 +30,7 @@ from typing import Dict, List, Optional
 import torch
 
 import synthetic as S
+from . import dist as DP
 from . import lib as L
 
 ALIGN = 256
@@ -52,7 +53,7 @@ class RecordLayout:
     dq: Optional[Dict[str, tuple]] = None   # name -> (codes8 offset, params offset, n blocks)
 
     @staticmethod
-    def of(shape: S.ModelShape, absmax: str = "fp32") -> "RecordLayout":
+    def of(shape: S.ModelShape, absmax: str = "fp32", record_align: int = 4096) -> "RecordLayout":
         if absmax not in ("fp32", "dq8"):
             raise ValueError(f"absmax must be 'fp32' or 'dq8', got {absmax!r}")
         off = 0
@@ -75,13 +76,13 @@ class RecordLayout:
         off = _al(off + shape.d * 2)
         ln2 = off
         off = _al(off + shape.d * 2)
-        nbytes = _al(off, 4096)
+        nbytes = _al(off, record_align)
         slot = nbytes
         if absmax == "dq8":
             for name, (n, k) in lin.items():
                 am[name] = slot
                 slot = _al(slot + n * (k // 64) * 4)
-        return RecordLayout(codes, am, ln1, ln2, nbytes, _al(slot, 4096), dq or None)
+        return RecordLayout(codes, am, ln1, ln2, nbytes, _al(slot, record_align), dq or None)
 
     def expand_items(self):
         """(codes8, params, fp32 out, n blocks) per weight, for the scheduler."""
@@ -159,7 +160,7 @@ class StreamedLoraTrainer:
 
     def __init__(self, shape: S.ModelShape, batch: int, seq: int, n_slots: Optional[int] = 2,
                  init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None,
-                 absmax: str = "fp32"):
+                 absmax: str = "fp32", shard: Optional[tuple] = None):
         self.shape, self.B, self.S = shape, batch, seq
         self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
         self.M = batch * seq
@@ -167,12 +168,16 @@ class StreamedLoraTrainer:
         self.dev = device
         self.resident = n_slots is None
         self.n_slots = shape.n_layers if self.resident else int(n_slots)
-        self.layout = RecordLayout.of(shape, absmax)
+        # shard = (rank, world): sharded upload over the default process group (each rank
+        # pins and copies 1/world of every record; an all-gather completes the slot)
+        self.shard = None if shard is None else (int(shard[0]), int(shard[1]))
+        align = 4096 if self.shard is None else math.lcm(4096, 256 * self.shard[1])
+        self.layout = RecordLayout.of(shape, absmax, align)
         self.absmax_kind = absmax
         self.compute = torch.cuda.current_stream()
         self.copy = torch.cuda.Stream()
-        if share is not None and share.absmax_kind != absmax:
-            raise ValueError("a shared host store must have the same absmax format")
+        if share is not None and (share.absmax_kind != absmax or share.shard != self.shard):
+            raise ValueError("a shared host store must have the same absmax format and sharding")
         if share is not None:       # reuse another trainer's host store and resident tensors
             self.host_records = share.host_records
             self.embed, self.lm_head, self.final_norm = share.embed, share.lm_head, share.final_norm
@@ -189,7 +194,8 @@ class StreamedLoraTrainer:
                       for _ in range(self.n_slots)]
         self.sched = L.lsq_stream_create(shape.n_layers, self.n_slots, self.layout.nbytes,
                                          [s.data_ptr() for s in self.slots],
-                                         [h.data_ptr() for h in self.host_records], self.compute, self.copy)
+                                         [h.data_ptr() for h in self.host_records], self.compute, self.copy,
+                                         shard=None if self.shard is None else (*self.shard, lambda *a: self._gather(*a)))
         if self.layout.dq:
             L.lsq_stream_set_absmax_expand(self.sched, self.layout.expand_items(), self.layout.slot_bytes)
         if self.resident:
@@ -199,6 +205,20 @@ class StreamedLoraTrainer:
         self.loss_dev = torch.zeros(1, dtype=torch.float32, device=device)
 
     # ------------------------------------------------------------------ setup
+    def shard_range(self):
+        """Bytes of every record this rank pins and copies: [lo, hi)."""
+        if self.shard is None:
+            return 0, self.layout.nbytes
+        return DP.shard_range(self.layout.nbytes, *self.shard)
+
+    def _gather(self, layer, slot, slot_ptr, nbytes, stream_handle):
+        """Sharded upload: after this rank's part of the record landed in the slot
+        (on the copy stream), complete the slot from the other ranks - an in-place
+        all-gather over the default process group, ordered on the copy stream."""
+        t = self.slots[slot]
+        assert t.data_ptr() == slot_ptr and stream_handle == self.copy.cuda_stream and nbytes == self.layout.nbytes
+        DP.gather_slot(t, nbytes, *self.shard, stream=self.copy)
+
     def _build_store(self, init: str):
         """Quantise every layer once on the GPU and keep the records pinned on the host."""
         sh, lay = self.shape, self.layout
@@ -221,8 +241,9 @@ class StreamedLoraTrainer:
             ones = torch.ones(sh.d, dtype=torch.bfloat16, device=self.dev)
             stage[lay.ln1:lay.ln1 + 2 * sh.d].copy_(ones.view(torch.uint8))
             stage[lay.ln2:lay.ln2 + 2 * sh.d].copy_(ones.view(torch.uint8))
-            rec = torch.empty(lay.nbytes, dtype=torch.uint8, pin_memory=True)
-            rec.copy_(stage[:lay.nbytes])
+            lo, hi = self.shard_range()
+            rec = torch.empty(hi - lo, dtype=torch.uint8, pin_memory=True)
+            rec.copy_(stage[lo:hi])
             self.host_records.append(rec)
         del stage
         torch.cuda.synchronize()
