@@ -66,6 +66,14 @@ def args_():
                    help="with several GPUs: every rank streams whole records over its own host link "
                         "(replicated), or each rank copies 1/N of every record and an NCCL all-gather over "
                         "NVLink completes the slot (sharded; the default when N > 1)")
+    p.add_argument("--source", default="ram", choices=["ram", "disk"],
+                   help="where the layer records live: page-locked RAM, or a store file read by the library's "
+                        "reader threads through page-locked staging buffers")
+    p.add_argument("--store-path", default=None,
+                   help="store file for --source disk (default: a file in the system temp directory, removed "
+                        "at exit)")
+    p.add_argument("--embed", default="hbm", choices=["hbm", "host"],
+                   help="untied embedding table in HBM, or in page-locked host RAM read in place by the gather")
     p.add_argument("--absmax", default="fp32", choices=["fp32", "dq8"],
                    help="absmax format of the streamed records: fp32, or double-quantised (8-bit E4M3 codes, "
                         "blocks of 256, expanded to fp32 in HBM after each upload)")
@@ -200,7 +208,9 @@ def workload_config(a, shape):
             f"off, run on each layer while it is resident)") if a.dpo else "causal-LM SFT"
     store_gb = shape.n_layers * record_bytes(shape, a.absmax) / 1e9
     am = "fp32 absmax" if a.absmax == "fp32" else "double-quantised absmax: E4M3 codes, blocks of 256"
-    return {"workload": f"{shape.name} shape, NF4 (bs64, {am}) base streamed from pinned host RAM through "
+    src = "pinned host RAM" if a.source == "ram" else "a store file (disk tier: reader threads, pinned staging)"
+    emb = "" if a.embed == "hbm" else ", embedding table in pinned host RAM (zero-copy gather)"
+    return {"workload": f"{shape.name} shape, NF4 (bs64, {am}) base streamed from {src}{emb} through "
                         f"{a.slots} HBM slots, grad checkpointing with re-stream, LoRA r={shape.r} on all linears, "
                         f"{task}, AdamW",
             "batch": a.batch, "seq_len": a.seq, "n_slots": a.slots, "parallelism": f"dp{a.gpus}",
@@ -225,6 +235,8 @@ def metric_name(a, shape):
     short = {"llama-3.1-8b": "8B", "dense-32b": "32B", "qwen2.5-3b": "3B", "smollm2-135m": "135M"}.get(shape.name,
                                                                                                       shape.name)
     dq = ", double-quantised absmax" if a.absmax == "dq8" else ""
+    dq += ", disk tier" if a.source == "disk" else ""
+    dq += ", host embedding" if a.embed == "host" else ""
     return f"streamed NF4-LoRA {task} tok/s ({short} shape, seq {a.seq}{dq})"
 
 
@@ -306,7 +318,13 @@ def our_arm(a):
     sharded = a.upload == "sharded" or (a.upload == "auto" and world > 1)
     a.upload = "sharded" if sharded else "replicated"
     shard = (rank, world) if sharded else None
-    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", absmax=a.absmax, shard=shard)
+    store_path = None
+    if a.source == "disk":
+        store_path = a.store_path or os.path.join(tempfile.gettempdir(), f"lsq_store_{os.getpid()}_r{rank}.bin")
+        if a.store_path and world > 1:
+            store_path = f"{a.store_path}.rank{rank}"
+    tiers = dict(absmax=a.absmax, shard=shard, source=a.source, store_path=store_path, embed=a.embed)
+    tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", **tiers)
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
         tr.set_ids(ids_list[i % 4])
@@ -368,8 +386,7 @@ def our_arm(a):
 
     # resident run on the same store: exposed copy time and peak HBM
     if not a.no_resident:
-        trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store,
-                                  absmax=a.absmax, shard=shard)
+        trr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=None, init="device", share=store, **tiers)
         for i in range(2):
             trr.set_ids(ids_list[i % 4])
             step_fb(trr, a)
@@ -386,8 +403,7 @@ def our_arm(a):
 
     batch1 = None
     if not a.no_batch1 and a.batch != 1 and not a.dpo:
-        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store, absmax=a.absmax,
-                                  shard=shard)
+        tr1 = StreamedLoraTrainer(shape, 1, a.seq, n_slots=a.slots, init="device", share=store, **tiers)
         ids1 = [t[:1] for t in ids_list]
         for i in range(2):
             tr1.train_step(ids1[i % 4])
@@ -426,6 +442,8 @@ def our_arm(a):
         if batch1:
             line["batch1"] = batch1
         print(json.dumps(line), flush=True)
+    if store_path and not a.store_path:
+        os.remove(store_path)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

@@ -338,11 +338,22 @@ typedef struct lsq_stream_cfg {
   size_t record_bytes;               /* bytes per layer record, > 0, a multiple of 256 x max(1, shard_world) */
   void* const* slots;                /* n_slots device pointers, 256-byte aligned, >= record_bytes each */
   const void* const* host_records;   /* n_layers host pointers, page-locked; with sharding each points
-                                        at this rank's record_bytes / shard_world bytes */
+                                        at this rank's record_bytes / shard_world bytes; NULL with disk_path */
   int32_t shard_rank;                /* sharded upload: this rank, 0 <= shard_rank < shard_world */
   int32_t shard_world;               /* ranks sharing each record; record_bytes % (256 shard_world) == 0 */
   lsq_gather_fn gather;              /* NULL: no sharding (shard_rank 0, shard_world 0 or 1) */
   void* gather_user;                 /* passed to gather */
+  /* Disk tier (host_records NULL): the parts are read from the file at
+   * disk_path, which holds n_layers parts of record_bytes / max(1, shard_world)
+   * bytes back to back (this rank's parts), by disk_threads host threads into
+   * n_staging page-locked staging buffers of one part each, in upload order;
+   * the copy stream waits for each part (host function, bounded) before its
+   * copy.  A failed read or a wait that runs out makes the next scheduler call
+   * return EINVAL / ETIMEOUT. */
+  const char* disk_path;             /* NULL: records come from host_records */
+  void* const* staging;              /* n_staging host pointers, page-locked */
+  int32_t n_staging;                 /* 2..8 */
+  int32_t disk_threads;              /* 1..16 reader threads (each reads one slice of every part) */
 } lsq_stream_cfg;
 
 /* Creates the scheduler; ENOTPINNED if any record is not page-locked (the

@@ -21,7 +21,7 @@ LIB = os.path.join(PKG, "liblsq.so")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC,-ffp-contract=off",
+    "-Xcompiler", "-fPIC,-ffp-contract=off,-pthread",
     "-Xptxas", "-warn-spills",
     "-shared",
 ]

@@ -15,6 +15,17 @@
 // The slot policy (which slot to fill, how far to prefetch) is a CUDA-free
 // core that emits actions; the scheduler executes them with CUDA calls and
 // lsq_stream_simulate returns them, so the policy is testable without a GPU.
+#include <fcntl.h>
+#include <sys/stat.h>
+#include <unistd.h>
+
+#include <chrono>
+#include <condition_variable>
+#include <cstring>
+#include <deque>
+#include <mutex>
+#include <string>
+#include <thread>
 #include <vector>
 
 #include "host_common.h"
@@ -105,8 +116,150 @@ struct Policy {
 }  // namespace sched
 }  // namespace lsq
 
+namespace lsq {
+namespace disk {
+
+// Disk tier: layer parts are read from a store file into a ring of
+// page-locked staging buffers by a small pool of host threads, in the order
+// the scheduler submits them; the copy stream waits for each part with a host
+// function before its host-to-device copy and hands the buffer back with
+// another one after it.  Part t (the t-th upload) uses buffer t % n; the
+// readers fill it only once part t - n has been handed back, and each reader
+// thread reads one contiguous piece of every part, in part order.  Every wait
+// is bounded (kWaitS); a wait that runs out, or a failed read, sets an error
+// that the next scheduler call returns.
+constexpr int kWaitS = 120;
+
+struct Reader {
+  int fd = -1;
+  size_t part_bytes = 0;           // bytes per upload (this rank's part of a record)
+  std::vector<void*> staging;      // page-locked, part_bytes each
+  int nthreads = 0;
+  std::mutex mu;
+  std::condition_variable cv;
+  std::vector<int> job_layer;      // layer of each submitted part (index = ticket)
+  std::vector<int64_t> filled;     // per buffer: the ticket whose bytes it holds, -1 none
+  std::vector<int64_t> released;   // per buffer: the last ticket handed back by the copy stream
+  std::vector<int> pieces;         // per buffer: pieces of the pending ticket read so far
+  bool stop = false;
+  lsq_status error = LSQ_OK;
+  std::string errmsg;
+  std::vector<std::thread> threads;
+  int64_t bytes_read = 0;
+
+  int n() const { return (int)staging.size(); }
+
+  void set_error(lsq_status e, const std::string& m) {
+    if (error == LSQ_OK) {
+      error = e;
+      errmsg = m;
+    }
+    cv.notify_all();
+  }
+
+  int64_t submit(int layer) {
+    std::lock_guard<std::mutex> g(mu);
+    job_layer.push_back(layer);
+    cv.notify_all();
+    return (int64_t)job_layer.size() - 1;
+  }
+
+  void worker(int w) {
+    const size_t per = (part_bytes + nthreads - 1) / nthreads;
+    const size_t lo = std::min(part_bytes, (size_t)w * per), hi = std::min(part_bytes, lo + per);
+    for (int64_t t = 0;; ++t) {
+      const int b = (int)(t % n());
+      int layer;
+      {
+        std::unique_lock<std::mutex> g(mu);
+        // the part is submitted and its buffer handed back by part t - n
+        for (;;) {
+          const bool ok = cv.wait_for(g, std::chrono::seconds(kWaitS), [&] {
+            return stop || error != LSQ_OK || ((int64_t)job_layer.size() > t && released[b] >= t - n());
+          });
+          if (stop || error != LSQ_OK) return;
+          if (ok) break;
+          if ((int64_t)job_layer.size() > t) {
+            set_error(LSQ_ETIMEOUT, "disk tier: a staging buffer was not handed back in time");
+            return;
+          }
+          // idle (nothing submitted yet): keep waiting on the host
+        }
+        layer = job_layer[t];
+      }
+      char* dst = static_cast<char*>(staging[b]) + lo;
+      off_t off = (off_t)((uint64_t)layer * part_bytes + lo);
+      size_t left = hi - lo;
+      while (left > 0) {
+        const ssize_t r = pread(fd, dst, left, off);
+        if (r <= 0) {
+          std::lock_guard<std::mutex> g(mu);
+          set_error(LSQ_EINVAL, std::string("disk tier: read of layer ") + std::to_string(layer) + " failed: " +
+                                    (r == 0 ? "end of file" : std::strerror(errno)));
+          return;
+        }
+        dst += r;
+        off += r;
+        left -= (size_t)r;
+      }
+      std::lock_guard<std::mutex> g(mu);
+      bytes_read += (int64_t)(hi - lo);
+      if (++pieces[b] == nthreads) {
+        pieces[b] = 0;
+        filled[b] = t;
+        cv.notify_all();
+      }
+    }
+  }
+
+  // host-function side (copy stream): wait until part t is in its buffer
+  void wait_filled(int64_t t) {
+    const int b = (int)(t % n());
+    std::unique_lock<std::mutex> g(mu);
+    if (!cv.wait_for(g, std::chrono::seconds(kWaitS), [&] { return stop || error != LSQ_OK || filled[b] == t; }))
+      set_error(LSQ_ETIMEOUT, "disk tier: a layer part was not read in time");
+  }
+  void release(int64_t t) {
+    std::lock_guard<std::mutex> g(mu);
+    released[t % n()] = t;
+    cv.notify_all();
+  }
+
+  void shutdown() {
+    {
+      std::lock_guard<std::mutex> g(mu);
+      stop = true;
+    }
+    cv.notify_all();
+    for (auto& th : threads)
+      if (th.joinable()) th.join();
+    threads.clear();
+    if (fd >= 0) close(fd);
+    fd = -1;
+  }
+};
+
+struct HostArg {
+  Reader* r;
+  int64_t t;
+};
+static void CUDART_CB wait_filled_cb(void* p) {
+  HostArg* a = static_cast<HostArg*>(p);
+  a->r->wait_filled(a->t);
+  delete a;
+}
+static void CUDART_CB release_cb(void* p) {
+  HostArg* a = static_cast<HostArg*>(p);
+  a->r->release(a->t);
+  delete a;
+}
+
+}  // namespace disk
+}  // namespace lsq
+
 struct lsq_stream {
   lsq::sched::Policy pol;
+  lsq::disk::Reader* reader = nullptr;  // disk tier, else records come from host_records
   size_t record_bytes = 0;
   // sharded upload: this rank copies shard_bytes at shard_rank * shard_bytes; gather completes the slot
   size_t shard_bytes = 0;
@@ -139,7 +292,16 @@ static lsq_status execute(lsq_stream* st) {
       if (st->free_recorded[a.slot]) LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[a.slot], 0));
       LSQ_CUDA_TRY(cudaEventRecord(st->up_start[a.layer], st->copy));
       char* dst = static_cast<char*>(st->slots[a.slot]) + (size_t)st->shard_rank * st->shard_bytes;
-      LSQ_CUDA_TRY(cudaMemcpyAsync(dst, st->host[a.layer], st->shard_bytes, cudaMemcpyHostToDevice, st->copy));
+      if (st->reader) {
+        disk::Reader* r = st->reader;
+        const int64_t t = r->submit(a.layer);
+        LSQ_CUDA_TRY(cudaLaunchHostFunc(st->copy, disk::wait_filled_cb, new disk::HostArg{r, t}));
+        LSQ_CUDA_TRY(cudaMemcpyAsync(dst, r->staging[t % r->n()], st->shard_bytes, cudaMemcpyHostToDevice,
+                                     st->copy));
+        LSQ_CUDA_TRY(cudaLaunchHostFunc(st->copy, disk::release_cb, new disk::HostArg{r, t}));
+      } else {
+        LSQ_CUDA_TRY(cudaMemcpyAsync(dst, st->host[a.layer], st->shard_bytes, cudaMemcpyHostToDevice, st->copy));
+      }
       if (st->gather) {
         const int32_t rc = st->gather(st->gather_user, a.layer, a.slot, st->slots[a.slot], st->record_bytes,
                                       (lsq_cuda_stream)st->copy);
@@ -170,6 +332,14 @@ static bool is_pinned_host(const void* p) {
   return a.type == cudaMemoryTypeHost;
 }
 
+// the disk tier's first error, if any (returned by the next scheduler call)
+static lsq_status disk_status(lsq_stream* st) {
+  if (!st->reader) return LSQ_OK;
+  std::lock_guard<std::mutex> g(st->reader->mu);
+  if (st->reader->error == LSQ_OK) return LSQ_OK;
+  return fail(st->reader->error, "%s", st->reader->errmsg.c_str());
+}
+
 static void destroy_events(lsq_stream* st) {
   for (auto* v : {&st->up_start, &st->up_done, &st->slot_free})
     for (cudaEvent_t e : *v)
@@ -188,7 +358,10 @@ using namespace lsq::sched;
 
 extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stream compute, lsq_cuda_stream copy,
                                         lsq_stream** out) {
-  if (!cfg || !out || !cfg->slots || !cfg->host_records) return fail(LSQ_EINVAL, "lsq_stream_create: NULL argument");
+  if (!cfg || !out || !cfg->slots || (!cfg->host_records && !cfg->disk_path))
+    return fail(LSQ_EINVAL, "lsq_stream_create: NULL argument");
+  if (cfg->host_records && cfg->disk_path)
+    return fail(LSQ_EINVAL, "lsq_stream_create: give host_records or disk_path, not both");
   *out = nullptr;
   if (cfg->n_layers < 1 || cfg->record_bytes == 0) return fail(LSQ_EINVAL, "lsq_stream_create: empty model");
   if (!valid_slots(cfg->n_layers, cfg->n_slots))
@@ -212,13 +385,43 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   if (cfg->record_bytes % (256 * (size_t)world) != 0)
     return fail(LSQ_EINVAL, "lsq_stream_create: record_bytes must be a multiple of 256 x shard_world");
   const size_t shard = cfg->record_bytes / world;
-  for (int l = 0; l < cfg->n_layers; ++l) {
+  for (int l = 0; cfg->host_records && l < cfg->n_layers; ++l) {
     const char* h = static_cast<const char*>(cfg->host_records[l]);
     if (!h) return fail(LSQ_EINVAL, "lsq_stream_create: record %d is NULL", l);
     if (!is_pinned_host(h) || !is_pinned_host(h + shard - 1))
       return fail(LSQ_ENOTPINNED, "lsq_stream_create: record %d is not page-locked host memory", l);
   }
+  disk::Reader* reader = nullptr;
+  if (cfg->disk_path) {
+    if (cfg->n_staging < 2 || cfg->n_staging > 8 || !cfg->staging || cfg->disk_threads < 1 || cfg->disk_threads > 16)
+      return fail(LSQ_EINVAL, "lsq_stream_create: the disk tier needs 2..8 staging buffers and 1..16 threads");
+    for (int i = 0; i < cfg->n_staging; ++i) {
+      const char* h = static_cast<const char*>(cfg->staging[i]);
+      if (!h || !is_pinned_host(h) || !is_pinned_host(h + shard - 1))
+        return fail(LSQ_ENOTPINNED, "lsq_stream_create: staging buffer %d is not page-locked host memory", i);
+    }
+    const int fd = open(cfg->disk_path, O_RDONLY | O_CLOEXEC);
+    if (fd < 0) return fail(LSQ_EINVAL, "lsq_stream_create: cannot open %s: %s", cfg->disk_path, std::strerror(errno));
+    struct stat sb;
+    if (fstat(fd, &sb) != 0 || (uint64_t)sb.st_size < (uint64_t)cfg->n_layers * shard) {
+      close(fd);
+      return fail(LSQ_EINVAL, "lsq_stream_create: %s holds less than %d layer parts of %zu bytes", cfg->disk_path,
+                  cfg->n_layers, shard);
+    }
+    posix_fadvise(fd, 0, 0, POSIX_FADV_SEQUENTIAL);
+    reader = new disk::Reader();
+    reader->fd = fd;
+    reader->part_bytes = shard;
+    reader->staging.assign(cfg->staging, cfg->staging + cfg->n_staging);
+    reader->nthreads = cfg->disk_threads;
+    reader->filled.assign(cfg->n_staging, -1);
+    reader->released.assign(cfg->n_staging, -1);
+    for (int b = 0; b < cfg->n_staging; ++b) reader->released[b] = b - cfg->n_staging;  // never used yet
+    reader->pieces.assign(cfg->n_staging, 0);
+    for (int w = 0; w < reader->nthreads; ++w) reader->threads.emplace_back(&disk::Reader::worker, reader, w);
+  }
   lsq_stream* st = new lsq_stream();
+  st->reader = reader;
   st->pol.init(cfg->n_layers, cfg->n_slots);
   st->record_bytes = cfg->record_bytes;
   st->shard_bytes = shard;
@@ -226,7 +429,7 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   st->gather = cfg->gather;
   st->gather_user = cfg->gather_user;
   st->slots.assign(cfg->slots, cfg->slots + cfg->n_slots);
-  st->host.assign(cfg->host_records, cfg->host_records + cfg->n_layers);
+  if (cfg->host_records) st->host.assign(cfg->host_records, cfg->host_records + cfg->n_layers);
   st->compute = (cudaStream_t)compute;
   st->copy = (cudaStream_t)copy;
   st->free_recorded.assign(cfg->n_slots, 0);
@@ -242,6 +445,10 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
     e = cudaEventCreateWithFlags(&st->slot_free[i], cudaEventDisableTiming);
   if (e != cudaSuccess) {
     destroy_events(st);
+    if (st->reader) {
+      st->reader->shutdown();
+      delete st->reader;
+    }
     delete st;
     return cuda_fail(e, "lsq_stream_create: cudaEventCreate");
   }
@@ -285,6 +492,8 @@ extern "C" lsq_status lsq_layer_upload_async(lsq_stream* st, int32_t layer, int3
   if (p.cur >= 0 && p.layer_slot[p.cur] == slot && p.cur != layer)
     return fail(LSQ_ESTATE, "lsq_layer_upload_async: slot %d holds layer %d, which is in use", slot, p.cur);
   if (p.layer_slot[layer] == slot) return LSQ_OK;  // already there
+  lsq_status ds = disk_status(st);
+  if (ds != LSQ_OK) return ds;
   p.place(layer, slot, st->acts);
   return execute(st);
 }
@@ -293,6 +502,8 @@ extern "C" lsq_status lsq_stream_step(lsq_stream* st, int32_t layer, int32_t dir
   if (!st || !slot_ptr) return fail(LSQ_EINVAL, "lsq_stream_step: NULL argument");
   if (layer < 0 || layer >= st->pol.n_layers) return fail(LSQ_EINVAL, "lsq_stream_step: layer %d out of range", layer);
   if (direction != 1 && direction != -1) return fail(LSQ_EINVAL, "lsq_stream_step: direction must be +1 or -1");
+  lsq_status ds = disk_status(st);
+  if (ds != LSQ_OK) return ds;
   st->pol.step(layer, direction, st->acts);
   lsq_status s = execute(st);
   if (s != LSQ_OK) return s;
@@ -355,7 +566,11 @@ extern "C" lsq_status lsq_stream_reset(lsq_stream* st) {
 
 extern "C" lsq_status lsq_stream_destroy(lsq_stream* st) {
   if (!st) return LSQ_OK;
-  cudaStreamSynchronize(st->copy);
+  cudaStreamSynchronize(st->copy);  // every host function of the disk tier has run
+  if (st->reader) {
+    st->reader->shutdown();
+    delete st->reader;
+  }
   destroy_events(st);
   delete st;
   return LSQ_OK;

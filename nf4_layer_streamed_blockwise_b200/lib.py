@@ -50,7 +50,8 @@ class lsq_stream_cfg(ctypes.Structure):
     _fields_ = [("n_layers", c_int32), ("n_slots", c_int32), ("record_bytes", c_size_t),
                 ("slots", ctypes.POINTER(c_void_p)), ("host_records", ctypes.POINTER(c_void_p)),
                 ("shard_rank", c_int32), ("shard_world", c_int32), ("gather", lsq_gather_fn),
-                ("gather_user", c_void_p)]
+                ("gather_user", c_void_p), ("disk_path", ctypes.c_char_p), ("staging", ctypes.POINTER(c_void_p)),
+                ("n_staging", c_int32), ("disk_threads", c_int32)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -412,12 +413,20 @@ _GATHERS = {}  # scheduler handle -> its ctypes callback (kept alive while the s
 
 
 def lsq_stream_create(n_layers: int, n_slots: int, record_bytes: int, slots: Sequence[int],
-                      host_records: Sequence[int], compute_stream, copy_stream, shard=None) -> int:
+                      host_records: Optional[Sequence[int]], compute_stream, copy_stream, shard=None,
+                      disk=None) -> int:
     """shard: None, or (rank, world, gather) for the sharded upload, where
     gather(layer, slot, slot_ptr, record_bytes, copy_stream_handle) enqueues the
-    completion of the slot on the copy stream (an all-gather) and raises on failure."""
+    completion of the slot on the copy stream (an all-gather) and raises on failure.
+    disk: None, or (path, staging buffers, reader threads) for the disk tier
+    (host_records None)."""
     sl = (c_void_p * len(slots))(*[_p(s) for s in slots])
-    hr = (c_void_p * len(host_records))(*[_p(h) for h in host_records])
+    hr = None if host_records is None else (c_void_p * len(host_records))(*[_p(h) for h in host_records])
+    path, stg, nthr = None, None, 0
+    if disk is not None:
+        path = str(disk[0]).encode()
+        stg = (c_void_p * len(disk[1]))(*[_p(b) for b in disk[1]])
+        nthr = int(disk[2])
     cb = lsq_gather_fn()
     rank = world = 0
     if shard is not None:
@@ -432,7 +441,8 @@ def lsq_stream_create(n_layers: int, n_slots: int, record_bytes: int, slots: Seq
                 print(f"lsq gather callback failed: {e!r}", file=sys.stderr)
                 return 1
         cb = lsq_gather_fn(_gather)
-    cfg = lsq_stream_cfg(n_layers, n_slots, record_bytes, sl, hr, rank, world, cb, None)
+    cfg = lsq_stream_cfg(n_layers, n_slots, record_bytes, sl, hr, rank, world, cb, None, path, stg,
+                         0 if disk is None else len(disk[1]), nthr)
     out = c_void_p()
     _call("lsq_stream_create", ctypes.byref(cfg), _stream(compute_stream), _stream(copy_stream), ctypes.byref(out))
     if shard is not None:

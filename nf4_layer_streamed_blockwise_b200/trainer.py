@@ -160,7 +160,8 @@ class StreamedLoraTrainer:
 
     def __init__(self, shape: S.ModelShape, batch: int, seq: int, n_slots: Optional[int] = 2,
                  init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None,
-                 absmax: str = "fp32", shard: Optional[tuple] = None):
+                 absmax: str = "fp32", shard: Optional[tuple] = None, source: str = "ram",
+                 store_path: Optional[str] = None, embed: str = "hbm"):
         self.shape, self.B, self.S = shape, batch, seq
         self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
         self.M = batch * seq
@@ -174,10 +175,21 @@ class StreamedLoraTrainer:
         align = 4096 if self.shard is None else math.lcm(4096, 256 * self.shard[1])
         self.layout = RecordLayout.of(shape, absmax, align)
         self.absmax_kind = absmax
+        # source "disk": the records live in a file (store_path) and reach the GPU through
+        # page-locked staging buffers filled by the library's reader threads
+        if source not in ("ram", "disk") or (source == "disk") != (store_path is not None):
+            raise ValueError("source must be 'ram', or 'disk' with a store_path")
+        self.source, self.store_path = source, store_path
+        # embed "host": an untied embedding table stays in page-locked host RAM and the
+        # gather reads the batch's rows straight over the host link (zero-copy)
+        if embed not in ("hbm", "host") or (embed == "host" and shape.tied):
+            raise ValueError("embed must be 'hbm', or 'host' for an untied embedding")
+        self.embed_kind = embed
         self.compute = torch.cuda.current_stream()
         self.copy = torch.cuda.Stream()
-        if share is not None and (share.absmax_kind != absmax or share.shard != self.shard):
-            raise ValueError("a shared host store must have the same absmax format and sharding")
+        if share is not None and (share.absmax_kind != absmax or share.shard != self.shard or
+                                  (share.source, share.store_path, share.embed_kind) != (source, store_path, embed)):
+            raise ValueError("a shared store must have the same absmax format, sharding, source and embed place")
         if share is not None:       # reuse another trainer's host store and resident tensors
             self.host_records = share.host_records
             self.embed, self.lm_head, self.final_norm = share.embed, share.lm_head, share.final_norm
@@ -192,10 +204,17 @@ class StreamedLoraTrainer:
         self._alloc_activations()
         self.slots = [torch.empty(self.layout.slot_bytes, dtype=torch.uint8, device=device)
                       for _ in range(self.n_slots)]
+        lo, hi = self.shard_range()
+        disk = None
+        if source == "disk":
+            self.staging = [torch.empty(hi - lo, dtype=torch.uint8, pin_memory=True) for _ in range(3)]
+            disk = (store_path, [b.data_ptr() for b in self.staging], 4)
         self.sched = L.lsq_stream_create(shape.n_layers, self.n_slots, self.layout.nbytes,
                                          [s.data_ptr() for s in self.slots],
-                                         [h.data_ptr() for h in self.host_records], self.compute, self.copy,
-                                         shard=None if self.shard is None else (*self.shard, lambda *a: self._gather(*a)))
+                                         None if source == "disk" else [h.data_ptr() for h in self.host_records],
+                                         self.compute, self.copy,
+                                         shard=None if self.shard is None else (*self.shard, lambda *a: self._gather(*a)),
+                                         disk=disk)
         if self.layout.dq:
             L.lsq_stream_set_absmax_expand(self.sched, self.layout.expand_items(), self.layout.slot_bytes)
         if self.resident:
@@ -220,11 +239,14 @@ class StreamedLoraTrainer:
         DP.gather_slot(t, nbytes, *self.shard, stream=self.copy)
 
     def _build_store(self, init: str):
-        """Quantise every layer once on the GPU and keep the records pinned on the host."""
+        """Quantise every layer once on the GPU and keep the records pinned on the host
+        (source "ram"), or write this rank's parts of them back to back to store_path
+        (source "disk")."""
         sh, lay = self.shape, self.layout
         stage = torch.zeros(lay.slot_bytes, dtype=torch.uint8, device=self.dev)
         base = stage.data_ptr()
         self.host_records: List[torch.Tensor] = []
+        fout = open(self.store_path, "wb") if self.source == "disk" else None
         for l in range(sh.n_layers):
             if init == "host":
                 Wl = S.layer_weights(sh, l)
@@ -242,9 +264,14 @@ class StreamedLoraTrainer:
             stage[lay.ln1:lay.ln1 + 2 * sh.d].copy_(ones.view(torch.uint8))
             stage[lay.ln2:lay.ln2 + 2 * sh.d].copy_(ones.view(torch.uint8))
             lo, hi = self.shard_range()
+            if fout is not None:
+                fout.write(stage[lo:hi].cpu().numpy().tobytes())
+                continue
             rec = torch.empty(hi - lo, dtype=torch.uint8, pin_memory=True)
             rec.copy_(stage[lo:hi])
             self.host_records.append(rec)
+        if fout is not None:
+            fout.close()
         del stage
         torch.cuda.synchronize()
 
@@ -258,6 +285,10 @@ class StreamedLoraTrainer:
             self.embed = S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD, S.WEIGHT_SEED, 11)
             self.lm_head = self.embed if sh.tied else S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD,
                                                                             S.WEIGHT_SEED, 12)
+        if self.embed_kind == "host":   # page-locked host copy; the gather reads it in place
+            host = torch.empty(self.embed.shape, dtype=self.embed.dtype, pin_memory=True)
+            host.copy_(self.embed)
+            self.embed = host
         self.final_norm = torch.ones(sh.d, dtype=torch.bfloat16, device=self.dev)
 
     def _alloc_activations(self):
