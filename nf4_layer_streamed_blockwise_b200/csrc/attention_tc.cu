@@ -15,8 +15,9 @@
 // Layouts as the mma.sync kernels: q, o [B, S, Hq, 128]; k, v [B, S, Hkv, 128];
 // lse [B, Hq, S].  Query head h reads kv head h / (Hq / Hkv).  K and V arrive
 // through a two-slot TMA ring (K chunks, then V chunks).  Warp 0: TMA; warp 1:
-// TMEM owner and MMA issuer; warps 2-5: softmax and epilogue, one query row
-// per thread (TMEM lane = row).  Every wait is bounded; no atomics.
+// TMEM owner and MMA issuer; warps 2-17: softmax and epilogue, one query row
+// per lane (TMEM lane = row), four warps per lane quarter splitting the key
+// columns.  Every wait is bounded; no atomics.
 #include "common.cuh"
 #include "host_common.h"
 
@@ -29,19 +30,29 @@ constexpr int BC = 128;          // keys per chunk
 constexpr int MAXC = 4;          // chunks: sequences of at most 512
 constexpr int TILE = BQ * D * 2; // 128 x 128 bf16 tile: two 64-column 128B-swizzled halves of 16 KB
 constexpr int HALF = TILE / 2;
-constexpr int OFF_Q = 0;
+constexpr int OFF_Q = 0;          // Q; once the score products are done, the row statistics
 constexpr int OFF_RING = OFF_Q + TILE;
 constexpr int OFF_P = OFF_RING + 2 * TILE;
 constexpr int OFF_BAR = OFF_P + MAXC * TILE;
-constexpr int NBAR = 1 + 2 + 2 + 1 + MAXC + 1;  // qfull, rfull[2], rempty[2], sfull, pready[4], ofull
+// qfull, rfull[2], rempty[2], sfull, pready[4], ofull, mxbar, smbar
+constexpr int NBAR = 1 + 2 + 2 + 1 + MAXC + 1 + 2;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-constexpr int NTHREADS = 192;
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr int EW = 16;                     // element-wise warps: four per TMEM lane quarter
+constexpr int FWD_THREADS = 32 * (2 + EW);
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 2^x in one special-function instruction (relative error about 2^-22, far
+// below the bf16 rounding of the probabilities); 0 for very negative x
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // smem descriptor of a K-major operand tile (rows x 128 elements as two
@@ -50,12 +61,17 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
   return smem_desc(base + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024, 2);
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                  const __grid_constant__ CUtensorMap kmap,
-                                                                  const __grid_constant__ CUtensorMap vmap,
-                                                                  __nv_bfloat16* __restrict__ o,
-                                                                  float* __restrict__ lse, int S, int Hq, int Hkv,
-                                                                  float scale_log2) {
+// Warp 0: TMA; warp 1: TMEM owner and MMA issuer; warps 2-17: softmax and
+// epilogue, four per TMEM lane quarter (one query row per lane, 32 of each
+// chunk's 128 key columns per warp); the four warps of a quarter combine
+// their partial row max and row sum through shared memory (an mbarrier each,
+// bounded waits).
+__global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                     const __grid_constant__ CUtensorMap kmap,
+                                                                     const __grid_constant__ CUtensorMap vmap,
+                                                                     __nv_bfloat16* __restrict__ o,
+                                                                     float* __restrict__ lse, int S, int Hq, int Hkv,
+                                                                     float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -64,6 +80,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_fwd_tc_kernel(const __grid_c
   uint64_t* sfull = rempty + 2;
   uint64_t* pready = sfull + 1;
   uint64_t* ofull = pready + MAXC;
+  uint64_t* mxbar = ofull + 1;
+  uint64_t* smbar = mxbar + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int nt = (S + BQ - 1) / BQ;
@@ -81,8 +99,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_fwd_tc_kernel(const __grid_c
       mbar_init(&rempty[i], 1);
     }
     mbar_init(sfull, 1);
-    for (int j = 0; j < MAXC; ++j) mbar_init(&pready[j], 4);  // one arrival per softmax warp
+    for (int j = 0; j < MAXC; ++j) mbar_init(&pready[j], EW);  // one arrival per softmax warp
     mbar_init(ofull, 1);
+    mbar_init(mxbar, EW);
+    mbar_init(smbar, EW);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -151,77 +171,98 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_fwd_tc_kernel(const __grid_c
       if (!ok) mbar_wait(ofull, 0, 565);
     }
   } else {
-    // softmax and epilogue: one query row per thread
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;
+    // softmax and epilogue: one query row per lane, key columns part*32 .. +31 of every chunk
+    const int quad = warp & 3, part = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;
     const int qi = q0 + r;
-    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    float* s_max = reinterpret_cast<float*>(smem + OFF_Q);  // [4][128], after the score products
+    float* s_sum = s_max + 4 * BQ;                          // [4][128]
     bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, 761));
     float m = -INFINITY, l = 0.0f;
     if (ok) {
       tc_fence_after();
       for (int j = 0; j < nc; ++j) {
-        for (int c4 = 0; c4 < BC / 32; ++c4) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + c4 * 32), v);
-          tc_wait_ld();
+        float v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + part * 32), v);
+        tc_wait_ld();
+        if (j < t) {  // a chunk before the diagonal: every key is visible
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m = fmaxf(m, v[e]);
+        } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int kj = j * BC + c4 * 32 + e;
-            if (kj <= qi && kj < S) m = fmaxf(m, v[e] * scale_log2);
+            const int kj = j * BC + part * 32 + e;
+            if (kj <= qi && kj < S) m = fmaxf(m, v[e]);
           }
         }
       }
+      m *= scale_log2;  // the scale is positive: max of scaled = scaled max
+      s_max[part * BQ + r] = m;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mxbar);
+      ok = __all_sync(0xffffffffu, mbar_wait(mxbar, 0, 762));
+    }
+    if (ok) {
+      m = fmaxf(fmaxf(s_max[r], s_max[BQ + r]), fmaxf(s_max[2 * BQ + r], s_max[3 * BQ + r]));
       for (int j = 0; j < nc; ++j) {
-        const uint32_t pbase = smem_u32(smem + OFF_P + j * TILE) + r * 128;
-        for (int c4 = 0; c4 < BC / 32; ++c4) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + c4 * 32), v);
-          tc_wait_ld();
-          uint32_t w[16];
+        float v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + part * 32), v);
+        tc_wait_ld();
+        uint32_t w[16];
+        if (j < t) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const int kj = j * BC + c4 * 32 + e;
-            const float p0 = (kj <= qi && kj < S) ? exp2f(v[e] * scale_log2 - m) : 0.0f;
-            const float p1 = (kj + 1 <= qi && kj + 1 < S) ? exp2f(v[e + 1] * scale_log2 - m) : 0.0f;
+            const float p0 = ex2(v[e] * scale_log2 - m), p1 = ex2(v[e + 1] * scale_log2 - m);
             l += p0 + p1;
             w[e / 2] = pack_bf16x2(p0, p1);
           }
-          // keys c4*32 .. +31 of this chunk: half c4 >> 1, 16-byte units (c4 & 1) * 4 .. + 3
-          const uint32_t hbase = pbase + (uint32_t)(c4 >> 1) * HALF;
+        } else {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int unit = (c4 & 1) * 4 + u;
-            st_shared_v4(hbase + ((uint32_t)(unit ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
-                         w[4 * u + 3]);
+          for (int e = 0; e < 32; e += 2) {
+            const int kj = j * BC + part * 32 + e;
+            const float p0 = (kj <= qi && kj < S) ? ex2(v[e] * scale_log2 - m) : 0.0f;
+            const float p1 = (kj + 1 <= qi && kj + 1 < S) ? ex2(v[e + 1] * scale_log2 - m) : 0.0f;
+            l += p0 + p1;
+            w[e / 2] = pack_bf16x2(p0, p1);
           }
+        }
+        // keys part*32 .. +31 of this chunk: half part >> 1, 16-byte units (part & 1) * 4 .. + 3
+        const uint32_t hbase = smem_u32(smem + OFF_P + j * TILE) + r * 128 + (uint32_t)(part >> 1) * HALF;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (part & 1) * 4 + u;
+          st_shared_v4(hbase + ((uint32_t)(unit ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
+                       w[4 * u + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pready[j]);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(ofull, 0, 762));
+      s_sum[part * BQ + r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smbar);
+      ok = __all_sync(0xffffffffu, mbar_wait(smbar, 0, 763)) && __all_sync(0xffffffffu, mbar_wait(ofull, 0, 764));
     }
     if (ok) {
       tc_fence_after();
+      l = (s_sum[r] + s_sum[BQ + r]) + (s_sum[2 * BQ + r] + s_sum[3 * BQ + r]);
       const float inv = 1.0f / l;
       __nv_bfloat16* orow = o + (((int64_t)b * S + qi) * Hq + h) * D;
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(c4 * 32), v);
-        tc_wait_ld();
-        if (qi < S) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + (uint32_t)(part * 32), v);
+      tc_wait_ld();
+      if (qi < S) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(orow + c4 * 32 + u * 8) =
-                make_uint4(pack_bf16x2(v[8 * u] * inv, v[8 * u + 1] * inv),
-                           pack_bf16x2(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
-                           pack_bf16x2(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
-                           pack_bf16x2(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
-        }
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(orow + part * 32 + u * 8) =
+              make_uint4(pack_bf16x2(v[8 * u] * inv, v[8 * u + 1] * inv),
+                         pack_bf16x2(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
+                         pack_bf16x2(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
+                         pack_bf16x2(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
+        if (part == 0) lse[((int64_t)b * Hq + h) * S + qi] = (m + log2f(l)) / LOG2E;
       }
-      if (qi < S) lse[((int64_t)b * Hq + h) * S + qi] = (m + log2f(l)) / LOG2E;
     }
   }
   tc_fence_before();
@@ -233,57 +274,106 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_fwd_tc_kernel(const __grid_c
 }
 
 // ================================================================ backward
-// dQ: one CTA per (128-query tile, query head, sequence); per key chunk j <= tile:
-//   S = Q K_j^T, dP = dO V_j^T (TMEM), dS = P (dP - Dvec) in bf16 (shared
-//   memory, K-major), dQ += dS K_j (TMEM); dq = dQ / sqrt(D).
+// Both backward kernels work through a list of 64-row sub-items with two
+// score accumulators in TMEM, so that the element-wise step of sub-item i
+// (sixteen warps) overlaps the
+// score products of sub-item i+1 and the accumulating products of i-1:
+//
+//   MMA issue order:  S(0)  S(1) A(0)  S(2) A(1)  ...  A(n-1)
+//   element-wise:           E(0)       E(1)      ...
+//
+// where S(i) writes score buffer i % 2 (after E(i-2) has read it), E(i) turns
+// it into bf16 operands in shared-memory buffer i % 2 (after A(i-2) has read
+// it) and A(i) accumulates from them.  A three-stage TMA ring feeds the 64-row
+// operand tiles.  Warp 0: TMA; warp 1: TMEM owner and MMA issuer; warps 2-17:
+// element-wise and epilogue, four per TMEM lane quarter, 16 columns each (four
+// warps per SM sub-partition hide the TMEM, exp and shuffle latencies).
+constexpr int SUB = 64;                     // rows per sub-item
+constexpr int ST = SUB * D * 2;             // 64 x 128 bf16 tile: two 64-column halves of 8 KB
+constexpr int SHALF = ST / 2;
+constexpr int PT = BC * SUB * 2;            // 128 x 64 bf16 operand (one 128-byte swizzled column block)
+constexpr int NRING = 3;
+constexpr int CW = SUB / (EW / 4);           // columns per element-wise warp
+constexpr int BWD_THREADS = 32 * (2 + EW);
+
+// K-major 128-row x 64-element operand at k-step kk (16 elements)
+__device__ __forceinline__ uint64_t desc_k64(uint32_t base, int kk) { return smem_desc(base + kk * 32, 16, 1024, 2); }
+// K-major 64-row x 128-element operand (two 64-element halves of 8 KB) at k-step kk
+__device__ __forceinline__ uint64_t desc_sub_kmajor(uint32_t base, int kk) {
+  return smem_desc(base + (kk >> 2) * SHALF + (kk & 3) * 32, 16, 1024, 2);
+}
+// MN-major 64-row (K) x 128-column (N) operand: N halves 8 KB apart, 16 rows per k-step
+__device__ __forceinline__ uint64_t desc_sub_mnmajor(uint32_t base, int kk) {
+  return smem_desc(base + kk * 2048, SHALF, 1024, 2);
+}
+
+// CW bf16 values (CW / 2 pairs) of row r into a 128-row x 64-column swizzled
+// operand: the row's 16-byte units part * CW / 8 onwards
+__device__ __forceinline__ void store_row_units(uint32_t row_base, int r, int part, const uint32_t (&w)[CW / 2]) {
+#pragma unroll
+  for (int u = 0; u < CW / 8; ++u)
+    st_shared_v4(row_base + ((uint32_t)((part * (CW / 8) + u) ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1],
+                 w[4 * u + 2], w[4 * u + 3]);
+}
+
+// ---------------------------------------------------------------- dQ
+// One CTA per (128-query tile, head, sequence); sub-items = 64-key slices of
+// the keys at or before the tile:  S = Q K_j^T, dP = dO V_j^T (TMEM), dS =
+// P (dP - D) (bf16, shared memory), dQ += dS K_j (TMEM); dq = dQ / sqrt(D).
 constexpr int Q_OFF_Q = 0;
 constexpr int Q_OFF_DO = Q_OFF_Q + TILE;
-constexpr int Q_OFF_RING = Q_OFF_DO + TILE;  // 2 slots of [K_j | V_j]
-constexpr int Q_OFF_DS = Q_OFF_RING + 4 * TILE;
-constexpr int Q_OFF_BAR = Q_OFF_DS + TILE;
-constexpr int Q_NBAR = 1 + 2 + 2 + 1 + 1 + 1 + 1;  // qfull, rfull[2], rempty[2], sfull, dsready, dsfree, dqfull
+constexpr int Q_OFF_RING = Q_OFF_DO + TILE;        // stage s: K at +s*2*ST, V at +s*2*ST + ST
+constexpr int Q_OFF_DS = Q_OFF_RING + NRING * 2 * ST;  // buffer b at +b*PT
+constexpr int Q_OFF_BAR = Q_OFF_DS + 2 * PT;
+// qfull, rfull[3], rempty[3], sfull[2], tfree[2], dsready[2], dsfree[2], done
+constexpr int Q_NBAR = 1 + 3 + 3 + 2 + 2 + 2 + 2 + 1;
 constexpr int Q_OFF_MISC = Q_OFF_BAR + 8 * Q_NBAR;
 constexpr int Q_SMEM = Q_OFF_MISC + 16 + 1024;
 static_assert(Q_SMEM <= 232448, "shared memory");
 
-__global__ void __launch_bounds__(NTHREADS, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                 const __grid_constant__ CUtensorMap kmap,
-                                                                 const __grid_constant__ CUtensorMap vmap,
-                                                                 const __grid_constant__ CUtensorMap domap,
-                                                                 const float* __restrict__ lse,
-                                                                 const float* __restrict__ dvec,
-                                                                 __nv_bfloat16* __restrict__ dq, int S, int Hq,
-                                                                 int Hkv, float scale, float scale_log2) {
+__global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                    const __grid_constant__ CUtensorMap kmap64,
+                                                                    const __grid_constant__ CUtensorMap vmap64,
+                                                                    const __grid_constant__ CUtensorMap domap,
+                                                                    const float* __restrict__ lse,
+                                                                    const float* __restrict__ dvec,
+                                                                    __nv_bfloat16* __restrict__ dq, int S, int Hq,
+                                                                    int Hkv, float scale, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + Q_OFF_BAR);
   uint64_t* rfull = qfull + 1;
-  uint64_t* rempty = rfull + 2;
-  uint64_t* sfull = rempty + 2;
-  uint64_t* dsready = sfull + 1;
-  uint64_t* dsfree = dsready + 1;
-  uint64_t* dqfull = dsfree + 1;
+  uint64_t* rempty = rfull + NRING;
+  uint64_t* sfull = rempty + NRING;
+  uint64_t* tfree = sfull + 2;
+  uint64_t* dsready = tfree + 2;
+  uint64_t* dsfree = dsready + 2;
+  uint64_t* done = dsfree + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Q_OFF_MISC);
 
   const int nt = (S + BQ - 1) / BQ;
-  const int t = nt - 1 - (int)blockIdx.x;
+  const int t = nt - 1 - (int)blockIdx.x;  // longest causal tiles first
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (Hq / Hkv);
   const int q0 = t * BQ;
-  const int nc = t + 1;
+  const int nkeys = min(q0 + BQ, S);
+  const int nsub = (nkeys + SUB - 1) / SUB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NRING; ++i) {
       mbar_init(&rfull[i], 1);
       mbar_init(&rempty[i], 1);
     }
-    mbar_init(sfull, 1);
-    mbar_init(dsready, 4);
-    mbar_init(dsfree, 1);
-    mbar_init(dqfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&tfree[i], EW);
+      mbar_init(&dsready[i], EW);
+      mbar_init(&dsfree[i], 1);
+    }
+    mbar_init(done, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -303,101 +393,113 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_dq_tc_kernel(const __grid_co
       tma_load_2d(smem + Q_OFF_Q + HALF, &qmap, qfull, h * D + 64, row0 + q0);
       tma_load_2d(smem + Q_OFF_DO, &domap, qfull, h * D, row0 + q0);
       tma_load_2d(smem + Q_OFF_DO + HALF, &domap, qfull, h * D + 64, row0 + q0);
-      for (int j = 0; j < nc; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&rempty[slot], ((uint32_t)(j >> 1) & 1u) ^ 1u, 471)) break;
-        uint8_t* dst = smem + Q_OFF_RING + slot * 2 * TILE;
-        mbar_arrive_expect_tx(&rfull[slot], 2u * TILE);
-        tma_load_2d(dst, &kmap, &rfull[slot], hk * D, row0 + j * BC);
-        tma_load_2d(dst + HALF, &kmap, &rfull[slot], hk * D + 64, row0 + j * BC);
-        tma_load_2d(dst + TILE, &vmap, &rfull[slot], hk * D, row0 + j * BC);
-        tma_load_2d(dst + TILE + HALF, &vmap, &rfull[slot], hk * D + 64, row0 + j * BC);
+      for (int j = 0; j < nsub; ++j) {
+        const int s = j % NRING;
+        if (!mbar_wait(&rempty[s], ((uint32_t)(j / NRING) & 1u) ^ 1u, 471)) break;
+        uint8_t* dst = smem + Q_OFF_RING + s * 2 * ST;
+        mbar_arrive_expect_tx(&rfull[s], 2u * ST);
+        tma_load_2d(dst, &kmap64, &rfull[s], hk * D, row0 + j * SUB);
+        tma_load_2d(dst + SHALF, &kmap64, &rfull[s], hk * D + 64, row0 + j * SUB);
+        tma_load_2d(dst + ST, &vmap64, &rfull[s], hk * D, row0 + j * SUB);
+        tma_load_2d(dst + ST + SHALF, &vmap64, &rfull[s], hk * D + 64, row0 + j * SUB);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = mbar_wait(qfull, 0, 571);
       const uint32_t qb = smem_u32(smem + Q_OFF_Q), dob = smem_u32(smem + Q_OFF_DO);
-      const uint32_t dsb = smem_u32(smem + Q_OFF_DS);
-      const uint32_t id_k = idesc_bf16(BQ, BC, 0, 0);  // S, dP: both operands K-major
-      const uint32_t id_q = idesc_bf16(BQ, D, 0, 1);   // dS K: K MN-major
-      for (int j = 0; ok && j < nc; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&rfull[slot], (uint32_t)(j >> 1) & 1u, 572)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t kb = smem_u32(smem + Q_OFF_RING + slot * 2 * TILE), vb = kb + TILE;
+      const uint32_t id_s = idesc_bf16(BQ, SUB, 0, 0);  // S, dP: both operands K-major
+      const uint32_t id_q = idesc_bf16(BQ, D, 0, 1);    // dS K: K MN-major
+      for (int j = 0; ok && j <= nsub; ++j) {
+        if (j < nsub) {
+          const int s = j % NRING, bb = j & 1;
+          if (!mbar_wait(&rfull[s], (uint32_t)(j / NRING) & 1u, 572) ||
+              (j >= 2 && !mbar_wait(&tfree[bb], (uint32_t)((j - 2) >> 1) & 1u, 573))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kb = smem_u32(smem + Q_OFF_RING + s * 2 * ST), vb = kb + ST;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          tc_mma(tmem + T_S, desc_kmajor(qb, kk), desc_kmajor(kb, kk), id_k, kk != 0);
-          tc_mma(tmem + T_DP, desc_kmajor(dob, kk), desc_kmajor(vb, kk), id_k, kk != 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            tc_mma(tmem + T_S + bb * SUB, desc_kmajor(qb, kk), desc_sub_kmajor(kb, kk), id_s, kk != 0);
+            tc_mma(tmem + T_DP + bb * SUB, desc_kmajor(dob, kk), desc_sub_kmajor(vb, kk), id_s, kk != 0);
+          }
+          tc_commit(&sfull[bb]);
         }
-        tc_commit(sfull);
-        if (!mbar_wait(dsready, (uint32_t)j & 1u, 573)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        if (j >= 1) {
+          const int p = j - 1, ps = p % NRING, pb = p & 1;
+          if (!mbar_wait(&dsready[pb], (uint32_t)(p >> 1) & 1u, 574)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dsb = smem_u32(smem + Q_OFF_DS + pb * PT);
+          const uint32_t kb = smem_u32(smem + Q_OFF_RING + ps * 2 * ST);
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk)
-          tc_mma(tmem + T_DQ, desc_kmajor(dsb, kk), smem_desc(kb + kk * 2048, HALF, 1024, 2), id_q, (j | kk) != 0);
-        tc_commit(dsfree);
-        tc_commit(&rempty[slot]);
+          for (int kk = 0; kk < SUB / 16; ++kk)
+            tc_mma(tmem + T_DQ, desc_k64(dsb, kk), desc_sub_mnmajor(kb, kk), id_q, (p | kk) != 0);
+          tc_commit(&dsfree[pb]);
+          tc_commit(&rempty[ps]);
+        }
       }
-      tc_commit(dqfull);
-      if (!ok) mbar_wait(dqfull, 0, 574);
+      tc_commit(done);  // also drains what was issued if a wait gave up
+      if (!ok) mbar_wait(done, 0, 575);
     }
   } else {
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;
+    const int quad = warp & 3, part = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;  // query row of the tile
     const int qi = q0 + r;
-    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int64_t ri = ((int64_t)b * Hq + h) * S + (qi < S ? qi : 0);
     const float lse2 = lse[ri] * LOG2E, dv = dvec[ri];
     bool ok = true;
-    for (int j = 0; ok && j < nc; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(sfull, (uint32_t)j & 1u, 771))) {
+    for (int j = 0; ok && j < nsub; ++j) {
+      const int bb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[bb], (uint32_t)(j >> 1) & 1u, 771))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(dsfree, (uint32_t)(j - 1) & 1u, 772))) {
-        ok = false;
-        break;
-      }
-      const uint32_t rbase = smem_u32(smem + Q_OFF_DS) + r * 128;
-      for (int c4 = 0; c4 < BC / 32; ++c4) {
-        float sv[32], pv[32];
-        tmem_ld32(tmem + lane_base + T_S + (uint32_t)(c4 * 32), sv);
-        tmem_ld32(tmem + lane_base + T_DP + (uint32_t)(c4 * 32), pv);
-        tc_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int kj = j * BC + c4 * 32 + e;
-          const bool ok0 = kj <= qi && kj < S && qi < S, ok1 = kj + 1 <= qi && kj + 1 < S && qi < S;
-          const float p0 = ok0 ? exp2f(sv[e] * scale_log2 - lse2) : 0.0f;
-          const float p1 = ok1 ? exp2f(sv[e + 1] * scale_log2 - lse2) : 0.0f;
-          w[e / 2] = pack_bf16x2(p0 * (pv[e] - dv), p1 * (pv[e + 1] - dv));
-        }
-        const uint32_t hbase = rbase + (uint32_t)(c4 >> 1) * HALF;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (c4 & 1) * 4 + u;
-          st_shared_v4(hbase + ((uint32_t)(unit ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
-      }
-      fence_proxy_async_smem();
+      float sv[CW], pv[CW];
+      tmem_ld16(tmem + lane_base + T_S + bb * SUB + part * CW, sv);
+      tmem_ld16(tmem + lane_base + T_DP + bb * SUB + part * CW, pv);
+      tc_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dsready);
+      if (lane == 0) mbar_arrive(&tfree[bb]);
+      uint32_t w[CW / 2];
+      if ((j + 1) * SUB <= q0 && q0 + BQ <= S) {  // keys all before the tile, rows all inside S: no mask
+#pragma unroll
+        for (int e = 0; e < CW; e += 2) {
+          const float p0 = ex2(sv[e] * scale_log2 - lse2), p1 = ex2(sv[e + 1] * scale_log2 - lse2);
+          w[e / 2] = pack_bf16x2(p0 * (pv[e] - dv), p1 * (pv[e + 1] - dv));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < CW; e += 2) {
+          const int kj = j * SUB + part * CW + e;
+          const bool ok0 = kj <= qi && kj < S && qi < S, ok1 = kj + 1 <= qi && kj + 1 < S && qi < S;
+          const float p0 = ok0 ? ex2(sv[e] * scale_log2 - lse2) : 0.0f;
+          const float p1 = ok1 ? ex2(sv[e + 1] * scale_log2 - lse2) : 0.0f;
+          w[e / 2] = pack_bf16x2(p0 * (pv[e] - dv), p1 * (pv[e + 1] - dv));
+        }
+      }
+      // buffer bb was read by the dQ product of sub-item j - 2
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&dsfree[bb], (uint32_t)((j - 2) >> 1) & 1u, 772))) {
+        ok = false;
+        break;
+      }
+      store_row_units(smem_u32(smem + Q_OFF_DS + bb * PT) + r * 128, r, part, w);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dsready[bb]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(dqfull, 0, 773))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(done, 0, 773))) {
       tc_fence_after();
       __nv_bfloat16* row = dq + (((int64_t)b * S + qi) * Hq + h) * D;
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      {
+        const int c4 = part;  // 32 of the 128 output columns per warp
         float v[32];
         tmem_ld32(tmem + lane_base + T_DQ + (uint32_t)(c4 * 32), v);
         tc_wait_ld();
@@ -421,57 +523,63 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_dq_tc_kernel(const __grid_co
   }
 }
 
-// dK, dV: one CTA per (128-key chunk, kv head, sequence); loops over the group's
-// query heads and the 128-query tiles at or after the chunk:
-//   S^T = K Q_i^T, dP^T = V dO_i^T (TMEM), P^T and dS^T = P^T (dP^T - Dvec) in
-//   bf16 (shared memory), dV += P^T dO_i, dK += dS^T Q_i (TMEM);
-//   dk = dK / sqrt(D), dv = dV.
+// ---------------------------------------------------------------- dK, dV
+// One CTA per (128-key chunk, kv head, sequence); sub-items = (query head of
+// the group, 64 queries at or after the chunk):  S^T = K Q_i^T, dP^T = V dO_i^T
+// (TMEM), P^T and dS^T = P^T (dP^T - D) (bf16, shared memory), dV += P^T dO_i,
+// dK += dS^T Q_i (TMEM); dk = dK / sqrt(D), dv = dV.
 constexpr int K_OFF_K = 0;
 constexpr int K_OFF_V = K_OFF_K + TILE;
-constexpr int K_OFF_Q = K_OFF_V + TILE;
-constexpr int K_OFF_DO = K_OFF_Q + TILE;
-constexpr int K_OFF_P = K_OFF_DO + TILE;
-constexpr int K_OFF_DS = K_OFF_P + TILE;
-constexpr int K_OFF_BAR = K_OFF_DS + TILE;
-constexpr int K_NBAR = 1 + 1 + 1 + 1 + 1 + 1;  // kvfull, qfull, qempty, sfull, psready, done
+constexpr int K_OFF_RING = K_OFF_V + TILE;          // stage s: Q at +s*2*ST, dO at +s*2*ST + ST
+constexpr int K_OFF_P = K_OFF_RING + NRING * 2 * ST;  // buffer b: P^T at +b*2*PT, dS^T at +b*2*PT + PT
+constexpr int K_OFF_BAR = K_OFF_P + 2 * 2 * PT;
+// kvfull, qfull[3], qempty[3], sfull[2], tfree[2], psready[2], pfree[2], done
+constexpr int K_NBAR = 1 + 3 + 3 + 2 + 2 + 2 + 2 + 1;
 constexpr int K_OFF_MISC = K_OFF_BAR + 8 * K_NBAR;
 constexpr int K_SMEM = K_OFF_MISC + 16 + 1024;
 static_assert(K_SMEM <= 232448, "shared memory");
 
-__global__ void __launch_bounds__(NTHREADS, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                  const __grid_constant__ CUtensorMap kmap,
-                                                                  const __grid_constant__ CUtensorMap vmap,
-                                                                  const __grid_constant__ CUtensorMap domap,
-                                                                  const float* __restrict__ lse,
-                                                                  const float* __restrict__ dvec,
-                                                                  __nv_bfloat16* __restrict__ dk,
-                                                                  __nv_bfloat16* __restrict__ dv_out, int S, int Hq,
-                                                                  int Hkv, float scale, float scale_log2) {
+__global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap64,
+                                                                     const __grid_constant__ CUtensorMap kmap,
+                                                                     const __grid_constant__ CUtensorMap vmap,
+                                                                     const __grid_constant__ CUtensorMap domap64,
+                                                                     const float* __restrict__ lse,
+                                                                     const float* __restrict__ dvec,
+                                                                     __nv_bfloat16* __restrict__ dk,
+                                                                     __nv_bfloat16* __restrict__ dv_out, int S, int Hq,
+                                                                     int Hkv, float scale, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + K_OFF_BAR);
   uint64_t* qfull = kvfull + 1;
-  uint64_t* qempty = qfull + 1;
-  uint64_t* sfull = qempty + 1;
-  uint64_t* psready = sfull + 1;
-  uint64_t* done = psready + 1;
+  uint64_t* qempty = qfull + NRING;
+  uint64_t* sfull = qempty + NRING;
+  uint64_t* tfree = sfull + 2;
+  uint64_t* psready = tfree + 2;
+  uint64_t* pfree = psready + 2;
+  uint64_t* done = pfree + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + K_OFF_MISC);
 
-  const int nt = (S + BQ - 1) / BQ;
   const int jc = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int group = Hq / Hkv;
   const int k0 = jc * BC;
-  const int nq = nt - jc;            // query tiles at or after the chunk
-  const int items = group * nq;
+  const int nsub = (S - k0 + SUB - 1) / SUB;  // 64-query slices at or after the chunk, per head
+  const int items = group * nsub;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 
   if (threadIdx.x == 0) {
     mbar_init(kvfull, 1);
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
-    mbar_init(sfull, 1);
-    mbar_init(psready, 4);
+    for (int i = 0; i < NRING; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&tfree[i], EW);
+      mbar_init(&psready[i], EW);
+      mbar_init(&pfree[i], 1);
+    }
     mbar_init(done, 1);
     fence_barrier_init();
   }
@@ -493,106 +601,136 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_dkv_tc_kernel(const __grid_c
       tma_load_2d(smem + K_OFF_V, &vmap, kvfull, hk * D, row0 + k0);
       tma_load_2d(smem + K_OFF_V + HALF, &vmap, kvfull, hk * D + 64, row0 + k0);
       for (int it = 0; it < items; ++it) {
-        if (!mbar_wait(qempty, ((uint32_t)it & 1u) ^ 1u, 481)) break;
-        const int h = hk * group + it / nq, qs = k0 + (it % nq) * BQ;
-        mbar_arrive_expect_tx(qfull, 2u * TILE);
-        tma_load_2d(smem + K_OFF_Q, &qmap, qfull, h * D, row0 + qs);
-        tma_load_2d(smem + K_OFF_Q + HALF, &qmap, qfull, h * D + 64, row0 + qs);
-        tma_load_2d(smem + K_OFF_DO, &domap, qfull, h * D, row0 + qs);
-        tma_load_2d(smem + K_OFF_DO + HALF, &domap, qfull, h * D + 64, row0 + qs);
+        const int s = it % NRING;
+        if (!mbar_wait(&qempty[s], ((uint32_t)(it / NRING) & 1u) ^ 1u, 481)) break;
+        const int h = hk * group + it / nsub, qs = k0 + (it % nsub) * SUB;
+        uint8_t* dst = smem + K_OFF_RING + s * 2 * ST;
+        mbar_arrive_expect_tx(&qfull[s], 2u * ST);
+        tma_load_2d(dst, &qmap64, &qfull[s], h * D, row0 + qs);
+        tma_load_2d(dst + SHALF, &qmap64, &qfull[s], h * D + 64, row0 + qs);
+        tma_load_2d(dst + ST, &domap64, &qfull[s], h * D, row0 + qs);
+        tma_load_2d(dst + ST + SHALF, &domap64, &qfull[s], h * D + 64, row0 + qs);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = mbar_wait(kvfull, 0, 581);
       const uint32_t kb = smem_u32(smem + K_OFF_K), vb = smem_u32(smem + K_OFF_V);
-      const uint32_t qb = smem_u32(smem + K_OFF_Q), dob = smem_u32(smem + K_OFF_DO);
-      const uint32_t pb = smem_u32(smem + K_OFF_P), dsb = smem_u32(smem + K_OFF_DS);
-      const uint32_t id_k = idesc_bf16(BC, BQ, 0, 0);  // S^T, dP^T: both K-major
-      const uint32_t id_m = idesc_bf16(BC, D, 0, 1);   // P^T dO, dS^T Q: dO / Q MN-major
-      for (int it = 0; ok && it < items; ++it) {
-        if (!mbar_wait(qfull, (uint32_t)it & 1u, 582)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      const uint32_t id_s = idesc_bf16(BC, SUB, 0, 0);  // S^T, dP^T: both K-major
+      const uint32_t id_m = idesc_bf16(BC, D, 0, 1);    // P^T dO, dS^T Q: dO / Q MN-major
+      for (int it = 0; ok && it <= items; ++it) {
+        if (it < items) {
+          const int s = it % NRING, bb = it & 1;
+          if (!mbar_wait(&qfull[s], (uint32_t)(it / NRING) & 1u, 582) ||
+              (it >= 2 && !mbar_wait(&tfree[bb], (uint32_t)((it - 2) >> 1) & 1u, 583))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = smem_u32(smem + K_OFF_RING + s * 2 * ST), dob = qb + ST;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          tc_mma(tmem + T_S, desc_kmajor(kb, kk), desc_kmajor(qb, kk), id_k, kk != 0);
-          tc_mma(tmem + T_DP, desc_kmajor(vb, kk), desc_kmajor(dob, kk), id_k, kk != 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            tc_mma(tmem + T_S + bb * SUB, desc_kmajor(kb, kk), desc_sub_kmajor(qb, kk), id_s, kk != 0);
+            tc_mma(tmem + T_DP + bb * SUB, desc_kmajor(vb, kk), desc_sub_kmajor(dob, kk), id_s, kk != 0);
+          }
+          tc_commit(&sfull[bb]);
         }
-        tc_commit(sfull);
-        if (!mbar_wait(psready, (uint32_t)it & 1u, 583)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        if (it >= 1) {
+          const int p = it - 1, ps = p % NRING, pb = p & 1;
+          if (!mbar_wait(&psready[pb], (uint32_t)(p >> 1) & 1u, 584)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pbase = smem_u32(smem + K_OFF_P + pb * 2 * PT), dsbase = pbase + PT;
+          const uint32_t qb = smem_u32(smem + K_OFF_RING + ps * 2 * ST), dob = qb + ST;
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          tc_mma(tmem + T_DV, desc_kmajor(pb, kk), smem_desc(dob + kk * 2048, HALF, 1024, 2), id_m, (it | kk) != 0);
-          tc_mma(tmem + T_DK, desc_kmajor(dsb, kk), smem_desc(qb + kk * 2048, HALF, 1024, 2), id_m, (it | kk) != 0);
+          for (int kk = 0; kk < SUB / 16; ++kk) {
+            tc_mma(tmem + T_DV, desc_k64(pbase, kk), desc_sub_mnmajor(dob, kk), id_m, (p | kk) != 0);
+            tc_mma(tmem + T_DK, desc_k64(dsbase, kk), desc_sub_mnmajor(qb, kk), id_m, (p | kk) != 0);
+          }
+          tc_commit(&pfree[pb]);
+          tc_commit(&qempty[ps]);
         }
-        tc_commit(qempty);
       }
       tc_commit(done);
-      if (!ok) mbar_wait(done, 0, 584);
+      if (!ok) mbar_wait(done, 0, 585);
     }
   } else {
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;  // key row of the chunk
+    const int quad = warp & 3, part = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;  // key row of the chunk
     const int kj = k0 + r;
-    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    // lse (as log2) and D of this warp's CW queries of sub-item it: lane l holds query
+    // l % CW (shuffles broadcast them); loaded one sub-item ahead
+    float l2own = 0.0f, dvown = 0.0f;
+    auto load_stats = [&](int it2, float& l2, float& dd) {
+      const int h2 = hk * group + it2 / nsub, q = k0 + (it2 % nsub) * SUB + part * CW + (lane % CW);
+      const int64_t ri = ((int64_t)b * Hq + h2) * S + (q < S ? q : 0);
+      l2 = lse[ri] * LOG2E;
+      dd = dvec[ri];
+    };
+    load_stats(0, l2own, dvown);
     bool ok = true;
     for (int it = 0; ok && it < items; ++it) {
-      const int h = hk * group + it / nq, qs = k0 + (it % nq) * BQ;
-      if (!__all_sync(0xffffffffu, mbar_wait(sfull, (uint32_t)it & 1u, 781))) {
+      const int bb = it & 1;
+      const int qs = k0 + (it % nsub) * SUB;
+      float l2next = 0.0f, dvnext = 0.0f;
+      if (it + 1 < items) load_stats(it + 1, l2next, dvnext);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[bb], (uint32_t)(it >> 1) & 1u, 781))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // the previous item's P^T / dS^T (and lse2 / Dvec rows) are free once its dV / dK products are done
-      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(qempty, (uint32_t)(it - 1) & 1u, 782))) {
-        ok = false;
-        break;
-      }
-      const uint32_t prow = smem_u32(smem + K_OFF_P) + r * 128, drow = smem_u32(smem + K_OFF_DS) + r * 128;
-      for (int c4 = 0; c4 < BQ / 32; ++c4) {
-        float sv[32], pv[32];
-        tmem_ld32(tmem + lane_base + T_S + (uint32_t)(c4 * 32), sv);
-        tmem_ld32(tmem + lane_base + T_DP + (uint32_t)(c4 * 32), pv);
-        // lse and Dvec of these 32 queries: lane l loads query l, shuffles broadcast
-        const int qown = qs + c4 * 32 + lane;
-        const int64_t rown = ((int64_t)b * Hq + h) * S + (qown < S ? qown : 0);
-        const float l2own = lse[rown] * LOG2E, dvown = dvec[rown];
-        tc_wait_ld();
-        uint32_t wp[16], wd[16];
+      float sv[CW], pv[CW];
+      tmem_ld16(tmem + lane_base + T_S + bb * SUB + part * CW, sv);
+      tmem_ld16(tmem + lane_base + T_DP + bb * SUB + part * CW, pv);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tfree[bb]);
+      uint32_t wp[CW / 2], wd[CW / 2];
+      if (qs >= k0 + BC && qs + SUB <= S && k0 + BC <= S) {  // every query after every key, all inside S
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int qi = qs + c4 * 32 + e;
+        for (int e = 0; e < CW; e += 2) {
           const float l20 = __shfl_sync(0xffffffffu, l2own, e), l21 = __shfl_sync(0xffffffffu, l2own, e + 1);
           const float d0 = __shfl_sync(0xffffffffu, dvown, e), d1 = __shfl_sync(0xffffffffu, dvown, e + 1);
-          const bool ok0 = kj <= qi && qi < S && kj < S, ok1 = kj <= qi + 1 && qi + 1 < S && kj < S;
-          const float p0 = ok0 ? exp2f(sv[e] * scale_log2 - l20) : 0.0f;
-          const float p1 = ok1 ? exp2f(sv[e + 1] * scale_log2 - l21) : 0.0f;
+          const float p0 = ex2(sv[e] * scale_log2 - l20), p1 = ex2(sv[e + 1] * scale_log2 - l21);
           wp[e / 2] = pack_bf16x2(p0, p1);
           wd[e / 2] = pack_bf16x2(p0 * (pv[e] - d0), p1 * (pv[e + 1] - d1));
         }
+      } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t off = (uint32_t)(c4 >> 1) * HALF + ((uint32_t)(((c4 & 1) * 4 + u) ^ (r & 7)) << 4);
-          st_shared_v4(prow + off, wp[4 * u], wp[4 * u + 1], wp[4 * u + 2], wp[4 * u + 3]);
-          st_shared_v4(drow + off, wd[4 * u], wd[4 * u + 1], wd[4 * u + 2], wd[4 * u + 3]);
+        for (int e = 0; e < CW; e += 2) {
+          const int qi = qs + part * CW + e;
+          const float l20 = __shfl_sync(0xffffffffu, l2own, e), l21 = __shfl_sync(0xffffffffu, l2own, e + 1);
+          const float d0 = __shfl_sync(0xffffffffu, dvown, e), d1 = __shfl_sync(0xffffffffu, dvown, e + 1);
+          const bool ok0 = kj <= qi && qi < S && kj < S, ok1 = kj <= qi + 1 && qi + 1 < S && kj < S;
+          const float p0 = ok0 ? ex2(sv[e] * scale_log2 - l20) : 0.0f;
+          const float p1 = ok1 ? ex2(sv[e + 1] * scale_log2 - l21) : 0.0f;
+          wp[e / 2] = pack_bf16x2(p0, p1);
+          wd[e / 2] = pack_bf16x2(p0 * (pv[e] - d0), p1 * (pv[e + 1] - d1));
         }
       }
+      l2own = l2next;
+      dvown = dvnext;
+      // buffer bb was read by the dV / dK products of sub-item it - 2
+      if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pfree[bb], (uint32_t)((it - 2) >> 1) & 1u, 782))) {
+        ok = false;
+        break;
+      }
+      const uint32_t prow = smem_u32(smem + K_OFF_P + bb * 2 * PT) + r * 128;
+      store_row_units(prow, r, part, wp);
+      store_row_units(prow + PT, r, part, wd);
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(psready);
+      if (lane == 0) mbar_arrive(&psready[bb]);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(done, 0, 783))) {
       tc_fence_after();
       const int64_t off = (((int64_t)b * S + kj) * Hkv + hk) * D;
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      {
+        const int c4 = part;  // 32 of the 128 output columns per warp
         float a[32], c[32];
         tmem_ld32(tmem + lane_base + T_DK + (uint32_t)(c4 * 32), a);
         tmem_ld32(tmem + lane_base + T_DV + (uint32_t)(c4 * 32), c);
@@ -621,9 +759,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_dkv_tc_kernel(const __grid_c
   }
 }
 
-static lsq_status tmap_heads(CUtensorMap* m, const void* base, int64_t rows, int64_t heads) {
+static lsq_status tmap_heads(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, int box_rows = BQ) {
   return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)(heads * D), (uint64_t)rows,
-                        (uint64_t)(heads * D * 2), 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B);
+                        (uint64_t)(heads * D * 2), 64, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // true when the tcgen05 path serves this shape
@@ -645,7 +783,7 @@ lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   if ((s = tmap_heads(&km, k, rows, Hkv)) != LSQ_OK) return s;
   if ((s = tmap_heads(&vm, v, rows, Hkv)) != LSQ_OK) return s;
   const float sl = LOG2E / sqrtf((float)D);
-  attn_fwd_tc_kernel<<<dim3((S + BQ - 1) / BQ, Hq, B), NTHREADS, SMEM_BYTES, st>>>(
+  attn_fwd_tc_kernel<<<dim3((S + BQ - 1) / BQ, Hq, B), FWD_THREADS, SMEM_BYTES, st>>>(
       qm, km, vm, static_cast<__nv_bfloat16*>(o), lse, S, Hq, Hkv, sl);
   LSQ_LAUNCH_CHECK("attn_fwd_tc_kernel");
   return LSQ_OK;
@@ -663,22 +801,27 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
     LSQ_CUDA_TRY(cudaFuncSetAttribute(attn_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM));
     cfg[dev] = 1;
   }
-  CUtensorMap qm, km, vm, dom;
+  CUtensorMap qm, km, vm, dom, qm64, km64, vm64, dom64;
   lsq_status s;
   const int64_t rows = (int64_t)B * S;
   if ((s = tmap_heads(&qm, q, rows, Hq)) != LSQ_OK) return s;
   if ((s = tmap_heads(&km, k, rows, Hkv)) != LSQ_OK) return s;
   if ((s = tmap_heads(&vm, v, rows, Hkv)) != LSQ_OK) return s;
   if ((s = tmap_heads(&dom, d_o, rows, Hq)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&qm64, q, rows, Hq, SUB)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&km64, k, rows, Hkv, SUB)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&vm64, v, rows, Hkv, SUB)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&dom64, d_o, rows, Hq, SUB)) != LSQ_OK) return s;
   const float scale = 1.0f / sqrtf((float)D), sl = LOG2E * scale;
   const int nt = (S + BQ - 1) / BQ;
-  attn_dq_tc_kernel<<<dim3(nt, Hq, B), NTHREADS, Q_SMEM, st>>>(qm, km, vm, dom, lse, dvec,
-                                                               static_cast<__nv_bfloat16*>(dq), S, Hq, Hkv, scale, sl);
+  attn_dq_tc_kernel<<<dim3(nt, Hq, B), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, lse, dvec,
+                                                                  static_cast<__nv_bfloat16*>(dq), S, Hq, Hkv, scale,
+                                                                  sl);
   LSQ_LAUNCH_CHECK("attn_dq_tc_kernel");
-  attn_dkv_tc_kernel<<<dim3(nt, Hkv, B), NTHREADS, K_SMEM, st>>>(qm, km, vm, dom, lse, dvec,
-                                                                 static_cast<__nv_bfloat16*>(dk),
-                                                                 static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv, scale,
-                                                                 sl);
+  attn_dkv_tc_kernel<<<dim3(nt, Hkv, B), BWD_THREADS, K_SMEM, st>>>(qm64, km, vm, dom64, lse, dvec,
+                                                                    static_cast<__nv_bfloat16*>(dk),
+                                                                    static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv,
+                                                                    scale, sl);
   LSQ_LAUNCH_CHECK("attn_dkv_tc_kernel");
   return LSQ_OK;
 }
