@@ -35,6 +35,8 @@
 // wait is bounded (common.cuh); there are no atomics, so results do not
 // depend on timing or on which SM ran which tile.
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstdlib>
 
 #include "common.cuh"
@@ -216,6 +218,15 @@ struct Params {
   int mtiles, tiles;
   __nv_bfloat16* dx;  // DX output [M, K]
   float cb[16];
+  // stream-K: the first dp_tiles tiles (whole rounds) go to the clusters
+  // whole, in the usual order; the weight blocks of the others are cut into
+  // one contiguous range per cluster, and a range that ends inside a tile
+  // leaves an fp32 partial that the cluster finishing the tile adds in cluster
+  // order (see piece_at)
+  int streamk, dp_tiles;
+  float* part;                  // per (cluster, CTA): [H x 8 column chunks][8 float4][128 rows] float4
+  unsigned long long* flags;    // per (cluster, CTA): the epoch once its partial is written
+  unsigned long long epoch;     // unique per launch
 };
 
 struct Maps {
@@ -230,6 +241,37 @@ __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
   int sg = 0;
   while (sg + 1 < p.nseg && i >= p.seg[sg + 1].first) ++sg;
   return sg;
+}
+
+// The j-th piece of work of cluster c of ncl: tile t, weight blocks [k0, k1)
+// (plus the LoRA block when k1 == nkb).  Whole tiles: c, c + ncl, ...  With
+// stream-K the whole tiles stop at dp_tiles; then comes the cluster's range
+// [W c / ncl, W (c+1) / ncl) of the W = (tiles - dp_tiles) x nkb remaining
+// blocks, walked from its last tile to its first, so that a range ending
+// inside a tile writes that tile's partial first and the cluster that
+// finishes the tile, whose range starts inside it, reaches it last.
+__device__ __forceinline__ int64_t sk_bound(const Params& p, int c, int ncl) {
+  return (int64_t)(p.tiles - p.dp_tiles) * p.nkb * c / ncl;
+}
+__device__ __forceinline__ bool piece_at(const Params& p, int c, int ncl, int j, int& t, int& k0, int& k1) {
+  const int whole = p.streamk ? p.dp_tiles : p.tiles;
+  if (c + j * ncl < whole) {
+    t = c + j * ncl;
+    k0 = 0;
+    k1 = p.nkb;
+    return true;
+  }
+  if (!p.streamk) return false;
+  j -= (whole - c + ncl - 1) / ncl;  // the cluster's whole tiles come first
+  const int64_t lo = sk_bound(p, c, ncl), hi = sk_bound(p, c + 1, ncl);
+  if (hi <= lo) return false;
+  const int tr = (int)((hi - 1) / p.nkb) - j;  // tile index within the stream-K part
+  if ((int64_t)tr < lo / p.nkb) return false;
+  const int64_t base = (int64_t)tr * p.nkb;
+  t = p.dp_tiles + tr;
+  k0 = (int)(max(lo, base) - base);
+  k1 = (int)(min(hi, base + p.nkb) - base);
+  return true;
 }
 
 template <int MODE, int H>
@@ -263,7 +305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
-  const int nkb_all = p.nkb + p.lora;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -292,11 +333,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       uint32_t g = 0;
       bool ok = true;
-      for (int t = cid; t < p.tiles && ok; t += ncl) {
+      int t, k0, k1;
+      for (int j = 0; ok && piece_at(p, cid, ncl, j, t, k0, k1); ++j) {
         int m0, sg, n0;
         tile_at<MODE, H>(p, t, m0, sg, n0);
         const int mrow = m0 + (int)rank * BMC, wcol = n0 + (int)rank * BNC;
-        for (int i = 0; i < nkb_all; ++i, ++g) {
+        const int kend = k1 + (k1 == p.nkb ? p.lora : 0);
+        for (int i = k0; i < kend; ++i, ++g) {
           const int s = (int)(g % NST);
           const uint32_t ph = (g / NST) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, 421)) {
@@ -333,9 +376,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const uint32_t id_k = idesc_bf16(2 * BMC, BT, 0, 0);   // both operands K-major
       const uint32_t id_mn = idesc_bf16(2 * BMC, BT, 0, 1);  // DX weight tile: MN-major
       uint32_t g = 0;
-      int j = 0;
       bool ok = true;
-      for (int t = cid; t < p.tiles && ok; t += ncl, ++j) {
+      int t, k0, k1;
+      for (int j = 0; ok && piece_at(p, cid, ncl, j, t, k0, k1); ++j) {
         const int buf = j % NBUF;
         const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
         if (!mbar_wait(&tempty[buf], tph ^ 1u, 521)) {
@@ -344,7 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * H * BT);
-        for (int i = 0; i < nkb_all; ++i, ++g) {
+        const int kend = k1 + (k1 == p.nkb ? p.lora : 0);
+        for (int i = k0; i < kend; ++i, ++g) {
           const int s = (int)(g % NST);
           const uint32_t ph = (g / NST) & 1u;
           if (!mbar_wait(&full[s], ph, 522)) {
@@ -362,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int h = 0; h < H; ++h)
               tc_mma_pair(d + (uint32_t)(h * BT), smem_desc(a_base + h * A_BYTES + kk * 32, 16, 1024, 2), bd,
-                          mn ? id_mn : id_k, (i | kk) != 0);
+                          mn ? id_mn : id_k, (i != k0 || kk != 0));
           }
           tc_commit_pair_mc(&empty[s], 0x3);
         }
@@ -379,10 +423,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int KB = p.K / 64;
     uint32_t g = 0;
     bool ok = true;
-    for (int tt = cid; tt < p.tiles && ok; tt += ncl) {
+    int tt, k0, k1;
+    for (int j = 0; ok && piece_at(p, cid, ncl, j, tt, k0, k1); ++j) {
       int m0, sg, n0;
       tile_at<MODE, H>(p, tt, m0, sg, n0);
       const int wcol = n0 + (int)rank * BNC;
+      const int kend = k1 + (k1 == p.nkb ? p.lora : 0);
       if (MODE == FWD) {
         // thread -> (row, half): consecutive lanes read consecutive 16-byte code
         // chunks and write conflict-free swizzled chunks
@@ -396,16 +442,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         float4 acur = make_float4(0.f, 0.f, 0.f, 0.f), anext = acur;
         float s0 = 0.f, s1 = 0.f, s2 = 0.f;
         if (valid) {
+          const int q0 = k0 & ~3;  // the float4 group of the piece's first block
           if (vec) {
-            acur = __ldg(reinterpret_cast<const float4*>(arow));
-            if (KB > 4) anext = __ldg(reinterpret_cast<const float4*>(arow + 4));
+            if (q0 < KB) acur = __ldg(reinterpret_cast<const float4*>(arow + q0));
+            if (q0 + 4 < KB) anext = __ldg(reinterpret_cast<const float4*>(arow + q0 + 4));
           } else {
-            s0 = __ldg(arow);
-            if (KB > 1) s1 = __ldg(arow + 1);
-            if (KB > 2) s2 = __ldg(arow + 2);
+            if (k0 < KB) s0 = __ldg(arow + k0);
+            if (k0 + 1 < KB) s1 = __ldg(arow + k0 + 1);
+            if (k0 + 2 < KB) s2 = __ldg(arow + k0 + 2);
           }
         }
-        for (int i = 0; i < nkb_all; ++i, ++g) {
+        for (int i = k0; i < kend; ++i, ++g) {
           const int s = (int)(g % NST);
           const uint32_t ph = (g / NST) & 1u;
           const uint32_t fl = cluster_addr(&full[s], 0);
@@ -456,11 +503,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           return (nrow < S.n && kcol < p.K) ? __ldg(S.absmax + (int64_t)nrow * KB + kcol / 64) : 0.0f;
         };
         // absmax of the next four blocks in flight (global-load latency > one block)
-        float a0 = absmax_of(0);
-        float a1 = p.nkb > 1 ? absmax_of(1) : 0.0f;
-        float a2 = p.nkb > 2 ? absmax_of(2) : 0.0f;
-        float a3 = p.nkb > 3 ? absmax_of(3) : 0.0f;
-        for (int i = 0; i < nkb_all; ++i, ++g) {
+        float a0 = k0 < p.nkb ? absmax_of(k0) : 0.0f;
+        float a1 = k0 + 1 < p.nkb ? absmax_of(k0 + 1) : 0.0f;
+        float a2 = k0 + 2 < p.nkb ? absmax_of(k0 + 2) : 0.0f;
+        float a3 = k0 + 3 < p.nkb ? absmax_of(k0 + 3) : 0.0f;
+        for (int i = k0; i < kend; ++i, ++g) {
           const int s = (int)(g % NST);
           const uint32_t ph = (g / NST) & 1u;
           const uint32_t fl = cluster_addr(&full[s], 0);
@@ -494,14 +541,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     // ---------------------------------------------------------------- epilogue (warps 0-3)
     const int e = threadIdx.x;  // TMEM lane = row within the CTA's 128
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    int j = 0;
-    for (int t = cid; t < p.tiles; t += ncl, ++j) {
+    constexpr int PART_FLOATS = H * (BT / 32) * 128 * 32;  // one CTA's accumulator
+    int t, k0, k1;
+    for (int j = 0; piece_at(p, cid, ncl, j, t, k0, k1); ++j) {
       int m0, sg, n0;
       tile_at<MODE, H>(p, t, m0, sg, n0);
       const int buf = j % NBUF;
       const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
       tc_fence_after();
+      if (k1 < p.nkb) {
+        // the range ends inside this tile: park the fp32 partial, then publish it
+        // row e's 32 values of chunk hc as 8 float4, each at [hc][q][e]: a warp's store covers 512
+        // contiguous bytes
+        float4* dst = reinterpret_cast<float4*>(p.part + (int64_t)(cid * 2 + (int)rank) * PART_FLOATS);
+        for (int hc = 0; hc < H * (BT / 32); ++hc) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)(buf * H * BT + hc * 32), v);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[((int64_t)hc * 8 + q) * 128 + e] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        __threadfence();
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        if (e == 0) {
+          asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p.flags + cid * 2 + (int)rank), "l"(p.epoch)
+                       : "memory");
+          mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+        }
+        continue;
+      }
+      // clusters whose ranges end inside this tile, before this one's: their partials, in cluster order
+      int cfirst = cid;
+      if (p.streamk && k0 > 0) {
+        const int64_t tstart = (int64_t)(t - p.dp_tiles) * p.nkb;
+        while (cfirst > 0 && sk_bound(p, cfirst, ncl) > tstart) --cfirst;
+        // ranges are not empty when stream-K runs (at least 4 blocks per cluster, see launch_pair); an
+        // empty one would leave no partial, so it is skipped here and below all the same
+        while (cfirst < cid && sk_bound(p, cfirst + 1, ncl) == sk_bound(p, cfirst, ncl)) ++cfirst;
+        for (int c2 = cfirst; c2 < cid; ++c2) {
+          if (sk_bound(p, c2 + 1, ncl) == sk_bound(p, c2, ncl)) continue;  // an empty range leaves no partial
+          const unsigned long long* f = p.flags + c2 * 2 + (int)rank;
+          unsigned long long v = 0;
+          const uint64_t t0 = globaltimer();
+          while (true) {
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+            if (v == p.epoch) break;
+            if (globaltimer() - t0 > LSQ_WAIT_NS) {
+              report(LSQ_ETIMEOUT, 735);
+              break;
+            }
+          }
+        }
+      }
       const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
       for (int hc = 0; hc < H * (BT / 32); ++hc) {
         const int h = hc / (BT / 32), c = hc % (BT / 32);
@@ -509,7 +603,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int m = m0 + h * BT + (int)rank * BMC + e;
         float v[32];
         tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
-        tc_wait_ld();
+        if (cfirst == cid) {
+          tc_wait_ld();
+        } else {
+          // the first contributor's partial is loaded while the TMEM load completes
+          const float4* src0 = reinterpret_cast<const float4*>(p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS) +
+                               (int64_t)hc * 8 * 128 + e;
+          float4 a[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) a[q] = __ldcg(src0 + q * 128);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            v[4 * q] += a[q].x;
+            v[4 * q + 1] += a[q].y;
+            v[4 * q + 2] += a[q].z;
+            v[4 * q + 3] += a[q].w;
+          }
+          for (int c2 = cfirst + 1; c2 < cid; ++c2) {
+            if (sk_bound(p, c2 + 1, ncl) == sk_bound(p, c2, ncl)) continue;
+            const float4* src = reinterpret_cast<const float4*>(p.part + (int64_t)(c2 * 2 + (int)rank) * PART_FLOATS) +
+                                (int64_t)hc * 8 * 128 + e;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) a[q] = __ldcg(src + q * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              v[4 * q] += a[q].x;
+              v[4 * q + 1] += a[q].y;
+              v[4 * q + 2] += a[q].z;
+              v[4 * q + 3] += a[q].w;
+            }
+          }
+        }
         if (m >= p.M) continue;
 #pragma unroll
         for (int gq = 0; gq < 4; ++gq) {
@@ -877,17 +1002,62 @@ static lsq_status max_pair_clusters(int* out) {
   return LSQ_OK;
 }
 
+// Workspace for stream-K: 4 KB of per-(cluster, CTA) flags, then one 512 x 256
+// fp32 partial per cluster (256 KB per CTA).
+static size_t sk_region_bytes() {
+  int n = 0;
+  if (max_pair_clusters(&n) != LSQ_OK || n < 1) {
+    (void)cudaGetLastError();
+    n = 74;
+  }
+  return 4096 + (size_t)n * 2 * (size_t)(2 * (BT / 32) * 128 * 32 * sizeof(float));
+}
+// unique per launch within the process (a partial's flag holds its launch's value)
+static unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{
+      (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull};
+  return ++counter;
+}
+
 // Rows per pair tile: 512 (H = 2) halves the NF4 decode work per FLOP but
 // leaves no second accumulator for the epilogue to overlap; 256 (H = 1) keeps
-// the overlap.  Pick the one with fewer rounds of work per cluster, an H = 2
+// the overlap.  With a stream-K workspace (sk_ws, at least sk_region_bytes())
+// the last one or two rounds' worth of tiles can be shared out as equal
+// ranges of weight blocks instead (stream-K, H = 2; see piece_at).  The fix-up
+// of the tiles split between clusters (a 256 KB partial written and read back
+// per CTA, one more accumulator hand-over) costs about 0.4 of a tile-time on
+// B200, so it is used where it saves more: at 2048 rows, 96 tiles of 512 rows
+// on 74 clusters take 1.3 + 0.4 tile-times instead of 2 rounds (q/k/v forward:
+// 138 -> 126 us), 448 take 6.05 + 0.4 instead of 7 (gate/up: 423 -> 390 us),
+// 224 take 3.03 + 0.4 instead of 4 (down's dX: 292 -> 257 us with the adapter
+// kernels), while 64 tiles (one round, 10 clusters idle) stay whole.
+// Otherwise pick the tile height with fewer rounds of whole tiles, an H = 2
 // tile costing 1.25 times an H = 1 tile (measured on B200 at the 8B shapes:
-// 1.4-1.7x the TFLOP/s of H = 1 at 2048 rows); LSQ_NF4_TILE_ROWS=256|512
-// overrides.
+// 1.4-1.7x the TFLOP/s of H = 1 at 2048 rows).  LSQ_NF4_TILE_ROWS=256|512
+// forces whole tiles of that height.
 template <int MODE>
-static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, cudaStream_t stream) {
+static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk_ws, size_t sk_bytes,
+                              cudaStream_t stream) {
   int ncl_max = 0;
   lsq_status st = max_pair_clusters(&ncl_max);
   if (st != LSQ_OK) return st;
+  const char* force = getenv("LSQ_NF4_TILE_ROWS");
+  const int64_t tiles2 = (int64_t)((p.M + 2 * BT - 1) / (2 * BT)) * ntiles_n;
+  p.streamk = 0;
+  const double rounds_sk = (double)tiles2 / ncl_max + 0.4;
+  const double rounds_whole = (double)((tiles2 + ncl_max - 1) / ncl_max);
+  const int64_t dp = std::max<int64_t>(0, tiles2 / ncl_max - 1) * ncl_max;
+  if (!force && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 && 2 * tiles2 >= ncl_max &&
+      (tiles2 - dp) * p.nkb >= 4 * (int64_t)ncl_max && rounds_sk < 0.97 * rounds_whole) {
+    p.streamk = 1;
+    p.dp_tiles = (int)dp;  // whole tiles for all but the last one or two rounds' worth
+    p.flags = reinterpret_cast<unsigned long long*>(sk_ws);
+    p.part = reinterpret_cast<float*>(sk_ws + 4096);
+    p.epoch = next_epoch();
+    p.mtiles = (p.M + 2 * BT - 1) / (2 * BT);
+    p.tiles = p.mtiles * ntiles_n;
+    return launch_pair_h<MODE, 2>(maps, p, ncl_max, stream);
+  }
   int64_t best = -1;
   int hbest = 1;
   for (int h = 1; h <= 2; ++h) {
@@ -899,7 +1069,7 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, cudaStre
       hbest = h;
     }
   }
-  if (const char* e = getenv("LSQ_NF4_TILE_ROWS")) {
+  if (const char* e = force) {
     const int rows = atoi(e);
     if (rows == 256) hbest = 1;
     if (rows == 512) hbest = 2;
@@ -1109,7 +1279,7 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
 
 // dX = sum_q dY_q deq(W_q) (+ (s G) A when sg != null)
 lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const __nv_bfloat16* sg,
-                     const __nv_bfloat16* at, void* dx, cudaStream_t stream) {
+                     const __nv_bfloat16* at, void* dx, char* sk_ws, size_t sk_bytes, cudaStream_t stream) {
   const int64_t K = W[0].k_in;
   Params p;
   memset(&p, 0, sizeof(p));
@@ -1139,7 +1309,7 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
     if ((st = tmap_act(&maps.lb[0], at, 64, K, BNC)) != LSQ_OK) return st;
   }
   p.nkb = blocks;
-  return launch_pair<DX>(maps, p, (int)((K + BT - 1) / BT), stream);
+  return launch_pair<DX>(maps, p, (int)((K + BT - 1) / BT), sk_ws, sk_bytes, stream);
 }
 
 }  // namespace tc
@@ -1147,8 +1317,8 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
 
 extern "C" size_t lsq_nf4_lora_fwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
-  return lsq::tc::fwd_plan(nseg, M, k_in, n_out, r).total;
+  if (nseg < 1 || nseg > 3 || r < 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
+  return (r > 0 ? lsq::tc::fwd_plan(nseg, M, k_in, n_out, r).total : 0) + lsq::nf4g::sk_region_bytes();
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
@@ -1178,9 +1348,17 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
   }
   const int rp = tc::rpad(r);
   const tc::FwdPlan f = tc::fwd_plan(nseg, M, K, ns, r);
-  if (r > 0 && (!workspace || workspace_bytes < f.total || !aligned(workspace, 256)))
-    return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, f.total,
+  const size_t base = r > 0 ? f.total : 0;
+  if (r > 0 && (!workspace || workspace_bytes < base || !aligned(workspace, 256)))
+    return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, base,
                 workspace_bytes);
+  // room past the rank-r part: the GEMM's stream-K partials
+  char* sk_ws = nullptr;
+  size_t sk_bytes = 0;
+  if (workspace && aligned(workspace, 256) && workspace_bytes > base) {
+    sk_ws = static_cast<char*>(workspace) + base;
+    sk_bytes = workspace_bytes - base;
+  }
   cudaStream_t cs = (cudaStream_t)stream;
 
   Params p;
@@ -1252,7 +1430,7 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
       if ((st = tmap_act(&maps.lb[i], bpad[i], 64, ns[i], BNC)) != LSQ_OK) return st;
     }
   }
-  return launch_pair<FWD>(maps, p, tiles_n, cs);
+  return launch_pair<FWD>(maps, p, tiles_n, sk_ws, sk_bytes, cs);
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A,

@@ -291,10 +291,18 @@ static lsq_status launch(int nseg, int64_t M, int64_t K, const int64_t* n_out, c
 
 using namespace lsq;
 
+namespace lsq {
+// bytes the backward must have (the rank-r part and the dA / dB partials; 0 without an adapter)
+size_t bwd_base_bytes(int nseg, int64_t M, int64_t k_in, const int64_t* n_out, int r) {
+  if (r <= 0) return 0;
+  return tc::bwd_rank_bytes(nseg, M, k_in, n_out, r) + lg::plan(nseg, M, k_in, n_out).total;
+}
+}  // namespace lsq
+
 extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out,
                                                   int32_t r) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
-  return tc::bwd_rank_bytes(nseg, M, k_in, n_out, r) + lg::plan(nseg, M, k_in, n_out).total;
+  if (nseg < 1 || nseg > 3 || r < 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
+  return bwd_base_bytes(nseg, M, k_in, n_out, r) + nf4g::sk_region_bytes();
 }
 
 extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x,
@@ -336,8 +344,14 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   __nv_bfloat16* su[3] = {nullptr, nullptr, nullptr};
   char* part = nullptr;
   cudaStream_t cs = (cudaStream_t)stream;
+  const size_t need = bwd_base_bytes(nseg, M, K, n_out, r);
+  char* sk_ws = nullptr;
+  size_t sk_bytes = 0;
+  if (workspace && aligned(workspace, 256) && workspace_bytes > need) {  // room for the dX GEMM's stream-K
+    sk_ws = static_cast<char*>(workspace) + need;
+    sk_bytes = workspace_bytes - need;
+  }
   if (r > 0) {
-    const size_t need = lsq_nf4_lora_bwd_workspace_size(nseg, M, K, n_out, r);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
       return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, need,
                   workspace_bytes);
@@ -346,7 +360,7 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, u, r, s, ws, &sg, su, &at, cs)) != LSQ_OK) return st;
     part = ws + tc::bwd_rank_bytes(nseg, M, K, n_out, r);
   }
-  if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, cs)) != LSQ_OK) return st;
+  if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, sk_ws, sk_bytes, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
   return lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, cs);
 }

@@ -60,7 +60,8 @@ extern "C" lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const vo
   using namespace lsq;
   if (!W) return fail(LSQ_EINVAL, "lsq_nf4_lora_bwd_noalloc: NULL weight");
   const int64_t n_out = W->n_out;
-  const size_t need = lsq_nf4_lora_bwd_workspace_size(1, M, W->k_in, &n_out, r);
+  if (M < 1 || r < 0 || r > 64 || W->k_in < 64) return fail(LSQ_EINVAL, "lsq_nf4_lora_bwd_noalloc: bad sizes");
+  const size_t need = bwd_base_bytes(1, M, W->k_in, &n_out, r);
   if (need > noalloc::SCRATCH_BYTES)
     return fail(LSQ_EINVAL,
                 "lsq_nf4_lora_bwd_noalloc: this size needs %zu bytes of scratch, more than the %zu-byte array the "
