@@ -194,6 +194,43 @@ lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
                                   int32_t accumulate, void* workspace, size_t workspace_bytes,
                                   lsq_cuda_stream stream);
 
+/* ------------------------------------------------------------------------
+ * The fused linear with its rank-r operands kept between passes.
+ *
+ * Under gradient checkpointing each layer's forward runs twice, with the
+ * same x, A and B (the pages' trainer recomputes the layer in the backward,
+ * soup-cli docs "Layer Streaming"; the adapters change only at the optimizer
+ * step).  The rank state of one call keeps what both passes and the backward
+ * need from the rank-r side: s*U of each segment [M, 64] bf16 (zero-padded),
+ * B of each segment padded to [n_out, 64], B^T [round16(r), n_out] and the
+ * A^T of all segments side by side [k_in, 64].
+ * lsq_nf4_lora_state_size: bytes of one call's state.
+ * lsq_nf4_lora_fwd_multi_ex: as lsq_nf4_lora_fwd_multi, with
+ *   state        device, 256-byte aligned, lsq_nf4_lora_state_size() bytes
+ *                (may be NULL when r = 0)
+ *   state_ready  0: compute the rank-r side (U into u_out, s*U, the padded
+ *                and transposed operands into state); 1: the state already
+ *                holds them from an earlier call with the same x, A, B, s and
+ *                shapes (the recompute): only the main GEMM runs, and u_out
+ *                is not written.  Y is bit-identical either way.
+ *   workspace    optional scratch (NULL, or lsq_nf4_lora_fwd_workspace_size
+ *                bytes, 256-byte aligned) that lets the GEMM balance its last
+ *                rounds (stream-K)
+ * lsq_nf4_lora_bwd_multi_ex: as lsq_nf4_lora_bwd_multi, reading s*U, B^T and
+ *   A^T from that state instead of rebuilding them (u may then be NULL);
+ *   results bit-identical to lsq_nf4_lora_bwd_multi. */
+size_t lsq_nf4_lora_state_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r);
+lsq_status lsq_nf4_lora_fwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                     const void* const* A, const void* const* B, int32_t r, float s,
+                                     const void* const* residual, void* const* y, float* const* u_out,
+                                     void* state, int32_t state_ready, void* workspace, size_t workspace_bytes,
+                                     lsq_cuda_stream stream);
+lsq_status lsq_nf4_lora_bwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, const void* x, const void* const* dy,
+                                     int64_t M, const void* const* A, const void* const* B, int32_t r, float s,
+                                     const float* const* u, const void* state, void* dx, float* const* dA,
+                                     float* const* dB, int32_t accumulate, void* workspace,
+                                     size_t workspace_bytes, lsq_cuda_stream stream);
+
 /* Backward of one fused linear for callers that cannot allocate device
  * memory.  The paper has no counterpart (its trainer allocates through
  * PyTorch); this entry point exists for code that runs where a cudaMalloc is

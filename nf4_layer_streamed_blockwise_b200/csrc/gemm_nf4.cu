@@ -1107,11 +1107,12 @@ static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int s
   return LSQ_OK;
 }
 
-static lsq_status launch_pad(const ldn::Pad& P, int64_t most, cudaStream_t stream) {
+// jobs 0 .. nseg-1: B^T of each segment; nseg: A^T of all segments; nseg+1 ..: s*U of each segment
+static lsq_status launch_pad(const ldn::Pad& P, int64_t most, cudaStream_t stream, int jobs = -1) {
   int64_t g = (most + 255) / 256;
   if (g > 512) g = 512;
   if (g < 1) g = 1;
-  ldn::lora_pad<<<dim3((unsigned)g, 2 * P.nseg + 1), 256, 0, stream>>>(P);
+  ldn::lora_pad<<<dim3((unsigned)g, jobs > 0 ? jobs : 2 * P.nseg + 1), 256, 0, stream>>>(P);
   LSQ_LAUNCH_CHECK("lora_pad");
   return LSQ_OK;
 }
@@ -1200,6 +1201,48 @@ static BwdPlan bwd_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, in
   return b;
 }
 
+// ---- rank state of one fused linear (the LoRA operands both passes read):
+// s*U per segment [M, 64] | padded B per segment [n, 64] | B^T per segment [rp, n] | A^T side by side [K, 64]
+struct StatePlan {
+  size_t su, bpad[3], bt[3], at, total;
+};
+static StatePlan state_plan(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
+  StatePlan sp;
+  memset(&sp, 0, sizeof(sp));
+  const int rp = rpad(r);
+  sp.su = ldn::round256((size_t)M * 64 * 2);
+  sp.at = ldn::round256((size_t)K * 64 * 2);
+  sp.total = (size_t)nseg * sp.su + sp.at;
+  for (int i = 0; i < nseg; ++i) {
+    sp.bpad[i] = ldn::round256((size_t)n_out[i] * 64 * 2);
+    sp.bt[i] = ldn::round256((size_t)rp * (size_t)n_out[i] * 2);
+    sp.total += sp.bpad[i] + sp.bt[i];
+  }
+  return sp;
+}
+struct StatePtrs {
+  __nv_bfloat16* su[3];
+  __nv_bfloat16* bpad[3];
+  __nv_bfloat16* bt[3];
+  __nv_bfloat16* at;
+};
+static StatePtrs state_ptrs(void* state, int nseg, const StatePlan& sp) {
+  StatePtrs q;
+  memset(&q, 0, sizeof(q));
+  char* cur = static_cast<char*>(state);
+  for (int i = 0; i < nseg; ++i, cur += sp.su) q.su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+  for (int i = 0; i < nseg; ++i) {
+    q.bpad[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+    cur += sp.bpad[i];
+  }
+  for (int i = 0; i < nseg; ++i) {
+    q.bt[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+    cur += sp.bt[i];
+  }
+  q.at = reinterpret_cast<__nv_bfloat16*>(cur);
+  return q;
+}
+
 size_t bwd_rank_bytes(int nseg, int64_t M, int64_t K, const int64_t* n_out, int r) {
   return bwd_plan(nseg, M, K, n_out, r).total;
 }
@@ -1210,7 +1253,7 @@ size_t bwd_rank_bytes(int nseg, int64_t M, int64_t K, const int64_t* n_out, int 
 // layout of bwd_plan.  The bf16 pointers come back through sg / su / at.
 lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* dy, int64_t M, const void* const* A,
                          const void* const* B, const float* const* U, int r, float s, char* ws, __nv_bfloat16** sg,
-                         __nv_bfloat16** su, __nv_bfloat16** at, cudaStream_t stream) {
+                         __nv_bfloat16** su, __nv_bfloat16** at, cudaStream_t stream, const StatePtrs* state) {
   const int64_t K = W[0].k_in;
   const int rp = rpad(r);
   int64_t n_out[3];
@@ -1231,13 +1274,20 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
     cur += b.su;
   }
   lsq_status st;
+  if (state) {  // the forward left B^T, A^T and s*U: only G remains to compute
+    *at = state->at;
+    for (int i = 0; i < nseg; ++i) {
+      bt[i] = state->bt[i];
+      su[i] = state->su[i];
+    }
+  }
   ldn::Pad P;
   memset(&P, 0, sizeof(P));
   int64_t most = K * 64;
   for (int i = 0; i < nseg; ++i) {
     P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
     P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
-    P.U[i] = U[i];
+    P.U[i] = U ? U[i] : nullptr;
     P.Bt[i] = bt[i];
     P.SU[i] = su[i];
     P.n[i] = n_out[i];
@@ -1251,7 +1301,7 @@ lsq_status bwd_rank_part(int nseg, const lsq_nf4_weight* W, const void* const* d
   P.nseg = nseg;
   P.r = r;
   P.rp = rp;
-  if ((st = launch_pad(P, most, stream)) != LSQ_OK) return st;
+  if (!state && (st = launch_pad(P, most, stream)) != LSQ_OK) return st;
 
   ldn::Maps maps;
   memset(&maps, 0, sizeof(maps));
@@ -1321,22 +1371,22 @@ extern "C" size_t lsq_nf4_lora_fwd_workspace_size(int32_t nseg, int64_t M, int64
   return (r > 0 ? lsq::tc::fwd_plan(nseg, M, k_in, n_out, r).total : 0) + lsq::nf4g::sk_region_bytes();
 }
 
-extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
-                                             const void* const* A, const void* const* B, int32_t r, float s,
-                                             const void* const* residual, void* const* y, float* const* u_out,
-                                             void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
-  using namespace lsq;
-  using namespace lsq::nf4g;
-  const char* who = "lsq_nf4_lora_fwd";
+namespace lsq {
+namespace tc {
+using namespace lsq::nf4g;
+
+// Argument checks shared by the forward entry points.
+static lsq_status fwd_checks(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                             const void* const* A, const void* const* B, int32_t r, const void* const* residual,
+                             void* const* y, int64_t* ns, const char* who) {
   if (nseg < 1 || nseg > 3) return fail(LSQ_EINVAL, "%s: 1..3 segments (got %d)", who, nseg);
   if (!W || !x || !y) return fail(LSQ_EINVAL, "%s: NULL argument", who);
   const int64_t K = W[0].k_in;
-  lsq_status st = tc::nf4_checks(M, K, r, who);
+  lsq_status st = nf4_checks(M, K, r, who);
   if (st != LSQ_OK) return st;
   if (!aligned(x, 16)) return fail(LSQ_EINVAL, "%s: x must be 16-byte aligned", who);
-  int64_t ns[3];
   for (int i = 0; i < nseg; ++i) {
-    if ((st = tc::check_weight(W[i], K, who)) != LSQ_OK) return st;
+    if ((st = check_weight(W[i], K, who)) != LSQ_OK) return st;
     ns[i] = W[i].n_out;
     if (!y[i] || !aligned(y[i], 16)) return fail(LSQ_EINVAL, "%s: y[%d] NULL or not 16-byte aligned", who, i);
     const void* res = residual ? residual[i] : nullptr;
@@ -1346,21 +1396,22 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
       if (!aligned(A[i], 16) || !aligned(B[i], 2)) return fail(LSQ_EINVAL, "%s: LoRA A must be 16-byte aligned", who);
     }
   }
-  const int rp = tc::rpad(r);
-  const tc::FwdPlan f = tc::fwd_plan(nseg, M, K, ns, r);
-  const size_t base = r > 0 ? f.total : 0;
-  if (r > 0 && (!workspace || workspace_bytes < base || !aligned(workspace, 256)))
-    return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, base,
-                workspace_bytes);
-  // room past the rank-r part: the GEMM's stream-K partials
-  char* sk_ws = nullptr;
-  size_t sk_bytes = 0;
-  if (workspace && aligned(workspace, 256) && workspace_bytes > base) {
-    sk_ws = static_cast<char*>(workspace) + base;
-    sk_bytes = workspace_bytes - base;
-  }
-  cudaStream_t cs = (cudaStream_t)stream;
+  return LSQ_OK;
+}
 
+// The forward proper.  su / bpad: where s*U and the padded B live (and are
+// written when rank_part); bt / at: when non-null, B^T and A^T are written
+// there too (the backward's operands); sk_ws: room for stream-K.
+static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M, const void* const* A,
+                           const void* const* B, int32_t r, float s, const void* const* residual, void* const* y,
+                           float* const* u_out, __nv_bfloat16* const* su, __nv_bfloat16* const* bpad,
+                           bool rank_part, __nv_bfloat16* const* bt, __nv_bfloat16* at, char* sk_ws,
+                           size_t sk_bytes, cudaStream_t cs) {
+  const int64_t K = W[0].k_in;
+  const int rp = rpad(r);
+  int64_t ns[3];
+  for (int i = 0; i < nseg; ++i) ns[i] = W[i].n_out;
+  lsq_status st;
   Params p;
   memset(&p, 0, sizeof(p));
   p.nseg = nseg;
@@ -1385,52 +1436,126 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
                              BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
   }
-
   if (r > 0) {
-    // workspace: s*U per segment | padded B per segment
-    char* cur = static_cast<char*>(workspace);
-    __nv_bfloat16* su[3];
-    __nv_bfloat16* bpad[3];
-    for (int i = 0; i < nseg; ++i) {
-      su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
-      cur += f.su;
+    if (rank_part) {
+      const FwdPlan f = fwd_plan(nseg, M, K, ns, r);
+      ldn::Maps dm;
+      memset(&dm, 0, sizeof(dm));
+      ldn::Params dp;
+      memset(&dp, 0, sizeof(dp));
+      if ((st = tmap_act(&dm.in[0], x, K, M, ldn::BM)) != LSQ_OK) return st;
+      for (int i = 0; i < nseg; ++i) {
+        if ((st = tmap_act(&dm.wl[i], A[i], K, r, (uint32_t)rp)) != LSQ_OK) return st;
+        dp.out32[i] = u_out ? u_out[i] : nullptr;
+        dp.out16[i] = su[i];
+        dp.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+        dp.Bpad[i] = bpad[i];
+        dp.nB[i] = ns[i];
+      }
+      dp.nprob = 1;
+      dp.M = (int)M;
+      dp.r = r;
+      dp.rp = rp;
+      dp.dx = 0;
+      dp.nseg = nseg;
+      dp.s = s;
+      dp.pr[0].nkb = (int)(K / 64);
+      dp.pr[0].kbps = f.kbps;
+      dp.pr[0].nsub = nseg;
+      dp.pr[0].first = 0;
+      if ((st = launch_down(dm, dp, f.splits, cs)) != LSQ_OK) return st;
+      if (bt && at) {  // B^T and A^T for the backward: the transposition jobs of lora_pad
+        ldn::Pad P;
+        memset(&P, 0, sizeof(P));
+        int64_t most = K * 64;
+        for (int i = 0; i < nseg; ++i) {
+          P.A[i] = static_cast<const __nv_bfloat16*>(A[i]);
+          P.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
+          P.Bt[i] = bt[i];
+          P.n[i] = ns[i];
+          most = std::max<int64_t>(most, (int64_t)rp * ns[i]);
+        }
+        P.At = at;
+        P.K = K;
+        P.M = M;
+        P.s = s;
+        P.nseg = nseg;
+        P.r = r;
+        P.rp = rp;
+        if ((st = launch_pad(P, most, cs, nseg + 1)) != LSQ_OK) return st;
+      }
     }
-    for (int i = 0; i < nseg; ++i) {
-      bpad[i] = reinterpret_cast<__nv_bfloat16*>(cur);
-      cur += f.bpad[i];
-    }
-    ldn::Maps dm;
-    memset(&dm, 0, sizeof(dm));
-    ldn::Params dp;
-    memset(&dp, 0, sizeof(dp));
-    if ((st = tmap_act(&dm.in[0], x, K, M, ldn::BM)) != LSQ_OK) return st;
-    for (int i = 0; i < nseg; ++i) {
-      if ((st = tmap_act(&dm.wl[i], A[i], K, r, (uint32_t)rp)) != LSQ_OK) return st;
-      dp.out32[i] = u_out ? u_out[i] : nullptr;
-      dp.out16[i] = su[i];
-      dp.B[i] = static_cast<const __nv_bfloat16*>(B[i]);
-      dp.Bpad[i] = bpad[i];
-      dp.nB[i] = ns[i];
-    }
-    dp.nprob = 1;
-    dp.M = (int)M;
-    dp.r = r;
-    dp.rp = rp;
-    dp.dx = 0;
-    dp.nseg = nseg;
-    dp.s = s;
-    dp.pr[0].nkb = (int)(K / 64);
-    dp.pr[0].kbps = f.kbps;
-    dp.pr[0].nsub = nseg;
-    dp.pr[0].first = 0;
-    if ((st = launch_down(dm, dp, f.splits, cs)) != LSQ_OK) return st;
-
     for (int i = 0; i < nseg; ++i) {
       if ((st = tmap_act(&maps.la[i], su[i], 64, M, BMC)) != LSQ_OK) return st;
       if ((st = tmap_act(&maps.lb[i], bpad[i], 64, ns[i], BNC)) != LSQ_OK) return st;
     }
   }
   return launch_pair<FWD>(maps, p, tiles_n, sk_ws, sk_bytes, cs);
+}
+
+}  // namespace tc
+}  // namespace lsq
+
+extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                             const void* const* A, const void* const* B, int32_t r, float s,
+                                             const void* const* residual, void* const* y, float* const* u_out,
+                                             void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
+  using namespace lsq;
+  const char* who = "lsq_nf4_lora_fwd";
+  int64_t ns[3];
+  lsq_status st = tc::fwd_checks(nseg, W, x, M, A, B, r, residual, y, ns, who);
+  if (st != LSQ_OK) return st;
+  const int64_t K = W[0].k_in;
+  const tc::FwdPlan f = tc::fwd_plan(nseg, M, K, ns, r);
+  const size_t base = r > 0 ? f.total : 0;
+  if (r > 0 && (!workspace || workspace_bytes < base || !aligned(workspace, 256)))
+    return fail(LSQ_EINVAL, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", who, base,
+                workspace_bytes);
+  // workspace: s*U per segment | padded B per segment | room past it for the GEMM's stream-K partials
+  __nv_bfloat16* su[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* bpad[3] = {nullptr, nullptr, nullptr};
+  char* cur = static_cast<char*>(workspace);
+  if (r > 0) {
+    for (int i = 0; i < nseg; ++i, cur += f.su) su[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+    for (int i = 0; i < nseg; ++i) {
+      bpad[i] = reinterpret_cast<__nv_bfloat16*>(cur);
+      cur += f.bpad[i];
+    }
+  }
+  char* sk_ws = nullptr;
+  size_t sk_bytes = 0;
+  if (workspace && aligned(workspace, 256) && workspace_bytes > base) {
+    sk_ws = static_cast<char*>(workspace) + base;
+    sk_bytes = workspace_bytes - base;
+  }
+  return tc::fwd_impl(nseg, W, x, M, A, B, r, s, residual, y, u_out, su, bpad, true, nullptr, nullptr, sk_ws,
+                      sk_bytes, (cudaStream_t)stream);
+}
+
+extern "C" size_t lsq_nf4_lora_state_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r) {
+  if (nseg < 1 || nseg > 3 || r <= 0 || r > 64 || M < 1 || k_in < 64 || !n_out) return 256;
+  return lsq::tc::state_plan(nseg, M, k_in, n_out, r).total;
+}
+
+extern "C" lsq_status lsq_nf4_lora_fwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                                const void* const* A, const void* const* B, int32_t r, float s,
+                                                const void* const* residual, void* const* y, float* const* u_out,
+                                                void* state, int32_t state_ready, void* workspace,
+                                                size_t workspace_bytes, lsq_cuda_stream stream) {
+  using namespace lsq;
+  const char* who = "lsq_nf4_lora_fwd_ex";
+  int64_t ns[3];
+  lsq_status st = tc::fwd_checks(nseg, W, x, M, A, B, r, residual, y, ns, who);
+  if (st != LSQ_OK) return st;
+  const int64_t K = W[0].k_in;
+  if (r > 0 && (!state || !aligned(state, 256)))
+    return fail(LSQ_EINVAL, "%s: a 256-byte aligned rank state is needed with r > 0", who);
+  if (workspace && !aligned(workspace, 256)) return fail(LSQ_EINVAL, "%s: workspace must be 256-byte aligned", who);
+  tc::StatePtrs q;
+  memset(&q, 0, sizeof(q));
+  if (r > 0) q = tc::state_ptrs(state, nseg, tc::state_plan(nseg, M, K, ns, r));
+  return tc::fwd_impl(nseg, W, x, M, A, B, r, s, residual, y, u_out, q.su, q.bpad, !state_ready, q.bt, q.at,
+                      static_cast<char*>(workspace), workspace ? workspace_bytes : 0, (cudaStream_t)stream);
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A,

@@ -305,12 +305,13 @@ extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64
   return bwd_base_bytes(nseg, M, k_in, n_out, r) + nf4g::sk_region_bytes();
 }
 
-extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x,
-                                             const void* const* dy, int64_t M, const void* const* A,
-                                             const void* const* B, int32_t r, float s, const float* const* u,
-                                             void* dx, float* const* dA, float* const* dB, int32_t accumulate,
-                                             void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
-  const char* who = "lsq_nf4_lora_bwd";
+namespace lsq {
+namespace tc {
+// state: the rank state a forward with lsq_nf4_lora_fwd_multi_ex left, or null
+static lsq_status bwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x, const void* const* dy, int64_t M,
+                           const void* const* A, const void* const* B, int32_t r, float s, const float* const* u,
+                           void* dx, float* const* dA, float* const* dB, int32_t accumulate, void* workspace,
+                           size_t workspace_bytes, cudaStream_t cs, void* state, const char* who) {
   if (nseg < 1 || nseg > 3) return fail(LSQ_EINVAL, "%s: 1..3 segments (got %d)", who, nseg);
   if (!W || !dy) return fail(LSQ_EINVAL, "%s: NULL argument", who);
   lsq_status st = check_device();
@@ -332,9 +333,9 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
     if (!dy[i] || !aligned(dy[i], 16)) return fail(LSQ_EINVAL, "%s: dy[%d] NULL or not 16-byte aligned", who, i);
     n_out[i] = w.n_out;
     if (r > 0) {
-      if (!A || !B || !u || !dA || !dB || !A[i] || !B[i] || !u[i] || !dA[i] || !dB[i])
+      if (!A || !B || !dA || !dB || !A[i] || !B[i] || !dA[i] || !dB[i] || (!state && (!u || !u[i])))
         return fail(LSQ_EINVAL, "%s: LoRA operands/gradients NULL with r > 0", who);
-      if (!aligned(A[i], 16) || !aligned(u[i], 16))
+      if (!aligned(A[i], 16) || (!state && !aligned(u[i], 16)))
         return fail(LSQ_EINVAL, "%s: LoRA A and U must be 16-byte aligned", who);
     }
   }
@@ -343,7 +344,6 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
   __nv_bfloat16* at = nullptr;
   __nv_bfloat16* su[3] = {nullptr, nullptr, nullptr};
   char* part = nullptr;
-  cudaStream_t cs = (cudaStream_t)stream;
   const size_t need = bwd_base_bytes(nseg, M, K, n_out, r);
   char* sk_ws = nullptr;
   size_t sk_bytes = 0;
@@ -357,12 +357,41 @@ extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight*
                   workspace_bytes);
     char* ws = static_cast<char*>(workspace);
     // s*G = s dY B (bf16, the dX kernel's LoRA block and dA's operand), s*U, A^T
-    if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, u, r, s, ws, &sg, su, &at, cs)) != LSQ_OK) return st;
+    StatePtrs sp;
+    if (state) {
+      if (!aligned(state, 256)) return fail(LSQ_EINVAL, "%s: rank state must be 256-byte aligned", who);
+      sp = state_ptrs(state, nseg, state_plan(nseg, M, K, n_out, r));
+    }
+    if ((st = tc::bwd_rank_part(nseg, W, dy, M, A, B, u, r, s, ws, &sg, su, &at, cs, state ? &sp : nullptr)) !=
+        LSQ_OK)
+      return st;
     part = ws + tc::bwd_rank_bytes(nseg, M, K, n_out, r);
   }
   if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, sk_ws, sk_bytes, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
   return lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, cs);
+}
+}  // namespace tc
+}  // namespace lsq
+
+extern "C" lsq_status lsq_nf4_lora_bwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x,
+                                             const void* const* dy, int64_t M, const void* const* A,
+                                             const void* const* B, int32_t r, float s, const float* const* u,
+                                             void* dx, float* const* dA, float* const* dB, int32_t accumulate,
+                                             void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
+  return tc::bwd_impl(nseg, W, x, dy, M, A, B, r, s, u, dx, dA, dB, accumulate, workspace, workspace_bytes,
+                      (cudaStream_t)stream, nullptr, "lsq_nf4_lora_bwd");
+}
+
+extern "C" lsq_status lsq_nf4_lora_bwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, const void* x,
+                                                const void* const* dy, int64_t M, const void* const* A,
+                                                const void* const* B, int32_t r, float s, const float* const* u,
+                                                const void* state, void* dx, float* const* dA, float* const* dB,
+                                                int32_t accumulate, void* workspace, size_t workspace_bytes,
+                                                lsq_cuda_stream stream) {
+  if (r > 0 && !state) return fail(LSQ_EINVAL, "lsq_nf4_lora_bwd_ex: a rank state is needed with r > 0");
+  return tc::bwd_impl(nseg, W, x, dy, M, A, B, r, s, u, dx, dA, dB, accumulate, workspace, workspace_bytes,
+                      (cudaStream_t)stream, const_cast<void*>(state), "lsq_nf4_lora_bwd_ex");
 }
 
 extern "C" lsq_status lsq_nf4_lora_bwd(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M,

@@ -71,6 +71,13 @@ _SIGS = {
     "lsq_nf4_lora_fwd_workspace_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
     "lsq_nf4_lora_fwd": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64, c_void_p, c_void_p, c_int32,
                                    c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "lsq_nf4_lora_state_size": (c_size_t, [c_int32, c_int64, c_int64, ctypes.POINTER(c_int64), c_int32]),
+    "lsq_nf4_lora_fwd_multi_ex": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
+                                            c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
+    "lsq_nf4_lora_bwd_multi_ex": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p, c_int64,
+                                            c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "lsq_nf4_lora_fwd_multi": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
                                          ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int32, c_float,
                                          ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
@@ -154,9 +161,11 @@ def _check(name: str, status: int):
 
 
 # kernel launches issued by the library, counted per call on this side
-# (with a LoRA adapter the fused linear's forward is 4 kernels: operand padding,
-# the split-K rank-r product, its reduction and the main GEMM; the backward is
-# those three, the dX GEMM when dx is wanted, and the dA/dB GEMM with its reduction)
+# (with a LoRA adapter the fused linear's forward is 2 kernels: the rank-r
+# product U = X A^T and the main GEMM, plus the operand transposition when a
+# rank state is filled, and only the main GEMM when the state is reused; the
+# backward is the operand padding (not with a state), G = dY B, the dX GEMM
+# when dx is wanted, and the dA/dB GEMM with its reduction)
 LAUNCHES = [0]
 _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_absmax_double_quantize": 1, "lsq_absmax_expand": 1,
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
@@ -277,7 +286,7 @@ def lsq_nf4_lora_fwd(W: NF4Weight, x, M: int, A, B, r: int, s: float, residual, 
     cw = W.c()
     ws = _fwd_workspace(workspace, [W.n_out], M, W.k_in, r, y.device)
     _call("lsq_nf4_lora_fwd", ctypes.byref(cw), _p(x), M, _p(A), _p(B), r, s, _p(residual), _p(y), _p(u_out),
-          _p(ws), _nbytes(ws), _stream(stream), launches=4 if r > 0 else 1)
+          _p(ws), _nbytes(ws), _stream(stream), launches=2 if r > 0 else 1)
 
 
 def lsq_nf4_lora_fwd_multi(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: float, residual, y, u_out,
@@ -288,7 +297,7 @@ def lsq_nf4_lora_fwd_multi(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: 
     uo = u_out if u_out is not None else [None] * n
     ws = _fwd_workspace(workspace, [w.n_out for w in Ws], M, Ws[0].k_in, r, y[0].device)
     _call("lsq_nf4_lora_fwd_multi", n, cws, _p(x), M, _ptrs(A), _ptrs(B), r, s, _ptrs(res), _ptrs(y), _ptrs(uo),
-          _p(ws), _nbytes(ws), _stream(stream), launches=4 if r > 0 else 1)
+          _p(ws), _nbytes(ws), _stream(stream), launches=2 if r > 0 else 1)
 
 
 def lsq_nf4_lora_bwd_workspace_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
@@ -304,8 +313,36 @@ def lsq_nf4_lora_bwd(W: NF4Weight, x, dy, M: int, A, B, r: int, s: float, u, dx,
           _p(dB), accumulate, _p(workspace), wsb, _stream(stream), launches=_bwd_launches(r, dx))
 
 
-def _bwd_launches(r: int, dx) -> int:
-    return (1 if dx is not None else 0) + (5 if r > 0 else 0)
+def _bwd_launches(r: int, dx, state=None) -> int:
+    return (1 if dx is not None else 0) + ((3 if state is not None else 4) if r > 0 else 0)
+
+
+def lsq_nf4_lora_state_size(n_outs: Sequence[int], M: int, k_in: int, r: int) -> int:
+    arr = (c_int64 * len(n_outs))(*n_outs)
+    return int(_fn("lsq_nf4_lora_state_size")(len(n_outs), M, k_in, arr, r))
+
+
+def lsq_nf4_lora_fwd_multi_ex(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: float, residual, y, u_out,
+                              state, state_ready: bool, workspace=None, stream=None):
+    """The fused forward with a rank state (see include/lsq.h): state_ready=False computes
+    the rank-r side into state (and U into u_out), True reuses it (the recompute)."""
+    n = len(Ws)
+    cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
+    res = residual if residual is not None else [None] * n
+    uo = u_out if u_out is not None else [None] * n
+    launches = 1 if (r == 0 or state_ready) else 3
+    _call("lsq_nf4_lora_fwd_multi_ex", n, cws, _p(x), M, _ptrs(A), _ptrs(B), r, s, _ptrs(res), _ptrs(y), _ptrs(uo),
+          _p(state), 1 if state_ready else 0, _p(workspace), _nbytes(workspace), _stream(stream), launches=launches)
+
+
+def lsq_nf4_lora_bwd_multi_ex(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, state, dx, dA, dB,
+                              accumulate: int, workspace, stream=None):
+    n = len(Ws)
+    cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
+    wsb = _nbytes(workspace)
+    _call("lsq_nf4_lora_bwd_multi_ex", n, cws, _p(x), _ptrs(dy), M, _ptrs(A), _ptrs(B), r, s, _ptrs(u), _p(state),
+          _p(dx), _ptrs(dA), _ptrs(dB), accumulate, _p(workspace), wsb, _stream(stream),
+          launches=_bwd_launches(r, dx, state))
 
 
 def lsq_nf4_lora_bwd_multi(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, dx, dA, dB,

@@ -304,6 +304,20 @@ class StreamedLoraTrainer:
         self.rstd1, self.rstd2, self.rstdf = (torch.empty(M, **f32) for _ in range(3))
         self.lse = torch.empty(self.B * sh.n_q * self.S, **f32)
         self.U = {n: torch.empty(M, r, **f32) for n in S.LINEARS}
+        # rank state of every fused linear of every layer: the first forward fills it, the
+        # checkpoint recompute and the backward read it (no rank-r kernels in the recompute)
+        self.keep_rank_state = True
+        self._groups = {"qkv": ([d, kv, kv], d), "o": ([d], d), "gateup": ([f, f], d), "down": ([d], f)}
+        sizes = {g: _al(L.lsq_nf4_lora_state_size(ns, M, k, r)) for g, (ns, k) in self._groups.items()}
+        per_layer = sum(sizes.values())
+        self.rank_state_buf = torch.empty(sh.n_layers * per_layer, dtype=torch.uint8, device=dev)
+        self.rank_state = []
+        for l in range(sh.n_layers):
+            off, views = l * per_layer, {}
+            for g, sz in sizes.items():
+                views[g] = self.rank_state_buf[off:off + sz]
+                off += sz
+            self.rank_state.append(views)
         self.dh, self.dhmid, self.dx, self.dq, self.da = (torch.empty(M, d, **bf) for _ in range(5))
         self.dk, self.dv = torch.empty(M, kv, **bf), torch.empty(M, kv, **bf)
         self.dmm = torch.empty(M, f, **bf)
@@ -334,9 +348,13 @@ class StreamedLoraTrainer:
         e.record(self.compute)
         self.timeline.append((kind, flops, start, e))
 
-    def _fwd_flops(self, ns, K, r=None):
-        M, r = self.M, self.shape.r if r is None else r
-        return sum(2.0 * M * n * K + 2.0 * M * r * K + 2.0 * M * n * r for n in ns)
+    def _fwd_flops(self, ns, K, r_down=None, r_up=None):
+        """FLOPs of one fused forward call: the base GEMM, U = X A^T when this call computes it
+        (r_down), and the LoRA-up block (r_up)."""
+        M = self.M
+        r_down = self.shape.r if r_down is None else r_down
+        r_up = r_down if r_up is None else r_up
+        return sum(2.0 * M * n * K + 2.0 * M * r_down * K + 2.0 * M * n * r_up for n in ns)
 
     def _bwd_flops(self, ns, K):
         M, r = self.M, self.shape.r
@@ -362,28 +380,36 @@ class StreamedLoraTrainer:
         hin = self.h[l] if hin is None else hin
         hout = self.h[l + 1] if hout is None else hout
         U = self.U if save and adapter else {n: None for n in S.LINEARS}
+        state = adapter and self.keep_rank_state
+        ready = save           # the recompute: the first forward of this step filled the rank state
+        rf = 0 if (state and ready) else r   # rank-r FLOPs done in this call
+
+        def fused(group, Ws, x, names, res, ys):
+            if state:
+                L.lsq_nf4_lora_fwd_multi_ex(Ws, x, M, [A[n] for n in names], [B[n] for n in names], r, s, res, ys,
+                                            None, self.rank_state[l][group], ready, workspace=self.ws_lora)
+            else:
+                L.lsq_nf4_lora_fwd_multi(Ws, x, M, [A[n] for n in names], [B[n] for n in names], r, s, res, ys,
+                                         [U[n] for n in names], workspace=self.ws_lora)
+
         L.lsq_rmsnorm_fwd(hin, W.ln1, self.x1, self.rstd1, M, sh.d, sh.eps)
         t = self._t0()
-        L.lsq_nf4_lora_fwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, M, [A["q"], A["k"], A["v"]],
-                                 [B["q"], B["k"], B["v"]], r, s, None, [self.q, self.k, self.v],
-                                 [U["q"], U["k"], U["v"]], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d, r))
+        fused("qkv", [W.W["q"], W.W["k"], W.W["v"]], self.x1, ["q", "k", "v"], None, [self.q, self.k, self.v])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d, rf, r))
         L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
         L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
         L.lsq_attention_fwd(self.q, self.k, self.v, self.a, self.lse, self.B, self.S, sh.n_q, sh.n_kv, sh.hd)
         t = self._t0()
-        L.lsq_nf4_lora_fwd(W.W["o"], self.a, M, A["o"], B["o"], r, s, hin, self.hmid, U["o"], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d, r))
+        fused("o", [W.W["o"]], self.a, ["o"], [hin], [self.hmid])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.d, rf, r))
         L.lsq_rmsnorm_fwd(self.hmid, W.ln2, self.x2, self.rstd2, M, sh.d, sh.eps)
         t = self._t0()
-        L.lsq_nf4_lora_fwd_multi([W.W["gate"], W.W["up"]], self.x2, M, [A["gate"], A["up"]], [B["gate"], B["up"]],
-                                 r, s, None, [self.g, self.u], [U["gate"], U["up"]], workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d, r))
+        fused("gateup", [W.W["gate"], W.W["up"]], self.x2, ["gate", "up"], None, [self.g, self.u])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.f, sh.f], sh.d, rf, r))
         L.lsq_swiglu_fwd(self.g, self.u, self.mm, M * sh.f)
         t = self._t0()
-        L.lsq_nf4_lora_fwd(W.W["down"], self.mm, M, A["down"], B["down"], r, s, self.hmid, hout, U["down"],
-                           workspace=self.ws_lora)
-        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f, r))
+        fused("down", [W.W["down"]], self.mm, ["down"], [self.hmid], [hout])
+        self._t1(t, "nf4_fwd", self._fwd_flops([sh.d], sh.f, rf, r))
 
     def _layer_bwd(self, l: int, W: LayerView):
         """self.dh holds dLoss/dh[l+1] on entry and dLoss/dh[l] on exit."""
@@ -393,32 +419,37 @@ class StreamedLoraTrainer:
         gA = {n: lp.view(lp.grad, l, n, "A") for n in S.LINEARS}
         gB = {n: lp.view(lp.grad, l, n, "B") for n in S.LINEARS}
         U = self.U
+
+        def fused_bwd(group, Ws, x, dys, names, dx):
+            if self.keep_rank_state:
+                L.lsq_nf4_lora_bwd_multi_ex(Ws, x, dys, M, [A[n] for n in names], [B[n] for n in names], r, s, None,
+                                            self.rank_state[l][group], dx, [gA[n] for n in names],
+                                            [gB[n] for n in names], 0, self.ws_lora)
+            else:
+                L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, [A[n] for n in names], [B[n] for n in names], r, s,
+                                         [U[n] for n in names], dx, [gA[n] for n in names], [gB[n] for n in names],
+                                         0, self.ws_lora)
+
         # down:  h_out = h_mid + down(m)
         t = self._t0()
-        L.lsq_nf4_lora_bwd(W.W["down"], self.mm, self.dh, M, A["down"], B["down"], r, s, U["down"], self.dmm,
-                           gA["down"], gB["down"], 0, self.ws_lora)
+        fused_bwd("down", [W.W["down"]], self.mm, [self.dh], ["down"], self.dmm)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.d], sh.f))
         L.lsq_swiglu_bwd(self.dmm, self.g, self.u, self.g, self.u, M * sh.f)   # g, u <- dg, du
         t = self._t0()
-        L.lsq_nf4_lora_bwd_multi([W.W["gate"], W.W["up"]], self.x2, [self.g, self.u], M, [A["gate"], A["up"]],
-                                 [B["gate"], B["up"]], r, s, [U["gate"], U["up"]], self.dx,
-                                 [gA["gate"], gA["up"]], [gB["gate"], gB["up"]], 0, self.ws_lora)
+        fused_bwd("gateup", [W.W["gate"], W.W["up"]], self.x2, [self.g, self.u], ["gate", "up"], self.dx)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.f, sh.f], sh.d))
         L.lsq_rmsnorm_bwd(self.dx, self.hmid, W.ln2, self.rstd2, self.dh, self.dhmid, M, sh.d)
         # o:  h_mid = h_in + o(a)
         t = self._t0()
-        L.lsq_nf4_lora_bwd(W.W["o"], self.a, self.dhmid, M, A["o"], B["o"], r, s, U["o"], self.da, gA["o"],
-                           gB["o"], 0, self.ws_lora)
+        fused_bwd("o", [W.W["o"]], self.a, [self.dhmid], ["o"], self.da)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.d], sh.d))
         L.lsq_attention_bwd(self.q, self.k, self.v, self.a, self.lse, self.da, self.dq, self.dk, self.dv, self.B,
                             self.S, sh.n_q, sh.n_kv, sh.hd, self.ws_attn)
         L.lsq_rope(self.dq, self.B, self.S, sh.n_q, sh.hd, sh.theta, 1)
         L.lsq_rope(self.dk, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 1)
         t = self._t0()
-        L.lsq_nf4_lora_bwd_multi([W.W["q"], W.W["k"], W.W["v"]], self.x1, [self.dq, self.dk, self.dv], M,
-                                 [A["q"], A["k"], A["v"]], [B["q"], B["k"], B["v"]], r, s,
-                                 [U["q"], U["k"], U["v"]], self.dx, [gA["q"], gA["k"], gA["v"]],
-                                 [gB["q"], gB["k"], gB["v"]], 0, self.ws_lora)
+        fused_bwd("qkv", [W.W["q"], W.W["k"], W.W["v"]], self.x1, [self.dq, self.dk, self.dv], ["q", "k", "v"],
+                  self.dx)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.d, sh.kv, sh.kv], sh.d))
         L.lsq_rmsnorm_bwd(self.dx, self.h[l], W.ln1, self.rstd1, self.dhmid, self.dh, M, sh.d)
 
