@@ -179,7 +179,11 @@ lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const v
  *  dA   device fp32 [r, k_in];  dB device fp32 [n_out, r]
  *  accumulate  0: overwrite dA/dB, 1: add into them
  *  workspace   device scratch of lsq_nf4_lora_bwd_workspace_size() bytes,
- *              256-byte aligned; contents undefined after the call. */
+ *              256-byte aligned; contents undefined after the call.
+ * With dx and r > 0 the dA / dB kernels run on a stream the library keeps
+ * per host thread and device, concurrently with the dX GEMM, ordered by
+ * events: everything enqueued on `stream` after the call sees dA and dB
+ * (also under stream capture, which records the fork and join). */
 size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r);
 lsq_status lsq_nf4_lora_bwd(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M, const void* A,
                             const void* B, int32_t r, float s, const float* u, void* dx, float* dA, float* dB,

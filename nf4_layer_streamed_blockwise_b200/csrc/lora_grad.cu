@@ -307,6 +307,30 @@ extern "C" size_t lsq_nf4_lora_bwd_workspace_size(int32_t nseg, int64_t M, int64
 
 namespace lsq {
 namespace tc {
+// A second stream of this host thread on the current device, with a fork and a
+// join event: the backward runs the dA / dB kernels there, concurrently with
+// the dX GEMM (they read the same s*G and neither writes what the other reads),
+// so that the SMs the dX GEMM leaves idle do that work.  Created on first use,
+// kept for the thread's life.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static lsq_status side_stream(SideStream** out) {
+  thread_local SideStream ss[64];
+  int dev = 0;
+  LSQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(LSQ_EUNSUPPORTED, "side stream: device %d out of range", dev);
+  SideStream& d = ss[dev];
+  if (!d.s) {
+    LSQ_CUDA_TRY(cudaStreamCreateWithFlags(&d.s, cudaStreamNonBlocking));
+    LSQ_CUDA_TRY(cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming));
+    LSQ_CUDA_TRY(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming));
+  }
+  *out = &d;
+  return LSQ_OK;
+}
+
 // state: the rank state a forward with lsq_nf4_lora_fwd_multi_ex left, or null
 static lsq_status bwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x, const void* const* dy, int64_t M,
                            const void* const* A, const void* const* B, int32_t r, float s, const float* const* u,
@@ -367,9 +391,19 @@ static lsq_status bwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
       return st;
     part = ws + tc::bwd_rank_bytes(nseg, M, K, n_out, r);
   }
+  SideStream* side = nullptr;
+  if (dx && r > 0 && (st = side_stream(&side)) != LSQ_OK) return st;
+  if (side) LSQ_CUDA_TRY(cudaEventRecord(side->fork, cs));  // s*G and the operands are in place
+  // dX first, so that its clusters are placed before the dA / dB kernels take the remaining SMs
   if (dx && (st = tc::launch_dx(nseg, W, dy, M, sg, at, dx, sk_ws, sk_bytes, cs)) != LSQ_OK) return st;
   if (r == 0) return LSQ_OK;
-  return lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, cs);
+  if (!side) return lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, cs);
+  LSQ_CUDA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
+  if ((st = lg::launch(nseg, M, K, n_out, x, dy, sg, su, dA, dB, r, rp, accumulate, part, side->s)) != LSQ_OK)
+    return st;
+  LSQ_CUDA_TRY(cudaEventRecord(side->join, side->s));
+  LSQ_CUDA_TRY(cudaStreamWaitEvent(cs, side->join, 0));  // the caller's stream sees dA / dB before anything later
+  return LSQ_OK;
 }
 }  // namespace tc
 }  // namespace lsq
