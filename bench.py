@@ -39,9 +39,11 @@ if ROOT not in sys.path:
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused forward
-# GEMM from an ncu capture (profiles/); None until a capture of the current
-# kernel exists.
-NCU_TRAFFIC = None
+# GEMM (nf4_pair_kernel<FWD>), the mean over the four calls of an 8B layer
+# (q/k/v, o, gate/up, down at 2048 tokens) from one ncu capture of the current
+# kernel (profiles/nf4_pair_kernel_fwd_gateup_8b_m2048.md); applies to the
+# 8B workload only.
+NCU_TRAFFIC_8B = 92.8e6
 
 REASON_COLS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
@@ -431,7 +433,9 @@ def our_arm(a):
                 "roofline": {"bound": "tensor",
                              "kernel": f"fused NF4-LoRA linear, {dom} (nf4_pair_kernel + lora_down_kernel)",
                              "achieved": ach, "peak": peak,
-                             "unit": "TFLOP/s", "frac": ach / peak, "traffic": NCU_TRAFFIC,
+                             "unit": "TFLOP/s", "frac": ach / peak,
+                             "traffic": NCU_TRAFFIC_8B if (shape.name == "llama-3.1-8b" and a.batch * a.seq == 2048)
+                             else None,
                              "peak_source": f"{peaks_src} bf16_tflops_sustained"},
                 "fused_gemm": {"frac_of_sustained_peak": (all_flops / (all_ms * 1e-3) / 1e12) / peak,
                                "frac_of_burst_peak": (all_flops / (all_ms * 1e-3) / 1e12) /
