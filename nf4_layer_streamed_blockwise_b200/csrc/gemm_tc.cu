@@ -6,6 +6,10 @@
 // One CTA computes a 128 x 256 output tile; contraction blocks of 64, 4
 // shared-memory stages filled by TMA (128-byte swizzle; for NN the weight
 // tile is loaded as four 64-column boxes in the MN-major canonical layout).
+// The row-tile index varies fastest across the grid, so the CTAs that share a
+// 256-row slice of the weight run together and read it from DRAM once (for
+// the logits, E [V, d] is 1 GB: with the column index fastest each slice came
+// back from DRAM once per row tile, 16 times at 2048 tokens).
 // Warps 0-3: epilogue (TMEM -> registers -> global, fp32 or bf16); warp 4:
 // TMA producer; warp 5: MMA issuer + TMEM owner.  Bounded waits; no atomics.
 #include "common.cuh"
@@ -46,7 +50,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) dense_gemm_kernel(const __grid_co
   uint64_t* drain = afull + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -195,7 +199,8 @@ extern "C" lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, in
   if ((st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, K, M, K * 2, BK, BM,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
     return st;
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  if ((N + BN - 1) / BN > 65535) return fail(LSQ_EINVAL, "%s: N too large for the grid", who);
+  dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)((N + BN - 1) / BN));
   if (!trans_b) {
     if ((st = encode_tmap_2d(&maps.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b, K, N, K * 2, BK, BN,
                              CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
