@@ -138,7 +138,9 @@ lsq_status lsq_absmax_expand(const uint8_t* codes, const float* params, int64_t 
  * cta_group::2, fp32 accumulation in TMEM).  U is computed first by a split-K
  * tensor-core kernel (kept in fp32 in u_out, and as s*U in bf16 in the
  * workspace); (s U) B^T then runs as one more contraction block of the main
- * GEMM, so Y is rounded to bf16 once.
+ * GEMM, so Y is rounded to bf16 once.  Workspace bytes beyond the rank-r part
+ * (lsq_nf4_lora_fwd_workspace_size includes them) let the GEMM share out its
+ * last rounds of tiles (stream-K); results stay deterministic.
  *  x        device bf16 [M, k_in], 16-byte aligned
  *  A        device bf16 [r, k_in]   (LoRA down), NULL with r = 0 disables LoRA
  *  B        device bf16 [n_out, r]  (LoRA up)

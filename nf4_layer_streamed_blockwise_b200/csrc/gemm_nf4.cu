@@ -3,24 +3,30 @@
 //   FWD: Y = residual + X deq(W)^T + s U B^T,          U = X A^T
 //   DX : dX = sum_seg dY_seg deq(W_seg) + s G A,       G = [G_seg] = [dY_seg B_seg]
 //
-// Main kernel (nf4_pair_kernel).  A cluster of two CTAs on two SMs computes a
-// 256 x 256 output tile with tcgen05.mma.cta_group::2 (M = 256, N = 256): each
-// CTA stages its own 128 activation rows and decodes its own 128 columns of
-// the weight tile into shared memory, and the pair's tensor cores read both
-// halves.  Per SM that is half the weight-operand reads and half the decode
-// work per FLOP of a one-SM 128 x 256 tile, and half the activation reads of
-// a 256 x 128 one.  The kernel is persistent: cluster c takes tiles c, c + C,
-// c + 2C, ... (C clusters, m index fastest so that the clusters in flight
-// share weight columns in L2); the two TMEM accumulators (2 x 256 fp32
-// columns) alternate, so the epilogue of one tile overlaps the main loop of
-// the next.  Six shared-memory stages of 64 contraction steps.
+// Main kernel (nf4_pair_kernel<MODE, H>).  A cluster of two CTAs on two SMs
+// computes a (256 H) x 256 output tile with tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, H instructions per k-step): each CTA stages its own H x 128
+// activation rows and decodes its own 128 columns of the weight tile into
+// shared memory, and the pair's tensor cores read both halves.  Per SM that is
+// half the weight-operand reads and half the decode work per FLOP of a one-SM
+// tile, and with H = 2 each decoded weight tile feeds two 128-row halves.  The
+// kernel is persistent: cluster c takes tiles c, c + C, c + 2C, ... (C
+// clusters, m index fastest so that the clusters in flight share weight
+// columns in L2).  H = 1 alternates two TMEM accumulators (the epilogue of one
+// tile overlaps the main loop of the next, six stages); H = 2 fills TMEM with
+// one 512-column accumulator pair (four stages).  With a stream-K workspace
+// the last round or two of tiles are shared out as equal ranges of weight
+// blocks (see piece_at and launch_pair).
 //
 // The rank-r products stay off the main loop: a split-K tcgen05 kernel
 // (lora_down_kernel) computes U = X A^T (or G = dY B), reduces its splits
-// inside a thread-block cluster and writes U in fp32 (kept for the backward)
-// and s*U (s*G) in bf16, zero-padded to 64 columns.  The main loop then runs (s U) B^T (or (s G) A) as one extra
-// contraction block of width 64 whose two operands are TMA-loaded like the
-// activation tile, so the output is still rounded to bf16 once.
+// inside a thread-block cluster and writes U in fp32 and s*U (s*G) in bf16,
+// zero-padded to 64 columns.  The main loop then runs (s U) B^T (or (s G) A)
+// as one extra contraction block of width 64 whose two operands are
+// TMA-loaded like the activation tile, so the output is still rounded to bf16
+// once.  A rank state (state_plan) keeps s*U and the padded / transposed
+// LoRA operands from a layer's first forward for its checkpoint recompute and
+// backward.
 //
 // Warp roles in each CTA of the pair:
 //   0-3   epilogue: TMEM lanes 0-127 -> the CTA's 128 output rows
@@ -33,7 +39,8 @@
 // have landed and all 16 decoder warps of the pair have arrived; the MMA
 // commit releases the stage in both CTAs at once (commit multicast).  Every
 // wait is bounded (common.cuh); there are no atomics, so results do not
-// depend on timing or on which SM ran which tile.
+// depend on timing or on which SM ran which tile (stream-K partials are added
+// in cluster order).
 #include <algorithm>
 #include <atomic>
 #include <chrono>
