@@ -85,8 +85,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int nt = (S + BQ - 1) / BQ;
-  const int t = nt - 1 - (int)blockIdx.x;  // longest causal tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (head, sequence, query tile), tiles reversed: every head's longest causal tile is dispatched
+  // before any shorter one
+  const int t = nt - 1 - (int)blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0 = t * BQ;
   const int nc = t + 1;  // key chunks at or before this query tile
@@ -352,8 +354,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Q_OFF_MISC);
 
   const int nt = (S + BQ - 1) / BQ;
-  const int t = nt - 1 - (int)blockIdx.x;  // longest causal tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (head, sequence, query tile), tiles reversed: every head's longest causal tile is dispatched
+  // before any shorter one
+  const int t = nt - 1 - (int)blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0 = t * BQ;
   const int nkeys = min(q0 + BQ, S);
@@ -528,6 +532,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
 // the group, 64 queries at or after the chunk):  S^T = K Q_i^T, dP^T = V dO_i^T
 // (TMEM), P^T and dS^T = P^T (dP^T - D) (bf16, shared memory), dV += P^T dO_i,
 // dK += dS^T Q_i (TMEM); dk = dK / sqrt(D), dv = dV.
+// With split = 2 (a GQA group of two or more query heads) the two CTAs of a
+// cluster take half of the group's heads each; both park their dK / dV
+// accumulators in their shared memory and each adds half of the rows of the
+// two through distributed shared memory, rank 0's partial first (the same
+// order in both CTAs).  The first key chunk's CTAs, which bound the kernel's
+// time, then have half as many sub-items.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem4(uint32_t caddr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(caddr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+constexpr int PSTRIDE = 132;  // floats per parked row: 33 x 16 bytes, conflict-free float4 stores
 constexpr int K_OFF_K = 0;
 constexpr int K_OFF_V = K_OFF_K + TILE;
 constexpr int K_OFF_RING = K_OFF_V + TILE;          // stage s: Q at +s*2*ST, dO at +s*2*ST + ST
@@ -538,6 +565,7 @@ constexpr int K_NBAR = 1 + 3 + 3 + 2 + 2 + 2 + 2 + 1;
 constexpr int K_OFF_MISC = K_OFF_BAR + 8 * K_NBAR;
 constexpr int K_SMEM = K_OFF_MISC + 16 + 1024;
 static_assert(K_SMEM <= 232448, "shared memory");
+static_assert(2 * BC * PSTRIDE * 4 <= K_OFF_BAR, "parked dK / dV partials stay below the barriers");
 
 __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap64,
                                                                      const __grid_constant__ CUtensorMap kmap,
@@ -547,7 +575,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
                                                                      const float* __restrict__ dvec,
                                                                      __nv_bfloat16* __restrict__ dk,
                                                                      __nv_bfloat16* __restrict__ dv_out, int S, int Hq,
-                                                                     int Hkv, float scale, float scale_log2) {
+                                                                     int Hkv, float scale, float scale_log2, int split) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + K_OFF_BAR);
@@ -560,11 +588,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
   uint64_t* done = pfree + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + K_OFF_MISC);
 
-  const int jc = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  // grid (kv head x split, sequence, key chunk): the chunks with the most sub-items (the first ones) are
+  // dispatched first, the short ones fill in behind them
+  const int jc = blockIdx.z, b = blockIdx.y;
+  const int hk = (int)blockIdx.x / split, half = (int)blockIdx.x % split;  // half = cluster rank when split
   const int group = Hq / Hkv;
+  const int gh = (group + split - 1) / split;  // query heads of the first half
+  const int h_begin = hk * group + half * gh, nheads = half == 0 ? gh : group - gh;
   const int k0 = jc * BC;
   const int nsub = (S - k0 + SUB - 1) / SUB;  // 64-query slices at or after the chunk, per head
-  const int items = group * nsub;
+  const int items = nheads * nsub;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 
@@ -603,7 +636,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
       for (int it = 0; it < items; ++it) {
         const int s = it % NRING;
         if (!mbar_wait(&qempty[s], ((uint32_t)(it / NRING) & 1u) ^ 1u, 481)) break;
-        const int h = hk * group + it / nsub, qs = k0 + (it % nsub) * SUB;
+        const int h = h_begin + it / nsub, qs = k0 + (it % nsub) * SUB;
         uint8_t* dst = smem + K_OFF_RING + s * 2 * ST;
         mbar_arrive_expect_tx(&qfull[s], 2u * ST);
         tma_load_2d(dst, &qmap64, &qfull[s], h * D, row0 + qs);
@@ -665,7 +698,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
     // l % CW (shuffles broadcast them); loaded one sub-item ahead
     float l2own = 0.0f, dvown = 0.0f;
     auto load_stats = [&](int it2, float& l2, float& dd) {
-      const int h2 = hk * group + it2 / nsub, q = k0 + (it2 % nsub) * SUB + part * CW + (lane % CW);
+      const int h2 = h_begin + it2 / nsub, q = k0 + (it2 % nsub) * SUB + part * CW + (lane % CW);
       const int64_t ri = ((int64_t)b * Hq + h2) * S + (q < S ? q : 0);
       l2 = lse[ri] * LOG2E;
       dd = dvec[ri];
@@ -726,7 +759,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
       __syncwarp();
       if (lane == 0) mbar_arrive(&psready[bb]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(done, 0, 783))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(done, 0, 783)) && split > 1) {
+      // park this CTA's partial dK / dV (fp32) in its shared memory, free now that every product is done
+      tc_fence_after();
+      float* pk = reinterpret_cast<float*>(smem) + (size_t)r * PSTRIDE + part * 32;
+      float* pv = pk + BC * PSTRIDE;
+      float a[32], c[32];
+      tmem_ld32(tmem + lane_base + T_DK + (uint32_t)(part * 32), a);
+      tmem_ld32(tmem + lane_base + T_DV + (uint32_t)(part * 32), c);
+      tc_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        reinterpret_cast<float4*>(pk)[u] = make_float4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+        reinterpret_cast<float4*>(pv)[u] = make_float4(c[4 * u], c[4 * u + 1], c[4 * u + 2], c[4 * u + 3]);
+      }
+    } else if (ok && split == 1) {
       tc_fence_after();
       const int64_t off = (((int64_t)b * S + kj) * Hkv + hk) * D;
       {
@@ -753,6 +800,27 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
   }
   tc_fence_before();
   __syncthreads();
+  if (split > 1) {
+    // rank q adds rows [64 q, 64 q + 64) of both partials, rank 0's first, and writes dK, dV
+    cluster_barrier();
+    const float* pk0 = reinterpret_cast<const float*>(smem);
+    for (int e = (int)threadIdx.x; e < (BC / 2) * 2 * (D / 4); e += blockDim.x) {
+      const int t = e / ((BC / 2) * (D / 4));              // 0: dK, 1: dV
+      const int rr = (e / (D / 4)) % (BC / 2) + half * (BC / 2), c4 = e % (D / 4);
+      const float* loc = pk0 + (size_t)t * BC * PSTRIDE + (size_t)rr * PSTRIDE + c4 * 4;
+      const float4 mine = *reinterpret_cast<const float4*>(loc);
+      const float4 peer = ld_dsmem4(dsmem_addr(loc, (uint32_t)(half ^ 1)));
+      const float4 lo = half == 0 ? mine : peer, hi = half == 0 ? peer : mine;
+      const float f = t == 0 ? scale : 1.0f;
+      const float x0 = (lo.x + hi.x) * f, x1 = (lo.y + hi.y) * f, x2 = (lo.z + hi.z) * f, x3 = (lo.w + hi.w) * f;
+      const int kr = k0 + rr;
+      if (kr < S) {
+        __nv_bfloat16* dst = (t == 0 ? dk : dv_out) + (((int64_t)b * S + kr) * Hkv + hk) * D + c4 * 4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(x0, x1), pack_bf16x2(x2, x3));
+      }
+    }
+    cluster_barrier();  // the peer has read this CTA's partials
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -783,7 +851,7 @@ lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   if ((s = tmap_heads(&km, k, rows, Hkv)) != LSQ_OK) return s;
   if ((s = tmap_heads(&vm, v, rows, Hkv)) != LSQ_OK) return s;
   const float sl = LOG2E / sqrtf((float)D);
-  attn_fwd_tc_kernel<<<dim3((S + BQ - 1) / BQ, Hq, B), FWD_THREADS, SMEM_BYTES, st>>>(
+  attn_fwd_tc_kernel<<<dim3(Hq, B, (S + BQ - 1) / BQ), FWD_THREADS, SMEM_BYTES, st>>>(
       qm, km, vm, static_cast<__nv_bfloat16*>(o), lse, S, Hq, Hkv, sl);
   LSQ_LAUNCH_CHECK("attn_fwd_tc_kernel");
   return LSQ_OK;
@@ -814,15 +882,26 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
   if ((s = tmap_heads(&dom64, d_o, rows, Hq, SUB)) != LSQ_OK) return s;
   const float scale = 1.0f / sqrtf((float)D), sl = LOG2E * scale;
   const int nt = (S + BQ - 1) / BQ;
-  attn_dq_tc_kernel<<<dim3(nt, Hq, B), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, lse, dvec,
+  attn_dq_tc_kernel<<<dim3(Hq, B, nt), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, lse, dvec,
                                                                   static_cast<__nv_bfloat16*>(dq), S, Hq, Hkv, scale,
                                                                   sl);
   LSQ_LAUNCH_CHECK("attn_dq_tc_kernel");
-  attn_dkv_tc_kernel<<<dim3(nt, Hkv, B), BWD_THREADS, K_SMEM, st>>>(qm64, km, vm, dom64, lse, dvec,
-                                                                    static_cast<__nv_bfloat16*>(dk),
-                                                                    static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv,
-                                                                    scale, sl);
-  LSQ_LAUNCH_CHECK("attn_dkv_tc_kernel");
+  const int split = Hq / Hkv >= 2 ? 2 : 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(Hkv * split, B, nt);
+  lc.blockDim = dim3(BWD_THREADS);
+  lc.dynamicSmemBytes = K_SMEM;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  LSQ_CUDA_TRY(cudaLaunchKernelEx(&lc, attn_dkv_tc_kernel, qm64, km, vm, dom64, lse, dvec,
+                                  static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv, scale,
+                                  sl, split));
   return LSQ_OK;
 }
 

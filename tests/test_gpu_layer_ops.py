@@ -89,7 +89,7 @@ def _attn_case(B, Sq, Hq, Hkv, hd, seed):
 
 @pytest.mark.parametrize("B,Sq,Hq,Hkv,hd", [(1, 512, 9, 3, 64), (2, 200, 4, 1, 128), (1, 64, 2, 2, 64),
                                             (1, 1, 4, 2, 128), (2, 130, 8, 2, 128), (2, 512, 32, 8, 128),
-                                            (1, 384, 4, 4, 128)])
+                                            (1, 384, 4, 4, 128), (1, 300, 7, 1, 128), (2, 256, 6, 2, 128)])
 def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
     q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, Sq)
     o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
