@@ -402,7 +402,10 @@ typedef struct lsq_stream_cfg {
 /* Creates the scheduler; ENOTPINNED if any record is not page-locked (the
  * pages fall back to pageable memory silently; here it is an error).  Upload
  * calls that run the gather callback return ECALLBACK if it fails (the slot
- * is then incomplete: destroy the scheduler). */
+ * is then incomplete: destroy the scheduler).  The first upload into each slot
+ * is ordered after all work queued on the compute stream when the scheduler
+ * is created (a caching allocator may hand out slot memory whose previous
+ * owner's kernels are still queued there). */
 lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stream compute, lsq_cuda_stream copy,
                              lsq_stream** out);
 /* Enqueue on the copy stream: wait until the compute stream is done with the

@@ -704,10 +704,13 @@ constexpr int A_BYTES = BM * BK * 2;    // 16 KB
 constexpr int B_BYTES = NMAX * BK * 2;  // 24 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + NST * A_BYTES;
-constexpr int OFF_BAR = OFF_B + NST * B_BYTES;
 constexpr int NBAR = 2 * NST + 1;
-constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+// the weight-side stages hold np_max rows of 128 bytes: sized per launch (bst bytes each), so that
+// narrow problems leave room for two or three CTAs per SM
+__host__ __device__ constexpr int off_bar(int bst) { return OFF_B + NST * bst; }
+__host__ __device__ constexpr int smem_bytes(int bst) { return off_bar(bst) + 8 * NBAR + 16 + 1024; }
+constexpr int OFF_BAR = off_bar(B_BYTES);
+constexpr int SMEM_BYTES = smem_bytes(B_BYTES);
 constexpr int NTHREADS = 192;
 constexpr int TARGET_CTAS = 296;
 constexpr int MAX_SPLITS = 8;  // portable cluster size
@@ -722,6 +725,7 @@ struct Prob {
 struct Params {
   Prob pr[3];
   int nprob, M, r, rp, dx, nseg;
+  int bst;  // bytes of one weight-side stage (np of the widest problem x 128), a multiple of 1024
   float s;
   float* out32[3];          // FWD: U of each segment (or null)
   __nv_bfloat16* out16[3];  // FWD: s*U of each segment [M, 64]; DX: s*G [M, 64] in out16[0]
@@ -756,10 +760,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + off_bar(p.bst));
   uint64_t* empty = full + NST;
   uint64_t* done = empty + NST;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + off_bar(p.bst) + 8 * NBAR);
   float* park = reinterpret_cast<float*>(smem);  // [128][ldp], over the stage buffers once the MMAs are done
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = np <= 32 ? 32u : np <= 64 ? 64u : np <= 128 ? 128u : 256u;
@@ -791,7 +795,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
         const int x = (kb0 + i) * BK;
         tma_load_2d(smem + OFF_A + s * A_BYTES, &maps.in[pi], &full[s], x, m0);
         for (int q = 0; q < P.nsub; ++q)
-          tma_load_2d(smem + OFF_B + s * B_BYTES + q * p.rp * 128, &maps.wl[P.first + q], &full[s], x, 0);
+          tma_load_2d(smem + OFF_B + s * p.bst + q * p.rp * 128, &maps.wl[P.first + q], &full[s], x, 0);
       }
     }
   } else if (warp == 1) {
@@ -807,7 +811,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) lora_down_kernel(const __grid_con
         }
         tc_fence_after();
         const uint32_t a_base = smem_u32(smem + OFF_A + s * A_BYTES);
-        const uint32_t b_base = smem_u32(smem + OFF_B + s * B_BYTES);
+        const uint32_t b_base = smem_u32(smem + OFF_B + s * p.bst);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
           tc_mma(tmem, smem_desc(a_base + kk * 32, 16, 1024, 2), smem_desc(b_base + kk * 32, 16, 1024, 2), id,
@@ -1088,20 +1092,27 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
 }
 
 // one cluster of `splits` CTAs per (row tile, problem)
-static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p, int splits, cudaStream_t stream) {
+static lsq_status launch_down(const ldn::Maps& maps, const ldn::Params& p_in, int splits, cudaStream_t stream) {
   static int configured[64] = {0};
   int dev = 0;
   LSQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     LSQ_CUDA_TRY(cudaFuncSetAttribute(ldn::lora_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       ldn::SMEM_BYTES));
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(ldn::lora_down_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      cudaSharedmemCarveoutMaxShared));
     configured[dev] = 1;
   }
+  ldn::Params p = p_in;
+  int np_max = 0;
+  for (int i = 0; i < p.nprob; ++i) np_max = std::max(np_max, p.pr[i].nsub * p.rp);
+  p.bst = np_max * 128;
+  if (np_max < 16 || np_max > ldn::NMAX || p.bst % 1024 != 0) return fail(LSQ_EINVAL, "lora_down: rank width");
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)((p.M + ldn::BM - 1) / ldn::BM), (unsigned)splits, (unsigned)p.nprob);
   cfg.blockDim = dim3(ldn::NTHREADS);
-  cfg.dynamicSmemBytes = ldn::SMEM_BYTES;
+  cfg.dynamicSmemBytes = ldn::smem_bytes(p.bst);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

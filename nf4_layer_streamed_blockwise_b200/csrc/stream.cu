@@ -443,6 +443,13 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   }
   for (int i = 0; i < cfg->n_slots && e == cudaSuccess; ++i)
     e = cudaEventCreateWithFlags(&st->slot_free[i], cudaEventDisableTiming);
+  // every slot starts out released at this point of the compute stream, so the first upload into it
+  // waits for the work queued there so far: the caller's allocator may have handed out the slots'
+  // memory while kernels that still write its previous contents are queued on that stream
+  for (int i = 0; i < cfg->n_slots && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(st->slot_free[i], st->compute);
+    st->free_recorded[i] = 1;
+  }
   if (e != cudaSuccess) {
     destroy_events(st);
     if (st->reader) {
@@ -450,7 +457,7 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
       delete st->reader;
     }
     delete st;
-    return cuda_fail(e, "lsq_stream_create: cudaEventCreate");
+    return cuda_fail(e, "lsq_stream_create: event create / record");
   }
   *out = st;
   return LSQ_OK;

@@ -6,7 +6,9 @@
   loss curve, for several slot counts (the pages' regression test: a
   streamed run feeds identical quantised bytes to identical kernels);
 * the first layer's LoRA gradients are not zero (the pages' other streaming
-  regression check).
+  regression check);
+* a pageable store is refused, and the first upload into a slot lands after
+  compute-stream work still queued on the slot's recycled memory.
 
 Gradient tolerance: the GPU keeps activations in bf16 between kernels (as the
 pages' bf16 trainer does) while the oracle is fp64 end to end; each bf16
@@ -123,3 +125,29 @@ def test_unpinned_store_is_rejected(lsq):
         lsq.lsq_stream_create(1, 2, 1 << 20, [s.data_ptr() for s in slots], [t.data_ptr()],
                               torch.cuda.current_stream(), torch.cuda.Stream())
     assert e.value.status == 2
+
+
+def test_first_upload_waits_for_queued_compute_work(lsq):
+    """The allocator may hand out a slot's memory while a kernel that writes
+    the block's previous tensor is still queued on the compute stream; the
+    first upload into the slot must land after it (the scheduler orders it
+    behind the compute stream's work at creation)."""
+    nbytes = 64 << 20
+    g = torch.Generator().manual_seed(5)
+    rec = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, generator=g).pin_memory()
+    compute, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    junk = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ptr = junk.data_ptr()
+    torch.cuda._sleep(100_000_000)       # about 50 ms of compute-stream work ahead of ...
+    junk.fill_(7)                        # ... a write into the block
+    del junk
+    slots = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    assert slots[0].data_ptr() == ptr    # the block was recycled with the write still queued
+    st = lsq.lsq_stream_create(1, 2, nbytes, [s.data_ptr() for s in slots], [rec.data_ptr()], compute, copy)
+    try:
+        lsq.lsq_layer_upload_async(st, 0, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(slots[0].cpu(), rec)
+    finally:
+        lsq.lsq_stream_destroy(st)
