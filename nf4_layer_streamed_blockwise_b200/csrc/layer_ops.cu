@@ -99,9 +99,11 @@ __global__ void __launch_bounds__(RN_T) rmsnorm_bwd_kernel(const uint4* __restri
 
 // ---------------------------------------------------------------- RoPE
 // one CTA per (batch, position): the hd/2 angles pos * theta^(-2i/hd) are
-// computed once in double, then every head at that position is rotated.
+// computed once in double, then every head at that position is rotated; with
+// vec (hd a multiple of 16, x 16-byte aligned) each thread moves 8 pairs per
+// 16-byte load and store.
 __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int seq, int heads, int hd,
-                                                   double log_theta, int inverse) {
+                                                   double log_theta, int inverse, int vec) {
   extern __shared__ float cs[];  // [hd/2] cos, [hd/2] sin
   const int half = hd / 2;
   const int64_t bs = blockIdx.x;
@@ -115,6 +117,26 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
   }
   __syncthreads();
   __nv_bfloat16* base = x + bs * (int64_t)heads * hd;
+  if (vec) {
+    const int nv = half / 8;  // 8-pair chunks per head
+    for (int idx = threadIdx.x; idx < heads * nv; idx += blockDim.x) {
+      const int h = idx / nv, i0 = (idx % nv) * 8;
+      uint4* p1 = reinterpret_cast<uint4*>(base + (int64_t)h * hd + i0);
+      uint4* p2 = reinterpret_cast<uint4*>(base + (int64_t)h * hd + half + i0);
+      float a[8], b[8], o1[8], o2[8];
+      unpack8(*p1, a);
+      unpack8(*p2, b);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float c = cs[i0 + k], sn = cs[half + i0 + k];
+        o1[k] = a[k] * c - b[k] * sn;
+        o2[k] = b[k] * c + a[k] * sn;
+      }
+      *p1 = pack8(o1);
+      *p2 = pack8(o2);
+    }
+    return;
+  }
   for (int idx = threadIdx.x; idx < heads * half; idx += blockDim.x) {
     const int h = idx / half, i = idx % half;
     __nv_bfloat16* p = base + (int64_t)h * hd + i;
@@ -417,7 +439,8 @@ extern "C" lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t head
   lsq_status st = check_device();
   if (st != LSQ_OK) return st;
   rope_kernel<<<(unsigned)(batch * seq), 128, (size_t)hd * sizeof(float), (cudaStream_t)stream>>>(
-      static_cast<__nv_bfloat16*>(x), (int)seq, (int)heads, (int)hd, log((double)theta), inverse ? 1 : 0);
+      static_cast<__nv_bfloat16*>(x), (int)seq, (int)heads, (int)hd, log((double)theta), inverse ? 1 : 0,
+      (hd % 16 == 0 && aligned(x, 16)) ? 1 : 0);
   LSQ_LAUNCH_CHECK("rope_kernel");
   return LSQ_OK;
 }

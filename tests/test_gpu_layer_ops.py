@@ -51,7 +51,7 @@ def test_rmsnorm_fwd_bwd(lsq, M, d):
     assert_close_ew(_np(out), dx.numpy() + _np(res), what="rmsnorm dx + res")
 
 
-@pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5)])
+@pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5), (1, 50, 3, 24, 1e4)])
 def test_rope_fwd_and_transpose(lsq, B, Sq, H, hd, theta):
     x = _rand((B, Sq, H, hd), 1.0, 5)
     dy = _rand((B, Sq, H, hd), 1.0, 6)
