@@ -244,23 +244,27 @@ __global__ void __launch_bounds__(128) fwd_kernel(const __nv_bfloat16* __restric
 
 // ---------------------------------------------------------------- backward
 // Dvec[b, h, i] = sum_d dO[b, i, h, d] * O[b, i, h, d]
+// D / 8 lanes per (b, i, h) row (D = 64 or 128: 8 or 16 lanes, a power of two
+// that divides the warp), each on one 16-byte chunk of both rows
 __global__ void __launch_bounds__(256) dvec_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ d_o,
                                                    float* __restrict__ dvec, int64_t rows, int S, int Hq, int D) {
-  // one warp per (b, i, h) row
-  const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= rows) return;
-  const __nv_bfloat16* a = o + w * D;
-  const __nv_bfloat16* g = d_o + w * D;
+  const int lpr = D / 8;
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t w = t / lpr;
+  const int part = (int)(t % lpr);
   float s = 0.0f;
-  for (int c = lane * 2; c < D; c += 64) {
-    const uint32_t av = *reinterpret_cast<const uint32_t*>(a + c), gv = *reinterpret_cast<const uint32_t*>(g + c);
-    s = fmaf(bf16lo(av), bf16lo(gv), s);
-    s = fmaf(bf16hi(av), bf16hi(gv), s);
-  }
+  if (w < rows) {
+    const uint4 av = *reinterpret_cast<const uint4*>(o + w * D + part * 8);
+    const uint4 gv = *reinterpret_cast<const uint4*>(d_o + w * D + part * 8);
+    const uint32_t a[4] = {av.x, av.y, av.z, av.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
-  for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
+    for (int k = 0; k < 4; ++k) {
+      s = fmaf(bf16lo(a[k]), bf16lo(g[k]), s);
+      s = fmaf(bf16hi(a[k]), bf16hi(g[k]), s);
+    }
+  }
+  for (int off = lpr / 2; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);  // within the row's lanes
+  if (w < rows && part == 0) {
     const int64_t h = w % Hq, bi = w / Hq, i = bi % S, b = bi / S;
     dvec[(b * Hq + h) * S + i] = s;
   }
@@ -595,7 +599,7 @@ extern "C" lsq_status lsq_attention_bwd(const void* q, const void* k, const void
   float* dvec = static_cast<float*>(workspace);
   const int64_t rows = batch * seq * hq;
   const cudaStream_t cs = (cudaStream_t)stream;
-  dvec_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, cs>>>((const __nv_bfloat16*)o, (const __nv_bfloat16*)d_o,
+  dvec_kernel<<<(unsigned)((rows * (hd / 8) + 255) / 256), 256, 0, cs>>>((const __nv_bfloat16*)o, (const __nv_bfloat16*)d_o,
                                                                   dvec, rows, (int)seq, (int)hq, (int)hd);
   LSQ_LAUNCH_CHECK("attention dvec_kernel");
   if (atc::bwd_supported(seq, hd))
