@@ -274,6 +274,9 @@ lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, int64_t M, in
  * only", soup-cli diff docs "Layer Streaming", "Honest scope").  Activations
  * bf16, reductions fp32.  Row-major [rows, d] unless stated.
  * ---------------------------------------------------------------------- */
+/* Shape and alignment rules of this section: device pointers; d (feature
+ * count) and n (element count) multiples of 8 with bf16 operands 16-byte
+ * aligned; anything else is EINVAL, with nothing enqueued. */
 /* y = x / sqrt(mean(x^2) + eps) * g;  rstd[row] = 1/sqrt(mean(x^2)+eps) (fp32, may be NULL). */
 lsq_status lsq_rmsnorm_fwd(const void* x, const void* g, void* y, float* rstd, int64_t rows, int64_t d, float eps,
                            lsq_cuda_stream stream);
@@ -282,15 +285,26 @@ lsq_status lsq_rmsnorm_fwd(const void* x, const void* g, void* y, float* rstd, i
 lsq_status lsq_rmsnorm_bwd(const void* dy, const void* x, const void* g, const float* rstd, const void* dres_in,
                            void* dres_out, int64_t rows, int64_t d, lsq_cuda_stream stream);
 /* In-place rotate-half RoPE on x viewed as [batch, seq, heads, hd] at
- * positions 0..seq-1; inverse = 1 applies the transpose (backward). */
+ * positions 0..seq-1; inverse = 1 applies the transpose (backward).  Angles
+ * pos * theta^(-2i/hd) in double, rotation in fp32.  hd even and <= 1024,
+ * theta > 1, else EINVAL; x 2-byte aligned (16-byte loads where hd % 16 == 0
+ * and x is 16-byte aligned). */
 lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t heads, int64_t hd, float theta, int32_t inverse,
                     lsq_cuda_stream stream);
 /* Causal GQA attention: q [B,S,Hq,hd], k,v [B,S,Hkv,hd] -> o [B,S,Hq,hd],
- * lse [B,Hq,S] fp32 (log-sum-exp of the scaled scores).  Scale 1/sqrt(hd). */
+ * lse [B,Hq,S] fp32 (log-sum-exp of the scaled scores).  Scale 1/sqrt(hd).
+ * Query head h reads kv head h / (Hq / Hkv).  hd 64 or 128 (else
+ * EUNSUPPORTED); Hq % Hkv == 0, S <= 2^20, B*S*Hq <= 2^31 and every bf16
+ * pointer 16-byte aligned (else EINVAL).  hd 128 with S <= 512 runs on the
+ * tensor cores (tcgen05), other shapes on mma.sync kernels; both exact
+ * softmax, no atomics. */
 lsq_status lsq_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t batch,
                              int64_t seq, int64_t hq, int64_t hkv, int64_t hd, lsq_cuda_stream stream);
-/* Gradients dq, dk, dv (bf16, same layouts) from do; deterministic.
- * workspace: lsq_attention_bwd_workspace_size() bytes (row dot products). */
+/* Gradients dq, dk, dv (bf16, same layouts) from do, given the forward's o
+ * and lse; deterministic (each output written by one CTA, fixed summation
+ * order).  Same limits as the forward; workspace:
+ * lsq_attention_bwd_workspace_size() bytes (row dot products D =
+ * rowsum(do * o), fp32 [B,Hq,S]); a smaller workspace is EINVAL. */
 size_t lsq_attention_bwd_workspace_size(int64_t batch, int64_t seq, int64_t hq);
 lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,
@@ -301,7 +315,11 @@ lsq_status lsq_swiglu_fwd(const void* g, const void* u, void* m, int64_t n, lsq_
 /* dg, du from dm (dg/du may alias g/u: in-place). */
 lsq_status lsq_swiglu_bwd(const void* dm, const void* g, const void* u, void* dg, void* du, int64_t n,
                           lsq_cuda_stream stream);
-/* h[i, :] = table[ids[i], :], ids int32 device [rows]; table bf16 [vocab, d]. */
+/* h[i, :] = table[ids[i], :], ids int32 device [rows]; table bf16 [vocab, d]
+ * (device memory, or page-locked host memory mapped into the device address
+ * space: the gather then reads the rows over the host link).  An id outside
+ * [0, vocab) gives a zero row and records EINVAL in the device status word
+ * (lsq_device_status). */
 lsq_status lsq_embed_gather(const int32_t* ids, const void* table, void* h, int64_t rows, int64_t d,
                             int64_t vocab, lsq_cuda_stream stream);
 /* Causal-LM cross entropy over logits fp32 [batch*seq, V]: target of row

@@ -1,8 +1,10 @@
 // Causal GQA attention on the 5th-generation tensor cores (tcgen05), for head
 // dim 128 and sequences of at most 512 positions (the 8B and 32B workloads of
-// the streamed trainer).  Forward: one CTA per (128-query tile, query head,
-// sequence).  Backward: a dQ kernel per query tile and a dK/dV kernel per key
-// chunk (below), each the sole owner of its outputs (no atomics).
+// the streamed trainer).  Forward: one CTA per (query head, sequence, 128-query
+// tile).  Backward: a dQ kernel per query tile and a dK/dV kernel per key chunk
+// (below; with a GQA group of two or more, a two-CTA cluster per chunk), each
+// the sole owner of its outputs (no atomics).  Every grid puts the causal tile
+// index slowest and reversed, so the longest tiles of all heads start first.
 //
 //   S_j = Q K_j^T              tcgen05, fp32 in TMEM, 128 columns per 128-key chunk j
 //   P   = exp2(S*c - max)      exact two-pass softmax over the whole row (all of S
