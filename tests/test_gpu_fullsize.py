@@ -1,10 +1,13 @@
-"""Parity at the full 8B sizes, in the launch configuration bench.py times.
+"""Parity at the full 8B and 32B sizes, in the launch configuration bench.py times.
 
-Every fused linear of one 8B decoder layer at 2048 tokens (q/k/v, o,
-gate/up, down), the lm_head GEMMs and the attention of 4 x 512 tokens with
-32 / 8 heads run exactly as in a training step (stream-K workspace, rank
-state filled by the forward and reused by the recompute and the backward,
-dA / dB beside dX).  The fp64 oracle checks sampled outputs it can compute
+Every fused linear of one 8B and one 32B decoder layer at 2048 tokens (q/k/v,
+o, gate/up, down), the 8B lm_head GEMMs and the attention of 4 x 512 tokens
+(32 / 8 and 40 / 8 heads) run exactly as in a training step (stream-K
+workspace, rank state filled by the forward and reused by the recompute and
+the backward, dA / dB beside dX).  The 32B layer's record is 274 MB, above
+the 165 MiB per layer where the pages report silently wrong NF4 gradients
+from the library they build on (Soup README, "Citing Soup": the repaired
+wrong-gradient defect); here its gradients are checked like the 8B ones.  The fp64 oracle checks sampled outputs it can compute
 one by one from its own quantisation of just the rows and blocks involved:
 
 * Y[m, n] for sampled rows m and columns n (oracle quantises W[n, :]);
@@ -58,9 +61,10 @@ def _wd_block(W, kb):
 GROUPS = {"qkv": (["q", "k", "v"], "d"), "o": (["o"], "d"), "gateup": (["gate", "up"], "d"), "down": (["down"], "f")}
 
 
+@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b"])
 @pytest.mark.parametrize("group", list(GROUPS))
-def test_fused_linear_fullsize_sampled(lsq, group):
-    sh = S.LLAMA8B
+def test_fused_linear_fullsize_sampled(lsq, shape, group):
+    sh = S.SHAPES[shape]
     names, kdim = GROUPS[group]
     shapes = sh.linear_shapes()
     K = sh.d if kdim == "d" else sh.f
@@ -136,8 +140,9 @@ def test_lm_head_fullsize_sampled(lsq):
     assert_close(dh.float().cpu().numpy()[np.ix_(rows, dcols)], DL @ E[:, dcols].double().numpy(), what="dh")
 
 
-def test_attention_fullsize_sampled(lsq):
-    sh, B, Sq = S.LLAMA8B, 4, 512
+@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b"])
+def test_attention_fullsize_sampled(lsq, shape):
+    sh, B, Sq = S.SHAPES[shape], 4, 512
     Hq, Hkv, hd = sh.n_q, sh.n_kv, sh.hd
     rng = np.random.default_rng(9)
     q = S.bf16(S.normal_f32(S.DATA_SEED, 520, (B, Sq, Hq, hd)))
