@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused forward
 # GEMM (nf4_pair_kernel<FWD>), the mean over the four calls of an 8B layer
 # (q/k/v, o, gate/up, down at 2048 tokens) from one ncu capture of the current
-# kernel (profiles/nf4_pair_kernel_fwd_gateup_8b_m2048.md); applies to the
+# kernel (the summary of that capture sits under profiles/); applies to the
 # 8B workload only.
 NCU_TRAFFIC_8B = 92.8e6
 
