@@ -60,6 +60,14 @@ int lsq_version(void);
  * synchronous cudaMemcpy): *status = LSQ_OK or the first device-side error
  * since the last read, *where = the site code of that error. */
 lsq_status lsq_device_status(int32_t* status, int32_t* where);
+/* Enqueues on `stream` one thread that waits until the device word *flag
+ * (8-byte aligned) equals value, read with acquire semantics at GPU scope, and
+ * gives up after limit_ns nanoseconds (1 .. 1e10) of the global timer,
+ * recording LSQ_ETIMEOUT at site 901 in the device status word; work after it
+ * on the stream then runs normally.  The same bounded wait guards the fused
+ * GEMM's stream-K partials; exposed for stream-ordered signalling and to test
+ * the timeout path without faulting the device. */
+lsq_status lsq_wait_flag(const uint64_t* flag, uint64_t value, int64_t limit_ns, lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
  * NF4 blockwise format.

@@ -175,6 +175,22 @@ lsq_status encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ba
   return LSQ_OK;
 }
 
+// One thread waits, in stream order, until *flag == value (acquire load at GPU
+// scope), giving up after limit_ns of the global timer with LSQ_ETIMEOUT at
+// site 901: the same bounded wait the stream-K finishers run on their flags.
+__global__ void wait_flag_kernel(const unsigned long long* flag, unsigned long long value, unsigned long long limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flag) : "memory");
+    if (v == value) return;
+    if (globaltimer() - t0 > limit_ns) {
+      report(LSQ_ETIMEOUT, 901);
+      return;
+    }
+  }
+}
+
 }  // namespace lsq
 
 extern "C" {
@@ -196,6 +212,18 @@ const char* lsq_status_str(lsq_status s) {
 const char* lsq_last_error(void) { return lsq::t_msg; }
 
 int lsq_version(void) { return 100; }
+
+lsq_status lsq_wait_flag(const uint64_t* flag, uint64_t value, int64_t limit_ns, lsq_cuda_stream stream) {
+  if (!flag || !lsq::aligned(flag, 8)) return lsq::fail(LSQ_EINVAL, "lsq_wait_flag: flag NULL or not 8-byte aligned");
+  if (limit_ns < 1 || limit_ns > 10000000000ll)
+    return lsq::fail(LSQ_EINVAL, "lsq_wait_flag: limit_ns must be in [1, 1e10] (got %lld)", (long long)limit_ns);
+  lsq_status st = lsq::check_device();
+  if (st != LSQ_OK) return st;
+  lsq::wait_flag_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(reinterpret_cast<const unsigned long long*>(flag),
+                                                          (unsigned long long)value, (unsigned long long)limit_ns);
+  LSQ_LAUNCH_CHECK("wait_flag_kernel");
+  return LSQ_OK;
+}
 
 lsq_status lsq_device_status(int32_t* status, int32_t* where) {
   if (!status || !where) return lsq::fail(LSQ_EINVAL, "NULL output");

@@ -63,6 +63,7 @@ _SIGS = {
     "lsq_last_error": (ctypes.c_char_p, []),
     "lsq_version": (c_int32, []),
     "lsq_device_status": (c_int32, [ctypes.POINTER(c_int32), ctypes.POINTER(c_int32)]),
+    "lsq_wait_flag": (c_int32, [c_void_p, ctypes.c_uint64, c_int64, c_void_p]),
     "lsq_nf4_codebook": (c_int32, [ctypes.POINTER(c_float)]),
     "lsq_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "lsq_nf4_dequantize": (c_int32, [ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p]),
@@ -171,7 +172,7 @@ _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_absmax_double_q
             "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
             "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
             "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1, "lsq_seq_logprob": 2,
-            "lsq_dpo_loss": 1, "lsq_seq_logprob_bwd": 1}
+            "lsq_dpo_loss": 1, "lsq_seq_logprob_bwd": 1, "lsq_wait_flag": 1}
 
 
 def _call(name, *args, launches=None):
@@ -237,6 +238,12 @@ def lsq_device_status():
     s, w = c_int32(0), c_int32(0)
     _call("lsq_device_status", ctypes.byref(s), ctypes.byref(w))
     return s.value, w.value
+
+
+def lsq_wait_flag(flag, value: int, limit_ns: int, stream=None):
+    """Stream-ordered wait until the 8-byte device word `flag` equals `value`; after limit_ns
+    the wait gives up and the device status word reads (LSQ_ETIMEOUT, 901)."""
+    _call("lsq_wait_flag", _p(flag), value, limit_ns, _stream(stream))
 
 
 def lsq_nf4_codebook():

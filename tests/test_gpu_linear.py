@@ -278,3 +278,24 @@ def test_bad_arguments_rejected_before_launch(lsq):
     with pytest.raises(lsq.LsqError):
         lsq.lsq_nf4_lora_fwd(w, x, 4, None, None, 65, 1.0, None, y, None)
     assert lsq.lsq_device_status() == (0, 0)
+
+
+def test_bounded_wait_times_out_and_the_context_survives(lsq):
+    """A wait on a flag that nothing sets runs out after its limit, records
+    LSQ_ETIMEOUT (site 901) in the device status word instead of faulting,
+    and the stream and context stay usable; a flag that is set passes."""
+    flag = torch.zeros(1, dtype=torch.int64, device="cuda")
+    torch.cuda.synchronize()
+    lsq.lsq_device_status()                                # clear anything earlier tests left
+    lsq.lsq_wait_flag(flag, 1, 20_000_000)                 # 20 ms, nothing sets the flag
+    after = torch.ones(8, device="cuda").sum()             # queued behind the wait
+    torch.cuda.synchronize()
+    assert lsq.lsq_device_status() == (4, 901)
+    assert after.item() == 8.0
+    flag.fill_(1)
+    lsq.lsq_wait_flag(flag, 1, 20_000_000)
+    torch.cuda.synchronize()
+    assert lsq.lsq_device_status() == (0, 0)
+    with pytest.raises(lsq.LsqError) as e:
+        lsq.lsq_wait_flag(flag, 1, 0)
+    assert e.value.status == 1
