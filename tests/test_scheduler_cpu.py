@@ -131,3 +131,20 @@ def test_record_layout_double_quant(name):
         assert abs(q.nbytes / 1e6 - 112.5) < 0.2 and abs(f.nbytes / 1e6 - 122.7) < 0.1
     with pytest.raises(ValueError):
         RecordLayout.of(sh, "int8")
+
+
+def test_store_sizes_match_the_pages():
+    """The whole pinned store with double-quantised records comes to the sizes
+    the pages print for the 8B and 3B runs (tests/golden/ram_store_sizes.json);
+    with fp32 absmax it is about 9% larger."""
+    import json
+    import os
+    import synthetic as S
+    from nf4_layer_streamed_blockwise_b200.trainer import RecordLayout
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "ram_store_sizes.json")))
+    for name, gb in gold["values"].items():
+        sh = S.SHAPES[name]
+        dq = sh.n_layers * RecordLayout.of(sh, "dq8").nbytes / 1e9
+        f32 = sh.n_layers * RecordLayout.of(sh, "fp32").nbytes / 1e9
+        assert round(dq, 2) == gb, (name, dq)
+        assert 1.08 < f32 / dq < 1.10, (name, f32, dq)
