@@ -18,6 +18,11 @@
  *    the current device; "host pinned" means page-locked host memory
  *    (cudaHostAlloc / cudaHostRegister).  The library allocates no device
  *    memory on any call below; scratch is passed in as `workspace`.
+ *  - A workspace (and a rank state) serves one call at a time: calls that
+ *    share one must be ordered on the GPU (the same stream, or events).  The
+ *    caller orders its own buffers the same way: memory a call reads or
+ *    writes must not be in use by work on another stream that the call's
+ *    stream does not wait for.
  *  - bf16 means IEEE bfloat16 (2 bytes); all matrices are row-major, dense,
  *    with the stated leading dimension equal to the row length.
  *  - Calls are asynchronous: they validate, enqueue on the given stream and
