@@ -21,11 +21,11 @@ import torch
 
 import synthetic as S
 from oracle import train as OT
-from tolerances import rel_fro
+from test_gpu_model import model_tolerance
+from tolerances import check_model_grads, rel_fro
 
 pytestmark = pytest.mark.gpu
 
-GRAD_REL = 3e-2
 BETA = 0.1
 
 
@@ -61,12 +61,8 @@ def test_dpo_matches_oracle(lsq, shape, B, Sq):
     err = (pi - opi).abs() + (ref - oref).abs()
     bound = BETA * float((err[0::2] + err[1::2]).max()) + 1e-6
     assert abs(loss - oloss) <= bound, (loss, oloss, bound)
-    for l in range(shape.n_layers):
-        for n in S.LINEARS:
-            for ab in ("A", "B"):
-                got = tr.lora.view(g, l, n, ab).cpu().numpy()
-                want = og[l][n][ab].numpy()
-                assert rel_fro(got, want) <= GRAD_REL, (l, n, ab, rel_fro(got, want))
+    check_model_grads(tr.lora, g, og, shape, model_tolerance(shape, B, Sq, og, dpo_beta=BETA, ids=ids),
+                      what=f"dpo {shape.name}")
     tr.close()
 
 

@@ -17,12 +17,12 @@ import torch
 import synthetic as S
 from oracle import nf4
 from oracle import train as OT
-from tolerances import rel_fro
+from test_gpu_model import model_tolerance
+from tolerances import check_model_grads, rel_fro
 
 pytestmark = pytest.mark.gpu
 
 F32 = np.float32
-GRAD_REL = 3e-2
 
 
 def _absmax_cases():
@@ -134,11 +134,8 @@ def test_dq_model_matches_oracle(lsq):
     ol, og, _ = OT.train(shape, layers, S.embeddings(shape), lora, ids, double_quant=True)
     for a, b in zip(losses, ol):
         assert abs(a - b) <= 1e-3 * abs(b), (losses, ol)
-    for l in range(shape.n_layers):
-        for n in S.LINEARS:
-            for ab in ("A", "B"):
-                got = tr.lora.view(g0, l, n, ab).cpu().numpy()
-                assert rel_fro(got, og[l][n][ab].numpy()) <= GRAD_REL, (l, n, ab)
+    check_model_grads(tr.lora, g0, og, shape, model_tolerance(shape, B, Sq, og, double_quant=True),
+                      what=f"dq8 {shape.name}")
     tr.close()
 
 

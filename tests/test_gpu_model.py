@@ -1,7 +1,7 @@
 """Whole-model streamed NF4-LoRA training on the GPU.
 
 * per-step loss against the fp64 oracle within 1e-3 relative (whole-model
-  configurations), LoRA gradients within the derived tolerance below;
+  configurations), LoRA gradients within the tolerance below;
 * streamed == resident bit for bit: logits, every LoRA gradient and a 5-step
   loss curve, for several slot counts (the pages' regression test: a
   streamed run feeds identical quantised bytes to identical kernels);
@@ -10,11 +10,13 @@
 * a pageable store is refused, and the first upload into a slot lands after
   compute-stream work still queued on the slot's recycled memory.
 
-Gradient tolerance: the GPU keeps activations in bf16 between kernels (as the
-pages' bf16 trainer does) while the oracle is fp64 end to end; each bf16
-rounding is a relative 2^-9, and a gradient at layer l passes through about
-10 (L - l) of them, so the whole-model gradient bound is 3e-2 relative
-Frobenius per tensor rather than the single-GEMM 5e-3.
+Gradient tolerance: the GPU keeps activations and their gradients in bf16
+between kernels (as the pages' bf16 trainer does) while the oracle is fp64
+end to end, and the LoRA gradients are sensitive to that storage rounding
+(0.5% to 3% relative Frobenius error per tensor).  bf16_model.py models it
+(the oracle's own forward and backward with bf16 rounding at the kernels'
+storage points); each tensor is held to twice that model's error against the
+oracle, never tighter than 5e-3.
 """
 import math
 
@@ -24,11 +26,11 @@ import torch
 
 import synthetic as S
 from oracle import train as OT
-from tolerances import rel_fro
+import bf16_model as BM
+from tolerances import check_model_grads, record, rel_fro
 
 pytestmark = pytest.mark.gpu
 
-GRAD_REL = 3e-2
 
 
 def _trainer(shape, B, Sq, n_slots, init="host"):
@@ -52,6 +54,27 @@ def _run(tr, shape, B, Sq, steps):
     return losses, grads0, logits0
 
 
+def _check_losses(losses, ref, what):
+    for t, (a, b) in enumerate(zip(losses, ref)):
+        record(f"{what} loss step {t}", "loss", rel=abs(a - b) / abs(b), rel_bound=1e-3)
+        assert abs(a - b) <= 1e-3 * abs(b), (losses, ref)
+
+
+def model_tolerance(shape, B, Sq, ref_grads, double_quant=False, dpo_beta=None, ids=None):
+    """Per-tensor gradient tolerance from the bf16 storage model (bf16_model.tolerance) on the
+    first step's inputs."""
+    from oracle import train as OT
+    layers = [OT.dequantized_layer(S.layer_weights(shape, l), double_quant) for l in range(shape.n_layers)]
+    emb = {k: v.to(torch.float64) for k, v in S.embeddings(shape).items()}
+    ops = [{n: {ab: OT.operand(t[ab]) for ab in ("A", "B")} for n, t in per.items()} for per in S.lora_init(shape)]
+    ids = S.tokens(shape, B, Sq, step=0) if ids is None else ids
+    if dpo_beta is None:
+        mg = BM.sft_grads(ids, layers, emb, ops, shape)
+    else:
+        mg = BM.dpo_grads(ids, layers, emb, ops, shape, dpo_beta)
+    return BM.tolerance(ref_grads, mg)
+
+
 def _oracle(shape, B, Sq, steps):
     layers = [S.layer_weights(shape, l) for l in range(shape.n_layers)]
     emb = S.embeddings(shape)
@@ -66,18 +89,8 @@ def test_model_matches_oracle(lsq, shape, B, Sq):
     tr = _trainer(shape, B, Sq, 2)
     losses, g0, _ = _run(tr, shape, B, Sq, steps)
     ol, og, _ = _oracle(shape, B, Sq, steps)
-    for a, b in zip(losses, ol):
-        assert abs(a - b) <= 1e-3 * abs(b), (losses, ol)
-    worst = 0.0
-    for l in range(shape.n_layers):
-        for n in S.LINEARS:
-            for ab in ("A", "B"):
-                got = tr.lora.view(g0, l, n, ab).cpu().numpy()
-                ref = og[l][n][ab].numpy()
-                rf = rel_fro(got, ref)
-                worst = max(worst, rf)
-                assert rf <= GRAD_REL, (l, n, ab, rf)
-                assert np.abs(got).max() > 0
+    _check_losses(losses, ol, shape.name)
+    check_model_grads(tr.lora, g0, og, shape, model_tolerance(shape, B, Sq, og), what=shape.name)
     tr.close()
 
 
@@ -86,14 +99,8 @@ def test_smollm2_shape_loss_matches_oracle(lsq):
     tr = _trainer(shape, B, Sq, 2)
     losses, g0, _ = _run(tr, shape, B, Sq, steps)
     ol, og, _ = _oracle(shape, B, Sq, steps)
-    for a, b in zip(losses, ol):
-        assert abs(a - b) <= 1e-3 * abs(b), (losses, ol)
-    # layer-0 gradients: non-zero and close to the oracle's
-    for n in S.LINEARS:
-        for ab in ("A", "B"):
-            got = tr.lora.view(g0, 0, n, ab).cpu().numpy()
-            assert np.abs(got).max() > 0
-            assert rel_fro(got, og[0][n][ab].numpy()) <= GRAD_REL
+    _check_losses(losses, ol, shape.name)
+    check_model_grads(tr.lora, g0, og, shape, model_tolerance(shape, B, Sq, og), what=shape.name)
     tr.close()
 
 
