@@ -40,10 +40,29 @@ if ROOT not in sys.path:
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused forward
 # GEMM (nf4_pair_kernel<FWD>), the mean over the four calls of an 8B layer
-# (q/k/v, o, gate/up, down at 2048 tokens) from one ncu capture of the current
-# kernel (the summary of that capture sits under profiles/); applies to the
-# 8B workload only.
-NCU_TRAFFIC_8B = 92.8e6
+# (q/k/v, o, gate/up, down at 2048 tokens), from one ncu capture of the kernel
+# built from the sources whose SHA-256 prefix is given; the figure is reported
+# only while those sources are unchanged (else traffic is null).
+NCU_TRAFFIC = {("llama-3.1-8b", 2048): (92.8e6, None)}
+TRAFFIC_SOURCES = ("nf4_layer_streamed_blockwise_b200/csrc/gemm_nf4.cu",
+                   "nf4_layer_streamed_blockwise_b200/csrc/common.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(shape, tokens):
+    entry = NCU_TRAFFIC.get((shape.name, tokens))
+    if entry is None or entry[1] != kernel_source_hash():
+        return None
+    return entry[0]
+
 
 REASON_COLS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
@@ -76,6 +95,10 @@ def args_():
                         "at exit)")
     p.add_argument("--embed", default="hbm", choices=["hbm", "host"],
                    help="untied embedding table in HBM, or in page-locked host RAM read in place by the gather")
+    p.add_argument("--head", default="hbm", choices=["hbm", "host"],
+                   help="lm_head resident in HBM, or in page-locked host RAM streamed in vocabulary chunks of "
+                        "--head-chunk rows through two HBM buffers for each of its GEMMs")
+    p.add_argument("--head-chunk", type=int, default=8192)
     p.add_argument("--absmax", default="fp32", choices=["fp32", "dq8"],
                    help="absmax format of the streamed records: fp32, or double-quantised (8-bit E4M3 codes, "
                         "blocks of 256, expanded to fp32 in HBM after each upload)")
@@ -187,19 +210,24 @@ def reference_arm(a):
     shape = S.SHAPES[a.shape]
     tokens = 128
     cores = torch.get_num_threads()
-    times = []
+    times, walls = [], []
     for i in range(a.warmup + a.steps):
+        t0 = time.perf_counter()
         t, _ = oracle_sample(shape, tokens)
         if i >= a.warmup:
             times.append(t)
+            walls.append(time.perf_counter() - t0)
     sec = statistics.median(times)
     value = tokens / sec
     sample = (f"one full-width {shape.name} decoder layer fwd+bwd (fp64 oracle) on batch 1 x {tokens} tokens, "
-              f"plus lm_head+CE on 1/32 of the vocabulary; extrapolated x{shape.n_layers} layers, x32 vocab; "
-              f"ms_per_step is a {a.batch} x {a.seq}-token step at that rate")
+              f"plus lm_head+CE on 1/32 of the vocabulary; each timed step is one such sample, and value is the "
+              f"whole-stack rate extrapolated from it (x{shape.n_layers} layers, x32 vocabulary)")
     line = {"impl": "reference", "metric": metric_name(a, shape), "value": value,
             "unit": "tok/s", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": a.batch * a.seq / value * 1e3,
+            "ms_per_step": statistics.median(walls) * 1e3,
+            "value_basis": "extrapolated",
+            "samples_run": a.warmup + a.steps,
+            "extrapolated_ms_per_full_step": a.batch * a.seq / value * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(a, shape),
             "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample},
@@ -214,6 +242,9 @@ def workload_config(a, shape):
     am = "fp32 absmax" if a.absmax == "fp32" else "double-quantised absmax: E4M3 codes, blocks of 256"
     src = "pinned host RAM" if a.source == "ram" else "a store file (disk tier: reader threads, pinned staging)"
     emb = "" if a.embed == "hbm" else ", embedding table in pinned host RAM (zero-copy gather)"
+    if a.head == "host":
+        emb += (f", lm_head in pinned host RAM streamed in {a.head_chunk}-row vocabulary chunks through two HBM "
+                f"buffers for each of its GEMMs")
     return {"workload": f"{shape.name} shape, NF4 (bs64, {am}) base streamed from {src}{emb} through "
                         f"{a.slots} HBM slots, grad checkpointing with re-stream, LoRA r={shape.r} on all linears, "
                         f"{task}, AdamW",
@@ -241,6 +272,7 @@ def metric_name(a, shape):
     dq = ", double-quantised absmax" if a.absmax == "dq8" else ""
     dq += ", disk tier" if a.source == "disk" else ""
     dq += ", host embedding" if a.embed == "host" else ""
+    dq += ", streamed lm_head" if a.head == "host" else ""
     return f"streamed NF4-LoRA {task} tok/s ({short} shape, seq {a.seq}{dq})"
 
 
@@ -327,7 +359,8 @@ def our_arm(a):
         store_path = a.store_path or os.path.join(tempfile.gettempdir(), f"lsq_store_{os.getpid()}_r{rank}.bin")
         if a.store_path and world > 1:
             store_path = f"{a.store_path}.rank{rank}"
-    tiers = dict(absmax=a.absmax, shard=shard, source=a.source, store_path=store_path, embed=a.embed)
+    tiers = dict(absmax=a.absmax, shard=shard, source=a.source, store_path=store_path, embed=a.embed, head=a.head,
+                 head_chunk=a.head_chunk)
     tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", **tiers)
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
@@ -335,22 +368,33 @@ def our_arm(a):
         step_fb(tr, a)
         DP.average_gradients(tr.lora.grad, world)
         tr.optimizer_step()
-    torch.cuda.synchronize()
+    tr.check_device()
     torch.cuda.reset_peak_memory_stats()
     up0, by0, re0 = tr.stats()
+    hb0 = tr.head_stats()[1]
+    # headline: the plain step loop (no timing events inside), clocks sampled beside it
     L.LAUNCHES[0] = 0
     clocks = ClockSampler(local)
     clocks.start()
-    ms, timeline = timed_steps(torch, dist, tr, a.steps, ids_list, world, instrument=True, a=a)
+    ms, _ = timed_steps(torch, dist, tr, a.steps, ids_list, world, a=a)
     clk = clocks.stop()
+    tr.check_device()               # no bounded wait in any kernel ran out during the timed steps
     launches = L.LAUNCHES[0]
     up1, by1, re1 = tr.stats()
+    hb1 = tr.head_stats()[1]
     peak_streamed = torch.cuda.max_memory_allocated()
     ms_step = ms / a.steps
     tokens = a.batch * a.seq
     value = world * tokens * a.steps / (ms * 1e-3)
 
-    # fused-GEMM roofline from the per-launch events of the timed region
+    # instrumented pass (separate): CUDA events around every fused linear (per-kind
+    # TFLOP/s, roofline) and around every compute-stream wait on an upload (exposed copy
+    # per direction)
+    L.lsq_stream_time_waits(tr.sched, 4 * shape.n_layers * a.steps)
+    ms_instr, timeline = timed_steps(torch, dist, tr, a.steps, ids_list, world, instrument=True, a=a)
+    wait_fwd, wait_bwd, n_waits, n_dropped = L.lsq_stream_wait_ms(tr.sched)
+    L.lsq_stream_time_waits(tr.sched, 0)
+    tr.check_device()
     kinds = {}
     for kind, flops, s0, s1 in timeline:
         d = kinds.setdefault(kind, [0.0, 0.0, 0])
@@ -372,7 +416,12 @@ def our_arm(a):
     up_ms = [L.lsq_stream_upload_ms(tr.sched, l) for l in range(shape.n_layers)]
     copy_gbs = rec / (statistics.median(up_ms) * 1e-3) / 1e9
     streaming = {"record_bytes": rec, "uploads_per_step": (up1 - up0) / a.steps,
-                 "h2d_bytes_per_step": (by1 - by0) / a.steps, "reused_per_step": (re1 - re0) / a.steps,
+                 "exposed_copy_ms_fwd": wait_fwd / a.steps, "exposed_copy_ms_bwd": wait_bwd / a.steps,
+                 "exposed_copy_frac": (wait_fwd + wait_bwd) / ms_instr,
+                 "exposed_copy_waits_timed": n_waits, "exposed_copy_waits_dropped": n_dropped,
+                 "ms_per_step_instrumented": ms_instr / a.steps,
+                 "h2d_bytes_per_step": (by1 - by0 + hb1 - hb0) / a.steps, "reused_per_step": (re1 - re0) / a.steps,
+                 "head_h2d_bytes_per_step": (hb1 - hb0) / a.steps,
                  "copy_gbs": copy_gbs, "pinned_h2d_gbs": h2d, "copy_frac_of_link": copy_gbs / h2d,
                  "peak_hbm_gb_streamed": peak_streamed / 1e9}
 
@@ -381,9 +430,12 @@ def our_arm(a):
     loss_host = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(a.steps)]
     ms_e2e, _ = timed_steps(torch, dist, tr, a.steps, ids_list, world, e2e=True, host_ids=host_ids,
                             loss_host=loss_host, a=a)
+    tr.check_device()
     e2e = {"value": world * tokens * a.steps / (ms_e2e * 1e-3), "unit": "tok/s",
            "h2d_bytes_per_step": tokens * 4 + streaming["h2d_bytes_per_step"], "d2h_bytes_per_step": 4,
-           "h2d_breakdown": {"token_ids": tokens * 4, "layer_records": streaming["h2d_bytes_per_step"]},
+           "h2d_breakdown": {"token_ids": tokens * 4,
+                             "layer_records": streaming["h2d_bytes_per_step"] - streaming["head_h2d_bytes_per_step"],
+                             "lm_head_chunks": streaming["head_h2d_bytes_per_step"]},
            "last_loss": float(loss_host[-1].item())}
     store = tr
     tr.close()
@@ -398,9 +450,9 @@ def our_arm(a):
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats()
         ms_r, _ = timed_steps(torch, dist, trr, a.steps, ids_list, world, a=a)
+        trr.check_device()
         streaming["ms_per_step_resident"] = ms_r / a.steps
-        streaming["exposed_copy_ms_per_step"] = max(0.0, ms_step - ms_r / a.steps)
-        streaming["exposed_copy_frac"] = streaming["exposed_copy_ms_per_step"] / ms_step
+        streaming["streamed_minus_resident_ms"] = max(0.0, ms_step - ms_r / a.steps)
         streaming["peak_hbm_gb_resident"] = torch.cuda.max_memory_allocated() / 1e9
         trr.close()
         del trr
@@ -411,7 +463,8 @@ def our_arm(a):
         ids1 = [t[:1] for t in ids_list]
         for i in range(2):
             tr1.train_step(ids1[i % 4])
-        ms1, _ = timed_steps(torch, dist, tr1, a.steps, ids1, world)
+        ms1, _ = timed_steps(torch, dist, tr1, a.steps, ids1, world, a=a)
+        tr1.check_device()
         batch1 = {"tok_s": world * a.seq * a.steps / (ms1 * 1e-3), "ms_per_step": ms1 / a.steps}
         tr1.close()
         del tr1
@@ -436,13 +489,12 @@ def our_arm(a):
                              "kernel": f"fused NF4-LoRA linear, {dom} (nf4_pair_kernel + lora_down_kernel)",
                              "achieved": ach, "peak": peak,
                              "unit": "TFLOP/s", "frac": ach / peak,
-                             "traffic": NCU_TRAFFIC_8B if (shape.name == "llama-3.1-8b" and a.batch * a.seq == 2048)
-                             else None,
+                             "traffic": measured_traffic(shape, a.batch * a.seq),
                              "peak_source": f"{peaks_src} bf16_tflops_sustained"},
                 "fused_gemm": {"frac_of_sustained_peak": (all_flops / (all_ms * 1e-3) / 1e12) / peak,
                                "frac_of_burst_peak": (all_flops / (all_ms * 1e-3) / 1e12) /
                                peaks.get("bf16_tflops", 1650.0),
-                               "share_of_step": all_ms / a.steps / ms_step, "by_kind": gemm},
+                               "share_of_step": all_ms / ms_instr, "by_kind": gemm},
                 "streaming": streaming, "clocks": clk, "e2e": e2e, "gpu_launches": launches,
                 "cpu_baseline": cpu}
         if batch1:

@@ -250,24 +250,66 @@ lsq_status lsq_nf4_lora_bwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, cons
                                      float* const* dB, int32_t accumulate, void* workspace,
                                      size_t workspace_bytes, lsq_cuda_stream stream);
 
+/* Rotate-half RoPE of some segments' outputs, applied in the fused GEMM's
+ * epilogue (the decoder layer rotates q and k right after their projections;
+ * Llama / Qwen stacks, soup-cli diff, docs "Layer Streaming", "Honest scope"):
+ * rows of y are (sequence, position) with position = row % seq, heads of hd
+ * columns; column i < hd/2 of a head pairs with column i + hd/2 and the pair
+ * is rotated by the angle position * theta^(-2i/hd), in fp32 on the
+ * accumulator, before the one bf16 rounding of the output.
+ *  table:    (cos, sin) fp32 pairs [seq][hd/2] from lsq_rope_table (device,
+ *            16-byte aligned)
+ *  seq, hd:  positions per sequence (M a multiple of seq); head dim 64, 128
+ *            or 256
+ *  segments: bit i set = rotate segment i (n_out a multiple of hd, no
+ *            residual) */
+typedef struct lsq_rope_spec {
+  const float* table;
+  int32_t seq, hd;
+  int32_t segments;
+} lsq_rope_spec;
+/* cos and sin of position * theta^(-2i/hd) for positions 0..seq-1 and
+ * i = 0..hd/2-1, computed in double and rounded to fp32 (the angles lsq_rope
+ * uses), written as (cos, sin) pairs into table [seq][hd/2][2] (device).
+ * hd even and <= 1024, theta > 1, seq >= 1, else EINVAL. */
+lsq_status lsq_rope_table(float theta, int64_t seq, int64_t hd, float* table, lsq_cuda_stream stream);
+/* lsq_nf4_lora_fwd_multi_ex with the RoPE of the segments `rope` marks
+ * (NULL or no bits: exactly lsq_nf4_lora_fwd_multi_ex); with state NULL,
+ * lsq_nf4_lora_fwd_multi (the rank-r operands rebuilt in the workspace of
+ * lsq_nf4_lora_fwd_workspace_size bytes) with that RoPE.  EINVAL for a bad
+ * spec, before anything is enqueued. */
+lsq_status lsq_nf4_lora_fwd_multi_ex2(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                      const void* const* A, const void* const* B, int32_t r, float s,
+                                      const void* const* residual, void* const* y, float* const* u_out,
+                                      void* state, int32_t state_ready, const lsq_rope_spec* rope,
+                                      void* workspace, size_t workspace_bytes, lsq_cuda_stream stream);
+
 /* Backward of one fused linear for callers that cannot allocate device
  * memory.  The paper has no counterpart (its trainer allocates through
  * PyTorch); this entry point exists for code that runs where a cudaMalloc is
  * unavailable or unsafe: inside a host framework that owns the whole device
- * pool and exposes no allocator, in a process held to a hard memory cap where
- * an extra allocation mid-step could fail, or while a stream is being
- * captured.
+ * pool and exposes no allocator, or in a process held to a hard memory cap
+ * where an extra allocation mid-step could fail.
  * Same arguments and results as lsq_nf4_lora_bwd without the workspace: the
- * scratch (G, the padded LoRA operands and the partial sums) is one fixed array
- * of lsq_nf4_lora_bwd_noalloc_max_scratch() bytes (32 MiB) in the device memory of
- * every GPU that loads the library, held until the process exits.  A size
- * whose scratch exceeds it is rejected with LSQ_EINVAL before anything is
- * enqueued.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current: make that first call
- * before any stream capture.  Every call shares the array and leaves its last
+ * scratch (G, the padded LoRA operands, the partial sums and the dX GEMM's
+ * stream-K partials) is one fixed array of
+ * lsq_nf4_lora_bwd_noalloc_max_scratch() bytes (64 MiB) in the device memory
+ * of every GPU that loads the library, held until the process exits.  Up to
+ * the sizes of any one linear of the 8B shape at 2048 tokens and r = 16 the
+ * call takes the plan lsq_nf4_lora_bwd takes with a workspace of
+ * lsq_nf4_lora_bwd_workspace_size() bytes, bit for bit the same results;
+ * beyond that, where the array has no room left for the stream-K partials,
+ * the dX GEMM runs whole tiles and its fp32 sums may differ in the last bits.
+ * A size whose scratch exceeds the array is rejected with LSQ_EINVAL before
+ * anything is enqueued.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current, and the
+ * first call on a host thread creates the library's per-thread side stream
+ * and events and queries device attributes: make those first calls before
+ * any stream capture.  Every call shares the array and leaves its last
  * contents there; nothing in it needs to start at zero (each call writes all
- * the scratch it reads).  Calls that overlap on the GPU (other streams or
- * host threads) race on the array: the caller must serialise them. */
+ * the scratch it reads, and stream-K flags carry a per-launch value).  Calls
+ * that overlap on the GPU (other streams or host threads) race on the array:
+ * the caller must serialise them. */
 size_t lsq_nf4_lora_bwd_noalloc_max_scratch(void);
 lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M,
                                     const void* A, const void* B, int32_t r, float s, const float* u, void* dx,
@@ -281,6 +323,21 @@ lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const void* x, cons
  *  out_f32 = 1: fp32 output, else bf16.  K % 8 == 0, N % 8 == 0. */
 lsq_status lsq_dense_gemm(const void* a, const void* b, void* out, int64_t M, int64_t N, int64_t K,
                           int32_t trans_b, int32_t out_f32, lsq_cuda_stream stream);
+/* The same GEMM on column blocks of wider row-major tensors, with a split
+ * contraction: the lm_head streamed in vocabulary chunks (the pages plan the
+ * untied embed_tokens and lm_head as streamed large layers, soup-cli diff,
+ * docs "Layer Streaming", "NF4 streaming").
+ *  a: rows of lda elements (lda >= K); out (and acc_in): rows of ldo elements
+ *  (ldo >= N); lda, ldo multiples of 8.
+ *  acc_in: NULL, or the fp32 accumulator [M, N] (row stride ldo, may alias an
+ *  fp32 out) that earlier calls over the preceding K range left: the call
+ *  continues the contraction from it.  With K ranges cut at multiples of 64 a
+ *  chain of calls gives bit for bit what one call over the whole K gives
+ *  (the accumulator enters the tensor memory exactly as it left it).
+ * Other rules as lsq_dense_gemm; EINVAL before anything is enqueued. */
+lsq_status lsq_dense_gemm_ex(const void* a, int64_t lda, const void* b, void* out, int64_t ldo, const float* acc_in,
+                             int64_t M, int64_t N, int64_t K, int32_t trans_b, int32_t out_f32,
+                             lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
  * Decoder-layer kernels around the linears (Llama / Qwen, "Llama / Qwen
@@ -323,6 +380,17 @@ lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const 
                              const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,
                              int64_t hkv, int64_t hd, void* workspace, size_t workspace_bytes,
                              lsq_cuda_stream stream);
+/* lsq_attention_bwd for q and k that the forward rotated with RoPE (the
+ * q / k projections of lsq_nf4_lora_fwd_multi_ex2): with rope_table (from
+ * lsq_rope_table for this seq and hd; NULL = plain lsq_attention_bwd), dq and
+ * dk come out as the gradients of the unrotated q and k - the transpose of the
+ * rotation applied to the fp32 gradient before its one bf16 rounding (head
+ * dim 128 up to 512 positions; other shapes rotate the bf16 gradients in a
+ * pass after the backward kernels).  rope_table 16-byte aligned. */
+lsq_status lsq_attention_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,
+                                int64_t hkv, int64_t hd, const float* rope_table, void* workspace,
+                                size_t workspace_bytes, lsq_cuda_stream stream);
 /* m = silu(g) * u over n elements. */
 lsq_status lsq_swiglu_fwd(const void* g, const void* u, void* m, int64_t n, lsq_cuda_stream stream);
 /* dg, du from dm (dg/du may alias g/u: in-place). */
@@ -378,6 +446,13 @@ lsq_status lsq_seq_logprob_bwd(const float* logits, const int32_t* ids, int64_t 
 lsq_status lsq_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int32_t step,
                           float lr, float beta1, float beta2, float eps, float weight_decay,
                           lsq_cuda_stream stream);
+/* The bf16 operand copies p_bf16 of n fp32 masters p (device pointers), each
+ * rounded to nearest even: the operand refresh that closes lsq_adamw_step,
+ * alone, for the operands' first fill before any step.  fp32 masters with
+ * bf16 operand copies are this library's reading of the optimizer step (the
+ * pages name only PagedAdamW8bit, CHANGELOG [0.72.2] benchmark setup).
+ * n >= 1, else EINVAL. */
+lsq_status lsq_lora_refresh_bf16(const float* p, void* p_bf16, int64_t n, lsq_cuda_stream stream);
 
 /* ------------------------------------------------------------------------
  * Layer streaming scheduler.
@@ -486,6 +561,21 @@ lsq_status lsq_stream_stats(const lsq_stream* st, int64_t* uploads, int64_t* byt
 /* Device time (ms) of the last completed upload of `layer` (event pair on the
  * copy stream); synchronises on that upload. */
 lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float* ms);
+/* Exposed-copy timing (the measure of copy time that compute could not hide):
+ * with capacity > 0, each compute-stream wait on an upload that
+ * lsq_stream_step enqueues is bracketed by two timing events recorded on the
+ * compute stream, before and after the wait, so the time between them is how
+ * long compute stood still for that layer's copy (the pages judge streaming by
+ * how long compute waits on copies, README "Citing Soup", measured share of
+ * the step).  Up to `capacity` waits are kept between two lsq_stream_wait_ms
+ * calls; later ones are counted as dropped.  capacity 0 turns it off.  Waits
+ * for the compute stream before it replaces the events.  capacity 0..2^20. */
+lsq_status lsq_stream_time_waits(lsq_stream* st, int32_t capacity);
+/* The summed time (ms) of the kept waits since the previous call, split by
+ * the walking direction of the step that enqueued them (+1: fwd_ms, -1:
+ * bwd_ms), their number and the number dropped; waits for those events and
+ * starts a new count.  ESTATE when timing is off. */
+lsq_status lsq_stream_wait_ms(lsq_stream* st, float* fwd_ms, float* bwd_ms, int32_t* n_waits, int32_t* n_dropped);
 /* Forget all residency (next step re-uploads); waits for pending copies. */
 lsq_status lsq_stream_reset(lsq_stream* st);
 lsq_status lsq_stream_destroy(lsq_stream* st);

@@ -583,14 +583,21 @@ extern "C" size_t lsq_attention_bwd_workspace_size(int64_t batch, int64_t seq, i
   return (size_t)((batch * seq * hq > 0 ? batch * seq * hq : 1) * sizeof(float) + 255) / 256 * 256;
 }
 
-extern "C" lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                                        const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq,
-                                        int64_t hq, int64_t hkv, int64_t hd, void* workspace, size_t workspace_bytes,
-                                        lsq_cuda_stream stream) {
+namespace lsq {
+namespace ops {
+lsq_status rope_from_table(void* x, const float* table, int64_t batch, int64_t seq, int64_t heads, int64_t hd,
+                           int inverse, cudaStream_t stream);
+}
+}  // namespace lsq
+
+extern "C" lsq_status lsq_attention_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                           const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq,
+                                           int64_t hq, int64_t hkv, int64_t hd, const float* rope_table,
+                                           void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
   if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv || !workspace)
     return fail(LSQ_EINVAL, "lsq_attention_bwd: NULL argument");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(d_o, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || (rope_table && !aligned(rope_table, 16)))
     return fail(LSQ_EINVAL, "lsq_attention_bwd: alignment");
   lsq_status st = check_args("lsq_attention_bwd", batch, seq, hq, hkv, hd);
   if (st != LSQ_OK) return st;
@@ -602,9 +609,21 @@ extern "C" lsq_status lsq_attention_bwd(const void* q, const void* k, const void
   dvec_kernel<<<(unsigned)((rows * (hd / 8) + 255) / 256), 256, 0, cs>>>((const __nv_bfloat16*)o, (const __nv_bfloat16*)d_o,
                                                                   dvec, rows, (int)seq, (int)hq, (int)hd);
   LSQ_LAUNCH_CHECK("attention dvec_kernel");
+  // the tcgen05 kernels apply the RoPE transpose in their epilogues; the others leave it to a pass after them
   if (atc::bwd_supported(seq, hd))
-    return atc::run_bwd(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
-  if (hd == 64)
-    return run_bwd<64>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
-  return run_bwd<128>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
+    return atc::run_bwd(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs,
+                        rope_table);
+  st = hd == 64 ? run_bwd<64>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs)
+                : run_bwd<128>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
+  if (st != LSQ_OK || !rope_table) return st;
+  if ((st = ops::rope_from_table(dq, rope_table, batch, seq, hq, hd, 1, cs)) != LSQ_OK) return st;
+  return ops::rope_from_table(dk, rope_table, batch, seq, hkv, hd, 1, cs);
+}
+
+extern "C" lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                        const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq,
+                                        int64_t hq, int64_t hkv, int64_t hd, void* workspace, size_t workspace_bytes,
+                                        lsq_cuda_stream stream) {
+  return lsq_attention_bwd_ex(q, k, v, o, lse, d_o, dq, dk, dv, batch, seq, hq, hkv, hd, nullptr, workspace,
+                              workspace_bytes, stream);
 }

@@ -320,6 +320,32 @@ __device__ __forceinline__ void store_row_units(uint32_t row_base, int r, int pa
                  w[4 * u + 2], w[4 * u + 3]);
 }
 
+// dx1 = g1 c + g2 s, dx2 = g2 c - g1 s (the transpose of rotate-half RoPE) for 16
+// column pairs (i, i + 64) of a head, g = f * accumulator; cs: (cos, sin) of
+// frequencies i..i+15; writes columns i.. at dst and i + 64.. at dst + 64
+__device__ __forceinline__ void rope_t_store(__nv_bfloat16* dst, const float (&g1)[16], const float (&g2)[16],
+                                             const float2* __restrict__ cs, float f) {
+  float o1[16], o2[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(cs) + q);
+    const float a0 = g1[2 * q] * f, a1 = g1[2 * q + 1] * f, b0 = g2[2 * q] * f, b1 = g2[2 * q + 1] * f;
+    o1[2 * q] = a0 * t.x + b0 * t.y;
+    o2[2 * q] = b0 * t.x - a0 * t.y;
+    o1[2 * q + 1] = a1 * t.z + b1 * t.w;
+    o2[2 * q + 1] = b1 * t.z - a1 * t.w;
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    *reinterpret_cast<uint4*>(dst + 8 * u) =
+        make_uint4(pack_bf16x2(o1[8 * u], o1[8 * u + 1]), pack_bf16x2(o1[8 * u + 2], o1[8 * u + 3]),
+                   pack_bf16x2(o1[8 * u + 4], o1[8 * u + 5]), pack_bf16x2(o1[8 * u + 6], o1[8 * u + 7]));
+    *reinterpret_cast<uint4*>(dst + 64 + 8 * u) =
+        make_uint4(pack_bf16x2(o2[8 * u], o2[8 * u + 1]), pack_bf16x2(o2[8 * u + 2], o2[8 * u + 3]),
+                   pack_bf16x2(o2[8 * u + 4], o2[8 * u + 5]), pack_bf16x2(o2[8 * u + 6], o2[8 * u + 7]));
+  }
+}
+
 // ---------------------------------------------------------------- dQ
 // One CTA per (128-query tile, head, sequence); sub-items = 64-key slices of
 // the keys at or before the tile:  S = Q K_j^T, dP = dO V_j^T (TMEM), dS =
@@ -342,7 +368,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
                                                                     const float* __restrict__ lse,
                                                                     const float* __restrict__ dvec,
                                                                     __nv_bfloat16* __restrict__ dq, int S, int Hq,
-                                                                    int Hkv, float scale, float scale_log2) {
+                                                                    int Hkv, float scale, float scale_log2,
+                                                                    const float2* __restrict__ rope) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + Q_OFF_BAR);
@@ -504,7 +531,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
     if (ok && __all_sync(0xffffffffu, mbar_wait(done, 0, 773))) {
       tc_fence_after();
       __nv_bfloat16* row = dq + (((int64_t)b * S + qi) * Hq + h) * D;
-      {
+      if (rope) {
+        // the transpose of the forward's RoPE, on the fp32 gradient before its one rounding:
+        // this warp takes columns [16 part, 16 part + 16) and their partners 64 further on
+        float x1[16], x2[16];
+        tmem_ld16(tmem + lane_base + T_DQ + (uint32_t)(part * 16), x1);
+        tmem_ld16(tmem + lane_base + T_DQ + (uint32_t)(64 + part * 16), x2);
+        tc_wait_ld();
+        if (qi < S) rope_t_store(row + part * 16, x1, x2, rope + (int64_t)qi * (D / 2) + part * 16, scale);
+      } else {
         const int c4 = part;  // 32 of the 128 output columns per warp
         float v[32];
         tmem_ld32(tmem + lane_base + T_DQ + (uint32_t)(c4 * 32), v);
@@ -577,7 +612,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
                                                                      const float* __restrict__ dvec,
                                                                      __nv_bfloat16* __restrict__ dk,
                                                                      __nv_bfloat16* __restrict__ dv_out, int S, int Hq,
-                                                                     int Hkv, float scale, float scale_log2, int split) {
+                                                                     int Hkv, float scale, float scale_log2, int split,
+                                                                     const float2* __restrict__ rope) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + K_OFF_BAR);
@@ -778,7 +814,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
     } else if (ok && split == 1) {
       tc_fence_after();
       const int64_t off = (((int64_t)b * S + kj) * Hkv + hk) * D;
-      {
+      if (rope) {
+        // dK with the transpose of the forward's RoPE (columns 16 part.. and 64 further on), dV as it is
+        float x1[16], x2[16], c[32];
+        tmem_ld16(tmem + lane_base + T_DK + (uint32_t)(part * 16), x1);
+        tmem_ld16(tmem + lane_base + T_DK + (uint32_t)(64 + part * 16), x2);
+        tmem_ld32(tmem + lane_base + T_DV + (uint32_t)(part * 32), c);
+        tc_wait_ld();
+        if (kj < S) {
+          rope_t_store(dk + off + part * 16, x1, x2, rope + (int64_t)kj * (D / 2) + part * 16, scale);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(dv_out + off + part * 32 + u * 8) =
+                make_uint4(pack_bf16x2(c[8 * u], c[8 * u + 1]), pack_bf16x2(c[8 * u + 2], c[8 * u + 3]),
+                           pack_bf16x2(c[8 * u + 4], c[8 * u + 5]), pack_bf16x2(c[8 * u + 6], c[8 * u + 7]));
+        }
+      } else {
         const int c4 = part;  // 32 of the 128 output columns per warp
         float a[32], c[32];
         tmem_ld32(tmem + lane_base + T_DK + (uint32_t)(c4 * 32), a);
@@ -809,17 +860,38 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
     for (int e = (int)threadIdx.x; e < (BC / 2) * 2 * (D / 4); e += blockDim.x) {
       const int t = e / ((BC / 2) * (D / 4));              // 0: dK, 1: dV
       const int rr = (e / (D / 4)) % (BC / 2) + half * (BC / 2), c4 = e % (D / 4);
-      const float* loc = pk0 + (size_t)t * BC * PSTRIDE + (size_t)rr * PSTRIDE + c4 * 4;
-      const float4 mine = *reinterpret_cast<const float4*>(loc);
-      const float4 peer = ld_dsmem4(dsmem_addr(loc, (uint32_t)(half ^ 1)));
-      const float4 lo = half == 0 ? mine : peer, hi = half == 0 ? peer : mine;
-      const float f = t == 0 ? scale : 1.0f;
-      const float x0 = (lo.x + hi.x) * f, x1 = (lo.y + hi.y) * f, x2 = (lo.z + hi.z) * f, x3 = (lo.w + hi.w) * f;
+      if (rope && t == 0 && c4 >= D / 8) continue;         // with RoPE each dK unit below D/2 takes its partner
       const int kr = k0 + rr;
-      if (kr < S) {
-        __nv_bfloat16* dst = (t == 0 ? dk : dv_out) + (((int64_t)b * S + kr) * Hkv + hk) * D + c4 * 4;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(x0, x1), pack_bf16x2(x2, x3));
+      auto sum4 = [&](int col) {                           // both CTAs' partials of 4 columns, rank 0's first
+        const float* loc = pk0 + (size_t)t * BC * PSTRIDE + (size_t)rr * PSTRIDE + col;
+        const float4 mine = *reinterpret_cast<const float4*>(loc);
+        const float4 peer = ld_dsmem4(dsmem_addr(loc, (uint32_t)(half ^ 1)));
+        const float4 lo = half == 0 ? mine : peer, hi = half == 0 ? peer : mine;
+        return make_float4(lo.x + hi.x, lo.y + hi.y, lo.z + hi.z, lo.w + hi.w);
+      };
+      const float4 a = sum4(c4 * 4);
+      __nv_bfloat16* dst = (t == 0 ? dk : dv_out) + (((int64_t)b * S + kr) * Hkv + hk) * D + c4 * 4;
+      if (rope && t == 0) {
+        const float4 g = sum4(c4 * 4 + D / 2);
+        const float a_[4] = {a.x * scale, a.y * scale, a.z * scale, a.w * scale};
+        const float g_[4] = {g.x * scale, g.y * scale, g.z * scale, g.w * scale};
+        float o1[4], o2[4];
+        const float2* cs = rope + (int64_t)kr * (D / 2) + c4 * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 tq = kr < S ? __ldg(cs + j) : make_float2(1.0f, 0.0f);
+          o1[j] = a_[j] * tq.x + g_[j] * tq.y;
+          o2[j] = g_[j] * tq.x - a_[j] * tq.y;
+        }
+        if (kr < S) {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o1[0], o1[1]), pack_bf16x2(o1[2], o1[3]));
+          *reinterpret_cast<uint2*>(dst + D / 2) = make_uint2(pack_bf16x2(o2[0], o2[1]), pack_bf16x2(o2[2], o2[3]));
+        }
+        continue;
       }
+      const float f = t == 0 ? scale : 1.0f;
+      if (kr < S)
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a.x * f, a.y * f), pack_bf16x2(a.z * f, a.w * f));
     }
     cluster_barrier();  // the peer has read this CTA's partials
   }
@@ -862,7 +934,9 @@ lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* 
 bool bwd_supported(int64_t S, int64_t hd) { return fwd_supported(S, hd); }
 
 lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o, const float* lse, const float* dvec,
-                   void* dq, void* dk, void* dv, int B, int S, int Hq, int Hkv, cudaStream_t st) {
+                   void* dq, void* dk, void* dv, int B, int S, int Hq, int Hkv, cudaStream_t st,
+                   const float* rope_table) {
+  const float2* rope = reinterpret_cast<const float2*>(rope_table);
   static int cfg[64];
   int dev = 0;
   LSQ_CUDA_TRY(cudaGetDevice(&dev));
@@ -886,7 +960,7 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
   const int nt = (S + BQ - 1) / BQ;
   attn_dq_tc_kernel<<<dim3(Hq, B, nt), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, lse, dvec,
                                                                   static_cast<__nv_bfloat16*>(dq), S, Hq, Hkv, scale,
-                                                                  sl);
+                                                                  sl, rope);
   LSQ_LAUNCH_CHECK("attn_dq_tc_kernel");
   const int split = Hq / Hkv >= 2 ? 2 : 1;
   cudaLaunchConfig_t lc = {};
@@ -903,7 +977,7 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
   lc.numAttrs = 1;
   LSQ_CUDA_TRY(cudaLaunchKernelEx(&lc, attn_dkv_tc_kernel, qm64, km, vm, dom64, lse, dvec,
                                   static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv, scale,
-                                  sl, split));
+                                  sl, split, rope));
   return LSQ_OK;
 }
 

@@ -215,6 +215,7 @@ struct Seg {
   const __nv_bfloat16* res;  // FWD residual [M, n] or null (may alias y)
   int n;                     // rows of W
   int first;                 // FWD: first n-tile of the segment; DX: first contraction block
+  int rope;                  // FWD: rotate this segment's output (heads of rope_hd columns)
 };
 
 struct Params {
@@ -225,6 +226,10 @@ struct Params {
   int mtiles, tiles;
   __nv_bfloat16* dx;  // DX output [M, K]
   float cb[16];
+  // FWD: rotate-half RoPE of the segments marked rope, position = row % rope_seq,
+  // cos / sin from the table [rope_seq][rope_hd / 2] (rope_hd 64, 128 or 256)
+  const float2* rope;
+  int rope_seq, rope_hd;
   // stream-K: the first dp_tiles tiles (whole rounds) go to the clusters
   // whole, in the usual order; the weight blocks of the others are cut into
   // one contiguous range per cluster, and a range that ends inside a tile
@@ -603,7 +608,89 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
+      // 16 columns (piece 0 or 1 of chunk hcc) of this tile's accumulator plus the partials of
+      // the clusters before this one, added in the same order as the 32-column path below
+      auto acc16 = [&](int hcc, int piece, float (&v)[16]) {
+        const int hh = hcc / (BT / 32), cc = hcc % (BT / 32);
+        tmem_ld16(tmem + lane_base + (uint32_t)((buf * H + hh) * BT + cc * 32 + piece * 16), v);
+        if (cfirst == cid) {
+          tc_wait_ld();
+          return;
+        }
+        const float4* src0 = reinterpret_cast<const float4*>(p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS) +
+                             ((int64_t)hcc * 8 + piece * 4) * 128 + e;
+        float4 a[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[q] = __ldcg(src0 + q * 128);
+        tc_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          v[4 * q] += a[q].x;
+          v[4 * q + 1] += a[q].y;
+          v[4 * q + 2] += a[q].z;
+          v[4 * q + 3] += a[q].w;
+        }
+        for (int c2 = cfirst + 1; c2 < cid; ++c2) {
+          if (sk_bound(p, c2 + 1, ncl) == sk_bound(p, c2, ncl)) continue;
+          const float4* src = reinterpret_cast<const float4*>(p.part + (int64_t)(c2 * 2 + (int)rank) * PART_FLOATS) +
+                              ((int64_t)hcc * 8 + piece * 4) * 128 + e;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) a[q] = __ldcg(src + q * 128);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            v[4 * q] += a[q].x;
+            v[4 * q + 1] += a[q].y;
+            v[4 * q + 2] += a[q].z;
+            v[4 * q + 3] += a[q].w;
+          }
+        }
+      };
       const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
+      if (MODE == FWD && p.seg[sg].rope) {
+        // RoPE in the epilogue: column i of a head pairs with column i + hd/2, which sits hd/64
+        // chunks of 32 further on in the same accumulator; each pair of chunks is rotated in
+        // fp32 (the accumulator plus earlier clusters' partials, as below) and rounded once
+        const int hc32 = p.rope_hd / 32, half = p.rope_hd / 2;
+        for (int hc = 0; hc < H * (BT / 32); ++hc) {
+          const int h = hc / (BT / 32), c = hc % (BT / 32);
+          if (c % hc32 >= hc32 / 2 || n0 + c * 32 >= ncols) continue;
+          const int m = m0 + h * BT + (int)rank * BMC + e;
+#pragma unroll 1
+          for (int piece = 0; piece < 2; ++piece) {
+            float x1[16], x2[16];
+            acc16(hc, piece, x1);
+            acc16(hc + hc32 / 2, piece, x2);
+            if (m >= p.M) continue;
+            const int i0 = (c % hc32) * 32 + piece * 16;  // frequency index of x1[0]
+            const float4* cs = reinterpret_cast<const float4*>(p.rope + (int64_t)(m % p.rope_seq) * half + i0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 t = __ldg(cs + q);  // (cos, sin) of frequencies i0 + 2q, i0 + 2q + 1
+              const float a0 = x1[2 * q], a1 = x1[2 * q + 1], b0 = x2[2 * q], b1 = x2[2 * q + 1];
+              x1[2 * q] = a0 * t.x - b0 * t.y;
+              x2[2 * q] = b0 * t.x + a0 * t.y;
+              x1[2 * q + 1] = a1 * t.z - b1 * t.w;
+              x2[2 * q + 1] = b1 * t.z + a1 * t.w;
+            }
+            const Seg& S = p.seg[sg];
+            __nv_bfloat16* y1 = S.y + (int64_t)m * S.n + n0 + c * 32 + piece * 16;
+            __nv_bfloat16* y2 = y1 + half;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              *reinterpret_cast<uint4*>(y1 + 8 * u) =
+                  make_uint4(pack_bf16x2(x1[8 * u], x1[8 * u + 1]), pack_bf16x2(x1[8 * u + 2], x1[8 * u + 3]),
+                             pack_bf16x2(x1[8 * u + 4], x1[8 * u + 5]), pack_bf16x2(x1[8 * u + 6], x1[8 * u + 7]));
+              *reinterpret_cast<uint4*>(y2 + 8 * u) =
+                  make_uint4(pack_bf16x2(x2[8 * u], x2[8 * u + 1]), pack_bf16x2(x2[8 * u + 2], x2[8 * u + 3]),
+                             pack_bf16x2(x2[8 * u + 4], x2[8 * u + 5]), pack_bf16x2(x2[8 * u + 6], x2[8 * u + 7]));
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+        continue;
+      }
       for (int hc = 0; hc < H * (BT / 32); ++hc) {
         const int h = hc / (BT / 32), c = hc % (BT / 32);
         if (n0 + c * 32 >= ncols) continue;
@@ -1058,8 +1145,13 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
   const double rounds_sk = (double)tiles2 / ncl_max + 0.4;
   const double rounds_whole = (double)((tiles2 + ncl_max - 1) / ncl_max);
   const int64_t dp = std::max<int64_t>(0, tiles2 / ncl_max - 1) * ncl_max;
-  if (!force && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 && 2 * tiles2 >= ncl_max &&
-      (tiles2 - dp) * p.nkb >= 4 * (int64_t)ncl_max && rounds_sk < 0.97 * rounds_whole) {
+  // LSQ_NF4_STREAMK=0 never shares tiles out, =1 does wherever it can (a tuning override)
+  const char* skenv = getenv("LSQ_NF4_STREAMK");
+  const int skmode = skenv ? atoi(skenv) : -1;
+  const bool sk_can = !force && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 &&
+                      (tiles2 - dp) * p.nkb >= 4 * (int64_t)ncl_max;
+  const bool sk_pays = 2 * tiles2 >= ncl_max && rounds_sk < 0.97 * rounds_whole;
+  if (sk_can && skmode != 0 && (skmode == 1 || sk_pays)) {
     p.streamk = 1;
     p.dp_tiles = (int)dp;  // whole tiles for all but the last one or two rounds' worth
     p.flags = reinterpret_cast<unsigned long long*>(sk_ws);
@@ -1424,7 +1516,7 @@ static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
                            const void* const* B, int32_t r, float s, const void* const* residual, void* const* y,
                            float* const* u_out, __nv_bfloat16* const* su, __nv_bfloat16* const* bpad,
                            bool rank_part, __nv_bfloat16* const* bt, __nv_bfloat16* at, char* sk_ws,
-                           size_t sk_bytes, cudaStream_t cs) {
+                           size_t sk_bytes, cudaStream_t cs, const lsq_rope_spec* rope = nullptr) {
   const int64_t K = W[0].k_in;
   const int rp = rpad(r);
   int64_t ns[3];
@@ -1438,6 +1530,11 @@ static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
   p.lora = r > 0 ? 1 : 0;
   p.nkb = (int)(K / BK);
   fill_cb(p);
+  if (rope) {
+    p.rope = reinterpret_cast<const float2*>(rope->table);
+    p.rope_seq = rope->seq;
+    p.rope_hd = rope->hd;
+  }
   Maps maps;
   memset(&maps, 0, sizeof(maps));
   if ((st = tmap_act(&maps.a[0], x, K, M, BMC)) != LSQ_OK) return st;
@@ -1449,6 +1546,7 @@ static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
     g.res = static_cast<const __nv_bfloat16*>(residual ? residual[i] : nullptr);
     g.n = (int)W[i].n_out;
     g.first = tiles_n;
+    g.rope = (rope && (rope->segments >> i) & 1) ? 1 : 0;
     tiles_n += (int)((W[i].n_out + BT - 1) / BT);
     if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
                              BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
@@ -1514,12 +1612,30 @@ static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
 }  // namespace tc
 }  // namespace lsq
 
+namespace lsq {
+namespace tc {
+// the workspace form of the fused forward (the rank-r operands rebuilt in the workspace), with optional RoPE
+static lsq_status fwd_multi_ws(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M, const void* const* A,
+                               const void* const* B, int32_t r, float s, const void* const* residual, void* const* y,
+                               float* const* u_out, void* workspace, size_t workspace_bytes, lsq_cuda_stream stream,
+                               const lsq_rope_spec* rope, const char* who);
+}  // namespace tc
+}  // namespace lsq
+
 extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
                                              const void* const* A, const void* const* B, int32_t r, float s,
                                              const void* const* residual, void* const* y, float* const* u_out,
                                              void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
+  return lsq::tc::fwd_multi_ws(nseg, W, x, M, A, B, r, s, residual, y, u_out, workspace, workspace_bytes, stream,
+                               nullptr, "lsq_nf4_lora_fwd");
+}
+
+static lsq_status lsq::tc::fwd_multi_ws(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                        const void* const* A, const void* const* B, int32_t r, float s,
+                                        const void* const* residual, void* const* y, float* const* u_out,
+                                        void* workspace, size_t workspace_bytes, lsq_cuda_stream stream,
+                                        const lsq_rope_spec* rope, const char* who) {
   using namespace lsq;
-  const char* who = "lsq_nf4_lora_fwd";
   int64_t ns[3];
   lsq_status st = tc::fwd_checks(nseg, W, x, M, A, B, r, residual, y, ns, who);
   if (st != LSQ_OK) return st;
@@ -1547,7 +1663,7 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi(int32_t nseg, const lsq_nf4_weight*
     sk_bytes = workspace_bytes - base;
   }
   return tc::fwd_impl(nseg, W, x, M, A, B, r, s, residual, y, u_out, su, bpad, true, nullptr, nullptr, sk_ws,
-                      sk_bytes, (cudaStream_t)stream);
+                      sk_bytes, (cudaStream_t)stream, rope);
 }
 
 extern "C" size_t lsq_nf4_lora_state_size(int32_t nseg, int64_t M, int64_t k_in, const int64_t* n_out, int32_t r) {
@@ -1574,6 +1690,42 @@ extern "C" lsq_status lsq_nf4_lora_fwd_multi_ex(int32_t nseg, const lsq_nf4_weig
   if (r > 0) q = tc::state_ptrs(state, nseg, tc::state_plan(nseg, M, K, ns, r));
   return tc::fwd_impl(nseg, W, x, M, A, B, r, s, residual, y, u_out, q.su, q.bpad, !state_ready, q.bt, q.at,
                       static_cast<char*>(workspace), workspace ? workspace_bytes : 0, (cudaStream_t)stream);
+}
+
+extern "C" lsq_status lsq_nf4_lora_fwd_multi_ex2(int32_t nseg, const lsq_nf4_weight* W, const void* x, int64_t M,
+                                                 const void* const* A, const void* const* B, int32_t r, float s,
+                                                 const void* const* residual, void* const* y, float* const* u_out,
+                                                 void* state, int32_t state_ready, const lsq_rope_spec* rope,
+                                                 void* workspace, size_t workspace_bytes, lsq_cuda_stream stream) {
+  using namespace lsq;
+  const char* who = "lsq_nf4_lora_fwd_ex2";
+  if (rope && rope->segments) {
+    if (!rope->table || !aligned(rope->table, 16) || (rope->hd != 64 && rope->hd != 128 && rope->hd != 256) ||
+        rope->seq < 1 || M % rope->seq != 0 || (rope->segments >> nseg) != 0)
+      return fail(LSQ_EINVAL, "%s: RoPE needs a 16-byte aligned table, hd 64, 128 or 256, M a multiple of seq "
+                  "and segment bits below nseg", who);
+    for (int i = 0; i < nseg; ++i)
+      if (((rope->segments >> i) & 1) && (!W || W[i].n_out % rope->hd != 0 || (residual && residual[i])))
+        return fail(LSQ_EINVAL, "%s: a rotated segment needs n_out a multiple of hd and no residual", who);
+  }
+  if (!state)  // no rank state: the operands are rebuilt in the workspace, as lsq_nf4_lora_fwd_multi does
+    return tc::fwd_multi_ws(nseg, W, x, M, A, B, r, s, residual, y, u_out, workspace, workspace_bytes, stream,
+                            rope && rope->segments ? rope : nullptr, who);
+  if (!rope || !rope->segments)
+    return lsq_nf4_lora_fwd_multi_ex(nseg, W, x, M, A, B, r, s, residual, y, u_out, state, state_ready, workspace,
+                                     workspace_bytes, stream);
+  int64_t ns[3];
+  lsq_status st = tc::fwd_checks(nseg, W, x, M, A, B, r, residual, y, ns, who);
+  if (st != LSQ_OK) return st;
+  const int64_t K = W[0].k_in;
+  if (r > 0 && (!state || !aligned(state, 256)))
+    return fail(LSQ_EINVAL, "%s: a 256-byte aligned rank state is needed with r > 0", who);
+  if (workspace && !aligned(workspace, 256)) return fail(LSQ_EINVAL, "%s: workspace must be 256-byte aligned", who);
+  tc::StatePtrs q;
+  memset(&q, 0, sizeof(q));
+  if (r > 0) q = tc::state_ptrs(state, nseg, tc::state_plan(nseg, M, K, ns, r));
+  return tc::fwd_impl(nseg, W, x, M, A, B, r, s, residual, y, u_out, q.su, q.bpad, !state_ready, q.bt, q.at,
+                      static_cast<char*>(workspace), workspace ? workspace_bytes : 0, (cudaStream_t)stream, rope);
 }
 
 extern "C" lsq_status lsq_nf4_lora_fwd(const lsq_nf4_weight* W, const void* x, int64_t M, const void* A,

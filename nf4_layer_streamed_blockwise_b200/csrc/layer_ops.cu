@@ -147,6 +147,48 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
   }
 }
 
+// (cos, sin) of pos * theta^(-2i/hd) for every position and frequency, with
+// rope_kernel's double-precision angle and rounding to fp32
+__global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ table, int64_t n, int half, int hd,
+                                                         double log_theta) {
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int pos = (int)(idx / half), i = (int)(idx % half);
+    const double inv = exp(-2.0 * i / hd * log_theta);
+    double sn, c;
+    sincos((double)pos * inv, &sn, &c);
+    table[idx] = make_float2((float)c, (float)sn);
+  }
+}
+
+// rope_kernel's rotation with the angles from a table (inverse: the transpose),
+// for heads of hd % 16 == 0 on 16-byte aligned rows; one CTA per (batch, position)
+__global__ void __launch_bounds__(128) rope_from_table_kernel(__nv_bfloat16* __restrict__ x,
+                                                              const float2* __restrict__ table, int seq, int heads,
+                                                              int hd, int inverse) {
+  const int half = hd / 2;
+  const int64_t bs = blockIdx.x;
+  const float2* cs = table + (int64_t)(bs % seq) * half;
+  __nv_bfloat16* base = x + bs * (int64_t)heads * hd;
+  const int nv = half / 8;
+  for (int idx = threadIdx.x; idx < heads * nv; idx += blockDim.x) {
+    const int h = idx / nv, i0 = (idx % nv) * 8;
+    uint4* p1 = reinterpret_cast<uint4*>(base + (int64_t)h * hd + i0);
+    uint4* p2 = reinterpret_cast<uint4*>(base + (int64_t)h * hd + half + i0);
+    float a[8], b[8], o1[8], o2[8];
+    unpack8(*p1, a);
+    unpack8(*p2, b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 t = cs[i0 + k];
+      const float c = t.x, sn = inverse ? -t.y : t.y;
+      o1[k] = a[k] * c - b[k] * sn;
+      o2[k] = b[k] * c + a[k] * sn;
+    }
+    *p1 = pack8(o1);
+    *p2 = pack8(o2);
+  }
+}
+
 // ---------------------------------------------------------------- SwiGLU
 __device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf(-g)); }
 
@@ -387,6 +429,14 @@ __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const
   }
 }
 
+// the bf16 operand copies of fp32 masters, refreshed without an optimizer step
+// (the rounding adamw_kernel applies after each update)
+__global__ void __launch_bounds__(256) refresh_bf16_kernel(const float* __restrict__ p, __nv_bfloat16* __restrict__ pb,
+                                                           int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    pb[i] = __float2bfloat16_rn(p[i]);
+}
+
 static unsigned grid_for(int64_t n, int threads) {
   int64_t g = (n + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms() * 32;
@@ -444,6 +494,34 @@ extern "C" lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t head
   LSQ_LAUNCH_CHECK("rope_kernel");
   return LSQ_OK;
 }
+
+extern "C" lsq_status lsq_rope_table(float theta, int64_t seq, int64_t hd, float* table, lsq_cuda_stream stream) {
+  if (!table) return fail(LSQ_EINVAL, "lsq_rope_table: NULL argument");
+  if (seq < 1 || seq > (1 << 24) || hd < 2 || hd % 2 != 0 || hd > 1024 || !(theta > 1.0f))
+    return fail(LSQ_EINVAL, "lsq_rope_table: bad shape or theta");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  const int64_t n = seq * (hd / 2);
+  rope_table_kernel<<<grid_for(n, 256), 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<float2*>(table), n,
+                                                                         (int)(hd / 2), (int)hd, log((double)theta));
+  LSQ_LAUNCH_CHECK("rope_table_kernel");
+  return LSQ_OK;
+}
+
+namespace lsq {
+namespace ops {
+// the rotation (or its transpose) of x [batch, seq, heads, hd] with a table from lsq_rope_table
+lsq_status rope_from_table(void* x, const float* table, int64_t batch, int64_t seq, int64_t heads, int64_t hd,
+                           int inverse, cudaStream_t stream) {
+  if (hd % 16 != 0 || !aligned(x, 16) || !aligned(table, 8))
+    return fail(LSQ_EINVAL, "rope from a table: hd a multiple of 16 and 16-byte aligned rows");
+  rope_from_table_kernel<<<(unsigned)(batch * seq), 128, 0, stream>>>(
+      static_cast<__nv_bfloat16*>(x), reinterpret_cast<const float2*>(table), (int)seq, (int)heads, (int)hd, inverse);
+  LSQ_LAUNCH_CHECK("rope_from_table_kernel");
+  return LSQ_OK;
+}
+}  // namespace ops
+}  // namespace lsq
 
 extern "C" lsq_status lsq_swiglu_fwd(const void* g, const void* u, void* m, int64_t n, lsq_cuda_stream stream) {
   if (!g || !u || !m) return fail(LSQ_EINVAL, "lsq_swiglu_fwd: NULL argument");
@@ -550,6 +628,16 @@ extern "C" lsq_status lsq_seq_logprob_bwd(const float* logits, const int32_t* id
   seqlp_bwd_kernel<<<(unsigned)(batch * seq), XE_T, 0, (cudaStream_t)stream>>>(
       logits, ids, (int)seq, V, row_lse, dseq, static_cast<__nv_bfloat16*>(dlogits));
   LSQ_LAUNCH_CHECK("seqlp_bwd_kernel");
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_lora_refresh_bf16(const float* p, void* p_bf16, int64_t n, lsq_cuda_stream stream) {
+  if (!p || !p_bf16) return fail(LSQ_EINVAL, "lsq_lora_refresh_bf16: NULL argument");
+  if (n < 1) return fail(LSQ_EINVAL, "lsq_lora_refresh_bf16: need n >= 1");
+  lsq_status st = check_device();
+  if (st != LSQ_OK) return st;
+  refresh_bf16_kernel<<<grid_for(n, 256), 256, 0, (cudaStream_t)stream>>>(p, static_cast<__nv_bfloat16*>(p_bf16), n);
+  LSQ_LAUNCH_CHECK("refresh_bf16_kernel");
   return LSQ_OK;
 }
 

@@ -278,6 +278,11 @@ struct lsq_stream {
   uint64_t ex_codes[8], ex_params[8], ex_out[8];
   int64_t ex_nb[8];
   int64_t expands = 0;
+  // exposed-copy timing: a pair of timing events around each compute-stream wait on an upload
+  int direction = 0;                 // walking direction of the lsq_stream_step being executed
+  std::vector<cudaEvent_t> wev;      // 2 per kept wait
+  std::vector<int> wdir;             // direction of each kept wait
+  int n_wait = 0, n_wait_dropped = 0;
 };
 
 namespace lsq {
@@ -316,7 +321,16 @@ static lsq_status execute(lsq_stream* st) {
       LSQ_CUDA_TRY(cudaEventRecord(st->up_done[a.layer], st->copy));
       st->bytes += (int64_t)st->shard_bytes;
     } else if (a.kind == WAIT) {
+      const bool timed = !st->wev.empty();
+      const bool kept = timed && 2 * (size_t)st->n_wait < st->wev.size();
+      if (kept) LSQ_CUDA_TRY(cudaEventRecord(st->wev[2 * st->n_wait], st->compute));
       LSQ_CUDA_TRY(cudaStreamWaitEvent(st->compute, st->up_done[a.layer], 0));
+      if (kept) {
+        LSQ_CUDA_TRY(cudaEventRecord(st->wev[2 * st->n_wait + 1], st->compute));
+        st->wdir[st->n_wait++] = st->direction;
+      } else if (timed) {
+        st->n_wait_dropped += 1;
+      }
     }
   }
   st->acts.clear();
@@ -340,7 +354,16 @@ static lsq_status disk_status(lsq_stream* st) {
   return fail(st->reader->error, "%s", st->reader->errmsg.c_str());
 }
 
+static void destroy_wait_events(lsq_stream* st) {
+  for (cudaEvent_t e : st->wev)
+    if (e) cudaEventDestroy(e);
+  st->wev.clear();
+  st->wdir.clear();
+  st->n_wait = st->n_wait_dropped = 0;
+}
+
 static void destroy_events(lsq_stream* st) {
+  destroy_wait_events(st);
   for (auto* v : {&st->up_start, &st->up_done, &st->slot_free})
     for (cudaEvent_t e : *v)
       if (e) cudaEventDestroy(e);
@@ -512,6 +535,7 @@ extern "C" lsq_status lsq_stream_step(lsq_stream* st, int32_t layer, int32_t dir
   lsq_status ds = disk_status(st);
   if (ds != LSQ_OK) return ds;
   st->pol.step(layer, direction, st->acts);
+  st->direction = direction;
   lsq_status s = execute(st);
   if (s != LSQ_OK) return s;
   *slot_ptr = st->slots[st->pol.layer_slot[layer]];
@@ -556,6 +580,44 @@ extern "C" lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float*
   if (layer < 0 || layer >= st->pol.n_layers) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: layer out of range");
   LSQ_CUDA_TRY(cudaEventSynchronize(st->up_done[layer]));
   LSQ_CUDA_TRY(cudaEventElapsedTime(ms, st->up_start[layer], st->up_done[layer]));
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_time_waits(lsq_stream* st, int32_t capacity) {
+  if (!st) return fail(LSQ_EINVAL, "lsq_stream_time_waits: NULL scheduler");
+  if (capacity < 0 || capacity > (1 << 20)) return fail(LSQ_EINVAL, "lsq_stream_time_waits: capacity %d", capacity);
+  LSQ_CUDA_TRY(cudaStreamSynchronize(st->compute));  // no kept wait is still pending on the old events
+  destroy_wait_events(st);
+  if (capacity == 0) return LSQ_OK;
+  st->wev.assign(2 * (size_t)capacity, nullptr);
+  st->wdir.assign(capacity, 0);
+  for (size_t i = 0; i < st->wev.size(); ++i) {
+    cudaError_t e = cudaEventCreate(&st->wev[i]);
+    if (e != cudaSuccess) {
+      st->wev[i] = nullptr;
+      destroy_wait_events(st);
+      return cuda_fail(e, "lsq_stream_time_waits: event create");
+    }
+  }
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_wait_ms(lsq_stream* st, float* fwd_ms, float* bwd_ms, int32_t* n_waits,
+                                         int32_t* n_dropped) {
+  if (!st || !fwd_ms || !bwd_ms || !n_waits || !n_dropped) return fail(LSQ_EINVAL, "lsq_stream_wait_ms: NULL argument");
+  if (st->wev.empty()) return fail(LSQ_ESTATE, "lsq_stream_wait_ms: wait timing is off (lsq_stream_time_waits)");
+  double f = 0.0, b = 0.0;
+  for (int i = 0; i < st->n_wait; ++i) {
+    float ms = 0.0f;
+    LSQ_CUDA_TRY(cudaEventSynchronize(st->wev[2 * i + 1]));
+    LSQ_CUDA_TRY(cudaEventElapsedTime(&ms, st->wev[2 * i], st->wev[2 * i + 1]));
+    (st->wdir[i] > 0 ? f : b) += ms;
+  }
+  *fwd_ms = (float)f;
+  *bwd_ms = (float)b;
+  *n_waits = st->n_wait;
+  *n_dropped = st->n_wait_dropped;
+  st->n_wait = st->n_wait_dropped = 0;
   return LSQ_OK;
 }
 

@@ -37,6 +37,10 @@ class lsq_nf4_weight(ctypes.Structure):
     _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
 
 
+class lsq_rope_spec(ctypes.Structure):
+    _fields_ = [("table", c_void_p), ("seq", c_int32), ("hd", c_int32), ("segments", c_int32)]
+
+
 class lsq_absmax_dq_item(ctypes.Structure):
     _fields_ = [("codes_off", ctypes.c_uint64), ("params_off", ctypes.c_uint64), ("out_off", ctypes.c_uint64),
                 ("nb", c_int64)]
@@ -76,6 +80,14 @@ _SIGS = {
     "lsq_nf4_lora_fwd_multi_ex": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
                                             c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
+    "lsq_nf4_lora_fwd_multi_ex2": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_int64,
+                                             c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
+                                             c_void_p, c_int32, ctypes.POINTER(lsq_rope_spec), c_void_p, c_size_t,
+                                             c_void_p]),
+    "lsq_rope_table": (c_int32, [c_float, c_int64, c_int64, c_void_p, c_void_p]),
+    "lsq_attention_bwd_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int64, c_void_p,
+                                       c_void_p, c_size_t, c_void_p]),
     "lsq_nf4_lora_bwd_multi_ex": (c_int32, [c_int32, ctypes.POINTER(lsq_nf4_weight), c_void_p, c_void_p, c_int64,
                                             c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
@@ -98,6 +110,8 @@ _SIGS = {
                                            c_int32, c_void_p]),
     "lsq_dense_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32,
                                  c_void_p]),
+    "lsq_dense_gemm_ex": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_int64, c_void_p, c_int64, c_int64,
+                                    c_int64, c_int32, c_int32, c_void_p]),
     "lsq_rmsnorm_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_float, c_void_p]),
     "lsq_rmsnorm_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                   c_void_p]),
@@ -120,6 +134,7 @@ _SIGS = {
     "lsq_dpo_loss": (c_int32, [c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p]),
     "lsq_seq_logprob_bwd": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                       c_void_p]),
+    "lsq_lora_refresh_bf16": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
     "lsq_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_float,
                                  c_float, c_float, c_float, c_float, c_void_p]),
     "lsq_stream_create": (c_int32, [ctypes.POINTER(lsq_stream_cfg), c_void_p, c_void_p, ctypes.POINTER(c_void_p)]),
@@ -131,6 +146,9 @@ _SIGS = {
     "lsq_stream_stats": (c_int32, [c_void_p, ctypes.POINTER(c_int64), ctypes.POINTER(c_int64),
                                    ctypes.POINTER(c_int64)]),
     "lsq_stream_upload_ms": (c_int32, [c_void_p, c_int32, ctypes.POINTER(c_float)]),
+    "lsq_stream_time_waits": (c_int32, [c_void_p, c_int32]),
+    "lsq_stream_wait_ms": (c_int32, [c_void_p, ctypes.POINTER(c_float), ctypes.POINTER(c_float),
+                                     ctypes.POINTER(c_int32), ctypes.POINTER(c_int32)]),
     "lsq_stream_reset": (c_int32, [c_void_p]),
     "lsq_stream_destroy": (c_int32, [c_void_p]),
 }
@@ -169,9 +187,9 @@ def _check(name: str, status: int):
 # when dx is wanted, and the dA/dB GEMM with its reduction)
 LAUNCHES = [0]
 _KERNELS = {"lsq_nf4_quantize": 1, "lsq_nf4_dequantize": 1, "lsq_absmax_double_quantize": 1, "lsq_absmax_expand": 1,
-            "lsq_dense_gemm": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1,
+            "lsq_dense_gemm": 1, "lsq_dense_gemm_ex": 1, "lsq_rmsnorm_fwd": 1, "lsq_rmsnorm_bwd": 1, "lsq_rope": 1, "lsq_rope_table": 1,
             "lsq_attention_fwd": 1, "lsq_attention_bwd": 3, "lsq_swiglu_fwd": 1, "lsq_swiglu_bwd": 1,
-            "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1, "lsq_seq_logprob": 2,
+            "lsq_embed_gather": 1, "lsq_xent_fwd_bwd": 2, "lsq_adamw_step": 1, "lsq_lora_refresh_bf16": 1, "lsq_seq_logprob": 2,
             "lsq_dpo_loss": 1, "lsq_seq_logprob_bwd": 1, "lsq_wait_flag": 1}
 
 
@@ -342,6 +360,32 @@ def lsq_nf4_lora_fwd_multi_ex(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, 
           _p(state), 1 if state_ready else 0, _p(workspace), _nbytes(workspace), _stream(stream), launches=launches)
 
 
+def lsq_nf4_lora_fwd_multi_ex2(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int, s: float, residual, y, u_out,
+                               state, state_ready: bool, rope, workspace=None, stream=None):
+    """lsq_nf4_lora_fwd_multi_ex with RoPE in the epilogue: rope = (table, seq, hd, segment bits) or None;
+    state None = the workspace form (lsq_nf4_lora_fwd_multi)."""
+    n = len(Ws)
+    cws = (lsq_nf4_weight * n)(*[w.c() for w in Ws])
+    res = residual if residual is not None else [None] * n
+    uo = u_out if u_out is not None else [None] * n
+    spec = None
+    if rope is not None:
+        spec = lsq_rope_spec(_p(rope[0]), int(rope[1]), int(rope[2]), int(rope[3]))
+    if state is None:
+        workspace = _fwd_workspace(workspace, [w.n_out for w in Ws], M, Ws[0].k_in, r, y[0].device)
+        launches = 2 if r > 0 else 1
+    else:
+        launches = 1 if (r == 0 or state_ready) else 3
+    _call("lsq_nf4_lora_fwd_multi_ex2", n, cws, _p(x), M, _ptrs(A), _ptrs(B), r, s, _ptrs(res), _ptrs(y),
+          _ptrs(uo), _p(state), 1 if state_ready else 0, None if spec is None else ctypes.byref(spec),
+          _p(workspace), _nbytes(workspace), _stream(stream), launches=launches)
+
+
+def lsq_rope_table(theta: float, seq: int, hd: int, table, stream=None):
+    """(cos, sin) fp32 pairs [seq][hd/2] of the RoPE angles into table (device)."""
+    _call("lsq_rope_table", theta, seq, hd, _p(table), _stream(stream))
+
+
 def lsq_nf4_lora_bwd_multi_ex(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, state, dx, dA, dB,
                               accumulate: int, workspace, stream=None):
     n = len(Ws)
@@ -379,6 +423,13 @@ def lsq_dense_gemm(a, b, out, M: int, N: int, K: int, trans_b: int, out_f32: int
 
 
 # ---------------------------------------------------------------------------- layer ops
+def lsq_dense_gemm_ex(a, lda: int, b, out, ldo: int, acc_in, M: int, N: int, K: int, trans_b: int, out_f32: int,
+                      stream=None):
+    """a, b, out, acc_in: tensors or raw device addresses (column blocks pass as addresses)."""
+    _call("lsq_dense_gemm_ex", _p(a), lda, _p(b), _p(out), ldo, _p(acc_in), M, N, K, trans_b, out_f32,
+          _stream(stream))
+
+
 def lsq_rmsnorm_fwd(x, g, y, rstd, rows: int, d: int, eps: float, stream=None):
     _call("lsq_rmsnorm_fwd", _p(x), _p(g), _p(y), _p(rstd), rows, d, eps, _stream(stream))
 
@@ -404,6 +455,16 @@ def lsq_attention_bwd(q, k, v, o, lse, d_o, dq, dk, dv, batch: int, seq: int, hq
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _call("lsq_attention_bwd", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(d_o), _p(dq), _p(dk), _p(dv), batch, seq,
           hq, hkv, hd, _p(workspace), wsb, _stream(stream))
+
+
+def lsq_attention_bwd_ex(q, k, v, o, lse, d_o, dq, dk, dv, batch: int, seq: int, hq: int, hkv: int, hd: int,
+                         rope_table, workspace, stream=None):
+    """lsq_attention_bwd returning the gradients of the unrotated q and k (rope_table from lsq_rope_table)."""
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    fused = hd == 128 and seq <= 512
+    _call("lsq_attention_bwd_ex", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(d_o), _p(dq), _p(dk), _p(dv), batch, seq,
+          hq, hkv, hd, _p(rope_table), _p(workspace), wsb, _stream(stream),
+          launches=3 if (rope_table is None or fused) else 5)
 
 
 def lsq_swiglu_fwd(g, u, m, n: int, stream=None):
@@ -444,6 +505,10 @@ def lsq_dpo_loss(policy_logp, ref_logp, npairs: int, beta: float, loss, dseq, st
 def lsq_seq_logprob_bwd(logits, ids, batch: int, seq: int, V: int, row_lse, dseq, dlogits, stream=None):
     _call("lsq_seq_logprob_bwd", _p(logits), _p(ids), batch, seq, V, _p(row_lse), _p(dseq), _p(dlogits),
           _stream(stream))
+
+
+def lsq_lora_refresh_bf16(p, p_bf16, n: int, stream=None):
+    _call("lsq_lora_refresh_bf16", _p(p), _p(p_bf16), n, _stream(stream))
 
 
 def lsq_adamw_step(p, g, m, v, p_bf16, n: int, step: int, lr: float, beta1: float, beta2: float, eps: float,
@@ -549,6 +614,17 @@ def lsq_stream_upload_ms(st: int, layer: int) -> float:
     ms = c_float(0)
     _call("lsq_stream_upload_ms", st, layer, ctypes.byref(ms))
     return ms.value
+
+
+def lsq_stream_time_waits(st: int, capacity: int):
+    _call("lsq_stream_time_waits", st, capacity)
+
+
+def lsq_stream_wait_ms(st: int):
+    """-> (forward ms, backward ms, waits kept, waits dropped) since the previous call."""
+    f, b, n, d = c_float(0), c_float(0), c_int32(0), c_int32(0)
+    _call("lsq_stream_wait_ms", st, ctypes.byref(f), ctypes.byref(b), ctypes.byref(n), ctypes.byref(d))
+    return f.value, b.value, n.value, d.value
 
 
 def lsq_stream_reset(st: int):

@@ -6,8 +6,10 @@ is quantised once, offline, to NF4 and kept in page-locked host RAM as one
 record per decoder layer; each training step streams the records through a
 small ring of HBM slots, forward 0 -> L-1, and under gradient checkpointing
 re-streams them L-1 -> 0 for the backward, recomputing each layer from its
-saved input; the embedding and lm_head remain on the GPU unquantised; the
-LoRA adapters are the only trained parameters (optimizer step at the end).
+saved input; the embedding and lm_head stay unquantised, on the GPU or (as the
+pages plan for them) in page-locked host RAM, the head then streamed in
+vocabulary chunks; the LoRA adapters are the only trained parameters
+(optimizer step at the end).
 
 This module only allocates memory (torch), builds the host store and calls
 the library in order.  Every arithmetic step runs in the library's kernels.
@@ -136,7 +138,7 @@ class LoraParams:
             for name, t in per.items():
                 for ab in ("A", "B"):
                     self.view(self.master, l, name, ab).copy_(t[ab])
-        self.op.copy_(self.master)
+        L.lsq_lora_refresh_bf16(self.master, self.op, self.numel)
 
     def init_device(self, seed: int = S.LORA_SEED):
         for l in range(self.shape.n_layers):
@@ -146,7 +148,7 @@ class LoraParams:
                     S.device_normal_f32((self.shape.r, k), 1.0 / math.sqrt(k), seed, st))
                 self.view(self.master, l, name, "B").copy_(
                     S.device_normal_f32((n, self.shape.r), S.LORA_B_STD, seed, st + 8))
-        self.op.copy_(self.master)
+        L.lsq_lora_refresh_bf16(self.master, self.op, self.numel)
 
 
 class StreamedLoraTrainer:
@@ -156,12 +158,18 @@ class StreamedLoraTrainer:
     resident run (one slot per layer, every layer uploaded once).
     init: "host" draws every weight from the seeded numpy streams that the
     oracle also reads; "device" draws them with the CUDA RNG (full-size runs).
+    head: "hbm" keeps the lm_head resident; "host" keeps it in page-locked
+    host RAM and streams it in vocabulary chunks of head_chunk rows through
+    two HBM chunk buffers on the copy stream, once for each of its GEMMs (with
+    a tied embedding the one host table also serves the gather, zero-copy).
+    The chunked GEMMs give bit for bit the resident head's results.
     """
 
     def __init__(self, shape: S.ModelShape, batch: int, seq: int, n_slots: Optional[int] = 2,
                  init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None,
                  absmax: str = "fp32", shard: Optional[tuple] = None, source: str = "ram",
-                 store_path: Optional[str] = None, embed: str = "hbm"):
+                 store_path: Optional[str] = None, embed: str = "hbm", head: str = "hbm",
+                 head_chunk: int = 8192):
         self.shape, self.B, self.S = shape, batch, seq
         self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
         self.M = batch * seq
@@ -185,11 +193,18 @@ class StreamedLoraTrainer:
         if embed not in ("hbm", "host") or (embed == "host" and shape.tied):
             raise ValueError("embed must be 'hbm', or 'host' for an untied embedding")
         self.embed_kind = embed
+        if head not in ("hbm", "host") or head_chunk < 64 or head_chunk % 256 != 0:
+            raise ValueError("head must be 'hbm' or 'host'; head_chunk a positive multiple of 256 rows")
+        self.head_kind, self.head_chunk = head, int(head_chunk)
+        if head == "host" and shape.tied:
+            self.embed_kind = embed = "host"   # one table: the head's host copy also serves the gather
         self.compute = torch.cuda.current_stream()
         self.copy = torch.cuda.Stream()
         if share is not None and (share.absmax_kind != absmax or share.shard != self.shard or
-                                  (share.source, share.store_path, share.embed_kind) != (source, store_path, embed)):
-            raise ValueError("a shared store must have the same absmax format, sharding, source and embed place")
+                                  (share.source, share.store_path, share.embed_kind, share.head_kind,
+                                   share.head_chunk) != (source, store_path, embed, head, self.head_chunk)):
+            raise ValueError("a shared store must have the same absmax format, sharding, source, embed and head "
+                             "places")
         if share is not None:       # reuse another trainer's host store and resident tensors
             self.host_records = share.host_records
             self.embed, self.lm_head, self.final_norm = share.embed, share.lm_head, share.final_norm
@@ -217,6 +232,18 @@ class StreamedLoraTrainer:
                                          disk=disk)
         if self.layout.dq:
             L.lsq_stream_set_absmax_expand(self.sched, self.layout.expand_items(), self.layout.slot_bytes)
+        self.head_sched = None
+        if self.head_kind == "host":
+            # the head's chunks are the "layers" of a second scheduler: same copy stream, two slots
+            C, d = self.head_chunk, shape.d
+            self.head_chunks = -(-shape.vocab // C)
+            cbytes = C * d * 2
+            self.head_slots = [torch.empty(cbytes, dtype=torch.uint8, device=device) for _ in range(2)]
+            base = self.lm_head.data_ptr()
+            self.head_sched = L.lsq_stream_create(self.head_chunks, 2, cbytes, [t.data_ptr() for t in self.head_slots],
+                                                  [base + c * cbytes for c in range(self.head_chunks)],
+                                                  self.compute, self.copy)
+            self.dh32 = torch.empty(self.M, d, dtype=torch.float32, device=device)
         if self.resident:
             for l in range(shape.n_layers):
                 L.lsq_layer_upload_async(self.sched, l, l)
@@ -285,7 +312,15 @@ class StreamedLoraTrainer:
             self.embed = S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD, S.WEIGHT_SEED, 11)
             self.lm_head = self.embed if sh.tied else S.device_normal_bf16((sh.vocab, sh.d), S.BASE_STD,
                                                                             S.WEIGHT_SEED, 12)
-        if self.embed_kind == "host":   # page-locked host copy; the gather reads it in place
+        if self.head_kind == "host":
+            # page-locked host copy, padded to whole chunks (every chunk upload copies the same bytes)
+            rows = -(-sh.vocab // self.head_chunk) * self.head_chunk
+            host = torch.zeros(rows, sh.d, dtype=self.lm_head.dtype, pin_memory=True)
+            host[:sh.vocab].copy_(self.lm_head)
+            if sh.tied:
+                self.embed = host
+            self.lm_head = host
+        if self.embed_kind == "host" and not self.embed.is_pinned():   # the gather reads it in place
             host = torch.empty(self.embed.shape, dtype=self.embed.dtype, pin_memory=True)
             host.copy_(self.embed)
             self.embed = host
@@ -332,6 +367,11 @@ class StreamedLoraTrainer:
         self.ws_attn = torch.empty(L.lsq_attention_bwd_workspace_size(self.B, self.S, sh.n_q), dtype=torch.uint8,
                                    device=dev)
         self.ws_xent = torch.empty(L.lsq_xent_workspace_size(M), dtype=torch.uint8, device=dev)
+        # RoPE: (cos, sin) per position and frequency; with head dims the fused GEMM epilogue serves,
+        # q and k are rotated there and the attention backward returns their unrotated gradients
+        self.rope_table = torch.empty(self.S * sh.hd, dtype=torch.float32, device=dev)
+        L.lsq_rope_table(sh.theta, self.S, sh.hd, self.rope_table)
+        self.fuse_rope = sh.hd in (64, 128, 256)
 
     # ------------------------------------------------------------------ timing
     def _t0(self):
@@ -384,8 +424,13 @@ class StreamedLoraTrainer:
         ready = save           # the recompute: the first forward of this step filled the rank state
         rf = 0 if (state and ready) else r   # rank-r FLOPs done in this call
 
-        def fused(group, Ws, x, names, res, ys):
-            if state:
+        def fused(group, Ws, x, names, res, ys, rope=None):
+            if rope is not None:
+                L.lsq_nf4_lora_fwd_multi_ex2(Ws, x, M, [A[n] for n in names], [B[n] for n in names], r, s, res, ys,
+                                             None if state else [U[n] for n in names],
+                                             self.rank_state[l][group] if state else None, ready, rope,
+                                             workspace=self.ws_lora)
+            elif state:
                 L.lsq_nf4_lora_fwd_multi_ex(Ws, x, M, [A[n] for n in names], [B[n] for n in names], r, s, res, ys,
                                             None, self.rank_state[l][group], ready, workspace=self.ws_lora)
             else:
@@ -394,10 +439,12 @@ class StreamedLoraTrainer:
 
         L.lsq_rmsnorm_fwd(hin, W.ln1, self.x1, self.rstd1, M, sh.d, sh.eps)
         t = self._t0()
-        fused("qkv", [W.W["q"], W.W["k"], W.W["v"]], self.x1, ["q", "k", "v"], None, [self.q, self.k, self.v])
+        rope = (self.rope_table, self.S, sh.hd, 0b011) if self.fuse_rope else None   # q and k
+        fused("qkv", [W.W["q"], W.W["k"], W.W["v"]], self.x1, ["q", "k", "v"], None, [self.q, self.k, self.v], rope)
         self._t1(t, "nf4_fwd", self._fwd_flops([sh.d, sh.kv, sh.kv], sh.d, rf, r))
-        L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
-        L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
+        if not self.fuse_rope:
+            L.lsq_rope(self.q, self.B, self.S, sh.n_q, sh.hd, sh.theta, 0)
+            L.lsq_rope(self.k, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 0)
         L.lsq_attention_fwd(self.q, self.k, self.v, self.a, self.lse, self.B, self.S, sh.n_q, sh.n_kv, sh.hd)
         t = self._t0()
         fused("o", [W.W["o"]], self.a, ["o"], [hin], [self.hmid])
@@ -443,15 +490,49 @@ class StreamedLoraTrainer:
         t = self._t0()
         fused_bwd("o", [W.W["o"]], self.a, [self.dhmid], ["o"], self.da)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.d], sh.d))
-        L.lsq_attention_bwd(self.q, self.k, self.v, self.a, self.lse, self.da, self.dq, self.dk, self.dv, self.B,
-                            self.S, sh.n_q, sh.n_kv, sh.hd, self.ws_attn)
-        L.lsq_rope(self.dq, self.B, self.S, sh.n_q, sh.hd, sh.theta, 1)
-        L.lsq_rope(self.dk, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 1)
+        L.lsq_attention_bwd_ex(self.q, self.k, self.v, self.a, self.lse, self.da, self.dq, self.dk, self.dv, self.B,
+                               self.S, sh.n_q, sh.n_kv, sh.hd, self.rope_table if self.fuse_rope else None,
+                               self.ws_attn)
+        if not self.fuse_rope:
+            L.lsq_rope(self.dq, self.B, self.S, sh.n_q, sh.hd, sh.theta, 1)
+            L.lsq_rope(self.dk, self.B, self.S, sh.n_kv, sh.hd, sh.theta, 1)
         t = self._t0()
         fused_bwd("qkv", [W.W["q"], W.W["k"], W.W["v"]], self.x1, [self.dq, self.dk, self.dv], ["q", "k", "v"],
                   self.dx)
         self._t1(t, "nf4_bwd", self._bwd_flops([sh.d, sh.kv, sh.kv], sh.d))
         L.lsq_rmsnorm_bwd(self.dx, self.h[l], W.ln1, self.rstd1, self.dhmid, self.dh, M, sh.d)
+
+    def _head_chunk_rows(self, c: int):
+        r0 = c * self.head_chunk
+        return r0, min(self.head_chunk, self.shape.vocab - r0)
+
+    def _head_logits(self):
+        """logits = hn E^T (fp32): one GEMM over the resident head, or one per streamed chunk,
+        each writing its block of logit columns."""
+        sh, M = self.shape, self.M
+        if self.head_sched is None:
+            L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+            return
+        for c in range(self.head_chunks):
+            Ec = L.lsq_stream_step(self.head_sched, c, +1)
+            r0, rows = self._head_chunk_rows(c)
+            L.lsq_dense_gemm_ex(self.hn, sh.d, Ec, self.logits.data_ptr() + 4 * r0, sh.vocab, None, M, rows, sh.d,
+                                0, 1)
+
+    def _head_dh(self):
+        """hn <- dlogits E: one GEMM over the resident head, or the contraction over the vocabulary
+        split at the streamed chunks, each call continuing from the fp32 accumulator the previous
+        left (bit-identical to the one GEMM)."""
+        sh, M = self.shape, self.M
+        if self.head_sched is None:
+            L.lsq_dense_gemm(self.dlogits, self.lm_head, self.hn, M, sh.d, sh.vocab, 1, 0)
+            return
+        last = self.head_chunks - 1
+        for c in range(self.head_chunks):
+            Ec = L.lsq_stream_step(self.head_sched, c, +1)
+            r0, rows = self._head_chunk_rows(c)
+            L.lsq_dense_gemm_ex(self.dlogits.data_ptr() + 2 * r0, sh.vocab, Ec, self.hn if c == last else self.dh32,
+                                sh.d, None if c == 0 else self.dh32, M, sh.d, rows, 1, 0 if c == last else 1)
 
     def _view(self, l: int, direction: int) -> LayerView:
         return LayerView(self.shape, self.layout, L.lsq_stream_step(self.sched, l, direction))
@@ -467,10 +548,10 @@ class StreamedLoraTrainer:
         for l in range(sh.n_layers):
             self._layer_fwd(l, self._view(l, +1), save=False)
         L.lsq_rmsnorm_fwd(self.h[sh.n_layers], self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
-        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        self._head_logits()
         L.lsq_xent_fwd_bwd(self.logits, self.ids, self.B, self.S, sh.vocab, self.loss_dev, self.dlogits,
                            self.ws_xent)
-        L.lsq_dense_gemm(self.dlogits, self.lm_head, self.hn, M, sh.d, sh.vocab, 1, 0)   # hn <- d hn
+        self._head_dh()   # hn <- d hn
         L.lsq_rmsnorm_bwd(self.hn, self.h[sh.n_layers], self.final_norm, self.rstdf, None, self.dh, M, sh.d)
         for l in reversed(range(sh.n_layers)):
             W = self._view(l, -1)
@@ -506,16 +587,16 @@ class StreamedLoraTrainer:
             self._layer_fwd(l, W, save=False, hin=self.h_ref, hout=self.h_ref, adapter=False)
         # reference sequence log-probabilities
         L.lsq_rmsnorm_fwd(self.h_ref, self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
-        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        self._head_logits()
         L.lsq_seq_logprob(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.ref_logp, self.ws_seqlp)
         # policy sequence log-probabilities, loss, d loss / d logits
         L.lsq_rmsnorm_fwd(self.h[sh.n_layers], self.final_norm, self.hn, self.rstdf, M, sh.d, sh.eps)
-        L.lsq_dense_gemm(self.hn, self.lm_head, self.logits, M, sh.vocab, sh.d, 0, 1)
+        self._head_logits()
         L.lsq_seq_logprob(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.pi_logp, self.ws_seqlp)
         L.lsq_dpo_loss(self.pi_logp, self.ref_logp, self.B // 2, beta, self.loss_dev, self.dseq)
         L.lsq_seq_logprob_bwd(self.logits, self.ids, self.B, self.S, sh.vocab, self.row_lse, self.dseq,
                               self.dlogits)
-        L.lsq_dense_gemm(self.dlogits, self.lm_head, self.hn, M, sh.d, sh.vocab, 1, 0)   # hn <- d hn
+        self._head_dh()   # hn <- d hn
         L.lsq_rmsnorm_bwd(self.hn, self.h[sh.n_layers], self.final_norm, self.rstdf, None, self.dh, M, sh.d)
         for l in reversed(range(sh.n_layers)):
             W = self._view(l, -1)
@@ -545,11 +626,31 @@ class StreamedLoraTrainer:
     def stats(self):
         return L.lsq_stream_stats(self.sched)
 
+    def head_stats(self):
+        """(uploads, bytes, reused) of the streamed head's chunks; zeros with a resident head."""
+        return L.lsq_stream_stats(self.head_sched) if self.head_sched is not None else (0, 0, 0)
+
+    def check_device(self):
+        """Raise LsqError if a bounded wait inside any kernel ran out since the
+        last check (the library's device status word, which the read clears):
+        a kernel that gave up leaves its outputs incomplete, so no loss,
+        gradient or timing of those steps stands.  Synchronises the device."""
+        torch.cuda.synchronize()
+        status, where = L.lsq_device_status()
+        if status != 0:
+            raise L.LsqError(status, "device status word",
+                             f"a bounded device wait gave up (site {where}); results since the last check are void")
+
     def close(self):
+        if getattr(self, "head_sched", None):
+            torch.cuda.synchronize()
+            L.lsq_stream_destroy(self.head_sched)
+            self.head_sched = None
         if getattr(self, "sched", None):
             torch.cuda.synchronize()
             L.lsq_stream_destroy(self.sched)
             self.sched = None
+            self.check_device()
 
     def __del__(self):
         try:

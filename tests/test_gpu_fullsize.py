@@ -1,8 +1,11 @@
-"""Parity at the full 8B and 32B sizes, in the launch configuration bench.py times.
+"""Parity at the full 8B, 32B and 3B sizes, in the launch configuration bench.py times.
 
-Every fused linear of one 8B and one 32B decoder layer at 2048 tokens (q/k/v,
-o, gate/up, down), the 8B lm_head GEMMs and the attention of 4 x 512 tokens
-(32 / 8 and 40 / 8 heads) run exactly as in a training step (stream-K
+Every fused linear of one 8B and one 32B decoder layer at 2048 tokens and of
+one Qwen2.5-3B layer at 512 tokens (q/k/v, o, gate/up, down; the 3B k and v
+projections are 256 wide, one SM-pair tile), the 8B lm_head GEMMs and the tied
+3B head (151936 x 2048), the attention of 4 x 512 tokens (32 / 8 and 40 / 8
+heads) and of 1 x 512 tokens at 16 / 2 heads (GQA groups of 8) run exactly as
+in a training step (stream-K
 workspace, rank state filled by the forward and reused by the recompute and
 the backward, dA / dB beside dX).  The 32B layer's record is 274 MB, above
 the 165 MiB per layer where the pages report silently wrong NF4 gradients
@@ -19,7 +22,8 @@ one by one from its own quantisation of just the rows and blocks involved:
 
 Tolerances as the single-linear tests (tolerances.assert_close: relative
 Frobenius 5e-3 and max-abs 2e-2 of the RMS on the sampled block; attention
-per row).
+element by element within the first-order bound of its bf16 roundings,
+attn_bounds.py, and relative Frobenius 5e-3).
 """
 import math
 
@@ -30,12 +34,12 @@ import torch
 import synthetic as S
 from oracle import decoder as D
 from oracle import nf4 as ON
-from tolerances import assert_close, assert_close_rows
+from attn_bounds import attention_bounds
+from tolerances import assert_close, assert_within_bound
 
 pytestmark = pytest.mark.gpu
 
 F64 = np.float64
-M = 2048
 R = 16
 SCALE = 1.0
 
@@ -61,10 +65,15 @@ def _wd_block(W, kb):
 GROUPS = {"qkv": (["q", "k", "v"], "d"), "o": (["o"], "d"), "gateup": (["gate", "up"], "d"), "down": (["down"], "f")}
 
 
-@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b"])
+# tokens per step of each shape's workload: batch 4 x 512 (8B, 32B), batch 1 x 512 (3B)
+TOKENS = {"llama-3.1-8b": 2048, "dense-32b": 2048, "qwen2.5-3b": 512}
+
+
+@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b", "qwen2.5-3b"])
 @pytest.mark.parametrize("group", list(GROUPS))
 def test_fused_linear_fullsize_sampled(lsq, shape, group):
     sh = S.SHAPES[shape]
+    M = TOKENS[shape]
     names, kdim = GROUPS[group]
     shapes = sh.linear_shapes()
     K = sh.d if kdim == "d" else sh.f
@@ -119,8 +128,12 @@ def test_fused_linear_fullsize_sampled(lsq, shape, group):
     assert_close(dx.float().cpu().numpy()[rows][:, ks], dx_ref, what=f"{group} dX")
 
 
-def test_lm_head_fullsize_sampled(lsq):
-    sh = S.LLAMA8B
+@pytest.mark.parametrize("shape", ["llama-3.1-8b", "qwen2.5-3b"])
+def test_lm_head_fullsize_sampled(lsq, shape):
+    """The untied 8B head (128256 x 4096) and the tied 3B embedding used as the
+    head (151936 x 2048), logits and input gradient."""
+    sh = S.SHAPES[shape]
+    M = TOKENS[shape]
     rng = np.random.default_rng(8)
     hn = S.bf16(S.normal_f32(S.DATA_SEED, 510, (M, sh.d)))
     E = S.bf16_weight(sh.vocab, sh.d, 610)
@@ -140,9 +153,10 @@ def test_lm_head_fullsize_sampled(lsq):
     assert_close(dh.float().cpu().numpy()[np.ix_(rows, dcols)], DL @ E[:, dcols].double().numpy(), what="dh")
 
 
-@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b"])
+@pytest.mark.parametrize("shape", ["llama-3.1-8b", "dense-32b", "qwen2.5-3b"])
 def test_attention_fullsize_sampled(lsq, shape):
-    sh, B, Sq = S.SHAPES[shape], 4, 512
+    sh, Sq = S.SHAPES[shape], 512
+    B = TOKENS[shape] // Sq
     Hq, Hkv, hd = sh.n_q, sh.n_kv, sh.hd
     rng = np.random.default_rng(9)
     q = S.bf16(S.normal_f32(S.DATA_SEED, 520, (B, Sq, Hq, hd)))
@@ -158,15 +172,22 @@ def test_attention_fullsize_sampled(lsq, shape):
     lsq.lsq_attention_bwd(qg, kg, vg, o, lse, do.cuda(), dq, dk, dv, B, Sq, Hq, Hkv, hd, ws)
     torch.cuda.synchronize()
     group = Hq // Hkv
-    for b, hk in [(0, 0), (3, Hkv - 1), (int(rng.integers(0, B)), int(rng.integers(0, Hkv)))]:
+    for b, hk in [(0, 0), (B - 1, Hkv - 1), (int(rng.integers(0, B)), int(rng.integers(0, Hkv)))]:
         heads = list(range(hk * group, (hk + 1) * group))
-        # the oracle on one sequence and the query heads of one kv head (the whole GQA group)
-        qs = q[b:b + 1, :, heads].double().requires_grad_(True)
-        ks = k[b:b + 1, :, hk:hk + 1].double().requires_grad_(True)
-        vs = v[b:b + 1, :, hk:hk + 1].double().requires_grad_(True)
-        out = D.causal_gqa_attention(qs, ks, vs)
-        out.backward(do[b:b + 1, :, heads].double())
-        assert_close_rows(o[b, :, heads].float().cpu().numpy(), out[0].detach().numpy(), what=f"o b{b} kv{hk}")
-        assert_close_rows(dq[b, :, heads].float().cpu().numpy(), qs.grad[0].numpy(), what=f"dq b{b} kv{hk}")
-        assert_close_rows(dk[b, :, hk:hk + 1].float().cpu().numpy(), ks.grad[0].numpy(), what=f"dk b{b} kv{hk}")
-        assert_close_rows(dv[b, :, hk:hk + 1].float().cpu().numpy(), vs.grad[0].numpy(), what=f"dv b{b} kv{hk}")
+        # the oracle on one sequence and the query heads of one kv head (the whole GQA group),
+        # element by element within the first-order bound of the kernels' bf16 roundings
+        qs, ks, vs, dos = q[b:b + 1, :, heads], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1], do[b:b + 1, :, heads]
+        bnd = attention_bounds(qs, ks, vs, dos)
+        xs = [t.double().requires_grad_(True) for t in (qs, ks, vs)]
+        out = D.causal_gqa_attention(*xs)
+        grads = torch.autograd.grad(out, xs, grad_outputs=dos.double())
+        for name, want in zip(("o", "dq", "dk", "dv"), (out.detach(), *grads)):
+            assert torch.allclose(bnd[name], want, rtol=1e-9, atol=1e-12), name   # the oracle's values
+        assert_within_bound(o[b:b + 1, :, heads].double().cpu().numpy(), bnd["o"].numpy(), bnd["b_o"].numpy(),
+                            what=f"o b{b} kv{hk}")
+        assert_within_bound(dq[b:b + 1, :, heads].double().cpu().numpy(), bnd["dq"].numpy(), bnd["b_dq"].numpy(),
+                            what=f"dq b{b} kv{hk}")
+        assert_within_bound(dk[b:b + 1, :, hk:hk + 1].double().cpu().numpy(), bnd["dk"].numpy(),
+                            bnd["b_dk"].numpy(), what=f"dk b{b} kv{hk}")
+        assert_within_bound(dv[b:b + 1, :, hk:hk + 1].double().cpu().numpy(), bnd["dv"].numpy(),
+                            bnd["b_dv"].numpy(), what=f"dv b{b} kv{hk}")

@@ -9,7 +9,8 @@ import torch
 
 import synthetic as S
 from oracle import decoder as D
-from tolerances import assert_close, assert_close_ew, assert_close_rows
+from attn_bounds import attention_bounds
+from tolerances import assert_close, assert_close_ew, assert_within_bound
 
 pytestmark = pytest.mark.gpu
 F64 = torch.float64
@@ -30,14 +31,13 @@ def _grad(fn, inputs, dy):
     return out.detach(), gr
 
 
-@pytest.mark.parametrize("M,d", [(130, 576), (64, 4096), (1, 256)])
-def test_rmsnorm_fwd_bwd(lsq, M, d):
+@pytest.mark.parametrize("M,d,eps", [(130, 576, 1e-5), (64, 4096, 1e-5), (1, 256, 1e-5), (512, 2048, 1e-6)])
+def test_rmsnorm_fwd_bwd(lsq, M, d, eps):
     x = _rand((M, d), 2.0, 1)
     g = _rand((d,), 0.3, 2) + 1
     g = g.to(torch.bfloat16)
     dy = _rand((M, d), 1.0, 3)
     res = _rand((M, d), 1.0, 4)
-    eps = 1e-5
     y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
     rstd = torch.empty(M, dtype=torch.float32, device="cuda")
     lsq.lsq_rmsnorm_fwd(x.cuda(), g.cuda(), y, rstd, M, d, eps)
@@ -51,7 +51,8 @@ def test_rmsnorm_fwd_bwd(lsq, M, d):
     assert_close_ew(_np(out), dx.numpy() + _np(res), what="rmsnorm dx + res")
 
 
-@pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5), (1, 50, 3, 24, 1e4)])
+@pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5), (1, 50, 3, 24, 1e4),
+                                             (1, 512, 16, 128, 1e6)])
 def test_rope_fwd_and_transpose(lsq, B, Sq, H, hd, theta):
     x = _rand((B, Sq, H, hd), 1.0, 5)
     dy = _rand((B, Sq, H, hd), 1.0, 6)
@@ -89,7 +90,8 @@ def _attn_case(B, Sq, Hq, Hkv, hd, seed):
 
 @pytest.mark.parametrize("B,Sq,Hq,Hkv,hd", [(1, 512, 9, 3, 64), (2, 200, 4, 1, 128), (1, 64, 2, 2, 64),
                                             (1, 1, 4, 2, 128), (2, 130, 8, 2, 128), (2, 512, 32, 8, 128),
-                                            (1, 384, 4, 4, 128), (1, 300, 7, 1, 128), (2, 256, 6, 2, 128)])
+                                            (1, 384, 4, 4, 128), (1, 300, 7, 1, 128), (2, 256, 6, 2, 128),
+                                            (1, 512, 16, 2, 128)])
 def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
     q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, Sq)
     o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
@@ -102,20 +104,22 @@ def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
     lsq.lsq_attention_bwd(q.cuda(), k.cuda(), v.cuda(), o, lse, do.cuda(), dq, dk, dv, B, Sq, Hq, Hkv, hd, ws)
     torch.cuda.synchronize()
     ref, (rq, rk, rv) = _grad(D.causal_gqa_attention, [q, k, v], do)
-    assert_close_ew(_np(o), ref.numpy(), what="attn out")
     # lse of the scaled scores
     kk = k.to(F64).repeat_interleave(Hq // Hkv, dim=2)
     sc = torch.einsum("bihd,bjhd->bhij", q.to(F64), kk) / math.sqrt(hd)
     sc = sc.masked_fill(torch.triu(torch.ones(Sq, Sq, dtype=torch.bool), 1), float("-inf"))
     assert_close(lse.cpu().numpy(), torch.logsumexp(sc, -1).numpy(), rel=1e-5, max_rms=1e-4, what="lse")
-    # P and dS enter the tensor cores as bf16: relative error up to ~2^-8 per
-    # term, so each gradient row (one position, one head) is checked against
-    # its own norm (tolerances.assert_close_rows).  With a single key the
-    # softmax gradient is exactly zero; the kernel leaves a residue of dP - D
-    # (two fp32 sums of the same products in different orders), about 1e-6.
-    assert_close_rows(_np(dq), rq.numpy(), what="dq")
-    assert_close_rows(_np(dk), rk.numpy(), what="dk")
-    assert_close_rows(_np(dv), rv.numpy(), what="dv")
+    # Element by element within the first-order bound of the kernels' bf16
+    # roundings (P and dS enter the tensor cores as bf16, D is formed from the
+    # bf16 output; attn_bounds.py), plus relative Frobenius 5e-3.  The bound's
+    # exact values are the oracle's (autograd through its forward).
+    bnd = attention_bounds(q, k, v, do)
+    for name, want in (("o", ref), ("dq", rq), ("dk", rk), ("dv", rv)):
+        assert torch.allclose(bnd[name], want, rtol=1e-9, atol=1e-12), name
+    assert_within_bound(_np(o), ref.numpy(), bnd["b_o"].numpy(), what="attn out")
+    assert_within_bound(_np(dq), rq.numpy(), bnd["b_dq"].numpy(), what="dq")
+    assert_within_bound(_np(dk), rk.numpy(), bnd["b_dk"].numpy(), what="dk")
+    assert_within_bound(_np(dv), rv.numpy(), bnd["b_dv"].numpy(), what="dv")
 
 
 def test_attention_deterministic(lsq):
@@ -176,3 +180,42 @@ def test_adamw_matches_oracle(lsq):
     torch.cuda.synchronize()
     assert_close(pg.cpu().numpy(), ref[0].numpy(), rel=1e-6, max_rms=1e-6, what="adamw p")
     assert torch.equal(pb.cpu(), pg.cpu().to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("B,Sq,Hq,Hkv,hd,theta", [(1, 384, 4, 4, 128, 5e5), (2, 130, 8, 2, 128, 1e4),
+                                                  (1, 300, 7, 1, 128, 1e6), (1, 512, 9, 3, 64, 1e4)])
+def test_attention_bwd_with_rope_transpose(lsq, B, Sq, Hq, Hkv, hd, theta):
+    """lsq_attention_bwd_ex with a RoPE table returns the gradients of the
+    unrotated q and k: the transpose of the rotation applied to the attention
+    gradients (in fp32 before the one rounding on the tcgen05 path, in a pass
+    over the bf16 gradients on the other), against the oracle's RoPE
+    transpose (autograd through oracle.decoder.rope) of its attention
+    gradients; dv is the plain attention's, bit for bit."""
+    q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, 3 * Sq)
+    qg, kg, vg, dog = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device="cuda")
+    lsq.lsq_attention_fwd(qg, kg, vg, o, lse, B, Sq, Hq, Hkv, hd)
+    table = torch.empty(Sq * hd, dtype=torch.float32, device="cuda")
+    lsq.lsq_rope_table(theta, Sq, hd, table)
+    ws = torch.empty(lsq.lsq_attention_bwd_workspace_size(B, Sq, Hq), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(o), torch.empty_like(kg), torch.empty_like(vg)
+    lsq.lsq_attention_bwd_ex(qg, kg, vg, o, lse, dog, dq, dk, dv, B, Sq, Hq, Hkv, hd, table, ws)
+    dq0, dk0, dv0 = torch.empty_like(o), torch.empty_like(kg), torch.empty_like(vg)
+    lsq.lsq_attention_bwd(qg, kg, vg, o, lse, dog, dq0, dk0, dv0, B, Sq, Hq, Hkv, hd, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(dv, dv0)
+    bnd = attention_bounds(q, k, v, do)
+
+    def rope_t(g):   # the oracle's RoPE transpose of g (autograd through its forward rotation)
+        z = torch.zeros_like(g, dtype=F64).requires_grad_(True)
+        return torch.autograd.grad(D.rope(z, theta), z, grad_outputs=g.to(F64))[0]
+
+    h = hd // 2
+    for name, got, g, b in (("dq rope", dq, bnd["dq"], bnd["b_dq"]), ("dk rope", dk, bnd["dk"], bnd["b_dk"])):
+        ref = rope_t(g)
+        # the unrotated gradient's bound carried through the rotation (|cos|, |sin| <= 1: column i
+        # takes the bounds of i and its partner), plus one more rounding of the rotated value
+        w = torch.cat([b[..., :h] + b[..., h:], b[..., h:] + b[..., :h]], dim=-1)
+        bound = w + 2.0 ** -8 * ref.abs()
+        assert_within_bound(_np(got), ref.numpy(), bound.numpy(), what=name)

@@ -299,3 +299,84 @@ def test_bounded_wait_times_out_and_the_context_survives(lsq):
     with pytest.raises(lsq.LsqError) as e:
         lsq.lsq_wait_flag(flag, 1, 0)
     assert e.value.status == 1
+
+
+@pytest.mark.parametrize("M,V,d,C", [(300, 3000, 512, 1024), (512, 1000, 256, 256)])
+def test_dense_gemm_chunked_equals_whole_bitwise(lsq, M, V, d, C):
+    """The lm_head GEMMs over vocabulary chunks (lsq_dense_gemm_ex): logits
+    column blocks written with a row stride, and the input gradient's
+    contraction split at the chunks, each call continuing from the fp32
+    accumulator the previous left - bit-identical to the single GEMMs, which
+    match the fp64 product."""
+    h = S.bf16(S.normal_f32(S.DATA_SEED, 530, (M, d))).cuda()
+    E = S.bf16_weight(V, d, 630).cuda()
+    dl = S.bf16(S.normal_f32(S.DATA_SEED, 531, (M, V), 1e-2)).cuda()
+    lg1 = torch.empty(M, V, dtype=torch.float32, device="cuda")
+    lg2 = torch.full((M, V), float("nan"), dtype=torch.float32, device="cuda")
+    dh1 = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    dh2 = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    acc = torch.empty(M, d, dtype=torch.float32, device="cuda")
+    lsq.lsq_dense_gemm(h, E, lg1, M, V, d, 0, 1)
+    lsq.lsq_dense_gemm(dl, E, dh1, M, d, V, 1, 0)
+    starts = list(range(0, V, C))
+    for i, r0 in enumerate(starts):
+        rows = min(C, V - r0)
+        Ec = E[r0:r0 + rows].contiguous()
+        lsq.lsq_dense_gemm_ex(h, d, Ec, lg2.data_ptr() + 4 * r0, V, None, M, rows, d, 0, 1)
+        last = i == len(starts) - 1
+        lsq.lsq_dense_gemm_ex(dl.data_ptr() + 2 * r0, V, Ec, dh2 if last else acc, d, None if i == 0 else acc,
+                              M, d, rows, 1, 0 if last else 1)
+    torch.cuda.synchronize()
+    assert torch.equal(lg1, lg2) and torch.equal(dh1, dh2)
+    Hd, Ed, Dd = h.double().cpu().numpy(), E.double().cpu().numpy(), dl.double().cpu().numpy()
+    assert_close(lg2.cpu().numpy(), Hd @ Ed.T, rel=5e-5, max_rms=2e-2, what="chunked logits")
+    assert_close(dh2.float().cpu().numpy(), Dd @ Ed, what="chunked dh")
+
+
+@pytest.mark.parametrize("M,seq,Ns,K,hd,r,theta", [(512, 256, [512, 256, 256], 512, 128, 16, 5e5),
+                                                   (384, 128, [256, 128, 128], 256, 64, 8, 1e4),
+                                                   (2048, 512, [4096, 1024, 1024], 4096, 128, 16, 5e5)])
+def test_fused_forward_with_rope_matches_oracle(lsq, M, seq, Ns, K, hd, r, theta):
+    """q and k rotated by RoPE in the fused GEMM's epilogue (segments 0 and 1;
+    v not rotated) against the oracle's linear followed by its RoPE
+    (oracle.decoder.rope) on whole sequences, on up to four sampled heads of
+    each segment; with the rank state and with the workspace form, bit for bit
+    the same; the 8B q/k/v shape at 2048 tokens runs the stream-K tail."""
+    from oracle import decoder as OD
+    s = 16.0 / r
+    x = S.bf16(S.normal_f32(S.DATA_SEED, 540, (M, K)))
+    Ws = [S.bf16_weight(n, K, 640 + i) for i, n in enumerate(Ns)]
+    As = [torch.from_numpy(S.normal_f32(S.LORA_SEED, 740 + i, (r, K), K ** -0.5)).to(torch.bfloat16) for i in range(3)]
+    Bs = [torch.from_numpy(S.normal_f32(S.LORA_SEED, 840 + i, (n, r), 0.02)).to(torch.bfloat16)
+          for i, n in enumerate(Ns)]
+    qw = []
+    for W in Ws:
+        w = lsq.NF4Weight.empty(W.shape[0], K)
+        lsq.lsq_nf4_quantize(W.cuda(), w.codes, w.absmax)
+        qw.append(w)
+    table = torch.empty(seq * hd, dtype=torch.float32, device="cuda")
+    lsq.lsq_rope_table(theta, seq, hd, table)
+    ws = torch.zeros(lsq.lsq_nf4_lora_fwd_workspace_size(Ns, M, K, r), dtype=torch.uint8, device="cuda")
+    state = torch.zeros(lsq.lsq_nf4_lora_state_size(Ns, M, K, r), dtype=torch.uint8, device="cuda")
+    xg, Ag, Bg = x.cuda(), [a.cuda() for a in As], [b.cuda() for b in Bs]
+    y1 = [torch.empty(M, n, dtype=torch.bfloat16, device="cuda") for n in Ns]
+    y2 = [torch.empty(M, n, dtype=torch.bfloat16, device="cuda") for n in Ns]
+    rope = (table, seq, hd, 0b011)
+    lsq.lsq_nf4_lora_fwd_multi_ex2(qw, xg, M, Ag, Bg, r, s, None, y1, None, state, False, rope, workspace=ws)
+    lsq.lsq_nf4_lora_fwd_multi_ex2(qw, xg, M, Ag, Bg, r, s, None, y2, None, None, False, rope, workspace=ws)
+    torch.cuda.synchronize()
+    X = x.double().numpy()
+    rng = np.random.default_rng(11)
+    for i, (W, n) in enumerate(zip(Ws, Ns)):
+        assert torch.equal(y1[i], y2[i])
+        heads = np.sort(rng.choice(n // hd, min(4, n // hd), replace=False))
+        cols = np.concatenate([np.arange(h * hd, (h + 1) * hd) for h in heads])
+        wd = W[cols].float().numpy()
+        packed, am = ON.quantize(wd)
+        Wd = ON.dequantize_f64(packed, am, wd.shape[0], K)
+        A, B = As[i].double().numpy(), Bs[i].double().numpy()
+        ref = X @ Wd.T + s * (X @ A.T) @ B[cols].T                  # [M, heads * hd]
+        if i < 2:
+            t = torch.from_numpy(ref).reshape(M // seq, seq, len(heads), hd)
+            ref = OD.rope(t, theta).reshape(M, -1).numpy()
+        assert_close(y1[i].float().cpu().numpy()[:, cols], ref, what=f"rope seg {i}")

@@ -6,7 +6,9 @@
   double-quantised absmax;
 * a store file shorter than the records it must hold is refused at creation;
 * an untied embedding gathered straight from page-locked host RAM (zero-copy)
-  trains bit-identically to one held in HBM.
+  trains bit-identically to one held in HBM;
+* the lm_head in page-locked host RAM, streamed in vocabulary chunks through
+  two HBM buffers, trains bit-identically to the resident head.
 """
 import pytest
 import torch
@@ -103,3 +105,39 @@ def test_host_embedding_equals_hbm_bitwise(lsq):
     assert al == bl and torch.equal(ag, bg)
     with pytest.raises(ValueError):
         StreamedLoraTrainer(S.TINY, 1, 64, n_slots=2, init="device", embed="host")   # tied: lm_head needs it
+
+
+@pytest.mark.parametrize("shape,B,Sq", [(S.TINY_UNTIED, 2, 128), (S.TINY, 2, 96)])
+def test_streamed_head_equals_resident_bitwise(lsq, shape, B, Sq):
+    """The lm_head in page-locked host RAM, streamed in vocabulary chunks (256
+    rows: 4 chunks with a ragged last one of 232 rows for the untied 1000-row
+    head, 2 for the tied 512-row table, which then also serves the gather),
+    trains bit-identically to the resident head: logits, loss curve,
+    gradients; also the DPO step, which runs the head three times."""
+    from nf4_layer_streamed_blockwise_b200.trainer import StreamedLoraTrainer
+    steps = 3
+    a = StreamedLoraTrainer(shape, B, Sq, n_slots=2, init="device")
+    al, ag = _run(a, shape, B, Sq, steps)
+    alog = a.logits.clone()
+    a.set_ids(S.tokens(shape, B, Sq, step=9).cuda())
+    a.forward_backward_dpo(0.1)
+    adpo = (a.loss_dev.clone(), a.lora.grad.clone())
+    a.close()
+    b = StreamedLoraTrainer(shape, B, Sq, n_slots=2, init="device", head="host", head_chunk=256)
+    assert not b.lm_head.is_cuda and b.lm_head.is_pinned()
+    assert b.embed.is_cuda != shape.tied
+    bl, bg = _run(b, shape, B, Sq, steps)
+    blog = b.logits.clone()
+    b.set_ids(S.tokens(shape, B, Sq, step=9).cuda())
+    b.forward_backward_dpo(0.1)
+    bdpo = (b.loss_dev.clone(), b.lora.grad.clone())
+    uploads, nbytes, _ = b.head_stats()
+    b.close()
+    n_chunks = -(-shape.vocab // 256)
+    # every pass over the head walks its chunks in order; more chunks than the two buffers means
+    # each pass uploads all of them (2 per training step, 3 for the DPO step), else they stay
+    passes = 2 * steps + 3
+    assert uploads == (passes * n_chunks if n_chunks > 2 else n_chunks), uploads
+    assert nbytes == uploads * 256 * shape.d * 2
+    assert al == bl and torch.equal(ag, bg) and torch.equal(alog, blog)
+    assert torch.equal(adpo[0], bdpo[0]) and torch.equal(adpo[1], bdpo[1])
