@@ -202,7 +202,7 @@ struct PCfg {
   static constexpr int OFF_W = OFF_A + NST * A_STAGE;
   static constexpr int OFF_C = OFF_W + NST * W_BYTES;
   static constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
-  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1;
+  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1 + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = OFF_MISC + 128 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -299,6 +299,53 @@ __device__ __forceinline__ void tile_at(const Params& p, int t, int& m0, int& sg
   }
 }
 
+// Bulk copies of stream-K unit u (32-column chunk u / G of the tile's valid chunks, partials
+// 4 (u % G) .. of the P contributors whose first partial is part0) into stage buffer u % 2
+__device__ __forceinline__ void sk_issue(uint8_t* stage, uint64_t* sbar, const float* part0, int u, int G, int P,
+                                         int cvalid) {
+  constexpr int PART_F = 2 * (BT / 32) * 128 * 32;  // one CTA's partial with 512-row tiles
+  const int k = u / G, g = u % G;
+  const int hc = (k / cvalid) * (BT / 32) + k % cvalid;
+  const int n = min(4, P - 4 * g);
+  mbar_arrive_expect_tx(&sbar[u & 1], (uint32_t)n * 16384u);
+  for (int i = 0; i < n; ++i)
+    bulk_g2s(stage + (u & 1) * 65536 + i * 16384, part0 + (int64_t)(4 * g + i) * 2 * PART_F + (int64_t)hc * 4096,
+             16384u, &sbar[u & 1]);
+}
+
+// bf16 output of 32 columns (chunk c) of row m of a tile whose first column is n0, with the residual (FWD)
+template <int MODE>
+__device__ __forceinline__ void store_chunk(const Params& p, int sg, int n0, int ncols, int m, int c, float (&v)[32]) {
+  if (m >= p.M) return;
+#pragma unroll
+  for (int gq = 0; gq < 4; ++gq) {
+    const int col = n0 + c * 32 + gq * 8;
+    if (col >= ncols) continue;
+    float* x = v + gq * 8;
+    if (MODE == FWD) {
+      const Seg& S = p.seg[sg];
+      const int64_t off = (int64_t)m * S.n + col;
+      if (S.res) {
+        const uint4 rv = *reinterpret_cast<const uint4*>(S.res + off);
+        x[0] += bf16lo(rv.x);
+        x[1] += bf16hi(rv.x);
+        x[2] += bf16lo(rv.y);
+        x[3] += bf16hi(rv.y);
+        x[4] += bf16lo(rv.z);
+        x[5] += bf16hi(rv.z);
+        x[6] += bf16lo(rv.w);
+        x[7] += bf16hi(rv.w);
+      }
+      *reinterpret_cast<uint4*>(S.y + off) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                                        pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+    } else {
+      *reinterpret_cast<uint4*>(p.dx + (int64_t)m * p.K + col) =
+          make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                     pack_bf16x2(x[6], x[7]));
+    }
+  }
+}
+
 template <int MODE, int H>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     nf4_pair_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
@@ -312,6 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   uint64_t* tfull = cfull + NST;
   uint64_t* tempty = tfull + NBUF;
   uint64_t* drain = tempty + NBUF;
+  uint64_t* sbar = drain + 1;  // [2]: stream-K partials pulled into the idle stages (finisher's last piece)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
 
   const uint32_t rank = cluster_ctarank();
@@ -329,6 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&tempty[b], 2);  // one epilogue arrival per CTA
     }
     mbar_init(drain, 1);
+    mbar_init(&sbar[0], 1);
+    mbar_init(&sbar[1], 1);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -608,83 +658,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      // 16 columns (piece 0 or 1 of chunk hcc) of this tile's accumulator plus the partials of
-      // the clusters before this one, added in the same order as the 32-column path below
-      auto acc16 = [&](int hcc, int piece, float (&v)[16]) {
-        const int hh = hcc / (BT / 32), cc = hcc % (BT / 32);
-        tmem_ld16(tmem + lane_base + (uint32_t)((buf * H + hh) * BT + cc * 32 + piece * 16), v);
+      // 16 columns (piece 0 or 1) of two chunks hca, hcb of this tile's accumulator plus the
+      // partials of the clusters before this one, added in the same order as the 32-column path
+      // below; the two chunks' loads are issued together
+      auto acc16x2 = [&](int hca, int hcb, int piece, float (&va)[16], float (&vb)[16]) {
+        tmem_ld16(tmem + lane_base + (uint32_t)((buf * H + hca / (BT / 32)) * BT + (hca % (BT / 32)) * 32 + piece * 16),
+                  va);
+        tmem_ld16(tmem + lane_base + (uint32_t)((buf * H + hcb / (BT / 32)) * BT + (hcb % (BT / 32)) * 32 + piece * 16),
+                  vb);
         if (cfirst == cid) {
           tc_wait_ld();
           return;
         }
-        const float4* src0 = reinterpret_cast<const float4*>(p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS) +
-                             ((int64_t)hcc * 8 + piece * 4) * 128 + e;
-        float4 a[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) a[q] = __ldcg(src0 + q * 128);
-        tc_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          v[4 * q] += a[q].x;
-          v[4 * q + 1] += a[q].y;
-          v[4 * q + 2] += a[q].z;
-          v[4 * q + 3] += a[q].w;
-        }
-        for (int c2 = cfirst + 1; c2 < cid; ++c2) {
-          if (sk_bound(p, c2 + 1, ncl) == sk_bound(p, c2, ncl)) continue;
-          const float4* src = reinterpret_cast<const float4*>(p.part + (int64_t)(c2 * 2 + (int)rank) * PART_FLOATS) +
-                              ((int64_t)hcc * 8 + piece * 4) * 128 + e;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) a[q] = __ldcg(src + q * 128);
+        bool first = true;
+        for (int c2 = cfirst; c2 < cid; ++c2) {
+          if (c2 > cfirst && sk_bound(p, c2 + 1, ncl) == sk_bound(p, c2, ncl)) continue;
+          const float4* base = reinterpret_cast<const float4*>(p.part + (int64_t)(c2 * 2 + (int)rank) * PART_FLOATS);
+          const float4* sa = base + ((int64_t)hca * 8 + piece * 4) * 128 + e;
+          const float4* sb = base + ((int64_t)hcb * 8 + piece * 4) * 128 + e;
+          float4 a[4], b[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            v[4 * q] += a[q].x;
-            v[4 * q + 1] += a[q].y;
-            v[4 * q + 2] += a[q].z;
-            v[4 * q + 3] += a[q].w;
+            a[q] = __ldcg(sa + q * 128);
+            b[q] = __ldcg(sb + q * 128);
+          }
+          if (first) tc_wait_ld();
+          first = false;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            va[4 * q] += a[q].x;
+            va[4 * q + 1] += a[q].y;
+            va[4 * q + 2] += a[q].z;
+            va[4 * q + 3] += a[q].w;
+            vb[4 * q] += b[q].x;
+            vb[4 * q + 1] += b[q].y;
+            vb[4 * q + 2] += b[q].z;
+            vb[4 * q + 3] += b[q].w;
           }
         }
       };
       const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
       if (MODE == FWD && p.seg[sg].rope) {
         // RoPE in the epilogue: column i of a head pairs with column i + hd/2, which sits hd/64
-        // chunks of 32 further on in the same accumulator; each pair of chunks is rotated in
-        // fp32 (the accumulator plus earlier clusters' partials, as below) and rounded once
-        const int hc32 = p.rope_hd / 32, half = p.rope_hd / 2;
-        for (int hc = 0; hc < H * (BT / 32); ++hc) {
-          const int h = hc / (BT / 32), c = hc % (BT / 32);
-          if (c % hc32 >= hc32 / 2 || n0 + c * 32 >= ncols) continue;
-          const int m = m0 + h * BT + (int)rank * BMC + e;
-#pragma unroll 1
-          for (int piece = 0; piece < 2; ++piece) {
-            float x1[16], x2[16];
-            acc16(hc, piece, x1);
-            acc16(hc + hc32 / 2, piece, x2);
-            if (m >= p.M) continue;
-            const int i0 = (c % hc32) * 32 + piece * 16;  // frequency index of x1[0]
-            const float4* cs = reinterpret_cast<const float4*>(p.rope + (int64_t)(m % p.rope_seq) * half + i0);
+        // chunks of 32 further on in the same accumulator; both are rotated in fp32 (the
+        // accumulator plus earlier clusters' partials) and rounded once.  The loop takes 16
+        // frequencies at a time for every head of the tile in turn, so the row's (cos, sin) of
+        // those frequencies come from the L1 cache after the first head.
+        const int hc32 = p.rope_hd / 32, half = p.rope_hd / 2, heads = BT / p.rope_hd;
+        for (int fb = 0; fb < half / 16; ++fb) {
+          const int cl = fb / 2, piece = fb % 2;
+          for (int h = 0; h < H; ++h) {
+            const int m = m0 + h * BT + (int)rank * BMC + e;
+            const float4* cs = reinterpret_cast<const float4*>(p.rope + (int64_t)(m % p.rope_seq) * half + fb * 16);
+            for (int hh = 0; hh < heads; ++hh) {
+              const int c = hh * hc32 + cl;
+              if (n0 + c * 32 >= ncols) continue;
+              float x1[16], x2[16];
+              acc16x2(h * (BT / 32) + c, h * (BT / 32) + c + hc32 / 2, piece, x1, x2);
+              if (m >= p.M) continue;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 t = __ldg(cs + q);  // (cos, sin) of frequencies i0 + 2q, i0 + 2q + 1
-              const float a0 = x1[2 * q], a1 = x1[2 * q + 1], b0 = x2[2 * q], b1 = x2[2 * q + 1];
-              x1[2 * q] = a0 * t.x - b0 * t.y;
-              x2[2 * q] = b0 * t.x + a0 * t.y;
-              x1[2 * q + 1] = a1 * t.z - b1 * t.w;
-              x2[2 * q + 1] = b1 * t.z + a1 * t.w;
-            }
-            const Seg& S = p.seg[sg];
-            __nv_bfloat16* y1 = S.y + (int64_t)m * S.n + n0 + c * 32 + piece * 16;
-            __nv_bfloat16* y2 = y1 + half;
+              for (int q = 0; q < 8; ++q) {
+                const float4 t = __ldg(cs + q);  // (cos, sin) of frequencies 2q, 2q + 1 of the block
+                const float a0 = x1[2 * q], a1 = x1[2 * q + 1], b0 = x2[2 * q], b1 = x2[2 * q + 1];
+                x1[2 * q] = a0 * t.x - b0 * t.y;
+                x2[2 * q] = b0 * t.x + a0 * t.y;
+                x1[2 * q + 1] = a1 * t.z - b1 * t.w;
+                x2[2 * q + 1] = b1 * t.z + a1 * t.w;
+              }
+              const Seg& S = p.seg[sg];
+              __nv_bfloat16* y1 = S.y + (int64_t)m * S.n + n0 + c * 32 + piece * 16;
+              __nv_bfloat16* y2 = y1 + half;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              *reinterpret_cast<uint4*>(y1 + 8 * u) =
-                  make_uint4(pack_bf16x2(x1[8 * u], x1[8 * u + 1]), pack_bf16x2(x1[8 * u + 2], x1[8 * u + 3]),
-                             pack_bf16x2(x1[8 * u + 4], x1[8 * u + 5]), pack_bf16x2(x1[8 * u + 6], x1[8 * u + 7]));
-              *reinterpret_cast<uint4*>(y2 + 8 * u) =
-                  make_uint4(pack_bf16x2(x2[8 * u], x2[8 * u + 1]), pack_bf16x2(x2[8 * u + 2], x2[8 * u + 3]),
-                             pack_bf16x2(x2[8 * u + 4], x2[8 * u + 5]), pack_bf16x2(x2[8 * u + 6], x2[8 * u + 7]));
+              for (int u = 0; u < 2; ++u) {
+                *reinterpret_cast<uint4*>(y1 + 8 * u) =
+                    make_uint4(pack_bf16x2(x1[8 * u], x1[8 * u + 1]), pack_bf16x2(x1[8 * u + 2], x1[8 * u + 3]),
+                               pack_bf16x2(x1[8 * u + 4], x1[8 * u + 5]), pack_bf16x2(x1[8 * u + 6], x1[8 * u + 7]));
+                *reinterpret_cast<uint4*>(y2 + 8 * u) =
+                    make_uint4(pack_bf16x2(x2[8 * u], x2[8 * u + 1]), pack_bf16x2(x2[8 * u + 2], x2[8 * u + 3]),
+                               pack_bf16x2(x2[8 * u + 4], x2[8 * u + 5]), pack_bf16x2(x2[8 * u + 6], x2[8 * u + 7]));
+              }
             }
           }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+        continue;
+      }
+      // A finisher that adds partials on its last piece (stream-K, 512-row tiles) pulls them into
+      // its idle activation stages with bulk copies: per 32-column chunk up to 4 partials of 16 KB
+      // per round, two rounds in flight, instead of one round trip per partial per chunk.  The
+      // partials are added in the same order as below, so the two paths agree bit for bit.
+      bool bulk = false;
+      if constexpr (H == 2) {
+        int tn, k0n, k1n;
+        bulk = cfirst < cid && cid - cfirst <= 16 && !piece_at(p, cid, ncl, j + 1, tn, k0n, k1n);
+        for (int c2 = cfirst; bulk && c2 < cid; ++c2) bulk = sk_bound(p, c2 + 1, ncl) > sk_bound(p, c2, ncl);
+      }
+      if (bulk) {
+        const int P = cid - cfirst, G = (P + 3) / 4;
+        const int cvalid = min(BT / 32, (ncols - n0 + 31) / 32);
+        const int nunits = H * cvalid * G;
+        uint8_t* stage = smem + C::OFF_A;  // 2 x 4 x 16 KB = the activation stages, idle now
+        const float* part0 = p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS;
+        if (e == 0) {
+          fence_proxy_async_all();  // the partials were published to this thread's acquires above
+          sk_issue(stage, sbar, part0, 0, G, P, cvalid);
+        }
+        bool okb = true;  // false once a wait ran out: every thread still passes every barrier, nothing is stored
+        int u = 0;
+        for (int k = 0; k < H * cvalid; ++k) {
+          const int h = k / cvalid, c = k % cvalid;
+          float v[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
+          for (int g = 0; g < G; ++g, ++u) {
+            if (e == 0 && u + 1 < nunits && okb) sk_issue(stage, sbar, part0, u + 1, G, P, cvalid);
+            okb = okb && mbar_wait(&sbar[u & 1], (uint32_t)(u >> 1) & 1u, 736);
+            if (g == 0) tc_wait_ld();
+            if (okb) {
+              const float4* sb = reinterpret_cast<const float4*>(stage + (u & 1) * 65536) + e;
+              const int n = min(4, P - 4 * g);
+              for (int i = 0; i < n; ++i) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float4 a = sb[i * 1024 + q * 128];
+                  v[4 * q] += a.x;
+                  v[4 * q + 1] += a.y;
+                  v[4 * q + 2] += a.z;
+                  v[4 * q + 3] += a.w;
+                }
+              }
+            }
+            named_bar_sync(1, 128);  // buffer u & 1 is read: unit u + 2 may refill it
+          }
+          if (okb) store_chunk<MODE>(p, sg, n0, ncols, m0 + h * BT + (int)rank * BMC + e, c, v);
         }
         tc_fence_before();
         named_bar_sync(1, 128);
@@ -729,34 +836,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        if (m >= p.M) continue;
-#pragma unroll
-        for (int gq = 0; gq < 4; ++gq) {
-          const int col = n0 + c * 32 + gq * 8;
-          if (col >= ncols) continue;
-          float* x = v + gq * 8;
-          if (MODE == FWD) {
-            const Seg& S = p.seg[sg];
-            const int64_t off = (int64_t)m * S.n + col;
-            if (S.res) {
-              const uint4 rv = *reinterpret_cast<const uint4*>(S.res + off);
-              x[0] += bf16lo(rv.x);
-              x[1] += bf16hi(rv.x);
-              x[2] += bf16lo(rv.y);
-              x[3] += bf16hi(rv.y);
-              x[4] += bf16lo(rv.z);
-              x[5] += bf16hi(rv.z);
-              x[6] += bf16lo(rv.w);
-              x[7] += bf16hi(rv.w);
-            }
-            *reinterpret_cast<uint4*>(S.y + off) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                                              pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-          } else {
-            *reinterpret_cast<uint4*>(p.dx + (int64_t)m * p.K + col) =
-                make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                           pack_bf16x2(x[6], x[7]));
-          }
-        }
+        store_chunk<MODE>(p, sg, n0, ncols, m, c, v);
       }
       tc_fence_before();
       named_bar_sync(1, 128);
@@ -1151,7 +1231,48 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
   const bool sk_can = !force && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 &&
                       (tiles2 - dp) * p.nkb >= 4 * (int64_t)ncl_max;
   const bool sk_pays = 2 * tiles2 >= ncl_max && rounds_sk < 0.97 * rounds_whole;
+  static const bool plan_log = getenv("LSQ_NF4_PLAN_LOG") != nullptr;   // prints each call's tile plan
+  // Few tiles (under half a round of 512-row tiles, e.g. 512 tokens): let S clusters share each
+  // tile (ncl = tiles x S, so each finisher adds at most about S partials).  Cost model in us,
+  // from the B200 launch lists: about 8 of fixed cost per launch, 1.0 per 64-wide weight block
+  // of a 512-row tile (0.73 for a 256-row one), and about 10 per partial the finisher adds
+  // (its four epilogue warps read them with one round trip per 32-column chunk each).
+  if (!force && skmode != 0 && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 &&
+      2 * tiles2 < ncl_max) {
+    const int64_t tiles1 = (int64_t)((p.M + BT - 1) / BT) * ntiles_n;
+    const double whole1 = 8.0 + (double)((tiles1 + ncl_max - 1) / ncl_max) * p.nkb * 0.73;
+    const double whole2 = 8.0 + (double)((tiles2 + ncl_max - 1) / ncl_max) * p.nkb * 1.0;
+    const double whole = std::min(whole1, whole2);
+    int sbest = 1;
+    double cbest = whole;
+    const char* splitenv = getenv("LSQ_NF4_SK_SPLIT");   // forces S (a tuning override)
+    for (int S = 2; S * tiles2 <= ncl_max; ++S) {
+      if (tiles2 * p.nkb < 4 * (int64_t)S * tiles2) break;  // at least 4 blocks per cluster
+      const double c = 8.0 + (double)p.nkb / S + 10.0 * (S - 1);
+      if (splitenv ? S == atoi(splitenv) : c < 0.85 * cbest) {
+        cbest = c;
+        sbest = S;
+      }
+    }
+    if (sbest > 1) {
+      const int ncl_s = (int)(tiles2 * sbest);
+      if (plan_log)
+        fprintf(stderr, "nf4 plan: mode %d M %d tiles %lld (512 rows) nkb %d: stream-K over %d clusters (%d per "
+                "tile)\n", MODE, p.M, (long long)tiles2, p.nkb, ncl_s, sbest);
+      p.streamk = 1;
+      p.dp_tiles = 0;
+      p.flags = reinterpret_cast<unsigned long long*>(sk_ws);
+      p.part = reinterpret_cast<float*>(sk_ws + 4096);
+      p.epoch = next_epoch();
+      p.mtiles = (p.M + 2 * BT - 1) / (2 * BT);
+      p.tiles = p.mtiles * ntiles_n;
+      return launch_pair_h<MODE, 2>(maps, p, ncl_s, stream);
+    }
+  }
   if (sk_can && skmode != 0 && (skmode == 1 || sk_pays)) {
+    if (plan_log)
+      fprintf(stderr, "nf4 plan: mode %d M %d tiles %lld (512 rows) nkb %d: stream-K, %lld whole tiles\n", MODE, p.M,
+              (long long)tiles2, p.nkb, (long long)dp);
     p.streamk = 1;
     p.dp_tiles = (int)dp;  // whole tiles for all but the last one or two rounds' worth
     p.flags = reinterpret_cast<unsigned long long*>(sk_ws);
@@ -1180,6 +1301,9 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
   p.mtiles = (p.M + BT * hbest - 1) / (BT * hbest);
   p.tiles = p.mtiles * ntiles_n;
   const int ncl = std::min(p.tiles, ncl_max);
+  if (plan_log)
+    fprintf(stderr, "nf4 plan: mode %d M %d tiles %d (%d rows) nkb %d: whole tiles on %d clusters%s\n", MODE, p.M,
+            p.tiles, 256 * hbest, p.nkb, ncl, sk_can ? "" : " (no stream-K: not possible)");
   return hbest == 2 ? launch_pair_h<MODE, 2>(maps, p, ncl, stream) : launch_pair_h<MODE, 1>(maps, p, ncl, stream);
 }
 
