@@ -32,12 +32,14 @@ constexpr int BC = 128;          // keys per chunk
 constexpr int MAXC = 4;          // chunks: sequences of at most 512
 constexpr int TILE = BQ * D * 2; // 128 x 128 bf16 tile: two 64-column 128B-swizzled halves of 16 KB
 constexpr int HALF = TILE / 2;
+constexpr int FRING = 4;          // forward K / V ring: every key chunk of a tile loads at once
+constexpr int FPB = 2;            // forward P buffers, reused every other chunk
 constexpr int OFF_Q = 0;          // Q; once the score products are done, the row statistics
 constexpr int OFF_RING = OFF_Q + TILE;
-constexpr int OFF_P = OFF_RING + 2 * TILE;
-constexpr int OFF_BAR = OFF_P + MAXC * TILE;
-// qfull, rfull[2], rempty[2], sfull, pready[4], ofull, mxbar, smbar
-constexpr int NBAR = 1 + 2 + 2 + 1 + MAXC + 1 + 2;
+constexpr int OFF_P = OFF_RING + FRING * TILE;
+constexpr int OFF_BAR = OFF_P + FPB * TILE;
+// qfull, rfull[4], rempty[4], sfull, pready[4], ofull, mxbar, smbar, pfree[2]
+constexpr int NBAR = 1 + FRING + FRING + 1 + MAXC + 1 + 2 + FPB;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -78,12 +80,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* rfull = qfull + 1;
-  uint64_t* rempty = rfull + 2;
-  uint64_t* sfull = rempty + 2;
+  uint64_t* rempty = rfull + FRING;
+  uint64_t* sfull = rempty + FRING;
   uint64_t* pready = sfull + 1;
   uint64_t* ofull = pready + MAXC;
   uint64_t* mxbar = ofull + 1;
   uint64_t* smbar = mxbar + 1;
+  uint64_t* pfree = smbar + 1;  // [FPB]: the P V product of the buffer's previous chunk is done
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int nt = (S + BQ - 1) / BQ;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < FRING; ++i) {
       mbar_init(&rfull[i], 1);
       mbar_init(&rempty[i], 1);
     }
@@ -107,6 +110,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
     mbar_init(ofull, 1);
     mbar_init(mxbar, EW);
     mbar_init(smbar, EW);
+    for (int i = 0; i < FPB; ++i) mbar_init(&pfree[i], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -125,8 +129,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
       tma_load_2d(smem + OFF_Q, &qmap, qfull, h * D, row0 + q0);
       tma_load_2d(smem + OFF_Q + HALF, &qmap, qfull, h * D + 64, row0 + q0);
       for (int it = 0; it < 2 * nc; ++it) {  // K chunks 0..nc-1, then V chunks 0..nc-1
-        const int slot = it & 1;
-        const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+        const int slot = it % FRING;
+        const uint32_t ph = (uint32_t)(it / FRING) & 1u;
         if (!mbar_wait(&rempty[slot], ph ^ 1u, 461)) break;
         const int j = it < nc ? it : it - nc;
         const CUtensorMap* m = it < nc ? &kmap : &vmap;
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
       const uint32_t id_s = idesc_bf16(BQ, BC, 0, 0);  // Q K^T: both K-major
       const uint32_t id_o = idesc_bf16(BQ, D, 0, 1);   // P V: P K-major, V MN-major
       for (int j = 0; ok && j < nc; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&rfull[slot], (uint32_t)(j >> 1) & 1u, 562)) {
+        const int slot = j % FRING;
+        if (!mbar_wait(&rfull[slot], (uint32_t)(j / FRING) & 1u, 562)) {
           ok = false;
           break;
         }
@@ -158,18 +162,19 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
       }
       if (ok) tc_commit(sfull);
       for (int j = 0; ok && j < nc; ++j) {
-        const int it = nc + j, slot = it & 1;
-        if (!mbar_wait(&rfull[slot], (uint32_t)(it >> 1) & 1u, 563) || !mbar_wait(&pready[j], 0, 564)) {
+        const int it = nc + j, slot = it % FRING;
+        if (!mbar_wait(&rfull[slot], (uint32_t)(it / FRING) & 1u, 563) || !mbar_wait(&pready[j], 0, 564)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t pb = smem_u32(smem + OFF_P + j * TILE);
+        const uint32_t pb = smem_u32(smem + OFF_P + (j % FPB) * TILE);
         const uint32_t vb = smem_u32(smem + OFF_RING + slot * TILE);
 #pragma unroll
         for (int kk = 0; kk < BC / 16; ++kk)
           tc_mma(tmem, desc_kmajor(pb, kk), smem_desc(vb + kk * 2048, HALF, 1024, 2), id_o, (j | kk) != 0);
         tc_commit(&rempty[slot]);
+        tc_commit(&pfree[j % FPB]);  // P buffer j % FPB may take chunk j + FPB
       }
       tc_commit(ofull);  // also drains what was issued if a wait gave up
       if (!ok) mbar_wait(ofull, 0, 565);
@@ -231,8 +236,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
             w[e / 2] = pack_bf16x2(p0, p1);
           }
         }
+        // P buffer j % FPB held chunk j - FPB until its P V product completed
+        if (j >= FPB && !__all_sync(0xffffffffu, mbar_wait(&pfree[j % FPB], (uint32_t)((j - FPB) / FPB) & 1u, 766))) {
+          ok = false;
+          break;
+        }
         // keys part*32 .. +31 of this chunk: half part >> 1, 16-byte units (part & 1) * 4 .. + 3
-        const uint32_t hbase = smem_u32(smem + OFF_P + j * TILE) + r * 128 + (uint32_t)(part >> 1) * HALF;
+        const uint32_t hbase = smem_u32(smem + OFF_P + (j % FPB) * TILE) + r * 128 + (uint32_t)(part >> 1) * HALF;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int unit = (part & 1) * 4 + u;
@@ -247,7 +257,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
       s_sum[part * BQ + r] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(smbar);
-      ok = __all_sync(0xffffffffu, mbar_wait(smbar, 0, 763)) && __all_sync(0xffffffffu, mbar_wait(ofull, 0, 764));
+      ok = __all_sync(0xffffffffu, mbar_wait(smbar, 0, 763)) && __all_sync(0xffffffffu, mbar_wait(ofull, 0, 764)) &&
+           ok;
     }
     if (ok) {
       tc_fence_after();

@@ -610,6 +610,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tile_at<MODE, H>(p, t, m0, sg, n0);
       const int buf = j % NBUF;
       const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
+      if (MODE == FWD && p.seg[sg].rope && k1 == p.nkb) {
+        // the rows' RoPE angles into L1 while the tile's MMAs finish
+        const int half = p.rope_hd / 2;
+        for (int h = 0; h < H; ++h) {
+          const int m = m0 + h * BT + (int)rank * BMC + e;
+          if (m >= p.M) continue;
+          const char* row = reinterpret_cast<const char*>(p.rope + (int64_t)(m % p.rope_seq) * half);
+          for (int b = 0; b < half * 8; b += 128) asm volatile("prefetch.global.L1 [%0];" ::"l"(row + b));
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
       tc_fence_after();
       if (k1 < p.nkb) {
@@ -698,7 +708,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       };
       const int ncols = (MODE == FWD) ? p.seg[sg].n : p.K;
-      if (MODE == FWD && p.seg[sg].rope) {
+      // A finisher that adds partials on its last piece (stream-K, 512-row tiles) pulls them into
+      // its idle activation stages with bulk copies: per 32-column chunk up to 4 partials of 16 KB
+      // per round, two rounds in flight, instead of one round trip per partial per chunk.  The
+      // partials are added in the same order as below, so the two paths agree bit for bit.
+      bool bulk = false;
+      if constexpr (H == 2) {
+        int tn, k0n, k1n;
+        bulk = cfirst < cid && cid - cfirst <= 16 && !piece_at(p, cid, ncl, j + 1, tn, k0n, k1n);
+        for (int c2 = cfirst; bulk && c2 < cid; ++c2) bulk = sk_bound(p, c2 + 1, ncl) > sk_bound(p, c2, ncl);
+      }
+      const bool rope_seg = MODE == FWD && p.seg[sg].rope;
+      if (bulk) {
+        const int P = cid - cfirst, G = (P + 3) / 4;
+        const int cvalid = min(BT / 32, (ncols - n0 + 31) / 32);
+        const int nunits = H * cvalid * G;
+        uint8_t* stage = smem + C::OFF_A;  // 2 x 4 x 16 KB = the activation stages, idle now
+        const float* part0 = p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS;
+        if (e == 0) {
+          fence_proxy_async_all();  // the partials were published to this thread's acquires above
+          sk_issue(stage, sbar, part0, 0, G, P, cvalid);
+        }
+        bool okb = true;  // false once a wait ran out: every thread still passes every barrier, nothing is stored
+        int u = 0;
+        for (int k = 0; k < H * cvalid; ++k) {
+          const int h = k / cvalid, c = k % cvalid;
+          float v[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
+          for (int g = 0; g < G; ++g, ++u) {
+            if (e == 0 && u + 1 < nunits && okb) sk_issue(stage, sbar, part0, u + 1, G, P, cvalid);
+            okb = okb && mbar_wait(&sbar[u & 1], (uint32_t)(u >> 1) & 1u, 736);
+            if (g == 0) tc_wait_ld();
+            if (okb) {
+              const float4* sb = reinterpret_cast<const float4*>(stage + (u & 1) * 65536) + e;
+              const int n = min(4, P - 4 * g);
+              for (int i = 0; i < n; ++i) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float4 a = sb[i * 1024 + q * 128];
+                  v[4 * q] += a.x;
+                  v[4 * q + 1] += a.y;
+                  v[4 * q + 2] += a.z;
+                  v[4 * q + 3] += a.w;
+                }
+              }
+            }
+            named_bar_sync(1, 128);  // buffer u & 1 is read: unit u + 2 may refill it
+          }
+          if (!okb) continue;
+          if (rope_seg)  // the sum goes back into the accumulator for the RoPE epilogue below
+            tmem_st32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
+          else
+            store_chunk<MODE>(p, sg, n0, ncols, m0 + h * BT + (int)rank * BMC + e, c, v);
+        }
+        if (rope_seg) {
+          tc_wait_st();
+          cfirst = cid;  // the accumulator holds the tile's whole sum now
+        } else {
+          tc_fence_before();
+          named_bar_sync(1, 128);
+          if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+          continue;
+        }
+      }
+      if (rope_seg) {
         // RoPE in the epilogue: column i of a head pairs with column i + hd/2, which sits hd/64
         // chunks of 32 further on in the same accumulator; both are rotated in fp32 (the
         // accumulator plus earlier clusters' partials) and rounded once.  The loop takes 16
@@ -739,59 +812,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               }
             }
           }
-        }
-        tc_fence_before();
-        named_bar_sync(1, 128);
-        if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
-        continue;
-      }
-      // A finisher that adds partials on its last piece (stream-K, 512-row tiles) pulls them into
-      // its idle activation stages with bulk copies: per 32-column chunk up to 4 partials of 16 KB
-      // per round, two rounds in flight, instead of one round trip per partial per chunk.  The
-      // partials are added in the same order as below, so the two paths agree bit for bit.
-      bool bulk = false;
-      if constexpr (H == 2) {
-        int tn, k0n, k1n;
-        bulk = cfirst < cid && cid - cfirst <= 16 && !piece_at(p, cid, ncl, j + 1, tn, k0n, k1n);
-        for (int c2 = cfirst; bulk && c2 < cid; ++c2) bulk = sk_bound(p, c2 + 1, ncl) > sk_bound(p, c2, ncl);
-      }
-      if (bulk) {
-        const int P = cid - cfirst, G = (P + 3) / 4;
-        const int cvalid = min(BT / 32, (ncols - n0 + 31) / 32);
-        const int nunits = H * cvalid * G;
-        uint8_t* stage = smem + C::OFF_A;  // 2 x 4 x 16 KB = the activation stages, idle now
-        const float* part0 = p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS;
-        if (e == 0) {
-          fence_proxy_async_all();  // the partials were published to this thread's acquires above
-          sk_issue(stage, sbar, part0, 0, G, P, cvalid);
-        }
-        bool okb = true;  // false once a wait ran out: every thread still passes every barrier, nothing is stored
-        int u = 0;
-        for (int k = 0; k < H * cvalid; ++k) {
-          const int h = k / cvalid, c = k % cvalid;
-          float v[32];
-          tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
-          for (int g = 0; g < G; ++g, ++u) {
-            if (e == 0 && u + 1 < nunits && okb) sk_issue(stage, sbar, part0, u + 1, G, P, cvalid);
-            okb = okb && mbar_wait(&sbar[u & 1], (uint32_t)(u >> 1) & 1u, 736);
-            if (g == 0) tc_wait_ld();
-            if (okb) {
-              const float4* sb = reinterpret_cast<const float4*>(stage + (u & 1) * 65536) + e;
-              const int n = min(4, P - 4 * g);
-              for (int i = 0; i < n; ++i) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  const float4 a = sb[i * 1024 + q * 128];
-                  v[4 * q] += a.x;
-                  v[4 * q + 1] += a.y;
-                  v[4 * q + 2] += a.z;
-                  v[4 * q + 3] += a.w;
-                }
-              }
-            }
-            named_bar_sync(1, 128);  // buffer u & 1 is read: unit u + 2 may refill it
-          }
-          if (okb) store_chunk<MODE>(p, sg, n0, ncols, m0 + h * BT + (int)rank * BMC + e, c, v);
         }
         tc_fence_before();
         named_bar_sync(1, 128);
@@ -1234,10 +1254,12 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
   static const bool plan_log = getenv("LSQ_NF4_PLAN_LOG") != nullptr;   // prints each call's tile plan
   // Few tiles (under half a round of 512-row tiles, e.g. 512 tokens): let S clusters share each
   // tile (ncl = tiles x S, so each finisher adds at most about S partials).  Cost model in us,
-  // from the B200 launch lists: about 8 of fixed cost per launch, 1.0 per 64-wide weight block
-  // of a 512-row tile (0.73 for a 256-row one), and about 10 per partial the finisher adds
-  // (its four epilogue warps read them with one round trip per 32-column chunk each).
-  if (!force && skmode != 0 && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 8 &&
+  // from B200 microbenchmarks at the 3B shapes: about 8 of fixed cost per launch, 1.0 per
+  // 64-wide weight block of a 512-row tile (0.73 for a 256-row one), and about 5 per partial the
+  // finisher adds (bulk copies into its idle stages; 10 with one round trip per partial).
+  // Only long contractions (at least 128 weight blocks, where it was measured to pay: 1.5-2.3x at
+  // the 3B shapes' 172 and 344 blocks) take it.
+  if (!force && skmode != 0 && sk_ws && sk_bytes >= sk_region_bytes() && p.M >= 2 * BT && p.nkb >= 128 &&
       2 * tiles2 < ncl_max) {
     const int64_t tiles1 = (int64_t)((p.M + BT - 1) / BT) * ntiles_n;
     const double whole1 = 8.0 + (double)((tiles1 + ncl_max - 1) / ncl_max) * p.nkb * 0.73;
@@ -1248,7 +1270,7 @@ static lsq_status launch_pair(const Maps& maps, Params p, int ntiles_n, char* sk
     const char* splitenv = getenv("LSQ_NF4_SK_SPLIT");   // forces S (a tuning override)
     for (int S = 2; S * tiles2 <= ncl_max; ++S) {
       if (tiles2 * p.nkb < 4 * (int64_t)S * tiles2) break;  // at least 4 blocks per cluster
-      const double c = 8.0 + (double)p.nkb / S + 10.0 * (S - 1);
+      const double c = 8.0 + (double)p.nkb / S + 5.0 * (S - 1);
       if (splitenv ? S == atoi(splitenv) : c < 0.85 * cbest) {
         cbest = c;
         sbest = S;
