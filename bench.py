@@ -40,10 +40,11 @@ if ROOT not in sys.path:
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused forward
 # GEMM (nf4_pair_kernel<FWD>), the mean over the four calls of an 8B layer
-# (q/k/v, o, gate/up, down at 2048 tokens), from one ncu capture of the kernel
-# built from the sources whose SHA-256 prefix is given; the figure is reported
-# only while those sources are unchanged (else traffic is null).
-NCU_TRAFFIC = {("llama-3.1-8b", 2048): (92.8e6, None)}
+# (q/k/v with RoPE, o, gate/up, down at 2048 tokens: 52.7, 27.1, 193.8 and 92.8
+# MB), from one ncu capture of the kernel built from the sources whose SHA-256
+# prefix is given; the figure is reported only while those sources are
+# unchanged (else traffic is null).
+NCU_TRAFFIC = {("llama-3.1-8b", 2048): (91.6e6, "aa55e5d1505ab1ab")}
 TRAFFIC_SOURCES = ("nf4_layer_streamed_blockwise_b200/csrc/gemm_nf4.cu",
                    "nf4_layer_streamed_blockwise_b200/csrc/common.cuh")
 
@@ -99,6 +100,8 @@ def args_():
                    help="lm_head resident in HBM, or in page-locked host RAM streamed in vocabulary chunks of "
                         "--head-chunk rows through two HBM buffers for each of its GEMMs")
     p.add_argument("--head-chunk", type=int, default=8192)
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch every kernel eagerly instead of replaying each step as a CUDA graph")
     p.add_argument("--absmax", default="fp32", choices=["fp32", "dq8"],
                    help="absmax format of the streamed records: fp32, or double-quantised (8-bit E4M3 codes, "
                         "blocks of 256, expanded to fp32 in HBM after each upload)")
@@ -250,7 +253,16 @@ def workload_config(a, shape):
                         f"{task}, AdamW",
             "batch": a.batch, "seq_len": a.seq, "n_slots": a.slots, "parallelism": f"dp{a.gpus}",
             "upload": a.upload if a.upload != "auto" else ("sharded" if a.gpus > 1 else "replicated"),
-            "l2": f"inputs larger than L2 ({store_gb:.2f} GB of layer records streamed per pass)"}
+            "l2": f"inputs larger than L2 ({store_gb:.2f} GB of layer records streamed per pass)",
+            "launch": ("eager launches" if not graph_on(a) else
+                       "each step replayed as one CUDA graph (kernels, layer uploads, their events) after one "
+                       "eager warm-up step; the instrumented pass runs eagerly")}
+
+
+def graph_on(a):
+    """Graph replay applies to the host-RAM tier without sharded uploads (the disk tier and the
+    all-gather do host work in each step)."""
+    return not a.no_graph and a.source == "ram" and a.upload != "sharded" and not (a.upload == "auto" and a.gpus > 1)
 
 
 def record_bytes(shape, absmax="fp32"):
@@ -334,6 +346,15 @@ def timed_steps(torch, dist, tr, steps, ids_list, world, instrument=False, e2e=F
 
 
 def our_arm(a):
+    """Everything runs on one non-default stream, the trainers' compute stream (stream capture
+    cannot record the legacy default stream)."""
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    with torch.cuda.stream(torch.cuda.Stream()):
+        _our_arm(a)
+
+
+def _our_arm(a):
     import torch
     import synthetic as S
     from nf4_layer_streamed_blockwise_b200 import lib as L
@@ -360,7 +381,7 @@ def our_arm(a):
         if a.store_path and world > 1:
             store_path = f"{a.store_path}.rank{rank}"
     tiers = dict(absmax=a.absmax, shard=shard, source=a.source, store_path=store_path, embed=a.embed, head=a.head,
-                 head_chunk=a.head_chunk)
+                 head_chunk=a.head_chunk, graph=graph_on(a))
     tr = StreamedLoraTrainer(shape, a.batch, a.seq, n_slots=a.slots, init="device", **tiers)
     ids_list = [S.tokens(shape, a.batch, a.seq, step=1000 * rank + t).cuda() for t in range(4)]
     for i in range(a.warmup):
@@ -395,6 +416,15 @@ def our_arm(a):
     wait_fwd, wait_bwd, n_waits, n_dropped = L.lsq_stream_wait_ms(tr.sched)
     L.lsq_stream_time_waits(tr.sched, 0)
     tr.check_device()
+    # host time to enqueue one step on an idle GPU (the library calls of the whole step), against
+    # the step's device time: a ratio near 1 means the host, not the GPU, sets the pace
+    t0 = time.perf_counter()
+    tr.set_ids(ids_list[0])
+    step_fb(tr, a)
+    tr.optimizer_step()
+    host_ms = (time.perf_counter() - t0) * 1e3
+    torch.cuda.synchronize()
+    tr.check_device()
     kinds = {}
     for kind, flops, s0, s1 in timeline:
         d = kinds.setdefault(kind, [0.0, 0.0, 0])
@@ -413,13 +443,19 @@ def our_arm(a):
 
     # streaming: copy GB/s from the copy-stream events of the last uploads
     rec = tr.layout.nbytes
-    up_ms = [L.lsq_stream_upload_ms(tr.sched, l) for l in range(shape.n_layers)]
+    up_ms = []
+    for l in range(shape.n_layers):   # the instrumented (eager) pass uploaded each layer it streams
+        try:
+            up_ms.append(L.lsq_stream_upload_ms(tr.sched, l))
+        except L.LsqError:
+            pass
     copy_gbs = rec / (statistics.median(up_ms) * 1e-3) / 1e9
     streaming = {"record_bytes": rec, "uploads_per_step": (up1 - up0) / a.steps,
                  "exposed_copy_ms_fwd": wait_fwd / a.steps, "exposed_copy_ms_bwd": wait_bwd / a.steps,
                  "exposed_copy_frac": (wait_fwd + wait_bwd) / ms_instr,
                  "exposed_copy_waits_timed": n_waits, "exposed_copy_waits_dropped": n_dropped,
                  "ms_per_step_instrumented": ms_instr / a.steps,
+                 "host_enqueue_ms_one_step": host_ms,
                  "h2d_bytes_per_step": (by1 - by0 + hb1 - hb0) / a.steps, "reused_per_step": (re1 - re0) / a.steps,
                  "head_h2d_bytes_per_step": (hb1 - hb0) / a.steps,
                  "copy_gbs": copy_gbs, "pinned_h2d_gbs": h2d, "copy_frac_of_link": copy_gbs / h2d,
@@ -452,6 +488,12 @@ def our_arm(a):
         ms_r, _ = timed_steps(torch, dist, trr, a.steps, ids_list, world, a=a)
         trr.check_device()
         streaming["ms_per_step_resident"] = ms_r / a.steps
+        # the fused linears' device time per step, resident against streamed (same instrumentation)
+        ms_ri, tl_r = timed_steps(torch, dist, trr, a.steps, ids_list, world, instrument=True, a=a)
+        trr.check_device()
+        streaming["fused_gemm_ms_per_step_resident"] = sum(s0.elapsed_time(s1) for _, _, s0, s1 in tl_r) / a.steps
+        streaming["fused_gemm_ms_per_step_streamed"] = all_ms / a.steps
+        streaming["ms_per_step_resident_instrumented"] = ms_ri / a.steps
         streaming["streamed_minus_resident_ms"] = max(0.0, ms_step - ms_r / a.steps)
         streaming["peak_hbm_gb_resident"] = torch.cuda.max_memory_allocated() / 1e9
         trr.close()

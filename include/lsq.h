@@ -257,8 +257,12 @@ lsq_status lsq_nf4_lora_bwd_multi_ex(int32_t nseg, const lsq_nf4_weight* W, cons
  * columns; column i < hd/2 of a head pairs with column i + hd/2 and the pair
  * is rotated by the angle position * theta^(-2i/hd), in fp32 on the
  * accumulator, before the one bf16 rounding of the output.
- *  table:    (cos, sin) fp32 pairs [seq][hd/2] from lsq_rope_table (device,
- *            16-byte aligned)
+ *  table:    lsq_rope_table's output for this seq and hd (device, 16-byte
+ *            aligned); the epilogue takes the frequencies after the pairs and
+ *            forms each angle as position x frequency in fp32, its cosine and
+ *            sine with a two-part reduction by 2 pi and the special-function
+ *            unit (error about 1e-6 of the rotated value, against 2^-8 for the
+ *            bf16 rounding after it)
  *  seq, hd:  positions per sequence (M a multiple of seq); head dim 64, 128
  *            or 256
  *  segments: bit i set = rotate segment i (n_out a multiple of hd, no
@@ -270,8 +274,10 @@ typedef struct lsq_rope_spec {
 } lsq_rope_spec;
 /* cos and sin of position * theta^(-2i/hd) for positions 0..seq-1 and
  * i = 0..hd/2-1, computed in double and rounded to fp32 (the angles lsq_rope
- * uses), written as (cos, sin) pairs into table [seq][hd/2][2] (device).
- * hd even and <= 1024, theta > 1, seq >= 1, else EINVAL. */
+ * uses), written as (cos, sin) pairs [seq][hd/2][2], followed by the hd/2
+ * frequencies theta^(-2i/hd) in fp32: lsq_rope_table_size(seq, hd) bytes of
+ * device memory.  hd even and <= 1024, theta > 1, seq >= 1, else EINVAL. */
+size_t lsq_rope_table_size(int64_t seq, int64_t hd);
 lsq_status lsq_rope_table(float theta, int64_t seq, int64_t hd, float* table, lsq_cuda_stream stream);
 /* lsq_nf4_lora_fwd_multi_ex with the RoPE of the segments `rope` marks
  * (NULL or no bits: exactly lsq_nf4_lora_fwd_multi_ex); with state NULL,
@@ -384,9 +390,10 @@ lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const 
  * q / k projections of lsq_nf4_lora_fwd_multi_ex2): with rope_table (from
  * lsq_rope_table for this seq and hd; NULL = plain lsq_attention_bwd), dq and
  * dk come out as the gradients of the unrotated q and k - the transpose of the
- * rotation applied to the fp32 gradient before its one bf16 rounding (head
- * dim 128 up to 512 positions; other shapes rotate the bf16 gradients in a
- * pass after the backward kernels).  rope_table 16-byte aligned. */
+ * rotation applied to the fp32 gradient before its one bf16 rounding, with
+ * the angles formed as in lsq_nf4_lora_fwd_multi_ex2 (head dim 128 up to 512
+ * positions; other shapes rotate the bf16 gradients with the table's pairs
+ * in a pass after the backward kernels).  rope_table 16-byte aligned. */
 lsq_status lsq_attention_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
                                 const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,
                                 int64_t hkv, int64_t hd, const float* rope_table, void* workspace,
@@ -576,8 +583,42 @@ lsq_status lsq_stream_time_waits(lsq_stream* st, int32_t capacity);
  * bwd_ms), their number and the number dropped; waits for those events and
  * starts a new count.  ESTATE when timing is off. */
 lsq_status lsq_stream_wait_ms(lsq_stream* st, float* fwd_ms, float* bwd_ms, int32_t* n_waits, int32_t* n_dropped);
-/* Forget all residency (next step re-uploads); waits for pending copies. */
+/* Forget all residency (next step re-uploads); waits for pending copies.
+ * ESTATE while a capture is open. */
 lsq_status lsq_stream_reset(lsq_stream* st);
+/* Recording one training step as a CUDA graph (stream capture), so that a
+ * step's several hundred kernels are launched from device memory: eager
+ * launches fetch their commands over the host link, which the layer copies
+ * keep busy, and measured on B200 they slow down by up to half under that
+ * load, while graph launches do not.
+ *
+ * lsq_stream_capture_begin, called after the caller began a capture on the
+ * compute stream (cudaStreamBeginCapture), brings the copy stream into that
+ * capture; lsq_stream_step then records its uploads, releases and waits into
+ * the graph instead of running them, and lsq_stream_capture_end, called
+ * before the capture ends, joins the copy stream back.  Inside the capture,
+ * a wait on a release or an upload recorded before it is left out: the graph
+ * starts after the compute stream's earlier work, and the caller makes the
+ * compute stream wait for the copy stream's earlier work before each launch
+ * of the graph.
+ *
+ * The captured step has not run: the policy's host state has advanced as if
+ * it had, so launch the graph once before any other use of the scheduler.
+ * Replaying it is only right when the step leaves the slot map (the layer
+ * each slot holds, their LRU order, the current layer) as it found it, which
+ * holds from the second step of a fixed 0 -> L-1 -> 0 walk on; capture_end
+ * checks this and returns ESTATE otherwise.  Events recorded in the capture
+ * are recorded again on the compute stream at the next eager use of the
+ * scheduler (lsq_stream_upload_ms then returns ESTATE for those layers until
+ * an eager step uploads them again).  Counters (lsq_stream_stats) advance at
+ * capture, not at replay.
+ *
+ * capture_begin: EINVAL with the disk tier, sharded uploads or wait timing
+ * on (they do host work in each step); ESTATE if the compute stream is not
+ * capturing or a capture is open.  capture_end: ESTATE if none is open or
+ * the slot map changed. */
+lsq_status lsq_stream_capture_begin(lsq_stream* st);
+lsq_status lsq_stream_capture_end(lsq_stream* st);
 lsq_status lsq_stream_destroy(lsq_stream* st);
 
 #ifdef __cplusplus

@@ -332,19 +332,18 @@ __device__ __forceinline__ void store_row_units(uint32_t row_base, int r, int pa
 }
 
 // dx1 = g1 c + g2 s, dx2 = g2 c - g1 s (the transpose of rotate-half RoPE) for 16
-// column pairs (i, i + 64) of a head, g = f * accumulator; cs: (cos, sin) of
-// frequencies i..i+15; writes columns i.. at dst and i + 64.. at dst + 64
+// column pairs (i, i + 64) of a head, g = f * accumulator; the angle of pair i is
+// pos * inv[i] (inv: the frequencies i..i+15), its cosine and sine from rope_cs;
+// writes columns i.. at dst and i + 64.. at dst + 64
 __device__ __forceinline__ void rope_t_store(__nv_bfloat16* dst, const float (&g1)[16], const float (&g2)[16],
-                                             const float2* __restrict__ cs, float f) {
+                                             const float* __restrict__ inv, float pos, float f) {
   float o1[16], o2[16];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float4 t = __ldg(reinterpret_cast<const float4*>(cs) + q);
-    const float a0 = g1[2 * q] * f, a1 = g1[2 * q + 1] * f, b0 = g2[2 * q] * f, b1 = g2[2 * q + 1] * f;
-    o1[2 * q] = a0 * t.x + b0 * t.y;
-    o2[2 * q] = b0 * t.x - a0 * t.y;
-    o1[2 * q + 1] = a1 * t.z + b1 * t.w;
-    o2[2 * q + 1] = b1 * t.z - a1 * t.w;
+  for (int i = 0; i < 16; ++i) {
+    const float2 t = rope_cs(pos * __ldg(inv + i));
+    const float a = g1[i] * f, b = g2[i] * f;
+    o1[i] = a * t.x + b * t.y;
+    o2[i] = b * t.x - a * t.y;
   }
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
@@ -549,7 +548,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
         tmem_ld16(tmem + lane_base + T_DQ + (uint32_t)(part * 16), x1);
         tmem_ld16(tmem + lane_base + T_DQ + (uint32_t)(64 + part * 16), x2);
         tc_wait_ld();
-        if (qi < S) rope_t_store(row + part * 16, x1, x2, rope + (int64_t)qi * (D / 2) + part * 16, scale);
+        if (qi < S)
+          rope_t_store(row + part * 16, x1, x2, reinterpret_cast<const float*>(rope) + (int64_t)S * D + part * 16,
+                       (float)qi, scale);
       } else {
         const int c4 = part;  // 32 of the 128 output columns per warp
         float v[32];
@@ -833,7 +834,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
         tmem_ld32(tmem + lane_base + T_DV + (uint32_t)(part * 32), c);
         tc_wait_ld();
         if (kj < S) {
-          rope_t_store(dk + off + part * 16, x1, x2, rope + (int64_t)kj * (D / 2) + part * 16, scale);
+          rope_t_store(dk + off + part * 16, x1, x2, reinterpret_cast<const float*>(rope) + (int64_t)S * D + part * 16,
+                       (float)kj, scale);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
             *reinterpret_cast<uint4*>(dv_out + off + part * 32 + u * 8) =
@@ -887,10 +889,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
         const float a_[4] = {a.x * scale, a.y * scale, a.z * scale, a.w * scale};
         const float g_[4] = {g.x * scale, g.y * scale, g.z * scale, g.w * scale};
         float o1[4], o2[4];
-        const float2* cs = rope + (int64_t)kr * (D / 2) + c4 * 4;
+        const float* inv = reinterpret_cast<const float*>(rope) + (int64_t)S * D + c4 * 4;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float2 tq = kr < S ? __ldg(cs + j) : make_float2(1.0f, 0.0f);
+          const float2 tq = rope_cs((float)kr * __ldg(inv + j));
           o1[j] = a_[j] * tq.x + g_[j] * tq.y;
           o2[j] = g_[j] * tq.x - a_[j] * tq.y;
         }

@@ -205,6 +205,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- RoPE angles
+// cos and sin of a RoPE angle (position x frequency, 0 <= a < 2^12 rad) in fp32: Cody-Waite additive
+// range reduction by 2 pi - a head of 8 significant bits, so that k * head is exact for the small
+// quotients k here, then the tail - followed by the special-function unit's sine and cosine on
+// [-pi, pi] (absolute error about 2^-21; the angle itself carries the fp32 rounding of position x
+// frequency, at most 2^-24 relative).  Both are far below the one bf16 rounding the rotation feeds.
+__device__ __forceinline__ float2 rope_cs(float a) {
+  constexpr float TWO_PI_HEAD = 6.28125f;                 // 201 / 32
+  constexpr float TWO_PI_TAIL = 1.93530717958647692e-3f;  // 2 pi - 201 / 32
+  constexpr float INV_TWO_PI = 0.159154943091895336f;     // 1 / (2 pi)
+  const float k = rintf(a * INV_TWO_PI);
+  float r = fmaf(-k, TWO_PI_HEAD, a);
+  r = fmaf(-k, TWO_PI_TAIL, r);
+  float sn, c;
+  __sincosf(r, &sn, &c);
+  return make_float2(c, sn);
+}
+
 // ---------------------------------------------------------------- bf16
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi

@@ -314,6 +314,15 @@ __device__ __forceinline__ void sk_issue(uint8_t* stage, uint64_t* sbar, const f
 }
 
 // bf16 output of 32 columns (chunk c) of row m of a tile whose first column is n0, with the residual (FWD)
+// A finisher that has seen the partials of clusters [c_lo, cid) for its rank clears their flags
+// once every epilogue thread is past its wait (each flag has this one reader).  Every flag is 0
+// again when the launch ends, so a launch replayed with the same epoch (a CUDA graph) cannot take
+// a flag left from an earlier replay for its own.
+__device__ __forceinline__ void clear_flags(const Params& p, int c_lo, int cid, unsigned rank) {
+  for (int c2 = c_lo; c2 < cid; ++c2)
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p.flags + c2 * 2 + (int)rank), "l"(0ull) : "memory");
+}
+
 template <int MODE>
 __device__ __forceinline__ void store_chunk(const Params& p, int sg, int n0, int ncols, int m, int c, float (&v)[32]) {
   if (m >= p.M) return;
@@ -610,16 +619,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tile_at<MODE, H>(p, t, m0, sg, n0);
       const int buf = j % NBUF;
       const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
-      if (MODE == FWD && p.seg[sg].rope && k1 == p.nkb) {
-        // the rows' RoPE angles into L1 while the tile's MMAs finish
-        const int half = p.rope_hd / 2;
-        for (int h = 0; h < H; ++h) {
-          const int m = m0 + h * BT + (int)rank * BMC + e;
-          if (m >= p.M) continue;
-          const char* row = reinterpret_cast<const char*>(p.rope + (int64_t)(m % p.rope_seq) * half);
-          for (int b = 0; b < half * 8; b += 128) asm volatile("prefetch.global.L1 [%0];" ::"l"(row + b));
-        }
-      }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
       tc_fence_after();
       if (k1 < p.nkb) {
@@ -647,6 +646,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       // clusters whose ranges end inside this tile, before this one's: their partials, in cluster order
       int cfirst = cid;
+      bool seen = true;  // every awaited flag held this launch's epoch
       if (p.streamk && k0 > 0) {
         const int64_t tstart = (int64_t)(t - p.dp_tiles) * p.nkb;
         while (cfirst > 0 && sk_bound(p, cfirst, ncl) > tstart) --cfirst;
@@ -663,11 +663,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (v == p.epoch) break;
             if (globaltimer() - t0 > LSQ_WAIT_NS) {
               report(LSQ_ETIMEOUT, 735);
+              seen = false;
               break;
             }
           }
         }
       }
+      const int cw = seen ? cfirst : cid;  // flags [cw, cid) are cleared at the end of this tile
       // 16 columns (piece 0 or 1) of two chunks hca, hcb of this tile's accumulator plus the
       // partials of the clusters before this one, added in the same order as the 32-column path
       // below; the two chunks' loads are issued together
@@ -767,22 +769,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         } else {
           tc_fence_before();
           named_bar_sync(1, 128);
-          if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+          if (e == 0) {
+            clear_flags(p, cw, cid, rank);
+            mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+          }
           continue;
         }
       }
       if (rope_seg) {
         // RoPE in the epilogue: column i of a head pairs with column i + hd/2, which sits hd/64
         // chunks of 32 further on in the same accumulator; both are rotated in fp32 (the
-        // accumulator plus earlier clusters' partials) and rounded once.  The loop takes 16
-        // frequencies at a time for every head of the tile in turn, so the row's (cos, sin) of
-        // those frequencies come from the L1 cache after the first head.
+        // accumulator plus earlier clusters' partials) and rounded once.  The angle of each
+        // pair is its row's position times the frequency, its cosine and sine computed here
+        // (rope_cs) from the table's per-frequency tail: no per-position table traffic.
         const int hc32 = p.rope_hd / 32, half = p.rope_hd / 2, heads = BT / p.rope_hd;
+        const float* inv = reinterpret_cast<const float*>(p.rope) + (int64_t)p.rope_seq * p.rope_hd;
         for (int fb = 0; fb < half / 16; ++fb) {
           const int cl = fb / 2, piece = fb % 2;
           for (int h = 0; h < H; ++h) {
             const int m = m0 + h * BT + (int)rank * BMC + e;
-            const float4* cs = reinterpret_cast<const float4*>(p.rope + (int64_t)(m % p.rope_seq) * half + fb * 16);
+            const float pos = (float)(m % p.rope_seq);
             for (int hh = 0; hh < heads; ++hh) {
               const int c = hh * hc32 + cl;
               if (n0 + c * 32 >= ncols) continue;
@@ -790,13 +796,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
               acc16x2(h * (BT / 32) + c, h * (BT / 32) + c + hc32 / 2, piece, x1, x2);
               if (m >= p.M) continue;
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 t = __ldg(cs + q);  // (cos, sin) of frequencies 2q, 2q + 1 of the block
-                const float a0 = x1[2 * q], a1 = x1[2 * q + 1], b0 = x2[2 * q], b1 = x2[2 * q + 1];
-                x1[2 * q] = a0 * t.x - b0 * t.y;
-                x2[2 * q] = b0 * t.x + a0 * t.y;
-                x1[2 * q + 1] = a1 * t.z - b1 * t.w;
-                x2[2 * q + 1] = b1 * t.z + a1 * t.w;
+              for (int i = 0; i < 16; ++i) {
+                const float2 t = rope_cs(pos * __ldg(inv + fb * 16 + i));
+                const float a = x1[i], b = x2[i];
+                x1[i] = a * t.x - b * t.y;
+                x2[i] = b * t.x + a * t.y;
               }
               const Seg& S = p.seg[sg];
               __nv_bfloat16* y1 = S.y + (int64_t)m * S.n + n0 + c * 32 + piece * 16;
@@ -815,7 +819,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_before();
         named_bar_sync(1, 128);
-        if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+        if (e == 0) {
+          clear_flags(p, cw, cid, rank);
+          mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+        }
         continue;
       }
       for (int hc = 0; hc < H * (BT / 32); ++hc) {
@@ -860,7 +867,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       named_bar_sync(1, 128);
-      if (e == 0) mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+      if (e == 0) {
+        clear_flags(p, cw, cid, rank);
+        mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
+      }
     }
   }
 
@@ -1210,7 +1220,8 @@ static size_t sk_region_bytes() {
   }
   return 4096 + (size_t)n * 2 * (size_t)(2 * (BT / 32) * 128 * 32 * sizeof(float));
 }
-// unique per launch within the process (a partial's flag holds its launch's value)
+// unique per launch within the process (a partial's flag holds its launch's value; its reader
+// clears it, see clear_flags, so a replayed launch may reuse the value)
 static unsigned long long next_epoch() {
   static std::atomic<unsigned long long> counter{
       (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull};

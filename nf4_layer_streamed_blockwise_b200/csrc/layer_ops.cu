@@ -148,10 +148,16 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
 }
 
 // (cos, sin) of pos * theta^(-2i/hd) for every position and frequency, with
-// rope_kernel's double-precision angle and rounding to fp32
+// rope_kernel's double-precision angle and rounding to fp32, then the hd/2
+// frequencies theta^(-2i/hd) themselves (fp32) after the n pairs
 __global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ table, int64_t n, int half, int hd,
                                                          double log_theta) {
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n + half;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    if (idx >= n) {
+      reinterpret_cast<float*>(table + n)[idx - n] = (float)exp(-2.0 * (int)(idx - n) / hd * log_theta);
+      continue;
+    }
     const int pos = (int)(idx / half), i = (int)(idx % half);
     const double inv = exp(-2.0 * i / hd * log_theta);
     double sn, c;
@@ -495,6 +501,11 @@ extern "C" lsq_status lsq_rope(void* x, int64_t batch, int64_t seq, int64_t head
   return LSQ_OK;
 }
 
+extern "C" size_t lsq_rope_table_size(int64_t seq, int64_t hd) {
+  if (seq < 1 || hd < 2) return 16;
+  return ((size_t)(seq * hd + hd / 2) * sizeof(float) + 15) / 16 * 16;
+}
+
 extern "C" lsq_status lsq_rope_table(float theta, int64_t seq, int64_t hd, float* table, lsq_cuda_stream stream) {
   if (!table) return fail(LSQ_EINVAL, "lsq_rope_table: NULL argument");
   if (seq < 1 || seq > (1 << 24) || hd < 2 || hd % 2 != 0 || hd > 1024 || !(theta > 1.0f))
@@ -502,7 +513,7 @@ extern "C" lsq_status lsq_rope_table(float theta, int64_t seq, int64_t hd, float
   lsq_status st = check_device();
   if (st != LSQ_OK) return st;
   const int64_t n = seq * (hd / 2);
-  rope_table_kernel<<<grid_for(n, 256), 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<float2*>(table), n,
+  rope_table_kernel<<<grid_for(n + hd / 2, 256), 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<float2*>(table), n,
                                                                          (int)(hd / 2), (int)hd, log((double)theta));
   LSQ_LAUNCH_CHECK("rope_table_kernel");
   return LSQ_OK;

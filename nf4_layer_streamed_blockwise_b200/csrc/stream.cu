@@ -283,18 +283,53 @@ struct lsq_stream {
   std::vector<cudaEvent_t> wev;      // 2 per kept wait
   std::vector<int> wdir;             // direction of each kept wait
   int n_wait = 0, n_wait_dropped = 0;
+  // stream capture of one step (lsq_stream_capture_begin / _end): the copy stream joins the compute
+  // stream's capture; only events recorded inside it order work inside it
+  bool capturing = false;
+  std::vector<char> cap_up, cap_free;  // up_done[layer] / slot_free[slot] recorded in this capture
+  cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
+  std::vector<int> cap_state;          // the policy's slot map when the capture began
+  // events last recorded inside a capture cannot be waited on or timed outside it: the first eager
+  // use after a capture records them again on the compute stream (after every replay queued there)
+  std::vector<char> stale_up, stale_free;
+  std::vector<char> untimed;           // the layer's upload events were re-recorded, not timed
 };
 
 namespace lsq {
 namespace sched {
 
+// Re-record, at the current point of the compute stream, the events a capture left behind: a
+// release or an upload recorded in a captured step is complete once the compute stream passes the
+// graph launches queued on it (the graph joins the copy stream back before it ends).
+static lsq_status refresh_after_capture(lsq_stream* st) {
+  for (size_t s = 0; s < st->stale_free.size(); ++s)
+    if (st->stale_free[s]) LSQ_CUDA_TRY(cudaEventRecord(st->slot_free[s], st->compute));
+  for (size_t l = 0; l < st->stale_up.size(); ++l)
+    if (st->stale_up[l]) {
+      LSQ_CUDA_TRY(cudaEventRecord(st->up_start[l], st->compute));
+      LSQ_CUDA_TRY(cudaEventRecord(st->up_done[l], st->compute));
+      st->untimed[l] = 1;
+    }
+  st->stale_free.clear();
+  st->stale_up.clear();
+  return LSQ_OK;
+}
+
 static lsq_status execute(lsq_stream* st) {
+  if (!st->capturing && (!st->stale_free.empty() || !st->stale_up.empty())) {
+    lsq_status s = refresh_after_capture(st);
+    if (s != LSQ_OK) return s;
+  }
   for (const Act& a : st->acts) {
     if (a.kind == RELEASE) {
       LSQ_CUDA_TRY(cudaEventRecord(st->slot_free[a.slot], st->compute));
       st->free_recorded[a.slot] = 1;
+      if (st->capturing) st->cap_free[a.slot] = 1;
     } else if (a.kind == UPLOAD) {
-      if (st->free_recorded[a.slot]) LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[a.slot], 0));
+      // in a capture, a release recorded before it is already ordered: the graph starts after the
+      // compute stream's earlier work
+      if (st->free_recorded[a.slot] && (!st->capturing || st->cap_free[a.slot]))
+        LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->slot_free[a.slot], 0));
       LSQ_CUDA_TRY(cudaEventRecord(st->up_start[a.layer], st->copy));
       char* dst = static_cast<char*>(st->slots[a.slot]) + (size_t)st->shard_rank * st->shard_bytes;
       if (st->reader) {
@@ -319,8 +354,13 @@ static lsq_status execute(lsq_stream* st) {
         st->expands += 1;
       }
       LSQ_CUDA_TRY(cudaEventRecord(st->up_done[a.layer], st->copy));
+      if (st->capturing) st->cap_up[a.layer] = 1;
+      st->untimed[a.layer] = 0;
       st->bytes += (int64_t)st->shard_bytes;
     } else if (a.kind == WAIT) {
+      // in a capture, an upload recorded before it is complete when the graph starts (the caller
+      // orders the compute stream after the copy stream's earlier work)
+      if (st->capturing && !st->cap_up[a.layer]) continue;
       const bool timed = !st->wev.empty();
       const bool kept = timed && 2 * (size_t)st->n_wait < st->wev.size();
       if (kept) LSQ_CUDA_TRY(cudaEventRecord(st->wev[2 * st->n_wait], st->compute));
@@ -367,6 +407,24 @@ static void destroy_events(lsq_stream* st) {
   for (auto* v : {&st->up_start, &st->up_done, &st->slot_free})
     for (cudaEvent_t e : *v)
       if (e) cudaEventDestroy(e);
+  if (st->fork_ev) cudaEventDestroy(st->fork_ev);
+  if (st->join_ev) cudaEventDestroy(st->join_ev);
+  st->fork_ev = st->join_ev = nullptr;
+}
+
+// The part of the policy's state that a step's actions depend on: which layer each slot holds, the
+// slots' LRU order, the layers stepped since their upload, the current layer.  (The tick counter
+// itself grows without bound; only the order it gives matters.)
+static std::vector<int> slot_map(const Policy& p) {
+  std::vector<int> v(p.slot_layer);
+  for (int s = 0; s < p.n_slots; ++s) {
+    int rank = 0;
+    for (int t = 0; t < p.n_slots; ++t) rank += p.slot_tick[t] < p.slot_tick[s];
+    v.push_back(rank);
+  }
+  for (char u : p.used_since_upload) v.push_back(u);
+  v.push_back(p.cur);
+  return v;
 }
 
 static bool valid_slots(int n_layers, int n_slots) {
@@ -458,6 +516,7 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   st->free_recorded.assign(cfg->n_slots, 0);
   st->up_start.assign(cfg->n_layers, nullptr);
   st->up_done.assign(cfg->n_layers, nullptr);
+  st->untimed.assign(cfg->n_layers, 0);
   st->slot_free.assign(cfg->n_slots, nullptr);
   cudaError_t e = cudaSuccess;
   for (int l = 0; l < cfg->n_layers && e == cudaSuccess; ++l) {
@@ -466,6 +525,8 @@ extern "C" lsq_status lsq_stream_create(const lsq_stream_cfg* cfg, lsq_cuda_stre
   }
   for (int i = 0; i < cfg->n_slots && e == cudaSuccess; ++i)
     e = cudaEventCreateWithFlags(&st->slot_free[i], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->fork_ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->join_ev, cudaEventDisableTiming);
   // every slot starts out released at this point of the compute stream, so the first upload into it
   // waits for the work queued there so far: the caller's allocator may have handed out the slots'
   // memory while kernels that still write its previous contents are queued on that stream
@@ -578,6 +639,8 @@ extern "C" lsq_status lsq_stream_stats(const lsq_stream* st, int64_t* uploads, i
 extern "C" lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float* ms) {
   if (!st || !ms) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: NULL argument");
   if (layer < 0 || layer >= st->pol.n_layers) return fail(LSQ_EINVAL, "lsq_stream_upload_ms: layer out of range");
+  if (st->capturing || ((size_t)layer < st->stale_up.size() && st->stale_up[layer]) || st->untimed[layer])
+    return fail(LSQ_ESTATE, "lsq_stream_upload_ms: layer %d was last uploaded inside a captured step", layer);
   LSQ_CUDA_TRY(cudaEventSynchronize(st->up_done[layer]));
   LSQ_CUDA_TRY(cudaEventElapsedTime(ms, st->up_start[layer], st->up_done[layer]));
   return LSQ_OK;
@@ -586,6 +649,7 @@ extern "C" lsq_status lsq_stream_upload_ms(lsq_stream* st, int32_t layer, float*
 extern "C" lsq_status lsq_stream_time_waits(lsq_stream* st, int32_t capacity) {
   if (!st) return fail(LSQ_EINVAL, "lsq_stream_time_waits: NULL scheduler");
   if (capacity < 0 || capacity > (1 << 20)) return fail(LSQ_EINVAL, "lsq_stream_time_waits: capacity %d", capacity);
+  if (st->capturing) return fail(LSQ_ESTATE, "lsq_stream_time_waits: a capture is open");
   LSQ_CUDA_TRY(cudaStreamSynchronize(st->compute));  // no kept wait is still pending on the old events
   destroy_wait_events(st);
   if (capacity == 0) return LSQ_OK;
@@ -623,6 +687,7 @@ extern "C" lsq_status lsq_stream_wait_ms(lsq_stream* st, float* fwd_ms, float* b
 
 extern "C" lsq_status lsq_stream_reset(lsq_stream* st) {
   if (!st) return fail(LSQ_EINVAL, "lsq_stream_reset: NULL scheduler");
+  if (st->capturing) return fail(LSQ_ESTATE, "lsq_stream_reset: a capture is open");
   LSQ_CUDA_TRY(cudaStreamSynchronize(st->copy));
   LSQ_CUDA_TRY(cudaStreamSynchronize(st->compute));
   const int64_t up = st->pol.uploads, re = st->pol.reused;
@@ -630,6 +695,39 @@ extern "C" lsq_status lsq_stream_reset(lsq_stream* st) {
   st->pol.uploads = up;
   st->pol.reused = re;
   std::fill(st->free_recorded.begin(), st->free_recorded.end(), 0);
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_capture_begin(lsq_stream* st) {
+  if (!st) return fail(LSQ_EINVAL, "lsq_stream_capture_begin: NULL scheduler");
+  if (st->capturing) return fail(LSQ_ESTATE, "lsq_stream_capture_begin: a capture is already open");
+  if (st->reader || st->gather)
+    return fail(LSQ_EINVAL, "lsq_stream_capture_begin: the disk tier and sharded uploads do host work in each step");
+  if (!st->wev.empty()) return fail(LSQ_EINVAL, "lsq_stream_capture_begin: exposed-copy timing is on");
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  LSQ_CUDA_TRY(cudaStreamIsCapturing(st->compute, &cs));
+  if (cs != cudaStreamCaptureStatusActive)
+    return fail(LSQ_ESTATE, "lsq_stream_capture_begin: the compute stream is not being captured");
+  st->cap_up.assign(st->pol.n_layers, 0);
+  st->cap_free.assign(st->pol.n_slots, 0);
+  LSQ_CUDA_TRY(cudaEventRecord(st->fork_ev, st->compute));
+  LSQ_CUDA_TRY(cudaStreamWaitEvent(st->copy, st->fork_ev, 0));
+  st->cap_state = slot_map(st->pol);
+  st->capturing = true;
+  return LSQ_OK;
+}
+
+extern "C" lsq_status lsq_stream_capture_end(lsq_stream* st) {
+  if (!st) return fail(LSQ_EINVAL, "lsq_stream_capture_end: NULL scheduler");
+  if (!st->capturing) return fail(LSQ_ESTATE, "lsq_stream_capture_end: no capture is open");
+  st->capturing = false;
+  st->stale_up = st->cap_up;
+  st->stale_free = st->cap_free;
+  LSQ_CUDA_TRY(cudaEventRecord(st->join_ev, st->copy));
+  LSQ_CUDA_TRY(cudaStreamWaitEvent(st->compute, st->join_ev, 0));
+  if (slot_map(st->pol) != st->cap_state)
+    return fail(LSQ_ESTATE, "lsq_stream_capture_end: the captured steps leave the slots holding other layers than "
+                "at the start, so a replay would compute on the wrong records (capture after a full warm-up step)");
   return LSQ_OK;
 }
 

@@ -85,6 +85,7 @@ _SIGS = {
                                              c_void_p, c_int32, ctypes.POINTER(lsq_rope_spec), c_void_p, c_size_t,
                                              c_void_p]),
     "lsq_rope_table": (c_int32, [c_float, c_int64, c_int64, c_void_p, c_void_p]),
+    "lsq_rope_table_size": (c_size_t, [c_int64, c_int64]),
     "lsq_attention_bwd_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int64, c_void_p,
                                        c_void_p, c_size_t, c_void_p]),
@@ -150,6 +151,8 @@ _SIGS = {
     "lsq_stream_wait_ms": (c_int32, [c_void_p, ctypes.POINTER(c_float), ctypes.POINTER(c_float),
                                      ctypes.POINTER(c_int32), ctypes.POINTER(c_int32)]),
     "lsq_stream_reset": (c_int32, [c_void_p]),
+    "lsq_stream_capture_begin": (c_int32, [c_void_p]),
+    "lsq_stream_capture_end": (c_int32, [c_void_p]),
     "lsq_stream_destroy": (c_int32, [c_void_p]),
 }
 
@@ -381,9 +384,21 @@ def lsq_nf4_lora_fwd_multi_ex2(Ws: Sequence[NF4Weight], x, M: int, A, B, r: int,
           _p(workspace), _nbytes(workspace), _stream(stream), launches=launches)
 
 
+def lsq_rope_table_size(seq: int, hd: int) -> int:
+    return _fn("lsq_rope_table_size")(seq, hd)
+
+
 def lsq_rope_table(theta: float, seq: int, hd: int, table, stream=None):
-    """(cos, sin) fp32 pairs [seq][hd/2] of the RoPE angles into table (device)."""
+    """(cos, sin) fp32 pairs [seq][hd/2] of the RoPE angles, then the hd/2 frequencies, into
+    table (device, lsq_rope_table_size bytes)."""
     _call("lsq_rope_table", theta, seq, hd, _p(table), _stream(stream))
+
+
+def rope_table(theta: float, seq: int, hd: int, device="cuda"):
+    """A device buffer of lsq_rope_table_size bytes filled by lsq_rope_table (fp32 view)."""
+    t = torch.empty(lsq_rope_table_size(seq, hd) // 4, dtype=torch.float32, device=device)
+    lsq_rope_table(theta, seq, hd, t)
+    return t
 
 
 def lsq_nf4_lora_bwd_multi_ex(Ws: Sequence[NF4Weight], x, dy, M: int, A, B, r: int, s: float, u, state, dx, dA, dB,
@@ -629,6 +644,15 @@ def lsq_stream_wait_ms(st: int):
 
 def lsq_stream_reset(st: int):
     _call("lsq_stream_reset", st)
+
+
+def lsq_stream_capture_begin(st: int):
+    """Bring the copy stream into the capture open on the compute stream (see lsq.h)."""
+    _call("lsq_stream_capture_begin", st)
+
+
+def lsq_stream_capture_end(st: int):
+    _call("lsq_stream_capture_end", st)
 
 
 def lsq_stream_destroy(st: int):

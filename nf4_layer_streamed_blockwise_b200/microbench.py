@@ -182,8 +182,7 @@ def main():
         wsf = torch.empty(L.lsq_nf4_lora_fwd_workspace_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
         run(f"fwd_{g}", fl, lambda: L.lsq_nf4_lora_fwd_multi(Ws, x, M, A, B, r, s, None, ys, us, workspace=wsf))
         if g == "qkv" and sh.hd in (64, 128, 256):   # the same call with q and k rotated in the epilogue
-            table = torch.empty(a.seq * sh.hd, dtype=torch.float32, device="cuda")
-            L.lsq_rope_table(sh.theta, a.seq, sh.hd, table)
+            table = L.rope_table(sh.theta, a.seq, sh.hd)
             run("fwd_qkv_rope", fl, lambda: L.lsq_nf4_lora_fwd_multi_ex2(Ws, x, M, A, B, r, s, None, ys, us, None,
                                                                           False, (table, a.seq, sh.hd, 0b011),
                                                                           workspace=wsf))

@@ -151,6 +151,19 @@ class LoraParams:
         L.lsq_lora_refresh_bf16(self.master, self.op, self.numel)
 
 
+@dataclasses.dataclass
+class _StepGraph:
+    """One recorded forward/backward: the graph, the kernels it launches, the scheduler counters
+    (uploads, bytes, reused per scheduler) one step advances, and whether it has run."""
+    graph: "torch.cuda.CUDAGraph"
+    launches: int
+    stats_delta: list
+    ran: bool = False
+
+    def replay(self):
+        self.graph.replay()
+
+
 class StreamedLoraTrainer:
     """One GPU, one batch of [batch, seq] token ids per step.
 
@@ -169,7 +182,7 @@ class StreamedLoraTrainer:
                  init: str = "device", lr: float = 2e-5, device: str = "cuda", share: "StreamedLoraTrainer" = None,
                  absmax: str = "fp32", shard: Optional[tuple] = None, source: str = "ram",
                  store_path: Optional[str] = None, embed: str = "hbm", head: str = "hbm",
-                 head_chunk: int = 8192):
+                 head_chunk: int = 8192, graph: bool = False):
         self.shape, self.B, self.S = shape, batch, seq
         self.timeline = None   # list of (kind, flops, start_event, end_event) when instrumented
         self.M = batch * seq
@@ -200,6 +213,16 @@ class StreamedLoraTrainer:
             self.embed_kind = embed = "host"   # one table: the head's host copy also serves the gather
         self.compute = torch.cuda.current_stream()
         self.copy = torch.cuda.Stream()
+        # graph: after a warm-up step, each kind of forward/backward is recorded once as a CUDA graph
+        # (the step's kernels, uploads and events) and replayed, so its launches are read from device
+        # memory instead of over the host link that the layer copies keep busy
+        self.graph = bool(graph)
+        if self.graph and (self.compute.cuda_stream == 0 or source == "disk" or shard is not None):
+            raise ValueError("graph replay needs a non-default compute stream (construct and drive the trainer "
+                             "under torch.cuda.stream(...)) and the host-RAM tier without sharding")
+        self._graphs = {}       # kind -> _StepGraph
+        self._stats_extra = [[0, 0, 0], [0, 0, 0]]   # counters of replays (layers, head)
+        self._warm = set()      # kinds that ran eagerly since the last residency change
         if share is not None and (share.absmax_kind != absmax or share.shard != self.shard or
                                   (share.source, share.store_path, share.embed_kind, share.head_kind,
                                    share.head_chunk) != (source, store_path, embed, head, self.head_chunk)):
@@ -369,8 +392,7 @@ class StreamedLoraTrainer:
         self.ws_xent = torch.empty(L.lsq_xent_workspace_size(M), dtype=torch.uint8, device=dev)
         # RoPE: (cos, sin) per position and frequency; with head dims the fused GEMM epilogue serves,
         # q and k are rotated there and the attention backward returns their unrotated gradients
-        self.rope_table = torch.empty(self.S * sh.hd, dtype=torch.float32, device=dev)
-        L.lsq_rope_table(sh.theta, self.S, sh.hd, self.rope_table)
+        self.rope_table = L.rope_table(sh.theta, self.S, sh.hd, device=dev)
         self.fuse_rope = sh.hd in (64, 128, 256)
 
     # ------------------------------------------------------------------ timing
@@ -541,8 +563,77 @@ class StreamedLoraTrainer:
     def set_ids(self, ids: torch.Tensor):
         self.ids.copy_(ids.reshape(-1).to(torch.int32), non_blocking=True)
 
+    # ------------------------------------------------------------------ graph replay
+    def _scheds(self):
+        return [s for s in (self.sched, self.head_sched) if s is not None]
+
+    def _raw_stats(self):
+        return [L.lsq_stream_stats(s) for s in self._scheds()]
+
+    def _graphed(self, kind, body):
+        """Run one forward/backward of this kind: eagerly while warming up or instrumented, else by
+        replaying its recorded graph (recorded at the first call after an eager warm-up step)."""
+        if not self.graph or self.timeline is not None:
+            body()
+            self._warm.add(kind)
+            return
+        g = self._graphs.get(kind)
+        if g is None:
+            if kind not in self._warm:      # the first step of a walk fills the slots: not periodic yet
+                body()
+                self._warm.add(kind)
+                return
+            g = self._capture(kind, body)
+        self.compute.wait_stream(self.copy)   # eager uploads queued before this step come first
+        g.replay()
+        if g.ran:                             # the capture advanced the counters once already
+            L.LAUNCHES[0] += g.launches
+            for k, d in enumerate(g.stats_delta):
+                self._stats_extra[k] = [a + b for a, b in zip(self._stats_extra[k], d)]
+        g.ran = True
+
+    def _capture(self, kind, body):
+        scheds = self._scheds()
+        before, launches0 = self._raw_stats(), L.LAUNCHES[0]
+        graph = torch.cuda.CUDAGraph()
+        opened = []
+        try:
+            with torch.cuda.graph(graph, stream=self.compute, capture_error_mode="thread_local"):
+                for sc in scheds:
+                    L.lsq_stream_capture_begin(sc)
+                    opened.append(sc)
+                body()
+                while opened:
+                    L.lsq_stream_capture_end(opened.pop(0))
+        except BaseException:
+            for sc in opened:
+                try:
+                    L.lsq_stream_capture_end(sc)
+                except L.LsqError:
+                    pass
+            # the policy advanced as if the captured step had run: forget residency so that the
+            # next step uploads what it needs
+            torch.cuda.synchronize()
+            for sc in scheds:
+                L.lsq_stream_reset(sc)
+            self._warm.clear()
+            raise
+        after = self._raw_stats()
+        g = _StepGraph(graph, L.LAUNCHES[0] - launches0,
+                       [[a - b for a, b in zip(x, y)] for x, y in zip(after, before)])
+        self._graphs[kind] = g
+        return g
+
+    def drop_graphs(self):
+        """Forget the recorded steps (the next step of each kind runs eagerly and records again)."""
+        torch.cuda.synchronize()
+        self._graphs.clear()
+
     def forward_backward(self):
         """Loss into self.loss_dev and LoRA gradients into self.lora.grad."""
+        self._graphed("sft", self._forward_backward)
+
+    def _forward_backward(self):
         sh, M = self.shape, self.M
         L.lsq_embed_gather(self.ids, self.embed, self.h[0], M, sh.d, sh.vocab)
         for l in range(sh.n_layers):
@@ -568,6 +659,12 @@ class StreamedLoraTrainer:
             self.ws_seqlp = torch.empty(L.lsq_seq_logprob_workspace_size(M), dtype=torch.uint8, device=dev)
 
     def forward_backward_dpo(self, beta: float = 0.1):
+        if self.B % 2:
+            raise ValueError("DPO needs an even batch (pairs of chosen / rejected sequences)")
+        self._dpo_buffers()
+        self._graphed(("dpo", float(beta)), lambda: self._forward_backward_dpo(beta))
+
+    def _forward_backward_dpo(self, beta: float = 0.1):
         """DPO over the batch as pairs (chosen = sequence 2i, rejected = 2i+1):
         loss into self.loss_dev, LoRA gradients into self.lora.grad.
 
@@ -624,11 +721,14 @@ class StreamedLoraTrainer:
         return self.logits
 
     def stats(self):
-        return L.lsq_stream_stats(self.sched)
+        """(uploads, bytes, reused) of the layer records since create, replayed steps included."""
+        return tuple(a + b for a, b in zip(L.lsq_stream_stats(self.sched), self._stats_extra[0]))
 
     def head_stats(self):
         """(uploads, bytes, reused) of the streamed head's chunks; zeros with a resident head."""
-        return L.lsq_stream_stats(self.head_sched) if self.head_sched is not None else (0, 0, 0)
+        if self.head_sched is None:
+            return (0, 0, 0)
+        return tuple(a + b for a, b in zip(L.lsq_stream_stats(self.head_sched), self._stats_extra[1]))
 
     def check_device(self):
         """Raise LsqError if a bounded wait inside any kernel ran out since the
@@ -638,10 +738,14 @@ class StreamedLoraTrainer:
         torch.cuda.synchronize()
         status, where = L.lsq_device_status()
         if status != 0:
+            self._graphs.clear()   # a recorded step is not replayed after a kernel gave up
             raise L.LsqError(status, "device status word",
                              f"a bounded device wait gave up (site {where}); results since the last check are void")
 
     def close(self):
+        if getattr(self, "_graphs", None):
+            torch.cuda.synchronize()
+            self._graphs.clear()
         if getattr(self, "head_sched", None):
             torch.cuda.synchronize()
             L.lsq_stream_destroy(self.head_sched)

@@ -196,8 +196,7 @@ def test_attention_bwd_with_rope_transpose(lsq, B, Sq, Hq, Hkv, hd, theta):
     o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device="cuda")
     lsq.lsq_attention_fwd(qg, kg, vg, o, lse, B, Sq, Hq, Hkv, hd)
-    table = torch.empty(Sq * hd, dtype=torch.float32, device="cuda")
-    lsq.lsq_rope_table(theta, Sq, hd, table)
+    table = lsq.rope_table(theta, Sq, hd)
     ws = torch.empty(lsq.lsq_attention_bwd_workspace_size(B, Sq, Hq), dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.empty_like(o), torch.empty_like(kg), torch.empty_like(vg)
     lsq.lsq_attention_bwd_ex(qg, kg, vg, o, lse, dog, dq, dk, dv, B, Sq, Hq, Hkv, hd, table, ws)

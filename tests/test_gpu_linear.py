@@ -354,8 +354,7 @@ def test_fused_forward_with_rope_matches_oracle(lsq, M, seq, Ns, K, hd, r, theta
         w = lsq.NF4Weight.empty(W.shape[0], K)
         lsq.lsq_nf4_quantize(W.cuda(), w.codes, w.absmax)
         qw.append(w)
-    table = torch.empty(seq * hd, dtype=torch.float32, device="cuda")
-    lsq.lsq_rope_table(theta, seq, hd, table)
+    table = lsq.rope_table(theta, seq, hd)
     ws = torch.zeros(lsq.lsq_nf4_lora_fwd_workspace_size(Ns, M, K, r), dtype=torch.uint8, device="cuda")
     state = torch.zeros(lsq.lsq_nf4_lora_state_size(Ns, M, K, r), dtype=torch.uint8, device="cuda")
     xg, Ag, Bg = x.cuda(), [a.cuda() for a in As], [b.cuda() for b in Bs]
