@@ -379,8 +379,9 @@ lsq_status lsq_attention_fwd(const void* q, const void* k, const void* v, void* 
 /* Gradients dq, dk, dv (bf16, same layouts) from do, given the forward's o
  * and lse; deterministic (each output written by one CTA, fixed summation
  * order).  Same limits as the forward; workspace:
- * lsq_attention_bwd_workspace_size() bytes (row dot products D =
- * rowsum(do * o), fp32 [B,Hq,S]); a smaller workspace is EINVAL. */
+ * lsq_attention_bwd_workspace_size() bytes, 16-byte aligned (per-row
+ * statistics: D = rowsum(do * o) and, for head dim 128 up to 512 positions,
+ * the log-sum-exp beside it); a smaller or misaligned workspace is EINVAL. */
 size_t lsq_attention_bwd_workspace_size(int64_t batch, int64_t seq, int64_t hq);
 lsq_status lsq_attention_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* d_o, void* dq, void* dk, void* dv, int64_t batch, int64_t seq, int64_t hq,

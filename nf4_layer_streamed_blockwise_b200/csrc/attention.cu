@@ -10,6 +10,8 @@
 // h / (Hq / Hkv).  Scale 1/sqrt(D).
 // Backward is deterministic: dQ and (dK, dV) are separate kernels that each
 // own their outputs; the GQA sum over query heads runs in a fixed order.
+#include <algorithm>
+
 #include "common.cuh"
 #include "host_common.h"
 
@@ -580,7 +582,10 @@ extern "C" lsq_status lsq_attention_fwd(const void* q, const void* k, const void
 }
 
 extern "C" size_t lsq_attention_bwd_workspace_size(int64_t batch, int64_t seq, int64_t hq) {
-  return (size_t)((batch * seq * hq > 0 ? batch * seq * hq : 1) * sizeof(float) + 255) / 256 * 256;
+  // the plain kernels' D [B, Hq, S] in fp32, or the tcgen05 kernels' row statistics table
+  const size_t plain = (size_t)(batch * seq * hq > 0 ? batch * seq * hq : 1) * sizeof(float);
+  const size_t tc = batch > 0 && seq > 0 && hq > 0 ? atc::bwd_stats_bytes(batch, seq, hq) : 0;
+  return (std::max(plain, tc) + 255) / 256 * 256;
 }
 
 namespace lsq {
@@ -601,18 +606,19 @@ extern "C" lsq_status lsq_attention_bwd_ex(const void* q, const void* k, const v
     return fail(LSQ_EINVAL, "lsq_attention_bwd: alignment");
   lsq_status st = check_args("lsq_attention_bwd", batch, seq, hq, hkv, hd);
   if (st != LSQ_OK) return st;
-  if (workspace_bytes < lsq_attention_bwd_workspace_size(batch, seq, hq))
-    return fail(LSQ_EINVAL, "lsq_attention_bwd: workspace too small");
+  if (workspace_bytes < lsq_attention_bwd_workspace_size(batch, seq, hq) || !aligned(workspace, 16))
+    return fail(LSQ_EINVAL, "lsq_attention_bwd: workspace too small or not 16-byte aligned");
+  const cudaStream_t cs = (cudaStream_t)stream;
+  // the tcgen05 kernels form their row statistics themselves and apply the RoPE transpose in their
+  // epilogues; the others take D from the pass below and leave RoPE to a pass after them
+  if (atc::bwd_supported(seq, hd))
+    return atc::run_bwd(q, k, v, o, d_o, lse, workspace, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs,
+                        rope_table);
   float* dvec = static_cast<float*>(workspace);
   const int64_t rows = batch * seq * hq;
-  const cudaStream_t cs = (cudaStream_t)stream;
   dvec_kernel<<<(unsigned)((rows * (hd / 8) + 255) / 256), 256, 0, cs>>>((const __nv_bfloat16*)o, (const __nv_bfloat16*)d_o,
                                                                   dvec, rows, (int)seq, (int)hq, (int)hd);
   LSQ_LAUNCH_CHECK("attention dvec_kernel");
-  // the tcgen05 kernels apply the RoPE transpose in their epilogues; the others leave it to a pass after them
-  if (atc::bwd_supported(seq, hd))
-    return atc::run_bwd(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs,
-                        rope_table);
   st = hd == 64 ? run_bwd<64>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs)
                 : run_bwd<128>(q, k, v, d_o, lse, dvec, dq, dk, dv, (int)batch, (int)seq, (int)hq, (int)hkv, cs);
   if (st != LSQ_OK || !rope_table) return st;

@@ -1,25 +1,15 @@
 // Causal GQA attention on the 5th-generation tensor cores (tcgen05), for head
 // dim 128 and sequences of at most 512 positions (the 8B and 32B workloads of
 // the streamed trainer).  Forward: one CTA per (query head, sequence, 128-query
-// tile).  Backward: a dQ kernel per query tile and a dK/dV kernel per key chunk
-// (below; with a GQA group of two or more, a two-CTA cluster per chunk), each
-// the sole owner of its outputs (no atomics).  Every grid puts the causal tile
-// index slowest and reversed, so the longest tiles of all heads start first.
-//
-//   S_j = Q K_j^T              tcgen05, fp32 in TMEM, 128 columns per 128-key chunk j
-//   P   = exp2(S*c - max)      exact two-pass softmax over the whole row (all of S
-//                               fits TMEM: 4 chunks x 128 columns), P in bf16 in
-//                               shared memory, 128-byte swizzled K-major
-//   O   = sum_j P_j V_j         tcgen05 into TMEM columns 0-127 (chunk 0's scores
-//                               are consumed before the first product lands)
-//   o   = O / l, lse = (max + log2 l) / log2(e)
+// tile), two per SM, online softmax over 64-key chunks (below).  Backward: a
+// dQ kernel per query tile and a dK/dV kernel per key chunk (with a GQA group
+// of two or more, a two-CTA cluster per chunk), each the sole owner of its
+// outputs (no atomics).  Every grid puts the causal tile index slowest and
+// reversed, so the longest tiles of all heads start first.
 //
 // Layouts as the mma.sync kernels: q, o [B, S, Hq, 128]; k, v [B, S, Hkv, 128];
-// lse [B, Hq, S].  Query head h reads kv head h / (Hq / Hkv).  K and V arrive
-// through a two-slot TMA ring (K chunks, then V chunks).  Warp 0: TMA; warp 1:
-// TMEM owner and MMA issuer; warps 2-17: softmax and epilogue, one query row
-// per lane (TMEM lane = row), four warps per lane quarter splitting the key
-// columns.  Every wait is bounded; no atomics.
+// lse [B, Hq, S].  Query head h reads kv head h / (Hq / Hkv).  Operands are
+// staged by TMA with the 128-byte swizzle; every wait is bounded.
 #include "common.cuh"
 #include "host_common.h"
 
@@ -28,24 +18,17 @@ namespace atc {
 
 constexpr int D = 128;           // head dim
 constexpr int BQ = 128;          // query rows per CTA
-constexpr int BC = 128;          // keys per chunk
-constexpr int MAXC = 4;          // chunks: sequences of at most 512
+constexpr int BC = 128;          // keys per backward chunk
+constexpr int MAXC = 4;          // 128-key chunks: sequences of at most 512
 constexpr int TILE = BQ * D * 2; // 128 x 128 bf16 tile: two 64-column 128B-swizzled halves of 16 KB
 constexpr int HALF = TILE / 2;
-constexpr int FRING = 4;          // forward K / V ring: every key chunk of a tile loads at once
-constexpr int FPB = 2;            // forward P buffers, reused every other chunk
-constexpr int OFF_Q = 0;          // Q; once the score products are done, the row statistics
-constexpr int OFF_RING = OFF_Q + TILE;
-constexpr int OFF_P = OFF_RING + FRING * TILE;
-constexpr int OFF_BAR = OFF_P + FPB * TILE;
-// qfull, rfull[4], rempty[4], sfull, pready[4], ofull, mxbar, smbar, pfree[2]
-constexpr int NBAR = 1 + FRING + FRING + 1 + MAXC + 1 + 2 + FPB;
-constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr int EW = 16;                     // element-wise warps: four per TMEM lane quarter
-constexpr int FWD_THREADS = 32 * (2 + EW);
-static_assert(SMEM_BYTES <= 232448, "shared memory");
+constexpr int EW = 16;                     // backward element-wise warps: four per TMEM lane quarter
+
+constexpr int SUB = 64;                     // keys per forward chunk, rows per backward sub-item
+constexpr int ST = SUB * D * 2;             // 64 x 128 bf16 tile: two 64-column halves of 8 KB
+constexpr int SHALF = ST / 2;
+constexpr int PT = BC * SUB * 2;            // 128 x 64 bf16 operand (one 128-byte swizzled column block)
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -64,30 +47,76 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
   return smem_desc(base + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024, 2);
 }
+// K-major 128-row x 64-element operand at k-step kk (16 elements)
+__device__ __forceinline__ uint64_t desc_k64(uint32_t base, int kk) { return smem_desc(base + kk * 32, 16, 1024, 2); }
+// K-major 64-row x 128-element operand (two 64-element halves of 8 KB) at k-step kk
+__device__ __forceinline__ uint64_t desc_sub_kmajor(uint32_t base, int kk) {
+  return smem_desc(base + (kk >> 2) * SHALF + (kk & 3) * 32, 16, 1024, 2);
+}
+// MN-major 64-row (K) x 128-column (N) operand: N halves 8 KB apart, 16 rows per k-step
+__device__ __forceinline__ uint64_t desc_sub_mnmajor(uint32_t base, int kk) {
+  return smem_desc(base + kk * 2048, SHALF, 1024, 2);
+}
 
-// Warp 0: TMA; warp 1: TMEM owner and MMA issuer; warps 2-17: softmax and
-// epilogue, four per TMEM lane quarter (one query row per lane, 32 of each
-// chunk's 128 key columns per warp); the four warps of a quarter combine
-// their partial row max and row sum through shared memory (an mbarrier each,
-// bounded waits).
-__global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                     const __grid_constant__ CUtensorMap kmap,
-                                                                     const __grid_constant__ CUtensorMap vmap,
+// ================================================================ forward
+// One CTA per (query head, sequence, 128-query tile), two CTAs per SM: while
+// one CTA's softmax warps turn scores into probabilities, the other's products
+// run on the tensor core.  Online softmax over 64-key chunks j:
+//
+//   S_j = Q K_j^T                 tcgen05 into one of two 64-column score buffers
+//   m   = running row max          (scaled to log2 units); kept while a chunk's
+//                                  max exceeds it by at most 8, so P_j <= 2^8 and
+//                                  O is rescaled only when the max jumps further
+//   P_j = exp2(S_j c - m)         bf16, written over K_j in its ring slot (the
+//                                  score product has read it)
+//   O  += P_j V_j                  tcgen05 into TMEM columns 0-127; l += rowsum P_j
+//   o   = O / l, lse = (m + log2 l) / log2(e)
+//
+// TMEM: O in columns 0-127, the score buffers in 128-191 and 192-255 (256 of
+// the SM's 512 per CTA).  Shared memory: Q (32 KB) and a five-slot ring of
+// 64-row K / V tiles (16 KB each), about 113 KB.  Warp 0: TMA (Q, then K_0, K_1,
+// and per chunk j: V_j, K_{j+2}, the order the products consume them); warp 1:
+// TMEM owner and MMA issuer (S_0, S_1, then per chunk: P_j V_j, S_{j+2}); warps
+// 2-5: softmax and epilogue, one query row per thread (TMEM lane = row).  Every
+// wait is bounded; no atomics.
+constexpr int FR = 5;                             // ring slots
+constexpr int F_OFF_Q = 0;
+constexpr int F_OFF_RING = F_OFF_Q + TILE;
+constexpr int F_OFF_BAR = F_OFF_RING + FR * ST;
+// qfull, rfull[FR], rempty[FR], sfull[2], pready[2], pvdone, drain
+constexpr int F_NBAR = 1 + 2 * FR + 2 + 2 + 1 + 1;
+constexpr int F_OFF_MISC = F_OFF_BAR + 8 * F_NBAR;
+constexpr int SMEM_BYTES = F_OFF_MISC + 16;
+constexpr int FWD_THREADS = 32 * 6;
+constexpr uint32_t F_T_O = 0, F_T_S = 128;       // TMEM columns
+constexpr float RESCALE_LOG2 = 8.0f;              // P_j <= 2^8 between rescales
+// two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA.  The tiles need 1024-byte
+// alignment for the 128-byte swizzle and there is no room to round the base up: the kernel checks it
+static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
+
+// ring position of K_j and V_j in the load order K_0, K_1, V_0, K_2, V_1, K_3, ..., V_{n-1}
+__device__ __forceinline__ int fwd_kidx(int j) { return j < 2 ? j : 2 * j - 1; }
+__device__ __forceinline__ int fwd_vidx(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 + 2 * j; }
+
+__global__ void __launch_bounds__(FWD_THREADS, 2) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                     const __grid_constant__ CUtensorMap kmap64,
+                                                                     const __grid_constant__ CUtensorMap vmap64,
                                                                      __nv_bfloat16* __restrict__ o,
                                                                      float* __restrict__ lse, int S, int Hq, int Hkv,
                                                                      float scale_log2) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + F_OFF_BAR);
   uint64_t* rfull = qfull + 1;
-  uint64_t* rempty = rfull + FRING;
-  uint64_t* sfull = rempty + FRING;
-  uint64_t* pready = sfull + 1;
-  uint64_t* ofull = pready + MAXC;
-  uint64_t* mxbar = ofull + 1;
-  uint64_t* smbar = mxbar + 1;
-  uint64_t* pfree = smbar + 1;  // [FPB]: the P V product of the buffer's previous chunk is done
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  uint64_t* rempty = rfull + FR;
+  uint64_t* sfull = rempty + FR;    // [2]: score buffer b holds S_j (j % 2 == b)
+  uint64_t* pready = sfull + 2;     // [2]: P_j written, S_j read, O rescaled (one arrival per softmax warp)
+  uint64_t* pvdone = pready + 2;    // one phase per chunk: P_j V_j (and everything before it) done
+  uint64_t* drain = pvdone + 1;     // error path: every product issued so far has completed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + F_OFF_MISC);
+  if (smem_u32(smem) & 1023u) {     // uniform over the CTA: nothing was started
+    if (threadIdx.x == 0) report(LSQ_EINVAL, 560);
+    return;
+  }
 
   const int nt = (S + BQ - 1) / BQ;
   // grid (head, sequence, query tile), tiles reversed: every head's longest causal tile is dispatched
@@ -96,25 +125,25 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
   const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0 = t * BQ;
-  const int nc = t + 1;  // key chunks at or before this query tile
+  const int n = (min(q0 + BQ, S) + SUB - 1) / SUB;  // 64-key chunks at or before the tile's last row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    for (int i = 0; i < FRING; ++i) {
+    for (int i = 0; i < FR; ++i) {
       mbar_init(&rfull[i], 1);
       mbar_init(&rempty[i], 1);
     }
-    mbar_init(sfull, 1);
-    for (int j = 0; j < MAXC; ++j) mbar_init(&pready[j], EW);  // one arrival per softmax warp
-    mbar_init(ofull, 1);
-    mbar_init(mxbar, EW);
-    mbar_init(smbar, EW);
-    for (int i = 0; i < FPB; ++i) mbar_init(&pfree[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pready[i], 4);
+    }
+    mbar_init(pvdone, 1);
+    mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, 512);
+    tmem_alloc(s_tmem, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -126,165 +155,193 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
     if (lane == 0) {
       const int row0 = b * S;
       mbar_arrive_expect_tx(qfull, (uint32_t)TILE);
-      tma_load_2d(smem + OFF_Q, &qmap, qfull, h * D, row0 + q0);
-      tma_load_2d(smem + OFF_Q + HALF, &qmap, qfull, h * D + 64, row0 + q0);
-      for (int it = 0; it < 2 * nc; ++it) {  // K chunks 0..nc-1, then V chunks 0..nc-1
-        const int slot = it % FRING;
-        const uint32_t ph = (uint32_t)(it / FRING) & 1u;
-        if (!mbar_wait(&rempty[slot], ph ^ 1u, 461)) break;
-        const int j = it < nc ? it : it - nc;
-        const CUtensorMap* m = it < nc ? &kmap : &vmap;
-        uint8_t* dst = smem + OFF_RING + slot * TILE;
-        mbar_arrive_expect_tx(&rfull[slot], (uint32_t)TILE);
-        tma_load_2d(dst, m, &rfull[slot], hk * D, row0 + j * BC);
-        tma_load_2d(dst + HALF, m, &rfull[slot], hk * D + 64, row0 + j * BC);
+      tma_load_2d(smem + F_OFF_Q, &qmap, qfull, h * D, row0 + q0);
+      tma_load_2d(smem + F_OFF_Q + HALF, &qmap, qfull, h * D + 64, row0 + q0);
+      int idx = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* m, int chunk) {
+        const int slot = idx % FR;
+        if (!ok || !mbar_wait(&rempty[slot], ((uint32_t)(idx / FR) & 1u) ^ 1u, 461)) {
+          ok = false;
+          return;
+        }
+        uint8_t* dst = smem + F_OFF_RING + slot * ST;
+        mbar_arrive_expect_tx(&rfull[slot], (uint32_t)ST);
+        tma_load_2d(dst, m, &rfull[slot], hk * D, row0 + chunk * SUB);
+        tma_load_2d(dst + SHALF, m, &rfull[slot], hk * D + 64, row0 + chunk * SUB);
+        ++idx;
+      };
+      load(&kmap64, 0);
+      if (n > 1) load(&kmap64, 1);
+      for (int j = 0; j < n; ++j) {
+        load(&vmap64, j);
+        if (j + 2 < n) load(&kmap64, j + 2);
       }
+      // no load may land after the CTA has gone: wait for the last one in each slot
+      for (int i = max(0, idx - FR); i < idx; ++i) mbar_wait(&rfull[i % FR], (uint32_t)(i / FR) & 1u, 462);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = mbar_wait(qfull, 0, 561);
-      if (ok) tc_fence_after();
-      const uint32_t qb = smem_u32(smem + OFF_Q);
-      const uint32_t id_s = idesc_bf16(BQ, BC, 0, 0);  // Q K^T: both K-major
-      const uint32_t id_o = idesc_bf16(BQ, D, 0, 1);   // P V: P K-major, V MN-major
-      for (int j = 0; ok && j < nc; ++j) {
-        const int slot = j % FRING;
-        if (!mbar_wait(&rfull[slot], (uint32_t)(j / FRING) & 1u, 562)) {
+      const uint32_t qb = smem_u32(smem + F_OFF_Q);
+      const uint32_t id_s = idesc_bf16(BQ, SUB, 0, 0);  // Q K^T: both K-major
+      const uint32_t id_o = idesc_bf16(BQ, D, 0, 1);    // P V: P K-major, V MN-major
+      auto score = [&](int j) {                          // S_j into buffer j % 2
+        const int c = fwd_kidx(j), slot = c % FR;
+        if (!ok || !mbar_wait(&rfull[slot], (uint32_t)(c / FR) & 1u, 562)) {
           ok = false;
-          break;
+          return;
         }
         tc_fence_after();
-        const uint32_t kb = smem_u32(smem + OFF_RING + slot * TILE);
+        const uint32_t kb = smem_u32(smem + F_OFF_RING + slot * ST);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          tc_mma(tmem + (uint32_t)(j * BC), desc_kmajor(qb, kk), desc_kmajor(kb, kk), id_s, kk != 0);
-        tc_commit(&rempty[slot]);
-      }
-      if (ok) tc_commit(sfull);
-      for (int j = 0; ok && j < nc; ++j) {
-        const int it = nc + j, slot = it % FRING;
-        if (!mbar_wait(&rfull[slot], (uint32_t)(it / FRING) & 1u, 563) || !mbar_wait(&pready[j], 0, 564)) {
+          tc_mma(tmem + F_T_S + (uint32_t)((j & 1) * SUB), desc_kmajor(qb, kk), desc_sub_kmajor(kb, kk), id_s,
+                 kk != 0);
+        tc_commit(&sfull[j & 1]);
+      };
+      if (ok) tc_fence_after();
+      score(0);
+      if (n > 1) score(1);
+      for (int j = 0; ok && j < n; ++j) {
+        const int c = fwd_vidx(j, n), vslot = c % FR, kslot = fwd_kidx(j) % FR;
+        if (!mbar_wait(&pready[j & 1], (uint32_t)(j >> 1) & 1u, 563) ||
+            !mbar_wait(&rfull[vslot], (uint32_t)(c / FR) & 1u, 564)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t pb = smem_u32(smem + OFF_P + (j % FPB) * TILE);
-        const uint32_t vb = smem_u32(smem + OFF_RING + slot * TILE);
+        const uint32_t pb = smem_u32(smem + F_OFF_RING + kslot * ST);  // P_j, written over K_j
+        const uint32_t vb = smem_u32(smem + F_OFF_RING + vslot * ST);
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk)
-          tc_mma(tmem, desc_kmajor(pb, kk), smem_desc(vb + kk * 2048, HALF, 1024, 2), id_o, (j | kk) != 0);
-        tc_commit(&rempty[slot]);
-        tc_commit(&pfree[j % FPB]);  // P buffer j % FPB may take chunk j + FPB
+        for (int kk = 0; kk < SUB / 16; ++kk)
+          tc_mma(tmem + F_T_O, desc_k64(pb, kk), desc_sub_mnmajor(vb, kk), id_o, (j | kk) != 0);
+        tc_commit(pvdone);
+        tc_commit(&rempty[kslot]);
+        tc_commit(&rempty[vslot]);
+        if (j + 2 < n) score(j + 2);
       }
-      tc_commit(ofull);  // also drains what was issued if a wait gave up
-      if (!ok) mbar_wait(ofull, 0, 565);
+      if (!ok) {  // let every product issued so far finish before TMEM is released
+        tc_commit(drain);
+        mbar_wait(drain, 0, 565);
+      }
     }
   } else {
-    // softmax and epilogue: one query row per lane, key columns part*32 .. +31 of every chunk
-    const int quad = warp & 3, part = (warp - 2) >> 2;
+    // softmax and epilogue: one query row per thread
+    const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int qi = q0 + r;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    float* s_max = reinterpret_cast<float*>(smem + OFF_Q);  // [4][128], after the score products
-    float* s_sum = s_max + 4 * BQ;                          // [4][128]
-    bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, 761));
     float m = -INFINITY, l = 0.0f;
-    if (ok) {
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int bb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[bb], (uint32_t)(j >> 1) & 1u, 761))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      for (int j = 0; j < nc; ++j) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + part * 32), v);
+      float s[64];
+      {
+        float lo[32], hi[32];
+        tmem_ld32(tmem + lane_base + F_T_S + (uint32_t)(bb * SUB), lo);
+        tmem_ld32(tmem + lane_base + F_T_S + (uint32_t)(bb * SUB + 32), hi);
         tc_wait_ld();
-        if (j < t) {  // a chunk before the diagonal: every key is visible
 #pragma unroll
-          for (int e = 0; e < 32; ++e) m = fmaxf(m, v[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int kj = j * BC + part * 32 + e;
-            if (kj <= qi && kj < S) m = fmaxf(m, v[e]);
-          }
+        for (int e = 0; e < 32; ++e) {
+          s[e] = lo[e];
+          s[32 + e] = hi[e];
         }
       }
-      m *= scale_log2;  // the scale is positive: max of scaled = scaled max
-      s_max[part * BQ + r] = m;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(mxbar);
-      ok = __all_sync(0xffffffffu, mbar_wait(mxbar, 0, 762));
-    }
-    if (ok) {
-      m = fmaxf(fmaxf(s_max[r], s_max[BQ + r]), fmaxf(s_max[2 * BQ + r], s_max[3 * BQ + r]));
-      for (int j = 0; j < nc; ++j) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(j * BC + part * 32), v);
-        tc_wait_ld();
-        uint32_t w[16];
-        if (j < t) {
+      const int k0 = j * SUB;
+      const bool full = k0 + SUB - 1 <= q0 && k0 + SUB <= S;  // every key of the chunk is visible to every row
+      if (!full) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(v[e] * scale_log2 - m), p1 = ex2(v[e + 1] * scale_log2 - m);
-            l += p0 + p1;
-            w[e / 2] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int kj = j * BC + part * 32 + e;
-            const float p0 = (kj <= qi && kj < S) ? ex2(v[e] * scale_log2 - m) : 0.0f;
-            const float p1 = (kj + 1 <= qi && kj + 1 < S) ? ex2(v[e + 1] * scale_log2 - m) : 0.0f;
-            l += p0 + p1;
-            w[e / 2] = pack_bf16x2(p0, p1);
-          }
-        }
-        // P buffer j % FPB held chunk j - FPB until its P V product completed
-        if (j >= FPB && !__all_sync(0xffffffffu, mbar_wait(&pfree[j % FPB], (uint32_t)((j - FPB) / FPB) & 1u, 766))) {
-          ok = false;
-          break;
-        }
-        // keys part*32 .. +31 of this chunk: half part >> 1, 16-byte units (part & 1) * 4 .. + 3
-        const uint32_t hbase = smem_u32(smem + OFF_P + (j % FPB) * TILE) + r * 128 + (uint32_t)(part >> 1) * HALF;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (part & 1) * 4 + u;
-          st_shared_v4(hbase + ((uint32_t)(unit ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
-                       w[4 * u + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pready[j]);
+        for (int e = 0; e < 64; ++e)
+          if (k0 + e > qi || k0 + e >= S) s[e] = -INFINITY;
       }
-      s_sum[part * BQ + r] = l;
+      float mxa = fmaxf(s[0], s[1]), mxb = fmaxf(s[2], s[3]);
+#pragma unroll
+      for (int e = 4; e < 64; e += 4) {
+        mxa = max3(mxa, s[e], s[e + 1]);
+        mxb = max3(mxb, s[e + 2], s[e + 3]);
+      }
+      const float mc = fmaxf(mxa, mxb) * scale_log2;  // the scale is positive: max of scaled = scaled max
+      const bool need = mc > m + RESCALE_LOG2;
+      // P_{j-1} V_{j-1} is done before O is rescaled or P_j may be consumed
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pvdone, (uint32_t)(j - 1) & 1u, 762))) {
+        ok = false;
+        break;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        tc_fence_after();
+        const float alpha = need ? ex2(m - mc) : 1.0f;
+        l *= alpha;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + F_T_O + (uint32_t)(c * 32), v);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tmem_st32(tmem + lane_base + F_T_O + (uint32_t)(c * 32), v);
+        }
+        tc_wait_st();
+      }
+      if (need) m = mc;
+      // p = 2^(s c - m), two columns per instruction but for the exponentials
+      uint32_t w[32];
+      const uint64_t c2 = f2(scale_log2, scale_log2), nm2 = f2(-m, -m);
+      uint64_t la = f2(0.0f, 0.0f), lb = la;
+#pragma unroll
+      for (int e = 0; e < 64; e += 4) {
+        const float2 xa = f2split(fma2(f2(s[e], s[e + 1]), c2, nm2));
+        const float2 xb = f2split(fma2(f2(s[e + 2], s[e + 3]), c2, nm2));
+        const uint64_t pa = f2(ex2(xa.x), ex2(xa.y)), pb = f2(ex2(xb.x), ex2(xb.y));
+        la = add2(la, pa);
+        lb = add2(lb, pb);
+        w[e / 2] = pack_bf16x2(pa);
+        w[e / 2 + 1] = pack_bf16x2(pb);
+      }
+      const float2 ls = f2split(add2(la, lb));
+      l += ls.x + ls.y;
+      // P_j over K_j (its score product completed before sfull): 128-byte rows, 16-byte units swizzled
+      const uint32_t prow = smem_u32(smem + F_OFF_RING + (fwd_kidx(j) % FR) * ST) + r * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(prow + ((uint32_t)(u ^ (r & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smbar);
-      ok = __all_sync(0xffffffffu, mbar_wait(smbar, 0, 763)) && __all_sync(0xffffffffu, mbar_wait(ofull, 0, 764)) &&
-           ok;
+      if (lane == 0) mbar_arrive(&pready[bb]);
     }
-    if (ok) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(pvdone, (uint32_t)(n - 1) & 1u, 763))) {
       tc_fence_after();
-      l = (s_sum[r] + s_sum[BQ + r]) + (s_sum[2 * BQ + r] + s_sum[3 * BQ + r]);
       const float inv = 1.0f / l;
       __nv_bfloat16* orow = o + (((int64_t)b * S + qi) * Hq + h) * D;
-      float v[32];
-      tmem_ld32(tmem + lane_base + (uint32_t)(part * 32), v);
-      tc_wait_ld();
-      if (qi < S) {
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + F_T_O + (uint32_t)(c * 32), v);
+        tc_wait_ld();
+        if (qi < S) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<uint4*>(orow + part * 32 + u * 8) =
-              make_uint4(pack_bf16x2(v[8 * u] * inv, v[8 * u + 1] * inv),
-                         pack_bf16x2(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
-                         pack_bf16x2(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
-                         pack_bf16x2(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
-        if (part == 0) lse[((int64_t)b * Hq + h) * S + qi] = (m + log2f(l)) / LOG2E;
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(orow + c * 32 + u * 8) =
+                make_uint4(pack_bf16x2(v[8 * u] * inv, v[8 * u + 1] * inv),
+                           pack_bf16x2(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
+                           pack_bf16x2(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
+                           pack_bf16x2(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
+        }
       }
+      if (qi < S) lse[((int64_t)b * Hq + h) * S + qi] = (m + log2f(l)) / LOG2E;
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -303,24 +360,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1) attn_fwd_tc_kernel(const __gri
 // operand tiles.  Warp 0: TMA; warp 1: TMEM owner and MMA issuer; warps 2-17:
 // element-wise and epilogue, four per TMEM lane quarter, 16 columns each (four
 // warps per SM sub-partition hide the TMEM, exp and shuffle latencies).
-constexpr int SUB = 64;                     // rows per sub-item
-constexpr int ST = SUB * D * 2;             // 64 x 128 bf16 tile: two 64-column halves of 8 KB
-constexpr int SHALF = ST / 2;
-constexpr int PT = BC * SUB * 2;            // 128 x 64 bf16 operand (one 128-byte swizzled column block)
 constexpr int NRING = 3;
 constexpr int CW = SUB / (EW / 4);           // columns per element-wise warp
 constexpr int BWD_THREADS = 32 * (2 + EW);
-
-// K-major 128-row x 64-element operand at k-step kk (16 elements)
-__device__ __forceinline__ uint64_t desc_k64(uint32_t base, int kk) { return smem_desc(base + kk * 32, 16, 1024, 2); }
-// K-major 64-row x 128-element operand (two 64-element halves of 8 KB) at k-step kk
-__device__ __forceinline__ uint64_t desc_sub_kmajor(uint32_t base, int kk) {
-  return smem_desc(base + (kk >> 2) * SHALF + (kk & 3) * 32, 16, 1024, 2);
-}
-// MN-major 64-row (K) x 128-column (N) operand: N halves 8 KB apart, 16 rows per k-step
-__device__ __forceinline__ uint64_t desc_sub_mnmajor(uint32_t base, int kk) {
-  return smem_desc(base + kk * 2048, SHALF, 1024, 2);
-}
 
 // CW bf16 values (CW / 2 pairs) of row r into a 128-row x 64-column swizzled
 // operand: the row's 16-byte units part * CW / 8 onwards
@@ -375,8 +417,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
                                                                     const __grid_constant__ CUtensorMap kmap64,
                                                                     const __grid_constant__ CUtensorMap vmap64,
                                                                     const __grid_constant__ CUtensorMap domap,
-                                                                    const float* __restrict__ lse,
-                                                                    const float* __restrict__ dvec,
+                                                                    const float4* __restrict__ stats, int Sp,
                                                                     __nv_bfloat16* __restrict__ dq, int S, int Hq,
                                                                     int Hkv, float scale, float scale_log2,
                                                                     const float2* __restrict__ rope) {
@@ -494,8 +535,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
     const int r = quad * 32 + lane;  // query row of the tile
     const int qi = q0 + r;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int64_t ri = ((int64_t)b * Hq + h) * S + (qi < S ? qi : 0);
-    const float lse2 = lse[ri] * LOG2E, dv = dvec[ri];
+    // this row's -lse (log2 units) and -D from the statistics table
+    const int64_t pr = ((int64_t)b * Hq + h) * Sp + (qi < S ? qi : 0);
+    const float4 st = stats[pr >> 1];
+    const float nl2 = (pr & 1) ? st.y : st.x, nd = (pr & 1) ? st.w : st.z;
+    const uint64_t c2 = f2(scale_log2, scale_log2), nl22 = f2(nl2, nl2), nd2 = f2(nd, nd);
     bool ok = true;
     for (int j = 0; ok && j < nsub; ++j) {
       const int bb = j & 1;
@@ -511,22 +555,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dq_tc_kernel(const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tfree[bb]);
+      // P = 2^(s c - lse), dS = P (dP - D), two columns per instruction but for the exponentials
       uint32_t w[CW / 2];
-      if ((j + 1) * SUB <= q0 && q0 + BQ <= S) {  // keys all before the tile, rows all inside S: no mask
+      const bool nomask = (j + 1) * SUB <= q0 && q0 + BQ <= S;  // keys all before the tile, rows inside S
 #pragma unroll
-        for (int e = 0; e < CW; e += 2) {
-          const float p0 = ex2(sv[e] * scale_log2 - lse2), p1 = ex2(sv[e + 1] * scale_log2 - lse2);
-          w[e / 2] = pack_bf16x2(p0 * (pv[e] - dv), p1 * (pv[e + 1] - dv));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < CW; e += 2) {
+      for (int e = 0; e < CW; e += 2) {
+        const float2 x = f2split(fma2(f2(sv[e], sv[e + 1]), c2, nl22));
+        float p0 = ex2(x.x), p1 = ex2(x.y);
+        if (!nomask) {
           const int kj = j * SUB + part * CW + e;
-          const bool ok0 = kj <= qi && kj < S && qi < S, ok1 = kj + 1 <= qi && kj + 1 < S && qi < S;
-          const float p0 = ok0 ? ex2(sv[e] * scale_log2 - lse2) : 0.0f;
-          const float p1 = ok1 ? ex2(sv[e + 1] * scale_log2 - lse2) : 0.0f;
-          w[e / 2] = pack_bf16x2(p0 * (pv[e] - dv), p1 * (pv[e + 1] - dv));
+          p0 = (kj <= qi && kj < S && qi < S) ? p0 : 0.0f;
+          p1 = (kj + 1 <= qi && kj + 1 < S && qi < S) ? p1 : 0.0f;
         }
+        w[e / 2] = pack_bf16x2(mul2(f2(p0, p1), add2(f2(pv[e], pv[e + 1]), nd2)));
       }
       // buffer bb was read by the dQ product of sub-item j - 2
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&dsfree[bb], (uint32_t)((j - 2) >> 1) & 1u, 772))) {
@@ -620,8 +661,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
                                                                      const __grid_constant__ CUtensorMap kmap,
                                                                      const __grid_constant__ CUtensorMap vmap,
                                                                      const __grid_constant__ CUtensorMap domap64,
-                                                                     const float* __restrict__ lse,
-                                                                     const float* __restrict__ dvec,
+                                                                     const float4* __restrict__ stats, int Sp,
                                                                      __nv_bfloat16* __restrict__ dk,
                                                                      __nv_bfloat16* __restrict__ dv_out, int S, int Hq,
                                                                      int Hkv, float scale, float scale_log2, int split,
@@ -744,22 +784,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
     const int r = quad * 32 + lane;  // key row of the chunk
     const int kj = k0 + r;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    // lse (as log2) and D of this warp's CW queries of sub-item it: lane l holds query
-    // l % CW (shuffles broadcast them); loaded one sub-item ahead
-    float l2own = 0.0f, dvown = 0.0f;
-    auto load_stats = [&](int it2, float& l2, float& dd) {
-      const int h2 = h_begin + it2 / nsub, q = k0 + (it2 % nsub) * SUB + part * CW + (lane % CW);
-      const int64_t ri = ((int64_t)b * Hq + h2) * S + (q < S ? q : 0);
-      l2 = lse[ri] * LOG2E;
-      dd = dvec[ri];
-    };
-    load_stats(0, l2own, dvown);
+    const uint64_t c2 = f2(scale_log2, scale_log2);
     bool ok = true;
     for (int it = 0; ok && it < items; ++it) {
       const int bb = it & 1;
       const int qs = k0 + (it % nsub) * SUB;
-      float l2next = 0.0f, dvnext = 0.0f;
-      if (it + 1 < items) load_stats(it + 1, l2next, dvnext);
+      // -lse (log2 units) and -D of this warp's CW queries, two queries per float4 of the statistics
+      // table (the same 16-byte loads in every lane), issued before the wait for the scores
+      float4 st[CW / 2];
+      {
+        const float4* src = stats + ((((int64_t)b * Hq + h_begin + it / nsub) * Sp + qs + part * CW) >> 1);
+#pragma unroll
+        for (int u = 0; u < CW / 2; ++u) st[u] = __ldg(src + u);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sfull[bb], (uint32_t)(it >> 1) & 1u, 781))) {
         ok = false;
         break;
@@ -772,31 +809,24 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tfree[bb]);
+      // P^T = 2^(s c - lse), dS^T = P^T (dP^T - D), two columns (queries) per instruction but for the
+      // exponentials
       uint32_t wp[CW / 2], wd[CW / 2];
-      if (qs >= k0 + BC && qs + SUB <= S && k0 + BC <= S) {  // every query after every key, all inside S
+      const bool nomask = qs >= k0 + BC && qs + SUB <= S && k0 + BC <= S;  // every query after every key
 #pragma unroll
-        for (int e = 0; e < CW; e += 2) {
-          const float l20 = __shfl_sync(0xffffffffu, l2own, e), l21 = __shfl_sync(0xffffffffu, l2own, e + 1);
-          const float d0 = __shfl_sync(0xffffffffu, dvown, e), d1 = __shfl_sync(0xffffffffu, dvown, e + 1);
-          const float p0 = ex2(sv[e] * scale_log2 - l20), p1 = ex2(sv[e + 1] * scale_log2 - l21);
-          wp[e / 2] = pack_bf16x2(p0, p1);
-          wd[e / 2] = pack_bf16x2(p0 * (pv[e] - d0), p1 * (pv[e + 1] - d1));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < CW; e += 2) {
+      for (int e = 0; e < CW; e += 2) {
+        const float4 t = st[e / 2];
+        const float2 x = f2split(fma2(f2(sv[e], sv[e + 1]), c2, f2(t.x, t.y)));
+        float p0 = ex2(x.x), p1 = ex2(x.y);
+        if (!nomask) {
           const int qi = qs + part * CW + e;
-          const float l20 = __shfl_sync(0xffffffffu, l2own, e), l21 = __shfl_sync(0xffffffffu, l2own, e + 1);
-          const float d0 = __shfl_sync(0xffffffffu, dvown, e), d1 = __shfl_sync(0xffffffffu, dvown, e + 1);
-          const bool ok0 = kj <= qi && qi < S && kj < S, ok1 = kj <= qi + 1 && qi + 1 < S && kj < S;
-          const float p0 = ok0 ? ex2(sv[e] * scale_log2 - l20) : 0.0f;
-          const float p1 = ok1 ? ex2(sv[e + 1] * scale_log2 - l21) : 0.0f;
-          wp[e / 2] = pack_bf16x2(p0, p1);
-          wd[e / 2] = pack_bf16x2(p0 * (pv[e] - d0), p1 * (pv[e + 1] - d1));
+          p0 = (kj <= qi && qi < S && kj < S) ? p0 : 0.0f;
+          p1 = (kj <= qi + 1 && qi + 1 < S && kj < S) ? p1 : 0.0f;
         }
+        const uint64_t p = f2(p0, p1);
+        wp[e / 2] = pack_bf16x2(p);
+        wd[e / 2] = pack_bf16x2(mul2(p, add2(f2(pv[e], pv[e + 1]), f2(t.z, t.w))));
       }
-      l2own = l2next;
-      dvown = dvnext;
       // buffer bb was read by the dV / dK products of sub-item it - 2
       if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pfree[bb], (uint32_t)((it - 2) >> 1) & 1u, 782))) {
         ok = false;
@@ -914,6 +944,47 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) attn_dkv_tc_kernel(const __gri
   }
 }
 
+// Row statistics for the backward kernels: per (sequence b, query head h, position q) -lse in log2
+// units and -D (D = rowsum(dO o), fp32, summed as the plain kernels sum it), stored as one float4
+// {-l2[q], -l2[q+1], -D[q], -D[q+1]} per even q, so that the dK/dV kernel reads two queries' values
+// with one 16-byte load and feeds them to the paired fp32 arithmetic as they are.  Each (b, h) row of
+// the table holds Sp positions (S rounded up to 64, zeros past S): every 64-query slice reads inside
+// it, and what it reads past S is finite.  16 lanes per row, 8 of its 128 columns each.
+__global__ void __launch_bounds__(256) rowstats_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ d_o,
+                                                       const float* __restrict__ lse, float* __restrict__ stats, int B,
+                                                       int S, int Sp, int Hq) {
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t w = t >> 4;  // row of [B][Sp][Hq]
+  const int part = (int)(t & 15);
+  const int64_t rows = (int64_t)B * Sp * Hq;
+  const int h = (int)(w % Hq);
+  const int q = (int)((w / Hq) % Sp);
+  const int b = (int)(w / ((int64_t)Hq * Sp));
+  const bool live = w < rows && q < S;
+  float sum = 0.0f;
+  if (live) {
+    const int64_t row = ((int64_t)b * S + q) * Hq + h;
+    const uint4 av = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+    const uint4 gv = *reinterpret_cast<const uint4*>(d_o + row * D + part * 8);
+    const uint32_t a[4] = {av.x, av.y, av.z, av.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sum = fmaf(bf16lo(a[k]), bf16lo(g[k]), sum);
+      sum = fmaf(bf16hi(a[k]), bf16hi(g[k]), sum);
+    }
+  }
+  for (int off = 8; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);  // the row's 16 lanes
+  if (w < rows && part == 0) {
+    const int64_t pr = ((int64_t)b * Hq + h) * Sp + q;
+    float* dst = stats + (pr >> 1) * 4 + (pr & 1);
+    dst[0] = live ? -lse[((int64_t)b * Hq + h) * S + q] * LOG2E : 0.0f;
+    dst[2] = live ? -sum : 0.0f;
+  }
+}
+
+size_t bwd_stats_bytes(int64_t B, int64_t S, int64_t Hq) { return (size_t)(B * Hq * ((S + SUB - 1) / SUB * SUB)) * 8; }
+
 static lsq_status tmap_heads(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, int box_rows = BQ) {
   return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)(heads * D), (uint64_t)rows,
                         (uint64_t)(heads * D * 2), 64, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -935,8 +1006,8 @@ lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   lsq_status s;
   const int64_t rows = (int64_t)B * S;
   if ((s = tmap_heads(&qm, q, rows, Hq)) != LSQ_OK) return s;
-  if ((s = tmap_heads(&km, k, rows, Hkv)) != LSQ_OK) return s;
-  if ((s = tmap_heads(&vm, v, rows, Hkv)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&km, k, rows, Hkv, SUB)) != LSQ_OK) return s;
+  if ((s = tmap_heads(&vm, v, rows, Hkv, SUB)) != LSQ_OK) return s;
   const float sl = LOG2E / sqrtf((float)D);
   attn_fwd_tc_kernel<<<dim3(Hq, B, (S + BQ - 1) / BQ), FWD_THREADS, SMEM_BYTES, st>>>(
       qm, km, vm, static_cast<__nv_bfloat16*>(o), lse, S, Hq, Hkv, sl);
@@ -946,8 +1017,8 @@ lsq_status run_fwd(const void* q, const void* k, const void* v, void* o, float* 
 
 bool bwd_supported(int64_t S, int64_t hd) { return fwd_supported(S, hd); }
 
-lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o, const float* lse, const float* dvec,
-                   void* dq, void* dk, void* dv, int B, int S, int Hq, int Hkv, cudaStream_t st,
+lsq_status run_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                   void* ws, void* dq, void* dk, void* dv, int B, int S, int Hq, int Hkv, cudaStream_t st,
                    const float* rope_table) {
   const float2* rope = reinterpret_cast<const float2*>(rope_table);
   static int cfg[64];
@@ -971,7 +1042,14 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
   if ((s = tmap_heads(&dom64, d_o, rows, Hq, SUB)) != LSQ_OK) return s;
   const float scale = 1.0f / sqrtf((float)D), sl = LOG2E * scale;
   const int nt = (S + BQ - 1) / BQ;
-  attn_dq_tc_kernel<<<dim3(Hq, B, nt), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, lse, dvec,
+  const int Sp = (S + SUB - 1) / SUB * SUB;
+  const int64_t srows = (int64_t)B * Sp * Hq;
+  rowstats_kernel<<<(unsigned)((srows * 16 + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse, static_cast<float*>(ws), B,
+      S, Sp, Hq);
+  LSQ_LAUNCH_CHECK("attention rowstats_kernel");
+  const float4* stats = static_cast<const float4*>(ws);
+  attn_dq_tc_kernel<<<dim3(Hq, B, nt), BWD_THREADS, Q_SMEM, st>>>(qm, km64, vm64, dom, stats, Sp,
                                                                   static_cast<__nv_bfloat16*>(dq), S, Hq, Hkv, scale,
                                                                   sl, rope);
   LSQ_LAUNCH_CHECK("attn_dq_tc_kernel");
@@ -988,7 +1066,7 @@ lsq_status run_bwd(const void* q, const void* k, const void* v, const void* d_o,
   attr[0].val.clusterDim.z = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  LSQ_CUDA_TRY(cudaLaunchKernelEx(&lc, attn_dkv_tc_kernel, qm64, km, vm, dom64, lse, dvec,
+  LSQ_CUDA_TRY(cudaLaunchKernelEx(&lc, attn_dkv_tc_kernel, qm64, km, vm, dom64, stats, Sp,
                                   static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), S, Hq, Hkv, scale,
                                   sl, split, rope));
   return LSQ_OK;

@@ -88,12 +88,18 @@ def _attn_case(B, Sq, Hq, Hkv, hd, seed):
     return q, k, v, do
 
 
-@pytest.mark.parametrize("B,Sq,Hq,Hkv,hd", [(1, 512, 9, 3, 64), (2, 200, 4, 1, 128), (1, 64, 2, 2, 64),
-                                            (1, 1, 4, 2, 128), (2, 130, 8, 2, 128), (2, 512, 32, 8, 128),
-                                            (1, 384, 4, 4, 128), (1, 300, 7, 1, 128), (2, 256, 6, 2, 128),
-                                            (1, 512, 16, 2, 128)])
-def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd):
+@pytest.mark.parametrize("B,Sq,Hq,Hkv,hd,ramp", [(1, 512, 9, 3, 64, False), (2, 200, 4, 1, 128, False),
+                                                 (1, 64, 2, 2, 64, False), (1, 1, 4, 2, 128, False),
+                                                 (2, 130, 8, 2, 128, False), (2, 512, 32, 8, 128, False),
+                                                 (1, 384, 4, 4, 128, False), (1, 300, 7, 1, 128, False),
+                                                 (2, 256, 6, 2, 128, False), (1, 512, 16, 2, 128, False),
+                                                 (1, 512, 8, 2, 128, True), (2, 300, 4, 1, 128, True)])
+def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd, ramp):
+    """ramp: key j scaled by 1 + 8 j / S, so that each 64-key chunk's max jumps past the running
+    one and the forward's online softmax rescales its accumulator again and again."""
     q, k, v, do = _attn_case(B, Sq, Hq, Hkv, hd, Sq)
+    if ramp:
+        k = (k.float() * (1.0 + 8.0 * torch.arange(Sq, dtype=torch.float32) / Sq)[None, :, None, None]).to(k.dtype)
     o = torch.empty(B, Sq, Hq, hd, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device="cuda")
     lsq.lsq_attention_fwd(q.cuda(), k.cuda(), v.cuda(), o, lse, B, Sq, Hq, Hkv, hd)
