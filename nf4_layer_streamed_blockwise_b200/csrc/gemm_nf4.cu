@@ -30,11 +30,14 @@
 //
 // Warp roles in each CTA of the pair:
 //   0-3   epilogue: TMEM lanes 0-127 -> the CTA's 128 output rows
-//   4     TMA producer: activation tile, packed codes, the LoRA block's tiles
+//   9     TMA producer: activation tile, packed codes, the LoRA block's tiles
 //   5     TMEM owner; in the leader CTA (rank 0) also the MMA issuer
-//   6-13  NF4 decoders: two threads per 64-value block of the stage, each
-//         writing half of one 128-byte row of the swizzled bf16 operand; the
-//         block's 16 possible values live in registers (byte-permute decode)
+//   4, 6-8, 10-12, 14  NF4 decoders: two threads per 64-value block of the
+//         stage, each writing half of one 128-byte row of the swizzled bf16
+//         operand; the block's 16 possible values live in registers
+//         (byte-permute decode, eight codes per step)
+//   13    idle: the issuing warps 5 and 9 have SM sub-partition 1 to
+//         themselves (see NTHREADS)
 // The leader's "full" barrier of a stage completes when both CTAs' TMA bytes
 // have landed and all 16 decoder warps of the pair have arrived; the MMA
 // commit releases the stage in both CTAs at once (commit multicast).  Every
@@ -164,10 +167,19 @@ __device__ __forceinline__ uint2 dq4(uint32_t ch, const DqTab& t) {
   // lo / hi bytes are ordered (code 1, code 0, code 3, code 2): interleave to bf16 words
   return make_uint2(prmt(lo, hi, 0x4051u), prmt(lo, hi, 0x6273u));
 }
-// eight codes (one 32-bit word) -> eight bf16
+// eight codes (one 32-bit word) -> eight bf16: dq4 of the low and the high half-word, with the
+// code and sign masks formed once on the whole word (prmt reads only the low 16 bits of its
+// selector, and the shifted sign bits stay inside their half-word)
 __device__ __forceinline__ uint4 dq8(uint32_t w, const DqTab& t) {
-  const uint2 a = dq4(w, t), b = dq4(w >> 16, t);
-  return make_uint4(a.x, a.y, b.x, b.y);
+  const uint32_t s7 = w & 0x77777777u, c8 = w & 0x88888888u;
+  const uint32_t sel = c8 | (c8 >> 1), s7h = s7 >> 16;
+  const uint32_t m0 = prmt(0u, 0x80u, sel), m1 = prmt(0u, 0x80u, sel >> 16);
+  const uint32_t lo0 = (prmt(t.lo[0], t.lo[1], s7) & ~m0) | (prmt(t.lo[2], t.lo[3], s7) & m0);
+  const uint32_t hi0 = (prmt(t.hi[0], t.hi[1], s7) & ~m0) | (prmt(t.hi[2], t.hi[3], s7) & m0);
+  const uint32_t lo1 = (prmt(t.lo[0], t.lo[1], s7h) & ~m1) | (prmt(t.lo[2], t.lo[3], s7h) & m1);
+  const uint32_t hi1 = (prmt(t.hi[0], t.hi[1], s7h) & ~m1) | (prmt(t.hi[2], t.hi[3], s7h) & m1);
+  return make_uint4(prmt(lo0, hi0, 0x4051u), prmt(lo0, hi0, 0x6273u), prmt(lo1, hi1, 0x4051u),
+                    prmt(lo1, hi1, 0x6273u));
 }
 
 // half of an NF4 block (32 values, 16 code bytes) -> 16-byte chunks
@@ -186,8 +198,18 @@ constexpr int BK = 64;
 constexpr int A_BYTES = BMC * BK * 2;  // 16 KB per 128-row activation tile
 constexpr int W_BYTES = BNC * BK * 2;  // 16 KB
 constexpr int C_BYTES = BNC * BK / 2;  // 4 KB
+// Warp roles: 0-3 epilogue (TMEM lane quarters), 5 TMEM owner and MMA issuer, 9 TMA producer,
+// 4, 6, 7, 8, 10, 11, 12, 14 NF4 decoders, 13 idle.  A warp stalled issuing tcgen05.mma (or a TMA)
+// holds back the shared-memory traffic of the other warps of its SM sub-partition (warp % 4):
+// decoders beside the MMA issuer ran about four times slower than the rest (2700 against 650
+// cycles per stage, measured on B200) and set the pace of every stage.  So the issuing warps share
+// sub-partition 1 and the decoders take the other three.
 constexpr int DQ_WARPS = 8;
-constexpr int NTHREADS = (6 + DQ_WARPS) * 32;
+constexpr int NTHREADS = 15 * 32;
+constexpr int W_MMA = 5, W_TMA = 9;
+__device__ __forceinline__ bool is_decoder(int warp) { return warp >= 4 && (warp & 3) != 1; }
+// decoder index 0 .. 7 of a decoder warp (4 -> 0, 6 -> 1, 7 -> 2, 8 -> 3, 10 -> 4, 11 -> 5, 12 -> 6, 14 -> 7)
+__device__ __forceinline__ int decoder_index(int warp) { return warp - 4 - (warp > 5) - (warp > 9) - (warp > 13); }
 
 // H = 256-row halves per pair tile.  H = 1: six stages and two accumulator
 // buffers, so the epilogue of one tile overlaps the main loop of the next.
@@ -390,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     mbar_init(&sbar[1], 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc_pair(s_tmem, 512);
     tmem_relinquish_pair();
   }
@@ -399,7 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == 4) {
+  if (warp == W_TMA) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t g = 0;
@@ -441,7 +463,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     // ---------------------------------------------------------------- MMA issuer (leader CTA)
     if (rank == 0 && lane == 0) {
       const uint32_t id_k = idesc_bf16(2 * BMC, BT, 0, 0);   // both operands K-major
@@ -488,9 +510,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_wait(drain, 0, 523);
       }
     }
-  } else if (warp >= 6) {
+  } else if (is_decoder(warp)) {
     // ---------------------------------------------------------------- NF4 decoders
-    const int t = threadIdx.x - 6 * 32;  // 0 .. 255
+    const int t = decoder_index(warp) * 32 + lane;  // 0 .. 255
     const int KB = p.K / 64;
     uint32_t g = 0;
     bool ok = true;
@@ -608,7 +630,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 4) {
     // ---------------------------------------------------------------- epilogue (warps 0-3)
     const int e = threadIdx.x;  // TMEM lane = row within the CTA's 128
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -876,7 +898,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
   tc_fence_before();
   cluster_sync_all();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
