@@ -1,0 +1,85 @@
+"""The attention kernels' arithmetic on the CPU (test infrastructure): fp32
+products and sums with bf16 roundings exactly where the CUDA kernels round -
+the probabilities entering P.V (the forward's online softmax over 64-key
+chunks, its running max kept while a chunk exceeds it by at most 8 in log2
+units) and P^T.dO, dS, the outputs, and D from the bf16 output.
+
+It serves two tests: test_attn_bounds_cpu.py checks that its errors sit
+inside the first-order bound of attn_bounds.py and that planted mistakes do
+not; the GPU attention test takes its relative Frobenius tolerance from it
+on inputs where the softmax is sharp.  There dS = P (dP - D) cancels, and
+the bf16 roundings alone move dq and dk by about 5e-3 relative Frobenius
+(this model: 4.9e-3 to 5.2e-3 on keys scaled by up to 9x), so such inputs
+are held to twice this model's error, never below the 5e-3 of the GEMMs.
+"""
+import math
+
+import torch
+
+def bf(t):
+    return t.to(torch.bfloat16).to(torch.float32)
+
+
+LOG2E = 1.4426950408889634
+
+
+def online_o(s, vv, chunk=64, thresh=8.0):
+    """The forward's online softmax: 64-key chunks, a running max in log2 units that is kept
+    while a chunk's max exceeds it by at most 8 (else O and l are rescaled), bf16 P into P.V."""
+    s2 = s * LOG2E
+    B, H, S, _ = s.shape
+    m = torch.full((B, H, S), float("-inf"))
+    l = torch.zeros(B, H, S)
+    O = torch.zeros(B, H, S, vv.shape[-1])
+    for j0 in range(0, S, chunk):
+        sc = s2[..., j0:j0 + chunk]
+        mc = sc.max(-1).values
+        need = mc > m + thresh
+        alpha = torch.where(need, torch.exp2(m - mc), torch.ones_like(m))
+        O, l = O * alpha[..., None], l * alpha
+        m = torch.where(need, mc, m)
+        p = torch.exp2(sc - m[..., None])
+        l = l + p.sum(-1)
+        O = O + torch.einsum("bhij,bjhd->bhid", bf(p), vv[:, j0:j0 + chunk])
+    return bf((O / l[..., None]).permute(0, 2, 1, 3)), m, l
+
+
+def model(q, k, v, do, shift_d=False, one_head_dv=False, mask_diag_off=False, online=False):
+    B, S, Hq, hd = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    kk, vv = k.repeat_interleave(g, 2), v.repeat_interleave(g, 2)
+    tau = 1.0 / math.sqrt(hd)
+    mask = torch.triu(torch.ones(S, S, dtype=torch.bool), 0 if mask_diag_off else 1)
+    mask[0, 0] = False
+    s = (torch.einsum("bihd,bjhd->bhij", q, kk) * tau).masked_fill(mask, float("-inf"))
+    m = s.max(-1, keepdim=True).values
+    p = torch.exp(s - m)
+    l = p.sum(-1, keepdim=True)
+    o = bf(torch.einsum("bhij,bjhd->bihd", bf(p), vv) / l.squeeze(-1).permute(0, 2, 1)[..., None])
+    if online:
+        o = online_o(s, vv)[0]
+    P = torch.exp(s - (m + torch.log(l)))
+    D = (do * o).sum(-1).permute(0, 2, 1)
+    if shift_d:
+        D = torch.roll(D, 1, dims=-1)
+    dP = torch.einsum("bihd,bjhd->bhij", do, vv)
+    dS = bf(P * (dP - D[..., None]))
+    dq = bf(tau * torch.einsum("bhij,bjhd->bihd", dS, kk))
+    dk = bf((tau * torch.einsum("bhij,bihd->bjhd", dS, q)).reshape(B, S, Hkv, g, hd).sum(3))
+    pdo = torch.einsum("bhij,bihd->bjhd", bf(P), do).reshape(B, S, Hkv, g, hd)
+    dv = bf(pdo[:, :, :, 0] * g if one_head_dv else pdo.sum(3))
+    return {"o": o, "dq": dq, "dk": dk, "dv": dv}
+
+
+def frobenius_tolerance(q, k, v, do, exact, floor=5e-3, factor=2.0):
+    """name -> max(floor, factor x this model's relative Frobenius error against the exact values
+    (attn_bounds.attention_bounds' o, dq, dk, dv))."""
+    got = model(q, k, v, do, online=True)
+    tol = {}
+    for name in ("o", "dq", "dk", "dv"):
+        ref = exact[name]
+        n = float(ref.norm())
+        rf = float((got[name].double() - ref).norm()) / n if n > 0 else 0.0
+        tol[name] = max(floor, factor * rf)
+    return tol

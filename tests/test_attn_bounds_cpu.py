@@ -1,70 +1,18 @@
 """The attention tolerance (attn_bounds.py) against a CPU model of the kernels'
-arithmetic: fp32 products and sums with bf16 roundings exactly where the CUDA
-kernels round (the probabilities entering P.V and P^T.dO, dS, the outputs; D
-from the bf16 output).  The model's errors must sit inside the bound, and
-plausible mistakes (D of the wrong row, dV from one head of a GQA group, a
-transposed mask) must fall far outside it."""
+arithmetic (attn_model.py: fp32 products and sums with bf16 roundings exactly
+where the CUDA kernels round).  The model's errors must sit inside the
+first-order bound, and plausible mistakes (D of the wrong row, dV from one
+head of a GQA group, a transposed mask) must fall far outside it.  On
+ordinary inputs the model also stays inside the GEMMs' 5e-3 relative
+Frobenius; on keys that make the softmax sharp its dq and dk do not (about
+5e-3 from the bf16 roundings alone), which is why the GPU test takes its
+Frobenius tolerance from the model there."""
 import math
 
 import torch
 
 from attn_bounds import attention_bounds
-
-
-def _bf(t):
-    return t.to(torch.bfloat16).to(torch.float32)
-
-
-LOG2E = 1.4426950408889634
-
-
-def _online_o(s, vv, chunk=64, thresh=8.0):
-    """The forward's online softmax: 64-key chunks, a running max in log2 units that is kept
-    while a chunk's max exceeds it by at most 8 (else O and l are rescaled), bf16 P into P.V."""
-    s2 = s * LOG2E
-    B, H, S, _ = s.shape
-    m = torch.full((B, H, S), float("-inf"))
-    l = torch.zeros(B, H, S)
-    O = torch.zeros(B, H, S, vv.shape[-1])
-    for j0 in range(0, S, chunk):
-        sc = s2[..., j0:j0 + chunk]
-        mc = sc.max(-1).values
-        need = mc > m + thresh
-        alpha = torch.where(need, torch.exp2(m - mc), torch.ones_like(m))
-        O, l = O * alpha[..., None], l * alpha
-        m = torch.where(need, mc, m)
-        p = torch.exp2(sc - m[..., None])
-        l = l + p.sum(-1)
-        O = O + torch.einsum("bhij,bjhd->bhid", _bf(p), vv[:, j0:j0 + chunk])
-    return _bf((O / l[..., None]).permute(0, 2, 1, 3)), m, l
-
-
-def _model(q, k, v, do, shift_d=False, one_head_dv=False, mask_diag_off=False, online=False):
-    B, S, Hq, hd = q.shape
-    Hkv = k.shape[2]
-    g = Hq // Hkv
-    kk, vv = k.repeat_interleave(g, 2), v.repeat_interleave(g, 2)
-    tau = 1.0 / math.sqrt(hd)
-    mask = torch.triu(torch.ones(S, S, dtype=torch.bool), 0 if mask_diag_off else 1)
-    mask[0, 0] = False
-    s = (torch.einsum("bihd,bjhd->bhij", q, kk) * tau).masked_fill(mask, float("-inf"))
-    m = s.max(-1, keepdim=True).values
-    p = torch.exp(s - m)
-    l = p.sum(-1, keepdim=True)
-    o = _bf(torch.einsum("bhij,bjhd->bihd", _bf(p), vv) / l.squeeze(-1).permute(0, 2, 1)[..., None])
-    if online:
-        o = _online_o(s, vv)[0]
-    P = torch.exp(s - (m + torch.log(l)))
-    D = (do * o).sum(-1).permute(0, 2, 1)
-    if shift_d:
-        D = torch.roll(D, 1, dims=-1)
-    dP = torch.einsum("bihd,bjhd->bhij", do, vv)
-    dS = _bf(P * (dP - D[..., None]))
-    dq = _bf(tau * torch.einsum("bhij,bjhd->bihd", dS, kk))
-    dk = _bf((tau * torch.einsum("bhij,bihd->bjhd", dS, q)).reshape(B, S, Hkv, g, hd).sum(3))
-    pdo = torch.einsum("bhij,bihd->bjhd", _bf(P), do).reshape(B, S, Hkv, g, hd)
-    dv = _bf(pdo[:, :, :, 0] * g if one_head_dv else pdo.sum(3))
-    return {"o": o, "dq": dq, "dk": dk, "dv": dv}
+from attn_model import LOG2E, bf as _bf, model as _model, online_o as _online_o
 
 
 def _inputs(B=1, S=192, Hq=4, Hkv=2, hd=128, seed=0):
@@ -110,9 +58,22 @@ def test_kernel_arithmetic_within_bound():
         got = _model(q, k, v, do, online=online)
         for name in ("o", "dq", "dk", "dv"):
             assert _worst(got, bnd, name) <= 1.0, (seed, name, _worst(got, bnd, name))
-            if bnd[name].norm() > 0:
+            if bnd[name].norm() > 0 and not ramped:
                 rf = float((got[name].double() - bnd[name]).norm() / bnd[name].norm())
                 assert rf <= 5e-3, (seed, name, rf)
+
+
+def test_frobenius_tolerance_from_the_model():
+    from attn_model import frobenius_tolerance
+    # ordinary inputs: the model's error is about half of 5e-3 (dq 2.5e-3), so the tolerance stays
+    # at about the floor
+    q, k, v, do = _inputs(seed=9)
+    tol = frobenius_tolerance(q, k, v, do, attention_bounds(q, k, v, do))
+    assert all(5e-3 <= t < 6e-3 for t in tol.values()), tol
+    # a sharp softmax: dq and dk get twice the model's own error, which is near 5e-3
+    q, k, v, do = _ramped(*_inputs(seed=10, S=256))
+    tol = frobenius_tolerance(q, k, v, do, attention_bounds(q, k, v, do))
+    assert 8e-3 < tol["dq"] < 1.2e-2 and 6e-3 < tol["dk"] < 1.2e-2 and tol["o"] == 5e-3, tol
 
 
 def test_planted_mistakes_fall_outside_bound():

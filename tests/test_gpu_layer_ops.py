@@ -10,6 +10,7 @@ import torch
 import synthetic as S
 from oracle import decoder as D
 from attn_bounds import attention_bounds
+from attn_model import frobenius_tolerance
 from tolerances import assert_close, assert_close_ew, assert_within_bound
 
 pytestmark = pytest.mark.gpu
@@ -122,10 +123,14 @@ def test_attention_fwd_bwd(lsq, B, Sq, Hq, Hkv, hd, ramp):
     bnd = attention_bounds(q, k, v, do)
     for name, want in (("o", ref), ("dq", rq), ("dk", rk), ("dv", rv)):
         assert torch.allclose(bnd[name], want, rtol=1e-9, atol=1e-12), name
-    assert_within_bound(_np(o), ref.numpy(), bnd["b_o"].numpy(), what="attn out")
-    assert_within_bound(_np(dq), rq.numpy(), bnd["b_dq"].numpy(), what="dq")
-    assert_within_bound(_np(dk), rk.numpy(), bnd["b_dk"].numpy(), what="dk")
-    assert_within_bound(_np(dv), rv.numpy(), bnd["b_dv"].numpy(), what="dv")
+    # relative Frobenius: the GEMMs' 5e-3; with a sharp softmax (ramped keys) dS = P (dP - D) cancels
+    # and the bf16 roundings alone move dq and dk by about that much, so there each output is held
+    # to twice the CPU model of the kernels' roundings (attn_model.py), never below 5e-3
+    tol = frobenius_tolerance(q, k, v, do, bnd) if ramp else {n: 5e-3 for n in ("o", "dq", "dk", "dv")}
+    assert_within_bound(_np(o), ref.numpy(), bnd["b_o"].numpy(), rel=tol["o"], what="attn out")
+    assert_within_bound(_np(dq), rq.numpy(), bnd["b_dq"].numpy(), rel=tol["dq"], what="dq")
+    assert_within_bound(_np(dk), rk.numpy(), bnd["b_dk"].numpy(), rel=tol["dk"], what="dk")
+    assert_within_bound(_np(dv), rv.numpy(), bnd["b_dv"].numpy(), rel=tol["dv"], what="dv")
 
 
 def test_attention_deterministic(lsq):
