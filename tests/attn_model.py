@@ -75,7 +75,7 @@ def model(q, k, v, do, shift_d=False, one_head_dv=False, mask_diag_off=False, on
 def frobenius_tolerance(q, k, v, do, exact, floor=5e-3, factor=2.0):
     """name -> max(floor, factor x this model's relative Frobenius error against the exact values
     (attn_bounds.attention_bounds' o, dq, dk, dv))."""
-    got = model(q, k, v, do, online=True)
+    got = model(*(t.float() for t in (q, k, v, do)), online=True)
     tol = {}
     for name in ("o", "dq", "dk", "dv"):
         ref = exact[name]
