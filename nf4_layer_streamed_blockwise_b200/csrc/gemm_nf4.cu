@@ -146,10 +146,11 @@ struct DqTab {
 };
 __device__ __forceinline__ DqTab dq_table(float a, const float (&cb)[16]) {
   DqTab t;
+  const uint64_t aa = f2(a, a);  // paired fp32 multiplies: each lane rounded as __fmul_rn
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t t0 = pack_bf16x2(__fmul_rn(cb[4 * j], a), __fmul_rn(cb[4 * j + 1], a));
-    const uint32_t t1 = pack_bf16x2(__fmul_rn(cb[4 * j + 2], a), __fmul_rn(cb[4 * j + 3], a));
+    const uint32_t t0 = pack_bf16x2(mul2(f2(cb[4 * j], cb[4 * j + 1]), aa));
+    const uint32_t t1 = pack_bf16x2(mul2(f2(cb[4 * j + 2], cb[4 * j + 3]), aa));
     t.lo[j] = prmt(t0, t1, 0x6420u);
     t.hi[j] = prmt(t0, t1, 0x7531u);
   }
