@@ -129,6 +129,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -198,6 +205,7 @@ constexpr int BT = 256;   // output columns of a pair tile (its rows: 256 * H)
 constexpr int BK = 64;
 constexpr int A_BYTES = BMC * BK * 2;  // 16 KB per 128-row activation tile
 constexpr int W_BYTES = BNC * BK * 2;  // 16 KB
+constexpr int STG_BYTES = 32 * 32 * 2;  // one warp's 32 rows x 32 columns of bf16 output
 constexpr int C_BYTES = BNC * BK / 2;  // 4 KB
 // Warp roles: 0-3 epilogue (TMEM lane quarters), 5 TMEM owner and MMA issuer, 9 TMA producer,
 // 4, 6, 7, 8, 10, 11, 12, 14 NF4 decoders, 13 idle.  A warp stalled issuing tcgen05.mma (or a TMA)
@@ -225,9 +233,14 @@ struct PCfg {
   static constexpr int OFF_W = OFF_A + NST * A_STAGE;
   static constexpr int OFF_C = OFF_W + NST * W_BYTES;
   static constexpr int OFF_BAR = OFF_C + NST * C_BYTES;
-  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1 + 2;
+  // H = 2: the epilogue stages each warp's 32 x 32 output chunk (bf16, 64-byte swizzle) in one of
+  // two 2 KB buffers per warp for a TMA store, the residual arriving there by TMA (one mbarrier
+  // per buffer)
+  static constexpr bool STG = H == 2;
+  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1 + 2 + (STG ? 8 : 0);
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
-  static constexpr int SMEM_BYTES = OFF_MISC + 128 + 1024;
+  static constexpr int OFF_STG = (OFF_MISC + 128 + 1023) / 1024 * 1024;
+  static constexpr int SMEM_BYTES = (STG ? OFF_STG + 4 * 2 * STG_BYTES : OFF_MISC + 128) + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(NBUF * H * BT <= 512, "TMEM columns");
 };
@@ -270,6 +283,9 @@ struct Maps {
   CUtensorMap la[3];  // LoRA block, activation side: FWD s*U of each segment [M, 64]; DX s*G [M, 64]
   CUtensorMap lb[3];  // LoRA block, weight side: FWD B of each segment, padded [n, 64]; DX A^T of all
                       // segments side by side [K, 64]
+  CUtensorMap y[3];    // output (H = 2 epilogue stores): FWD y of each segment [M, n]; DX dx [M, K] in y[0]
+                       // (box 32 x 32 rows, 64B swizzle)
+  CUtensorMap res[3];  // FWD residual of each segment [M, n] (same box), where there is one
 };
 
 __device__ __forceinline__ int seg_of_block(const Params& p, int i) {
@@ -346,6 +362,43 @@ __device__ __forceinline__ void clear_flags(const Params& p, int c_lo, int cid, 
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p.flags + c2 * 2 + (int)rank), "l"(0ull) : "memory");
 }
 
+// The epilogue's hand-back of a TMEM accumulator: every epilogue thread of the CTA is past its
+// last load of it; one thread clears the stream-K flags it consumed and arrives on the leader's
+// tempty barrier.
+__device__ __forceinline__ void release_acc(const Params& p, int cw, int cid, unsigned rank, int e,
+                                            uint64_t* tempty_b) {
+  tc_fence_before();
+  named_bar_sync(1, 128);
+  if (e == 0) {
+    clear_flags(p, cw, cid, rank);
+    mbar_arrive_cluster(cluster_addr(tempty_b, 0));
+  }
+}
+
+// One lane's row of a staged 32 x 32 output chunk: the accumulator values v (plus the residual row
+// at r_addr when res) rounded once to bf16 and written at s_addr (both rows of 64-byte-swizzled
+// boxes, 16-byte piece q at (q ^ (row / 2 % 4)) * 16; r_addr may equal s_addr).
+__device__ __forceinline__ void stage_chunk(float (&v)[32], bool res, uint32_t r_addr, uint32_t s_addr, int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t sw = (uint32_t)(q ^ ((lane >> 1) & 3)) << 4;
+    float* x = v + q * 8;
+    if (res) {
+      const uint4 rv = ld_shared_v4(r_addr + sw);
+      x[0] += bf16lo(rv.x);
+      x[1] += bf16hi(rv.x);
+      x[2] += bf16lo(rv.y);
+      x[3] += bf16hi(rv.y);
+      x[4] += bf16lo(rv.z);
+      x[5] += bf16hi(rv.z);
+      x[6] += bf16lo(rv.w);
+      x[7] += bf16hi(rv.w);
+    }
+    st_shared_v4(s_addr + sw, make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                         pack_bf16x2(x[6], x[7])));
+  }
+}
+
 template <int MODE>
 __device__ __forceinline__ void store_chunk(const Params& p, int sg, int n0, int ncols, int m, int c, float (&v)[32]) {
   if (m >= p.M) return;
@@ -392,6 +445,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   uint64_t* tempty = tfull + NBUF;
   uint64_t* drain = tempty + NBUF;
   uint64_t* sbar = drain + 1;  // [2]: stream-K partials pulled into the idle stages (finisher's last piece)
+  uint64_t* rbar = sbar + 2;   // [4 x 2] (H = 2): residual chunks landing in the epilogue's staging buffers
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
 
   const uint32_t rank = cluster_ctarank();
@@ -411,6 +465,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     mbar_init(&sbar[0], 1);
     mbar_init(&sbar[1], 1);
+    if constexpr (C::STG)
+      for (int b = 0; b < 8; ++b) mbar_init(&rbar[b], 1);
     fence_barrier_init();
   }
   if (warp == W_MMA) {
@@ -636,12 +692,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int e = threadIdx.x;  // TMEM lane = row within the CTA's 128
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     constexpr int PART_FLOATS = H * (BT / 32) * 128 * 32;  // one CTA's accumulator
+    uint32_t rph = 0;          // H = 2 staging: parity of the warp's residual barrier
+    bool stg_ok = true;        // false once a residual wait ran out: nothing more is stored
     int t, k0, k1;
     for (int j = 0; piece_at(p, cid, ncl, j, t, k0, k1); ++j) {
       int m0, sg, n0;
       tile_at<MODE, H>(p, t, m0, sg, n0);
       const int buf = j % NBUF;
       const uint32_t tph = (uint32_t)(j / NBUF) & 1u;
+      if constexpr (C::STG) {
+        // the tile's residual, needed only after its products, is brought into L2 meanwhile
+        if (MODE == FWD && lane == 0 && k1 == p.nkb && p.seg[sg].res) {
+          const int wrow = m0 + (int)rank * BMC + warp * 32;
+          for (int h = 0; h < H; ++h)
+            if (wrow + h * BT < p.M)
+              for (int c = 0; c < BT / 32 && n0 + c * 32 < p.seg[sg].n; ++c)
+                tma_prefetch_l2_2d(&maps.res[sg], n0 + c * 32, wrow + h * BT);
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, 731))) break;
       tc_fence_after();
       if (k1 < p.nkb) {
@@ -848,6 +916,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         continue;
       }
+      if constexpr (C::STG) {
+        if (cfirst == cid) {
+          // The whole sum is in TMEM.  Each warp takes its 32 rows two 32-column chunks at a time:
+          // both TMEM loads in flight together, then each chunk written to one of the warp's two
+          // staging buffers (bf16, 64-byte swizzle: 16-byte piece q of row i at
+          // i * 64 + (q ^ (i / 2 % 4)) * 16, conflict-free with one row per lane) and stored by
+          // one lane with TMA, so the output leaves as whole lines.  The accumulator goes back to
+          // the MMA issuer as soon as its last chunks are in registers.  A residual comes in by
+          // TMA: when no piece follows this one, the tile's whole residual at once into the idle
+          // activation stages (box (h, c) of warp w at ((w * H + h) * 8 + c) * 2 KB), else each
+          // pair's boxes into the staging buffers just ahead of their use.
+          const int si = MODE == FWD ? sg : 0;
+          const bool res = MODE == FWD && p.seg[si].res != nullptr;
+          const int cvalid = min(BT / 32, (ncols - n0 + 31) / 32);  // chunks of each half inside n
+          const int wrow = m0 + (int)rank * BMC + warp * 32;        // the warp's first row in half 0
+          uint8_t* stg = smem + C::OFF_STG + warp * 2 * STG_BYTES;
+          uint64_t* rb = &rbar[warp * 2];
+          int tn, k0n, k1n;
+          const bool res_all = res && !piece_at(p, cid, ncl, j + 1, tn, k0n, k1n);
+          uint8_t* rall = smem + C::OFF_A + warp * H * (BT / 32) * STG_BYTES;
+          bool rpend = false;  // a residual load on rb not yet waited for
+          if (res_all && stg_ok) {
+            if (lane == 0) {
+              uint32_t bytes = 0;
+              for (int h = 0; h < H; ++h)
+                if (wrow + h * BT < p.M) bytes += (uint32_t)cvalid * STG_BYTES;
+              if (bytes) {
+                mbar_arrive_expect_tx(rb, bytes);
+                for (int h = 0; h < H; ++h)
+                  if (wrow + h * BT < p.M)
+                    for (int c = 0; c < cvalid; ++c)
+                      tma_load_2d(rall + (h * (BT / 32) + c) * STG_BYTES, &maps.res[si], rb, n0 + c * 32, wrow + h * BT);
+              }
+            }
+            rpend = wrow < p.M;  // warp-uniform: half 0's rows decide whether anything was loaded
+          }
+          for (int h = 0; h < H; ++h) {
+            const int row = wrow + h * BT;
+            for (int c = 0; c < cvalid; c += 2) {
+              const bool two = c + 1 < cvalid;
+              float va[32], vb[32];
+              // (chunk c + 1 < BT / 32 always exists in TMEM; past n it is loaded but not stored)
+              tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), va);
+              tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + (c + 1) * 32), vb);
+              const bool pair_res = res && !res_all && stg_ok && row < p.M;
+              if (lane == 0) {
+                bulk_wait_read<0>();  // the last pair's stores have read both buffers
+                if (pair_res) {
+                  mbar_arrive_expect_tx(rb, (two ? 2u : 1u) * STG_BYTES);
+                  tma_load_2d(stg, &maps.res[si], rb, n0 + c * 32, row);
+                  if (two) tma_load_2d(stg + STG_BYTES, &maps.res[si], rb, n0 + (c + 1) * 32, row);
+                }
+              }
+              __syncwarp();
+              tc_wait_ld_regs(va);
+              tc_wait_ld_regs(vb);
+              if (h + 1 == H && c + 2 >= cvalid) release_acc(p, cw, cid, rank, e, &tempty[buf]);
+              if (row >= p.M) continue;  // the warp's rows are all past M (warp-uniform)
+              if ((pair_res || rpend) && stg_ok) {
+                stg_ok = __all_sync(0xffffffffu, mbar_wait(rb, rph & 1u, 737));
+                rph ^= 1u;
+                rpend = false;
+              }
+              if (!stg_ok) continue;
+              const uint32_t lrow = (uint32_t)lane * 64;
+              const uint32_t s0 = smem_u32(stg) + lrow;
+              const uint32_t r0 = res_all ? smem_u32(rall + (h * (BT / 32) + c) * STG_BYTES) + lrow : s0;
+              stage_chunk(va, res, r0, s0, lane);
+              if (two) stage_chunk(vb, res, r0 + STG_BYTES, s0 + STG_BYTES, lane);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&maps.y[si], stg, n0 + c * 32, row);
+                if (two) tma_store_2d(&maps.y[si], stg + STG_BYTES, n0 + (c + 1) * 32, row);
+                bulk_commit();
+              }
+            }
+          }
+          continue;
+        }
+      }
       for (int hc = 0; hc < H * (BT / 32); ++hc) {
         const int h = hc / (BT / 32), c = hc % (BT / 32);
         if (n0 + c * 32 >= ncols) continue;
@@ -894,6 +1043,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         clear_flags(p, cw, cid, rank);
         mbar_arrive_cluster(cluster_addr(&tempty[buf], 0));
       }
+    }
+    if constexpr (C::STG) {
+      if (lane == 0) bulk_wait_all();  // the staged stores are written before the CTA exits
     }
   }
 
@@ -1416,6 +1568,11 @@ static lsq_status tmap_act(CUtensorMap* m, const void* base, int64_t inner, int6
   return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)inner, (uint64_t)outer,
                         (uint64_t)inner * 2, 64, box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// an output (or residual) [rows, cols] bf16 as the H = 2 epilogue moves it: 32 x 32 boxes, 64B swizzle
+static lsq_status tmap_out(CUtensorMap* m, const void* base, int64_t cols, int64_t rows) {
+  return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)cols, (uint64_t)rows,
+                        (uint64_t)cols * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
 
 }  // namespace nf4g
 
@@ -1648,6 +1805,7 @@ lsq_status launch_dx(int nseg, const lsq_nf4_weight* W, const void* const* dy, i
     if ((st = tmap_act(&maps.la[0], sg, 64, M, BMC)) != LSQ_OK) return st;
     if ((st = tmap_act(&maps.lb[0], at, 64, K, BNC)) != LSQ_OK) return st;
   }
+  if ((st = tmap_out(&maps.y[0], dx, K, M)) != LSQ_OK) return st;
   p.nkb = blocks;
   return launch_pair<DX>(maps, p, (int)((K + BT - 1) / BT), sk_ws, sk_bytes, stream);
 }
@@ -1731,6 +1889,8 @@ static lsq_status fwd_impl(int32_t nseg, const lsq_nf4_weight* W, const void* x,
     if ((st = encode_tmap_2d(&maps.c[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, W[i].codes, K / 2, W[i].n_out, K / 2,
                              BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE)) != LSQ_OK)
       return st;
+    if ((st = tmap_out(&maps.y[i], g.y, g.n, M)) != LSQ_OK) return st;
+    if (g.res && (st = tmap_out(&maps.res[i], g.res, g.n, M)) != LSQ_OK) return st;
   }
   if (r > 0) {
     if (rank_part) {

@@ -181,6 +181,10 @@ def main():
         fl = sum(2.0 * M * n * K + 2.0 * M * r * K + 2.0 * M * n * r for n in ns)
         wsf = torch.empty(L.lsq_nf4_lora_fwd_workspace_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
         run(f"fwd_{g}", fl, lambda: L.lsq_nf4_lora_fwd_multi(Ws, x, M, A, B, r, s, None, ys, us, workspace=wsf))
+        if g in ("o", "down"):   # as in the decoder layer: the residual stream added in the epilogue
+            res = [torch.randn(M, n, **bf) for n in ns]
+            run(f"fwd_{g}_res", fl, lambda: L.lsq_nf4_lora_fwd_multi(Ws, x, M, A, B, r, s, res, ys, us, workspace=wsf))
+            del res
         if g == "qkv" and sh.hd in (64, 128, 256):   # the same call with q and k rotated in the epilogue
             table = L.rope_table(sh.theta, a.seq, sh.hd)
             run("fwd_qkv_rope", fl, lambda: L.lsq_nf4_lora_fwd_multi_ex2(Ws, x, M, A, B, r, s, None, ys, us, None,
