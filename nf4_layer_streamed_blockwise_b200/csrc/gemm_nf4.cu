@@ -867,6 +867,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           continue;
         }
       }
+      if constexpr (C::STG) {
+        if (rope_seg && cfirst == cid) {
+          // RoPE with the staged stores of the path below: the two 32-column chunks of a head
+          // whose columns pair up (c and c + hd/64) are loaded together, rotated in fp32 (the
+          // same arithmetic as the unstaged RoPE path below) and rounded once, staged and stored
+          // by TMA.
+          const int hc32 = p.rope_hd / 32, heads = BT / p.rope_hd;
+          const float* inv = reinterpret_cast<const float*>(p.rope) + (int64_t)p.rope_seq * p.rope_hd;
+          const int wrow = m0 + (int)rank * BMC + warp * 32;
+          uint8_t* stg = smem + C::OFF_STG + warp * 2 * STG_BYTES;
+          const int npairs = H * heads * (hc32 / 2);
+          int pi = 0;
+          for (int h = 0; h < H; ++h) {
+            const int row = wrow + h * BT;
+            const float pos = (float)((row + lane) % p.rope_seq);
+            for (int hh = 0; hh < heads; ++hh) {
+              for (int cl = 0; cl < hc32 / 2; ++cl, ++pi) {
+                const int ca = hh * hc32 + cl, cb = ca + hc32 / 2;
+                float va[32], vb[32];
+                tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + ca * 32), va);
+                tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + cb * 32), vb);
+                if (lane == 0) bulk_wait_read<0>();  // the last pair's stores have read both buffers
+                __syncwarp();
+                tc_wait_ld_regs(va);
+                tc_wait_ld_regs(vb);
+                if (pi + 1 == npairs) release_acc(p, cw, cid, rank, e, &tempty[buf]);
+                if (row >= p.M || n0 + ca * 32 >= ncols) continue;  // warp-uniform
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const float2 t = rope_cs(pos * __ldg(inv + cl * 32 + i));
+                  const float a = va[i], b = vb[i];
+                  va[i] = a * t.x - b * t.y;
+                  vb[i] = b * t.x + a * t.y;
+                }
+                const uint32_t s0 = smem_u32(stg) + (uint32_t)lane * 64;
+                stage_chunk(va, false, s0, s0, lane);
+                stage_chunk(vb, false, s0 + STG_BYTES, s0 + STG_BYTES, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(&maps.y[sg], stg, n0 + ca * 32, row);
+                  tma_store_2d(&maps.y[sg], stg + STG_BYTES, n0 + cb * 32, row);
+                  bulk_commit();
+                }
+              }
+            }
+          }
+          continue;
+        }
+      }
       if (rope_seg) {
         // RoPE in the epilogue: column i of a head pairs with column i + hd/2, which sits hd/64
         // chunks of 32 further on in the same accumulator; both are rotated in fp32 (the
