@@ -399,6 +399,57 @@ __device__ __forceinline__ void stage_chunk(float (&v)[32], bool res, uint32_t r
   }
 }
 
+// The residual of row m's 32-column chunk c (FWD with a residual): four 16-byte words of bf16
+// (the residual may alias y: each address is read before it is written).
+template <int MODE>
+__device__ __forceinline__ void load_res_chunk(const Params& p, int sg, int n0, int ncols, int m, int c,
+                                               uint4 (&r)[4]) {
+  if (MODE != FWD || m >= p.M) return;
+  const Seg& S = p.seg[sg];
+  if (!S.res) return;
+#pragma unroll
+  for (int gq = 0; gq < 4; ++gq) {
+    const int col = n0 + c * 32 + gq * 8;
+    if (col < ncols) r[gq] = *reinterpret_cast<const uint4*>(S.res + (int64_t)m * S.n + col);
+  }
+}
+
+// One epilogue warp's 32 rows (from row0) of a finished 32-column chunk c through the warp's
+// staging buffers (512-row tiles): the residual added per row from global memory (FWD), then
+// staged in buffer nst & 1 and stored by TMA; nothing for rows past M.  All lanes call it.
+template <int MODE>
+__device__ __forceinline__ void staged_store(const Params& p, const CUtensorMap* ymap, int sg, int n0, int ncols,
+                                             int row0, int c, float (&v)[32], uint8_t* stg, uint32_t& nst, int lane) {
+  const int b = (int)(nst++ & 1u);
+  if (lane == 0) bulk_wait_read<0>();  // every earlier store (a pair's included) has read its buffer
+  __syncwarp();
+  if (row0 >= p.M) return;  // warp-uniform
+  if (MODE == FWD && p.seg[sg].res) {
+    uint4 r[4] = {};
+    load_res_chunk<MODE>(p, sg, n0, ncols, row0 + lane, c, r);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float* x = v + q * 8;
+      x[0] += bf16lo(r[q].x);
+      x[1] += bf16hi(r[q].x);
+      x[2] += bf16lo(r[q].y);
+      x[3] += bf16hi(r[q].y);
+      x[4] += bf16lo(r[q].z);
+      x[5] += bf16hi(r[q].z);
+      x[6] += bf16lo(r[q].w);
+      x[7] += bf16hi(r[q].w);
+    }
+  }
+  const uint32_t s0 = smem_u32(stg + b * STG_BYTES) + (uint32_t)lane * 64;
+  stage_chunk(v, false, s0, s0, lane);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(ymap, stg + b * STG_BYTES, n0 + c * 32, row0);
+    bulk_commit();
+  }
+}
+
 template <int MODE>
 __device__ __forceinline__ void store_chunk(const Params& p, int sg, int n0, int ncols, int m, int c, float (&v)[32]) {
   if (m >= p.M) return;
@@ -693,6 +744,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     constexpr int PART_FLOATS = H * (BT / 32) * 128 * 32;  // one CTA's accumulator
     uint32_t rph = 0;          // H = 2 staging: parity of the warp's residual barrier
+    uint32_t nst = 0;          // staged stores of the single-chunk paths (buffer nst & 1)
     bool stg_ok = true;        // false once a residual wait ran out: nothing more is stored
     int t, k0, k1;
     for (int j = 0; piece_at(p, cid, ncl, j, t, k0, k1); ++j) {
@@ -848,11 +900,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             named_bar_sync(1, 128);  // buffer u & 1 is read: unit u + 2 may refill it
           }
-          if (!okb) continue;
-          if (rope_seg)  // the sum goes back into the accumulator for the RoPE epilogue below
+          if (!__all_sync(0xffffffffu, okb)) continue;
+          if (rope_seg) {  // the sum goes back into the accumulator for the RoPE epilogue below
             tmem_st32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
-          else
+          } else if constexpr (C::STG) {
+            staged_store<MODE>(p, &maps.y[MODE == FWD ? sg : 0], sg, n0, ncols, m0 + h * BT + (int)rank * BMC + warp * 32,
+                               c, v, smem + C::OFF_STG + warp * 2 * STG_BYTES, nst, lane);
+          } else {
             store_chunk<MODE>(p, sg, n0, ncols, m0 + h * BT + (int)rank * BMC + e, c, v);
+          }
         }
         if (rope_seg) {
           tc_wait_st();
@@ -1085,7 +1141,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        store_chunk<MODE>(p, sg, n0, ncols, m, c, v);
+        if constexpr (C::STG)
+          staged_store<MODE>(p, &maps.y[MODE == FWD ? sg : 0], sg, n0, ncols, m0 + h * BT + (int)rank * BMC + warp * 32, c,
+                             v, smem + C::OFF_STG + warp * 2 * STG_BYTES, nst, lane);
+        else
+          store_chunk<MODE>(p, sg, n0, ncols, m, c, v);
       }
       tc_fence_before();
       named_bar_sync(1, 128);
