@@ -97,6 +97,99 @@ __global__ void __launch_bounds__(RN_T) rmsnorm_bwd_kernel(const uint4* __restri
   }
 }
 
+// The same two RMSNorm passes with the row held in registers between the reduction and the
+// output (one read of x, dy and the residual gradient per row) and all of a thread's loads issued
+// before its first use: RN2_T threads per row, V 16-byte words per thread (d <= 8 V RN2_T).
+constexpr int RN2_T = 128;
+
+template <int V>
+__global__ void __launch_bounds__(RN2_T) rmsnorm_fwd_reg_kernel(const uint4* __restrict__ x,
+                                                                const uint4* __restrict__ g, uint4* __restrict__ y,
+                                                                float* __restrict__ rstd, int d8, float inv_d,
+                                                                float eps) {
+  __shared__ float red[RN2_T / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * d8;
+  uint4 xv[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int c = threadIdx.x + i * RN2_T;
+    xv[i] = c < d8 ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    float f[8];
+    unpack8(xv[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+  }
+  const float tot = block_sum<RN2_T>(ss, red);
+  const float rs = 1.0f / sqrtf(tot * inv_d + eps);
+  if (threadIdx.x == 0 && rstd) rstd[row] = rs;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int c = threadIdx.x + i * RN2_T;
+    if (c >= d8) break;
+    float f[8], gv[8];
+    unpack8(xv[i], f);
+    unpack8(g[c], gv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = f[j] * rs * gv[j];
+    y[row * d8 + c] = pack8(f);
+  }
+}
+
+template <int V>
+__global__ void __launch_bounds__(RN2_T) rmsnorm_bwd_reg_kernel(const uint4* __restrict__ dy,
+                                                                const uint4* __restrict__ x,
+                                                                const uint4* __restrict__ g,
+                                                                const float* __restrict__ rstd,
+                                                                const uint4* dres_in, uint4* dres_out, int d8,
+                                                                float inv_d) {
+  __shared__ float red[RN2_T / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * d8;
+  const uint4* dr = dy + row * d8;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  uint4 xv[V], dv4[V], gv4[V], rv[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int c = threadIdx.x + i * RN2_T;
+    const bool in = c < d8;
+    xv[i] = in ? xr[c] : z;
+    dv4[i] = in ? dr[c] : z;
+    gv4[i] = in ? g[c] : z;
+    rv[i] = (in && dres_in) ? dres_in[row * d8 + c] : z;  // in flight across the reduction
+  }
+  float dot = 0.0f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    float f[8], dv[8], gv[8];
+    unpack8(xv[i], f);
+    unpack8(dv4[i], dv);
+    unpack8(gv4[i], gv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dot = fmaf(dv[j] * gv[j], f[j], dot);
+  }
+  const float tot = block_sum<RN2_T>(dot, red);
+  const float rs = rstd[row];
+  const float k = rs * rs * rs * tot * inv_d;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int c = threadIdx.x + i * RN2_T;
+    if (c >= d8) break;
+    float f[8], dv[8], gv[8], o[8];
+    unpack8(xv[i], f);
+    unpack8(dv4[i], dv);
+    unpack8(gv4[i], gv);
+    unpack8(rv[i], o);  // zero without a residual gradient
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] += rs * dv[j] * gv[j] - f[j] * k;
+    dres_out[row * d8 + c] = pack8(o);
+  }
+}
+
 // ---------------------------------------------------------------- RoPE
 // one CTA per (batch, position): the hd/2 angles pos * theta^(-2i/hd) are
 // computed once in double, then every head at that position is rotated; with
@@ -464,8 +557,17 @@ extern "C" lsq_status lsq_rmsnorm_fwd(const void* x, const void* g, void* y, flo
   if (!aligned(x, 16) || !aligned(g, 16) || !aligned(y, 16)) return fail(LSQ_EINVAL, "lsq_rmsnorm_fwd: alignment");
   lsq_status st = check_device();
   if (st != LSQ_OK) return st;
-  rmsnorm_fwd_kernel<<<(unsigned)rows, RN_T, 0, (cudaStream_t)stream>>>(
-      (const uint4*)x, (const uint4*)g, (uint4*)y, rstd, (int)(d / 8), 1.0f / (float)d, eps);
+  const int d8 = (int)(d / 8), v = (d8 + RN2_T - 1) / RN2_T;
+  const unsigned nb = (unsigned)rows;
+  const float inv_d = 1.0f / (float)d;
+  cudaStream_t cs = (cudaStream_t)stream;
+  const uint4 *xx = (const uint4*)x, *gg = (const uint4*)g;
+  uint4* yy = (uint4*)y;
+  if (v <= 1) rmsnorm_fwd_reg_kernel<1><<<nb, RN2_T, 0, cs>>>(xx, gg, yy, rstd, d8, inv_d, eps);
+  else if (v <= 2) rmsnorm_fwd_reg_kernel<2><<<nb, RN2_T, 0, cs>>>(xx, gg, yy, rstd, d8, inv_d, eps);
+  else if (v <= 4) rmsnorm_fwd_reg_kernel<4><<<nb, RN2_T, 0, cs>>>(xx, gg, yy, rstd, d8, inv_d, eps);
+  else if (v <= 8) rmsnorm_fwd_reg_kernel<8><<<nb, RN2_T, 0, cs>>>(xx, gg, yy, rstd, d8, inv_d, eps);
+  else rmsnorm_fwd_kernel<<<nb, RN_T, 0, cs>>>(xx, gg, yy, rstd, d8, inv_d, eps);
   LSQ_LAUNCH_CHECK("rmsnorm_fwd_kernel");
   return LSQ_OK;
 }
@@ -480,9 +582,17 @@ extern "C" lsq_status lsq_rmsnorm_bwd(const void* dy, const void* x, const void*
     return fail(LSQ_EINVAL, "lsq_rmsnorm_bwd: alignment");
   lsq_status st = check_device();
   if (st != LSQ_OK) return st;
-  rmsnorm_bwd_kernel<<<(unsigned)rows, RN_T, 0, (cudaStream_t)stream>>>(
-      (const uint4*)dy, (const uint4*)x, (const uint4*)g, rstd, (const uint4*)dres_in, (uint4*)dres_out, (int)(d / 8),
-      1.0f / (float)d);
+  const int d8 = (int)(d / 8), v = (d8 + RN2_T - 1) / RN2_T;
+  const unsigned nb = (unsigned)rows;
+  const float inv_d = 1.0f / (float)d;
+  cudaStream_t cs = (cudaStream_t)stream;
+  const uint4 *dd = (const uint4*)dy, *xx = (const uint4*)x, *gg = (const uint4*)g, *ri = (const uint4*)dres_in;
+  uint4* ro = (uint4*)dres_out;
+  if (v <= 1) rmsnorm_bwd_reg_kernel<1><<<nb, RN2_T, 0, cs>>>(dd, xx, gg, rstd, ri, ro, d8, inv_d);
+  else if (v <= 2) rmsnorm_bwd_reg_kernel<2><<<nb, RN2_T, 0, cs>>>(dd, xx, gg, rstd, ri, ro, d8, inv_d);
+  else if (v <= 4) rmsnorm_bwd_reg_kernel<4><<<nb, RN2_T, 0, cs>>>(dd, xx, gg, rstd, ri, ro, d8, inv_d);
+  else if (v <= 8) rmsnorm_bwd_reg_kernel<8><<<nb, RN2_T, 0, cs>>>(dd, xx, gg, rstd, ri, ro, d8, inv_d);
+  else rmsnorm_bwd_kernel<<<nb, RN_T, 0, cs>>>(dd, xx, gg, rstd, ri, ro, d8, inv_d);
   LSQ_LAUNCH_CHECK("rmsnorm_bwd_kernel");
   return LSQ_OK;
 }

@@ -32,7 +32,8 @@ def _grad(fn, inputs, dy):
     return out.detach(), gr
 
 
-@pytest.mark.parametrize("M,d,eps", [(130, 576, 1e-5), (64, 4096, 1e-5), (1, 256, 1e-5), (512, 2048, 1e-6)])
+@pytest.mark.parametrize("M,d,eps", [(130, 576, 1e-5), (64, 4096, 1e-5), (1, 256, 1e-5), (512, 2048, 1e-6),
+                                     (8, 5120, 1e-5), (3, 9216, 1e-5)])
 def test_rmsnorm_fwd_bwd(lsq, M, d, eps):
     x = _rand((M, d), 2.0, 1)
     g = _rand((d,), 0.3, 2) + 1
@@ -50,6 +51,10 @@ def test_rmsnorm_fwd_bwd(lsq, M, d, eps):
     rr = 1.0 / np.sqrt((_np(x) ** 2).mean(-1) + eps)
     assert_close(rstd.cpu().numpy(), rr, rel=1e-6, max_rms=1e-5, what="rstd")
     assert_close_ew(_np(out), dx.numpy() + _np(res), what="rmsnorm dx + res")
+    out0 = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")   # no residual gradient to add
+    lsq.lsq_rmsnorm_bwd(dy.cuda(), x.cuda(), g.cuda(), rstd, None, out0, M, d)
+    torch.cuda.synchronize()
+    assert_close_ew(_np(out0), dx.numpy(), what="rmsnorm dx")
 
 
 @pytest.mark.parametrize("B,Sq,H,hd,theta", [(2, 300, 4, 64, 1e4), (1, 512, 8, 128, 5e5), (1, 50, 3, 24, 1e4),
