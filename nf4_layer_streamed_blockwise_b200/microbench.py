@@ -199,6 +199,20 @@ def main():
         fl0 = sum(2.0 * M * n * K for n in ns)
         run(f"dx_{g}", fl0, lambda: L.lsq_nf4_lora_bwd_multi(Ws, x, dys, M, None, None, 0, 0.0, None, dx, None, None,
                                                                 0, None))
+        # the calls of a training step's backward half: the layer's first forward leaves a rank state
+        # (s*U and the padded LoRA operands), which its checkpoint recompute (rfwd: the fused GEMM
+        # alone, with the residual or RoPE the layer uses) and its backward (sbwd: G, dX, dA, dB) reuse
+        st = torch.zeros(L.lsq_nf4_lora_state_size(ns, M, K, r), dtype=torch.uint8, device="cuda")
+        resr = [torch.randn(M, n, **bf) for n in ns] if g in ("o", "down") else None
+        roper = ((L.rope_table(sh.theta, a.seq, sh.hd), a.seq, sh.hd, 0b011)
+                 if g == "qkv" and sh.hd in (64, 128, 256) else None)
+        L.lsq_nf4_lora_fwd_multi_ex2(Ws, x, M, A, B, r, s, resr, ys, None, st, False, roper, workspace=wsf)
+        flr = sum(2.0 * M * n * K + 2.0 * M * n * r for n in ns)
+        run(f"rfwd_{g}", flr, lambda: L.lsq_nf4_lora_fwd_multi_ex2(Ws, x, M, A, B, r, s, resr, ys, None, st, True, roper,
+                                                                   workspace=wsf))
+        run(f"sbwd_{g}", fl, lambda: L.lsq_nf4_lora_bwd_multi_ex(Ws, x, dys, M, A, B, r, s, None, st, dx, dA, dB, 0,
+                                                                  ws))
+        del st, resr, roper
         del Ws, x, A, B, ys, us, dys, dx, dA, dB, ws, wsf
     # causal GQA attention of one layer (the batch's sequences), forward and backward
     Hq, Hkv, hd, Bt, Sq = sh.n_q, sh.n_kv, sh.hd, a.batch, a.seq
