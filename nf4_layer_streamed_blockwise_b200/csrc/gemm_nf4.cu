@@ -206,6 +206,7 @@ constexpr int BK = 64;
 constexpr int A_BYTES = BMC * BK * 2;  // 16 KB per 128-row activation tile
 constexpr int W_BYTES = BNC * BK * 2;  // 16 KB
 constexpr int STG_BYTES = 32 * 32 * 2;  // one warp's 32 rows x 32 columns of bf16 output
+constexpr int SKB = 8;                  // 16 KB buffers of stream-K partials a finisher keeps in flight
 constexpr int C_BYTES = BNC * BK / 2;  // 4 KB
 // Warp roles: 0-3 epilogue (TMEM lane quarters), 5 TMEM owner and MMA issuer, 9 TMA producer,
 // 4, 6, 7, 8, 10, 11, 12, 14 NF4 decoders, 13 idle.  A warp stalled issuing tcgen05.mma (or a TMA)
@@ -237,7 +238,7 @@ struct PCfg {
   // two 2 KB buffers per warp for a TMA store, the residual arriving there by TMA (one mbarrier
   // per buffer)
   static constexpr bool STG = H == 2;
-  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1 + 2 + (STG ? 8 : 0);
+  static constexpr int NBAR = 3 * NST + 2 * NBUF + 1 + SKB + (STG ? 8 : 0);
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_STG = (OFF_MISC + 128 + 1023) / 1024 * 1024;
   static constexpr int SMEM_BYTES = (STG ? OFF_STG + 4 * 2 * STG_BYTES : OFF_MISC + 128) + 1024;
@@ -338,19 +339,6 @@ __device__ __forceinline__ void tile_at(const Params& p, int t, int& m0, int& sg
   }
 }
 
-// Bulk copies of stream-K unit u (32-column chunk u / G of the tile's valid chunks, partials
-// 4 (u % G) .. of the P contributors whose first partial is part0) into stage buffer u % 2
-__device__ __forceinline__ void sk_issue(uint8_t* stage, uint64_t* sbar, const float* part0, int u, int G, int P,
-                                         int cvalid) {
-  constexpr int PART_F = 2 * (BT / 32) * 128 * 32;  // one CTA's partial with 512-row tiles
-  const int k = u / G, g = u % G;
-  const int hc = (k / cvalid) * (BT / 32) + k % cvalid;
-  const int n = min(4, P - 4 * g);
-  mbar_arrive_expect_tx(&sbar[u & 1], (uint32_t)n * 16384u);
-  for (int i = 0; i < n; ++i)
-    bulk_g2s(stage + (u & 1) * 65536 + i * 16384, part0 + (int64_t)(4 * g + i) * 2 * PART_F + (int64_t)hc * 4096,
-             16384u, &sbar[u & 1]);
-}
 
 // bf16 output of 32 columns (chunk c) of row m of a tile whose first column is n0, with the residual (FWD)
 // A finisher that has seen the partials of clusters [c_lo, cid) for its rank clears their flags
@@ -495,8 +483,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   uint64_t* tfull = cfull + NST;
   uint64_t* tempty = tfull + NBUF;
   uint64_t* drain = tempty + NBUF;
-  uint64_t* sbar = drain + 1;  // [2]: stream-K partials pulled into the idle stages (finisher's last piece)
-  uint64_t* rbar = sbar + 2;   // [4 x 2] (H = 2): residual chunks landing in the epilogue's staging buffers
+  uint64_t* sbar = drain + 1;   // [SKB]: stream-K partials pulled into the idle stages (finisher's last piece)
+  uint64_t* rbar = sbar + SKB;  // [4 x 2] (H = 2): residual chunks landing in the epilogue's staging buffers
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
 
   const uint32_t rank = cluster_ctarank();
@@ -514,8 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&tempty[b], 2);  // one epilogue arrival per CTA
     }
     mbar_init(drain, 1);
-    mbar_init(&sbar[0], 1);
-    mbar_init(&sbar[1], 1);
+    for (int b = 0; b < SKB; ++b) mbar_init(&sbar[b], 1);
     if constexpr (C::STG)
       for (int b = 0; b < 8; ++b) mbar_init(&rbar[b], 1);
     fence_barrier_init();
@@ -865,14 +852,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       const bool rope_seg = MODE == FWD && p.seg[sg].rope;
       if (bulk) {
-        const int P = cid - cfirst, G = (P + 3) / 4;
+        // units u = (chunk k, contributor i), chunk-major: the 16 KB of contributor i's partial for
+        // chunk k, bulk-copied into one of SKB buffers of the idle activation stages, SKB units in
+        // flight (so the L2 round trips overlap); added in cluster order, as in the path below
+        const int P = cid - cfirst;
         const int cvalid = min(BT / 32, (ncols - n0 + 31) / 32);
-        const int nunits = H * cvalid * G;
-        uint8_t* stage = smem + C::OFF_A;  // 2 x 4 x 16 KB = the activation stages, idle now
+        const int nunits = H * cvalid * P;
+        uint8_t* stage = smem + C::OFF_A;  // SKB x 16 KB of the activation stages, idle now
         const float* part0 = p.part + (int64_t)(cfirst * 2 + (int)rank) * PART_FLOATS;
+        auto issue = [&](int uu) {  // thread e == 0
+          const int k = uu / P, i = uu % P;
+          const int hc = (k / cvalid) * (BT / 32) + k % cvalid;
+          mbar_arrive_expect_tx(&sbar[uu % SKB], 16384u);
+          bulk_g2s(stage + (uu % SKB) * 16384, part0 + (int64_t)i * 2 * PART_FLOATS + (int64_t)hc * 4096, 16384u,
+                   &sbar[uu % SKB]);
+        };
         if (e == 0) {
           fence_proxy_async_all();  // the partials were published to this thread's acquires above
-          sk_issue(stage, sbar, part0, 0, G, P, cvalid);
+          for (int uu = 0; uu < min(SKB, nunits); ++uu) issue(uu);
         }
         bool okb = true;  // false once a wait ran out: every thread still passes every barrier, nothing is stored
         int u = 0;
@@ -880,25 +877,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const int h = k / cvalid, c = k % cvalid;
           float v[32];
           tmem_ld32(tmem + lane_base + (uint32_t)((buf * H + h) * BT + c * 32), v);
-          for (int g = 0; g < G; ++g, ++u) {
-            if (e == 0 && u + 1 < nunits && okb) sk_issue(stage, sbar, part0, u + 1, G, P, cvalid);
-            okb = okb && mbar_wait(&sbar[u & 1], (uint32_t)(u >> 1) & 1u, 736);
-            if (g == 0) tc_wait_ld();
+          for (int i = 0; i < P; ++i, ++u) {
+            okb = okb && mbar_wait(&sbar[u % SKB], (uint32_t)(u / SKB) & 1u, 736);
+            if (i == 0) tc_wait_ld();
             if (okb) {
-              const float4* sb = reinterpret_cast<const float4*>(stage + (u & 1) * 65536) + e;
-              const int n = min(4, P - 4 * g);
-              for (int i = 0; i < n; ++i) {
+              const float4* sb = reinterpret_cast<const float4*>(stage + (u % SKB) * 16384) + e;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  const float4 a = sb[i * 1024 + q * 128];
-                  v[4 * q] += a.x;
-                  v[4 * q + 1] += a.y;
-                  v[4 * q + 2] += a.z;
-                  v[4 * q + 3] += a.w;
-                }
+              for (int q = 0; q < 8; ++q) {
+                const float4 a = sb[q * 128];
+                v[4 * q] += a.x;
+                v[4 * q + 1] += a.y;
+                v[4 * q + 2] += a.z;
+                v[4 * q + 3] += a.w;
               }
             }
-            named_bar_sync(1, 128);  // buffer u & 1 is read: unit u + 2 may refill it
+            // buffer u % SKB is read (unit u + SKB may refill it); a wait that ran out anywhere stops all
+            okb = named_bar_and(1, 128, okb);
+            if (e == 0 && okb && u + SKB < nunits) issue(u + SKB);
           }
           if (!__all_sync(0xffffffffu, okb)) continue;
           if (rope_seg) {  // the sum goes back into the accumulator for the RoPE epilogue below
