@@ -41,11 +41,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused forward
 # GEMM (nf4_pair_kernel<FWD>), the mean over the four calls of an 8B layer as
 # the checkpoint recompute runs them (q/k/v with RoPE, o and down adding their
-# residual, gate/up, at 2048 tokens: 56.1, 43.9, 201.0 and 126.0 MB), from one
+# residual, gate/up, at 2048 tokens: 51.1, 43.9, 197.7 and 126.3 MB), from one
 # ncu capture of the kernel built from the sources whose SHA-256 prefix is
 # given; the figure is reported only while those sources are unchanged (else
 # traffic is null).
-NCU_TRAFFIC = {("llama-3.1-8b", 2048): (106.8e6, "98b96dfbc8ddc34f")}
+NCU_TRAFFIC = {("llama-3.1-8b", 2048): (104.8e6, "736a214a541a1cb0")}
 TRAFFIC_SOURCES = ("nf4_layer_streamed_blockwise_b200/csrc/gemm_nf4.cu",
                    "nf4_layer_streamed_blockwise_b200/csrc/common.cuh")
 
