@@ -310,8 +310,8 @@ lsq_status lsq_nf4_lora_fwd_multi_ex2(int32_t nseg, const lsq_nf4_weight* W, con
  * anything is enqueued.  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current, and the
  * first call on a host thread creates the library's per-thread side stream
- * and events and queries device attributes.  Every call shares the array and leaves its last
- * contents there; nothing in it needs to start at zero (each call writes all
+ * and events and queries device attributes.  Every call shares the array
+ * and leaves its last contents there; nothing in it needs to start at zero (each call writes all
  * the scratch it reads, and stream-K flags carry a per-launch value).  Calls
  * that overlap on the GPU (other streams or host threads) race on the array:
  * the caller must serialise them. */
