@@ -311,10 +311,10 @@ lsq_status lsq_nf4_lora_fwd_multi_ex2(int32_t nseg, const lsq_nf4_weight* W, con
  * device address (cudaGetSymbolAddress) with that device current, and the
  * first call on a host thread creates the library's per-thread side stream
  * and events and queries device attributes.  Every call shares the array
- * and leaves its last contents there; nothing in it needs to start at zero (each call writes all
- * the scratch it reads, and stream-K flags carry a per-launch value).  Calls
- * that overlap on the GPU (other streams or host threads) race on the array:
- * the caller must serialise them. */
+ * and leaves its last contents there; nothing in it needs to start at zero
+ * (each call writes all the scratch it reads, and stream-K flags carry a
+ * per-launch value).  Calls that overlap on the GPU (other streams or host
+ * threads) race on the array: the caller must serialise them. */
 size_t lsq_nf4_lora_bwd_noalloc_max_scratch(void);
 lsq_status lsq_nf4_lora_bwd_noalloc(const lsq_nf4_weight* W, const void* x, const void* dy, int64_t M,
                                     const void* A, const void* B, int32_t r, float s, const float* u, void* dx,
