@@ -15,10 +15,11 @@ are cut into two and three pieces and some ranges lie wholly inside a tile):
 * the same call with whole tiles (no workspace room) agrees within the GEMM
   tolerance.
 
-The last case of each test has few tiles and a long contraction (512 rows, 6
-tiles of 512 x 256, 128 weight blocks each): there a small number of clusters
-shares each tile (five per tile by the plan's cost model), so every finisher
-adds about four partials, pulled into its idle stages with bulk copies.
+The last two cases of each test have few tiles and a long contraction (512
+rows; 6 tiles of 128 weight blocks, then 2 tiles of 256): there several
+clusters share each tile (by the plan's cost model five and four per tile),
+so every finisher adds up to four partials, pulled into its idle stages with
+bulk copies.
 """
 import numpy as np
 import pytest
@@ -54,7 +55,8 @@ def _fwd(lsq, ws_list, x, M, A, B, r, s, ys, us, workspace):
         lsq.lsq_nf4_lora_fwd_multi(ws_list, x, M, A, B, r, s, None, ys, us, workspace=workspace)
 
 
-@pytest.mark.parametrize("M,Ns,K", [(1000, [4800], 1024), (1024, [2048, 1536, 1216], 1024), (512, [1536], 8192)])
+@pytest.mark.parametrize("M,Ns,K", [(1000, [4800], 1024), (1024, [2048, 1536, 1216], 1024), (512, [1536], 8192),
+                                    (512, [512], 16384)])
 def test_streamk_fwd_matches_oracle_and_is_deterministic(lsq, M, Ns, K):
     r = 16
     cases = [S.linear_case(M, n, K, r, s=1.0, seed=300 + i) for i, n in enumerate(Ns)]
@@ -103,7 +105,8 @@ def test_streamk_b_zero_equals_base_bitwise(lsq, M, N, K):
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("M,Ns,K", [(1000, [1024], 4800), (1024, [512, 256, 256], 4800), (512, [4096, 4096], 1536)])
+@pytest.mark.parametrize("M,Ns,K", [(1000, [1024], 4800), (1024, [512, 256, 256], 4800), (512, [4096, 4096], 1536),
+                                    (512, [16384], 512)])
 def test_streamk_dx_matches_oracle_and_is_deterministic(lsq, M, Ns, K):
     r = 16
     cases = [S.linear_case(M, n, K, r, s=1.0, seed=320 + i) for i, n in enumerate(Ns)]
