@@ -138,6 +138,31 @@ def test_fwd_with_residual_and_no_lora(lsq):
     assert_close(y.float().cpu().numpy(), ref, what="Y+res")
 
 
+@pytest.mark.parametrize("M,N,K", [(1000, 4104, 256), (2048, 8200, 128)])
+def test_fwd_residual_512_row_tiles(lsq, monkeypatch, M, N, K):
+    """512-row tiles (forced) with the residual added in the staged epilogue,
+    against the oracle: 34 tiles (one per cluster: the tile's whole residual
+    comes in by TMA before its stores) and 132 (two per cluster for most: the
+    first tile's residual a pair of chunks at a time); M and N ragged (rows
+    past M and a last tile of 8 columns); the residual aliasing y gives the
+    same bits."""
+    monkeypatch.setenv("LSQ_NF4_TILE_ROWS", "512")
+    r = 16
+    case = S.linear_case(M, N, K, r, s=16.0 / r, seed=M + N + 5)
+    w = _gpu_quant(lsq, case["W"])
+    A, B = _lora_bf16(case)
+    res = S.bf16(S.normal_f32(9, 11, (M, N)))
+    x, Ag, Bg, rg = case["X"].cuda(), A.cuda(), B.cuda(), res.cuda()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    lsq.lsq_nf4_lora_fwd(w, x, M, Ag, Bg, r, case["s"], rg, y, None)
+    y2 = rg.clone()                               # residual aliases y
+    lsq.lsq_nf4_lora_fwd(w, x, M, Ag, Bg, r, case["s"], y2, y2, None)
+    torch.cuda.synchronize()
+    Y, _, _ = _oracle_fwd(case, *_oracle_quant(case["W"]), residual=res)
+    assert_close(y.float().cpu().numpy(), Y, what="Y + residual")
+    assert torch.equal(y, y2)
+
+
 def test_b_zero_equals_base_bitwise(lsq):
     M, N, K, r = 128, 512, 512, 8
     case = S.linear_case(M, N, K, r)
