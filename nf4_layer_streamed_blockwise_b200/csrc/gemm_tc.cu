@@ -193,6 +193,221 @@ __global__ void __launch_bounds__(NTHREADS, 1) dense_gemm_kernel(const __grid_co
   }
 }
 
+// ---------------------------------------------------------------- persistent form
+// Without acc_in the tiles go to a persistent grid (one CTA per SM, tile t, t + G, ... with the row
+// tile fastest, as above) whose two TMEM accumulators (2 x 256 columns) alternate, so the epilogue
+// of one tile runs under the products of the next.  The epilogue stages each warp's 32 rows x 32
+// columns in shared memory (two buffers per warp; fp32 rows of 128 bytes in the 128-byte swizzle,
+// bf16 rows of 64 bytes in the 64-byte one) and one lane stores the box with TMA, so the output
+// leaves as whole lines; the accumulator goes back to the MMA issuer once its last columns are in
+// registers.
+constexpr int PSTG = 2;  // staging buffers per epilogue warp
+template <int F32>
+struct PCfg {
+  static constexpr int STG = 32 * 32 * (F32 ? 4 : 2);
+  static constexpr int OFF_STG = OFF_B + NST * B_BYTES;
+  static constexpr int OFF_PBAR = OFF_STG + 4 * PSTG * STG;
+  static constexpr int NPBAR = 2 * NST + 4;  // full, empty, tfull[2], tempty[2]
+  static constexpr int OFF_PMISC = OFF_PBAR + 8 * NPBAR;
+  static constexpr int PBYTES = OFF_PMISC + 64 + 1024;
+  static_assert(PBYTES <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void wait_ld_dep(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]),
+                 "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
+                 "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]),
+                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
+}
+// one lane's row of a 32 x 32 output chunk into its staged row at s_row: fp32 as eight 16-byte
+// pieces, piece q at (q ^ (row % 8)) * 16; bf16 as four, piece q at (q ^ (row / 2 % 4)) * 16
+template <int F32>
+__device__ __forceinline__ void stage_row(const float (&v)[32], uint32_t s_row, int lane) {
+  if (F32) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      sts_v4(s_row + ((uint32_t)(q ^ (lane & 7)) << 4),
+             make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                        __float_as_uint(v[4 * q + 3])));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      sts_v4(s_row + ((uint32_t)(q ^ ((lane >> 1) & 3)) << 4),
+             make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                        pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7])));
+  }
+}
+
+struct PMaps {
+  CUtensorMap a, b, out;  // out: [M, N] with row stride ldo, box 32 x 32 (swizzle as staged)
+};
+
+template <int NN, int F32>
+__global__ void __launch_bounds__(NTHREADS, 1) dense_pgemm_kernel(const __grid_constant__ PMaps maps,
+                                                                  const __grid_constant__ Params p) {
+  using C = PCfg<F32>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_PBAR);
+  uint64_t* empty = full + NST;
+  uint64_t* tfull = empty + NST;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_PMISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntm = (p.M + BM - 1) / BM, ntn = (p.N + BN - 1) / BN, tiles = ntm * ntn;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const int m0 = (t % ntm) * BM, n0 = (t / ntm) * BN;
+        for (int i = 0; i < p.nkb; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, 425)) {
+            ok = false;
+            break;
+          }
+          uint8_t* b_dst = smem + OFF_B + s * B_BYTES;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES));
+          tma_load_2d(smem + OFF_A + s * A_BYTES, &maps.a, &full[s], i * BK, m0);
+          if (!NN) {
+            tma_load_2d(b_dst, &maps.b, &full[s], i * BK, n0);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &maps.b, &full[s], n0 + c * 64, i * BK);
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(BM, BN, 0, NN);
+      uint32_t g = 0;
+      bool ok = true;
+      int j = 0;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++j) {
+        const int buf = j & 1;
+        if (!mbar_wait(&tempty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, 526)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BN);
+        for (int i = 0; i < p.nkb; ++i, ++g) {
+          const int s = (int)(g % NST);
+          const uint32_t ph = (g / NST) & 1u;
+          if (!mbar_wait(&full[s], ph, 527)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + OFF_A + s * A_BYTES);
+          const uint32_t b_base = smem_u32(smem + OFF_B + s * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bd =
+                NN ? smem_desc(b_base + kk * 2048, 8192, 1024, 2) : smem_desc(b_base + kk * 32, 16, 1024, 2);
+            tc_mma(d, smem_desc(a_base + kk * 32, 16, 1024, 2), bd, id, (i | kk) != 0);
+          }
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&tfull[buf]);  // also when a wait gave up: the epilogue is not left waiting
+      }
+    }
+  } else {
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    uint8_t* stg = smem + C::OFF_STG + warp * PSTG * C::STG;
+    int j = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+      const int m0 = (t % ntm) * BM, n0 = (t / ntm) * BN;
+      const int buf = j & 1;
+      const int row = m0 + warp * 32;  // the warp's first row
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (uint32_t)(j >> 1) & 1u, 726))) break;
+      tc_fence_after();
+      const int cvalid = min(BN / 32, (p.N - n0 + 31) / 32);
+      for (int c = 0; c < cvalid; c += 2) {
+        // chunk c + 1 < BN / 32 always exists in TMEM; past N it is loaded but not stored
+        float va[32], vb[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(buf * BN + c * 32), va);
+        tmem_ld32(tmem + lane_base + (uint32_t)(buf * BN + (c + 1) * 32), vb);
+        if (lane == 0) bulk_wait_read<0>();  // the last stores have read both buffers
+        __syncwarp();
+        wait_ld_dep(va);
+        wait_ld_dep(vb);
+        if (c + 2 >= cvalid) {  // the accumulator is in registers: hand it back
+          tc_fence_before();
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 0) mbar_arrive(&tempty[buf]);
+        }
+        if (row >= p.M) continue;  // warp-uniform
+        const bool two = c + 1 < cvalid;
+        const uint32_t s0 = smem_u32(stg) + (uint32_t)lane * (F32 ? 128 : 64);
+        stage_row<F32>(va, s0, lane);
+        if (two) stage_row<F32>(vb, s0 + C::STG, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&maps.out, stg, n0 + c * 32, row);
+          if (two) tma_store_2d(&maps.out, stg + C::STG, n0 + (c + 1) * 32, row);
+          bulk_commit();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_all();  // the staged stores are written before the CTA exits
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int NN, int F32>
+static lsq_status launch_p(const PMaps& maps, const Params& p, cudaStream_t stream) {
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    LSQ_CUDA_TRY(cudaFuncSetAttribute(dense_pgemm_kernel<NN, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PCfg<F32>::PBYTES));
+    configured[dev] = 1;
+  }
+  const int64_t tiles = (int64_t)((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+  const int grid = (int)std::min<int64_t>(tiles, (int64_t)num_sms());
+  dense_pgemm_kernel<NN, F32><<<grid, NTHREADS, PCfg<F32>::PBYTES, stream>>>(maps, p);
+  LSQ_LAUNCH_CHECK("dense_pgemm_kernel");
+  return LSQ_OK;
+}
+
 template <int NN>
 static lsq_status launch(const Maps& maps, const Params& p, dim3 grid, cudaStream_t stream) {
   static int configured[64] = {0};
@@ -242,6 +457,29 @@ extern "C" lsq_status lsq_dense_gemm_ex(const void* a, int64_t lda, const void* 
   if ((st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, K, M, lda * 2, BK, BM,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
     return st;
+  if (!acc_in) {  // the persistent form (two accumulators, staged TMA stores)
+    PMaps pm;
+    memset(&pm, 0, sizeof(pm));
+    pm.a = maps.a;
+    if (!trans_b) {
+      if ((st = encode_tmap_2d(&pm.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b, K, N, K * 2, BK, BN,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+        return st;
+    } else if ((st = encode_tmap_2d(&pm.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b, N, K, N * 2, 64, BK,
+                                    CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK) {
+      return st;
+    }
+    if (out_f32) {
+      if ((st = encode_tmap_2d(&pm.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, N, M, ldo * 4, 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != LSQ_OK)
+        return st;
+      return trans_b ? launch_p<1, 1>(pm, p, (cudaStream_t)stream) : launch_p<0, 1>(pm, p, (cudaStream_t)stream);
+    }
+    if ((st = encode_tmap_2d(&pm.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_64B)) != LSQ_OK)
+      return st;
+    return trans_b ? launch_p<1, 0>(pm, p, (cudaStream_t)stream) : launch_p<0, 0>(pm, p, (cudaStream_t)stream);
+  }
   if ((N + BN - 1) / BN > 65535) return fail(LSQ_EINVAL, "%s: N too large for the grid", who);
   dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)((N + BN - 1) / BN));
   if (!trans_b) {
