@@ -155,8 +155,9 @@ def test_attention_deterministic(lsq):
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("B,Sq,V", [(2, 64, 1000), (1, 512, 49152)])
+@pytest.mark.parametrize("B,Sq,V", [(2, 64, 1000), (1, 512, 49152), (1, 96, 128256), (2, 40, 1002)])
 def test_cross_entropy(lsq, B, Sq, V):
+    """Small, odd and 8B-sized vocabularies (128256) against the oracle's loss and gradient."""
     logits = torch.from_numpy(S.normal_f32(S.DATA_SEED, 77, (B * Sq, V), 2.0))
     ids = S.uniform_ids(S.DATA_SEED, 78, (B, Sq), V)
     loss = torch.zeros(1, dtype=torch.float32, device="cuda")
